@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the ragged paged decode library on B200.
+
+One step = one decode step of one layer over the whole batch: the split-K decode kernel plus
+the log-sum-exp merge, through the C ABI (tg_ragged_paged_decode / tg_tiered_decode). The
+batch's KV cache, page tables and plan are resident in HBM before timing (admission happens
+once, as in serving); the step's inputs are the queries.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run, one rank per GPU. The batch is sharded by sequence with
+the library's ahead-of-time placement (per-GPU work fixed: weak scaling); the decode has no
+data-path collective, the ranks only agree on timing (barrier + max over ranks).
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "ragged paged decode attn: KV-read GB/s vs HBM peak; decode tokens/s per layer"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2**20
+
+WORKLOAD_NAMES = {
+    1: "tiny ragged MHA decode: 1 seq, 8/8 heads, d 64, retained U[16,256] per head, page 16",
+    2: "GQA decode layer, ragged budgets: batch 64/GPU, 32 q / 8 KV heads, d 128, context "
+       "U[2048,8192], retention ratio ranked onto [0.1,0.9] +-0.05 per (seq, KV head), "
+       "4 budget groups, page 16, pool 90% occupied, shuffled",
+    3: "multi-turn serving step, one layer: batch 256/GPU, 32 q / 8 KV heads, d 128, context "
+       "U[4096,32768], ratios [0.05,0.5] over 256 (layer, head) ranks, 8 budget groups",
+    4: "prefix-shared decode: 512 seqs/GPU, 32 q / 8 KV heads, d 128, 2000-token system prefix "
+       "+ 1 of 8 500-token docs + private 80-100 tokens, full retention",
+    5: "tiered long-context decode: batch 4/GPU, context 131072, 32 q / 8 KV heads, d 128, last "
+       "8192 tokens bf16, older INT8 per token per head, >= 64 chunks per head",
+}
+
+
+def _env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def _plan_kw(cfg):
+    return dict(min_splits=64, max_chunk_pages=128) if cfg == 5 else {}
+
+
+def _global_spec(cfg, world):
+    sp = synth.preset(cfg)
+    if world > 1:
+        from dataclasses import replace
+        sp = replace(sp, B=sp.B * world)
+    return sp
+
+
+def _my_sequences(sp, rank, world, kv_len, fast_len):
+    """Ahead-of-time placement of sequences on ranks by retained K/V bytes."""
+    if world == 1:
+        return None
+    import non_uniform_paged_flash_b200 as tg
+    if fast_len is None:
+        per_seq = kv_len.astype(np.int64).sum(1) * 2 * sp.D * 2
+    else:
+        f = fast_len.astype(np.int64)
+        per_seq = ((kv_len - f) * 2 * (sp.D + 4) + f * 2 * sp.D * 2).sum(1)
+    gpu = tg.tg_place_sequences(per_seq, world)
+    return np.nonzero(gpu == rank)[0]
+
+
+def _measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _traffic(cfg):
+    """DRAM bytes per launch of the decode kernel from a committed ncu capture, if the kernel
+    source is unchanged since the capture; else None."""
+    src = os.path.join(ROOT, "non_uniform_paged_flash_b200", "csrc", "tg_kernels.cu")
+    path = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+    try:
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        with open(path) as f:
+            j = json.load(f)
+        e = j.get(f"config{cfg}")
+        if e and e.get("kernel_sha") == sha:
+            return float(e["traffic_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = str(gpu_index)
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"bench_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------
+# Reference arm: the CPU oracle, as it stands, on bounded samples of the same workload.
+# ------------------------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = _env_int("RANK", 0)
+    if rank != 0:
+        return 0
+    import oracle
+    from oracle import workload as ow
+    cfg = args.config
+    sp = synth.preset(cfg)
+    o = ow.layout(sp, 0)
+    q = ow.q_bits(sp)
+    G = sp.Hq // sp.Hkv
+    # Each step: the query rows of one sequence (round-robin over the batch).
+    if o.fast_len is None:
+        k = synth.pool_bits(sp, "k", o.num_pages)
+        v = synth.pool_bits(sp, "v", o.num_pages)
+
+        def step(b):
+            sel = np.arange(b * sp.Hq, (b + 1) * sp.Hq)
+            oracle.decode(q, k, v, o.table, o.head_off, o.kv_len, sp.scale, sel=sel)
+            return int(o.kv_len[b].astype(np.int64).sum()) * 2 * sp.D * 2
+    else:
+        k = synth.pool_bits(sp, "k", o.num_pages)
+        v = synth.pool_bits(sp, "v", o.num_pages)
+        kq, ks = oracle.quantize_int8(synth.pool_bits(sp, "kslow", o.num_slow_pages))
+        vq, vs = oracle.quantize_int8(synth.pool_bits(sp, "vslow", o.num_slow_pages))
+
+        def step(b):
+            # one KV head of one sequence per step (bounded: the heads are 131072 tokens)
+            h = b % sp.Hkv
+            bb = (b // sp.Hkv) % sp.B
+            sel = np.arange(bb * sp.Hq + h * G, bb * sp.Hq + (h + 1) * G)
+            oracle.tiered_decode(q, kq, vq, ks, vs, o.slow_table, o.slow_off, k, v, o.table,
+                                 o.head_off, o.kv_len, o.fast_len, sp.scale, sel=sel)
+            n, f = int(o.kv_len[bb, h]), int(o.fast_len[bb, h])
+            return (n - f) * 2 * (sp.D + 4) + f * 2 * sp.D * 2
+    for i in range(args.warmup):
+        step(i % sp.B)
+    t0 = time.perf_counter()
+    nbytes = 0
+    for i in range(args.steps):
+        nbytes += step(i % sp.B)
+    dt = time.perf_counter() - t0
+    value = nbytes / dt / 1e9
+    cores = oracle.num_threads()
+    sample = ("per step: all query rows of one sequence" if o.fast_len is None else
+              "per step: the query rows of one (sequence, KV head)") + \
+        f"; fp64 oracle over {cores} threads"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAMES[cfg], "config_id": cfg},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------
+# Our arm
+# ------------------------------------------------------------------------------------------
+
+def cpu_baseline(cfg, budget_s=20.0):
+    """The oracle as it stands on a bounded sample of this workload (rank 0, N = 1)."""
+    import oracle
+    from oracle import workload as ow
+    sp = synth.preset(cfg)
+    o = ow.layout(sp, 0)
+    q = ow.q_bits(sp)
+    cores = oracle.num_threads()
+    if o.fast_len is not None:
+        return None
+    k = synth.pool_bits(sp, "k", o.num_pages)
+    v = synth.pool_bits(sp, "v", o.num_pages)
+    done, nbytes, t_used = 0, 0, 0.0
+    chunk = max(1, sp.B // 16)
+    while done < sp.B and t_used < budget_s:
+        b1 = min(sp.B, done + chunk)
+        sel = np.arange(done * sp.Hq, b1 * sp.Hq)
+        t0 = time.perf_counter()
+        oracle.decode(q, k, v, o.table, o.head_off, o.kv_len, sp.scale, sel=sel)
+        t_used += time.perf_counter() - t0
+        nbytes += int(o.kv_len[done:b1].astype(np.int64).sum()) * 2 * sp.D * 2
+        done = b1
+    return {"value": nbytes / t_used / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"sequences 0..{done - 1} of the batch (all their query rows), "
+                      f"{t_used:.1f} s of fp64 oracle time on {cores} host threads"}
+
+
+def run_ours(args):
+    import torch
+    import non_uniform_paged_flash_b200 as tg
+    from non_uniform_paged_flash_b200 import workload
+
+    rank, world = _env_int("RANK", 0), _env_int("WORLD_SIZE", 1)
+    local = _env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    cfg = args.config
+    sp = _global_spec(cfg, world)
+    kv_all, fast_all = workload.retained(sp, 0)
+    seqs = _my_sequences(sp, rank, world, kv_all, fast_all)
+    lay = workload.layout(sp, 0, seqs)
+    db = workload.to_device(sp, lay, 0, device=f"cuda:{local}", seqs=seqs, **_plan_kw(cfg))
+    info = tg.tg_plan_get_info(db.plan)
+    alg = workload.algorithmic_bytes(sp, lay)
+    B_local = lay.kv_len.shape[0]
+    stream = torch.cuda.current_stream()
+
+    # L2: inputs larger than L2 need no flush; smaller ones get a flush between steps.
+    flush = None
+    if alg["kv"] < 2 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=f"cuda:{local}")
+
+    def step():
+        if flush is not None:
+            flush.zero_()
+        db.run(stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert tg.tg_plan_status(db.plan) == tg.TG_OK, "device error word set during warm-up"
+
+    n_timed = min(args.steps, 4096)
+    tg.tg_plan_timing_enable(db.plan, n_timed)
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    ms_total = ev0.elapsed_time(ev1)
+    n_rec, dec_ms, mrg_ms = tg.tg_plan_timing_read(db.plan)
+    tg.tg_plan_timing_enable(db.plan, 0)
+    status = tg.tg_plan_status(db.plan)
+
+    # End to end through the public call with host buffers: pinned q in, out + lse back.
+    q_host = db.q.cpu().pin_memory()
+    out_host = torch.empty(db.out.shape, dtype=db.out.dtype).pin_memory()
+    lse_host = torch.empty(db.lse.shape, dtype=db.lse.dtype).pin_memory()
+    k_e2e = min(args.steps, 2000)
+
+    def e2e_step():
+        if flush is not None:
+            flush.zero_()
+        db.q.copy_(q_host, non_blocking=True)
+        db.run(stream)
+        out_host.copy_(db.out, non_blocking=True)
+        lse_host.copy_(db.lse, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(k_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+
+    # Max over ranks (time) and sums (work).
+    vals = torch.tensor([ms_total, e2e_ms, dec_ms / max(n_rec, 1), float(alg["kv"]),
+                         float(B_local), float(status != tg.TG_OK)], dtype=torch.float64,
+                        device=f"cuda:{local}")
+    if dist is not None:
+        mx = vals.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        sm = vals.clone()
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+        ms_total, e2e_ms, dec_avg = mx[0].item(), mx[1].item(), mx[2].item()
+        kv_total, b_total, bad = sm[3].item(), sm[4].item(), mx[5].item()
+    else:
+        dec_avg = vals[2].item()
+        kv_total, b_total, bad = float(alg["kv"]), float(B_local), float(status != tg.TG_OK)
+
+    ms_step = ms_total / args.steps
+    value = kv_total / (ms_step * 1e-3) / 1e9
+    e2e_value = kv_total / (e2e_ms / k_e2e * 1e-3) / 1e9
+
+    if rank == 0:
+        peak, peak_kind = _measured_peak()
+        achieved = alg["total"] / (dec_avg * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if lay.fast_len is None else "bf16+int8", "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAMES[cfg], "config_id": cfg,
+                       "global_batch": int(b_total), "parallelism":
+                       "sequence shards by AOT byte placement, no collective" if world > 1
+                       else "single GPU",
+                       "l2": ("inputs larger than L2 (%.2f GB K/V per step vs 126 MB)" %
+                              (alg["kv"] / 1e9)) if flush is None else "L2 flushed between steps"},
+            "tokens_per_s_per_layer": b_total / (ms_step * 1e-3),
+            "kv_bytes_per_step": int(kv_total),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": _traffic(cfg) if world == 1 else None,
+                         "peak_kind": peak_kind, "kernel": "decode_kernel",
+                         "algorithmic_bytes_per_launch": alg["total"],
+                         "avg_launch_ms": dec_avg, "merge_avg_ms": mrg_ms / max(n_rec, 1),
+                         "launches_timed": n_rec},
+            "e2e": {"value": e2e_value, "unit": "GB/s",
+                    "h2d_bytes_per_step": int(db.q.numel() * db.q.element_size()),
+                    "d2h_bytes_per_step": int(db.out.numel() * db.out.element_size() +
+                                              db.lse.numel() * db.lse.element_size()),
+                    "steps": k_e2e},
+            "gpu_launches": args.steps * (1 + (1 if info["n_merge"] > 0 else 0)),
+            "plan": {k: info[k] for k in ("n_items", "n_partials", "n_merge", "n_workers",
+                                          "grid", "stages", "smem_bytes")},
+            "device_status": "ok" if not bad else "error word set",
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cfg)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,276 @@
+/*
+ * tg.h — C ABI of the B200 ragged / prefix-shared / tiered paged decode library (libtg.so).
+ *
+ * One decode step of attention for a batch of sequences whose KV cache is paged, where every
+ * (sequence, KV head) keeps its own number of tokens:
+ *   - per-head budgets fixed at admission and ragged page tables grouped by budget
+ *     ("Tangram" explainer, arXiv 2606.06302: 核心方法 / 三大机制 1 Budget Reservation,
+ *     2 Ragged Paging, 3 Ahead-of-Time Load Balancing);
+ *   - prefix pages shared across sequences through their page tables (RadixAttention lesson,
+ *     Phase 17 · 06: the radix tree as KV index and its worked example);
+ *   - a recent bf16 tier and an older INT8 tier dequantised inside the attention loop
+ *     ("TTKV" explainer, arXiv 2604.19769: 核心方法 1 Tier Layout, 2 Tier Content,
+ *     3 Tier Interaction);
+ *   - split-K over each head's tokens merged by log-sum-exp (CAP survey, arXiv 2405.11299,
+ *     §2.4.3 "加速单个请求": the online normaliser; Fig. 5 Dist Attention).
+ *
+ * Conventions for every function:
+ *   - Return value: TG_OK (0) or one of the TG_E* codes below. Nothing throws across the ABI.
+ *   - Host pointers are read during the call only. Device pointers are caller-owned device
+ *     memory (allocate them with any allocator); the library never frees them.
+ *   - Device calls are stream-ordered and asynchronous on the given stream; they allocate
+ *     nothing, synchronise nothing and re-plan nothing per call. Pass the stream as the
+ *     cudaStream_t value cast to tg_stream (NULL = legacy default stream).
+ *   - Layouts are row-major and contiguous unless stated. "bf16" = IEEE bfloat16 bits.
+ *   - Device base pointers must be 16-byte aligned (TG_EINVAL otherwise).
+ *   - Query head hq uses KV head hq / (Hq/Hkv) (contiguous GQA groups of G = Hq/Hkv).
+ *   - Supported by the kernels: page = 16 tokens, D in {64, 128}, G in {1, 2, 4, 8};
+ *     the tiered kernel needs D = 128. Other shapes return TG_EUNSUPPORTED.
+ *   - Not thread-safe per object: one host thread at a time per tg_alloc / tg_plan.
+ */
+#ifndef TG_H
+#define TG_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TG_OK 0
+#define TG_EINVAL 1        /* bad argument: null/misaligned pointer, inconsistent sizes */
+#define TG_ENOSPC 2        /* page pool exhausted; the allocator state is unchanged */
+#define TG_EBADPAGE 3      /* a kernel met a page id outside the pool, a table row outside its
+                              group table, or lengths that differ from the plan; the offending
+                              pages were skipped (never read), the affected rows are unspecified */
+#define TG_ECUDA 4         /* a CUDA runtime call failed (message via tg_last_cuda_error) */
+#define TG_ETIMEOUT 5      /* a kernel wait exceeded its bound; the kernel returned early */
+#define TG_ENOMEM 6        /* host or device allocation failed */
+#define TG_ENOTFOUND 7     /* unknown sequence or segment id */
+#define TG_EUNSUPPORTED 8  /* shape outside what the kernels support */
+#define TG_EEXIST 9        /* sequence id already holds a reservation */
+
+typedef struct CUstream_st *tg_stream; /* == cudaStream_t */
+
+/* Shape of one decode step over one layer. */
+typedef struct tg_shape {
+    int32_t B;              /* sequences */
+    int32_t Hq;             /* query heads */
+    int32_t Hkv;            /* KV heads; Hq % Hkv == 0 */
+    int32_t D;              /* head dimension */
+    int32_t page;           /* tokens per page (16) */
+    int32_t reserved;       /* 0 */
+    int64_t num_pages;      /* pages in the bf16 pools (k_pages, v_pages / k_fast, v_fast) */
+    int64_t num_slow_pages; /* pages in the INT8 pools (tiered decode only; else 0) */
+} tg_shape;
+
+/* Human-readable text of a status code (static storage). */
+const char *tg_strerror(int status);
+/* Text of the last CUDA error seen by this library on the calling thread ("" if none). */
+const char *tg_last_cuda_error(void);
+
+/* =====================================================================================
+ * Host-side admission steps (pure host code; no device needed).
+ * ===================================================================================== */
+
+/* Retained length from the budget table ("Tangram" 关键发现: per-head retention ratios from
+ * an input-invariant head ranking; 三大机制 1: footprint fixed at admission).
+ * For i < n: kv_len[i] = 0 if full_len[i] <= 0, else
+ *   min(full_len[i], max(1, floor((ratio_ppm[i] * full_len[i] + 500000) / 1000000))).
+ * ratio_ppm in [0, 1000000]; out of range -> TG_EINVAL. Arrays host, length n. */
+int tg_retained_lengths(int64_t n, const int32_t *full_len, const int32_t *ratio_ppm,
+                        int32_t *kv_len);
+
+/* Budget groups ("Tangram" 三大机制 2, Ragged Paging: heads with similar budgets share one
+ * page table). Heads ranked by budget ascending (ties by index); rank p of n_heads goes to
+ * group floor(p * n_groups / n_heads). budget_ppm, group_of_head: host, length n_heads.
+ * 1 <= n_groups <= n_heads, else TG_EINVAL. */
+int tg_budget_groups(int32_t n_heads, const int32_t *budget_ppm, int32_t n_groups,
+                     int32_t *group_of_head);
+
+/* ---- Budget-reservation page allocator ("Tangram" 三大机制 1; RadixAttention worked
+ * example for shared segments). A FIFO free list of page ids: reservations take pages from
+ * the front, releases append freed pages at the back in release order. Owns only host
+ * memory. */
+typedef struct tg_alloc tg_alloc;
+
+/* num_pages >= 1; page = tokens per page (>= 1). free_order: a permutation of
+ * 0..num_pages-1 giving the initial free-list order (NULL = ascending). A non-permutation
+ * returns TG_EINVAL. */
+int tg_alloc_create(int64_t num_pages, int32_t page, const int32_t *free_order, tg_alloc **out);
+void tg_alloc_destroy(tg_alloc *a);
+int64_t tg_alloc_free_pages(const tg_alloc *a);   /* pages currently on the free list */
+/* References held on a page (0 = free; a shared page counts its segment plus each reader). */
+int32_t tg_alloc_refcount(const tg_alloc *a, int32_t page_id);
+
+/* Shared segment of n_tokens tokens for n_heads KV heads: floor(n_tokens/page) full pages per
+ * head, taken head ascending, page ascending. Only full pages are shared; a partial tail goes
+ * into each reader's private pages. *seg_id receives the segment id; page_ids (may be NULL)
+ * receives [n_heads][floor(n_tokens/page)]. All-or-nothing: TG_ENOSPC leaves state unchanged. */
+int tg_alloc_share_segment(tg_alloc *a, int32_t n_tokens, int32_t n_heads, int32_t *seg_id,
+                           int32_t *page_ids);
+
+/* Reservation of sequence seq_id at admission: for each KV head h (ascending), its page list
+ * is the full pages of each segment in prefix_segs[0..n_prefix) (in order; a negative id is
+ * skipped), followed by ceil((kv_len[h] - shared tokens)/page) private pages from the free
+ * list. kv_len[h] must be >= the shared tokens (TG_EINVAL otherwise). All-or-nothing:
+ * TG_ENOSPC leaves state unchanged. page_ids (host, capacity entries) receives the lists
+ * head after head; *n_written the total. Each head's count is ceil(kv_len[h]/page) when every
+ * shared segment holds whole pages. seq_id must be new (TG_EEXIST). */
+int tg_alloc_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads, const int32_t *kv_len,
+                     int32_t n_prefix, const int32_t *prefix_segs, int32_t *page_ids,
+                     int64_t capacity, int64_t *n_written);
+/* Release a sequence: private pages return to the free list, shared pages drop one reference. */
+int tg_alloc_release(tg_alloc *a, int32_t seq_id);
+/* Drop a segment's own reference; its pages return once no sequence reads them. */
+int tg_alloc_release_segment(tg_alloc *a, int32_t seg_id);
+
+/* Group page tables ("Tangram" 三大机制 2). For B sequences x Hkv heads with head_count[b][h]
+ * pages whose ids are listed in page_ids (flat: b ascending, h ascending, page ascending —
+ * the order tg_alloc_reserve writes them for b = 0, 1, ...): group g's table is dense
+ * [B][H_g][P_g] (heads of g ascending, P_g = max page count in g, unused slots -1); tables
+ * concatenated in group order. Writes head_off[B*Hkv] (start of each row) and
+ * group_off[n_groups+1] (start of each group table; group_off[n_groups] = total length).
+ * table may be NULL to query the length (head_off then may be NULL too); otherwise it must
+ * hold group_off[n_groups] entries. All arrays host. */
+int tg_group_tables(int32_t B, int32_t Hkv, const int32_t *head_count,
+                    const int32_t *group_of_head, int32_t n_groups, const int32_t *page_ids,
+                    int32_t *table, int64_t *head_off, int64_t *group_off);
+
+/* Ahead-of-time placement of sequences on GPUs ("Tangram" 三大机制 3): longest-processing-
+ * time greedy over seq_bytes (descending, ties by index) onto the least-loaded GPU (ties by
+ * lowest index). gpu_of_seq: host, length n_seq. */
+int tg_place_sequences(int32_t n_seq, const int64_t *seq_bytes, int32_t n_gpus,
+                       int32_t *gpu_of_seq);
+
+/* =====================================================================================
+ * Plan: the static work list of one layer's decode step (single-GPU form of "Tangram"
+ * 三大机制 3: balanced ahead of time, never re-planned per step).
+ * ===================================================================================== */
+typedef struct tg_plan tg_plan;
+
+typedef struct tg_plan_opts {
+    int32_t num_workers;      /* 0: (SM count) x (workers per CTA) of the device */
+    int32_t min_splits;       /* cut every head into at least this many chunks (>= 1) */
+    int32_t max_chunk_pages;  /* 0: no cap; else chunks hold at most this many pages */
+    int32_t host_only;        /* 1: build the work list on the host only (inspection; decode
+                                 calls reject such a plan); 0: also create device state */
+    int32_t device;           /* CUDA device ordinal, -1 = current */
+    int32_t reserved[3];
+} tg_plan_opts;
+
+/* Build a plan. kv_len[B*Hkv] (host): retained tokens per (sequence, KV head); the decode
+ * calls check the device copy against it. fast_len[B*Hkv] (host) or NULL: tiered plan whose
+ * last min(fast_len, kv_len) tokens of each head are in the bf16 tier and the rest in the INT8
+ * tier. group_of_head[Hkv] and group_off[n_groups+1] (host; from tg_budget_groups /
+ * tg_group_tables) bound every row of the bf16 (fast) table to its group table; for a tiered
+ * plan slow_table_len bounds the INT8 tier's table (ignored otherwise).
+ * Each head's tokens are cut into chunks (min_splits, max_chunk_pages; chunks never cross a
+ * tier boundary), and the byte cost of all chunks is partitioned into num_workers equal
+ * contiguous ranges; a head cut into several items is merged by log-sum-exp after the decode.
+ * The plan owns one device allocation (work list, merge list, partial results, error word),
+ * made here; nothing is allocated per call. */
+int tg_plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,
+                   const int32_t *group_of_head, const int64_t *group_off, int32_t n_groups,
+                   int64_t slow_table_len, const tg_plan_opts *opts, tg_plan **out);
+void tg_plan_destroy(tg_plan *p);
+
+typedef struct tg_plan_info {
+    int64_t n_items;          /* work items */
+    int64_t n_partials;       /* items that write a partial result (heads with > 1 item) */
+    int64_t n_merge;          /* heads finished by the merge kernel (split or empty) */
+    int32_t n_workers;        /* workers that have items */
+    int32_t grid;             /* CTAs of the decode kernel */
+    int32_t block;            /* threads per CTA */
+    int32_t smem_bytes;       /* dynamic shared memory per CTA */
+    int32_t stages;           /* pipeline stages per worker */
+    int32_t reserved;
+    int64_t device_bytes;     /* bytes of the plan's device allocation */
+    int64_t kv_bytes;         /* retained K/V bytes one step reads (scales included) */
+} tg_plan_info;
+int tg_plan_get_info(const tg_plan *p, tg_plan_info *info);
+
+/* Work list export for inspection: items (host, n_items x 8 int32): per item
+ * {b*Hkv + h, page_begin, page_end, tier_tokens, partial slot (-1 = final), flags (bit 0 =
+ * INT8 tier), worker, 0}; page indices are within the head's row of its tier's table. */
+int tg_plan_items(const tg_plan *p, int32_t *items);
+
+/* Read and clear the plan's device error word after the work queued on stream: returns
+ * TG_OK, TG_EBADPAGE or TG_ETIMEOUT. Synchronises the stream (a debugging aid). */
+int tg_plan_status(tg_plan *p, tg_stream stream);
+
+/* Kernel timing (a profiling aid). With max_calls > 0, the next max_calls decode calls on this
+ * plan record CUDA events on their stream before the decode kernel, between it and the merge
+ * kernel, and after the merge; later calls record nothing. The events are created here (no
+ * device memory); max_calls = 0 destroys them. tg_plan_timing_read waits for the last
+ * recorded event, returns the number of calls recorded and the summed decode-kernel and
+ * merge-kernel times in milliseconds, and restarts the count. */
+int tg_plan_timing_enable(tg_plan *p, int32_t max_calls);
+int tg_plan_timing_read(tg_plan *p, int32_t *n_calls, double *decode_ms, double *merge_ms);
+
+/* =====================================================================================
+ * Decode entry points (device).
+ * ===================================================================================== */
+
+/* Ragged paged decode ("Tangram" 三大机制 2 Ragged Paging; CAP §2.4.3 online normaliser):
+ * for every query row (b, hq), h = hq / G, n = head_kv_len[b*Hkv+h], the retained tokens
+ * t < n are read through the page table (page = page_table[head_page_off[b*Hkv+h] + t/16],
+ * slot t % 16) and
+ *   lse = ln sum_t exp(s_t),  s_t = scale * q . K_t,   out = sum_t exp(s_t - lse) V_t.
+ * n = 0 gives out = 0, lse = -inf.
+ *   plan        from tg_plan_create with fast_len = NULL and this shape.
+ *   q           device bf16 [B][Hq][D]
+ *   k_pages     device bf16 [num_pages][16][D];   v_pages likewise
+ *   page_table  device int32, the concatenated group tables (tg_group_tables)
+ *   head_page_off device int64 [B*Hkv];  head_kv_len device int32 [B*Hkv] (must equal the
+ *               plan's kv_len); group_of_head device int32 [Hkv]
+ *   scale       softmax scale applied in fp32 (e.g. 1/sqrt(D))
+ *   out         device bf16 [B][Hq][D];  lse device fp32 [B][Hq] (natural log)
+ * Reads each page once per item with the Tensor Memory Accelerator; computes q.K and P.V on
+ * tensor cores (bf16 in, fp32 accumulate; P rounded to bf16); writes out/lse for single-item
+ * heads and partials for split heads, then runs the merge. */
+int tg_ragged_paged_decode(tg_plan *plan, const void *q, const void *k_pages,
+                           const void *v_pages, const int32_t *page_table,
+                           const int64_t *head_page_off, const int32_t *head_kv_len,
+                           const int32_t *group_of_head, float scale, void *out, float *lse,
+                           tg_stream stream);
+
+/* Tiered decode ("TTKV" 核心方法 1-3): as tg_ragged_paged_decode over the union of two tiers.
+ * Per head, f = min(head_fast_len, n): tokens [0, n - f) are in the INT8 tier (row starts at
+ * slot 0 of slow_page_table[slow_head_off[b*Hkv+h]]), tokens [n - f, n) in the bf16 tier
+ * (row starts at slot 0 of fast_page_table[fast_head_off[b*Hkv+h]]).
+ *   k_q8, v_q8       device int8 [num_slow_pages][16][D] (symmetric codes)
+ *   k_scale, v_scale device fp32 [num_slow_pages][16] (per token per head): K_t = code * scale
+ *   k_fast, v_fast   device bf16 [num_pages][16][D]
+ * The INT8 rows are converted exactly to fp16 in registers; the K scale multiplies the score
+ * and the V scale multiplies the probability before P.V (both in fp32). plan from
+ * tg_plan_create with this fast_len. D must be 128. */
+int tg_tiered_decode(tg_plan *plan, const void *q, const int8_t *k_q8, const int8_t *v_q8,
+                     const float *k_scale, const float *v_scale, const int32_t *slow_page_table,
+                     const int64_t *slow_head_off, const void *k_fast, const void *v_fast,
+                     const int32_t *fast_page_table, const int64_t *fast_head_off,
+                     const int32_t *head_kv_len, const int32_t *head_fast_len, float scale,
+                     void *out, float *lse, tg_stream stream);
+
+/* Log-sum-exp merge of split results (CAP §2.4.3 online normaliser; Fig. 5 Dist Attention):
+ * for each of n_rows rows, its splits j = row_split_off[r] .. row_split_off[r+1]-1 hold a
+ * normalised partial part_o[j][D] (fp32) and part_lse[j] (fp32, natural log):
+ *   lse = ln sum_j exp(part_lse[j]),  out = sum_j exp(part_lse[j] - lse) part_o[j]
+ * in split order; a row with no splits (or only -inf splits) gets out = 0, lse = -inf.
+ * All pointers device; row_split_off int64 [n_rows+1]; out bf16 [n_rows][D]; lse fp32. */
+int tg_lse_merge(int64_t n_rows, int32_t D, const int64_t *row_split_off, const float *part_o,
+                 const float *part_lse, void *out, float *lse, tg_stream stream);
+
+/* INT8 slow-tier quantisation ("TTKV" 核心方法 1/3: older tokens stored quantised; scheme
+ * left open by the page): per row (token of one head) of D bf16 values,
+ *   amax = max |x|, scale = amax / 127 (fp32), code = clamp(rint(x / scale), -127, 127)
+ * with an IEEE fp32 quotient and ties to even; amax = 0 gives scale 0 and zero codes.
+ * src device bf16 [n_rows][D]; codes device int8 [n_rows][D]; scale device fp32 [n_rows].
+ * A page of the INT8 pool is 16 consecutive rows. */
+int tg_quantize_int8(int64_t n_rows, int32_t D, const void *src, int8_t *codes, float *scale,
+                     tg_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TG_H */

@@ -1,0 +1,352 @@
+"""Python binding of libtg, the B200 ragged / prefix-shared / tiered paged decode library.
+
+Argument marshalling only: every step runs in libtg.so (host C++ for admission-time steps,
+sm_100a CUDA kernels for the decode). There is no fallback: if libtg.so is missing or fails
+to load, importing the library raises. The C ABI is declared in include/tg.h; each function
+here has the same name and documents only how Python arguments map onto it.
+
+Host arrays are numpy arrays (converted to contiguous arrays of the ABI's dtype). Device
+arrays are CUDA tensors (anything with .data_ptr()); the stream defaults to torch's current
+stream on the current device.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtg.so")
+
+TG_OK, TG_EINVAL, TG_ENOSPC, TG_EBADPAGE, TG_ECUDA, TG_ETIMEOUT = 0, 1, 2, 3, 4, 5
+TG_ENOMEM, TG_ENOTFOUND, TG_EUNSUPPORTED, TG_EEXIST = 6, 7, 8, 9
+
+
+class TGError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib().tg_strerror(status).decode()
+        if status == TG_ECUDA:
+            msg += " — " + _lib().tg_last_cuda_error().decode()
+        super().__init__(f"{where}: {msg} (status {status})")
+
+
+class tg_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("page", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("num_pages", ctypes.c_int64), ("num_slow_pages", ctypes.c_int64)]
+
+
+class tg_plan_opts(ctypes.Structure):
+    _fields_ = [("num_workers", ctypes.c_int32), ("min_splits", ctypes.c_int32),
+                ("max_chunk_pages", ctypes.c_int32), ("host_only", ctypes.c_int32),
+                ("device", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+
+
+class tg_plan_info(ctypes.Structure):
+    _fields_ = [("n_items", ctypes.c_int64), ("n_partials", ctypes.c_int64),
+                ("n_merge", ctypes.c_int64), ("n_workers", ctypes.c_int32),
+                ("grid", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("smem_bytes", ctypes.c_int32), ("stages", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("device_bytes", ctypes.c_int64),
+                ("kv_bytes", ctypes.c_int64)]
+
+
+_L = None
+
+# (name, restype, argtypes)
+_P, _I32, _I64, _F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+_SIGS = [
+    ("tg_strerror", ctypes.c_char_p, [ctypes.c_int]),
+    ("tg_last_cuda_error", ctypes.c_char_p, []),
+    ("tg_retained_lengths", ctypes.c_int, [_I64, _P, _P, _P]),
+    ("tg_budget_groups", ctypes.c_int, [_I32, _P, _I32, _P]),
+    ("tg_alloc_create", ctypes.c_int, [_I64, _I32, _P, ctypes.POINTER(_P)]),
+    ("tg_alloc_destroy", None, [_P]),
+    ("tg_alloc_free_pages", _I64, [_P]),
+    ("tg_alloc_refcount", _I32, [_P, _I32]),
+    ("tg_alloc_share_segment", ctypes.c_int, [_P, _I32, _I32, _P, _P]),
+    ("tg_alloc_reserve", ctypes.c_int, [_P, _I32, _I32, _P, _I32, _P, _P, _I64, _P]),
+    ("tg_alloc_release", ctypes.c_int, [_P, _I32]),
+    ("tg_alloc_release_segment", ctypes.c_int, [_P, _I32]),
+    ("tg_group_tables", ctypes.c_int, [_I32, _I32, _P, _P, _I32, _P, _P, _P, _P]),
+    ("tg_place_sequences", ctypes.c_int, [_I32, _P, _I32, _P]),
+    ("tg_plan_create", ctypes.c_int, [ctypes.POINTER(tg_shape), _P, _P, _P, _P, _I32, _I64,
+                                      ctypes.POINTER(tg_plan_opts), ctypes.POINTER(_P)]),
+    ("tg_plan_destroy", None, [_P]),
+    ("tg_plan_get_info", ctypes.c_int, [_P, ctypes.POINTER(tg_plan_info)]),
+    ("tg_plan_items", ctypes.c_int, [_P, _P]),
+    ("tg_plan_status", ctypes.c_int, [_P, _P]),
+    ("tg_plan_timing_enable", ctypes.c_int, [_P, _I32]),
+    ("tg_plan_timing_read", ctypes.c_int, [_P, _P, _P, _P]),
+    ("tg_ragged_paged_decode", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _F32, _P, _P, _P]),
+    ("tg_tiered_decode", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                        _F32, _P, _P, _P]),
+    ("tg_lse_merge", ctypes.c_int, [_I64, _I32, _P, _P, _P, _P, _P, _P]),
+    ("tg_quantize_int8", ctypes.c_int, [_I64, _I32, _P, _P, _P, _P]),
+]
+
+#: Symbols the C ABI exports (include/tg.h).
+ABI_SYMBOLS = tuple(n for n, _, _ in _SIGS)
+
+
+def _lib():
+    global _L
+    if _L is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libtg.so not built ({LIB_PATH}); run "
+                              "`python -m non_uniform_paged_flash_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, res, args in _SIGS:
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _L = lib
+    return _L
+
+
+def load():
+    """Load libtg.so (raises if it is missing)."""
+    return _lib()
+
+
+def _check(status: int, where: str):
+    if status != TG_OK:
+        raise TGError(status, where)
+
+
+def _h(a, dtype):
+    """Host array as a contiguous numpy array of dtype."""
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _hp(a):
+    return None if a is None else a.ctypes.data
+
+
+def _dp(t):
+    """Device pointer of a CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not getattr(t, "is_cuda", False):
+        raise ValueError("expected a CUDA tensor for a device argument")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+# ------------------------------------------------------------------------------------------
+# Host-side admission steps
+# ------------------------------------------------------------------------------------------
+
+def tg_retained_lengths(full_len, ratio_ppm) -> np.ndarray:
+    L = _h(full_len, np.int32)
+    r = _h(ratio_ppm, np.int32)
+    if L.shape != r.shape:
+        raise ValueError("shape mismatch")
+    out = np.empty(L.shape, dtype=np.int32)
+    _check(_lib().tg_retained_lengths(L.size, _hp(L), _hp(r), _hp(out)), "tg_retained_lengths")
+    return out
+
+
+def tg_budget_groups(budget_ppm, n_groups: int) -> np.ndarray:
+    b = _h(budget_ppm, np.int32).reshape(-1)
+    out = np.empty(b.size, dtype=np.int32)
+    _check(_lib().tg_budget_groups(b.size, _hp(b), n_groups, _hp(out)), "tg_budget_groups")
+    return out
+
+
+def tg_alloc_create(num_pages: int, page: int = 16, free_order=None):
+    fo = None if free_order is None else _h(free_order, np.int32)
+    h = ctypes.c_void_p()
+    _check(_lib().tg_alloc_create(num_pages, page, _hp(fo), ctypes.byref(h)), "tg_alloc_create")
+    return h
+
+
+def tg_alloc_destroy(a):
+    _lib().tg_alloc_destroy(a)
+
+
+def tg_alloc_free_pages(a) -> int:
+    return int(_lib().tg_alloc_free_pages(a))
+
+
+def tg_alloc_refcount(a, page_id: int) -> int:
+    return int(_lib().tg_alloc_refcount(a, page_id))
+
+
+def tg_alloc_share_segment(a, n_tokens: int, n_heads: int, page: int = 16):
+    """Returns (seg_id, page_ids int32[n_heads, n_tokens // page])."""
+    full = n_tokens // page
+    ids = np.empty((n_heads, full), dtype=np.int32)
+    sid = ctypes.c_int32()
+    _check(_lib().tg_alloc_share_segment(a, n_tokens, n_heads, ctypes.byref(sid), _hp(ids)),
+           "tg_alloc_share_segment")
+    return sid.value, ids
+
+
+def tg_alloc_reserve(a, seq_id: int, kv_len, prefix_segs=(), page: int = 16) -> np.ndarray:
+    """Reserve all heads of one sequence; returns its page ids (flat, head after head)."""
+    kv = _h(kv_len, np.int32).reshape(-1)
+    segs = _h(np.asarray(prefix_segs, dtype=np.int32).reshape(-1), np.int32)
+    cap = int(kv.astype(np.int64).sum() // page + kv.size * (1 + max(1, segs.size)))
+    ids = np.empty(cap, dtype=np.int32)
+    n = ctypes.c_int64()
+    _check(_lib().tg_alloc_reserve(a, seq_id, kv.size, _hp(kv), segs.size,
+                                   _hp(segs) if segs.size else None, _hp(ids), cap,
+                                   ctypes.byref(n)), "tg_alloc_reserve")
+    return ids[:n.value].copy()
+
+
+def tg_alloc_release(a, seq_id: int):
+    _check(_lib().tg_alloc_release(a, seq_id), "tg_alloc_release")
+
+
+def tg_alloc_release_segment(a, seg_id: int):
+    _check(_lib().tg_alloc_release_segment(a, seg_id), "tg_alloc_release_segment")
+
+
+def tg_group_tables(head_count, group_of_head, n_groups: int, page_ids):
+    """Returns (table int32[len], head_off int64[B, Hkv], group_off int64[n_groups + 1])."""
+    hc = _h(head_count, np.int32)
+    B, Hkv = hc.shape
+    goh = _h(group_of_head, np.int32)
+    ids = _h(page_ids, np.int32)
+    goff = np.empty(n_groups + 1, dtype=np.int64)
+    _check(_lib().tg_group_tables(B, Hkv, _hp(hc), _hp(goh), n_groups, None, None, None,
+                                  _hp(goff)), "tg_group_tables")
+    table = np.empty(max(1, int(goff[-1])), dtype=np.int32)
+    off = np.empty((B, Hkv), dtype=np.int64)
+    _check(_lib().tg_group_tables(B, Hkv, _hp(hc), _hp(goh), n_groups, _hp(ids), _hp(table),
+                                  _hp(off), _hp(goff)), "tg_group_tables")
+    return table[:int(goff[-1])].copy(), off, goff
+
+
+def tg_place_sequences(seq_bytes, n_gpus: int) -> np.ndarray:
+    b = _h(seq_bytes, np.int64)
+    out = np.empty(b.size, dtype=np.int32)
+    _check(_lib().tg_place_sequences(b.size, _hp(b), n_gpus, _hp(out)), "tg_place_sequences")
+    return out
+
+
+# ------------------------------------------------------------------------------------------
+# Plan
+# ------------------------------------------------------------------------------------------
+
+@dataclass
+class Plan:
+    """Owns a tg_plan handle; destroy() (or garbage collection) frees it."""
+    handle: ctypes.c_void_p
+    shape: tg_shape
+    tiered: bool
+
+    def destroy(self):
+        if self.handle:
+            _lib().tg_plan_destroy(self.handle)
+            self.handle = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def make_shape(B, Hq, Hkv, D, num_pages, num_slow_pages=0, page=16) -> tg_shape:
+    return tg_shape(B, Hq, Hkv, D, page, 0, num_pages, num_slow_pages)
+
+
+def tg_plan_create(shape: tg_shape, kv_len, group_of_head, group_off, fast_len=None,
+                   slow_table_len: int = 0, num_workers: int = 0, min_splits: int = 1,
+                   max_chunk_pages: int = 0, host_only: bool = False, device: int = -1) -> Plan:
+    kv = _h(kv_len, np.int32).reshape(-1)
+    fl = None if fast_len is None else _h(fast_len, np.int32).reshape(-1)
+    goh = _h(group_of_head, np.int32).reshape(-1)
+    goff = _h(group_off, np.int64).reshape(-1)
+    opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device)
+    h = ctypes.c_void_p()
+    _check(_lib().tg_plan_create(ctypes.byref(shape), _hp(kv), _hp(fl), _hp(goh), _hp(goff),
+                                 goff.size - 1, slow_table_len, ctypes.byref(opts),
+                                 ctypes.byref(h)), "tg_plan_create")
+    return Plan(h, shape, fl is not None)
+
+
+def tg_plan_destroy(plan: Plan):
+    plan.destroy()
+
+
+def tg_plan_get_info(plan: Plan) -> dict:
+    info = tg_plan_info()
+    _check(_lib().tg_plan_get_info(plan.handle, ctypes.byref(info)), "tg_plan_get_info")
+    return {f: getattr(info, f) for f, _ in tg_plan_info._fields_ if f != "reserved"}
+
+
+def tg_plan_items(plan: Plan) -> np.ndarray:
+    """int32[n_items, 8]: bh, page_begin, page_end, tier_tokens, slot, flags, worker, 0."""
+    n = tg_plan_get_info(plan)["n_items"]
+    out = np.empty((max(n, 1), 8), dtype=np.int32)
+    _check(_lib().tg_plan_items(plan.handle, _hp(out)), "tg_plan_items")
+    return out[:n]
+
+
+def tg_plan_status(plan: Plan, stream=None) -> int:
+    """Read and clear the device error word (synchronises the stream); returns the status."""
+    return int(_lib().tg_plan_status(plan.handle, _stream(stream)))
+
+
+def tg_plan_timing_enable(plan: Plan, max_calls: int):
+    _check(_lib().tg_plan_timing_enable(plan.handle, max_calls), "tg_plan_timing_enable")
+
+
+def tg_plan_timing_read(plan: Plan):
+    """(n_calls, decode_ms_total, merge_ms_total) of the calls recorded since enable/read."""
+    n = ctypes.c_int32()
+    d = ctypes.c_double()
+    m = ctypes.c_double()
+    _check(_lib().tg_plan_timing_read(plan.handle, ctypes.byref(n), ctypes.byref(d),
+                                      ctypes.byref(m)), "tg_plan_timing_read")
+    return n.value, d.value, m.value
+
+
+# ------------------------------------------------------------------------------------------
+# Device entry points
+# ------------------------------------------------------------------------------------------
+
+def tg_ragged_paged_decode(plan: Plan, q, k_pages, v_pages, page_table, head_page_off,
+                           head_kv_len, group_of_head, scale: float, out, lse, stream=None):
+    _check(_lib().tg_ragged_paged_decode(
+        plan.handle, _dp(q), _dp(k_pages), _dp(v_pages), _dp(page_table), _dp(head_page_off),
+        _dp(head_kv_len), _dp(group_of_head), float(scale), _dp(out), _dp(lse),
+        _stream(stream)), "tg_ragged_paged_decode")
+
+
+def tg_tiered_decode(plan: Plan, q, k_q8, v_q8, k_scale, v_scale, slow_page_table,
+                     slow_head_off, k_fast, v_fast, fast_page_table, fast_head_off, head_kv_len,
+                     head_fast_len, scale: float, out, lse, stream=None):
+    _check(_lib().tg_tiered_decode(
+        plan.handle, _dp(q), _dp(k_q8), _dp(v_q8), _dp(k_scale), _dp(v_scale),
+        _dp(slow_page_table), _dp(slow_head_off), _dp(k_fast), _dp(v_fast),
+        _dp(fast_page_table), _dp(fast_head_off), _dp(head_kv_len), _dp(head_fast_len),
+        float(scale), _dp(out), _dp(lse), _stream(stream)), "tg_tiered_decode")
+
+
+def tg_lse_merge(row_split_off, part_o, part_lse, out, lse, stream=None):
+    n_rows = row_split_off.numel() - 1
+    D = part_o.shape[-1]
+    _check(_lib().tg_lse_merge(n_rows, D, _dp(row_split_off), _dp(part_o), _dp(part_lse),
+                               _dp(out), _dp(lse), _stream(stream)), "tg_lse_merge")
+
+
+def tg_quantize_int8(src, codes, scale, stream=None):
+    D = src.shape[-1]
+    n_rows = src.numel() // D
+    _check(_lib().tg_quantize_int8(n_rows, D, _dp(src), _dp(codes), _dp(scale), _stream(stream)),
+           "tg_quantize_int8")

@@ -1,0 +1,513 @@
+// Host side of libtg: admission-time steps (retained lengths, budget groups, the
+// budget-reservation allocator, group page tables, AOT placement) and the static work-list
+// planner. Pure host C++; the CUDA side lives in tg_kernels.cu.
+#include <algorithm>
+#include <climits>
+#include <cstring>
+#include <deque>
+#include <new>
+#include <numeric>
+#include <unordered_map>
+#include <vector>
+
+#include "tg_internal.h"
+
+// ------------------------------------------------------------------------------------------
+// Status text
+// ------------------------------------------------------------------------------------------
+extern "C" const char *tg_strerror(int s) {
+    switch (s) {
+        case TG_OK: return "ok";
+        case TG_EINVAL: return "invalid argument";
+        case TG_ENOSPC: return "page pool exhausted";
+        case TG_EBADPAGE: return "page id, table row or length outside the plan (pages skipped)";
+        case TG_ECUDA: return "CUDA runtime error";
+        case TG_ETIMEOUT: return "kernel wait timed out";
+        case TG_ENOMEM: return "out of memory";
+        case TG_ENOTFOUND: return "unknown sequence or segment";
+        case TG_EUNSUPPORTED: return "unsupported shape";
+        case TG_EEXIST: return "sequence already reserved";
+        default: return "unknown status";
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Retained length from the budget table ("Tangram": per-head ratio fixed at admission).
+// ------------------------------------------------------------------------------------------
+extern "C" int tg_retained_lengths(int64_t n, const int32_t *full_len, const int32_t *ratio_ppm,
+                                   int32_t *kv_len) {
+    if (n < 0 || (n > 0 && (!full_len || !ratio_ppm || !kv_len))) return TG_EINVAL;
+    for (int64_t i = 0; i < n; ++i)
+        if (ratio_ppm[i] < 0 || ratio_ppm[i] > 1000000) return TG_EINVAL;
+    for (int64_t i = 0; i < n; ++i) {
+        const int64_t L = full_len[i];
+        if (L <= 0) { kv_len[i] = 0; continue; }
+        int64_t r = (static_cast<int64_t>(ratio_ppm[i]) * L + 500000) / 1000000;
+        kv_len[i] = static_cast<int32_t>(std::min<int64_t>(L, std::max<int64_t>(1, r)));
+    }
+    return TG_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Budget groups (Ragged Paging): equal-count quantiles of the budget ranking.
+// ------------------------------------------------------------------------------------------
+extern "C" int tg_budget_groups(int32_t n, const int32_t *budget_ppm, int32_t n_groups,
+                                int32_t *group_of_head) {
+    if (n <= 0 || !budget_ppm || !group_of_head || n_groups < 1 || n_groups > n) return TG_EINVAL;
+    std::vector<int32_t> order(n);
+    std::iota(order.begin(), order.end(), 0);
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int32_t a, int32_t b) { return budget_ppm[a] < budget_ppm[b]; });
+    for (int32_t pos = 0; pos < n; ++pos)
+        group_of_head[order[pos]] = static_cast<int32_t>(static_cast<int64_t>(pos) * n_groups / n);
+    return TG_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Budget-reservation allocator.
+// ------------------------------------------------------------------------------------------
+struct tg_alloc {
+    int64_t num_pages = 0;
+    int32_t page = 16;
+    std::deque<int32_t> free_list;
+    std::vector<int32_t> refs;
+    struct Segment {
+        int32_t n_heads = 0, full = 0;
+        bool alive = false;
+        std::vector<int32_t> pages;  // [n_heads][full]
+    };
+    std::vector<Segment> segs;
+    struct Seq {
+        std::vector<int32_t> priv;    // private pages in allocation order
+        std::vector<int32_t> shared;  // shared page references held
+    };
+    std::unordered_map<int32_t, Seq> seqs;
+
+    void unref(int32_t p) {
+        if (--refs[p] == 0) free_list.push_back(p);
+    }
+};
+
+extern "C" int tg_alloc_create(int64_t num_pages, int32_t page, const int32_t *free_order,
+                               tg_alloc **out) {
+    if (!out || num_pages < 1 || num_pages > INT32_MAX || page < 1) return TG_EINVAL;
+    tg_alloc *a = new (std::nothrow) tg_alloc;
+    if (!a) return TG_ENOMEM;
+    a->num_pages = num_pages;
+    a->page = page;
+    a->refs.assign(static_cast<size_t>(num_pages), 0);
+    std::vector<char> seen(static_cast<size_t>(num_pages), 0);
+    for (int64_t i = 0; i < num_pages; ++i) {
+        const int32_t p = free_order ? free_order[i] : static_cast<int32_t>(i);
+        if (p < 0 || p >= num_pages || seen[p]) { delete a; return TG_EINVAL; }
+        seen[p] = 1;
+        a->free_list.push_back(p);
+    }
+    *out = a;
+    return TG_OK;
+}
+
+extern "C" void tg_alloc_destroy(tg_alloc *a) { delete a; }
+
+extern "C" int64_t tg_alloc_free_pages(const tg_alloc *a) {
+    return a ? static_cast<int64_t>(a->free_list.size()) : -1;
+}
+
+extern "C" int32_t tg_alloc_refcount(const tg_alloc *a, int32_t page_id) {
+    if (!a || page_id < 0 || page_id >= a->num_pages) return -1;
+    return a->refs[page_id];
+}
+
+extern "C" int tg_alloc_share_segment(tg_alloc *a, int32_t n_tokens, int32_t n_heads,
+                                      int32_t *seg_id, int32_t *page_ids) {
+    if (!a || !seg_id || n_tokens < 0 || n_heads < 1) return TG_EINVAL;
+    const int32_t full = n_tokens / a->page;
+    const int64_t need = static_cast<int64_t>(full) * n_heads;
+    if (need > static_cast<int64_t>(a->free_list.size())) return TG_ENOSPC;
+    tg_alloc::Segment s;
+    s.n_heads = n_heads;
+    s.full = full;
+    s.alive = true;
+    s.pages.reserve(static_cast<size_t>(need));
+    for (int64_t i = 0; i < need; ++i) {
+        const int32_t p = a->free_list.front();
+        a->free_list.pop_front();
+        a->refs[p] = 1;  // the segment's own reference
+        s.pages.push_back(p);
+    }
+    if (page_ids) std::memcpy(page_ids, s.pages.data(), sizeof(int32_t) * static_cast<size_t>(need));
+    *seg_id = static_cast<int32_t>(a->segs.size());
+    a->segs.push_back(std::move(s));
+    return TG_OK;
+}
+
+extern "C" int tg_alloc_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads,
+                                const int32_t *kv_len, int32_t n_prefix,
+                                const int32_t *prefix_segs, int32_t *page_ids, int64_t capacity,
+                                int64_t *n_written) {
+    if (!a || n_heads < 1 || !kv_len || n_prefix < 0 || (n_prefix > 0 && !prefix_segs) ||
+        (capacity > 0 && !page_ids) || capacity < 0)
+        return TG_EINVAL;
+    if (a->seqs.count(seq_id)) return TG_EEXIST;
+    int64_t shared_pages = 0;
+    for (int32_t c = 0; c < n_prefix; ++c) {
+        const int32_t s = prefix_segs[c];
+        if (s < 0) continue;
+        if (s >= static_cast<int32_t>(a->segs.size()) || !a->segs[s].alive) return TG_ENOTFOUND;
+        if (a->segs[s].n_heads != n_heads) return TG_EINVAL;
+        shared_pages += a->segs[s].full;
+    }
+    const int64_t shared_tokens = shared_pages * a->page;
+    int64_t priv_total = 0, total = 0;
+    for (int32_t h = 0; h < n_heads; ++h) {
+        if (kv_len[h] < shared_tokens) return TG_EINVAL;
+        const int64_t priv = (kv_len[h] - shared_tokens + a->page - 1) / a->page;
+        priv_total += priv;
+        total += shared_pages + priv;
+    }
+    if (total > capacity) return TG_EINVAL;
+    if (priv_total > static_cast<int64_t>(a->free_list.size())) return TG_ENOSPC;
+
+    tg_alloc::Seq sq;
+    int64_t w = 0;
+    for (int32_t h = 0; h < n_heads; ++h) {
+        for (int32_t c = 0; c < n_prefix; ++c) {
+            const int32_t s = prefix_segs[c];
+            if (s < 0) continue;
+            const tg_alloc::Segment &sg = a->segs[s];
+            for (int32_t p = 0; p < sg.full; ++p) {
+                const int32_t id = sg.pages[static_cast<size_t>(h) * sg.full + p];
+                ++a->refs[id];
+                sq.shared.push_back(id);
+                page_ids[w++] = id;
+            }
+        }
+        const int64_t priv = (kv_len[h] - shared_tokens + a->page - 1) / a->page;
+        for (int64_t p = 0; p < priv; ++p) {
+            const int32_t id = a->free_list.front();
+            a->free_list.pop_front();
+            a->refs[id] = 1;
+            sq.priv.push_back(id);
+            page_ids[w++] = id;
+        }
+    }
+    if (n_written) *n_written = w;
+    a->seqs.emplace(seq_id, std::move(sq));
+    return TG_OK;
+}
+
+extern "C" int tg_alloc_release(tg_alloc *a, int32_t seq_id) {
+    if (!a) return TG_EINVAL;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return TG_ENOTFOUND;
+    for (int32_t p : it->second.priv) a->unref(p);
+    for (int32_t p : it->second.shared) a->unref(p);
+    a->seqs.erase(it);
+    return TG_OK;
+}
+
+extern "C" int tg_alloc_release_segment(tg_alloc *a, int32_t seg_id) {
+    if (!a) return TG_EINVAL;
+    if (seg_id < 0 || seg_id >= static_cast<int32_t>(a->segs.size()) || !a->segs[seg_id].alive)
+        return TG_ENOTFOUND;
+    tg_alloc::Segment &s = a->segs[seg_id];
+    s.alive = false;
+    for (int32_t p : s.pages) a->unref(p);
+    return TG_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Group page tables (Ragged Paging).
+// ------------------------------------------------------------------------------------------
+extern "C" int tg_group_tables(int32_t B, int32_t Hkv, const int32_t *head_count,
+                               const int32_t *group_of_head, int32_t n_groups,
+                               const int32_t *page_ids, int32_t *table, int64_t *head_off,
+                               int64_t *group_off) {
+    if (B < 0 || Hkv < 1 || !head_count || !group_of_head || n_groups < 1 || !group_off)
+        return TG_EINVAL;
+    for (int32_t h = 0; h < Hkv; ++h)
+        if (group_of_head[h] < 0 || group_of_head[h] >= n_groups) return TG_EINVAL;
+    const int64_t BH = static_cast<int64_t>(B) * Hkv;
+    std::vector<int64_t> src(static_cast<size_t>(BH) + 1, 0);
+    for (int64_t i = 0; i < BH; ++i) {
+        if (head_count[i] < 0) return TG_EINVAL;
+        src[i + 1] = src[i] + head_count[i];
+    }
+    if (table && (!page_ids || !head_off)) return TG_EINVAL;
+    int64_t pos = 0;
+    for (int32_t g = 0; g < n_groups; ++g) {
+        group_off[g] = pos;
+        std::vector<int32_t> heads;
+        int64_t Pg = 0;
+        for (int32_t h = 0; h < Hkv; ++h) {
+            if (group_of_head[h] != g) continue;
+            heads.push_back(h);
+            for (int32_t b = 0; b < B; ++b)
+                Pg = std::max<int64_t>(Pg, head_count[static_cast<int64_t>(b) * Hkv + h]);
+        }
+        const int64_t Hg = static_cast<int64_t>(heads.size());
+        if (table) {
+            for (int32_t b = 0; b < B; ++b)
+                for (int64_t j = 0; j < Hg; ++j) {
+                    const int64_t bh = static_cast<int64_t>(b) * Hkv + heads[j];
+                    const int64_t row = pos + (static_cast<int64_t>(b) * Hg + j) * Pg;
+                    head_off[bh] = row;
+                    const int64_t cnt = head_count[bh];
+                    for (int64_t p = 0; p < Pg; ++p)
+                        table[row + p] = p < cnt ? page_ids[src[bh] + p] : -1;
+                }
+        } else if (head_off) {
+            for (int32_t b = 0; b < B; ++b)
+                for (int64_t j = 0; j < Hg; ++j)
+                    head_off[static_cast<int64_t>(b) * Hkv + heads[j]] =
+                        pos + (static_cast<int64_t>(b) * Hg + j) * Pg;
+        }
+        pos += static_cast<int64_t>(B) * Hg * Pg;
+    }
+    group_off[n_groups] = pos;
+    return TG_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// AOT placement of sequences on GPUs (LPT greedy).
+// ------------------------------------------------------------------------------------------
+extern "C" int tg_place_sequences(int32_t n_seq, const int64_t *seq_bytes, int32_t n_gpus,
+                                  int32_t *gpu_of_seq) {
+    if (n_seq < 0 || n_gpus < 1 || (n_seq > 0 && (!seq_bytes || !gpu_of_seq))) return TG_EINVAL;
+    std::vector<int32_t> order(n_seq);
+    std::iota(order.begin(), order.end(), 0);
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int32_t a, int32_t b) { return seq_bytes[a] > seq_bytes[b]; });
+    std::vector<int64_t> load(n_gpus, 0);
+    for (int32_t s : order) {
+        const int32_t g = static_cast<int32_t>(std::min_element(load.begin(), load.end()) - load.begin());
+        gpu_of_seq[s] = g;
+        load[g] += seq_bytes[s];
+    }
+    return TG_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Static work-list planner.
+//
+// Each head's tokens are cut into chunks (per tier; chunks never cross the tier boundary),
+// then the byte cost of the chunks, in (sequence, head, tier, chunk) order, is cut into
+// num_workers contiguous ranges of equal cost. A chunk that straddles a range boundary is
+// cut at the page nearest the boundary. Every resulting (worker, chunk piece) is an item.
+// ------------------------------------------------------------------------------------------
+namespace tg {
+
+int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
+                    int32_t num_workers, int32_t min_splits, int32_t max_chunk_pages) {
+    const tg_shape &s = p->shape;
+    const int64_t BH = static_cast<int64_t>(s.B) * s.Hkv;
+    const int32_t page = s.page;
+    const int64_t bf16_page_cost = 2LL * page * s.D * 2;            // K + V bytes of a page
+    const int64_t i8_page_cost = 2LL * (page * s.D + page * 4);     // codes + fp32 scales
+    const int64_t item_cost = static_cast<int64_t>(p->G) * s.D * 6; // q in + partial out
+
+    struct Chunk {
+        int32_t bh, pb, pe, tier_tokens, flags, kv, fl;
+        int64_t page_cost;
+    };
+    std::vector<Chunk> chunks;
+    p->planned_kv.assign(static_cast<size_t>(BH), 0);
+    int64_t total_pages = 0, kv_bytes = 0;
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        const int32_t n = kv_len[bh];
+        if (n < 0) return TG_EINVAL;
+        p->planned_kv[bh] = n;
+        const int32_t f = fast_len ? std::max(0, std::min(fast_len[bh], n)) : 0;
+        if (fast_len && fast_len[bh] < 0) return TG_EINVAL;
+        struct Run { int32_t tokens, flags; int64_t cost; };
+        Run runs[2];
+        int nr = 0;
+        if (fast_len) {
+            runs[nr++] = {n - f, kItemSlow, i8_page_cost};
+            runs[nr++] = {f, 0, bf16_page_cost};
+            kv_bytes += static_cast<int64_t>(n - f) * 2 * (s.D + 4) + static_cast<int64_t>(f) * 2 * s.D * 2;
+        } else {
+            runs[nr++] = {n, 0, bf16_page_cost};
+            kv_bytes += static_cast<int64_t>(n) * 2 * s.D * 2;
+        }
+        int64_t head_pages = 0;
+        for (int r = 0; r < nr; ++r) head_pages += (runs[r].tokens + page - 1) / page;
+        int64_t cap = max_chunk_pages > 0 ? max_chunk_pages : INT32_MAX;
+        if (min_splits > 1 && head_pages > 0)
+            cap = std::min<int64_t>(cap, std::max<int64_t>(1, head_pages / min_splits));
+        for (int r = 0; r < nr; ++r) {
+            const int32_t pages = (runs[r].tokens + page - 1) / page;
+            if (pages == 0) continue;
+            const int64_t k = (pages + cap - 1) / cap;
+            int32_t at = 0;
+            for (int64_t c = 0; c < k; ++c) {
+                const int32_t sz = static_cast<int32_t>(pages / k + (c < pages % k ? 1 : 0));
+                chunks.push_back({static_cast<int32_t>(bh), at, at + sz, runs[r].tokens,
+                                  runs[r].flags, n, fast_len ? fast_len[bh] : 0, runs[r].cost});
+                at += sz;
+            }
+            total_pages += pages;
+        }
+    }
+    p->kv_bytes = kv_bytes;
+
+    int64_t W = std::max<int64_t>(1, num_workers);
+    W = std::max<int64_t>(1, std::min<int64_t>(W, total_pages / 2));
+    // Cost of all pages plus one item overhead per chunk and per worker cut.
+    long double total_cost = static_cast<long double>(W - 1) * item_cost;
+    for (const Chunk &c : chunks) total_cost += static_cast<long double>(c.pe - c.pb) * c.page_cost + item_cost;
+
+    p->items.clear();
+    p->worker_of_item.clear();
+    int64_t w = 0;
+    long double cum = 0;
+    auto emit = [&](const Chunk &c, int32_t pb, int32_t pe) {
+        Item it{};
+        it.bh = c.bh;
+        it.page_begin = pb;
+        it.page_end = pe;
+        it.tier_tokens = c.tier_tokens;
+        it.slot = -1;
+        it.flags = c.flags;
+        it.kv_len = c.kv;
+        it.fast_len = c.fl;
+        p->items.push_back(it);
+        p->worker_of_item.push_back(static_cast<int32_t>(w));
+        cum += static_cast<long double>(pe - pb) * c.page_cost + item_cost;
+    };
+    for (const Chunk &c : chunks) {
+        int32_t at = c.pb;
+        while (at < c.pe) {
+            if (w == W - 1) { emit(c, at, c.pe); at = c.pe; break; }
+            const long double target = total_cost * static_cast<long double>(w + 1) / W;
+            const long double room = target - cum - item_cost;
+            const int64_t k = room <= 0 ? 0 : static_cast<int64_t>(room / c.page_cost + 0.5L);
+            if (k >= c.pe - at) {
+                emit(c, at, c.pe);
+                at = c.pe;
+            } else if (k >= 1) {
+                emit(c, at, at + static_cast<int32_t>(k));
+                at += static_cast<int32_t>(k);
+                ++w;
+            } else {
+                ++w;
+            }
+        }
+    }
+    p->n_workers = p->items.empty() ? 0 : p->worker_of_item.back() + 1;
+    p->worker_off.assign(static_cast<size_t>(p->n_workers) + 1, 0);
+    for (size_t i = 0; i < p->items.size(); ++i) p->worker_off[p->worker_of_item[i] + 1] = static_cast<int32_t>(i + 1);
+    for (int32_t i = 1; i <= p->n_workers; ++i)
+        p->worker_off[i] = std::max(p->worker_off[i], p->worker_off[i - 1]);
+
+    // Partial slots and the merge list: a head's items are consecutive in the list.
+    std::vector<int32_t> cnt(static_cast<size_t>(BH), 0), first(static_cast<size_t>(BH), -1);
+    for (size_t i = 0; i < p->items.size(); ++i) {
+        const int32_t bh = p->items[i].bh;
+        if (first[bh] < 0) first[bh] = static_cast<int32_t>(i);
+        ++cnt[bh];
+    }
+    p->merge.clear();
+    int64_t slot = 0;
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        if (cnt[bh] == 0) {
+            p->merge.push_back({static_cast<int32_t>(bh), 0, 0, 0});
+        } else if (cnt[bh] > 1) {
+            p->merge.push_back({static_cast<int32_t>(bh), static_cast<int32_t>(slot), cnt[bh], 0});
+            for (int32_t j = 0; j < cnt[bh]; ++j) p->items[first[bh] + j].slot = static_cast<int32_t>(slot++);
+        }
+    }
+    p->n_partials = slot;
+    return TG_OK;
+}
+
+}  // namespace tg
+
+// ------------------------------------------------------------------------------------------
+// Plan creation (host part) and inspection.
+// ------------------------------------------------------------------------------------------
+extern "C" int tg_plan_create(const tg_shape *shape, const int32_t *kv_len,
+                              const int32_t *fast_len, const int32_t *group_of_head,
+                              const int64_t *group_off, int32_t n_groups,
+                              int64_t slow_table_len, const tg_plan_opts *opts,
+                              tg_plan **out) {
+    if (!shape || !kv_len || !out || !group_of_head || !group_off || n_groups < 1) return TG_EINVAL;
+    const tg_shape &s = *shape;
+    if (s.B < 0 || s.Hkv < 1 || s.Hq < 1 || s.Hq % s.Hkv != 0 || s.D < 1 || s.page < 1 ||
+        s.num_pages < 0 || s.num_slow_pages < 0)
+        return TG_EINVAL;
+    const int32_t G = s.Hq / s.Hkv;
+    if (s.page != 16 || (s.D != 64 && s.D != 128) || (G != 1 && G != 2 && G != 4 && G != 8))
+        return TG_EUNSUPPORTED;
+    if (fast_len && s.D != 128) return TG_EUNSUPPORTED;
+    if (s.num_pages > (INT64_C(1) << 28) || s.num_slow_pages > (INT64_C(1) << 28)) return TG_EUNSUPPORTED;
+    for (int32_t h = 0; h < s.Hkv; ++h)
+        if (group_of_head[h] < 0 || group_of_head[h] >= n_groups) return TG_EINVAL;
+    tg_plan_opts o{};
+    o.min_splits = 1;
+    o.device = -1;
+    if (opts) o = *opts;
+    if (o.min_splits < 1) o.min_splits = 1;
+
+    tg_plan *p = new (std::nothrow) tg_plan;
+    if (!p) return TG_ENOMEM;
+    p->shape = s;
+    p->G = G;
+    p->tiered = fast_len != nullptr;
+    p->host_only = o.host_only != 0;
+    p->n_groups = n_groups;
+    p->slow_table_len = slow_table_len;
+    p->group_off.assign(group_off, group_off + n_groups + 1);
+    p->device = o.device;
+
+    int32_t workers = o.num_workers;
+    if (!p->host_only) {
+        int rc = tg::device_num_sms(o.device, &p->num_sms);
+        if (rc != TG_OK) { delete p; return rc; }
+        if (workers <= 0) workers = p->num_sms * tg::kPairs;
+    } else if (workers <= 0) {
+        workers = 148 * tg::kPairs;
+    }
+    int rc = tg::build_work_list(p, kv_len, fast_len, workers, o.min_splits, o.max_chunk_pages);
+    if (rc != TG_OK) { delete p; return rc; }
+    p->grid = (p->n_workers + tg::kPairs - 1) / tg::kPairs;
+    if (!p->host_only) {
+        rc = tg::device_init_plan(p);
+        if (rc != TG_OK) { tg::device_free_plan(p); delete p; return rc; }
+    }
+    *out = p;
+    return TG_OK;
+}
+
+extern "C" void tg_plan_destroy(tg_plan *p) {
+    if (!p) return;
+    if (!p->host_only) tg::device_free_plan(p);
+    delete p;
+}
+
+extern "C" int tg_plan_get_info(const tg_plan *p, tg_plan_info *info) {
+    if (!p || !info) return TG_EINVAL;
+    std::memset(info, 0, sizeof(*info));
+    info->n_items = static_cast<int64_t>(p->items.size());
+    info->n_partials = p->n_partials;
+    info->n_merge = static_cast<int64_t>(p->merge.size());
+    info->n_workers = p->n_workers;
+    info->grid = p->grid;
+    info->block = tg::kThreads;
+    info->smem_bytes = p->smem_bytes;
+    info->stages = p->stages;
+    info->device_bytes = p->dev_bytes;
+    info->kv_bytes = p->kv_bytes;
+    return TG_OK;
+}
+
+extern "C" int tg_plan_items(const tg_plan *p, int32_t *items) {
+    if (!p || !items) return TG_EINVAL;
+    for (size_t i = 0; i < p->items.size(); ++i) {
+        const tg::Item &it = p->items[i];
+        int32_t *o = items + 8 * i;
+        o[0] = it.bh; o[1] = it.page_begin; o[2] = it.page_end; o[3] = it.tier_tokens;
+        o[4] = it.slot; o[5] = it.flags; o[6] = p->worker_of_item[i]; o[7] = 0;
+    }
+    return TG_OK;
+}

@@ -1,0 +1,105 @@
+// Internal declarations shared by the host library (tg_host.cpp) and the CUDA side
+// (tg_kernels.cu) of libtg. Not part of the ABI.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "tg.h"
+
+namespace tg {
+
+// One work item: a contiguous page range of one (sequence, KV head) row in one tier.
+struct Item {
+    int32_t bh;          // b * Hkv + h
+    int32_t page_begin;  // first page (index within the head's row of its tier's table)
+    int32_t page_end;    // one past the last page
+    int32_t tier_tokens; // tokens held by this head's row in this tier (tail-page mask)
+    int32_t slot;        // partial-result slot, -1 = this item writes the final output
+    int32_t flags;       // kItemSlow: INT8 tier
+    int32_t kv_len;      // planned retained length of the head (checked on device)
+    int32_t fast_len;    // planned fast-tier length (tiered plans), else 0
+};
+static_assert(sizeof(Item) == 32, "Item is 32 bytes");
+constexpr int32_t kItemSlow = 1;
+
+// A head whose result is finished by the merge kernel: split over nsplit consecutive slots,
+// or empty (nsplit = 0).
+struct MergeHead {
+    int32_t bh;
+    int32_t first_slot;
+    int32_t nsplit;
+    int32_t pad;
+};
+
+// Device error-word bits.
+constexpr uint32_t kErrBadPage = 1u;   // page id outside the pool
+constexpr uint32_t kErrBadRow = 2u;    // row outside its group table / table
+constexpr uint32_t kErrPlan = 4u;      // device lengths differ from the plan
+constexpr uint32_t kErrTimeout = 8u;   // a bounded wait gave up
+
+// Launch geometry of the decode kernels (see tg_kernels.cu).
+constexpr int kPairs = 4;              // (producer warp, consumer warp) pairs per CTA
+constexpr int kThreads = kPairs * 64;  // threads per CTA
+
+}  // namespace tg
+
+struct tg_plan {
+    tg_shape shape{};
+    int32_t G = 0;
+    bool tiered = false;
+    bool host_only = true;
+    int device = 0;
+    int num_sms = 0;
+    int32_t n_groups = 0;
+    int64_t slow_table_len = 0;
+
+    // host copies
+    std::vector<tg::Item> items;
+    std::vector<int32_t> worker_of_item;
+    std::vector<int32_t> worker_off;  // [n_workers + 1]
+    std::vector<tg::MergeHead> merge;
+    std::vector<int64_t> group_off;   // [n_groups + 1]
+    std::vector<int32_t> planned_kv;  // [B*Hkv]
+    int64_t n_partials = 0;
+    int32_t n_workers = 0;
+    int64_t kv_bytes = 0;
+
+    // launch geometry
+    int32_t grid = 0;
+    int32_t stages = 0;
+    int32_t stage_bytes = 0;
+    int32_t smem_bytes = 0;
+
+    // device state: one allocation carved into these
+    void *dev_base = nullptr;
+    int64_t dev_bytes = 0;
+    tg::Item *d_items = nullptr;
+    int32_t *d_worker_off = nullptr;
+    tg::MergeHead *d_merge = nullptr;
+    int64_t *d_group_off = nullptr;
+    float *d_part_o = nullptr;    // [n_partials][G][D]
+    float *d_part_lse = nullptr;  // [n_partials][G]
+    uint32_t *d_err = nullptr;
+
+    // kernel timing: 3 events per recorded call (cudaEvent_t stored as void*)
+    std::vector<void *> tev;
+    int32_t tev_cap = 0;
+    int32_t tev_count = 0;
+
+    // tensor-map cache keyed by the pool pointers of the last call
+    const void *tm_key[4] = {nullptr, nullptr, nullptr, nullptr};
+    alignas(64) unsigned char tmaps[4][128];
+};
+
+namespace tg {
+// Host planner (tg_host.cpp): fills items / worker_off / merge / n_partials / kv_bytes.
+int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
+                    int32_t num_workers, int32_t min_splits, int32_t max_chunk_pages);
+// Device side (tg_kernels.cu).
+int device_init_plan(tg_plan *p);
+void device_free_plan(tg_plan *p);
+int device_num_sms(int device, int *num_sms);
+void set_cuda_error(const char *what, int code);
+}  // namespace tg

@@ -1,0 +1,1199 @@
+// CUDA side of libtg (sm_100a): split-K ragged / tiered paged decode, the log-sum-exp merge,
+// the INT8 slow-tier quantiser, plan device state and launchers.
+//
+// Decode kernel design (one layer, one step):
+//   * Persistent CTAs of kPairs (producer warp, consumer warp) pairs; each pair is one worker
+//     of the static plan and walks its items (page ranges of one (sequence, KV head) row).
+//   * The producer warp reads the page ids through the table and streams each page's K and V
+//     into a per-pair ring of shared-memory stages with the Tensor Memory Accelerator
+//     (2-D tiled loads, 128-byte swizzle, mbarrier transaction counts; no clusters, no
+//     multicast). The first page of an item also brings the item's G query rows; INT8 pages
+//     also bring their per-token fp32 scales.
+//   * The consumer warp computes S = K q^T for 16 tokens x (up to) 8 query heads with
+//     mma.m16n8k16 (tokens on M, the GQA heads of the KV head on N), an online softmax in
+//     the log2 domain, and O^T += V^T P^T with the head dimension on M. INT8 rows are
+//     converted exactly to fp16 in registers; their scales multiply the score (K) and the
+//     probability (V) in fp32.
+//   * Items that cover a whole head write bf16 out + fp32 lse; split heads write normalised
+//     fp32 partials that the merge kernel combines by log-sum-exp in split order.
+//   * Every wait is bounded (globaltimer); every page id and table row is range-checked
+//     before a copy is issued. Faults turn into bits of the plan's error word.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "tg_internal.h"
+
+namespace tg {
+
+// ------------------------------------------------------------------------------------------
+// Error reporting
+// ------------------------------------------------------------------------------------------
+static thread_local char g_cuda_msg[256] = "";
+
+void set_cuda_error(const char *what, int code) {
+    std::snprintf(g_cuda_msg, sizeof(g_cuda_msg), "%s: %s (%d)", what,
+                  cudaGetErrorString(static_cast<cudaError_t>(code)), code);
+}
+
+#define TG_CUDA_TRY(expr)                                   \
+    do {                                                    \
+        cudaError_t e_ = (expr);                            \
+        if (e_ != cudaSuccess) {                            \
+            set_cuda_error(#expr, static_cast<int>(e_));    \
+            return TG_ECUDA;                                \
+        }                                                   \
+    } while (0)
+
+// ------------------------------------------------------------------------------------------
+// Device helpers (inline PTX)
+// ------------------------------------------------------------------------------------------
+namespace dev {
+
+constexpr uint64_t kWaitNs = 4000000000ull;  // bound of any single wait: 4 s
+constexpr uint64_t kDrainNs = 200000000ull;  // bound of the drain after a timeout: 0.2 s
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase of the given parity; false after `limit` ns.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer();
+    while (!mbar_try_wait(bar, parity))
+        if (global_timer() - t0 > limit) return false;
+    return true;
+}
+
+// 2-D tiled TMA load into this CTA's shared memory, completing on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int32_t x, int32_t y,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// 1-D bulk copy global -> this CTA's shared memory (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(dst),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                          uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t movm_t(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Hardware base-2 exponential and logarithm (PTX ex2.approx / lg2.approx).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+__device__ __forceinline__ float f16_lo(uint32_t v) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xFFFFu)));
+}
+__device__ __forceinline__ float f16_hi(uint32_t v) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
+}
+
+// Four signed 8-bit integers (|x| <= 128) -> two fp16x2, exactly: bias each byte to x + 128,
+// place it in the low mantissa byte of fp16 1024 (0x6400), subtract 1152.
+__device__ __forceinline__ void i8x4_to_f16x4(uint32_t v, uint32_t &lo, uint32_t &hi) {
+    const uint32_t u = v ^ 0x80808080u;
+    uint32_t a, b;
+    asm("prmt.b32 %0, %1, %2, 0x4140;" : "=r"(a) : "r"(u), "r"(0x64646464u));
+    asm("prmt.b32 %0, %1, %2, 0x4342;" : "=r"(b) : "r"(u), "r"(0x64646464u));
+    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+    __half2 ha = __hsub2(*reinterpret_cast<__half2 *>(&a), bias);
+    __half2 hb = __hsub2(*reinterpret_cast<__half2 *>(&b), bias);
+    lo = *reinterpret_cast<uint32_t *>(&ha);
+    hi = *reinterpret_cast<uint32_t *>(&hb);
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a box of 128-byte rows written by TMA
+// with 128-byte swizzle (the box base is 1024-byte aligned).
+__device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {
+    return row * 128u + (((chunk ^ row) & 7u) << 4);
+}
+
+}  // namespace dev
+
+// ------------------------------------------------------------------------------------------
+// Kernel arguments
+// ------------------------------------------------------------------------------------------
+struct DecodeArgs {
+    const Item *items;
+    const int32_t *worker_off;
+    int32_t n_workers;
+    int32_t B, Hq, Hkv, G;
+    int32_t stages, stage_bytes;
+    float scale_log2;                // softmax scale * log2(e)
+    const __nv_bfloat16 *q;          // [B][Hq][D]
+    const int32_t *table;            // bf16 (fast) tier table
+    const int64_t *head_off;         // [B*Hkv]
+    const int32_t *group_of_head;    // [Hkv]; null = bound rows by the whole table
+    const int64_t *group_off;        // [n_groups + 1] (device copy in the plan)
+    int32_t n_groups;
+    const int32_t *slow_table;       // INT8 tier table (tiered)
+    const int64_t *slow_off;         // [B*Hkv] (tiered)
+    int64_t slow_table_len;
+    const float *k_scale, *v_scale;  // [num_slow_pages][16] (tiered)
+    const int32_t *kv_len_dev;       // [B*Hkv]
+    const int32_t *fast_len_dev;     // [B*Hkv] (tiered) or null
+    int64_t num_pages, num_slow_pages;
+    __nv_bfloat16 *out;              // [B][Hq][D]
+    float *lse;                      // [B][Hq]
+    float *part_o;                   // [n_partials][G][D]
+    float *part_lse;                 // [n_partials][G]
+    uint32_t *err;
+};
+
+// Per-stage header written by the producer before it arrives on the stage's full barrier.
+struct StageHdr {
+    int32_t valid;  // valid tokens in this page (0 when the page was skipped)
+    int32_t flags;  // kHdr* bits
+    int32_t bh;
+    int32_t slot;
+};
+constexpr int32_t kHdrSlow = 1, kHdrFirst = 2, kHdrLast = 4, kHdrWorkerLast = 8;
+
+// Shared-memory stage layout (offsets within a stage; D = 128 shown, D = 64 halves the bf16
+// regions): K bf16 [0, KB) as D/64 boxes of 16 rows x 128 B; V bf16 [KB, 2KB); q [2KB, +QB).
+// INT8 pages reuse it: K codes [0, 2048), K scales [2048, 2112), V scales [2112, 2176),
+// V codes [KB, KB + 2048).
+template <int D>
+struct Layout {
+    static constexpr int KB = 16 * D * 2;
+    static constexpr int kI8 = 16 * D;  // one INT8 page of one tensor
+    static constexpr int kKScale = 2048, kVScale = 2112;
+};
+
+// ------------------------------------------------------------------------------------------
+// Decode kernel
+// ------------------------------------------------------------------------------------------
+template <int D, bool TIERED>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_kq,
+                  const __grid_constant__ CUtensorMap tm_vq) {
+    using L = Layout<D>;
+    constexpr int KSTEPS = D / 16;  // k-steps of q.K and m-tiles of P.V
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int pair = warp >> 1;
+    const bool producer = (warp & 1) != 0;
+    const int stages = a.stages;
+    const int worker = blockIdx.x * kPairs + pair;
+
+    unsigned char *ring = smem + static_cast<size_t>(pair) * stages * a.stage_bytes;
+    StageHdr *hdr = reinterpret_cast<StageHdr *>(smem + static_cast<size_t>(kPairs) * stages * a.stage_bytes) +
+                    pair * stages;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(
+                         smem + static_cast<size_t>(kPairs) * stages * a.stage_bytes +
+                         static_cast<size_t>(kPairs) * stages * sizeof(StageHdr)) +
+                     static_cast<size_t>(pair) * stages * 2;
+    volatile int32_t *ctl = reinterpret_cast<volatile int32_t *>(
+                                smem + static_cast<size_t>(kPairs) * stages * a.stage_bytes +
+                                static_cast<size_t>(kPairs) * stages * (sizeof(StageHdr) + 16)) +
+                            pair * 2;  // [0] = pages issued, [1] = abort
+
+    const uint32_t full0 = dev::smem_addr(bars), empty0 = dev::smem_addr(bars + stages);
+    if (lane == 0 && !producer) {
+        for (int s = 0; s < stages; ++s) {
+            dev::mbar_init(full0 + 8 * s, 1);
+            dev::mbar_init(empty0 + 8 * s, 1);
+        }
+        ctl[0] = 0;
+        ctl[1] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (worker >= a.n_workers) return;
+    const int it0 = a.worker_off[worker], it1 = a.worker_off[worker + 1];
+    if (it0 >= it1) return;
+
+    if (producer) {
+        // ================================ producer warp ================================
+        uint32_t seq = 0;
+        for (int it = it0; it < it1; ++it) {
+            const Item item = a.items[it];
+            const int32_t bh = item.bh;
+            const int32_t b = bh / a.Hkv, h = bh - b * a.Hkv;
+            const bool slow = TIERED && (item.flags & kItemSlow);
+            const int32_t row_pages = (item.tier_tokens + 15) >> 4;
+            // Row of this head in its tier's table, bounds-checked.
+            int64_t row;
+            bool row_ok;
+            if (slow) {
+                row = a.slow_off[bh];
+                row_ok = row >= 0 && row + row_pages <= a.slow_table_len;
+            } else {
+                row = a.head_off[bh];
+                int64_t lo = a.group_off[0], hi = a.group_off[a.n_groups];
+                if (a.group_of_head) {
+                    const int32_t g = a.group_of_head[h];
+                    if (g >= 0 && g < a.n_groups) {
+                        lo = a.group_off[g];
+                        hi = a.group_off[g + 1];
+                    } else {
+                        hi = lo - 1;  // invalid group: reject the row
+                    }
+                }
+                row_ok = row >= lo && row + row_pages <= hi;
+            }
+            if (lane == 0) {
+                if (!row_ok) atomicOr(a.err, kErrBadRow);
+                bool plan_ok = a.kv_len_dev[bh] == item.kv_len;
+                if (TIERED) plan_ok = plan_ok && a.fast_len_dev[bh] == item.fast_len;
+                if (!plan_ok) atomicOr(a.err, kErrPlan);
+            }
+            const int32_t *table = slow ? a.slow_table : a.table;
+            const int64_t npool = slow ? a.num_slow_pages : a.num_pages;
+            for (int32_t p0 = item.page_begin; p0 < item.page_end; p0 += 32) {
+                const int32_t cnt = min(32, item.page_end - p0);
+                int32_t pid = -1;
+                if (row_ok && lane < cnt) {
+                    pid = __ldg(table + row + p0 + lane);
+                    if (pid < 0 || pid >= npool) {
+                        atomicOr(a.err, kErrBadPage);
+                        pid = -1;
+                    }
+                }
+                for (int32_t j = 0; j < cnt; ++j) {
+                    const int32_t page_id = __shfl_sync(0xffffffffu, pid, j);
+                    const int32_t pg = p0 + j;
+                    const int stage = seq % stages;
+                    const uint32_t phase = (seq / stages) & 1u;
+                    bool ok = dev::mbar_wait(empty0 + 8 * stage, phase ^ 1u, dev::kWaitNs);
+                    if (!ok || ctl[1]) {
+                        if (lane == 0) { atomicOr(a.err, kErrTimeout); ctl[1] = 1; }
+                        return;
+                    }
+                    if (lane == 0) {
+                        const bool first = pg == item.page_begin;
+                        const bool last = pg == item.page_end - 1;
+                        StageHdr hd;
+                        hd.valid = page_id >= 0 ? min(16, item.tier_tokens - pg * 16) : 0;
+                        hd.flags = (slow ? kHdrSlow : 0) | (first ? kHdrFirst : 0) |
+                                   (last ? kHdrLast : 0) |
+                                   (last && it == it1 - 1 ? kHdrWorkerLast : 0);
+                        hd.bh = bh;
+                        hd.slot = item.slot;
+                        hdr[stage] = hd;
+                        const uint32_t st = dev::smem_addr(ring + static_cast<size_t>(stage) * a.stage_bytes);
+                        const uint32_t fb = full0 + 8 * stage;
+                        const uint32_t qbytes = static_cast<uint32_t>(a.G * D * 2);
+                        uint32_t bytes = first ? qbytes : 0u;
+                        if (page_id >= 0) bytes += slow ? 2u * (L::kI8 + 64u) : 2u * L::KB;
+                        if (bytes == 0) {
+                            dev::mbar_arrive(fb);
+                        } else {
+                            dev::mbar_arrive_expect_tx(fb, bytes);
+                            if (first)
+                                dev::bulk_load(st + 2 * L::KB,
+                                               a.q + (static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * a.G) * D,
+                                               qbytes, fb);
+                            if (page_id >= 0) {
+                                const int32_t y = page_id * 16;
+                                if (slow) {
+                                    dev::tma_load_2d(st, &tm_kq, 0, y, fb);
+                                    dev::tma_load_2d(st + L::KB, &tm_vq, 0, y, fb);
+                                    dev::bulk_load(st + L::kKScale, a.k_scale + static_cast<int64_t>(page_id) * 16, 64, fb);
+                                    dev::bulk_load(st + L::kVScale, a.v_scale + static_cast<int64_t>(page_id) * 16, 64, fb);
+                                } else {
+#pragma unroll
+                                    for (int bx = 0; bx < D / 64; ++bx) {
+                                        dev::tma_load_2d(st + bx * 2048, &tm_k, bx * 64, y, fb);
+                                        dev::tma_load_2d(st + L::KB + bx * 2048, &tm_v, bx * 64, y, fb);
+                                    }
+                                }
+                            }
+                        }
+                        ctl[0] = static_cast<int32_t>(seq + 1);
+                    }
+                    __syncwarp();
+                    ++seq;
+                }
+            }
+        }
+        return;
+    }
+
+    // ================================ consumer warp ================================
+    const int g = lane >> 2, t = lane & 3;
+    uint32_t qf[KSTEPS][2];
+    float o[KSTEPS][4];
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    bool item_slow = false;
+    uint32_t seq = 0;
+
+    while (true) {
+        const int stage = seq % stages;
+        const uint32_t phase = (seq / stages) & 1u;
+        if (!dev::mbar_wait(full0 + 8 * stage, phase, dev::kWaitNs)) {
+            // Timed out: stop the producer and drain the copies it issued, then leave.
+            if (lane == 0) {
+                atomicOr(a.err, kErrTimeout);
+                ctl[1] = 1;
+            }
+            __syncwarp();
+            const uint32_t issued = static_cast<uint32_t>(ctl[0]);
+            for (uint32_t s = seq; s < issued; ++s)
+                dev::mbar_wait(full0 + 8 * (s % stages), (s / stages) & 1u, dev::kDrainNs);
+            return;
+        }
+        const StageHdr hd = hdr[stage];
+        const unsigned char *st = ring + static_cast<size_t>(stage) * a.stage_bytes;
+        const uint32_t st_a = dev::smem_addr(st);
+        const bool slow = TIERED && (hd.flags & kHdrSlow);
+
+        if (hd.flags & kHdrFirst) {
+            // New item: query fragments (B operand, N = head g of this KV head) and state.
+            item_slow = slow;
+            const unsigned char *qs = st + 2 * L::KB;
+#pragma unroll
+            for (int j = 0; j < KSTEPS; ++j) {
+                if (g < a.G) {
+                    if (!slow) {
+                        qf[j][0] = *reinterpret_cast<const uint32_t *>(qs + (g * D + 16 * j + 2 * t) * 2);
+                        qf[j][1] = *reinterpret_cast<const uint32_t *>(qs + (g * D + 16 * j + 2 * t + 8) * 2);
+                    } else {
+                        // INT8 tier: fp16 q, k-slots (2t, 2t+1, 2t+8, 2t+9) <-> d = 16j + 4t + 0..3
+                        const uint2 v = *reinterpret_cast<const uint2 *>(qs + (g * D + 16 * j + 4 * t) * 2);
+                        qf[j][0] = dev::pack_f16(dev::bf16_lo(v.x), dev::bf16_hi(v.x));
+                        qf[j][1] = dev::pack_f16(dev::bf16_lo(v.y), dev::bf16_hi(v.y));
+                    }
+                } else {
+                    qf[j][0] = 0u;
+                    qf[j][1] = 0u;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < KSTEPS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+            m0 = m1 = -INFINITY;
+            l0 = l1 = 0.f;
+        }
+
+        const int valid = hd.valid;
+        // ---- S = K q^T : 16 tokens x 8 heads ----
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        float ks0 = 1.f, ks1 = 1.f, vs0 = 1.f, vs1 = 1.f;
+        if (!slow) {
+#pragma unroll
+            for (int j = 0; j < KSTEPS; ++j) {
+                const int mi = lane >> 3;
+                const uint32_t row = (mi & 1) * 8 + (lane & 7);
+                const uint32_t cc = 2 * j + (mi >> 1);  // 16-byte chunk over the row of D
+                uint32_t a0, a1, a2, a3;
+                dev::ldsm_x4(st_a + (cc >> 3) * 2048 + dev::swz(row, cc & 7), a0, a1, a2, a3);
+                dev::mma_bf16(s, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+            }
+        } else if (TIERED) {
+#pragma unroll
+            for (int j = 0; j < KSTEPS; j += 2) {
+                const int mi = lane >> 3;
+                const uint32_t row = (mi & 1) * 8 + (lane & 7);
+                const uint32_t cc = j + (mi >> 1);
+                uint32_t r0, r1, r2, r3;
+                dev::ldsm_x4(st_a + dev::swz(row, cc), r0, r1, r2, r3);
+                uint32_t a0, a1, a2, a3;
+                dev::i8x4_to_f16x4(r0, a0, a2);
+                dev::i8x4_to_f16x4(r1, a1, a3);
+                dev::mma_f16(s, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+                dev::i8x4_to_f16x4(r2, a0, a2);
+                dev::i8x4_to_f16x4(r3, a1, a3);
+                dev::mma_f16(s, a0, a1, a2, a3, qf[j + 1][0], qf[j + 1][1]);
+            }
+            const float *ksc = reinterpret_cast<const float *>(st + L::kKScale);
+            const float *vsc = reinterpret_cast<const float *>(st + L::kVScale);
+            ks0 = ksc[g];
+            ks1 = ksc[g + 8];
+            vs0 = vsc[g];
+            vs1 = vsc[g + 8];
+        }
+        // s[0]: token g head 2t; s[1]: token g head 2t+1; s[2]/s[3]: token g+8.
+        const bool v0 = g < valid, v1 = g + 8 < valid;
+        float x0 = v0 ? s[0] * ks0 * a.scale_log2 : -INFINITY;
+        float x1 = v0 ? s[1] * ks0 * a.scale_log2 : -INFINITY;
+        float x2 = v1 ? s[2] * ks1 * a.scale_log2 : -INFINITY;
+        float x3 = v1 ? s[3] * ks1 * a.scale_log2 : -INFINITY;
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        // Lazy rescale: the running max moves only when a tile exceeds it by more than the
+        // threshold (2^8 for bf16 probabilities; exact for the fp16 INT8 path).
+        const float thr = slow ? 0.f : 8.f;
+        const bool up0 = mx0 > m0 + thr, up1 = mx1 > m1 + thr;
+        if (__any_sync(0xffffffffu, up0 || up1)) {
+            const float n0 = up0 ? mx0 : m0, n1 = up1 ? mx1 : m1;
+            const float c0 = (m0 == -INFINITY) ? 0.f : dev::ex2(m0 - n0);
+            const float c1 = (m1 == -INFINITY) ? 0.f : dev::ex2(m1 - n1);
+#pragma unroll
+            for (int i = 0; i < KSTEPS; ++i) {
+                o[i][0] *= c0;
+                o[i][1] *= c1;
+                o[i][2] *= c0;
+                o[i][3] *= c1;
+            }
+            l0 *= c0;
+            l1 *= c1;
+            m0 = n0;
+            m1 = n1;
+        }
+        const float p0 = x0 == -INFINITY ? 0.f : dev::ex2(x0 - m0);
+        const float p1 = x1 == -INFINITY ? 0.f : dev::ex2(x1 - m1);
+        const float p2 = x2 == -INFINITY ? 0.f : dev::ex2(x2 - m0);
+        const float p3 = x3 == -INFINITY ? 0.f : dev::ex2(x3 - m1);
+
+        if (!slow) {
+            const uint32_t r0 = dev::pack_bf16(p0, p1), r1 = dev::pack_bf16(p2, p3);
+            l0 += dev::bf16_lo(r0) + dev::bf16_lo(r1);
+            l1 += dev::bf16_hi(r0) + dev::bf16_hi(r1);
+            const uint32_t b0 = dev::movm_t(r0), b1 = dev::movm_t(r1);
+            // token masks of this thread's A-fragment halves (tokens 2t, 2t+1 | 2t+8, 2t+9)
+            const uint32_t mk01 = (2 * t < valid ? 0xFFFFu : 0u) | (2 * t + 1 < valid ? 0xFFFF0000u : 0u);
+            const uint32_t mk23 = (2 * t + 8 < valid ? 0xFFFFu : 0u) | (2 * t + 9 < valid ? 0xFFFF0000u : 0u);
+            const bool tail = valid < 16;
+#pragma unroll
+            for (int i = 0; i < KSTEPS; ++i) {
+                const int mi = lane >> 3;
+                const uint32_t row = (mi >> 1) * 8 + (lane & 7);  // token
+                const uint32_t cc = 2 * i + (mi & 1);             // d chunk
+                uint32_t a0, a1, a2, a3;
+                dev::ldsm_x4_t(st_a + L::KB + (cc >> 3) * 2048 + dev::swz(row, cc & 7), a0, a1, a2, a3);
+                if (tail) {
+                    a0 &= mk01;
+                    a1 &= mk01;
+                    a2 &= mk23;
+                    a3 &= mk23;
+                }
+                dev::mma_bf16(o[i], a0, a1, a2, a3, b0, b1);
+            }
+        } else if (TIERED) {
+            // p' = p * v_scale (fp32) -> fp16; the normaliser keeps the unscaled p.
+            l0 += p0 + p2;
+            l1 += p1 + p3;
+            const float q0 = v0 ? p0 * vs0 : 0.f, q1 = v0 ? p1 * vs0 : 0.f;
+            const float q2 = v1 ? p2 * vs1 : 0.f, q3 = v1 ? p3 * vs1 : 0.f;
+            const uint32_t b0 = dev::movm_t(dev::pack_f16(q0, q1));
+            const uint32_t b1 = dev::movm_t(dev::pack_f16(q2, q3));
+#pragma unroll
+            for (int i = 0; i < KSTEPS; i += 2) {
+                const int mi = lane >> 3;
+                const uint32_t row = (mi & 1) * 8 + (lane & 7);  // token
+                const uint32_t cc = i + (mi >> 1);
+                uint32_t r0, r1, r2, r3;
+                dev::ldsm_x4(st_a + L::KB + dev::swz(row, cc), r0, r1, r2, r3);
+                // r0: tokens 0-7 chunk i; r1: tokens 8-15 chunk i; r2/r3: chunk i+1
+                uint32_t x0l, x0h, x1l, x1h;
+                dev::i8x4_to_f16x4(r0, x0l, x0h);
+                dev::i8x4_to_f16x4(r1, x1l, x1h);
+                dev::mma_f16(o[i], dev::movm_t(x0l), dev::movm_t(x0h), dev::movm_t(x1l),
+                             dev::movm_t(x1h), b0, b1);
+                dev::i8x4_to_f16x4(r2, x0l, x0h);
+                dev::i8x4_to_f16x4(r3, x1l, x1h);
+                dev::mma_f16(o[i + 1], dev::movm_t(x0l), dev::movm_t(x0h), dev::movm_t(x1l),
+                             dev::movm_t(x1h), b0, b1);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(empty0 + 8 * stage);
+
+        if (hd.flags & kHdrLast) {
+            // ---- finish the item ----
+            float L0 = l0, L1 = l1;
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                L0 += __shfl_xor_sync(0xffffffffu, L0, off);
+                L1 += __shfl_xor_sync(0xffffffffu, L1, off);
+            }
+            const float inv0 = L0 > 0.f ? 1.f / L0 : 0.f, inv1 = L1 > 0.f ? 1.f / L1 : 0.f;
+            constexpr float kLn2 = 0.69314718055994530942f;
+            const float lse0 = L0 > 0.f ? (m0 + dev::lg2(L0)) * kLn2 : -INFINITY;
+            const float lse1 = L1 > 0.f ? (m1 + dev::lg2(L1)) * kLn2 : -INFINITY;
+            const int32_t b = hd.bh / a.Hkv, h = hd.bh - b * a.Hkv;
+            const int n0 = 2 * t, n1 = 2 * t + 1;
+            if (hd.slot < 0) {
+                __nv_bfloat16 *ob = a.out + (static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * a.G) * D;
+#pragma unroll
+                for (int i = 0; i < KSTEPS; ++i) {
+                    int dlo, dhi;
+                    if (!item_slow) {
+                        dlo = 16 * i + g;
+                        dhi = dlo + 8;
+                    } else {
+                        dlo = 16 * i + 4 * (g >> 1) + (g & 1);
+                        dhi = dlo + 2;
+                    }
+                    if (n0 < a.G) {
+                        ob[n0 * D + dlo] = __float2bfloat16_rn(o[i][0] * inv0);
+                        ob[n0 * D + dhi] = __float2bfloat16_rn(o[i][2] * inv0);
+                    }
+                    if (n1 < a.G) {
+                        ob[n1 * D + dlo] = __float2bfloat16_rn(o[i][1] * inv1);
+                        ob[n1 * D + dhi] = __float2bfloat16_rn(o[i][3] * inv1);
+                    }
+                }
+                if (g == 0) {
+                    float *lb = a.lse + static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * a.G;
+                    if (n0 < a.G) lb[n0] = lse0;
+                    if (n1 < a.G) lb[n1] = lse1;
+                }
+            } else {
+                float *po = a.part_o + static_cast<int64_t>(hd.slot) * a.G * D;
+#pragma unroll
+                for (int i = 0; i < KSTEPS; ++i) {
+                    int dlo, dhi;
+                    if (!item_slow) {
+                        dlo = 16 * i + g;
+                        dhi = dlo + 8;
+                    } else {
+                        dlo = 16 * i + 4 * (g >> 1) + (g & 1);
+                        dhi = dlo + 2;
+                    }
+                    if (n0 < a.G) {
+                        po[n0 * D + dlo] = o[i][0] * inv0;
+                        po[n0 * D + dhi] = o[i][2] * inv0;
+                    }
+                    if (n1 < a.G) {
+                        po[n1 * D + dlo] = o[i][1] * inv1;
+                        po[n1 * D + dhi] = o[i][3] * inv1;
+                    }
+                }
+                if (g == 0) {
+                    float *pl = a.part_lse + static_cast<int64_t>(hd.slot) * a.G;
+                    if (n0 < a.G) pl[n0] = lse0;
+                    if (n1 < a.G) pl[n1] = lse1;
+                }
+            }
+        }
+        ++seq;
+        if (hd.flags & kHdrWorkerLast) break;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Merge of the plan's split heads (and zero output for empty heads): one warp per query row.
+// ------------------------------------------------------------------------------------------
+__global__ void plan_merge_kernel(const MergeHead *mh, int32_t n_merge, int32_t G, int32_t D,
+                                  int32_t Hq, int32_t Hkv, const float *part_o,
+                                  const float *part_lse, __nv_bfloat16 *out, float *lse) {
+    const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (r >= static_cast<int64_t>(n_merge) * G) return;
+    const MergeHead m = mh[r / G];
+    const int n = static_cast<int>(r % G);
+    const int32_t b = m.bh / Hkv, h = m.bh - b * Hkv;
+    __nv_bfloat16 *ob = out + ((static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * G + n) * D);
+    float mx = -INFINITY;
+    for (int j = 0; j < m.nsplit; ++j) mx = fmaxf(mx, part_lse[static_cast<int64_t>(m.first_slot + j) * G + n]);
+    if (mx == -INFINITY) {
+        for (int d = lane; d < D; d += 32) ob[d] = __float2bfloat16_rn(0.f);
+        if (lane == 0) lse[static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * G + n] = -INFINITY;
+        return;
+    }
+    float sum = 0.f;
+    for (int j = 0; j < m.nsplit; ++j) sum += expf(part_lse[static_cast<int64_t>(m.first_slot + j) * G + n] - mx);
+    const float tot = mx + logf(sum);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < m.nsplit; ++j) {
+        const int64_t sl = m.first_slot + j;
+        const float w = expf(part_lse[sl * G + n] - tot);
+        const float *po = part_o + (sl * G + n) * D;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int d = lane + 32 * k;
+            if (d < D) acc[k] += w * po[d];
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int d = lane + 32 * k;
+        if (d < D) ob[d] = __float2bfloat16_rn(acc[k]);
+    }
+    if (lane == 0) lse[static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * G + n] = tot;
+}
+
+// Generic merge (exported as tg_lse_merge): rows with contiguous split ranges.
+__global__ void lse_merge_kernel(int64_t n_rows, int32_t D, const int64_t *off, const float *po,
+                                 const float *pl, __nv_bfloat16 *out, float *lse) {
+    const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (r >= n_rows) return;
+    const int64_t j0 = off[r], j1 = off[r + 1];
+    float mx = -INFINITY;
+    for (int64_t j = j0; j < j1; ++j) mx = fmaxf(mx, pl[j]);
+    if (mx == -INFINITY) {
+        for (int d = lane; d < D; d += 32) out[r * D + d] = __float2bfloat16_rn(0.f);
+        if (lane == 0) lse[r] = -INFINITY;
+        return;
+    }
+    float sum = 0.f;
+    for (int64_t j = j0; j < j1; ++j) sum += expf(pl[j] - mx);
+    const float tot = mx + logf(sum);
+    for (int d = lane; d < D; d += 32) {
+        float acc = 0.f;
+        for (int64_t j = j0; j < j1; ++j) acc += expf(pl[j] - tot) * po[j * D + d];
+        out[r * D + d] = __float2bfloat16_rn(acc);
+    }
+    if (lane == 0) lse[r] = tot;
+}
+
+// ------------------------------------------------------------------------------------------
+// INT8 quantiser: one warp per row of D bf16 values.
+// ------------------------------------------------------------------------------------------
+template <int D>
+__global__ void quantize_kernel(int64_t n_rows, const __nv_bfloat16 *src, int8_t *codes,
+                                float *scale) {
+    constexpr int PER = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < n_rows; r += warps) {
+        float x[PER];
+        float amax = 0.f;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            x[k] = __bfloat162float(src[r * D + lane * PER + k]);
+            amax = fmaxf(amax, fabsf(x[k]));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        const float sc = __fdiv_rn(amax, 127.f);
+        int8_t c[PER];
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            int v = 0;
+            if (amax != 0.f) v = max(-127, min(127, __float2int_rn(__fdiv_rn(x[k], sc))));
+            c[k] = static_cast<int8_t>(v);
+        }
+#pragma unroll
+        for (int k = 0; k < PER; ++k) codes[r * D + lane * PER + k] = c[k];
+        if (lane == 0) scale[r] = sc;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Host: tensor maps, plan device state, launchers
+// ------------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// Tensor map over a pool of pages [rows = pages * 16][inner] with 128-byte swizzled boxes of
+// box_inner elements x 16 rows.
+static int make_pool_map(CUtensorMap *tm, const void *base, CUtensorMapDataType dt, int elem,
+                         uint64_t inner, uint64_t rows, uint32_t box_inner) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        set_cuda_error("cuTensorMapEncodeTiled unavailable", 0);
+        return TG_ECUDA;
+    }
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elem)};
+    cuuint32_t box[2] = {box_inner, 16};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_cuda_msg, sizeof(g_cuda_msg), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+        return TG_ECUDA;
+    }
+    return TG_OK;
+}
+
+int device_num_sms(int device, int *num_sms) {
+    int dev = device;
+    if (dev < 0) TG_CUDA_TRY(cudaGetDevice(&dev));
+    TG_CUDA_TRY(cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev));
+    return TG_OK;
+}
+
+static constexpr int kSmemBudget = 232448;  // 227 KB opt-in dynamic shared memory per CTA
+
+template <int D, bool TIERED>
+static int set_smem_attr(int bytes) {
+    TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<D, TIERED>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+    return TG_OK;
+}
+
+int device_init_plan(tg_plan *p) {
+    const tg_shape &s = p->shape;
+    int cur = 0;
+    TG_CUDA_TRY(cudaGetDevice(&cur));
+    if (p->device < 0) p->device = cur;
+    if (p->device != cur) TG_CUDA_TRY(cudaSetDevice(p->device));
+
+    // Stage geometry.
+    const int KB = 16 * s.D * 2;
+    const int QB = ((p->G * s.D * 2) + 1023) / 1024 * 1024;
+    p->stage_bytes = 2 * KB + QB;
+    const int per_stage_extra = static_cast<int>(sizeof(StageHdr)) + 16;  // header + 2 barriers
+    int stages = (kSmemBudget - 1024 - kPairs * 8) / (kPairs * (p->stage_bytes + per_stage_extra));
+    stages = stages > 8 ? 8 : stages;
+    if (stages < 2) {
+        if (p->device != cur) cudaSetDevice(cur);
+        return TG_EUNSUPPORTED;
+    }
+    p->stages = stages;
+    p->smem_bytes = 1024 + kPairs * stages * (p->stage_bytes + per_stage_extra) + kPairs * 8;
+
+    int rc = TG_OK;
+    if (s.D == 128 && !p->tiered) rc = set_smem_attr<128, false>(p->smem_bytes);
+    else if (s.D == 128 && p->tiered) rc = set_smem_attr<128, true>(p->smem_bytes);
+    else if (s.D == 64 && !p->tiered) rc = set_smem_attr<64, false>(p->smem_bytes);
+    else rc = TG_EUNSUPPORTED;
+    if (rc != TG_OK) {
+        if (p->device != cur) cudaSetDevice(cur);
+        return rc;
+    }
+
+    // One device allocation for the plan.
+    auto al = [](int64_t x) { return (x + 255) / 256 * 256; };
+    const int64_t n_items = static_cast<int64_t>(p->items.size());
+    const int64_t b_items = al(n_items * static_cast<int64_t>(sizeof(Item)));
+    const int64_t b_woff = al((p->n_workers + 1) * 4LL);
+    const int64_t b_merge = al(static_cast<int64_t>(p->merge.size()) * static_cast<int64_t>(sizeof(MergeHead)));
+    const int64_t b_goff = al((p->n_groups + 1) * 8LL);
+    const int64_t b_po = al(p->n_partials * p->G * s.D * 4LL);
+    const int64_t b_pl = al(p->n_partials * p->G * 4LL);
+    const int64_t b_err = 256;
+    p->dev_bytes = b_items + b_woff + b_merge + b_goff + b_po + b_pl + b_err;
+    cudaError_t e = cudaMalloc(&p->dev_base, static_cast<size_t>(p->dev_bytes));
+    if (e != cudaSuccess) {
+        set_cuda_error("cudaMalloc(plan)", static_cast<int>(e));
+        p->dev_base = nullptr;
+        if (p->device != cur) cudaSetDevice(cur);
+        return TG_ENOMEM;
+    }
+    char *base = static_cast<char *>(p->dev_base);
+    p->d_items = reinterpret_cast<Item *>(base);
+    base += b_items;
+    p->d_worker_off = reinterpret_cast<int32_t *>(base);
+    base += b_woff;
+    p->d_merge = reinterpret_cast<MergeHead *>(base);
+    base += b_merge;
+    p->d_group_off = reinterpret_cast<int64_t *>(base);
+    base += b_goff;
+    p->d_part_o = reinterpret_cast<float *>(base);
+    base += b_po;
+    p->d_part_lse = reinterpret_cast<float *>(base);
+    base += b_pl;
+    p->d_err = reinterpret_cast<uint32_t *>(base);
+
+    rc = TG_OK;
+    auto up = [&](void *dst, const void *src, int64_t bytes) {
+        if (bytes <= 0 || rc != TG_OK) return;
+        cudaError_t ee = cudaMemcpy(dst, src, static_cast<size_t>(bytes), cudaMemcpyHostToDevice);
+        if (ee != cudaSuccess) {
+            set_cuda_error("cudaMemcpy(plan)", static_cast<int>(ee));
+            rc = TG_ECUDA;
+        }
+    };
+    up(p->d_items, p->items.data(), n_items * static_cast<int64_t>(sizeof(Item)));
+    up(p->d_worker_off, p->worker_off.data(), (p->n_workers + 1) * 4LL);
+    up(p->d_merge, p->merge.data(), static_cast<int64_t>(p->merge.size()) * static_cast<int64_t>(sizeof(MergeHead)));
+    up(p->d_group_off, p->group_off.data(), (p->n_groups + 1) * 8LL);
+    if (rc == TG_OK) {
+        cudaError_t ee = cudaMemset(p->d_err, 0, 4);
+        if (ee != cudaSuccess) { set_cuda_error("cudaMemset(plan)", static_cast<int>(ee)); rc = TG_ECUDA; }
+    }
+    if (p->device != cur) cudaSetDevice(cur);
+    return rc;
+}
+
+static void timing_free(tg_plan *p) {
+    for (void *e : p->tev) cudaEventDestroy(static_cast<cudaEvent_t>(e));
+    p->tev.clear();
+    p->tev_cap = 0;
+    p->tev_count = 0;
+}
+
+void device_free_plan(tg_plan *p) {
+    timing_free(p);
+    if (p->dev_base) {
+        int cur = 0;
+        cudaGetDevice(&cur);
+        if (p->device >= 0 && p->device != cur) cudaSetDevice(p->device);
+        cudaFree(p->dev_base);
+        if (p->device >= 0 && p->device != cur) cudaSetDevice(cur);
+        p->dev_base = nullptr;
+    }
+}
+
+static bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+static int get_map(tg_plan *p, int idx, const void *base, CUtensorMapDataType dt, int elem,
+                   uint64_t pages, uint32_t box_inner) {
+    if (p->tm_key[idx] == base) return TG_OK;
+    int rc = make_pool_map(reinterpret_cast<CUtensorMap *>(p->tmaps[idx]), base, dt, elem,
+                           static_cast<uint64_t>(p->shape.D), pages * 16, box_inner);
+    if (rc == TG_OK) p->tm_key[idx] = base;
+    return rc;
+}
+
+static int check_device(const tg_plan *p) {
+    int cur = 0;
+    TG_CUDA_TRY(cudaGetDevice(&cur));
+    return cur == p->device ? TG_OK : TG_EINVAL;
+}
+
+// Timing hook: event k (0 = before decode, 1 = before merge, 2 = after merge) of this call.
+static void timing_mark(tg_plan *p, int k, cudaStream_t stream) {
+    if (p->tev_count >= p->tev_cap) return;
+    cudaEventRecord(static_cast<cudaEvent_t>(p->tev[3 * p->tev_count + k]), stream);
+    if (k == 2) ++p->tev_count;
+}
+
+static int launch_merge(tg_plan *p, void *out, float *lse, cudaStream_t stream) {
+    timing_mark(p, 1, stream);
+    if (p->merge.empty()) {
+        timing_mark(p, 2, stream);
+        return TG_OK;
+    }
+    const int64_t rows = static_cast<int64_t>(p->merge.size()) * p->G;
+    const int threads = 256;
+    const int64_t blocks = (rows * 32 + threads - 1) / threads;
+    plan_merge_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        p->d_merge, static_cast<int32_t>(p->merge.size()), p->G, p->shape.D, p->shape.Hq,
+        p->shape.Hkv, p->d_part_o, p->d_part_lse, static_cast<__nv_bfloat16 *>(out), lse);
+    TG_CUDA_TRY(cudaGetLastError());
+    timing_mark(p, 2, stream);
+    return TG_OK;
+}
+
+static DecodeArgs base_args(const tg_plan *p, const void *q, const int32_t *kv, float scale,
+                            void *out, float *lse) {
+    DecodeArgs a{};
+    a.items = p->d_items;
+    a.worker_off = p->d_worker_off;
+    a.n_workers = p->n_workers;
+    a.B = p->shape.B;
+    a.Hq = p->shape.Hq;
+    a.Hkv = p->shape.Hkv;
+    a.G = p->G;
+    a.stages = p->stages;
+    a.stage_bytes = p->stage_bytes;
+    a.scale_log2 = scale * 1.44269504088896340736f;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.group_off = p->d_group_off;
+    a.n_groups = p->n_groups;
+    a.kv_len_dev = kv;
+    a.num_pages = p->shape.num_pages;
+    a.num_slow_pages = p->shape.num_slow_pages;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.lse = lse;
+    a.part_o = p->d_part_o;
+    a.part_lse = p->d_part_lse;
+    a.err = p->d_err;
+    return a;
+}
+
+}  // namespace tg
+
+// ------------------------------------------------------------------------------------------
+// ABI entry points (device)
+// ------------------------------------------------------------------------------------------
+using namespace tg;
+
+extern "C" const char *tg_last_cuda_error(void) { return g_cuda_msg; }
+
+extern "C" int tg_ragged_paged_decode(tg_plan *p, const void *q, const void *k_pages,
+                                      const void *v_pages, const int32_t *page_table,
+                                      const int64_t *head_page_off, const int32_t *head_kv_len,
+                                      const int32_t *group_of_head, float scale, void *out,
+                                      float *lse, tg_stream stream_) {
+    if (!p || p->host_only || p->tiered) return TG_EINVAL;
+    if (!q || !out || !lse || !head_kv_len || !aligned16(q) || !aligned16(out) || !aligned16(lse))
+        return TG_EINVAL;
+    const bool any_items = !p->items.empty();
+    if (any_items && (!k_pages || !v_pages || !page_table || !head_page_off || !group_of_head ||
+                      !aligned16(k_pages) || !aligned16(v_pages) || p->shape.num_pages < 1))
+        return TG_EINVAL;
+    int rc = check_device(p);
+    if (rc != TG_OK) return rc;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (any_items) {
+        rc = get_map(p, 0, k_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
+        if (rc == TG_OK) rc = get_map(p, 1, v_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
+        if (rc != TG_OK) return rc;
+        DecodeArgs a = base_args(p, q, head_kv_len, scale, out, lse);
+        timing_mark(p, 0, stream);
+        a.table = page_table;
+        a.head_off = head_page_off;
+        a.group_of_head = group_of_head;
+        const CUtensorMap &tk = *reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
+        const CUtensorMap &tv = *reinterpret_cast<const CUtensorMap *>(p->tmaps[1]);
+        if (p->shape.D == 128)
+            decode_kernel<128, false><<<p->grid, kThreads, p->smem_bytes, stream>>>(a, tk, tv, tk, tv);
+        else
+            decode_kernel<64, false><<<p->grid, kThreads, p->smem_bytes, stream>>>(a, tk, tv, tk, tv);
+        TG_CUDA_TRY(cudaGetLastError());
+    } else {
+        timing_mark(p, 0, stream);
+    }
+    return launch_merge(p, out, lse, stream);
+}
+
+extern "C" int tg_tiered_decode(tg_plan *p, const void *q, const int8_t *k_q8,
+                                const int8_t *v_q8, const float *k_scale, const float *v_scale,
+                                const int32_t *slow_page_table, const int64_t *slow_head_off,
+                                const void *k_fast, const void *v_fast,
+                                const int32_t *fast_page_table, const int64_t *fast_head_off,
+                                const int32_t *head_kv_len, const int32_t *head_fast_len,
+                                float scale, void *out, float *lse, tg_stream stream_) {
+    if (!p || p->host_only || !p->tiered) return TG_EINVAL;
+    if (!q || !out || !lse || !head_kv_len || !head_fast_len || !aligned16(q) || !aligned16(out) ||
+        !aligned16(lse))
+        return TG_EINVAL;
+    bool has_slow = false, has_fast = false;
+    for (const Item &it : p->items) (it.flags & kItemSlow ? has_slow : has_fast) = true;
+    if (has_slow && (!k_q8 || !v_q8 || !k_scale || !v_scale || !slow_page_table || !slow_head_off ||
+                     !aligned16(k_q8) || !aligned16(v_q8) || !aligned16(k_scale) ||
+                     !aligned16(v_scale) || p->shape.num_slow_pages < 1))
+        return TG_EINVAL;
+    if (has_fast && (!k_fast || !v_fast || !fast_page_table || !fast_head_off ||
+                     !aligned16(k_fast) || !aligned16(v_fast) || p->shape.num_pages < 1))
+        return TG_EINVAL;
+    int rc = check_device(p);
+    if (rc != TG_OK) return rc;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!p->items.empty()) {
+        if (has_fast) {
+            rc = get_map(p, 0, k_fast, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
+            if (rc == TG_OK) rc = get_map(p, 1, v_fast, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
+        }
+        if (rc == TG_OK && has_slow) {
+            rc = get_map(p, 2, k_q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p->shape.num_slow_pages, 128);
+            if (rc == TG_OK) rc = get_map(p, 3, v_q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p->shape.num_slow_pages, 128);
+        }
+        if (rc != TG_OK) return rc;
+        DecodeArgs a = base_args(p, q, head_kv_len, scale, out, lse);
+        timing_mark(p, 0, stream);
+        a.table = fast_page_table;
+        a.head_off = fast_head_off;
+        a.group_of_head = nullptr;
+        a.slow_table = slow_page_table;
+        a.slow_off = slow_head_off;
+        a.slow_table_len = p->slow_table_len;
+        a.k_scale = k_scale;
+        a.v_scale = v_scale;
+        a.fast_len_dev = head_fast_len;
+        // The fast tier's rows are bounded by its whole table [group_off[0], group_off[n]).
+        const CUtensorMap *maps = reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
+        decode_kernel<128, true><<<p->grid, kThreads, p->smem_bytes, stream>>>(
+            a, maps[has_fast ? 0 : 2], maps[has_fast ? 1 : 3], maps[has_slow ? 2 : 0],
+            maps[has_slow ? 3 : 1]);
+        TG_CUDA_TRY(cudaGetLastError());
+    } else {
+        timing_mark(p, 0, stream);
+    }
+    return launch_merge(p, out, lse, stream);
+}
+
+extern "C" int tg_plan_status(tg_plan *p, tg_stream stream_) {
+    if (!p || p->host_only) return TG_EINVAL;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    uint32_t err = 0;
+    TG_CUDA_TRY(cudaMemcpyAsync(&err, p->d_err, 4, cudaMemcpyDeviceToHost, stream));
+    TG_CUDA_TRY(cudaStreamSynchronize(stream));
+    TG_CUDA_TRY(cudaMemsetAsync(p->d_err, 0, 4, stream));
+    TG_CUDA_TRY(cudaStreamSynchronize(stream));
+    if (err & kErrTimeout) return TG_ETIMEOUT;
+    if (err & (kErrBadPage | kErrBadRow | kErrPlan)) return TG_EBADPAGE;
+    return TG_OK;
+}
+
+extern "C" int tg_lse_merge(int64_t n_rows, int32_t D, const int64_t *row_split_off,
+                            const float *part_o, const float *part_lse, void *out, float *lse,
+                            tg_stream stream_) {
+    if (n_rows < 0 || D < 1 || D > 4096) return TG_EINVAL;
+    if (n_rows == 0) return TG_OK;
+    if (!row_split_off || !out || !lse) return TG_EINVAL;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    const int threads = 256;
+    const int64_t blocks = (n_rows * 32 + threads - 1) / threads;
+    lse_merge_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        n_rows, D, row_split_off, part_o, part_lse, static_cast<__nv_bfloat16 *>(out), lse);
+    TG_CUDA_TRY(cudaGetLastError());
+    return TG_OK;
+}
+
+extern "C" int tg_quantize_int8(int64_t n_rows, int32_t D, const void *src, int8_t *codes,
+                                float *scale, tg_stream stream_) {
+    if (n_rows < 0 || (D != 64 && D != 128)) return n_rows < 0 ? TG_EINVAL : TG_EUNSUPPORTED;
+    if (n_rows == 0) return TG_OK;
+    if (!src || !codes || !scale) return TG_EINVAL;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int threads = 256;
+    int64_t blocks = (n_rows * 32 + threads - 1) / threads;
+    if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
+    if (D == 128)
+        quantize_kernel<128><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+            n_rows, static_cast<const __nv_bfloat16 *>(src), codes, scale);
+    else
+        quantize_kernel<64><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+            n_rows, static_cast<const __nv_bfloat16 *>(src), codes, scale);
+    TG_CUDA_TRY(cudaGetLastError());
+    return TG_OK;
+}
+
+extern "C" int tg_plan_timing_enable(tg_plan *p, int32_t max_calls) {
+    if (!p || p->host_only || max_calls < 0) return TG_EINVAL;
+    timing_free(p);
+    if (max_calls == 0) return TG_OK;
+    p->tev.assign(static_cast<size_t>(max_calls) * 3, nullptr);
+    for (auto &e : p->tev) {
+        cudaEvent_t ev;
+        cudaError_t r = cudaEventCreate(&ev);
+        if (r != cudaSuccess) {
+            set_cuda_error("cudaEventCreate", static_cast<int>(r));
+            for (void *x : p->tev)
+                if (x) cudaEventDestroy(static_cast<cudaEvent_t>(x));
+            p->tev.clear();
+            return TG_ECUDA;
+        }
+        e = ev;
+    }
+    p->tev_cap = max_calls;
+    p->tev_count = 0;
+    return TG_OK;
+}
+
+extern "C" int tg_plan_timing_read(tg_plan *p, int32_t *n_calls, double *decode_ms,
+                                   double *merge_ms) {
+    if (!p || !n_calls || !decode_ms || !merge_ms) return TG_EINVAL;
+    *n_calls = p->tev_count;
+    *decode_ms = 0.0;
+    *merge_ms = 0.0;
+    if (p->tev_count == 0) return TG_OK;
+    TG_CUDA_TRY(cudaEventSynchronize(static_cast<cudaEvent_t>(p->tev[3 * p->tev_count - 1])));
+    for (int32_t i = 0; i < p->tev_count; ++i) {
+        float a = 0.f, b = 0.f;
+        TG_CUDA_TRY(cudaEventElapsedTime(&a, static_cast<cudaEvent_t>(p->tev[3 * i]),
+                                         static_cast<cudaEvent_t>(p->tev[3 * i + 1])));
+        TG_CUDA_TRY(cudaEventElapsedTime(&b, static_cast<cudaEvent_t>(p->tev[3 * i + 1]),
+                                         static_cast<cudaEvent_t>(p->tev[3 * i + 2])));
+        *decode_ms += a;
+        *merge_ms += b;
+    }
+    p->tev_count = 0;
+    return TG_OK;
+}

@@ -1,0 +1,276 @@
+"""CPU tests of the C ABI: the library loads and exports every declared symbol, and its host
+steps (retained lengths, groups, reservation, group tables, placement, the planner) agree bit
+for bit with the oracle's own derivation. No device calls."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import non_uniform_paged_flash_b200 as tg
+import oracle
+import synth
+from non_uniform_paged_flash_b200 import workload
+from tests import _oracle_side as ors
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_library_exports_every_declared_symbol():
+    hdr = open(os.path.join(ROOT, "include", "tg.h")).read()
+    hdr = re.sub(r"/\*.*?\*/", "", hdr, flags=re.S)
+    declared = set(re.findall(r"\b(tg_[a-z0-9_]+)\s*\(", hdr))
+    assert declared, "no declarations parsed"
+    lib = tg.load()
+    for name in sorted(declared):
+        assert hasattr(lib, name), f"libtg.so does not export {name}"
+    assert declared == set(tg.ABI_SYMBOLS), declared ^ set(tg.ABI_SYMBOLS)
+
+
+def test_strerror_covers_codes():
+    for code in range(10):
+        assert tg.load().tg_strerror(code).decode() != "unknown status"
+
+
+def test_retained_lengths_match_oracle():
+    rng = np.random.default_rng(20)
+    L = rng.integers(-3, 300_000, 20_000).astype(np.int32)
+    r = rng.integers(0, 1_000_001, 20_000).astype(np.int32)
+    np.testing.assert_array_equal(tg.tg_retained_lengths(L, r), oracle.retained_lengths(L, r))
+    with pytest.raises(tg.TGError):
+        tg.tg_retained_lengths([10], [1_000_001])
+
+
+def test_budget_groups_match_oracle():
+    rng = np.random.default_rng(21)
+    for n, G in [(8, 4), (256, 8), (13, 5), (8, 8), (1, 1)]:
+        b = rng.integers(0, 50, n).astype(np.int32)   # many ties
+        np.testing.assert_array_equal(tg.tg_budget_groups(b, G), oracle.budget_groups(b, G))
+    with pytest.raises(tg.TGError):
+        tg.tg_budget_groups([1, 2], 3)
+
+
+def _lib_reservation(num_pages, order, kv, segs=(), chain=None, page=16):
+    a = tg.tg_alloc_create(num_pages, page, order)
+    try:
+        seg_ids = []
+        seg_pages = []
+        for s in segs:
+            sid, ids = tg.tg_alloc_share_segment(a, s, kv.shape[1], page)
+            seg_ids.append(sid)
+            seg_pages.append(ids.reshape(-1))
+        out = []
+        for b in range(kv.shape[0]):
+            pre = [] if chain is None else [seg_ids[c] if c >= 0 else -1 for c in chain[b]]
+            out.append(tg.tg_alloc_reserve(a, b, kv[b], pre, page))
+        return np.concatenate(out), (np.concatenate(seg_pages) if seg_pages else np.zeros(0, np.int32))
+    finally:
+        tg.tg_alloc_destroy(a)
+
+
+def test_reservation_matches_oracle_plain_and_prefix():
+    rng = np.random.default_rng(22)
+    kv = rng.integers(0, 400, (11, 3)).astype(np.int32)
+    need = int(((kv + 15) // 16).sum())
+    order = rng.permutation(need + 5).astype(np.int32)
+    ids, _ = _lib_reservation(need + 5, order, kv)
+    oids, _, _ = oracle.reservation_layout(need + 5, order, 16, kv)
+    np.testing.assert_array_equal(ids, oids)
+    # prefix sharing with partial segments and an absent chain entry
+    segs = [100, 37, 64]
+    chain = np.array([[0, 1], [0, 2], [0, -1], [-1, 2], [0, 1]])
+    shared = np.array([sum(segs[c] // 16 * 16 for c in row if c >= 0) for row in chain])
+    kv = (shared[:, None] + rng.integers(0, 70, (5, 2))).astype(np.int32)
+    order = rng.permutation(400).astype(np.int32)
+    ids, segp = _lib_reservation(400, order, kv, segs, chain)
+    oids, _, osegp = oracle.reservation_layout(400, order, 16, kv, segs, chain)
+    np.testing.assert_array_equal(ids, oids)
+    np.testing.assert_array_equal(segp, osegp)
+
+
+def test_reservation_is_all_or_nothing():
+    a = tg.tg_alloc_create(10, 16, np.arange(10)[::-1])
+    try:
+        tg.tg_alloc_reserve(a, 0, [40, 16])                       # 3 + 1 pages
+        assert tg.tg_alloc_free_pages(a) == 6
+        with pytest.raises(tg.TGError) as e:
+            tg.tg_alloc_reserve(a, 1, [64, 64])                   # needs 8 > 6
+        assert e.value.status == tg.TG_ENOSPC
+        assert tg.tg_alloc_free_pages(a) == 6                     # unchanged
+        ids = tg.tg_alloc_reserve(a, 1, [32, 1])                  # same as if no failure
+        np.testing.assert_array_equal(ids, [5, 4, 3])
+        with pytest.raises(tg.TGError) as e:
+            tg.tg_alloc_reserve(a, 1, [1])
+        assert e.value.status == tg.TG_EEXIST
+        with pytest.raises(tg.TGError) as e:
+            tg.tg_alloc_release(a, 7)
+        assert e.value.status == tg.TG_ENOTFOUND
+    finally:
+        tg.tg_alloc_destroy(a)
+
+
+def test_free_order_must_be_a_permutation():
+    with pytest.raises(tg.TGError):
+        tg.tg_alloc_create(4, 16, [0, 1, 1, 2])
+    with pytest.raises(tg.TGError):
+        tg.tg_alloc_create(3, 16, [0, 1, 3])
+
+
+def test_shared_segment_refcounts_and_release_order():
+    a = tg.tg_alloc_create(40, 16)
+    try:
+        sid, sp = tg.tg_alloc_share_segment(a, 40, 2, 16)         # 2 full pages per head
+        np.testing.assert_array_equal(sp, [[0, 1], [2, 3]])
+        r0 = tg.tg_alloc_reserve(a, 0, [50, 33], [sid])          # shared 32 tokens
+        r1 = tg.tg_alloc_reserve(a, 1, [32, 40], [sid])
+        np.testing.assert_array_equal(r0, [0, 1, 4, 5, 2, 3, 6])
+        np.testing.assert_array_equal(r1, [0, 1, 2, 3, 7])
+        for p in (0, 1, 2, 3):
+            assert tg.tg_alloc_refcount(a, p) == 3                # segment + 2 readers
+        assert tg.tg_alloc_refcount(a, 4) == 1
+        tg.tg_alloc_release(a, 0)
+        assert tg.tg_alloc_refcount(a, 0) == 2 and tg.tg_alloc_refcount(a, 4) == 0
+        free_before = tg.tg_alloc_free_pages(a)
+        tg.tg_alloc_release_segment(a, sid)
+        assert tg.tg_alloc_free_pages(a) == free_before           # reader 1 still holds them
+        tg.tg_alloc_release(a, 1)
+        assert all(tg.tg_alloc_refcount(a, p) == 0 for p in range(8))
+        assert tg.tg_alloc_free_pages(a) == 40
+        # released pages are appended at the back, in release order: the front is unchanged
+        ids = tg.tg_alloc_reserve(a, 2, [16])
+        np.testing.assert_array_equal(ids, [8])
+        with pytest.raises(tg.TGError):
+            tg.tg_alloc_reserve(a, 3, [16], [sid])               # dead segment
+    finally:
+        tg.tg_alloc_destroy(a)
+
+
+def test_group_tables_match_oracle():
+    rng = np.random.default_rng(23)
+    for B, H, G in [(7, 8, 4), (3, 5, 5), (4, 4, 1), (6, 8, 8)]:
+        cnt = rng.integers(0, 9, (B, H)).astype(np.int32)
+        goh = rng.integers(0, G, H).astype(np.int32)
+        ids = rng.permutation(int(cnt.sum()) + 3)[: int(cnt.sum())].astype(np.int32)
+        t, off, goff = tg.tg_group_tables(cnt, goh, G, ids)
+        ot, ooff, ogoff = oracle.group_tables(goh, G, ids, cnt)
+        np.testing.assert_array_equal(t, ot)
+        np.testing.assert_array_equal(goff, ogoff)
+        # head_off of empty groups' heads is only meaningful where the head has pages
+        np.testing.assert_array_equal(off, ooff)
+
+
+def test_place_sequences_match_oracle():
+    rng = np.random.default_rng(24)
+    for n, g in [(64, 2), (513, 8), (5, 7), (1000, 3)]:
+        b = rng.integers(0, 10**7, n)
+        b[::7] = b[0]                                              # ties
+        np.testing.assert_array_equal(tg.tg_place_sequences(b, g), oracle.place_sequences(b, g))
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
+def test_small_workload_layout_matches_oracle(cfg):
+    sp = synth.small(cfg)
+    for layer in range(min(sp.layers, 3)):
+        ors.assert_same_layout(workload.layout(sp, layer), ors.layout(sp, layer))
+
+
+@pytest.mark.parametrize("cfg", [2, 4, 5])
+def test_full_size_layout_matches_oracle(cfg):
+    sp = synth.preset(cfg)
+    ors.assert_same_layout(workload.layout(sp, 0), ors.layout(sp, 0))
+
+
+def test_full_size_layout_matches_oracle_multi_layer():
+    sp = synth.preset(3)
+    for layer in (0, 31):
+        ors.assert_same_layout(workload.layout(sp, layer), ors.layout(sp, layer))
+
+
+# ---------------------------------------------------------------------------------------
+# Planner (host-only plans)
+# ---------------------------------------------------------------------------------------
+
+def _plan(sp, lay, **kw):
+    shape = tg.make_shape(sp.B, sp.Hq, sp.Hkv, sp.D, lay.num_pages, lay.num_slow_pages, sp.page)
+    return tg.tg_plan_create(shape, lay.kv_len, lay.group_of_head, lay.group_off,
+                             fast_len=lay.fast_len,
+                             slow_table_len=0 if lay.slow_table is None else lay.slow_table.size,
+                             host_only=True, **kw)
+
+
+def _check_coverage(sp, lay, items, min_splits=1, max_chunk=0):
+    """Every (head, tier, page) is covered exactly once; items stay in one tier; slots of a
+    split head are consecutive in item order; single-item heads write the final output."""
+    kv = lay.kv_len.reshape(-1).astype(np.int64)
+    fl = None if lay.fast_len is None else lay.fast_len.reshape(-1).astype(np.int64)
+    seen = {}
+    for bh, pb, pe, tier_tok, slot, flags, worker, _ in items:
+        assert 0 <= pb < pe
+        slow = bool(flags & 1)
+        n = kv[bh] if fl is None else (kv[bh] - min(fl[bh], kv[bh]) if slow else min(fl[bh], kv[bh]))
+        assert tier_tok == n
+        assert pe <= -(-n // 16)
+        if max_chunk:
+            assert pe - pb <= max_chunk
+        for p in range(pb, pe):
+            key = (bh, slow, p)
+            assert key not in seen, key
+            seen[key] = slot
+    want = 0
+    for bh in range(kv.size):
+        if fl is None:
+            want += -(-kv[bh] // 16)
+        else:
+            f = min(fl[bh], kv[bh])
+            want += -(-(kv[bh] - f) // 16) + -(-f // 16)
+    assert len(seen) == want
+    by_head = {}
+    for row in items:
+        by_head.setdefault(int(row[0]), []).append(int(row[4]))
+    for bh, slots in by_head.items():
+        if len(slots) == 1:
+            assert slots == [-1]
+        else:
+            assert slots == list(range(slots[0], slots[0] + len(slots)))
+            if min_splits > 1:
+                assert len(slots) >= min(min_splits, sum(1 for r in items if r[0] == bh))
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("workers", [1, 7, 592])
+def test_plan_coverage(cfg, workers):
+    sp = synth.small(cfg)
+    lay = workload.layout(sp, 0)
+    p = _plan(sp, lay, num_workers=workers)
+    items = tg.tg_plan_items(p)
+    _check_coverage(sp, lay, items)
+    info = tg.tg_plan_get_info(p)
+    assert info["n_items"] == len(items) and info["n_workers"] <= workers
+
+
+def test_plan_min_splits_and_chunk_cap():
+    sp = synth.preset(5)
+    lay = workload.layout(sp, 0)
+    p = _plan(sp, lay, num_workers=592, min_splits=64, max_chunk_pages=128)
+    items = tg.tg_plan_items(p)
+    _check_coverage(sp, lay, items, max_chunk=128)
+    for bh in range(sp.B * sp.Hkv):
+        assert (items[:, 0] == bh).sum() >= 64                   # >= 64 chunks per head
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+def test_plan_balances_bytes_across_workers(cfg):
+    sp = synth.preset(cfg)
+    lay = workload.layout(sp, 0)
+    W = 592
+    kw = dict(min_splits=64, max_chunk_pages=128) if cfg == 5 else {}
+    p = _plan(sp, lay, num_workers=W, **kw)
+    items = tg.tg_plan_items(p)
+    _check_coverage(sp, lay, items, **({"max_chunk": 128} if cfg == 5 else {}))
+    page_bytes = np.where(items[:, 5] & 1, 2 * (16 * sp.D + 64), 2 * 16 * sp.D * 2)
+    work = np.zeros(W, np.float64)
+    np.add.at(work, items[:, 6], (items[:, 2] - items[:, 1]) * page_bytes)
+    assert items[:, 6].max() + 1 == W
+    # equal-cost contiguous ranges: every worker within a few bf16 pages of the mean
+    assert work.max() - work.mean() <= 4 * 2 * 16 * sp.D * 2
+    assert work.mean() - work.min() <= 4 * 2 * 16 * sp.D * 2

@@ -156,7 +156,18 @@ typedef struct tg_plan_opts {
     int32_t host_only;        /* 1: build the work list on the host only (inspection; decode
                                  calls reject such a plan); 0: also create device state */
     int32_t device;           /* CUDA device ordinal, -1 = current */
-    int32_t reserved[3];
+    int32_t static_permille;  /* share of the bytes assigned to workers ahead of time, in
+                                 1/1000 (0 = default 800; 1000 = all static); the rest is
+                                 cut into dynamic items that workers take in order */
+    int32_t dyn_chunk_pages;  /* pages per dynamic item, at most (0 = default 16) */
+    int32_t early_prologue;   /* decode kernels are launched as programmatic dependents (CUDA
+                                 programmatic dependent launch) of the preceding kernel in the
+                                 stream. 0 (default): they wait for it before doing anything.
+                                 1: before waiting they already read this plan and the page
+                                 tables, head offsets, lengths and group map; queries, K/V and
+                                 every output are touched only after the wait. Use 1 only if no
+                                 preceding kernel that triggers its dependents early writes
+                                 those tables (this library's own kernels never do). */
 } tg_plan_opts;
 
 /* Build a plan. kv_len[B*Hkv] (host): retained tokens per (sequence, KV head); the decode
@@ -166,8 +177,12 @@ typedef struct tg_plan_opts {
  * tg_group_tables) bound every row of the bf16 (fast) table to its group table; for a tiered
  * plan slow_table_len bounds the INT8 tier's table (ignored otherwise).
  * Each head's tokens are cut into chunks (min_splits, max_chunk_pages; chunks never cross a
- * tier boundary), and the byte cost of all chunks is partitioned into num_workers equal
- * contiguous ranges; a head cut into several items is merged by log-sum-exp after the decode.
+ * tier boundary). The first static_permille of the chunks' byte cost is partitioned into
+ * num_workers equal contiguous ranges assigned ahead of time (at least ~8 pages per worker;
+ * fewer workers for tiny batches); the rest is cut into dynamic items of at most
+ * dyn_chunk_pages pages that workers take from a shared ticket when their own range is done
+ * (absorbing per-SM bandwidth differences). A head cut into several items is merged
+ * by log-sum-exp inside the decode kernel.
  * The plan owns one device allocation (work list, merge list, partial results, error word),
  * made here; nothing is allocated per call. */
 int tg_plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,
@@ -178,7 +193,9 @@ void tg_plan_destroy(tg_plan *p);
 typedef struct tg_plan_info {
     int64_t n_items;          /* work items */
     int64_t n_partials;       /* items that write a partial result (heads with > 1 item) */
-    int64_t n_merge;          /* heads finished by the merge kernel (split or empty) */
+    int64_t n_merge;          /* heads split over several items (merged in the kernel) */
+    int64_t n_empty;          /* heads with no retained token (out = 0, lse = -inf) */
+    int64_t n_dynamic;        /* items taken from the shared ticket at run time */
     int32_t n_workers;        /* workers that have items */
     int32_t grid;             /* CTAs of the decode kernel */
     int32_t block;            /* threads per CTA */
@@ -191,22 +208,34 @@ typedef struct tg_plan_info {
 int tg_plan_get_info(const tg_plan *p, tg_plan_info *info);
 
 /* Work list export for inspection: items (host, n_items x 8 int32): per item
- * {b*Hkv + h, page_begin, page_end, tier_tokens, partial slot (-1 = final), flags (bit 0 =
- * INT8 tier), worker, 0}; page indices are within the head's row of its tier's table. */
+ * {b*Hkv + h, page_begin, page_end, tier_tokens, partial slot (-1 = final), INT8 tier (0/1),
+ * worker (-1 = dynamic), merge-list index (-1 = final)}; page indices are within the head's
+ * row of its tier's table. */
 int tg_plan_items(const tg_plan *p, int32_t *items);
 
 /* Read and clear the plan's device error word after the work queued on stream: returns
- * TG_OK, TG_EBADPAGE or TG_ETIMEOUT. Synchronises the stream (a debugging aid). */
+ * TG_OK, TG_EBADPAGE or TG_ETIMEOUT. Synchronises the stream (a debugging aid). After a
+ * timeout it also resets the split heads' arrival tickets, so the plan can be used again. */
 int tg_plan_status(tg_plan *p, tg_stream stream);
 
 /* Kernel timing (a profiling aid). With max_calls > 0, the next max_calls decode calls on this
  * plan record CUDA events on their stream before the decode kernel, between it and the merge
- * kernel, and after the merge; later calls record nothing. The events are created here (no
- * device memory); max_calls = 0 destroys them. tg_plan_timing_read waits for the last
- * recorded event, returns the number of calls recorded and the summed decode-kernel and
- * merge-kernel times in milliseconds, and restarts the count. */
+ * kernel, and after the merge kernel (a recorded call gives up the merge kernel's launch
+ * overlap); later calls record nothing. The events are created here (no device memory);
+ * max_calls = 0 destroys them. tg_plan_timing_read waits for the last recorded event, returns
+ * the number of calls recorded and the summed decode-kernel and merge-kernel times in
+ * milliseconds, and restarts the count. */
 int tg_plan_timing_enable(tg_plan *p, int32_t max_calls);
 int tg_plan_timing_read(tg_plan *p, int32_t *n_calls, double *decode_ms, double *merge_ms);
+
+/* Worker timeline (a profiling aid). With on = 1 the plan allocates n_workers x 8 uint64
+ * device words (here, not per call) and every later decode call records, per worker: the
+ * global timer (ns) at CTA start, first copy issued, first page ready, stop marker seen and
+ * worker done; then the number of dynamic items it took, the number of split heads it merged
+ * and the ns it spent merging. tg_plan_trace_read synchronises the stream and copies the
+ * last call's words to trace (host, n_workers x 8). on = 0 frees the buffer. */
+int tg_plan_trace_enable(tg_plan *p, int32_t on);
+int tg_plan_trace_read(tg_plan *p, uint64_t *trace, tg_stream stream);
 
 /* =====================================================================================
  * Decode entry points (device).
@@ -226,9 +255,11 @@ int tg_plan_timing_read(tg_plan *p, int32_t *n_calls, double *decode_ms, double 
  *               plan's kv_len); group_of_head device int32 [Hkv]
  *   scale       softmax scale applied in fp32 (e.g. 1/sqrt(D))
  *   out         device bf16 [B][Hq][D];  lse device fp32 [B][Hq] (natural log)
- * Reads each page once per item with the Tensor Memory Accelerator; computes q.K and P.V on
- * tensor cores (bf16 in, fp32 accumulate; P rounded to bf16); writes out/lse for single-item
- * heads and partials for split heads, then runs the merge. */
+ * One kernel launch: reads each page once with the Tensor Memory Accelerator; computes q.K
+ * and P.V on tensor cores (bf16 in, fp32 accumulate; P rounded to bf16); heads covered by one
+ * item write out/lse directly; split heads write one partial per item, and a second kernel
+ * (a programmatic dependent launch, so its launch overlaps the decode's tail) merges them by
+ * log-sum-exp in split order, so results are deterministic. */
 int tg_ragged_paged_decode(tg_plan *plan, const void *q, const void *k_pages,
                            const void *v_pages, const int32_t *page_table,
                            const int64_t *head_page_off, const int32_t *head_kv_len,

@@ -43,12 +43,15 @@ class tg_shape(ctypes.Structure):
 class tg_plan_opts(ctypes.Structure):
     _fields_ = [("num_workers", ctypes.c_int32), ("min_splits", ctypes.c_int32),
                 ("max_chunk_pages", ctypes.c_int32), ("host_only", ctypes.c_int32),
-                ("device", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+                ("device", ctypes.c_int32), ("static_permille", ctypes.c_int32),
+                ("dyn_chunk_pages", ctypes.c_int32), ("early_prologue", ctypes.c_int32)]
 
 
 class tg_plan_info(ctypes.Structure):
     _fields_ = [("n_items", ctypes.c_int64), ("n_partials", ctypes.c_int64),
-                ("n_merge", ctypes.c_int64), ("n_workers", ctypes.c_int32),
+                ("n_merge", ctypes.c_int64), ("n_empty", ctypes.c_int64),
+                ("n_dynamic", ctypes.c_int64),
+                ("n_workers", ctypes.c_int32),
                 ("grid", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("smem_bytes", ctypes.c_int32), ("stages", ctypes.c_int32),
                 ("reserved", ctypes.c_int32), ("device_bytes", ctypes.c_int64),
@@ -82,6 +85,8 @@ _SIGS = [
     ("tg_plan_status", ctypes.c_int, [_P, _P]),
     ("tg_plan_timing_enable", ctypes.c_int, [_P, _I32]),
     ("tg_plan_timing_read", ctypes.c_int, [_P, _P, _P, _P]),
+    ("tg_plan_trace_enable", ctypes.c_int, [_P, _I32]),
+    ("tg_plan_trace_read", ctypes.c_int, [_P, _P, _P]),
     ("tg_ragged_paged_decode", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _F32, _P, _P, _P]),
     ("tg_tiered_decode", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                         _F32, _P, _P, _P]),
@@ -266,12 +271,15 @@ def make_shape(B, Hq, Hkv, D, num_pages, num_slow_pages=0, page=16) -> tg_shape:
 
 def tg_plan_create(shape: tg_shape, kv_len, group_of_head, group_off, fast_len=None,
                    slow_table_len: int = 0, num_workers: int = 0, min_splits: int = 1,
-                   max_chunk_pages: int = 0, host_only: bool = False, device: int = -1) -> Plan:
+                   max_chunk_pages: int = 0, host_only: bool = False, device: int = -1,
+                   static_permille: int = 0, dyn_chunk_pages: int = 0,
+                   early_prologue: bool = False) -> Plan:
     kv = _h(kv_len, np.int32).reshape(-1)
     fl = None if fast_len is None else _h(fast_len, np.int32).reshape(-1)
     goh = _h(group_of_head, np.int32).reshape(-1)
     goff = _h(group_off, np.int64).reshape(-1)
-    opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device)
+    opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
+                        static_permille, dyn_chunk_pages, int(early_prologue))
     h = ctypes.c_void_p()
     _check(_lib().tg_plan_create(ctypes.byref(shape), _hp(kv), _hp(fl), _hp(goh), _hp(goff),
                                  goff.size - 1, slow_table_len, ctypes.byref(opts),
@@ -290,7 +298,8 @@ def tg_plan_get_info(plan: Plan) -> dict:
 
 
 def tg_plan_items(plan: Plan) -> np.ndarray:
-    """int32[n_items, 8]: bh, page_begin, page_end, tier_tokens, slot, flags, worker, 0."""
+    """int32[n_items, 8]: bh, page_begin, page_end, tier_tokens, slot, int8 tier, worker (-1 =
+    dynamic), merge index (-1 for items that write the final output)."""
     n = tg_plan_get_info(plan)["n_items"]
     out = np.empty((max(n, 1), 8), dtype=np.int32)
     _check(_lib().tg_plan_items(plan.handle, _hp(out)), "tg_plan_items")
@@ -314,6 +323,20 @@ def tg_plan_timing_read(plan: Plan):
     _check(_lib().tg_plan_timing_read(plan.handle, ctypes.byref(n), ctypes.byref(d),
                                       ctypes.byref(m)), "tg_plan_timing_read")
     return n.value, d.value, m.value
+
+
+def tg_plan_trace_enable(plan: Plan, on: bool = True):
+    _check(_lib().tg_plan_trace_enable(plan.handle, int(on)), "tg_plan_trace_enable")
+
+
+def tg_plan_trace_read(plan: Plan, stream=None) -> np.ndarray:
+    """uint64[n_workers, 8] of the last call: global-timer stamps (ns) of CTA start, first copy
+    issued, first page ready, stop marker seen, worker done; dynamic items taken, split heads
+    merged, ns spent merging."""
+    n = tg_plan_get_info(plan)["n_workers"]
+    out = np.zeros((max(n, 1), 8), dtype=np.uint64)
+    _check(_lib().tg_plan_trace_read(plan.handle, _hp(out), _stream(stream)), "tg_plan_trace_read")
+    return out[:n]
 
 
 # ------------------------------------------------------------------------------------------

@@ -298,7 +298,8 @@ extern "C" int tg_place_sequences(int32_t n_seq, const int64_t *seq_bytes, int32
 namespace tg {
 
 int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
-                    int32_t num_workers, int32_t min_splits, int32_t max_chunk_pages) {
+                    int32_t num_workers, int32_t min_splits, int32_t max_chunk_pages,
+                    int32_t static_permille, int32_t dyn_chunk_pages) {
     const tg_shape &s = p->shape;
     const int64_t BH = static_cast<int64_t>(s.B) * s.Hkv;
     const int32_t page = s.page;
@@ -351,17 +352,39 @@ int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
     }
     p->kv_bytes = kv_bytes;
 
+    // Workers: as many as asked, but at least ~8 pages each (tiny batches are not worth the
+    // partials and the merge).
     int64_t W = std::max<int64_t>(1, num_workers);
-    W = std::max<int64_t>(1, std::min<int64_t>(W, total_pages / 2));
-    // Cost of all pages plus one item overhead per chunk and per worker cut.
+    W = std::max<int64_t>(1, std::min<int64_t>(W, total_pages / 8));
+    // Cost of all pages plus one item overhead per (head, tier) run and per worker cut
+    // (adjacent chunks of a run on one worker form a single item).
     long double total_cost = static_cast<long double>(W - 1) * item_cost;
-    for (const Chunk &c : chunks) total_cost += static_cast<long double>(c.pe - c.pb) * c.page_cost + item_cost;
+    for (size_t i = 0; i < chunks.size(); ++i) {
+        const Chunk &c = chunks[i];
+        total_cost += static_cast<long double>(c.pe - c.pb) * c.page_cost;
+        if (i == 0 || chunks[i - 1].bh != c.bh || chunks[i - 1].flags != c.flags) total_cost += item_cost;
+    }
+
+    const bool hybrid = static_permille < 1000;
+    const long double sfrac = hybrid ? static_permille / 1000.0L : 1.0L;
+    const int32_t dyn_pages = std::max(1, dyn_chunk_pages);
+    std::vector<Item> dyn;
 
     p->items.clear();
     p->worker_of_item.clear();
     int64_t w = 0;
     long double cum = 0;
     auto emit = [&](const Chunk &c, int32_t pb, int32_t pe) {
+        // A worker running adjacent chunks of the same head and tier continues the online
+        // softmax across them: one item, no partial in between.
+        if (!p->items.empty() && p->worker_of_item.back() == static_cast<int32_t>(w)) {
+            Item &prev = p->items.back();
+            if (prev.bh == c.bh && prev.flags == c.flags && prev.page_end == pb) {
+                prev.page_end = pe;
+                cum += static_cast<long double>(pe - pb) * c.page_cost;
+                return;
+            }
+        }
         Item it{};
         it.bh = c.bh;
         it.page_begin = pb;
@@ -375,11 +398,19 @@ int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
         p->worker_of_item.push_back(static_cast<int32_t>(w));
         cum += static_cast<long double>(pe - pb) * c.page_cost + item_cost;
     };
+    // The dynamic region (the cost line after every worker's static share) is collected as
+    // spans and cut into dynamic items afterwards.
+    struct Span { size_t chunk; int32_t pb, pe; };
+    std::vector<Span> dyn_spans;
+    auto emit_dyn = [&](const Chunk &c, int32_t pb, int32_t pe) {
+        dyn_spans.push_back({static_cast<size_t>(&c - chunks.data()), pb, pe});
+    };
     for (const Chunk &c : chunks) {
         int32_t at = c.pb;
         while (at < c.pe) {
-            if (w == W - 1) { emit(c, at, c.pe); at = c.pe; break; }
-            const long double target = total_cost * static_cast<long double>(w + 1) / W;
+            if (hybrid && w == W) { emit_dyn(c, at, c.pe); at = c.pe; break; }
+            if (!hybrid && w == W - 1) { emit(c, at, c.pe); at = c.pe; break; }
+            const long double target = total_cost * sfrac * static_cast<long double>(w + 1) / W;
             const long double room = target - cum - item_cost;
             const int64_t k = room <= 0 ? 0 : static_cast<int64_t>(room / c.page_cost + 0.5L);
             if (k >= c.pe - at) {
@@ -394,11 +425,41 @@ int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
             }
         }
     }
+    // Dynamic items: each span of the dynamic region cut into near-equal pieces of at most
+    // dyn_pages pages (pieces never cross a (head, tier) chunk).
+    for (const Span &sp : dyn_spans) {
+        const Chunk &c = chunks[sp.chunk];
+        const int32_t n = sp.pe - sp.pb;
+        const int32_t k = (n + dyn_pages - 1) / dyn_pages;
+        int32_t at = sp.pb;
+        for (int32_t i = 0; i < k; ++i) {
+            const int32_t sz = n / k + (i < n % k ? 1 : 0);
+            Item it{};
+            it.bh = c.bh;
+            it.page_begin = at;
+            it.page_end = at + sz;
+            it.tier_tokens = c.tier_tokens;
+            it.slot = -1;
+            it.flags = c.flags;
+            it.kv_len = c.kv;
+            it.fast_len = c.fl;
+            dyn.push_back(it);
+            at += sz;
+        }
+    }
     p->n_workers = p->items.empty() ? 0 : p->worker_of_item.back() + 1;
+    if (hybrid && !dyn.empty()) p->n_workers = static_cast<int32_t>(W);
     p->worker_off.assign(static_cast<size_t>(p->n_workers) + 1, 0);
     for (size_t i = 0; i < p->items.size(); ++i) p->worker_off[p->worker_of_item[i] + 1] = static_cast<int32_t>(i + 1);
     for (int32_t i = 1; i <= p->n_workers; ++i)
         p->worker_off[i] = std::max(p->worker_off[i], p->worker_off[i - 1]);
+    // Dynamic items follow the static ones; they belong to no worker until run time.
+    p->dyn_first = static_cast<int32_t>(p->items.size());
+    p->n_dyn = static_cast<int32_t>(dyn.size());
+    for (const Item &it : dyn) {
+        p->items.push_back(it);
+        p->worker_of_item.push_back(-1);
+    }
 
     // Partial slots and the merge list: a head's items are consecutive in the list.
     std::vector<int32_t> cnt(static_cast<size_t>(BH), 0), first(static_cast<size_t>(BH), -1);
@@ -408,13 +469,22 @@ int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
         ++cnt[bh];
     }
     p->merge.clear();
+    p->empties.clear();
+    p->merge_warps = 1;
     int64_t slot = 0;
     for (int64_t bh = 0; bh < BH; ++bh) {
         if (cnt[bh] == 0) {
-            p->merge.push_back({static_cast<int32_t>(bh), 0, 0, 0});
+            p->empties.push_back(static_cast<int32_t>(bh));
         } else if (cnt[bh] > 1) {
+            const int32_t mi = static_cast<int32_t>(p->merge.size());
             p->merge.push_back({static_cast<int32_t>(bh), static_cast<int32_t>(slot), cnt[bh], 0});
-            for (int32_t j = 0; j < cnt[bh]; ++j) p->items[first[bh] + j].slot = static_cast<int32_t>(slot++);
+            for (int32_t j = 0; j < cnt[bh]; ++j) {
+                Item &it = p->items[first[bh] + j];
+                it.slot = static_cast<int32_t>(slot++);
+                it.flags |= mi << 1;
+            }
+            // warps per merge CTA: up to 8 splits per warp, at most 32 warps
+            p->merge_warps = std::max(p->merge_warps, std::min(32, (cnt[bh] + 7) / 8));
         }
     }
     p->n_partials = slot;
@@ -459,6 +529,7 @@ extern "C" int tg_plan_create(const tg_shape *shape, const int32_t *kv_len,
     p->slow_table_len = slow_table_len;
     p->group_off.assign(group_off, group_off + n_groups + 1);
     p->device = o.device;
+    p->early_prologue = o.early_prologue != 0;
 
     int32_t workers = o.num_workers;
     if (!p->host_only) {
@@ -468,9 +539,13 @@ extern "C" int tg_plan_create(const tg_shape *shape, const int32_t *kv_len,
     } else if (workers <= 0) {
         workers = 148 * tg::kPairs;
     }
-    int rc = tg::build_work_list(p, kv_len, fast_len, workers, o.min_splits, o.max_chunk_pages);
+    const int32_t sp = o.static_permille <= 0 ? 800 : std::min(1000, o.static_permille);
+    const int32_t dc = o.dyn_chunk_pages <= 0 ? 16 : o.dyn_chunk_pages;
+    int rc = tg::build_work_list(p, kv_len, fast_len, workers, o.min_splits, o.max_chunk_pages, sp, dc);
     if (rc != TG_OK) { delete p; return rc; }
     p->grid = (p->n_workers + tg::kPairs - 1) / tg::kPairs;
+    if (p->n_dyn > 0 && p->grid == 0) p->grid = 1;
+    if (p->grid == 0 && !p->empties.empty()) p->grid = 1;  // the kernel also writes empty heads
     if (!p->host_only) {
         rc = tg::device_init_plan(p);
         if (rc != TG_OK) { tg::device_free_plan(p); delete p; return rc; }
@@ -491,6 +566,8 @@ extern "C" int tg_plan_get_info(const tg_plan *p, tg_plan_info *info) {
     info->n_items = static_cast<int64_t>(p->items.size());
     info->n_partials = p->n_partials;
     info->n_merge = static_cast<int64_t>(p->merge.size());
+    info->n_empty = static_cast<int64_t>(p->empties.size());
+    info->n_dynamic = p->n_dyn;
     info->n_workers = p->n_workers;
     info->grid = p->grid;
     info->block = tg::kThreads;
@@ -507,7 +584,8 @@ extern "C" int tg_plan_items(const tg_plan *p, int32_t *items) {
         const tg::Item &it = p->items[i];
         int32_t *o = items + 8 * i;
         o[0] = it.bh; o[1] = it.page_begin; o[2] = it.page_end; o[3] = it.tier_tokens;
-        o[4] = it.slot; o[5] = it.flags; o[6] = p->worker_of_item[i]; o[7] = 0;
+        o[4] = it.slot; o[5] = it.flags & tg::kItemSlow; o[6] = p->worker_of_item[i];
+        o[7] = it.slot >= 0 ? (it.flags >> 1) : -1;
     }
     return TG_OK;
 }

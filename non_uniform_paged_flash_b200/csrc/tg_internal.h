@@ -17,15 +17,14 @@ struct Item {
     int32_t page_end;    // one past the last page
     int32_t tier_tokens; // tokens held by this head's row in this tier (tail-page mask)
     int32_t slot;        // partial-result slot, -1 = this item writes the final output
-    int32_t flags;       // kItemSlow: INT8 tier
+    int32_t flags;       // bit 0 kItemSlow (INT8 tier); bits 1.. merge-list index
     int32_t kv_len;      // planned retained length of the head (checked on device)
     int32_t fast_len;    // planned fast-tier length (tiered plans), else 0
 };
 static_assert(sizeof(Item) == 32, "Item is 32 bytes");
 constexpr int32_t kItemSlow = 1;
 
-// A head whose result is finished by the merge kernel: split over nsplit consecutive slots,
-// or empty (nsplit = 0).
+// A head split over nsplit >= 2 consecutive partial slots, merged after the decode kernel.
 struct MergeHead {
     int32_t bh;
     int32_t first_slot;
@@ -42,6 +41,7 @@ constexpr uint32_t kErrTimeout = 8u;   // a bounded wait gave up
 // Launch geometry of the decode kernels (see tg_kernels.cu).
 constexpr int kPairs = 4;              // (producer warp, consumer warp) pairs per CTA
 constexpr int kThreads = kPairs * 64;  // threads per CTA
+constexpr int kTraceWords = 8;         // worker timeline words (see tg_plan_trace_enable)
 
 }  // namespace tg
 
@@ -58,11 +58,16 @@ struct tg_plan {
     // host copies
     std::vector<tg::Item> items;
     std::vector<int32_t> worker_of_item;
-    std::vector<int32_t> worker_off;  // [n_workers + 1]
+    std::vector<int32_t> worker_off;  // [n_workers + 1] (static items)
+    int32_t dyn_first = 0;            // dynamic items: items[dyn_first ..]
+    int32_t n_dyn = 0;
     std::vector<tg::MergeHead> merge;
+    std::vector<int32_t> empties;     // heads with no retained token
     std::vector<int64_t> group_off;   // [n_groups + 1]
     std::vector<int32_t> planned_kv;  // [B*Hkv]
     int64_t n_partials = 0;
+    int32_t merge_warps = 1;          // warps per (split head, row) CTA of the merge kernel
+    bool early_prologue = false;      // see tg_plan_opts.early_prologue
     int32_t n_workers = 0;
     int64_t kv_bytes = 0;
 
@@ -81,12 +86,15 @@ struct tg_plan {
     int64_t *d_group_off = nullptr;
     float *d_part_o = nullptr;    // [n_partials][G][D]
     float *d_part_lse = nullptr;  // [n_partials][G]
+    int32_t *d_empties = nullptr;   // [n_empty]
+    uint32_t *d_dyn = nullptr;      // [2] dynamic ticket, producers done
     uint32_t *d_err = nullptr;
 
-    // kernel timing: 3 events per recorded call (cudaEvent_t stored as void*)
+    // kernel timing: 2 events per recorded call (cudaEvent_t stored as void*)
     std::vector<void *> tev;
     int32_t tev_cap = 0;
     int32_t tev_count = 0;
+    uint64_t *d_trace = nullptr;  // worker timeline, n_workers x kTraceWords (when enabled)
 
     // tensor-map cache keyed by the pool pointers of the last call
     const void *tm_key[4] = {nullptr, nullptr, nullptr, nullptr};
@@ -96,7 +104,8 @@ struct tg_plan {
 namespace tg {
 // Host planner (tg_host.cpp): fills items / worker_off / merge / n_partials / kv_bytes.
 int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
-                    int32_t num_workers, int32_t min_splits, int32_t max_chunk_pages);
+                    int32_t num_workers, int32_t min_splits, int32_t max_chunk_pages,
+                    int32_t static_permille, int32_t dyn_chunk_pages);
 // Device side (tg_kernels.cu).
 int device_init_plan(tg_plan *p);
 void device_free_plan(tg_plan *p);

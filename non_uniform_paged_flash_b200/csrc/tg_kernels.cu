@@ -208,7 +208,6 @@ __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {
 }
 
 }  // namespace dev
-
 // ------------------------------------------------------------------------------------------
 // Kernel arguments
 // ------------------------------------------------------------------------------------------
@@ -236,7 +235,13 @@ struct DecodeArgs {
     float *lse;                      // [B][Hq]
     float *part_o;                   // [n_partials][G][D]
     float *part_lse;                 // [n_partials][G]
+    const int32_t *empties;          // heads with no tokens
+    int32_t n_empty;
+    int32_t dyn_first, n_dyn;        // dynamic items: items[dyn_first .. dyn_first + n_dyn)
+    uint32_t *dyn_next;              // [0] next dynamic item, [1] producers done (zero between calls)
+    int32_t early_prologue;          // read plan/table metadata before the predecessor finishes
     uint32_t *err;
+    uint64_t *trace;                 // worker timeline (n_workers x kTraceWords) or null
 };
 
 // Per-stage header written by the producer before it arrives on the stage's full barrier.
@@ -246,7 +251,8 @@ struct StageHdr {
     int32_t bh;
     int32_t slot;
 };
-constexpr int32_t kHdrSlow = 1, kHdrFirst = 2, kHdrLast = 4, kHdrWorkerLast = 8;
+constexpr int32_t kHdrSlow = 1, kHdrFirst = 2, kHdrLast = 4, kHdrStop = 8;
+constexpr int32_t kNoLoad = -2;  // page id placeholder of a row that failed its bounds check
 
 // Shared-memory stage layout (offsets within a stage; D = 128 shown, D = 64 halves the bf16
 // regions): K bf16 [0, KB) as D/64 boxes of 16 rows x 128 B; V bf16 [KB, 2KB); q [2KB, +QB).
@@ -270,6 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tm_vq) {
     using L = Layout<D>;
     constexpr int KSTEPS = D / 16;  // k-steps of q.K and m-tiles of P.V
+    constexpr unsigned FULL = 0xffffffffu;
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -304,78 +311,155 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
+    // Programmatic dependent launch: the kernel that follows in the stream may be scheduled
+    // now (it waits for this grid before touching what this grid writes). This grid waits for
+    // its predecessor here, or, with early_prologue, only the producers read the plan and the
+    // tables first and wait just before their first copy (queries, K/V and every write come
+    // after the wait).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (!a.early_prologue || !producer) asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    if (worker >= a.n_workers) return;
-    const int it0 = a.worker_off[worker], it1 = a.worker_off[worker + 1];
-    if (it0 >= it1) return;
+    // Heads with no retained token: out = 0, lse = -inf (consumer warps).
+    if (a.n_empty > 0 && !producer) {
+        const int64_t per = static_cast<int64_t>(a.G) * D;
+        const int64_t total = static_cast<int64_t>(a.n_empty) * per;
+        const int64_t nthr = static_cast<int64_t>(gridDim.x) * kPairs * 32;
+        for (int64_t i = (static_cast<int64_t>(blockIdx.x) * kPairs + pair) * 32 + lane; i < total; i += nthr) {
+            const int32_t bh = a.empties[i / per];
+            const int32_t b = bh / a.Hkv, h = bh - b * a.Hkv;
+            const int64_t r = i % per;
+            const int64_t row = static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * a.G + r / D;
+            a.out[row * D + r % D] = __float2bfloat16_rn(0.f);
+            if (r % D == 0) a.lse[row] = -INFINITY;
+        }
+    }
+
+    // Static items of this worker (none for pairs beyond the plan's workers), then dynamic
+    // items taken from a shared ticket until they run out, then a stop marker.
+    const int it0 = worker < a.n_workers ? a.worker_off[worker] : 0;
+    const int it1 = worker < a.n_workers ? a.worker_off[worker + 1] : 0;
+    uint64_t *trace = (a.trace && worker < a.n_workers) ? a.trace + static_cast<size_t>(worker) * kTraceWords : nullptr;
+    if (trace && lane == 0 && !producer) {
+        trace[0] = dev::global_timer();
+        trace[6] = trace[7] = 0;
+    }
+    if (trace && lane == 0 && producer) trace[5] = 0;
 
     if (producer) {
         // ================================ producer warp ================================
+        // Items are taken up to 32 at a time: lane j holds item j's metadata and its row
+        // offset, checked against its (group) table; page ids are read 32 at a time, one
+        // block ahead.
         uint32_t seq = 0;
-        for (int it = it0; it < it1; ++it) {
-            const Item item = a.items[it];
-            const int32_t bh = item.bh;
-            const int32_t b = bh / a.Hkv, h = bh - b * a.Hkv;
-            const bool slow = TIERED && (item.flags & kItemSlow);
-            const int32_t row_pages = (item.tier_tokens + 15) >> 4;
-            // Row of this head in its tier's table, bounds-checked.
-            int64_t row;
-            bool row_ok;
-            if (slow) {
-                row = a.slow_off[bh];
-                row_ok = row >= 0 && row + row_pages <= a.slow_table_len;
-            } else {
-                row = a.head_off[bh];
-                int64_t lo = a.group_off[0], hi = a.group_off[a.n_groups];
-                if (a.group_of_head) {
-                    const int32_t g = a.group_of_head[h];
-                    if (g >= 0 && g < a.n_groups) {
-                        lo = a.group_off[g];
-                        hi = a.group_off[g + 1];
-                    } else {
-                        hi = lo - 1;  // invalid group: reject the row
+        bool aborted = false;
+        bool waited = !a.early_prologue;
+        auto wait_predecessor = [&]() {
+            if (!waited) {
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                waited = true;
+            }
+        };
+        auto run_items = [&](int c0, int nc) {
+            Item mi{};
+            int64_t mrow = 0;
+            int32_t mok = 0;
+            if (lane < nc) {
+                mi = a.items[c0 + lane];
+                const bool slow = TIERED && (mi.flags & kItemSlow);
+                const int32_t h = mi.bh % a.Hkv;
+                const int32_t row_pages = (mi.tier_tokens + 15) >> 4;
+                int64_t lo = 0, hi;
+                if (slow) {
+                    mrow = a.slow_off[mi.bh];
+                    hi = a.slow_table_len;
+                } else {
+                    mrow = a.head_off[mi.bh];
+                    lo = a.group_off[0];
+                    hi = a.group_off[a.n_groups];
+                    if (a.group_of_head) {
+                        const int32_t g = a.group_of_head[h];
+                        if (g >= 0 && g < a.n_groups) {
+                            lo = a.group_off[g];
+                            hi = a.group_off[g + 1];
+                        } else {
+                            hi = lo - 1;  // invalid group: reject the row
+                        }
                     }
                 }
-                row_ok = row >= lo && row + row_pages <= hi;
-            }
-            if (lane == 0) {
-                if (!row_ok) atomicOr(a.err, kErrBadRow);
-                bool plan_ok = a.kv_len_dev[bh] == item.kv_len;
-                if (TIERED) plan_ok = plan_ok && a.fast_len_dev[bh] == item.fast_len;
+                mok = (mrow >= lo && mrow + row_pages <= hi) ? 1 : 0;
+                if (!mok) atomicOr(a.err, kErrBadRow);
+                bool plan_ok = a.kv_len_dev[mi.bh] == mi.kv_len;
+                if (TIERED) plan_ok = plan_ok && a.fast_len_dev[mi.bh] == mi.fast_len;
                 if (!plan_ok) atomicOr(a.err, kErrPlan);
             }
-            const int32_t *table = slow ? a.slow_table : a.table;
-            const int64_t npool = slow ? a.num_slow_pages : a.num_pages;
-            for (int32_t p0 = item.page_begin; p0 < item.page_end; p0 += 32) {
-                const int32_t cnt = min(32, item.page_end - p0);
-                int32_t pid = -1;
-                if (row_ok && lane < cnt) {
-                    pid = __ldg(table + row + p0 + lane);
-                    if (pid < 0 || pid >= npool) {
-                        atomicOr(a.err, kErrBadPage);
-                        pid = -1;
-                    }
+            // Page ids of block (item j, pages p0 .. p0+31): lane k gets page p0 + k. The value
+            // is not inspected here, so the load stays in flight until the block is issued.
+            auto ids_of = [&](int j, int32_t p0) -> int32_t {
+                const int64_t row = __shfl_sync(FULL, mrow, j);
+                const int32_t ok = __shfl_sync(FULL, mok, j);
+                const int32_t pe = __shfl_sync(FULL, mi.page_end, j);
+                const int32_t fl = __shfl_sync(FULL, mi.flags, j);
+                const bool slow = TIERED && (fl & kItemSlow);
+                int32_t pid = kNoLoad;
+                if (ok && lane < pe - p0) pid = __ldg((slow ? a.slow_table : a.table) + row + p0 + lane);
+                return pid;
+            };
+            auto next_block = [&](int j, int32_t p0, int &jn, int32_t &pn) {
+                const int32_t pe = __shfl_sync(FULL, mi.page_end, j);
+                if (p0 + 32 < pe) {
+                    jn = j;
+                    pn = p0 + 32;
+                } else {
+                    jn = j + 1;
+                    pn = jn < nc ? __shfl_sync(FULL, mi.page_begin, jn) : 0;
                 }
-                for (int32_t j = 0; j < cnt; ++j) {
-                    const int32_t page_id = __shfl_sync(0xffffffffu, pid, j);
-                    const int32_t pg = p0 + j;
+            };
+            int j = 0;
+            int32_t p0 = __shfl_sync(FULL, mi.page_begin, 0);
+            int32_t ids = ids_of(0, p0);
+            int jn;
+            int32_t pn;
+            next_block(j, p0, jn, pn);
+            int32_t ids_n = jn < nc ? ids_of(jn, pn) : kNoLoad;
+            while (j < nc) {
+                const int32_t bh = __shfl_sync(FULL, mi.bh, j);
+                const int32_t pb = __shfl_sync(FULL, mi.page_begin, j);
+                const int32_t pe = __shfl_sync(FULL, mi.page_end, j);
+                const int32_t tt = __shfl_sync(FULL, mi.tier_tokens, j);
+                const int32_t slot = __shfl_sync(FULL, mi.slot, j);
+                const int32_t fl = __shfl_sync(FULL, mi.flags, j);
+                const bool slow = TIERED && (fl & kItemSlow);
+                const int32_t b = bh / a.Hkv, h = bh - b * a.Hkv;
+                const int32_t cnt = min(32, pe - p0);
+                for (int32_t k = 0; k < cnt; ++k) {
+                    int32_t page_id = __shfl_sync(FULL, ids, k);
+                    const int32_t pg = p0 + k;
                     const int stage = seq % stages;
                     const uint32_t phase = (seq / stages) & 1u;
-                    bool ok = dev::mbar_wait(empty0 + 8 * stage, phase ^ 1u, dev::kWaitNs);
+                    wait_predecessor();
+                    const bool ok = dev::mbar_wait(empty0 + 8 * stage, phase ^ 1u, dev::kWaitNs);
                     if (!ok || ctl[1]) {
-                        if (lane == 0) { atomicOr(a.err, kErrTimeout); ctl[1] = 1; }
+                        if (lane == 0) {
+                            atomicOr(a.err, kErrTimeout);
+                            ctl[1] = 1;
+                        }
+                        aborted = true;
                         return;
                     }
                     if (lane == 0) {
-                        const bool first = pg == item.page_begin;
-                        const bool last = pg == item.page_end - 1;
+                        if (page_id != kNoLoad &&
+                            (page_id < 0 || page_id >= (slow ? a.num_slow_pages : a.num_pages))) {
+                            atomicOr(a.err, kErrBadPage);
+                            page_id = kNoLoad;
+                        }
+                        const bool first = pg == pb;
+                        const bool last = pg == pe - 1;
                         StageHdr hd;
-                        hd.valid = page_id >= 0 ? min(16, item.tier_tokens - pg * 16) : 0;
+                        hd.valid = page_id >= 0 ? min(16, tt - pg * 16) : 0;
                         hd.flags = (slow ? kHdrSlow : 0) | (first ? kHdrFirst : 0) |
-                                   (last ? kHdrLast : 0) |
-                                   (last && it == it1 - 1 ? kHdrWorkerLast : 0);
+                                   (last ? kHdrLast : 0);
                         hd.bh = bh;
-                        hd.slot = item.slot;
+                        hd.slot = slot;
                         hdr[stage] = hd;
                         const uint32_t st = dev::smem_addr(ring + static_cast<size_t>(stage) * a.stage_bytes);
                         const uint32_t fb = full0 + 8 * stage;
@@ -407,9 +491,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                         ctl[0] = static_cast<int32_t>(seq + 1);
+                        if (trace && seq == 0) trace[1] = dev::global_timer();
                     }
                     __syncwarp();
                     ++seq;
+                }
+                j = jn;
+                p0 = pn;
+                ids = ids_n;
+                if (j < nc) {
+                    next_block(j, p0, jn, pn);
+                    ids_n = jn < nc ? ids_of(jn, pn) : kNoLoad;
+                }
+            }
+        };
+        for (int c0 = it0; c0 < it1 && !aborted; c0 += 32) run_items(c0, min(32, it1 - c0));
+        wait_predecessor();
+        while (!aborted && a.n_dyn > 0) {
+            uint32_t idx = 0;
+            if (lane == 0) idx = atomicAdd(a.dyn_next, 1u);
+            idx = __shfl_sync(FULL, idx, 0);
+            if (idx >= static_cast<uint32_t>(a.n_dyn)) break;
+            run_items(a.dyn_first + static_cast<int>(idx), 1);
+            if (trace && lane == 0) trace[5] += 1;
+        }
+        if (!aborted) {
+            // Stop marker for the consumer.
+            const int stage = seq % stages;
+            const uint32_t phase = (seq / stages) & 1u;
+            if (!dev::mbar_wait(empty0 + 8 * stage, phase ^ 1u, dev::kWaitNs) || ctl[1]) {
+                if (lane == 0) {
+                    atomicOr(a.err, kErrTimeout);
+                    ctl[1] = 1;
+                }
+            } else if (lane == 0) {
+                StageHdr hd;
+                hd.valid = 0;
+                hd.flags = kHdrStop;
+                hd.bh = 0;
+                hd.slot = -1;
+                hdr[stage] = hd;
+                dev::mbar_arrive(full0 + 8 * stage);
+                ctl[0] = static_cast<int32_t>(seq + 1);
+            }
+            // The last producer of the launch to finish resets the dynamic queue.
+            if (lane == 0 && a.n_dyn > 0) {
+                __threadfence();
+                const uint32_t total = gridDim.x * kPairs;
+                if (atomicAdd(a.dyn_next + 1, 1u) == total - 1) {
+                    a.dyn_next[0] = 0;
+                    a.dyn_next[1] = 0;
                 }
             }
         }
@@ -420,7 +551,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = lane >> 2, t = lane & 3;
     uint32_t qf[KSTEPS][2];
     float o[KSTEPS][4];
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    // running max (log2 units) and normalisers of heads 2t, 2t+1: le = sum of fp32 p (for
+    // lse), lr = sum of the p actually multiplied into V (bf16-rounded on the bf16 path)
+    float m0 = -INFINITY, m1 = -INFINITY, le0 = 0.f, le1 = 0.f, lr0 = 0.f, lr1 = 0.f;
     bool item_slow = false;
     uint32_t seq = 0;
 
@@ -439,7 +572,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 dev::mbar_wait(full0 + 8 * (s % stages), (s / stages) & 1u, dev::kDrainNs);
             return;
         }
+        if (trace && seq == 0 && lane == 0) trace[2] = dev::global_timer();
         const StageHdr hd = hdr[stage];
+        if (hd.flags & kHdrStop) {
+            if (trace && lane == 0) trace[3] = dev::global_timer();
+            break;
+        }
         const unsigned char *st = ring + static_cast<size_t>(stage) * a.stage_bytes;
         const uint32_t st_a = dev::smem_addr(st);
         const bool slow = TIERED && (hd.flags & kHdrSlow);
@@ -468,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < KSTEPS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
             m0 = m1 = -INFINITY;
-            l0 = l1 = 0.f;
+            le0 = le1 = lr0 = lr1 = 0.f;
         }
 
         const int valid = hd.valid;
@@ -510,21 +648,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // s[0]: token g head 2t; s[1]: token g head 2t+1; s[2]/s[3]: token g+8.
         const bool v0 = g < valid, v1 = g + 8 < valid;
-        float x0 = v0 ? s[0] * ks0 * a.scale_log2 : -INFINITY;
-        float x1 = v0 ? s[1] * ks0 * a.scale_log2 : -INFINITY;
-        float x2 = v1 ? s[2] * ks1 * a.scale_log2 : -INFINITY;
-        float x3 = v1 ? s[3] * ks1 * a.scale_log2 : -INFINITY;
+        const float x0 = v0 ? s[0] * ks0 * a.scale_log2 : -INFINITY;
+        const float x1 = v0 ? s[1] * ks0 * a.scale_log2 : -INFINITY;
+        const float x2 = v1 ? s[2] * ks1 * a.scale_log2 : -INFINITY;
+        const float x3 = v1 ? s[3] * ks1 * a.scale_log2 : -INFINITY;
         float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
         }
         // Lazy rescale: the running max moves only when a tile exceeds it by more than the
         // threshold (2^8 for bf16 probabilities; exact for the fp16 INT8 path).
         const float thr = slow ? 0.f : 8.f;
         const bool up0 = mx0 > m0 + thr, up1 = mx1 > m1 + thr;
-        if (__any_sync(0xffffffffu, up0 || up1)) {
+        if (__any_sync(FULL, up0 || up1)) {
             const float n0 = up0 ? mx0 : m0, n1 = up1 ? mx1 : m1;
             const float c0 = (m0 == -INFINITY) ? 0.f : dev::ex2(m0 - n0);
             const float c1 = (m1 == -INFINITY) ? 0.f : dev::ex2(m1 - n1);
@@ -535,8 +673,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 o[i][2] *= c0;
                 o[i][3] *= c1;
             }
-            l0 *= c0;
-            l1 *= c1;
+            le0 *= c0;
+            le1 *= c1;
+            lr0 *= c0;
+            lr1 *= c1;
             m0 = n0;
             m1 = n1;
         }
@@ -544,11 +684,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float p1 = x1 == -INFINITY ? 0.f : dev::ex2(x1 - m1);
         const float p2 = x2 == -INFINITY ? 0.f : dev::ex2(x2 - m0);
         const float p3 = x3 == -INFINITY ? 0.f : dev::ex2(x3 - m1);
+        le0 += p0 + p2;
+        le1 += p1 + p3;
 
         if (!slow) {
             const uint32_t r0 = dev::pack_bf16(p0, p1), r1 = dev::pack_bf16(p2, p3);
-            l0 += dev::bf16_lo(r0) + dev::bf16_lo(r1);
-            l1 += dev::bf16_hi(r0) + dev::bf16_hi(r1);
+            lr0 += dev::bf16_lo(r0) + dev::bf16_lo(r1);
+            lr1 += dev::bf16_hi(r0) + dev::bf16_hi(r1);
             const uint32_t b0 = dev::movm_t(r0), b1 = dev::movm_t(r1);
             // token masks of this thread's A-fragment halves (tokens 2t, 2t+1 | 2t+8, 2t+9)
             const uint32_t mk01 = (2 * t < valid ? 0xFFFFu : 0u) | (2 * t + 1 < valid ? 0xFFFF0000u : 0u);
@@ -571,8 +713,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         } else if (TIERED) {
             // p' = p * v_scale (fp32) -> fp16; the normaliser keeps the unscaled p.
-            l0 += p0 + p2;
-            l1 += p1 + p3;
+            lr0 += p0 + p2;
+            lr1 += p1 + p3;
             const float q0 = v0 ? p0 * vs0 : 0.f, q1 = v0 ? p1 * vs0 : 0.f;
             const float q2 = v1 ? p2 * vs1 : 0.f, q3 = v1 ? p3 * vs1 : 0.f;
             const uint32_t b0 = dev::movm_t(dev::pack_f16(q0, q1));
@@ -601,16 +743,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         if (hd.flags & kHdrLast) {
             // ---- finish the item ----
-            float L0 = l0, L1 = l1;
+            float E0 = le0, E1 = le1, R0 = lr0, R1 = lr1;
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) {
-                L0 += __shfl_xor_sync(0xffffffffu, L0, off);
-                L1 += __shfl_xor_sync(0xffffffffu, L1, off);
+                E0 += __shfl_xor_sync(FULL, E0, off);
+                E1 += __shfl_xor_sync(FULL, E1, off);
+                R0 += __shfl_xor_sync(FULL, R0, off);
+                R1 += __shfl_xor_sync(FULL, R1, off);
             }
-            const float inv0 = L0 > 0.f ? 1.f / L0 : 0.f, inv1 = L1 > 0.f ? 1.f / L1 : 0.f;
+            const float inv0 = R0 > 0.f ? 1.f / R0 : 0.f, inv1 = R1 > 0.f ? 1.f / R1 : 0.f;
             constexpr float kLn2 = 0.69314718055994530942f;
-            const float lse0 = L0 > 0.f ? (m0 + dev::lg2(L0)) * kLn2 : -INFINITY;
-            const float lse1 = L1 > 0.f ? (m1 + dev::lg2(L1)) * kLn2 : -INFINITY;
+            const float lse0 = E0 > 0.f ? (m0 + dev::lg2(E0)) * kLn2 : -INFINITY;
+            const float lse1 = E1 > 0.f ? (m1 + dev::lg2(E1)) * kLn2 : -INFINITY;
             const int32_t b = hd.bh / a.Hkv, h = hd.bh - b * a.Hkv;
             const int n0 = 2 * t, n1 = 2 * t + 1;
             if (hd.slot < 0) {
@@ -668,50 +812,105 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         ++seq;
-        if (hd.flags & kHdrWorkerLast) break;
     }
+    if (trace && lane == 0) trace[4] = dev::global_timer();
 }
 
 // ------------------------------------------------------------------------------------------
-// Merge of the plan's split heads (and zero output for empty heads): one warp per query row.
+// Merge of split heads (log-sum-exp): one CTA per (split head, query row). Warp w owns the
+// contiguous splits [w*k, (w+1)*k); it loads them 4 at a time (all loads in flight), keeps a
+// running maximum and sum, and the warps' results are combined through shared memory in warp
+// order, so the result does not depend on timing. Launched as a programmatic dependent of
+// the decode kernel: it waits for that grid before reading.
 // ------------------------------------------------------------------------------------------
-__global__ void plan_merge_kernel(const MergeHead *mh, int32_t n_merge, int32_t G, int32_t D,
-                                  int32_t Hq, int32_t Hkv, const float *part_o,
-                                  const float *part_lse, __nv_bfloat16 *out, float *lse) {
-    const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (r >= static_cast<int64_t>(n_merge) * G) return;
-    const MergeHead m = mh[r / G];
-    const int n = static_cast<int>(r % G);
-    const int32_t b = m.bh / Hkv, h = m.bh - b * Hkv;
-    __nv_bfloat16 *ob = out + ((static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * G + n) * D);
-    float mx = -INFINITY;
-    for (int j = 0; j < m.nsplit; ++j) mx = fmaxf(mx, part_lse[static_cast<int64_t>(m.first_slot + j) * G + n]);
-    if (mx == -INFINITY) {
-        for (int d = lane; d < D; d += 32) ob[d] = __float2bfloat16_rn(0.f);
-        if (lane == 0) lse[static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * G + n] = -INFINITY;
+template <int D>
+__global__ void __launch_bounds__(1024) split_merge_kernel(const MergeHead *mh, int32_t G, int32_t Hq,
+                                                           int32_t Hkv, const float *part_o,
+                                                           const float *part_lse,
+                                                           __nv_bfloat16 *out, float *lse) {
+    constexpr int VEC = D / 32;
+    constexpr int U = 4;
+    extern __shared__ float s_dyn[];  // [nw] maxima, [nw] sums, [nw][D] sums of V (nw > 1)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // Every CTA of this grid has started: the next kernel may be scheduled.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const MergeHead h = mh[blockIdx.x / G];
+    const int n = blockIdx.x % G;
+    const float *pl = part_lse + static_cast<int64_t>(h.first_slot) * G + n;
+    const float *po = part_o + (static_cast<int64_t>(h.first_slot) * G + n) * D + lane * VEC;
+    const int64_t pstride = static_cast<int64_t>(G) * D;
+    const int k = (h.nsplit + nw - 1) / nw;
+    const int j0 = warp * k, j1 = min(h.nsplit, j0 + k);
+
+    float m = -INFINITY, sum = 0.f, acc[VEC];
+#pragma unroll
+    for (int c = 0; c < VEC; ++c) acc[c] = 0.f;
+    for (int j = j0; j < j1; j += U) {
+        float l[U], v[U][VEC];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const bool in = j + u < j1;
+            l[u] = in ? pl[static_cast<int64_t>(j + u) * G] : -INFINITY;
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) v[u][c] = in ? po[(j + u) * pstride + c] : 0.f;
+        }
+        float mc = m;
+#pragma unroll
+        for (int u = 0; u < U; ++u) mc = fmaxf(mc, l[u]);
+        if (mc == -INFINITY) continue;
+        const float r = m == -INFINITY ? 0.f : expf(m - mc);
+        sum *= r;
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) acc[c] *= r;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const float w = expf(l[u] - mc);  // 0 for an empty or absent split
+            sum += w;
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) acc[c] += w * v[u][c];
+        }
+        m = mc;
+    }
+    const int32_t b = h.bh / Hkv, hh = h.bh - b * Hkv;
+    const int64_t row = static_cast<int64_t>(b) * Hq + static_cast<int64_t>(hh) * G + n;
+    if (nw > 1) {
+        float *s_m = s_dyn, *s_s = s_dyn + nw;
+        float(*s_acc)[D] = reinterpret_cast<float(*)[D]>(s_dyn + 2 * nw);
+        if (lane == 0) {
+            s_m[warp] = m;
+            s_s[warp] = sum;
+        }
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) s_acc[warp][lane * VEC + c] = acc[c];
+        __syncthreads();
+        if (warp != 0) return;
+        float M = -INFINITY;
+        for (int w = 0; w < nw; ++w) M = fmaxf(M, s_m[w]);
+        sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) acc[c] = 0.f;
+        if (M != -INFINITY) {
+            for (int w = 0; w < nw; ++w) {
+                if (s_m[w] == -INFINITY) continue;
+                const float r = expf(s_m[w] - M);
+                sum += r * s_s[w];
+#pragma unroll
+                for (int c = 0; c < VEC; ++c) acc[c] += r * s_acc[w][lane * VEC + c];
+            }
+        }
+        m = M;
+    }
+    if (m == -INFINITY) {
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) out[row * D + lane * VEC + c] = __float2bfloat16_rn(0.f);
+        if (lane == 0) lse[row] = -INFINITY;
         return;
     }
-    float sum = 0.f;
-    for (int j = 0; j < m.nsplit; ++j) sum += expf(part_lse[static_cast<int64_t>(m.first_slot + j) * G + n] - mx);
-    const float tot = mx + logf(sum);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < m.nsplit; ++j) {
-        const int64_t sl = m.first_slot + j;
-        const float w = expf(part_lse[sl * G + n] - tot);
-        const float *po = part_o + (sl * G + n) * D;
+    const float inv = 1.f / sum;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int d = lane + 32 * k;
-            if (d < D) acc[k] += w * po[d];
-        }
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int d = lane + 32 * k;
-        if (d < D) ob[d] = __float2bfloat16_rn(acc[k]);
-    }
-    if (lane == 0) lse[static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * G + n] = tot;
+    for (int c = 0; c < VEC; ++c) out[row * D + lane * VEC + c] = __float2bfloat16_rn(acc[c] * inv);
+    if (lane == 0) lse[row] = m + logf(sum);
 }
 
 // Generic merge (exported as tg_lse_merge): rows with contiguous split ranges.
@@ -871,8 +1070,9 @@ int device_init_plan(tg_plan *p) {
     const int64_t b_goff = al((p->n_groups + 1) * 8LL);
     const int64_t b_po = al(p->n_partials * p->G * s.D * 4LL);
     const int64_t b_pl = al(p->n_partials * p->G * 4LL);
-    const int64_t b_err = 256;
-    p->dev_bytes = b_items + b_woff + b_merge + b_goff + b_po + b_pl + b_err;
+    const int64_t b_emp = al(static_cast<int64_t>(p->empties.size()) * 4LL);
+    const int64_t b_err = 256;  // error word + dynamic ticket counters
+    p->dev_bytes = b_items + b_woff + b_merge + b_goff + b_po + b_pl + b_emp + b_err;
     cudaError_t e = cudaMalloc(&p->dev_base, static_cast<size_t>(p->dev_bytes));
     if (e != cudaSuccess) {
         set_cuda_error("cudaMalloc(plan)", static_cast<int>(e));
@@ -893,7 +1093,10 @@ int device_init_plan(tg_plan *p) {
     base += b_po;
     p->d_part_lse = reinterpret_cast<float *>(base);
     base += b_pl;
+    p->d_empties = reinterpret_cast<int32_t *>(base);
+    base += b_emp;
     p->d_err = reinterpret_cast<uint32_t *>(base);
+    p->d_dyn = p->d_err + 16;
 
     rc = TG_OK;
     auto up = [&](void *dst, const void *src, int64_t bytes) {
@@ -908,8 +1111,9 @@ int device_init_plan(tg_plan *p) {
     up(p->d_worker_off, p->worker_off.data(), (p->n_workers + 1) * 4LL);
     up(p->d_merge, p->merge.data(), static_cast<int64_t>(p->merge.size()) * static_cast<int64_t>(sizeof(MergeHead)));
     up(p->d_group_off, p->group_off.data(), (p->n_groups + 1) * 8LL);
+    up(p->d_empties, p->empties.data(), static_cast<int64_t>(p->empties.size()) * 4LL);
     if (rc == TG_OK) {
-        cudaError_t ee = cudaMemset(p->d_err, 0, 4);
+        cudaError_t ee = cudaMemset(p->d_err, 0, 256);
         if (ee != cudaSuccess) { set_cuda_error("cudaMemset(plan)", static_cast<int>(ee)); rc = TG_ECUDA; }
     }
     if (p->device != cur) cudaSetDevice(cur);
@@ -925,6 +1129,10 @@ static void timing_free(tg_plan *p) {
 
 void device_free_plan(tg_plan *p) {
     timing_free(p);
+    if (p->d_trace) {
+        cudaFree(p->d_trace);
+        p->d_trace = nullptr;
+    }
     if (p->dev_base) {
         int cur = 0;
         cudaGetDevice(&cur);
@@ -952,26 +1160,56 @@ static int check_device(const tg_plan *p) {
     return cur == p->device ? TG_OK : TG_EINVAL;
 }
 
-// Timing hook: event k (0 = before decode, 1 = before merge, 2 = after merge) of this call.
+// Timing hook: event k (0 = before the decode kernel, 1 = after it, 2 = after the merge
+// kernel) of this call. A recorded call loses the launch overlap of the merge kernel.
 static void timing_mark(tg_plan *p, int k, cudaStream_t stream) {
     if (p->tev_count >= p->tev_cap) return;
     cudaEventRecord(static_cast<cudaEvent_t>(p->tev[3 * p->tev_count + k]), stream);
     if (k == 2) ++p->tev_count;
 }
 
-static int launch_merge(tg_plan *p, void *out, float *lse, cudaStream_t stream) {
+// Decode kernel launch, as a programmatic dependent of whatever precedes it in the stream.
+typedef void (*DecodeFn)(DecodeArgs, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap);
+static int launch_decode(tg_plan *p, DecodeFn fn, const DecodeArgs &a, const CUtensorMap &m0,
+                         const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3,
+                         cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(p->grid));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(p->smem_bytes);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, fn, a, m0, m1, m2, m3));
+    return TG_OK;
+}
+
+// Merge kernel of the split heads, as a programmatic dependent launch of the decode kernel;
+// then close the call's timing record.
+static int finish_call(tg_plan *p, void *out, float *lse, cudaStream_t stream) {
     timing_mark(p, 1, stream);
-    if (p->merge.empty()) {
-        timing_mark(p, 2, stream);
-        return TG_OK;
+    if (!p->merge.empty()) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(p->merge.size() * p->G));
+        cfg.blockDim = dim3(static_cast<unsigned>(32 * p->merge_warps));
+        cfg.dynamicSmemBytes = p->merge_warps > 1 ? static_cast<size_t>(p->merge_warps) * (2 + p->shape.D) * 4 : 0;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const int32_t G = p->G, Hq = p->shape.Hq, Hkv = p->shape.Hkv;
+        const float *po = p->d_part_o, *pl = p->d_part_lse;
+        __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
+        if (p->shape.D == 128)
+            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<128>, (const MergeHead *)p->d_merge, G, Hq, Hkv, po, pl, o, lse));
+        else
+            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<64>, (const MergeHead *)p->d_merge, G, Hq, Hkv, po, pl, o, lse));
     }
-    const int64_t rows = static_cast<int64_t>(p->merge.size()) * p->G;
-    const int threads = 256;
-    const int64_t blocks = (rows * 32 + threads - 1) / threads;
-    plan_merge_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-        p->d_merge, static_cast<int32_t>(p->merge.size()), p->G, p->shape.D, p->shape.Hq,
-        p->shape.Hkv, p->d_part_o, p->d_part_lse, static_cast<__nv_bfloat16 *>(out), lse);
-    TG_CUDA_TRY(cudaGetLastError());
     timing_mark(p, 2, stream);
     return TG_OK;
 }
@@ -999,7 +1237,14 @@ static DecodeArgs base_args(const tg_plan *p, const void *q, const int32_t *kv, 
     a.lse = lse;
     a.part_o = p->d_part_o;
     a.part_lse = p->d_part_lse;
+    a.empties = p->d_empties;
+    a.n_empty = static_cast<int32_t>(p->empties.size());
     a.err = p->d_err;
+    a.trace = p->d_trace;
+    a.dyn_first = p->dyn_first;
+    a.n_dyn = p->n_dyn;
+    a.dyn_next = p->d_dyn;
+    a.early_prologue = p->early_prologue ? 1 : 0;
     return a;
 }
 
@@ -1021,15 +1266,16 @@ extern "C" int tg_ragged_paged_decode(tg_plan *p, const void *q, const void *k_p
     if (!q || !out || !lse || !head_kv_len || !aligned16(q) || !aligned16(out) || !aligned16(lse))
         return TG_EINVAL;
     const bool any_items = !p->items.empty();
+    const bool launch = p->grid > 0;
     if (any_items && (!k_pages || !v_pages || !page_table || !head_page_off || !group_of_head ||
                       !aligned16(k_pages) || !aligned16(v_pages) || p->shape.num_pages < 1))
         return TG_EINVAL;
     int rc = check_device(p);
     if (rc != TG_OK) return rc;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    if (any_items) {
-        rc = get_map(p, 0, k_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
-        if (rc == TG_OK) rc = get_map(p, 1, v_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
+    if (launch) {
+        if (any_items) rc = get_map(p, 0, k_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
+        if (rc == TG_OK && any_items) rc = get_map(p, 1, v_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
         if (rc != TG_OK) return rc;
         DecodeArgs a = base_args(p, q, head_kv_len, scale, out, lse);
         timing_mark(p, 0, stream);
@@ -1039,14 +1285,14 @@ extern "C" int tg_ragged_paged_decode(tg_plan *p, const void *q, const void *k_p
         const CUtensorMap &tk = *reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
         const CUtensorMap &tv = *reinterpret_cast<const CUtensorMap *>(p->tmaps[1]);
         if (p->shape.D == 128)
-            decode_kernel<128, false><<<p->grid, kThreads, p->smem_bytes, stream>>>(a, tk, tv, tk, tv);
+            rc = launch_decode(p, decode_kernel<128, false>, a, tk, tv, tk, tv, stream);
         else
-            decode_kernel<64, false><<<p->grid, kThreads, p->smem_bytes, stream>>>(a, tk, tv, tk, tv);
-        TG_CUDA_TRY(cudaGetLastError());
+            rc = launch_decode(p, decode_kernel<64, false>, a, tk, tv, tk, tv, stream);
+        if (rc != TG_OK) return rc;
     } else {
         timing_mark(p, 0, stream);
     }
-    return launch_merge(p, out, lse, stream);
+    return finish_call(p, out, lse, stream);
 }
 
 extern "C" int tg_tiered_decode(tg_plan *p, const void *q, const int8_t *k_q8,
@@ -1072,7 +1318,7 @@ extern "C" int tg_tiered_decode(tg_plan *p, const void *q, const int8_t *k_q8,
     int rc = check_device(p);
     if (rc != TG_OK) return rc;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    if (!p->items.empty()) {
+    if (p->grid > 0) {
         if (has_fast) {
             rc = get_map(p, 0, k_fast, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
             if (rc == TG_OK) rc = get_map(p, 1, v_fast, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
@@ -1095,14 +1341,13 @@ extern "C" int tg_tiered_decode(tg_plan *p, const void *q, const int8_t *k_q8,
         a.fast_len_dev = head_fast_len;
         // The fast tier's rows are bounded by its whole table [group_off[0], group_off[n]).
         const CUtensorMap *maps = reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
-        decode_kernel<128, true><<<p->grid, kThreads, p->smem_bytes, stream>>>(
-            a, maps[has_fast ? 0 : 2], maps[has_fast ? 1 : 3], maps[has_slow ? 2 : 0],
-            maps[has_slow ? 3 : 1]);
-        TG_CUDA_TRY(cudaGetLastError());
+        rc = launch_decode(p, decode_kernel<128, true>, a, maps[has_fast ? 0 : 2], maps[has_fast ? 1 : 3],
+                           maps[has_slow ? 2 : 0], maps[has_slow ? 3 : 1], stream);
+        if (rc != TG_OK) return rc;
     } else {
         timing_mark(p, 0, stream);
     }
-    return launch_merge(p, out, lse, stream);
+    return finish_call(p, out, lse, stream);
 }
 
 extern "C" int tg_plan_status(tg_plan *p, tg_stream stream_) {
@@ -1112,6 +1357,8 @@ extern "C" int tg_plan_status(tg_plan *p, tg_stream stream_) {
     TG_CUDA_TRY(cudaMemcpyAsync(&err, p->d_err, 4, cudaMemcpyDeviceToHost, stream));
     TG_CUDA_TRY(cudaStreamSynchronize(stream));
     TG_CUDA_TRY(cudaMemsetAsync(p->d_err, 0, 4, stream));
+    // A timed-out call may leave the dynamic ticket part-counted: reset it.
+    if (err & kErrTimeout) TG_CUDA_TRY(cudaMemsetAsync(p->d_dyn, 0, 8, stream));
     TG_CUDA_TRY(cudaStreamSynchronize(stream));
     if (err & kErrTimeout) return TG_ETIMEOUT;
     if (err & (kErrBadPage | kErrBadRow | kErrPlan)) return TG_EBADPAGE;
@@ -1195,5 +1442,32 @@ extern "C" int tg_plan_timing_read(tg_plan *p, int32_t *n_calls, double *decode_
         *merge_ms += b;
     }
     p->tev_count = 0;
+    return TG_OK;
+}
+
+extern "C" int tg_plan_trace_enable(tg_plan *p, int32_t on) {
+    if (!p || p->host_only) return TG_EINVAL;
+    if (p->d_trace) {
+        cudaFree(p->d_trace);
+        p->d_trace = nullptr;
+    }
+    if (!on || p->n_workers == 0) return TG_OK;
+    const size_t bytes = static_cast<size_t>(p->n_workers) * kTraceWords * sizeof(uint64_t);
+    cudaError_t e = cudaMalloc(&p->d_trace, bytes);
+    if (e != cudaSuccess) {
+        set_cuda_error("cudaMalloc(trace)", static_cast<int>(e));
+        p->d_trace = nullptr;
+        return TG_ENOMEM;
+    }
+    TG_CUDA_TRY(cudaMemset(p->d_trace, 0, bytes));
+    return TG_OK;
+}
+
+extern "C" int tg_plan_trace_read(tg_plan *p, uint64_t *trace, tg_stream stream_) {
+    if (!p || !trace || !p->d_trace) return TG_EINVAL;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    TG_CUDA_TRY(cudaMemcpyAsync(trace, p->d_trace, static_cast<size_t>(p->n_workers) * kTraceWords * 8,
+                                cudaMemcpyDeviceToHost, stream));
+    TG_CUDA_TRY(cudaStreamSynchronize(stream));
     return TG_OK;
 }

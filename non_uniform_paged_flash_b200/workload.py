@@ -200,7 +200,8 @@ def _pool_to_device(sp, which, n, layer, device, chunk_pages=1 << 16):
 
 
 def to_device(sp: synth.Spec, lay: Layout, layer: int = 0, device="cuda", num_workers: int = 0,
-              min_splits: int = 1, max_chunk_pages: int = 0, seqs=None) -> DeviceBatch:
+              min_splits: int = 1, max_chunk_pages: int = 0, seqs=None, static_permille: int = 0,
+              dyn_chunk_pages: int = 0, early_prologue: bool = False) -> DeviceBatch:
     import torch
     dev = torch.device(device)
     B = lay.kv_len.shape[0]
@@ -209,7 +210,8 @@ def to_device(sp: synth.Spec, lay: Layout, layer: int = 0, device="cuda", num_wo
                           fast_len=lay.fast_len,
                           slow_table_len=0 if lay.slow_table is None else lay.slow_table.size,
                           num_workers=num_workers, min_splits=min_splits,
-                          max_chunk_pages=max_chunk_pages,
+                          max_chunk_pages=max_chunk_pages, static_permille=static_permille,
+                          dyn_chunk_pages=dyn_chunk_pages, early_prologue=early_prologue,
                           device=dev.index if dev.index is not None else -1)
     qb = synth.q_bits(sp, layer)
     q = _bf16_tensor(qb if seqs is None else np.ascontiguousarray(qb[seqs]), dev)

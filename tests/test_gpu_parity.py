@@ -51,9 +51,10 @@ def _run(sp, layer=0, sel=None, **plan_kw):
 
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
 @pytest.mark.parametrize("workers", [0, 1, 13])
-def test_small_configs_match_oracle(cfg, workers):
+@pytest.mark.parametrize("static_permille", [1000, 800, 200])
+def test_small_configs_match_oracle(cfg, workers, static_permille):
     sp = synth.small(cfg)
-    kw = dict(num_workers=workers)
+    kw = dict(num_workers=workers, static_permille=static_permille, dyn_chunk_pages=4)
     if cfg == 5:
         kw.update(min_splits=8, max_chunk_pages=16)
     for layer in range(min(sp.layers, 2)):
@@ -98,8 +99,10 @@ def test_split_heads_every_partition_size():
 
 
 def test_deterministic_repeat():
+    """Dynamic items land on different workers from call to call; the merge order (split
+    order) keeps the results bit-identical."""
     sp = synth.small(2)
-    db, _ = _run(sp)
+    db, _ = _run(sp, static_permille=300, dyn_chunk_pages=2)
     a = db.out.clone(), db.lse.clone()
     for _ in range(3):
         db.run()

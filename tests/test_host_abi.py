@@ -190,6 +190,24 @@ def test_full_size_layout_matches_oracle_multi_layer():
 # Planner (host-only plans)
 # ---------------------------------------------------------------------------------------
 
+def test_hybrid_plan_static_share():
+    """With static_permille = 800 every worker's static bytes are ~80% of its fair share."""
+    sp = synth.preset(2)
+    lay = workload.layout(sp, 0)
+    W = 592
+    p = _plan(sp, lay, num_workers=W, static_permille=800)
+    items = tg.tg_plan_items(p)
+    _check_coverage(sp, lay, items)
+    _check_merge_indices(items)
+    st = items[:, 6] >= 0
+    pages = (items[:, 2] - items[:, 1]).astype(np.int64)
+    per_w = np.bincount(items[st, 6], weights=pages[st], minlength=W)
+    total = pages.sum()
+    assert abs(per_w.mean() - 0.8 * total / W) <= 2
+    assert per_w.max() - per_w.min() <= 4
+    assert abs(pages[~st].sum() - 0.2 * total) <= 0.01 * total
+
+
 def _plan(sp, lay, **kw):
     shape = tg.make_shape(sp.B, sp.Hq, sp.Hkv, sp.D, lay.num_pages, lay.num_slow_pages, sp.page)
     return tg.tg_plan_create(shape, lay.kv_len, lay.group_of_head, lay.group_off,
@@ -236,37 +254,75 @@ def _check_coverage(sp, lay, items, min_splits=1, max_chunk=0):
                 assert len(slots) >= min(min_splits, sum(1 for r in items if r[0] == bh))
 
 
+def _check_merge_indices(items):
+    """Split heads: one merge index per head, distinct across heads; final items have none."""
+    by_head = {}
+    for bh, pb, pe, tt, slot, tier, worker, mi in items:
+        if slot < 0:
+            assert mi == -1
+        else:
+            assert mi >= 0
+            by_head.setdefault(int(bh), set()).add(int(mi))
+    idx = [next(iter(v)) for v in by_head.values()]
+    assert all(len(v) == 1 for v in by_head.values())
+    assert sorted(idx) == list(range(len(idx)))
+
+
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
 @pytest.mark.parametrize("workers", [1, 7, 592])
-def test_plan_coverage(cfg, workers):
+@pytest.mark.parametrize("static_permille", [1000, 800, 300])
+def test_plan_coverage(cfg, workers, static_permille):
     sp = synth.small(cfg)
     lay = workload.layout(sp, 0)
-    p = _plan(sp, lay, num_workers=workers)
+    p = _plan(sp, lay, num_workers=workers, static_permille=static_permille)
     items = tg.tg_plan_items(p)
     _check_coverage(sp, lay, items)
+    _check_merge_indices(items)
     info = tg.tg_plan_get_info(p)
     assert info["n_items"] == len(items) and info["n_workers"] <= workers
+    assert info["n_empty"] == int((lay.kv_len == 0).sum())
+    dyn = items[:, 6] == -1
+    assert info["n_dynamic"] == int(dyn.sum())
+    if static_permille == 1000:
+        assert not dyn.any()
+    if dyn.any():
+        # dynamic items come last, hold at most 16 pages, and follow every static item
+        first = int(np.argmax(dyn))
+        assert dyn[first:].all()
+        assert ((items[dyn, 2] - items[dyn, 1]) <= 16).all()
 
 
-def test_plan_min_splits_and_chunk_cap():
+def test_plan_min_splits_and_chunk_fusion():
+    """Config 5 is cut into >= 64 chunks per head (128 pages each at most); a worker running
+    adjacent chunks of one head and tier carries its softmax state across them, so its
+    static items never hold two adjacent pieces of the same (head, tier)."""
     sp = synth.preset(5)
     lay = workload.layout(sp, 0)
-    p = _plan(sp, lay, num_workers=592, min_splits=64, max_chunk_pages=128)
+    p = _plan(sp, lay, num_workers=592, min_splits=64, max_chunk_pages=128, static_permille=1000)
     items = tg.tg_plan_items(p)
-    _check_coverage(sp, lay, items, max_chunk=128)
-    for bh in range(sp.B * sp.Hkv):
-        assert (items[:, 0] == bh).sum() >= 64                   # >= 64 chunks per head
+    _check_coverage(sp, lay, items)
+    _check_merge_indices(items)
+    for a, b in zip(items[:-1], items[1:]):
+        if a[6] == b[6] and a[6] >= 0:
+            assert not (a[0] == b[0] and a[5] == b[5] and a[2] == b[1])
+    # the chunking still bounds dynamic items
+    p = _plan(sp, lay, num_workers=592, min_splits=64, max_chunk_pages=128, static_permille=800)
+    items = tg.tg_plan_items(p)
+    _check_coverage(sp, lay, items)
+    dyn = items[:, 6] == -1
+    assert dyn.any() and ((items[dyn, 2] - items[dyn, 1]) <= 16).all()
 
 
 @pytest.mark.parametrize("cfg", [2, 3, 4, 5])
 def test_plan_balances_bytes_across_workers(cfg):
+    """Fully static plans: equal-cost contiguous ranges."""
     sp = synth.preset(cfg)
     lay = workload.layout(sp, 0)
     W = 592
     kw = dict(min_splits=64, max_chunk_pages=128) if cfg == 5 else {}
-    p = _plan(sp, lay, num_workers=W, **kw)
+    p = _plan(sp, lay, num_workers=W, static_permille=1000, **kw)
     items = tg.tg_plan_items(p)
-    _check_coverage(sp, lay, items, **({"max_chunk": 128} if cfg == 5 else {}))
+    _check_coverage(sp, lay, items)
     page_bytes = np.where(items[:, 5] & 1, 2 * (16 * sp.D + 64), 2 * 16 * sp.D * 2)
     work = np.zeros(W, np.float64)
     np.add.at(work, items[:, 6], (items[:, 2] - items[:, 1]) * page_bytes)

@@ -266,6 +266,28 @@ int tg_ragged_paged_decode(tg_plan *plan, const void *q, const void *k_pages,
                            const int32_t *group_of_head, float scale, void *out, float *lse,
                            tg_stream stream);
 
+/* Ragged paged decode that allocates no device memory. The source pages have no counterpart:
+ * this entry exists for callers that cannot allocate device memory after start-up — an engine
+ * that reserves the whole device for its KV pool and treats any later cudaMalloc as a failure,
+ * a plug-in whose host framework owns every device allocation, a runtime that permits
+ * allocation only during initialisation. Arguments and results are those of
+ * tg_ragged_paged_decode; plan may be a host-only plan (tg_plan_opts.host_only = 1), which holds
+ * no device memory. The kernels' scratch (the plan's work list, copied in by plain host-to-
+ * device copies on the stream, and the split heads' partial results) lives in one fixed
+ * 16 MiB device array inside this library, which every GPU that loads the library holds
+ * until the process exits; a plan that needs more returns TG_ENOMEM (the message says how
+ * much it needs) without launching anything. The first call on a device also looks up the
+ * array's device address and sets the kernels' shared-memory limit on that device; make that
+ * first call before any stream capture. All calls share the array and each call overwrites
+ * it: calls whose work overlaps on the GPU (other streams, other host threads) race and must
+ * be serialised by the caller. Kernel-side range errors are skipped as in the plan-based
+ * entry but are not reported. Calls no cudaMalloc, cudaFree or allocating library routine. */
+int tg_ragged_paged_decode_noalloc(tg_plan *plan, const void *q, const void *k_pages,
+                                   const void *v_pages, const int32_t *page_table,
+                                   const int64_t *head_page_off, const int32_t *head_kv_len,
+                                   const int32_t *group_of_head, float scale, void *out,
+                                   float *lse, tg_stream stream);
+
 /* Tiered decode ("TTKV" 核心方法 1-3): as tg_ragged_paged_decode over the union of two tiers.
  * Per head, f = min(head_fast_len, n): tokens [0, n - f) are in the INT8 tier (row starts at
  * slot 0 of slow_page_table[slow_head_off[b*Hkv+h]]), tokens [n - f, n) in the bf16 tier

@@ -88,6 +88,8 @@ _SIGS = [
     ("tg_plan_trace_enable", ctypes.c_int, [_P, _I32]),
     ("tg_plan_trace_read", ctypes.c_int, [_P, _P, _P]),
     ("tg_ragged_paged_decode", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _F32, _P, _P, _P]),
+    ("tg_ragged_paged_decode_noalloc", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _F32, _P,
+                                                      _P, _P]),
     ("tg_tiered_decode", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                         _F32, _P, _P, _P]),
     ("tg_lse_merge", ctypes.c_int, [_I64, _I32, _P, _P, _P, _P, _P, _P]),
@@ -349,6 +351,17 @@ def tg_ragged_paged_decode(plan: Plan, q, k_pages, v_pages, page_table, head_pag
         plan.handle, _dp(q), _dp(k_pages), _dp(v_pages), _dp(page_table), _dp(head_page_off),
         _dp(head_kv_len), _dp(group_of_head), float(scale), _dp(out), _dp(lse),
         _stream(stream)), "tg_ragged_paged_decode")
+
+
+def tg_ragged_paged_decode_noalloc(plan: Plan, q, k_pages, v_pages, page_table, head_page_off,
+                                   head_kv_len, group_of_head, scale: float, out, lse,
+                                   stream=None):
+    """As tg_ragged_paged_decode, for callers that cannot allocate device memory: the plan may
+    be host-only; the scratch is the library's fixed 16 MiB device array."""
+    _check(_lib().tg_ragged_paged_decode_noalloc(
+        plan.handle, _dp(q), _dp(k_pages), _dp(v_pages), _dp(page_table), _dp(head_page_off),
+        _dp(head_kv_len), _dp(group_of_head), float(scale), _dp(out), _dp(lse),
+        _stream(stream)), "tg_ragged_paged_decode_noalloc")
 
 
 def tg_tiered_decode(plan: Plan, q, k_q8, v_q8, k_scale, v_scale, slow_page_table,

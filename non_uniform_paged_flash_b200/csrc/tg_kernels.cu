@@ -26,6 +26,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "tg_internal.h"
 
@@ -1469,5 +1470,199 @@ extern "C" int tg_plan_trace_read(tg_plan *p, uint64_t *trace, tg_stream stream_
     TG_CUDA_TRY(cudaMemcpyAsync(trace, p->d_trace, static_cast<size_t>(p->n_workers) * kTraceWords * 8,
                                 cudaMemcpyDeviceToHost, stream));
     TG_CUDA_TRY(cudaStreamSynchronize(stream));
+    return TG_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Decode without device allocation.
+//
+// For callers that must not allocate device memory after start-up (an engine that reserves
+// the whole device for its KV pool and treats any later cudaMalloc as a failure, a plug-in
+// whose host framework owns every device allocation, a runtime that allows allocation only
+// during initialisation). Their scratch lives in one file-scope device array of fixed size;
+// every GPU that loads this library holds it until the process exits. The host code below
+// never names the array as a device address: it asks the runtime for the array's device
+// address once per device and passes that address to the kernels.
+// ------------------------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// One-time set-up on the current device: the array's device address, and the decode
+// kernels' shared-memory limit.
+int noalloc_setup(int dev, void **ptr) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p) {
+            set_cuda_error("cudaGetSymbolAddress(scratch)", static_cast<int>(e));
+            return TG_ECUDA;
+        }
+        TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<128, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget));
+        TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<64, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget));
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return TG_OK;
+}
+}  // namespace
+
+extern "C" int tg_ragged_paged_decode_noalloc(tg_plan *p, const void *q, const void *k_pages,
+                                              const void *v_pages, const int32_t *page_table,
+                                              const int64_t *head_page_off,
+                                              const int32_t *head_kv_len,
+                                              const int32_t *group_of_head, float scale,
+                                              void *out, float *lse, tg_stream stream_) {
+    if (!p || p->tiered) return TG_EINVAL;
+    if (!q || !out || !lse || !head_kv_len || !aligned16(q) || !aligned16(out) || !aligned16(lse))
+        return TG_EINVAL;
+    const bool any_items = !p->items.empty();
+    if (any_items && (!k_pages || !v_pages || !page_table || !head_page_off || !group_of_head ||
+                      !aligned16(k_pages) || !aligned16(v_pages) || p->shape.num_pages < 1))
+        return TG_EINVAL;
+
+    // Scratch layout: [0, 256) error word and dynamic tickets, then the work list, worker
+    // offsets, merge list, group offsets, empty heads, partial results.
+    auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t b_items = al(p->items.size() * sizeof(Item));
+    const size_t b_woff = al((static_cast<size_t>(p->n_workers) + 1) * 4);
+    const size_t b_merge = al(p->merge.size() * sizeof(MergeHead));
+    const size_t b_goff = al((static_cast<size_t>(p->n_groups) + 1) * 8);
+    const size_t b_emp = al(p->empties.size() * 4);
+    const size_t b_po = al(static_cast<size_t>(p->n_partials) * p->G * p->shape.D * 4);
+    const size_t b_pl = al(static_cast<size_t>(p->n_partials) * p->G * 4);
+    const size_t need = 256 + b_items + b_woff + b_merge + b_goff + b_emp + b_po + b_pl;
+    if (need > kNoAllocScratchBytes) {
+        std::snprintf(g_cuda_msg, sizeof(g_cuda_msg),
+                      "tg_ragged_paged_decode_noalloc: plan needs %zu bytes of scratch, the "
+                      "fixed scratch holds %zu",
+                      need, kNoAllocScratchBytes);
+        return TG_ENOMEM;
+    }
+    // Stage geometry (as for a device plan).
+    const tg_shape &s = p->shape;
+    const int KB = 16 * s.D * 2;
+    const int QB = ((p->G * s.D * 2) + 1023) / 1024 * 1024;
+    const int stage_bytes = 2 * KB + QB;
+    const int per_stage_extra = static_cast<int>(sizeof(StageHdr)) + 16;
+    int stages = (kSmemBudget - 1024 - kPairs * 8) / (kPairs * (stage_bytes + per_stage_extra));
+    stages = stages > 8 ? 8 : stages;
+    if (stages < 2) return TG_EUNSUPPORTED;
+    const int smem_bytes = 1024 + kPairs * stages * (stage_bytes + per_stage_extra) + kPairs * 8;
+
+    int dev = 0;
+    TG_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return TG_EUNSUPPORTED;
+    void *base_v = nullptr;
+    int rc = noalloc_setup(dev, &base_v);
+    if (rc != TG_OK) return rc;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+
+    char *base = static_cast<char *>(base_v);
+    uint32_t *d_err = reinterpret_cast<uint32_t *>(base);
+    uint32_t *d_dyn = d_err + 16;
+    char *at = base + 256;
+    Item *d_items = reinterpret_cast<Item *>(at);
+    at += b_items;
+    int32_t *d_woff = reinterpret_cast<int32_t *>(at);
+    at += b_woff;
+    MergeHead *d_merge = reinterpret_cast<MergeHead *>(at);
+    at += b_merge;
+    int64_t *d_goff = reinterpret_cast<int64_t *>(at);
+    at += b_goff;
+    int32_t *d_emp = reinterpret_cast<int32_t *>(at);
+    at += b_emp;
+    float *d_po = reinterpret_cast<float *>(at);
+    at += b_po;
+    float *d_pl = reinterpret_cast<float *>(at);
+
+    // The scratch keeps the previous call's contents: the error word and the dynamic tickets
+    // must start at zero; the work list is written afresh (plain copies, no allocation).
+    TG_CUDA_TRY(cudaMemsetAsync(base, 0, 256, stream));
+    if (!p->items.empty())
+        TG_CUDA_TRY(cudaMemcpyAsync(d_items, p->items.data(), p->items.size() * sizeof(Item),
+                                    cudaMemcpyHostToDevice, stream));
+    TG_CUDA_TRY(cudaMemcpyAsync(d_woff, p->worker_off.data(), (p->worker_off.size()) * 4,
+                                cudaMemcpyHostToDevice, stream));
+    if (!p->merge.empty())
+        TG_CUDA_TRY(cudaMemcpyAsync(d_merge, p->merge.data(), p->merge.size() * sizeof(MergeHead),
+                                    cudaMemcpyHostToDevice, stream));
+    TG_CUDA_TRY(cudaMemcpyAsync(d_goff, p->group_off.data(), p->group_off.size() * 8,
+                                cudaMemcpyHostToDevice, stream));
+    if (!p->empties.empty())
+        TG_CUDA_TRY(cudaMemcpyAsync(d_emp, p->empties.data(), p->empties.size() * 4,
+                                    cudaMemcpyHostToDevice, stream));
+
+    if (p->grid > 0) {
+        if (any_items) {
+            rc = get_map(p, 0, k_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.num_pages, 64);
+            if (rc == TG_OK) rc = get_map(p, 1, v_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.num_pages, 64);
+            if (rc != TG_OK) return rc;
+        }
+        DecodeArgs a{};
+        a.items = d_items;
+        a.worker_off = d_woff;
+        a.n_workers = p->n_workers;
+        a.B = s.B;
+        a.Hq = s.Hq;
+        a.Hkv = s.Hkv;
+        a.G = p->G;
+        a.stages = stages;
+        a.stage_bytes = stage_bytes;
+        a.scale_log2 = scale * 1.44269504088896340736f;
+        a.q = static_cast<const __nv_bfloat16 *>(q);
+        a.table = page_table;
+        a.head_off = head_page_off;
+        a.group_of_head = group_of_head;
+        a.group_off = d_goff;
+        a.n_groups = p->n_groups;
+        a.kv_len_dev = head_kv_len;
+        a.num_pages = s.num_pages;
+        a.num_slow_pages = s.num_slow_pages;
+        a.out = static_cast<__nv_bfloat16 *>(out);
+        a.lse = lse;
+        a.part_o = d_po;
+        a.part_lse = d_pl;
+        a.empties = d_emp;
+        a.n_empty = static_cast<int32_t>(p->empties.size());
+        a.err = d_err;
+        a.trace = nullptr;
+        a.dyn_first = p->dyn_first;
+        a.n_dyn = p->n_dyn;
+        a.dyn_next = d_dyn;
+        a.early_prologue = 0;
+        const CUtensorMap &tk = *reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
+        const CUtensorMap &tv = *reinterpret_cast<const CUtensorMap *>(p->tmaps[1]);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(p->grid));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
+        cfg.stream = stream;
+        if (s.D == 128)
+            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel<128, false>, a, tk, tv, tk, tv));
+        else
+            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel<64, false>, a, tk, tv, tk, tv));
+    }
+    if (!p->merge.empty()) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(p->merge.size() * p->G));
+        cfg.blockDim = dim3(static_cast<unsigned>(32 * p->merge_warps));
+        cfg.dynamicSmemBytes = p->merge_warps > 1 ? static_cast<size_t>(p->merge_warps) * (2 + s.D) * 4 : 0;
+        cfg.stream = stream;
+        __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
+        if (s.D == 128)
+            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<128>, (const MergeHead *)d_merge,
+                                           p->G, s.Hq, s.Hkv, (const float *)d_po, (const float *)d_pl, o, lse));
+        else
+            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<64>, (const MergeHead *)d_merge,
+                                           p->G, s.Hq, s.Hkv, (const float *)d_po, (const float *)d_pl, o, lse));
+    }
     return TG_OK;
 }

@@ -252,7 +252,7 @@ struct StageHdr {
     int32_t bh;
     int32_t slot;
 };
-constexpr int32_t kHdrSlow = 1, kHdrFirst = 2, kHdrLast = 4, kHdrStop = 8;
+constexpr int32_t kHdrSlow = 1, kHdrFirst = 2, kHdrLast = 4, kHdrStop = 8, kHdrPair = 16;
 constexpr int32_t kNoLoad = -2;  // page id placeholder of a row that failed its bounds check
 
 // Shared-memory stage layout (offsets within a stage; D = 128 shown, D = 64 halves the bf16
@@ -266,6 +266,193 @@ struct Layout {
     static constexpr int kKScale = 2048, kVScale = 2112;
 };
 
+// Online-softmax state of the two query heads (2t, 2t+1) a consumer lane accumulates.
+struct PageState {
+    float m0, m1;    // running maxima, log2 units
+    float le0, le1;  // sums of fp32 probabilities (for the lse)
+    float lr0, lr1;  // sums of the probabilities multiplied into V
+    __device__ __forceinline__ void reset() {
+        m0 = m1 = -INFINITY;
+        le0 = le1 = lr0 = lr1 = 0.f;
+    }
+};
+
+// One consumer step over NP pages (1 or 2) of the same item: S = K q^T per page (16 tokens x
+// 8 heads, tokens on M), one max reduction and rescale check for all NP pages, then O^T +=
+// V^T P^T per page. With NP = 2 the two pages' instruction streams interleave (independent
+// chains). SLOW: INT8 pages (codes converted to fp16 in registers, per-token scales).
+template <int D, int NP, bool SLOW>
+__device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const int (&valid)[NP],
+                                              const uint32_t (&qf)[D / 16][2],
+                                              float (&o)[D / 16][4], PageState &ps,
+                                              const uint32_t (&offK)[D / 16],
+                                              const uint32_t (&offV)[D / 16],
+                                              const uint32_t (&off8)[D / 32], float scale_log2,
+                                              int lane) {
+    using L = Layout<D>;
+    constexpr int KS = D / 16;
+    constexpr unsigned FULL = 0xffffffffu;
+    const int g = lane >> 2, t = lane & 3;
+    float s[NP][4];
+    float ks[NP][2], vs[NP][2];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        s[p][0] = s[p][1] = s[p][2] = s[p][3] = 0.f;
+        ks[p][0] = ks[p][1] = vs[p][0] = vs[p][1] = 1.f;
+    }
+    if (!SLOW) {
+#pragma unroll
+        for (int j = 0; j < KS; ++j) {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                uint32_t a0, a1, a2, a3;
+                dev::ldsm_x4(sa[p] + offK[j], a0, a1, a2, a3);
+                dev::mma_bf16(s[p], a0, a1, a2, a3, qf[j][0], qf[j][1]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int jj = 0; jj < KS / 2; ++jj) {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                uint32_t r0, r1, r2, r3;
+                dev::ldsm_x4(sa[p] + off8[jj], r0, r1, r2, r3);
+                uint32_t a0, a1, a2, a3;
+                dev::i8x4_to_f16x4(r0, a0, a2);
+                dev::i8x4_to_f16x4(r1, a1, a3);
+                dev::mma_f16(s[p], a0, a1, a2, a3, qf[2 * jj][0], qf[2 * jj][1]);
+                dev::i8x4_to_f16x4(r2, a0, a2);
+                dev::i8x4_to_f16x4(r3, a1, a3);
+                dev::mma_f16(s[p], a0, a1, a2, a3, qf[2 * jj + 1][0], qf[2 * jj + 1][1]);
+            }
+        }
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            float k0, k1, v0, v1;
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(k0) : "r"(sa[p] + L::kKScale + 4 * g));
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(k1) : "r"(sa[p] + L::kKScale + 4 * (g + 8)));
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v0) : "r"(sa[p] + L::kVScale + 4 * g));
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v1) : "r"(sa[p] + L::kVScale + 4 * (g + 8)));
+            ks[p][0] = k0;
+            ks[p][1] = k1;
+            vs[p][0] = v0;
+            vs[p][1] = v1;
+        }
+    }
+    // s[p][0]: token g head 2t; s[p][1]: token g head 2t+1; s[p][2]/s[p][3]: token g+8.
+    float x[NP][4];
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        const bool v0 = g < valid[p], v1 = g + 8 < valid[p];
+        x[p][0] = v0 ? s[p][0] * ks[p][0] * scale_log2 : -INFINITY;
+        x[p][1] = v0 ? s[p][1] * ks[p][0] * scale_log2 : -INFINITY;
+        x[p][2] = v1 ? s[p][2] * ks[p][1] * scale_log2 : -INFINITY;
+        x[p][3] = v1 ? s[p][3] * ks[p][1] * scale_log2 : -INFINITY;
+        mx0 = fmaxf(mx0, fmaxf(x[p][0], x[p][2]));
+        mx1 = fmaxf(mx1, fmaxf(x[p][1], x[p][3]));
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
+    }
+    // Lazy rescale: the running max moves only when a tile exceeds it by more than the
+    // threshold (2^8 for bf16 probabilities; exact for the fp16 INT8 path).
+    const float thr = SLOW ? 0.f : 8.f;
+    const bool up0 = mx0 > ps.m0 + thr, up1 = mx1 > ps.m1 + thr;
+    if (__any_sync(FULL, up0 || up1)) {
+        const float n0 = up0 ? mx0 : ps.m0, n1 = up1 ? mx1 : ps.m1;
+        const float c0 = (ps.m0 == -INFINITY) ? 0.f : dev::ex2(ps.m0 - n0);
+        const float c1 = (ps.m1 == -INFINITY) ? 0.f : dev::ex2(ps.m1 - n1);
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+            o[i][0] *= c0;
+            o[i][1] *= c1;
+            o[i][2] *= c0;
+            o[i][3] *= c1;
+        }
+        ps.le0 *= c0;
+        ps.le1 *= c1;
+        ps.lr0 *= c0;
+        ps.lr1 *= c1;
+        ps.m0 = n0;
+        ps.m1 = n1;
+    }
+    float pv[NP][4];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        pv[p][0] = x[p][0] == -INFINITY ? 0.f : dev::ex2(x[p][0] - ps.m0);
+        pv[p][1] = x[p][1] == -INFINITY ? 0.f : dev::ex2(x[p][1] - ps.m1);
+        pv[p][2] = x[p][2] == -INFINITY ? 0.f : dev::ex2(x[p][2] - ps.m0);
+        pv[p][3] = x[p][3] == -INFINITY ? 0.f : dev::ex2(x[p][3] - ps.m1);
+        ps.le0 += pv[p][0] + pv[p][2];
+        ps.le1 += pv[p][1] + pv[p][3];
+    }
+    if (!SLOW) {
+        uint32_t b0[NP], b1[NP], mk01[NP], mk23[NP];
+        bool tail[NP];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            const uint32_t r0 = dev::pack_bf16(pv[p][0], pv[p][1]), r1 = dev::pack_bf16(pv[p][2], pv[p][3]);
+            ps.lr0 += dev::bf16_lo(r0) + dev::bf16_lo(r1);
+            ps.lr1 += dev::bf16_hi(r0) + dev::bf16_hi(r1);
+            b0[p] = dev::movm_t(r0);
+            b1[p] = dev::movm_t(r1);
+            // token masks of this thread's A-fragment halves (tokens 2t, 2t+1 | 2t+8, 2t+9)
+            mk01[p] = (2 * t < valid[p] ? 0xFFFFu : 0u) | (2 * t + 1 < valid[p] ? 0xFFFF0000u : 0u);
+            mk23[p] = (2 * t + 8 < valid[p] ? 0xFFFFu : 0u) | (2 * t + 9 < valid[p] ? 0xFFFF0000u : 0u);
+            tail[p] = valid[p] < 16;
+        }
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                uint32_t a0, a1, a2, a3;
+                dev::ldsm_x4_t(sa[p] + offV[i], a0, a1, a2, a3);
+                if (tail[p]) {
+                    a0 &= mk01[p];
+                    a1 &= mk01[p];
+                    a2 &= mk23[p];
+                    a3 &= mk23[p];
+                }
+                dev::mma_bf16(o[i], a0, a1, a2, a3, b0[p], b1[p]);
+            }
+        }
+    } else {
+        uint32_t b0[NP], b1[NP];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            // p' = p * v_scale (fp32) -> fp16; the normaliser keeps the unscaled p.
+            ps.lr0 += pv[p][0] + pv[p][2];
+            ps.lr1 += pv[p][1] + pv[p][3];
+            const bool v0 = g < valid[p], v1 = g + 8 < valid[p];
+            const float q0 = v0 ? pv[p][0] * vs[p][0] : 0.f, q1 = v0 ? pv[p][1] * vs[p][0] : 0.f;
+            const float q2 = v1 ? pv[p][2] * vs[p][1] : 0.f, q3 = v1 ? pv[p][3] * vs[p][1] : 0.f;
+            b0[p] = dev::movm_t(dev::pack_f16(q0, q1));
+            b1[p] = dev::movm_t(dev::pack_f16(q2, q3));
+        }
+#pragma unroll
+        for (int ii = 0; ii < KS / 2; ++ii) {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                uint32_t r0, r1, r2, r3;
+                dev::ldsm_x4(sa[p] + L::KB + off8[ii], r0, r1, r2, r3);
+                // r0: tokens 0-7 chunk 2ii; r1: tokens 8-15 chunk 2ii; r2/r3: chunk 2ii+1
+                uint32_t x0l, x0h, x1l, x1h;
+                dev::i8x4_to_f16x4(r0, x0l, x0h);
+                dev::i8x4_to_f16x4(r1, x1l, x1h);
+                dev::mma_f16(o[2 * ii], dev::movm_t(x0l), dev::movm_t(x0h), dev::movm_t(x1l),
+                             dev::movm_t(x1h), b0[p], b1[p]);
+                dev::i8x4_to_f16x4(r2, x0l, x0h);
+                dev::i8x4_to_f16x4(r3, x1l, x1h);
+                dev::mma_f16(o[2 * ii + 1], dev::movm_t(x0l), dev::movm_t(x0h), dev::movm_t(x1l),
+                             dev::movm_t(x1h), b0[p], b1[p]);
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------------------------------
 // Decode kernel
 // ------------------------------------------------------------------------------------------
@@ -276,7 +463,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tm_kq,
                   const __grid_constant__ CUtensorMap tm_vq) {
     using L = Layout<D>;
-    constexpr int KSTEPS = D / 16;  // k-steps of q.K and m-tiles of P.V
     constexpr unsigned FULL = 0xffffffffu;
 
     extern __shared__ unsigned char smem_raw[];
@@ -352,6 +538,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // offset, checked against its (group) table; page ids are read 32 at a time, one
         // block ahead.
         uint32_t seq = 0;
+        int pstage = 0;        // seq % stages
+        uint32_t pphase = 0;   // (seq / stages) & 1
         bool aborted = false;
         bool waited = !a.early_prologue;
         auto wait_predecessor = [&]() {
@@ -435,8 +623,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int32_t k = 0; k < cnt; ++k) {
                     int32_t page_id = __shfl_sync(FULL, ids, k);
                     const int32_t pg = p0 + k;
-                    const int stage = seq % stages;
-                    const uint32_t phase = (seq / stages) & 1u;
+                    const int stage = pstage;
+                    const uint32_t phase = pphase;
                     wait_predecessor();
                     const bool ok = dev::mbar_wait(empty0 + 8 * stage, phase ^ 1u, dev::kWaitNs);
                     if (!ok || ctl[1]) {
@@ -455,10 +643,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         const bool first = pg == pb;
                         const bool last = pg == pe - 1;
+                        // pages (pb, pb+1), (pb+2, pb+3), ... of an item are consumed together
+                        const bool pair = ((pg - pb) & 1) == 0 && pg + 1 < pe;
                         StageHdr hd;
                         hd.valid = page_id >= 0 ? min(16, tt - pg * 16) : 0;
                         hd.flags = (slow ? kHdrSlow : 0) | (first ? kHdrFirst : 0) |
-                                   (last ? kHdrLast : 0);
+                                   (last ? kHdrLast : 0) | (pair ? kHdrPair : 0);
                         hd.bh = bh;
                         hd.slot = slot;
                         hdr[stage] = hd;
@@ -496,6 +686,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     __syncwarp();
                     ++seq;
+                    if (++pstage == stages) {
+                        pstage = 0;
+                        pphase ^= 1u;
+                    }
                 }
                 j = jn;
                 p0 = pn;
@@ -518,8 +712,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!aborted) {
             // Stop marker for the consumer.
-            const int stage = seq % stages;
-            const uint32_t phase = (seq / stages) & 1u;
+            const int stage = pstage;
+            const uint32_t phase = pphase;
             if (!dev::mbar_wait(empty0 + 8 * stage, phase ^ 1u, dev::kWaitNs) || ctl[1]) {
                 if (lane == 0) {
                     atomicOr(a.err, kErrTimeout);
@@ -550,43 +744,87 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ================================ consumer warp ================================
     const int g = lane >> 2, t = lane & 3;
+    // Per-lane ldmatrix row offsets within a stage (128-byte swizzled boxes), fixed for the
+    // whole kernel: bf16 K per k-step, bf16 V per m-tile, INT8 K/V per pair of 16-byte chunks.
+    constexpr int KSTEPS = D / 16;
+    uint32_t offK[KSTEPS], offV[KSTEPS], off8[KSTEPS / 2];
+    {
+        const int lm = lane >> 3;
+#pragma unroll
+        for (int j = 0; j < KSTEPS; ++j) {
+            const uint32_t rk = (lm & 1) * 8 + (lane & 7), ck = 2 * j + (lm >> 1);
+            offK[j] = (ck >> 3) * 2048 + dev::swz(rk, ck & 7);
+            const uint32_t rv = (lm >> 1) * 8 + (lane & 7), cv = 2 * j + (lm & 1);
+            offV[j] = L::KB + (cv >> 3) * 2048 + dev::swz(rv, cv & 7);
+        }
+#pragma unroll
+        for (int j = 0; j < KSTEPS / 2; ++j)
+            off8[j] = dev::swz((lm & 1) * 8 + (lane & 7), 2 * j + (lm >> 1));
+    }
     uint32_t qf[KSTEPS][2];
     float o[KSTEPS][4];
     // running max (log2 units) and normalisers of heads 2t, 2t+1: le = sum of fp32 p (for
     // lse), lr = sum of the p actually multiplied into V (bf16-rounded on the bf16 path)
-    float m0 = -INFINITY, m1 = -INFINITY, le0 = 0.f, le1 = 0.f, lr0 = 0.f, lr1 = 0.f;
+    PageState ps;
     bool item_slow = false;
     uint32_t seq = 0;
+    int cstage = 0;
+    uint32_t cphase = 0;
+    auto advance = [&]() {
+        ++seq;
+        if (++cstage == stages) {
+            cstage = 0;
+            cphase ^= 1u;
+        }
+    };
+    auto timed_out = [&]() {
+        // Stop the producer and drain the copies it issued, then leave.
+        if (lane == 0) {
+            atomicOr(a.err, kErrTimeout);
+            ctl[1] = 1;
+        }
+        __syncwarp();
+        const uint32_t issued = static_cast<uint32_t>(ctl[0]);
+        for (uint32_t s = seq; s < issued; ++s)
+            dev::mbar_wait(full0 + 8 * (s % stages), (s / stages) & 1u, dev::kDrainNs);
+    };
 
     while (true) {
-        const int stage = seq % stages;
-        const uint32_t phase = (seq / stages) & 1u;
-        if (!dev::mbar_wait(full0 + 8 * stage, phase, dev::kWaitNs)) {
-            // Timed out: stop the producer and drain the copies it issued, then leave.
-            if (lane == 0) {
-                atomicOr(a.err, kErrTimeout);
-                ctl[1] = 1;
-            }
-            __syncwarp();
-            const uint32_t issued = static_cast<uint32_t>(ctl[0]);
-            for (uint32_t s = seq; s < issued; ++s)
-                dev::mbar_wait(full0 + 8 * (s % stages), (s / stages) & 1u, dev::kDrainNs);
+        if (!dev::mbar_wait(full0 + 8 * cstage, cphase, dev::kWaitNs)) {
+            timed_out();
             return;
         }
         if (trace && seq == 0 && lane == 0) trace[2] = dev::global_timer();
-        const StageHdr hd = hdr[stage];
+        const StageHdr hd = hdr[cstage];
         if (hd.flags & kHdrStop) {
             if (trace && lane == 0) trace[3] = dev::global_timer();
             break;
         }
-        const unsigned char *st = ring + static_cast<size_t>(stage) * a.stage_bytes;
-        const uint32_t st_a = dev::smem_addr(st);
+        const int sA = cstage;
+        advance();
+        int sB = sA;
+        int validB = 0;
+        int32_t last_flags = hd.flags;
+        const bool pair = (hd.flags & kHdrPair) != 0;
+        if (pair) {
+            if (!dev::mbar_wait(full0 + 8 * cstage, cphase, dev::kWaitNs)) {
+                timed_out();
+                return;
+            }
+            const StageHdr hb = hdr[cstage];
+            sB = cstage;
+            validB = hb.valid;
+            last_flags = hb.flags;
+            advance();
+        }
+        const unsigned char *stA = ring + static_cast<size_t>(sA) * a.stage_bytes;
+        const unsigned char *stB = ring + static_cast<size_t>(sB) * a.stage_bytes;
         const bool slow = TIERED && (hd.flags & kHdrSlow);
 
         if (hd.flags & kHdrFirst) {
             // New item: query fragments (B operand, N = head g of this KV head) and state.
             item_slow = slow;
-            const unsigned char *qs = st + 2 * L::KB;
+            const unsigned char *qs = stA + 2 * L::KB;
 #pragma unroll
             for (int j = 0; j < KSTEPS; ++j) {
                 if (g < a.G) {
@@ -606,145 +844,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
 #pragma unroll
             for (int i = 0; i < KSTEPS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-            m0 = m1 = -INFINITY;
-            le0 = le1 = lr0 = lr1 = 0.f;
+            ps.reset();
         }
 
-        const int valid = hd.valid;
-        // ---- S = K q^T : 16 tokens x 8 heads ----
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
-        float ks0 = 1.f, ks1 = 1.f, vs0 = 1.f, vs1 = 1.f;
+        const uint32_t aA = dev::smem_addr(stA), aB = dev::smem_addr(stB);
         if (!slow) {
-#pragma unroll
-            for (int j = 0; j < KSTEPS; ++j) {
-                const int mi = lane >> 3;
-                const uint32_t row = (mi & 1) * 8 + (lane & 7);
-                const uint32_t cc = 2 * j + (mi >> 1);  // 16-byte chunk over the row of D
-                uint32_t a0, a1, a2, a3;
-                dev::ldsm_x4(st_a + (cc >> 3) * 2048 + dev::swz(row, cc & 7), a0, a1, a2, a3);
-                dev::mma_bf16(s, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+            if (pair) {
+                const uint32_t sa[2] = {aA, aB};
+                const int va[2] = {hd.valid, validB};
+                consume_pages<D, 2, false>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
+            } else {
+                const uint32_t sa[1] = {aA};
+                const int va[1] = {hd.valid};
+                consume_pages<D, 1, false>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
             }
         } else if (TIERED) {
-#pragma unroll
-            for (int j = 0; j < KSTEPS; j += 2) {
-                const int mi = lane >> 3;
-                const uint32_t row = (mi & 1) * 8 + (lane & 7);
-                const uint32_t cc = j + (mi >> 1);
-                uint32_t r0, r1, r2, r3;
-                dev::ldsm_x4(st_a + dev::swz(row, cc), r0, r1, r2, r3);
-                uint32_t a0, a1, a2, a3;
-                dev::i8x4_to_f16x4(r0, a0, a2);
-                dev::i8x4_to_f16x4(r1, a1, a3);
-                dev::mma_f16(s, a0, a1, a2, a3, qf[j][0], qf[j][1]);
-                dev::i8x4_to_f16x4(r2, a0, a2);
-                dev::i8x4_to_f16x4(r3, a1, a3);
-                dev::mma_f16(s, a0, a1, a2, a3, qf[j + 1][0], qf[j + 1][1]);
-            }
-            const float *ksc = reinterpret_cast<const float *>(st + L::kKScale);
-            const float *vsc = reinterpret_cast<const float *>(st + L::kVScale);
-            ks0 = ksc[g];
-            ks1 = ksc[g + 8];
-            vs0 = vsc[g];
-            vs1 = vsc[g + 8];
-        }
-        // s[0]: token g head 2t; s[1]: token g head 2t+1; s[2]/s[3]: token g+8.
-        const bool v0 = g < valid, v1 = g + 8 < valid;
-        const float x0 = v0 ? s[0] * ks0 * a.scale_log2 : -INFINITY;
-        const float x1 = v0 ? s[1] * ks0 * a.scale_log2 : -INFINITY;
-        const float x2 = v1 ? s[2] * ks1 * a.scale_log2 : -INFINITY;
-        const float x3 = v1 ? s[3] * ks1 * a.scale_log2 : -INFINITY;
-        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
-        }
-        // Lazy rescale: the running max moves only when a tile exceeds it by more than the
-        // threshold (2^8 for bf16 probabilities; exact for the fp16 INT8 path).
-        const float thr = slow ? 0.f : 8.f;
-        const bool up0 = mx0 > m0 + thr, up1 = mx1 > m1 + thr;
-        if (__any_sync(FULL, up0 || up1)) {
-            const float n0 = up0 ? mx0 : m0, n1 = up1 ? mx1 : m1;
-            const float c0 = (m0 == -INFINITY) ? 0.f : dev::ex2(m0 - n0);
-            const float c1 = (m1 == -INFINITY) ? 0.f : dev::ex2(m1 - n1);
-#pragma unroll
-            for (int i = 0; i < KSTEPS; ++i) {
-                o[i][0] *= c0;
-                o[i][1] *= c1;
-                o[i][2] *= c0;
-                o[i][3] *= c1;
-            }
-            le0 *= c0;
-            le1 *= c1;
-            lr0 *= c0;
-            lr1 *= c1;
-            m0 = n0;
-            m1 = n1;
-        }
-        const float p0 = x0 == -INFINITY ? 0.f : dev::ex2(x0 - m0);
-        const float p1 = x1 == -INFINITY ? 0.f : dev::ex2(x1 - m1);
-        const float p2 = x2 == -INFINITY ? 0.f : dev::ex2(x2 - m0);
-        const float p3 = x3 == -INFINITY ? 0.f : dev::ex2(x3 - m1);
-        le0 += p0 + p2;
-        le1 += p1 + p3;
-
-        if (!slow) {
-            const uint32_t r0 = dev::pack_bf16(p0, p1), r1 = dev::pack_bf16(p2, p3);
-            lr0 += dev::bf16_lo(r0) + dev::bf16_lo(r1);
-            lr1 += dev::bf16_hi(r0) + dev::bf16_hi(r1);
-            const uint32_t b0 = dev::movm_t(r0), b1 = dev::movm_t(r1);
-            // token masks of this thread's A-fragment halves (tokens 2t, 2t+1 | 2t+8, 2t+9)
-            const uint32_t mk01 = (2 * t < valid ? 0xFFFFu : 0u) | (2 * t + 1 < valid ? 0xFFFF0000u : 0u);
-            const uint32_t mk23 = (2 * t + 8 < valid ? 0xFFFFu : 0u) | (2 * t + 9 < valid ? 0xFFFF0000u : 0u);
-            const bool tail = valid < 16;
-#pragma unroll
-            for (int i = 0; i < KSTEPS; ++i) {
-                const int mi = lane >> 3;
-                const uint32_t row = (mi >> 1) * 8 + (lane & 7);  // token
-                const uint32_t cc = 2 * i + (mi & 1);             // d chunk
-                uint32_t a0, a1, a2, a3;
-                dev::ldsm_x4_t(st_a + L::KB + (cc >> 3) * 2048 + dev::swz(row, cc & 7), a0, a1, a2, a3);
-                if (tail) {
-                    a0 &= mk01;
-                    a1 &= mk01;
-                    a2 &= mk23;
-                    a3 &= mk23;
-                }
-                dev::mma_bf16(o[i], a0, a1, a2, a3, b0, b1);
-            }
-        } else if (TIERED) {
-            // p' = p * v_scale (fp32) -> fp16; the normaliser keeps the unscaled p.
-            lr0 += p0 + p2;
-            lr1 += p1 + p3;
-            const float q0 = v0 ? p0 * vs0 : 0.f, q1 = v0 ? p1 * vs0 : 0.f;
-            const float q2 = v1 ? p2 * vs1 : 0.f, q3 = v1 ? p3 * vs1 : 0.f;
-            const uint32_t b0 = dev::movm_t(dev::pack_f16(q0, q1));
-            const uint32_t b1 = dev::movm_t(dev::pack_f16(q2, q3));
-#pragma unroll
-            for (int i = 0; i < KSTEPS; i += 2) {
-                const int mi = lane >> 3;
-                const uint32_t row = (mi & 1) * 8 + (lane & 7);  // token
-                const uint32_t cc = i + (mi >> 1);
-                uint32_t r0, r1, r2, r3;
-                dev::ldsm_x4(st_a + L::KB + dev::swz(row, cc), r0, r1, r2, r3);
-                // r0: tokens 0-7 chunk i; r1: tokens 8-15 chunk i; r2/r3: chunk i+1
-                uint32_t x0l, x0h, x1l, x1h;
-                dev::i8x4_to_f16x4(r0, x0l, x0h);
-                dev::i8x4_to_f16x4(r1, x1l, x1h);
-                dev::mma_f16(o[i], dev::movm_t(x0l), dev::movm_t(x0h), dev::movm_t(x1l),
-                             dev::movm_t(x1h), b0, b1);
-                dev::i8x4_to_f16x4(r2, x0l, x0h);
-                dev::i8x4_to_f16x4(r3, x1l, x1h);
-                dev::mma_f16(o[i + 1], dev::movm_t(x0l), dev::movm_t(x0h), dev::movm_t(x1l),
-                             dev::movm_t(x1h), b0, b1);
+            if (pair) {
+                const uint32_t sa[2] = {aA, aB};
+                const int va[2] = {hd.valid, validB};
+                consume_pages<D, 2, true>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
+            } else {
+                const uint32_t sa[1] = {aA};
+                const int va[1] = {hd.valid};
+                consume_pages<D, 1, true>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
             }
         }
         __syncwarp();
-        if (lane == 0) dev::mbar_arrive(empty0 + 8 * stage);
+        if (lane == 0) {
+            dev::mbar_arrive(empty0 + 8 * sA);
+            if (pair) dev::mbar_arrive(empty0 + 8 * sB);
+        }
 
-        if (hd.flags & kHdrLast) {
+        if (last_flags & kHdrLast) {
             // ---- finish the item ----
-            float E0 = le0, E1 = le1, R0 = lr0, R1 = lr1;
+            float E0 = ps.le0, E1 = ps.le1, R0 = ps.lr0, R1 = ps.lr1;
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) {
                 E0 += __shfl_xor_sync(FULL, E0, off);
@@ -754,8 +887,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float inv0 = R0 > 0.f ? 1.f / R0 : 0.f, inv1 = R1 > 0.f ? 1.f / R1 : 0.f;
             constexpr float kLn2 = 0.69314718055994530942f;
-            const float lse0 = E0 > 0.f ? (m0 + dev::lg2(E0)) * kLn2 : -INFINITY;
-            const float lse1 = E1 > 0.f ? (m1 + dev::lg2(E1)) * kLn2 : -INFINITY;
+            const float lse0 = E0 > 0.f ? (ps.m0 + dev::lg2(E0)) * kLn2 : -INFINITY;
+            const float lse1 = E1 > 0.f ? (ps.m1 + dev::lg2(E1)) * kLn2 : -INFINITY;
             const int32_t b = hd.bh / a.Hkv, h = hd.bh - b * a.Hkv;
             const int n0 = 2 * t, n1 = 2 * t + 1;
             if (hd.slot < 0) {
@@ -812,7 +945,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-        ++seq;
     }
     if (trace && lane == 0) trace[4] = dev::global_timer();
 }

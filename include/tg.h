@@ -168,6 +168,12 @@ typedef struct tg_plan_opts {
                                  every output are touched only after the wait. Use 1 only if no
                                  preceding kernel that triggers its dependents early writes
                                  those tables (this library's own kernels never do). */
+    int32_t wait_limit_us;    /* bound of any single wait inside the decode kernel, in µs
+                                 (0 = default 4 s); a wait that runs out stops the kernel and
+                                 the call reports TG_ETIMEOUT through tg_plan_status */
+    int32_t test_withhold_page; /* testing only (0 = off): worker 0's producer never signals
+                                 its page number test_withhold_page (1-based), so a bounded
+                                 wait runs out on purpose; no copy is issued for that page */
 } tg_plan_opts;
 
 /* Build a plan. kv_len[B*Hkv] (host): retained tokens per (sequence, KV head); the decode

@@ -44,7 +44,8 @@ class tg_plan_opts(ctypes.Structure):
     _fields_ = [("num_workers", ctypes.c_int32), ("min_splits", ctypes.c_int32),
                 ("max_chunk_pages", ctypes.c_int32), ("host_only", ctypes.c_int32),
                 ("device", ctypes.c_int32), ("static_permille", ctypes.c_int32),
-                ("dyn_chunk_pages", ctypes.c_int32), ("early_prologue", ctypes.c_int32)]
+                ("dyn_chunk_pages", ctypes.c_int32), ("early_prologue", ctypes.c_int32),
+                ("wait_limit_us", ctypes.c_int32), ("test_withhold_page", ctypes.c_int32)]
 
 
 class tg_plan_info(ctypes.Structure):
@@ -275,13 +276,15 @@ def tg_plan_create(shape: tg_shape, kv_len, group_of_head, group_off, fast_len=N
                    slow_table_len: int = 0, num_workers: int = 0, min_splits: int = 1,
                    max_chunk_pages: int = 0, host_only: bool = False, device: int = -1,
                    static_permille: int = 0, dyn_chunk_pages: int = 0,
-                   early_prologue: bool = False) -> Plan:
+                   early_prologue: bool = False, wait_limit_us: int = 0,
+                   test_withhold_page: int = 0) -> Plan:
     kv = _h(kv_len, np.int32).reshape(-1)
     fl = None if fast_len is None else _h(fast_len, np.int32).reshape(-1)
     goh = _h(group_of_head, np.int32).reshape(-1)
     goff = _h(group_off, np.int64).reshape(-1)
     opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
-                        static_permille, dyn_chunk_pages, int(early_prologue))
+                        static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us,
+                        test_withhold_page)
     h = ctypes.c_void_p()
     _check(_lib().tg_plan_create(ctypes.byref(shape), _hp(kv), _hp(fl), _hp(goh), _hp(goff),
                                  goff.size - 1, slow_table_len, ctypes.byref(opts),

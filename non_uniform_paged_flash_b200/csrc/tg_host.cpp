@@ -524,26 +524,29 @@ extern "C" int tg_plan_create(const tg_shape *shape, const int32_t *kv_len,
     p->shape = s;
     p->G = G;
     p->tiered = fast_len != nullptr;
+    p->pairs = p->tiered ? tg::kPairsTiered : tg::kPairs;
     p->host_only = o.host_only != 0;
     p->n_groups = n_groups;
     p->slow_table_len = slow_table_len;
     p->group_off.assign(group_off, group_off + n_groups + 1);
     p->device = o.device;
     p->early_prologue = o.early_prologue != 0;
+    if (o.wait_limit_us > 0) p->wait_ns = static_cast<uint64_t>(o.wait_limit_us) * 1000ull;
+    p->withhold = o.test_withhold_page > 0 ? o.test_withhold_page : 0;
 
     int32_t workers = o.num_workers;
     if (!p->host_only) {
         int rc = tg::device_num_sms(o.device, &p->num_sms);
         if (rc != TG_OK) { delete p; return rc; }
-        if (workers <= 0) workers = p->num_sms * tg::kPairs;
+        if (workers <= 0) workers = p->num_sms * p->pairs;
     } else if (workers <= 0) {
-        workers = 148 * tg::kPairs;
+        workers = 148 * p->pairs;
     }
     const int32_t sp = o.static_permille <= 0 ? 800 : std::min(1000, o.static_permille);
     const int32_t dc = o.dyn_chunk_pages <= 0 ? 16 : o.dyn_chunk_pages;
     int rc = tg::build_work_list(p, kv_len, fast_len, workers, o.min_splits, o.max_chunk_pages, sp, dc);
     if (rc != TG_OK) { delete p; return rc; }
-    p->grid = (p->n_workers + tg::kPairs - 1) / tg::kPairs;
+    p->grid = (p->n_workers + p->pairs - 1) / p->pairs;
     if (p->n_dyn > 0 && p->grid == 0) p->grid = 1;
     if (p->grid == 0 && !p->empties.empty()) p->grid = 1;  // the kernel also writes empty heads
     if (!p->host_only) {
@@ -570,7 +573,7 @@ extern "C" int tg_plan_get_info(const tg_plan *p, tg_plan_info *info) {
     info->n_dynamic = p->n_dyn;
     info->n_workers = p->n_workers;
     info->grid = p->grid;
-    info->block = tg::kThreads;
+    info->block = p->pairs * 64;
     info->smem_bytes = p->smem_bytes;
     info->stages = p->stages;
     info->device_bytes = p->dev_bytes;

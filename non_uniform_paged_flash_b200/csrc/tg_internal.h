@@ -38,9 +38,12 @@ constexpr uint32_t kErrBadRow = 2u;    // row outside its group table / table
 constexpr uint32_t kErrPlan = 4u;      // device lengths differ from the plan
 constexpr uint32_t kErrTimeout = 8u;   // a bounded wait gave up
 
-// Launch geometry of the decode kernels (see tg_kernels.cu).
-constexpr int kPairs = 4;              // (producer warp, consumer warp) pairs per CTA
-constexpr int kThreads = kPairs * 64;  // threads per CTA
+// Launch geometry of the decode kernels (see tg_kernels.cu): (producer warp, consumer warp)
+// pairs per CTA. (8 pairs for the tiered kernel were tried: at 128 registers per thread its
+// consumer spills, and ptxas does not raise the consumer's budget past a register split.)
+constexpr int kPairs = 4;              // bf16 decode kernel
+constexpr int kPairsTiered = 4;        // tiered decode kernel
+constexpr int kThreads = kPairs * 64;  // threads per CTA of the bf16 decode kernel
 constexpr int kTraceWords = 8;         // worker timeline words (see tg_plan_trace_enable)
 
 }  // namespace tg
@@ -67,7 +70,10 @@ struct tg_plan {
     std::vector<int32_t> planned_kv;  // [B*Hkv]
     int64_t n_partials = 0;
     int32_t merge_warps = 1;          // warps per (split head, row) CTA of the merge kernel
+    int32_t pairs = tg::kPairs;       // worker pairs per CTA of this plan's decode kernel
     bool early_prologue = false;      // see tg_plan_opts.early_prologue
+    uint64_t wait_ns = 4000000000ull; // bound of any single wait in the decode kernel
+    int32_t withhold = 0;             // see tg_plan_opts.test_withhold_page
     int32_t n_workers = 0;
     int64_t kv_bytes = 0;
 

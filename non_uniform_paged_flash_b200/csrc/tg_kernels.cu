@@ -56,7 +56,7 @@ void set_cuda_error(const char *what, int code) {
 // ------------------------------------------------------------------------------------------
 namespace dev {
 
-constexpr uint64_t kWaitNs = 4000000000ull;  // bound of any single wait: 4 s
+constexpr uint64_t kWaitNs = 4000000000ull;  // default bound of any single wait: 4 s
 constexpr uint64_t kDrainNs = 200000000ull;  // bound of the drain after a timeout: 0.2 s
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
@@ -241,6 +241,8 @@ struct DecodeArgs {
     int32_t dyn_first, n_dyn;        // dynamic items: items[dyn_first .. dyn_first + n_dyn)
     uint32_t *dyn_next;              // [0] next dynamic item, [1] producers done (zero between calls)
     int32_t early_prologue;          // read plan/table metadata before the predecessor finishes
+    uint64_t wait_ns;                // bound of any single wait
+    int32_t withhold;                // testing: worker 0 never signals its page number withhold
     uint32_t *err;
     uint64_t *trace;                 // worker timeline (n_workers x kTraceWords) or null
 };
@@ -456,8 +458,8 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
 // ------------------------------------------------------------------------------------------
 // Decode kernel
 // ------------------------------------------------------------------------------------------
-template <int D, bool TIERED>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, bool TIERED, int NPAIRS>
+__global__ void __launch_bounds__(NPAIRS * 64, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ CUtensorMap tm_kq,
@@ -469,22 +471,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
+    // Warps [0, NPAIRS) consume, warps [NPAIRS, 2 NPAIRS) produce; pair p = warps p, NPAIRS + p.
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int pair = warp >> 1;
-    const bool producer = (warp & 1) != 0;
+    const int pair = warp % NPAIRS;
+    const bool producer = warp >= NPAIRS;
     const int stages = a.stages;
-    const int worker = blockIdx.x * kPairs + pair;
+    const int worker = blockIdx.x * NPAIRS + pair;
 
     unsigned char *ring = smem + static_cast<size_t>(pair) * stages * a.stage_bytes;
-    StageHdr *hdr = reinterpret_cast<StageHdr *>(smem + static_cast<size_t>(kPairs) * stages * a.stage_bytes) +
+    StageHdr *hdr = reinterpret_cast<StageHdr *>(smem + static_cast<size_t>(NPAIRS) * stages * a.stage_bytes) +
                     pair * stages;
     uint64_t *bars = reinterpret_cast<uint64_t *>(
-                         smem + static_cast<size_t>(kPairs) * stages * a.stage_bytes +
-                         static_cast<size_t>(kPairs) * stages * sizeof(StageHdr)) +
+                         smem + static_cast<size_t>(NPAIRS) * stages * a.stage_bytes +
+                         static_cast<size_t>(NPAIRS) * stages * sizeof(StageHdr)) +
                      static_cast<size_t>(pair) * stages * 2;
     volatile int32_t *ctl = reinterpret_cast<volatile int32_t *>(
-                                smem + static_cast<size_t>(kPairs) * stages * a.stage_bytes +
-                                static_cast<size_t>(kPairs) * stages * (sizeof(StageHdr) + 16)) +
+                                smem + static_cast<size_t>(NPAIRS) * stages * a.stage_bytes +
+                                static_cast<size_t>(NPAIRS) * stages * (sizeof(StageHdr) + 16)) +
                             pair * 2;  // [0] = pages issued, [1] = abort
 
     const uint32_t full0 = dev::smem_addr(bars), empty0 = dev::smem_addr(bars + stages);
@@ -510,8 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (a.n_empty > 0 && !producer) {
         const int64_t per = static_cast<int64_t>(a.G) * D;
         const int64_t total = static_cast<int64_t>(a.n_empty) * per;
-        const int64_t nthr = static_cast<int64_t>(gridDim.x) * kPairs * 32;
-        for (int64_t i = (static_cast<int64_t>(blockIdx.x) * kPairs + pair) * 32 + lane; i < total; i += nthr) {
+        const int64_t nthr = static_cast<int64_t>(gridDim.x) * NPAIRS * 32;
+        for (int64_t i = (static_cast<int64_t>(blockIdx.x) * NPAIRS + pair) * 32 + lane; i < total; i += nthr) {
             const int32_t bh = a.empties[i / per];
             const int32_t b = bh / a.Hkv, h = bh - b * a.Hkv;
             const int64_t r = i % per;
@@ -626,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int stage = pstage;
                     const uint32_t phase = pphase;
                     wait_predecessor();
-                    const bool ok = dev::mbar_wait(empty0 + 8 * stage, phase ^ 1u, dev::kWaitNs);
+                    const bool ok = dev::mbar_wait(empty0 + 8 * stage, phase ^ 1u, a.wait_ns);
                     if (!ok || ctl[1]) {
                         if (lane == 0) {
                             atomicOr(a.err, kErrTimeout);
@@ -657,7 +660,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t qbytes = static_cast<uint32_t>(a.G * D * 2);
                         uint32_t bytes = first ? qbytes : 0u;
                         if (page_id >= 0) bytes += slow ? 2u * (L::kI8 + 64u) : 2u * L::KB;
-                        if (bytes == 0) {
+                        if (a.withhold && worker == 0 && seq + 1 == static_cast<uint32_t>(a.withhold)) {
+                            // testing: this stage is never signalled; the consumer's bounded
+                            // wait runs out and the call reports a timeout
+                        } else if (bytes == 0) {
                             dev::mbar_arrive(fb);
                         } else {
                             dev::mbar_arrive_expect_tx(fb, bytes);
@@ -714,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Stop marker for the consumer.
             const int stage = pstage;
             const uint32_t phase = pphase;
-            if (!dev::mbar_wait(empty0 + 8 * stage, phase ^ 1u, dev::kWaitNs) || ctl[1]) {
+            if (!dev::mbar_wait(empty0 + 8 * stage, phase ^ 1u, a.wait_ns) || ctl[1]) {
                 if (lane == 0) {
                     atomicOr(a.err, kErrTimeout);
                     ctl[1] = 1;
@@ -732,7 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // The last producer of the launch to finish resets the dynamic queue.
             if (lane == 0 && a.n_dyn > 0) {
                 __threadfence();
-                const uint32_t total = gridDim.x * kPairs;
+                const uint32_t total = gridDim.x * NPAIRS;
                 if (atomicAdd(a.dyn_next + 1, 1u) == total - 1) {
                     a.dyn_next[0] = 0;
                     a.dyn_next[1] = 0;
@@ -786,11 +792,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         const uint32_t issued = static_cast<uint32_t>(ctl[0]);
         for (uint32_t s = seq; s < issued; ++s)
-            dev::mbar_wait(full0 + 8 * (s % stages), (s / stages) & 1u, dev::kDrainNs);
+            dev::mbar_wait(full0 + 8 * (s % stages), (s / stages) & 1u,
+                           a.wait_ns < dev::kDrainNs ? a.wait_ns : dev::kDrainNs);
     };
 
     while (true) {
-        if (!dev::mbar_wait(full0 + 8 * cstage, cphase, dev::kWaitNs)) {
+        if (!dev::mbar_wait(full0 + 8 * cstage, cphase, a.wait_ns)) {
             timed_out();
             return;
         }
@@ -807,7 +814,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int32_t last_flags = hd.flags;
         const bool pair = (hd.flags & kHdrPair) != 0;
         if (pair) {
-            if (!dev::mbar_wait(full0 + 8 * cstage, cphase, dev::kWaitNs)) {
+            if (!dev::mbar_wait(full0 + 8 * cstage, cphase, a.wait_ns)) {
                 timed_out();
                 return;
             }
@@ -1156,9 +1163,9 @@ int device_num_sms(int device, int *num_sms) {
 
 static constexpr int kSmemBudget = 232448;  // 227 KB opt-in dynamic shared memory per CTA
 
-template <int D, bool TIERED>
+template <int D, bool TIERED, int NPAIRS>
 static int set_smem_attr(int bytes) {
-    TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<D, TIERED>,
+    TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<D, TIERED, NPAIRS>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
     return TG_OK;
 }
@@ -1175,19 +1182,20 @@ int device_init_plan(tg_plan *p) {
     const int QB = ((p->G * s.D * 2) + 1023) / 1024 * 1024;
     p->stage_bytes = 2 * KB + QB;
     const int per_stage_extra = static_cast<int>(sizeof(StageHdr)) + 16;  // header + 2 barriers
-    int stages = (kSmemBudget - 1024 - kPairs * 8) / (kPairs * (p->stage_bytes + per_stage_extra));
+    const int np = p->pairs;
+    int stages = (kSmemBudget - 1024 - np * 8) / (np * (p->stage_bytes + per_stage_extra));
     stages = stages > 8 ? 8 : stages;
-    if (stages < 2) {
+    if (stages < 3) {  // a page pair plus one page in flight
         if (p->device != cur) cudaSetDevice(cur);
         return TG_EUNSUPPORTED;
     }
     p->stages = stages;
-    p->smem_bytes = 1024 + kPairs * stages * (p->stage_bytes + per_stage_extra) + kPairs * 8;
+    p->smem_bytes = 1024 + np * stages * (p->stage_bytes + per_stage_extra) + np * 8;
 
     int rc = TG_OK;
-    if (s.D == 128 && !p->tiered) rc = set_smem_attr<128, false>(p->smem_bytes);
-    else if (s.D == 128 && p->tiered) rc = set_smem_attr<128, true>(p->smem_bytes);
-    else if (s.D == 64 && !p->tiered) rc = set_smem_attr<64, false>(p->smem_bytes);
+    if (s.D == 128 && !p->tiered) rc = set_smem_attr<128, false, kPairs>(p->smem_bytes);
+    else if (s.D == 128 && p->tiered) rc = set_smem_attr<128, true, kPairsTiered>(p->smem_bytes);
+    else if (s.D == 64 && !p->tiered) rc = set_smem_attr<64, false, kPairs>(p->smem_bytes);
     else rc = TG_EUNSUPPORTED;
     if (rc != TG_OK) {
         if (p->device != cur) cudaSetDevice(cur);
@@ -1308,7 +1316,7 @@ static int launch_decode(tg_plan *p, DecodeFn fn, const DecodeArgs &a, const CUt
                          cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(p->grid));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(static_cast<unsigned>(p->pairs * 64));
     cfg.dynamicSmemBytes = static_cast<size_t>(p->smem_bytes);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -1378,6 +1386,8 @@ static DecodeArgs base_args(const tg_plan *p, const void *q, const int32_t *kv, 
     a.n_dyn = p->n_dyn;
     a.dyn_next = p->d_dyn;
     a.early_prologue = p->early_prologue ? 1 : 0;
+    a.wait_ns = p->wait_ns;
+    a.withhold = p->withhold;
     return a;
 }
 
@@ -1418,9 +1428,9 @@ extern "C" int tg_ragged_paged_decode(tg_plan *p, const void *q, const void *k_p
         const CUtensorMap &tk = *reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
         const CUtensorMap &tv = *reinterpret_cast<const CUtensorMap *>(p->tmaps[1]);
         if (p->shape.D == 128)
-            rc = launch_decode(p, decode_kernel<128, false>, a, tk, tv, tk, tv, stream);
+            rc = launch_decode(p, decode_kernel<128, false, kPairs>, a, tk, tv, tk, tv, stream);
         else
-            rc = launch_decode(p, decode_kernel<64, false>, a, tk, tv, tk, tv, stream);
+            rc = launch_decode(p, decode_kernel<64, false, kPairs>, a, tk, tv, tk, tv, stream);
         if (rc != TG_OK) return rc;
     } else {
         timing_mark(p, 0, stream);
@@ -1474,7 +1484,7 @@ extern "C" int tg_tiered_decode(tg_plan *p, const void *q, const int8_t *k_q8,
         a.fast_len_dev = head_fast_len;
         // The fast tier's rows are bounded by its whole table [group_off[0], group_off[n]).
         const CUtensorMap *maps = reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
-        rc = launch_decode(p, decode_kernel<128, true>, a, maps[has_fast ? 0 : 2], maps[has_fast ? 1 : 3],
+        rc = launch_decode(p, decode_kernel<128, true, kPairsTiered>, a, maps[has_fast ? 0 : 2], maps[has_fast ? 1 : 3],
                            maps[has_slow ? 2 : 0], maps[has_slow ? 3 : 1], stream);
         if (rc != TG_OK) return rc;
     } else {
@@ -1635,9 +1645,9 @@ int noalloc_setup(int dev, void **ptr) {
             set_cuda_error("cudaGetSymbolAddress(scratch)", static_cast<int>(e));
             return TG_ECUDA;
         }
-        TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<128, false>,
+        TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<128, false, tg::kPairs>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget));
-        TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<64, false>,
+        TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<64, false, tg::kPairs>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget));
         g_noalloc_ptr[dev] = p;
     }
@@ -1684,10 +1694,10 @@ extern "C" int tg_ragged_paged_decode_noalloc(tg_plan *p, const void *q, const v
     const int QB = ((p->G * s.D * 2) + 1023) / 1024 * 1024;
     const int stage_bytes = 2 * KB + QB;
     const int per_stage_extra = static_cast<int>(sizeof(StageHdr)) + 16;
-    int stages = (kSmemBudget - 1024 - kPairs * 8) / (kPairs * (stage_bytes + per_stage_extra));
+    int stages = (kSmemBudget - 1024 - tg::kPairs * 8) / (tg::kPairs * (stage_bytes + per_stage_extra));
     stages = stages > 8 ? 8 : stages;
     if (stages < 2) return TG_EUNSUPPORTED;
-    const int smem_bytes = 1024 + kPairs * stages * (stage_bytes + per_stage_extra) + kPairs * 8;
+    const int smem_bytes = 1024 + tg::kPairs * stages * (stage_bytes + per_stage_extra) + tg::kPairs * 8;
 
     int dev = 0;
     TG_CUDA_TRY(cudaGetDevice(&dev));
@@ -1770,6 +1780,8 @@ extern "C" int tg_ragged_paged_decode_noalloc(tg_plan *p, const void *q, const v
         a.n_dyn = p->n_dyn;
         a.dyn_next = d_dyn;
         a.early_prologue = 0;
+        a.wait_ns = dev::kWaitNs;
+        a.withhold = 0;
         const CUtensorMap &tk = *reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
         const CUtensorMap &tv = *reinterpret_cast<const CUtensorMap *>(p->tmaps[1]);
         cudaLaunchConfig_t cfg = {};
@@ -1778,9 +1790,9 @@ extern "C" int tg_ragged_paged_decode_noalloc(tg_plan *p, const void *q, const v
         cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
         cfg.stream = stream;
         if (s.D == 128)
-            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel<128, false>, a, tk, tv, tk, tv));
+            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel<128, false, tg::kPairs>, a, tk, tv, tk, tv));
         else
-            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel<64, false>, a, tk, tv, tk, tv));
+            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel<64, false, tg::kPairs>, a, tk, tv, tk, tv));
     }
     if (!p->merge.empty()) {
         cudaLaunchConfig_t cfg = {};

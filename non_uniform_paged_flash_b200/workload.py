@@ -201,7 +201,8 @@ def _pool_to_device(sp, which, n, layer, device, chunk_pages=1 << 16):
 
 def to_device(sp: synth.Spec, lay: Layout, layer: int = 0, device="cuda", num_workers: int = 0,
               min_splits: int = 1, max_chunk_pages: int = 0, seqs=None, static_permille: int = 0,
-              dyn_chunk_pages: int = 0, early_prologue: bool = False) -> DeviceBatch:
+              dyn_chunk_pages: int = 0, early_prologue: bool = False, wait_limit_us: int = 0,
+              test_withhold_page: int = 0) -> DeviceBatch:
     import torch
     dev = torch.device(device)
     B = lay.kv_len.shape[0]
@@ -212,6 +213,7 @@ def to_device(sp: synth.Spec, lay: Layout, layer: int = 0, device="cuda", num_wo
                           num_workers=num_workers, min_splits=min_splits,
                           max_chunk_pages=max_chunk_pages, static_permille=static_permille,
                           dyn_chunk_pages=dyn_chunk_pages, early_prologue=early_prologue,
+                          wait_limit_us=wait_limit_us, test_withhold_page=test_withhold_page,
                           device=dev.index if dev.index is not None else -1)
     qb = synth.q_bits(sp, layer)
     q = _bf16_tensor(qb if seqs is None else np.ascontiguousarray(qb[seqs]), dev)

@@ -197,6 +197,28 @@ def test_length_mismatch_with_plan_is_reported():
     assert tg.tg_plan_status(db.plan) == tg.TG_EBADPAGE
 
 
+def test_bounded_wait_runs_out_and_context_survives():
+    """A page that is never signalled (a flag nothing sets) makes the consumer's bounded wait
+    run out: the kernel drains what it issued, returns, and the call reports TG_ETIMEOUT; the
+    context stays usable and a normal plan afterwards gives correct results."""
+    sp = synth.small(2)
+    lay = workload.layout(sp, 0)
+    ol = ors.layout(sp, 0)
+    for withhold in (1, 3):
+        db = workload.to_device(sp, lay, 0, num_workers=16, wait_limit_us=20000,
+                                test_withhold_page=withhold)
+        db.run()
+        torch.cuda.synchronize()
+        assert tg.tg_plan_status(db.plan) == tg.TG_ETIMEOUT
+        del db
+    db = workload.to_device(sp, lay, 0, num_workers=16, wait_limit_us=20000)
+    db.run()
+    torch.cuda.synchronize()
+    assert tg.tg_plan_status(db.plan) == tg.TG_OK
+    ref_out, ref_lse = ors.reference(sp, ol, 0)
+    _compare(db, ref_out, ref_lse)
+
+
 def test_argument_validation():
     sp = synth.small(1)
     db = workload.admit(sp)

@@ -159,6 +159,14 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                       uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // Hardware base-2 exponential and logarithm (PTX ex2.approx / lg2.approx).
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -270,6 +278,7 @@ struct Layout {
 
 // Online-softmax state of the two query heads (2t, 2t+1) a consumer lane accumulates.
 struct PageState {
+    float sq0, sq1;  // INT8 tier: scale of the integer q digits of heads 2t, 2t+1
     float m0, m1;    // running maxima, log2 units
     float le0, le1;  // sums of fp32 probabilities (for the lse)
     float lr0, lr1;  // sums of the probabilities multiplied into V
@@ -313,20 +322,28 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
             }
         }
     } else {
+        // INT8 codes straight into the integer tensor-core path: K (tokens x 32 d, as stored)
+        // times the two int8 digits of q; S = s_q * (K.q1 + K.q2 / 254), exact in int32.
+        int32_t s1[NP][4], s2[NP][4];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) s1[p][0] = s1[p][1] = s1[p][2] = s1[p][3] = s2[p][0] = s2[p][1] = s2[p][2] = s2[p][3] = 0;
 #pragma unroll
         for (int jj = 0; jj < KS / 2; ++jj) {
 #pragma unroll
             for (int p = 0; p < NP; ++p) {
                 uint32_t r0, r1, r2, r3;
                 dev::ldsm_x4(sa[p] + off8[jj], r0, r1, r2, r3);
-                uint32_t a0, a1, a2, a3;
-                dev::i8x4_to_f16x4(r0, a0, a2);
-                dev::i8x4_to_f16x4(r1, a1, a3);
-                dev::mma_f16(s[p], a0, a1, a2, a3, qf[2 * jj][0], qf[2 * jj][1]);
-                dev::i8x4_to_f16x4(r2, a0, a2);
-                dev::i8x4_to_f16x4(r3, a1, a3);
-                dev::mma_f16(s[p], a0, a1, a2, a3, qf[2 * jj + 1][0], qf[2 * jj + 1][1]);
+                dev::mma_s8(s1[p], r0, r1, r2, r3, qf[jj][0], qf[jj][1]);
+                dev::mma_s8(s2[p], r0, r1, r2, r3, qf[KS / 2 + jj][0], qf[KS / 2 + jj][1]);
             }
+        }
+        constexpr float kInv254 = 1.f / 254.f;
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            s[p][0] = ps.sq0 * fmaf(static_cast<float>(s2[p][0]), kInv254, static_cast<float>(s1[p][0]));
+            s[p][1] = ps.sq1 * fmaf(static_cast<float>(s2[p][1]), kInv254, static_cast<float>(s1[p][1]));
+            s[p][2] = ps.sq0 * fmaf(static_cast<float>(s2[p][2]), kInv254, static_cast<float>(s1[p][2]));
+            s[p][3] = ps.sq1 * fmaf(static_cast<float>(s2[p][3]), kInv254, static_cast<float>(s1[p][3]));
         }
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
@@ -838,16 +855,56 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                     if (!slow) {
                         qf[j][0] = *reinterpret_cast<const uint32_t *>(qs + (g * D + 16 * j + 2 * t) * 2);
                         qf[j][1] = *reinterpret_cast<const uint32_t *>(qs + (g * D + 16 * j + 2 * t + 8) * 2);
-                    } else {
-                        // INT8 tier: fp16 q, k-slots (2t, 2t+1, 2t+8, 2t+9) <-> d = 16j + 4t + 0..3
-                        const uint2 v = *reinterpret_cast<const uint2 *>(qs + (g * D + 16 * j + 4 * t) * 2);
-                        qf[j][0] = dev::pack_f16(dev::bf16_lo(v.x), dev::bf16_hi(v.x));
-                        qf[j][1] = dev::pack_f16(dev::bf16_lo(v.y), dev::bf16_hi(v.y));
                     }
                 } else {
                     qf[j][0] = 0u;
                     qf[j][1] = 0u;
                 }
+            }
+            if (slow) {
+                // INT8 tier: q of head g as s_q * (q1 + q2 / 254) with int8 digits q1, q2
+                // (|error| <= max|q| / 64516 per element); B fragments of mma.m16n8k32.s8:
+                // qf[jj] = q1 and qf[KS/2 + jj] = q2 at d = 32 jj + 4t + (0..3 | 16..19).
+                float qv[KSTEPS / 2][8];
+                float amax = 0.f;
+#pragma unroll
+                for (int jj = 0; jj < KSTEPS / 2; ++jj) {
+                    if (g < a.G) {
+                        const uint2 v0 = *reinterpret_cast<const uint2 *>(qs + (g * D + 32 * jj + 4 * t) * 2);
+                        const uint2 v1 = *reinterpret_cast<const uint2 *>(qs + (g * D + 32 * jj + 16 + 4 * t) * 2);
+                        qv[jj][0] = dev::bf16_lo(v0.x); qv[jj][1] = dev::bf16_hi(v0.x);
+                        qv[jj][2] = dev::bf16_lo(v0.y); qv[jj][3] = dev::bf16_hi(v0.y);
+                        qv[jj][4] = dev::bf16_lo(v1.x); qv[jj][5] = dev::bf16_hi(v1.x);
+                        qv[jj][6] = dev::bf16_lo(v1.y); qv[jj][7] = dev::bf16_hi(v1.y);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) qv[jj][e] = 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(qv[jj][e]));
+                }
+                amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
+                amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
+                const float inv = amax > 0.f ? 127.f / amax : 0.f;
+                const float sq = amax / 127.f;
+#pragma unroll
+                for (int jj = 0; jj < KSTEPS / 2; ++jj) {
+                    uint32_t d1[2] = {0u, 0u}, d2[2] = {0u, 0u};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float y = qv[jj][e] * inv;
+                        const int c1 = max(-127, min(127, __float2int_rn(y)));
+                        const int c2 = max(-127, min(127, __float2int_rn((y - static_cast<float>(c1)) * 254.f)));
+                        d1[e >> 2] |= (static_cast<uint32_t>(c1) & 0xFFu) << (8 * (e & 3));
+                        d2[e >> 2] |= (static_cast<uint32_t>(c2) & 0xFFu) << (8 * (e & 3));
+                    }
+                    qf[jj][0] = d1[0];
+                    qf[jj][1] = d1[1];
+                    qf[KSTEPS / 2 + jj][0] = d2[0];
+                    qf[KSTEPS / 2 + jj][1] = d2[1];
+                }
+                ps.sq0 = __shfl_sync(FULL, sq, 8 * t);      // head 2t lives in lanes 4 * 2t + ...
+                ps.sq1 = __shfl_sync(FULL, sq, 8 * t + 4);  // head 2t+1
             }
 #pragma unroll
             for (int i = 0; i < KSTEPS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;

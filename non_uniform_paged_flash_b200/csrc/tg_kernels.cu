@@ -196,13 +196,14 @@ __device__ __forceinline__ float f16_hi(uint32_t v) {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
 }
 
-// Four signed 8-bit integers (|x| <= 128) -> two fp16x2, exactly: bias each byte to x + 128,
-// place it in the low mantissa byte of fp16 1024 (0x6400), subtract 1152.
-__device__ __forceinline__ void i8x4_to_f16x4(uint32_t v, uint32_t &lo, uint32_t &hi) {
+// One ldmatrix.trans register of INT8 V codes, bytes (x[t][d], x[t][d+1], x[t+1][d], x[t+1][d+1]),
+// -> two fp16x2 registers (x[t][d], x[t+1][d]) and (x[t][d+1], x[t+1][d+1]), exactly: bias each
+// byte to x + 128, place it in the low mantissa byte of fp16 1024 (0x6400), subtract 1152.
+__device__ __forceinline__ void i8pair_to_f16(uint32_t v, uint32_t &lo, uint32_t &hi) {
     const uint32_t u = v ^ 0x80808080u;
     uint32_t a, b;
-    asm("prmt.b32 %0, %1, %2, 0x4140;" : "=r"(a) : "r"(u), "r"(0x64646464u));
-    asm("prmt.b32 %0, %1, %2, 0x4342;" : "=r"(b) : "r"(u), "r"(0x64646464u));
+    asm("prmt.b32 %0, %1, %2, 0x4240;" : "=r"(a) : "r"(u), "r"(0x64646464u));
+    asm("prmt.b32 %0, %1, %2, 0x4341;" : "=r"(b) : "r"(u), "r"(0x64646464u));
     const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
     __half2 ha = __hsub2(*reinterpret_cast<__half2 *>(&a), bias);
     __half2 hb = __hsub2(*reinterpret_cast<__half2 *>(&b), bias);
@@ -278,7 +279,7 @@ struct Layout {
 
 // Online-softmax state of the two query heads (2t, 2t+1) a consumer lane accumulates.
 struct PageState {
-    float sq0, sq1;  // INT8 tier: scale of the integer q digits of heads 2t, 2t+1
+    float sq0, sq1;  // INT8 tier: s_q * scale * log2(e) / 254 of heads 2t, 2t+1
     float m0, m1;    // running maxima, log2 units
     float le0, le1;  // sums of fp32 probabilities (for the lse)
     float lr0, lr1;  // sums of the probabilities multiplied into V
@@ -291,7 +292,8 @@ struct PageState {
 // One consumer step over NP pages (1 or 2) of the same item: S = K q^T per page (16 tokens x
 // 8 heads, tokens on M), one max reduction and rescale check for all NP pages, then O^T +=
 // V^T P^T per page. With NP = 2 the two pages' instruction streams interleave (independent
-// chains). SLOW: INT8 pages (codes converted to fp16 in registers, per-token scales).
+// chains). SLOW: INT8 pages (K codes on the s8 tensor path against two int8 digits of q, V codes
+// widened to fp16 in registers, per-token scales).
 template <int D, int NP, bool SLOW>
 __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const int (&valid)[NP],
                                               const uint32_t (&qf)[D / 16][2],
@@ -337,13 +339,11 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
                 dev::mma_s8(s2[p], r0, r1, r2, r3, qf[KS / 2 + jj][0], qf[KS / 2 + jj][1]);
             }
         }
-        constexpr float kInv254 = 1.f / 254.f;
+        // 254 s1 + s2 is exact in int32 (|s1| < 2^21); ps.sq* carries s_q * scale * log2(e) / 254.
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
-            s[p][0] = ps.sq0 * fmaf(static_cast<float>(s2[p][0]), kInv254, static_cast<float>(s1[p][0]));
-            s[p][1] = ps.sq1 * fmaf(static_cast<float>(s2[p][1]), kInv254, static_cast<float>(s1[p][1]));
-            s[p][2] = ps.sq0 * fmaf(static_cast<float>(s2[p][2]), kInv254, static_cast<float>(s1[p][2]));
-            s[p][3] = ps.sq1 * fmaf(static_cast<float>(s2[p][3]), kInv254, static_cast<float>(s1[p][3]));
+#pragma unroll
+            for (int c = 0; c < 4; ++c) s[p][c] = static_cast<float>(s1[p][c] * 254 + s2[p][c]);
         }
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
@@ -364,10 +364,12 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
         const bool v0 = g < valid[p], v1 = g + 8 < valid[p];
-        x[p][0] = v0 ? s[p][0] * ks[p][0] * scale_log2 : -INFINITY;
-        x[p][1] = v0 ? s[p][1] * ks[p][0] * scale_log2 : -INFINITY;
-        x[p][2] = v1 ? s[p][2] * ks[p][1] * scale_log2 : -INFINITY;
-        x[p][3] = v1 ? s[p][3] * ks[p][1] * scale_log2 : -INFINITY;
+        const float f0 = SLOW ? ks[p][0] * ps.sq0 : scale_log2, f1 = SLOW ? ks[p][0] * ps.sq1 : scale_log2;
+        const float f2 = SLOW ? ks[p][1] * ps.sq0 : scale_log2, f3 = SLOW ? ks[p][1] * ps.sq1 : scale_log2;
+        x[p][0] = v0 ? s[p][0] * f0 : -INFINITY;
+        x[p][1] = v0 ? s[p][1] * f1 : -INFINITY;
+        x[p][2] = v1 ? s[p][2] * f2 : -INFINITY;
+        x[p][3] = v1 ? s[p][3] * f3 : -INFINITY;
         mx0 = fmaxf(mx0, fmaxf(x[p][0], x[p][2]));
         mx1 = fmaxf(mx1, fmaxf(x[p][1], x[p][3]));
     }
@@ -456,17 +458,16 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
 #pragma unroll
             for (int p = 0; p < NP; ++p) {
                 uint32_t r0, r1, r2, r3;
-                dev::ldsm_x4(sa[p] + L::KB + off8[ii], r0, r1, r2, r3);
-                // r0: tokens 0-7 chunk 2ii; r1: tokens 8-15 chunk 2ii; r2/r3: chunk 2ii+1
-                uint32_t x0l, x0h, x1l, x1h;
-                dev::i8x4_to_f16x4(r0, x0l, x0h);
-                dev::i8x4_to_f16x4(r1, x1l, x1h);
-                dev::mma_f16(o[2 * ii], dev::movm_t(x0l), dev::movm_t(x0h), dev::movm_t(x1l),
-                             dev::movm_t(x1h), b0[p], b1[p]);
-                dev::i8x4_to_f16x4(r2, x0l, x0h);
-                dev::i8x4_to_f16x4(r3, x1l, x1h);
-                dev::mma_f16(o[2 * ii + 1], dev::movm_t(x0l), dev::movm_t(x0h), dev::movm_t(x1l),
-                             dev::movm_t(x1h), b0[p], b1[p]);
+                dev::ldsm_x4_t(sa[p] + L::KB + off8[ii], r0, r1, r2, r3);
+                // r0/r1: tokens (2t, 2t+1) / (8+2t, 9+2t) at d = 32ii + 2g, +1 (chunk 2ii);
+                // r2/r3: the same for chunk 2ii+1. Tile i rows: g -> d 16i + 2g, g+8 -> +1.
+                uint32_t a0, a1, a2, a3;
+                dev::i8pair_to_f16(r0, a0, a1);
+                dev::i8pair_to_f16(r1, a2, a3);
+                dev::mma_f16(o[2 * ii], a0, a1, a2, a3, b0[p], b1[p]);
+                dev::i8pair_to_f16(r2, a0, a1);
+                dev::i8pair_to_f16(r3, a2, a3);
+                dev::mma_f16(o[2 * ii + 1], a0, a1, a2, a3, b0[p], b1[p]);
             }
         }
     }
@@ -903,8 +904,10 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                     qf[KSTEPS / 2 + jj][0] = d2[0];
                     qf[KSTEPS / 2 + jj][1] = d2[1];
                 }
-                ps.sq0 = __shfl_sync(FULL, sq, 8 * t);      // head 2t lives in lanes 4 * 2t + ...
-                ps.sq1 = __shfl_sync(FULL, sq, 8 * t + 4);  // head 2t+1
+                // per-head factor of the integer scores: s_q * scale * log2(e) / 254
+                const float sqf = sq * (a.scale_log2 * (1.f / 254.f));
+                ps.sq0 = __shfl_sync(FULL, sqf, 8 * t);      // head 2t lives in lanes 4 * 2t + ...
+                ps.sq1 = __shfl_sync(FULL, sqf, 8 * t + 4);  // head 2t+1
             }
 #pragma unroll
             for (int i = 0; i < KSTEPS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
@@ -964,8 +967,8 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         dlo = 16 * i + g;
                         dhi = dlo + 8;
                     } else {
-                        dlo = 16 * i + 4 * (g >> 1) + (g & 1);
-                        dhi = dlo + 2;
+                        dlo = 16 * i + 2 * g;
+                        dhi = dlo + 1;
                     }
                     if (n0 < a.G) {
                         ob[n0 * D + dlo] = __float2bfloat16_rn(o[i][0] * inv0);
@@ -990,8 +993,8 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         dlo = 16 * i + g;
                         dhi = dlo + 8;
                     } else {
-                        dlo = 16 * i + 4 * (g >> 1) + (g & 1);
-                        dhi = dlo + 2;
+                        dlo = 16 * i + 2 * g;
+                        dhi = dlo + 1;
                     }
                     if (n0 < a.G) {
                         po[n0 * D + dlo] = o[i][0] * inv0;

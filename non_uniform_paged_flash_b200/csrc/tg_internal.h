@@ -42,7 +42,7 @@ constexpr uint32_t kErrTimeout = 8u;   // a bounded wait gave up
 // pairs per CTA. (8 pairs for the tiered kernel were tried: at 128 registers per thread its
 // consumer spills, and ptxas does not raise the consumer's budget past a register split.)
 constexpr int kPairs = 4;              // bf16 decode kernel
-constexpr int kPairsTiered = 4;        // tiered decode kernel
+constexpr int kPairsTiered = 6;        // tiered decode kernel (12 warps; 4 ring stages at D = 128)
 constexpr int kThreads = kPairs * 64;  // threads per CTA of the bf16 decode kernel
 constexpr int kTraceWords = 8;         // worker timeline words (see tg_plan_trace_enable)
 

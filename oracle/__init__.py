@@ -54,6 +54,13 @@ def _L():
         lib.or_quantize_int8.argtypes = [i64, i32, p, p, p]
         lib.or_lse_merge.argtypes = [i32, i64, i32, p, p, p, p]
         lib.or_place_sequences.argtypes = [i32, p, i32, p]
+        lib.or_sink_recent_slot.argtypes = [i32, i32, i32, p]
+        lib.or_sink_recent_slot.restype = i32
+        lib.or_h2o_victim.argtypes = [i32, i32, i32, p, p, i32]
+        lib.or_h2o_victim.restype = i32
+        lib.or_token_scores.argtypes = [i32, i32, i32, i32, i32, p, p, i64, p, p, p, f64, p]
+        lib.or_token_scores.restype = ctypes.c_int
+        lib.or_h2o_accumulate.argtypes = [i32, i32, p, p, p, p]
         _lib = lib
     return _lib
 
@@ -214,4 +221,51 @@ def place_sequences(seq_bytes, n_gpus: int) -> np.ndarray:
     b = _c(seq_bytes, np.int64)
     out = np.empty(b.size, dtype=np.int32)
     _L().or_place_sequences(b.size, _ptr(b), n_gpus, _ptr(out))
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+# Decode-step write path.
+# ---------------------------------------------------------------------------------------
+
+def sink_recent_slot(budget: int, sink: int, kv_len: int, slot_pos) -> int:
+    """Slot that receives a head's new token under the sink + recent rule (or -1)."""
+    sp = _c(slot_pos, np.int32)
+    return int(_L().or_sink_recent_slot(int(budget), int(sink), int(kv_len), _ptr(sp)))
+
+
+def h2o_victim(budget: int, recent: int, kv_len: int, slot_pos, score, new_pos: int) -> int:
+    """Slot that receives a head's new token under the H2O rule (or -1)."""
+    sp = _c(slot_pos, np.int32)
+    sc = _c(score, np.float32)
+    return int(_L().or_h2o_victim(int(budget), int(recent), int(kv_len), _ptr(sp), _ptr(sc),
+                                  int(new_pos)))
+
+
+def token_scores(q_bits, k_bits, table, head_off, kv_len, scale, table_len: int, page: int = 16):
+    """Per-token scores of every retained token, float64[table_len * page, G]; NaN where no
+    token is retained."""
+    q = _c(q_bits, np.uint16)
+    k = _c(k_bits, np.uint16)
+    B, Hq, D = q.shape
+    kl = _c(kv_len, np.int32)
+    Hkv = kl.size // B
+    G = Hq // Hkv
+    out = np.full((int(table_len) * page, G), np.nan, dtype=np.float64)
+    rc = _L().or_token_scores(B, Hq, Hkv, D, page, _ptr(q), _ptr(k), k.shape[0],
+                              _ptr(_c(table, np.int32)), _ptr(_c(head_off, np.int64)), _ptr(kl),
+                              float(scale), _ptr(out))
+    if rc:
+        raise ValueError(f"or_token_scores failed ({rc})")
+    return out
+
+
+def h2o_accumulate(s, lse, score):
+    """score[t] + sum_g exp(s[t, g] - lse[g]) for one head, float32[n]."""
+    s_ = _c(s, np.float64)
+    n, G = s_.shape
+    l_ = _c(lse, np.float64)
+    sc = _c(score, np.float32)
+    out = np.empty(n, dtype=np.float32)
+    _L().or_h2o_accumulate(n, G, _ptr(s_), _ptr(l_), _ptr(sc), _ptr(out))
     return out

@@ -477,3 +477,98 @@ void or_place_sequences(int32_t n_seq, const int64_t *seq_bytes, int32_t n_gpus,
     free(order);
     free(load);
 }
+
+/* ---------------------------------------------------------------------------------------
+ * Decode-step write path: where the token of a new decode step goes in a head whose
+ * footprint is fixed. [Tangram] 三大机制 1 (Budget Reservation): each head's post-compression
+ * footprint is fixed when the request starts, so a decode step never reclaims or grows pages;
+ * a head whose reserved slots are all in use replaces one retained token. Which one is the
+ * compression algorithm's choice; Tangram plugs in H2O and others unchanged (落地形态). The
+ * two rules below are the ones [CAP] §2.4.1 describes for decoder-only models:
+ *  (3) static: LM-Infinite / StreamingLLM keep the first tokens and the last L tokens;
+ *  (4) dynamic: H2O keeps the last L tokens plus the tokens with the largest attention
+ *      accumulated at run time.
+ * A head is described by its `budget` reserved slots, `kv_len` of them in use (slots
+ * 0 .. kv_len-1), and slot_pos[i] = sequence position of the token in slot i.
+ * ------------------------------------------------------------------------------------- */
+
+/* Sink + recent. Readings used: the first s = min(sink, budget - 1) positions of the
+ * sequence are the sinks; with a free slot the new token takes slot kv_len; otherwise it
+ * replaces the oldest non-sink token (smallest position >= s), so that the head keeps
+ * positions 0 .. s-1 and the budget - s most recent ones. Returns the slot, or -1 when
+ * budget < 1. */
+int32_t or_sink_recent_slot(int32_t budget, int32_t sink, int32_t kv_len, const int32_t *slot_pos) {
+    if (budget < 1) return -1;
+    if (kv_len < budget) return kv_len;
+    int32_t s = sink < budget - 1 ? sink : budget - 1;
+    if (s < 0) s = 0;
+    int32_t best = -1;
+    for (int32_t i = 0; i < kv_len; ++i) {
+        if (slot_pos[i] < s) continue;
+        if (best < 0 || slot_pos[i] < slot_pos[best]) best = i;
+    }
+    return best;
+}
+
+/* H2O. Readings used: the protected recent window is the last `recent` positions before the
+ * new token (positions >= new_pos - recent); with a free slot the new token takes slot
+ * kv_len; otherwise the victim is the slot with the lowest accumulated score among the older
+ * tokens (ties: the lowest slot); if every token is recent, the slot of the oldest token.
+ * The comparison is on the fp32 scores as stored. Returns the slot, or -1 when budget < 1. */
+int32_t or_h2o_victim(int32_t budget, int32_t recent, int32_t kv_len, const int32_t *slot_pos,
+                      const float *score, int32_t new_pos) {
+    if (budget < 1) return -1;
+    if (kv_len < budget) return kv_len;
+    int32_t best = -1, oldest = 0;
+    for (int32_t i = 0; i < kv_len; ++i) {
+        if (slot_pos[i] < slot_pos[oldest]) oldest = i;
+        if ((int64_t)slot_pos[i] >= (int64_t)new_pos - recent) continue;
+        if (best < 0 || score[i] < score[best]) best = i;
+    }
+    return best >= 0 ? best : oldest;
+}
+
+/* Attention scores of every retained token, fp64: s[t][g] = scale * q[b][h*G+g] . K[t] for
+ * the tokens of every (b, h), t < kv_len[b][h], gathered through the table as in or_decode.
+ * Output out[(head_off[b][h] * page + t) * G + g]; slots beyond kv_len are left untouched.
+ * Returns 0, 3 on a page id outside the pool, 1 on a bad argument. */
+int or_token_scores(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t page, const uint16_t *q,
+                    const uint16_t *k_pool, int64_t num_pages, const int32_t *table,
+                    const int64_t *head_off, const int32_t *kv_len, double scale, double *out) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || page <= 0) return 1;
+    int32_t G = Hq / Hkv;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < (int64_t)B * Hkv; ++bh) {
+        int32_t b = (int32_t)(bh / Hkv), h = (int32_t)(bh % Hkv);
+        for (int64_t t = 0; t < kv_len[bh]; ++t) {
+            int64_t pid = table[head_off[bh] + t / page];
+            if (pid < 0 || pid >= num_pages) {
+#pragma omp atomic write
+                err = 3;
+                break;
+            }
+            const uint16_t *kr = k_pool + (pid * page + t % page) * D;
+            for (int32_t g = 0; g < G; ++g) {
+                const uint16_t *qr = q + ((int64_t)b * Hq + (int64_t)h * G + g) * D;
+                double dot = 0.0;
+                for (int32_t d = 0; d < D; ++d) dot += or_bf16(qr[d]) * or_bf16(kr[d]);
+                out[(head_off[bh] * page + t) * G + g] = scale * dot;
+            }
+        }
+    }
+    return err;
+}
+
+/* H2O accumulation for one head: each retained token's score grows by the attention the
+ * current step's queries pay it, summed over the G query heads of the KV head:
+ *     score[t] += sum_g exp(s[t][g] - lse[g]),
+ * in fp64 from the fp32 score, rounded to fp32 once. s is [n][G], lse [G]. */
+void or_h2o_accumulate(int32_t n, int32_t G, const double *s, const double *lse,
+                       const float *score_in, float *score_out) {
+    for (int32_t t = 0; t < n; ++t) {
+        double acc = (double)score_in[t];
+        for (int32_t g = 0; g < G; ++g) acc += exp(s[(int64_t)t * G + g] - lse[g]);
+        score_out[t] = (float)acc;
+    }
+}

@@ -36,6 +36,10 @@ S_V = 9          # V page contents (bf16 pool)
 S_KSLOW = 10     # K contents of slow-tier pages before INT8 quantisation
 S_VSLOW = 11     # V contents of slow-tier pages before INT8 quantisation
 S_FREE_SLOW = 12 # free-list order of the slow-tier pool
+S_NEWK = 13      # K row of the token a decode step appends (sub = step)
+S_NEWV = 14      # V row of the token a decode step appends (sub = step)
+S_SCORE = 15     # initial accumulated attention score of each retained slot (H2O)
+S_PICK = 16      # which older positions a head retained at admission (H2O)
 
 
 def stream_id(kind: int, sub: int = 0) -> int:
@@ -298,4 +302,43 @@ def pool_page_bits(sp: Spec, which: str, pages: np.ndarray, layer: int = 0) -> n
     for i, p in enumerate(np.asarray(pages, dtype=np.int64)):
         normal_bf16(sp.seed, stream_id(kind, layer), per, i0=int(p) * per,
                     out=out[i].reshape(-1))
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+# Decode-step write path inputs.
+# ---------------------------------------------------------------------------------------
+
+def new_kv_bits(sp: Spec, step: int, which: str, layer: int = 0) -> np.ndarray:
+    """K or V row of the token appended at decode step `step`, per (sequence, KV head):
+    bf16 bits uint16[B, Hkv, D], N(0, 1)."""
+    kind = {"k": S_NEWK, "v": S_NEWV}[which]
+    n = sp.B * sp.Hkv * sp.D
+    return normal_bf16(sp.seed, stream_id(kind, (layer << 16) | step), n).reshape(sp.B, sp.Hkv, sp.D)
+
+
+def init_scores(sp: Spec, n: int, layer: int = 0) -> np.ndarray:
+    """n accumulated attention scores float32 in [0, 4), 24-bit resolution (exact in fp32)."""
+    d = draws(sp.seed, stream_id(S_SCORE, layer), n)
+    return ((d >> np.uint64(40)).astype(np.float64) * 2.0 ** -22).astype(np.float32)
+
+
+def retained_positions(sp: Spec, kv_len: np.ndarray, seen: np.ndarray, recent: int,
+                       layer: int = 0) -> list:
+    """Admission state of each head for the score-based policy: the positions its kv_len
+    retained slots hold, given `seen` tokens so far. The last min(recent, kv_len) positions
+    are kept and the rest is a seeded choice among the older ones; slots hold them in
+    increasing position order. Returns one int32 array per (b, h), row-major."""
+    out = []
+    kv = np.asarray(kv_len).reshape(-1)
+    sn = np.asarray(seen).reshape(-1)
+    for i in range(kv.size):
+        n, L = int(kv[i]), int(sn[i])
+        r = min(recent, n, L)
+        older = L - r
+        k = min(n - r, older)
+        pick = permutation(sp.seed, stream_id(S_PICK, (layer << 20) | i), older)[:k] if k > 0 else \
+            np.zeros(0, np.int64)
+        pos = np.concatenate([np.sort(pick.astype(np.int64)), np.arange(L - r, L)]).astype(np.int32)
+        out.append(pos)
     return out

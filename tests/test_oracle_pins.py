@@ -413,3 +413,123 @@ def test_tiered_equals_untiered_on_exact_values():
                                     fast, 0.125)
     np.testing.assert_allclose(out, ref, atol=1e-12)
     np.testing.assert_allclose(lse, rlse, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------
+# Decode-step write path (sink + recent, H2O): hand-worked cases, closed forms, invariants.
+# ---------------------------------------------------------------------------------------
+
+def _run_sink_recent(budget, sink, kv_len, slot_pos, new_positions):
+    pos = list(slot_pos) + [-1] * (budget - len(slot_pos))
+    n = kv_len
+    slots = []
+    for p in new_positions:
+        s = oracle.sink_recent_slot(budget, sink, n, np.array(pos[:max(n, 1)], np.int32))
+        slots.append(s)
+        pos[s] = p
+        n = max(n, s + 1)
+    return slots, pos[:n]
+
+
+def test_sink_recent_golden():
+    for c in gold("write_path.json")["sink_recent"]:
+        slots, final = _run_sink_recent(c["budget"], c["sink"], c["kv_len"], c["slot_pos"], c["new_pos"])
+        assert slots == c["slots"], c["work"]
+        assert final == c["final_pos"], c["work"]
+
+
+def test_sink_recent_keeps_first_and_last_tokens():
+    """Closed form of the rule the pages describe: after any number of steps a full head holds
+    exactly the first s positions and the last budget - s positions."""
+    rng = np.random.default_rng(40)
+    for _ in range(200):
+        budget = int(rng.integers(1, 40))
+        sink = int(rng.integers(0, 6))
+        L = int(rng.integers(budget, 200))
+        s = min(sink, budget - 1)
+        start = list(range(s)) + list(range(L - (budget - s), L))
+        T = int(rng.integers(0, 120))
+        _, final = _run_sink_recent(budget, sink, budget, start, range(L, L + T))
+        want = set(range(s)) | set(range(L + T - (budget - s), L + T))
+        assert sorted(final) == sorted(want)
+
+
+def test_h2o_golden():
+    for c in gold("write_path.json")["h2o"]:
+        got = oracle.h2o_victim(c["budget"], c["recent"], c["kv_len"], np.array(c["slot_pos"], np.int32),
+                                np.array(c["score"], np.float32), c["new_pos"])
+        assert got == c["slot"], c["work"]
+
+
+def test_h2o_with_age_scores_is_a_sliding_window():
+    """Special case: when every token's score equals its position, the lowest-scored candidate
+    is the oldest token, so H2O reduces to a sliding window of the last `budget` positions."""
+    rng = np.random.default_rng(41)
+    for _ in range(100):
+        budget = int(rng.integers(1, 30))
+        recent = int(rng.integers(0, 40))
+        L = int(rng.integers(budget, 100))
+        pos = np.arange(L - budget, L, dtype=np.int32)
+        rng.shuffle(pos)
+        for p in range(L, L + int(rng.integers(1, 80))):
+            v = oracle.h2o_victim(budget, recent, budget, pos, pos.astype(np.float32), p)
+            pos[v] = p
+        assert sorted(pos.tolist()) == list(range(p + 1 - budget, p + 1))
+
+
+def test_h2o_never_evicts_the_recent_window():
+    rng = np.random.default_rng(42)
+    for _ in range(300):
+        budget = int(rng.integers(2, 50))
+        recent = int(rng.integers(0, budget))
+        L = budget + int(rng.integers(0, 100))
+        pos = np.sort(rng.choice(L, size=budget, replace=False)).astype(np.int32)
+        pos[-min(recent, budget):] = np.arange(L - min(recent, budget), L) if recent else pos[-1:]
+        pos = np.unique(pos)
+        if pos.size < budget:
+            continue
+        score = rng.random(budget).astype(np.float32)
+        v = oracle.h2o_victim(budget, recent, budget, pos, score, L)
+        older = pos < L - recent
+        if older.any():
+            assert older[v]
+            assert score[v] == score[older].min()
+            assert v == np.flatnonzero(older & (score == score[older].min()))[0]
+        else:
+            assert pos[v] == pos.min()
+
+
+def test_token_scores_logsumexp_equals_decode_lse():
+    """The per-token scores tie to the (pinned) decode: ln sum_t exp(s_t) is its lse."""
+    sp = synth.small(2)
+    from tests import _oracle_side as ors
+    lay = ors.layout(sp, 0)
+    q = synth.q_bits(sp)
+    k = synth.pool_bits(sp, "k", lay.num_pages)
+    s = oracle.token_scores(q, k, lay.table, lay.head_off, lay.kv_len, sp.scale, lay.table.size)
+    _, ref_lse = ors.reference(sp, lay, 0)
+    G = sp.Hq // sp.Hkv
+    for b in range(sp.B):
+        for h in range(sp.Hkv):
+            n = int(lay.kv_len[b, h])
+            base = int(lay.head_off[b, h]) * sp.page
+            st = s[base:base + n]
+            assert not np.isnan(st).any()
+            for g in range(G):
+                want = ref_lse[b * sp.Hq + h * G + g]
+                got = np.logaddexp.reduce(st[:, g]) if n else -np.inf
+                assert got == pytest.approx(want, abs=1e-9)
+
+
+def test_h2o_accumulate_adds_one_per_query_head():
+    """Each query head's attention sums to 1 over the retained tokens, so the scores of a head
+    grow by G in total per step."""
+    rng = np.random.default_rng(43)
+    for n, G in ((1, 1), (7, 4), (300, 8)):
+        s = rng.normal(size=(n, G)) * 3
+        lse = np.logaddexp.reduce(s, axis=0)
+        sc0 = (rng.random(n) * 4).astype(np.float32)
+        sc1 = oracle.h2o_accumulate(s, lse, sc0)
+        assert (sc1 >= sc0).all()
+        inc = sc1.astype(np.float64) - sc0.astype(np.float64)
+        assert inc.sum() == pytest.approx(G, abs=n * 4 * 2.0 ** -23)

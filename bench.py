@@ -427,6 +427,119 @@ def run_ours(args):
     return 0
 
 
+def run_write_path(args):
+    """Decode step with the write path on one GPU: append one token per (sequence, KV head)
+    into the full, fixed-budget heads, then the decode (+ merge); with --path h2o the decode
+    also writes the token scores and the H2O update accumulates them and picks the next step's
+    victims. Prints one JSON line with the step time and each kernel's time and bytes."""
+    import torch
+    import non_uniform_paged_flash_b200 as tg
+    from non_uniform_paged_flash_b200 import workload
+
+    cfg = args.config
+    sp = synth.preset(cfg)
+    if sp.kind == "tiered":
+        raise SystemExit("the write path is built for the bf16 tier")
+    lay = workload.layout(sp, 0)
+    db = workload.to_device(sp, lay, 0, **_plan_kw(cfg))
+    B, Hkv = lay.kv_len.shape
+    G = sp.Hq // sp.Hkv
+    dev = db.q.device
+    stream = torch.cuda.current_stream()
+    shape = tg.make_shape(B, sp.Hq, sp.Hkv, sp.D, lay.num_pages)
+    it = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).to(dev)
+    budget = it(lay.kv_len, np.int32)
+    k_new = workload._bf16_tensor(synth.new_kv_bits(sp, 0, "k"), dev)
+    v_new = workload._bf16_tensor(synth.new_kv_bits(sp, 0, "v"), dev)
+    slot_out = torch.empty(B * Hkv, dtype=torch.int32, device=dev)
+    cursor = torch.zeros(B * Hkv, dtype=torch.int32, device=dev)
+    slots = lay.table.size * 16
+    L = synth.full_lengths(sp).astype(np.int64)
+    recent = 64
+    h2o = args.path == "h2o"
+    if h2o:
+        pos = np.full(slots, -1, np.int32)
+        for bh, pp in enumerate(synth.retained_positions(sp, lay.kv_len, np.repeat(L, Hkv), recent)):
+            o = int(lay.head_off.reshape(-1)[bh]) * 16
+            pos[o:o + pp.size] = pp
+        slot_pos = it(pos, np.int32)
+        slot_score = it(synth.init_scores(sp, slots), np.float32)
+        ts = torch.zeros((slots, G), dtype=torch.float32, device=dev)
+        victim = torch.empty(B * Hkv, dtype=torch.int32, device=dev)
+        n_pos = args.warmup + args.steps + 1
+        positions = it(L[None, :] + np.arange(n_pos)[:, None], np.int32)  # [step][B]
+        tg.tg_h2o_update(shape, recent, None, None, db.head_off, budget, db.kv_len, slot_pos,
+                         slot_score, positions[0], victim)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    n_ev = min(args.steps, 256)
+    marks = [[ev() for _ in range(5)] for _ in range(n_ev)]
+
+    def step(i, m=None):
+        if m: m[0].record(stream)
+        if h2o:
+            tg.tg_append_h2o(shape, k_new, v_new, db.k, db.v, db.table, db.head_off, budget,
+                             db.kv_len, victim, slot_pos, slot_score, positions[i], slot_out, stream)
+        else:
+            tg.tg_append_sink_recent(shape, 4, k_new, v_new, db.k, db.v, db.table, db.head_off,
+                                     budget, db.kv_len, cursor, slot_out, stream)
+        if m: m[1].record(stream)
+        if h2o:
+            tg.tg_ragged_paged_decode_scores(db.plan, db.q, db.k, db.v, db.table, db.head_off,
+                                             db.kv_len, db.group_of_head, sp.scale, db.out,
+                                             db.lse, ts, stream)
+        else:
+            db.run(stream)
+        if m: m[2].record(stream)
+        if h2o:
+            tg.tg_h2o_update(shape, recent, ts, db.lse, db.head_off, budget, db.kv_len, slot_pos,
+                             slot_score, positions[i + 1], victim, stream)
+        if m: m[3].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert tg.tg_plan_status(db.plan) == tg.TG_OK
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms_step = e0.elapsed_time(e1) / args.steps
+    for i in range(n_ev):                       # per-kernel times, separate (marked) steps
+        step(args.warmup + i, marks[i])
+    torch.cuda.synchronize()
+    assert tg.tg_plan_status(db.plan) == tg.TG_OK
+    avg = lambda a, b: statistics.mean(m[a].elapsed_time(m[b]) for m in marks)
+    t_app, t_dec, t_upd = avg(0, 1), avg(1, 2), avg(2, 3)
+    alg = workload.algorithmic_bytes(sp, lay)
+    tokens = int(lay.kv_len.sum())
+    app_bytes = B * Hkv * (4 * sp.D * 2 + 12 + (8 if h2o else 4))
+    upd_bytes = tokens * (4 * G + 12) + B * Hkv * 16 if h2o else 0
+    dec_bytes = alg["total"] + (tokens * 4 * G if h2o else 0)
+    peak, peak_kind = _measured_peak()
+    line = {
+        "metric": "decode step with %s write path: step time" % ("H2O" if h2o else "sink+recent"),
+        "value": ms_step * 1e3, "unit": "us", "higher_is_better": False, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup,
+        "config": {"workload": WORKLOAD_NAMES[cfg], "config_id": cfg, "recent": recent if h2o else None,
+                   "sink": None if h2o else 4},
+        "kernels_us": {"append": t_app * 1e3, "decode+merge": t_dec * 1e3,
+                       "h2o_update": t_upd * 1e3 if h2o else None},
+        "bytes": {"append": app_bytes, "decode": dec_bytes, "h2o_update": upd_bytes},
+        "achieved_gbs": {"append": app_bytes / (t_app * 1e-3) / 1e9,
+                         "h2o_update": upd_bytes / (t_upd * 1e-3) / 1e9 if h2o else None},
+        "peak_gbs": peak, "peak_kind": peak_kind, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,11 +548,16 @@ def main():
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="decode", choices=["decode", "sink", "h2o"],
+                    help="decode: the decode step (default); sink / h2o: the decode step with "
+                         "the write path (one GPU, separate JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.path != "decode":
+        return run_write_path(args)
     return run_ours(args)
 
 

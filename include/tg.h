@@ -288,6 +288,17 @@ int tg_ragged_paged_decode(tg_plan *plan, const void *q, const void *k_pages,
  * it: calls whose work overlaps on the GPU (other streams, other host threads) race and must
  * be serialised by the caller. Kernel-side range errors are skipped as in the plan-based
  * entry but are not reported. Calls no cudaMalloc, cudaFree or allocating library routine. */
+/* tg_ragged_paged_decode that also writes every retained token's scores for the H2O rule
+ * below: token_scores (device fp32, 4-byte aligned, [table_len*16][G]) gets, at entry
+ * (head_page_off[b*Hkv+h]*16 + t)*G + g, s = scale * q[b][h*G+g] . K_t (natural-log units, as
+ * computed for the softmax) for every retained t < head_kv_len; other entries are untouched.
+ * Costs 4*G bytes of writes per retained token. */
+int tg_ragged_paged_decode_scores(tg_plan *plan, const void *q, const void *k_pages,
+                                  const void *v_pages, const int32_t *page_table,
+                                  const int64_t *head_page_off, const int32_t *head_kv_len,
+                                  const int32_t *group_of_head, float scale, void *out, float *lse,
+                                  float *token_scores, tg_stream stream);
+
 int tg_ragged_paged_decode_noalloc(tg_plan *plan, const void *q, const void *k_pages,
                                    const void *v_pages, const int32_t *page_table,
                                    const int64_t *head_page_off, const int32_t *head_kv_len,
@@ -301,9 +312,11 @@ int tg_ragged_paged_decode_noalloc(tg_plan *plan, const void *q, const void *k_p
  *   k_q8, v_q8       device int8 [num_slow_pages][16][D] (symmetric codes)
  *   k_scale, v_scale device fp32 [num_slow_pages][16] (per token per head): K_t = code * scale
  *   k_fast, v_fast   device bf16 [num_pages][16][D]
- * The INT8 rows are converted exactly to fp16 in registers; the K scale multiplies the score
- * and the V scale multiplies the probability before P.V (both in fp32). plan from
- * tg_plan_create with this fast_len. D must be 128. */
+ * INT8 K codes enter an integer tensor-core product against q written per row as two int8
+ * digits, q = s_q (q1 + q2/254) (|error| <= max|q| / 64516 per element), exact in int32; INT8
+ * V codes are converted exactly to fp16 in registers; the K scale multiplies the score and the
+ * V scale multiplies the probability before P.V (both in fp32). plan from tg_plan_create with
+ * this fast_len. D must be 128. */
 int tg_tiered_decode(tg_plan *plan, const void *q, const int8_t *k_q8, const int8_t *v_q8,
                      const float *k_scale, const float *v_scale, const int32_t *slow_page_table,
                      const int64_t *slow_head_off, const void *k_fast, const void *v_fast,
@@ -328,6 +341,59 @@ int tg_lse_merge(int64_t n_rows, int32_t D, const int64_t *row_split_off, const 
  * A page of the INT8 pool is 16 consecutive rows. */
 int tg_quantize_int8(int64_t n_rows, int32_t D, const void *src, int8_t *codes, float *scale,
                      tg_stream stream);
+
+/* =====================================================================================
+ * Decode-step write path ("Tangram" 三大机制 1 Budget Reservation and 落地形态; CAP §2.4.1
+ * (3) static and (4) dynamic sparsity of decoder-only models).
+ * A head's footprint is fixed when its request starts: head_budget[b*Hkv+h] slots, laid out
+ * like the retained tokens (slot t in page page_table[head_page_off[b*Hkv+h] + t/16], row
+ * t % 16; the caller reserved ceil(budget/16) pages). head_kv_len counts the slots in use,
+ * 0 .. kv_len-1. A decode step appends one token per (sequence, KV head): a head with a free
+ * slot takes it (kv_len grows by one); a full head overwrites one retained token and keeps
+ * kv_len = budget, so no page is ever reclaimed or added. Per-slot metadata (slot_pos,
+ * slot_score) is indexed by table position: entry head_page_off[b*Hkv+h]*16 + t.
+ * Common arguments: shape (B, Hq, Hkv, D with D % 8 == 0, page = 16, num_pages); k_new, v_new
+ * device bf16 [B][Hkv][D], 16-byte aligned: the step's new rows; k_pages, v_pages the bf16
+ * pool (written); slot_out device int32 [B*Hkv]: the slot written, or -1 when nothing was
+ * written (budget < 1, or the table's page id outside [0, num_pages)). All device pointers;
+ * calls are stream-ordered and allocate nothing. Returns TG_EINVAL on a null/misaligned
+ * pointer or bad shape, TG_ECUDA on a launch error.
+ * ===================================================================================== */
+
+/* Static rule (LM-Infinite / StreamingLLM): keep the first s = min(sink, budget-1) positions of
+ * the sequence and the budget - s most recent. A full head overwrites slot s + cursor and
+ * advances cursor modulo budget - s; head_cursor (int32 [B*Hkv], in/out) is 0 for a head whose
+ * retained tokens sit in slots in position order, sinks first. One launch, one warp per head;
+ * moves 4*D bytes per head. */
+int tg_append_sink_recent(const tg_shape *shape, int32_t sink, const void *k_new,
+                          const void *v_new, void *k_pages, void *v_pages,
+                          const int32_t *page_table, const int64_t *head_page_off,
+                          const int32_t *head_budget, int32_t *head_kv_len, int32_t *head_cursor,
+                          int32_t *slot_out, tg_stream stream);
+
+/* Score-based rule (H2O), append half: a full head overwrites slot head_victim[b*Hkv+h] (int32
+ * [B*Hkv], from tg_h2o_update; ignored while the head has a free slot, which is taken
+ * instead); the written slot's slot_pos (int32, in/out) becomes new_pos[b] (int32 [B]) and its
+ * slot_score (fp32, in/out) 0. One launch, one warp per head. */
+int tg_append_h2o(const tg_shape *shape, const void *k_new, const void *v_new, void *k_pages,
+                  void *v_pages, const int32_t *page_table, const int64_t *head_page_off,
+                  const int32_t *head_budget, int32_t *head_kv_len, const int32_t *head_victim,
+                  int32_t *slot_pos, float *slot_score, const int32_t *new_pos,
+                  int32_t *slot_out, tg_stream stream);
+
+/* Score-based rule (H2O), bookkeeping half, run after a decode step: each retained token's
+ * score grows by the attention the step's G query heads paid it,
+ *   slot_score += sum_g exp(token_scores[entry][g] - lse[b][h*G+g])
+ * (token_scores from tg_ragged_paged_decode_scores, lse from the same call; token_scores =
+ * NULL skips this), then head_victim[b*Hkv+h] gets the slot the next token takes: kv_len while
+ * the head has a free slot; else, among tokens older than the last `recent` positions
+ * (slot_pos < next_pos[b] - recent), the lowest score (ties: lowest slot); if every token is
+ * recent, the oldest one; -1 for budget < 1. One launch, one CTA per head; reads 8 + 4*G bytes
+ * and writes 4 per retained token. */
+int tg_h2o_update(const tg_shape *shape, int32_t recent, const float *token_scores,
+                  const float *lse, const int64_t *head_page_off, const int32_t *head_budget,
+                  const int32_t *head_kv_len, const int32_t *slot_pos, float *slot_score,
+                  const int32_t *next_pos, int32_t *head_victim, tg_stream stream);
 
 #ifdef __cplusplus
 }

@@ -95,6 +95,14 @@ _SIGS = [
                                         _F32, _P, _P, _P]),
     ("tg_lse_merge", ctypes.c_int, [_I64, _I32, _P, _P, _P, _P, _P, _P]),
     ("tg_quantize_int8", ctypes.c_int, [_I64, _I32, _P, _P, _P, _P]),
+    ("tg_ragged_paged_decode_scores", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _F32, _P,
+                                                     _P, _P, _P]),
+    ("tg_append_sink_recent", ctypes.c_int, [ctypes.POINTER(tg_shape), _I32, _P, _P, _P, _P, _P,
+                                             _P, _P, _P, _P, _P, _P]),
+    ("tg_append_h2o", ctypes.c_int, [ctypes.POINTER(tg_shape), _P, _P, _P, _P, _P, _P, _P, _P,
+                                     _P, _P, _P, _P, _P, _P]),
+    ("tg_h2o_update", ctypes.c_int, [ctypes.POINTER(tg_shape), _I32, _P, _P, _P, _P, _P, _P, _P,
+                                     _P, _P, _P]),
 ]
 
 #: Symbols the C ABI exports (include/tg.h).
@@ -365,6 +373,47 @@ def tg_ragged_paged_decode_noalloc(plan: Plan, q, k_pages, v_pages, page_table, 
         plan.handle, _dp(q), _dp(k_pages), _dp(v_pages), _dp(page_table), _dp(head_page_off),
         _dp(head_kv_len), _dp(group_of_head), float(scale), _dp(out), _dp(lse),
         _stream(stream)), "tg_ragged_paged_decode_noalloc")
+
+
+def tg_ragged_paged_decode_scores(plan: Plan, q, k_pages, v_pages, page_table, head_page_off,
+                                  head_kv_len, group_of_head, scale: float, out, lse,
+                                  token_scores, stream=None):
+    """As tg_ragged_paged_decode, also writing every retained token's scores
+    s = scale * q . K_t to token_scores (fp32 [table_len * 16, G])."""
+    _check(_lib().tg_ragged_paged_decode_scores(
+        plan.handle, _dp(q), _dp(k_pages), _dp(v_pages), _dp(page_table), _dp(head_page_off),
+        _dp(head_kv_len), _dp(group_of_head), float(scale), _dp(out), _dp(lse),
+        _dp(token_scores), _stream(stream)), "tg_ragged_paged_decode_scores")
+
+
+def tg_append_sink_recent(shape: tg_shape, sink: int, k_new, v_new, k_pages, v_pages,
+                          page_table, head_page_off, head_budget, head_kv_len, head_cursor,
+                          slot_out, stream=None):
+    """Decode-step append under the sink + recent rule (see include/tg.h)."""
+    _check(_lib().tg_append_sink_recent(
+        ctypes.byref(shape), int(sink), _dp(k_new), _dp(v_new), _dp(k_pages), _dp(v_pages),
+        _dp(page_table), _dp(head_page_off), _dp(head_budget), _dp(head_kv_len),
+        _dp(head_cursor), _dp(slot_out), _stream(stream)), "tg_append_sink_recent")
+
+
+def tg_append_h2o(shape: tg_shape, k_new, v_new, k_pages, v_pages, page_table, head_page_off,
+                  head_budget, head_kv_len, head_victim, slot_pos, slot_score, new_pos,
+                  slot_out, stream=None):
+    """Decode-step append under the H2O rule, into the slots tg_h2o_update chose."""
+    _check(_lib().tg_append_h2o(
+        ctypes.byref(shape), _dp(k_new), _dp(v_new), _dp(k_pages), _dp(v_pages),
+        _dp(page_table), _dp(head_page_off), _dp(head_budget), _dp(head_kv_len),
+        _dp(head_victim), _dp(slot_pos), _dp(slot_score), _dp(new_pos), _dp(slot_out),
+        _stream(stream)), "tg_append_h2o")
+
+
+def tg_h2o_update(shape: tg_shape, recent: int, token_scores, lse, head_page_off, head_budget,
+                  head_kv_len, slot_pos, slot_score, next_pos, head_victim, stream=None):
+    """H2O score accumulation (token_scores may be None) and the next step's victims."""
+    _check(_lib().tg_h2o_update(
+        ctypes.byref(shape), int(recent), _dp(token_scores), _dp(lse), _dp(head_page_off),
+        _dp(head_budget), _dp(head_kv_len), _dp(slot_pos), _dp(slot_score), _dp(next_pos),
+        _dp(head_victim), _stream(stream)), "tg_h2o_update")
 
 
 def tg_tiered_decode(plan: Plan, q, k_q8, v_q8, k_scale, v_scale, slow_page_table,

@@ -254,14 +254,17 @@ struct DecodeArgs {
     int32_t withhold;                // testing: worker 0 never signals its page number withhold
     uint32_t *err;
     uint64_t *trace;                 // worker timeline (n_workers x kTraceWords) or null
+    float *token_scores;             // bf16 kernel: per-token scores [table_len*16][G], or null
 };
 
 // Per-stage header written by the producer before it arrives on the stage's full barrier.
-struct StageHdr {
+struct alignas(16) StageHdr {
     int32_t valid;  // valid tokens in this page (0 when the page was skipped)
     int32_t flags;  // kHdr* bits
     int32_t bh;
     int32_t slot;
+    int64_t tpos;   // table position of the page (head row offset + page index in the row)
+    int64_t pad;
 };
 constexpr int32_t kHdrSlow = 1, kHdrFirst = 2, kHdrLast = 4, kHdrStop = 8, kHdrPair = 16;
 constexpr int32_t kNoLoad = -2;  // page id placeholder of a row that failed its bounds check
@@ -301,7 +304,8 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
                                               const uint32_t (&offK)[D / 16],
                                               const uint32_t (&offV)[D / 16],
                                               const uint32_t (&off8)[D / 32], float scale_log2,
-                                              int lane) {
+                                              int lane, float *ts = nullptr, int64_t tpos = 0,
+                                              int32_t G = 0) {
     using L = Layout<D>;
     constexpr int KS = D / 16;
     constexpr unsigned FULL = 0xffffffffu;
@@ -377,6 +381,24 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
     for (int off = 4; off < 32; off <<= 1) {
         mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
         mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
+    }
+    if (!SLOW && ts != nullptr) {
+        // Per-token scores s = x * ln 2 of the valid tokens, entry (tpos * 16 + token) * G + head.
+        constexpr float kLn2f = 0.69314718055994530942f;
+        const int n0 = 2 * t, n1 = 2 * t + 1;
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            float *e0 = ts + ((tpos + p) * 16 + g) * G;
+            float *e1 = e0 + 8 * G;
+            if (g < valid[p]) {
+                if (n0 < G) e0[n0] = x[p][0] * kLn2f;
+                if (n1 < G) e0[n1] = x[p][1] * kLn2f;
+            }
+            if (g + 8 < valid[p]) {
+                if (n0 < G) e1[n0] = x[p][2] * kLn2f;
+                if (n1 < G) e1[n1] = x[p][3] * kLn2f;
+            }
+        }
     }
     // Lazy rescale: the running max moves only when a tile exceeds it by more than the
     // threshold (2^8 for bf16 probabilities; exact for the fp16 INT8 path).
@@ -633,6 +655,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
             int32_t ids_n = jn < nc ? ids_of(jn, pn) : kNoLoad;
             while (j < nc) {
                 const int32_t bh = __shfl_sync(FULL, mi.bh, j);
+                const int64_t row_j = __shfl_sync(FULL, mrow, j);
                 const int32_t pb = __shfl_sync(FULL, mi.page_begin, j);
                 const int32_t pe = __shfl_sync(FULL, mi.page_end, j);
                 const int32_t tt = __shfl_sync(FULL, mi.tier_tokens, j);
@@ -672,6 +695,8 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                                    (last ? kHdrLast : 0) | (pair ? kHdrPair : 0);
                         hd.bh = bh;
                         hd.slot = slot;
+                        hd.tpos = row_j + pg;
+                        hd.pad = 0;
                         hdr[stage] = hd;
                         const uint32_t st = dev::smem_addr(ring + static_cast<size_t>(stage) * a.stage_bytes);
                         const uint32_t fb = full0 + 8 * stage;
@@ -749,6 +774,8 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                 hd.flags = kHdrStop;
                 hd.bh = 0;
                 hd.slot = -1;
+                hd.tpos = 0;
+                hd.pad = 0;
                 hdr[stage] = hd;
                 dev::mbar_arrive(full0 + 8 * stage);
                 ctl[0] = static_cast<int32_t>(seq + 1);
@@ -919,11 +946,13 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
             if (pair) {
                 const uint32_t sa[2] = {aA, aB};
                 const int va[2] = {hd.valid, validB};
-                consume_pages<D, 2, false>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
+                consume_pages<D, 2, false>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane,
+                                           a.token_scores, hd.tpos, a.G);
             } else {
                 const uint32_t sa[1] = {aA};
                 const int va[1] = {hd.valid};
-                consume_pages<D, 1, false>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
+                consume_pages<D, 1, false>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane,
+                                           a.token_scores, hd.tpos, a.G);
             }
         } else if (TIERED) {
             if (pair) {
@@ -1460,11 +1489,10 @@ using namespace tg;
 
 extern "C" const char *tg_last_cuda_error(void) { return g_cuda_msg; }
 
-extern "C" int tg_ragged_paged_decode(tg_plan *p, const void *q, const void *k_pages,
-                                      const void *v_pages, const int32_t *page_table,
-                                      const int64_t *head_page_off, const int32_t *head_kv_len,
-                                      const int32_t *group_of_head, float scale, void *out,
-                                      float *lse, tg_stream stream_) {
+static int decode_bf16(tg_plan *p, const void *q, const void *k_pages, const void *v_pages,
+                       const int32_t *page_table, const int64_t *head_page_off,
+                       const int32_t *head_kv_len, const int32_t *group_of_head, float scale,
+                       void *out, float *lse, float *token_scores, tg_stream stream_) {
     if (!p || p->host_only || p->tiered) return TG_EINVAL;
     if (!q || !out || !lse || !head_kv_len || !aligned16(q) || !aligned16(out) || !aligned16(lse))
         return TG_EINVAL;
@@ -1485,6 +1513,7 @@ extern "C" int tg_ragged_paged_decode(tg_plan *p, const void *q, const void *k_p
         a.table = page_table;
         a.head_off = head_page_off;
         a.group_of_head = group_of_head;
+        a.token_scores = token_scores;
         const CUtensorMap &tk = *reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
         const CUtensorMap &tv = *reinterpret_cast<const CUtensorMap *>(p->tmaps[1]);
         if (p->shape.D == 128)
@@ -1496,6 +1525,27 @@ extern "C" int tg_ragged_paged_decode(tg_plan *p, const void *q, const void *k_p
         timing_mark(p, 0, stream);
     }
     return finish_call(p, out, lse, stream);
+}
+
+extern "C" int tg_ragged_paged_decode(tg_plan *p, const void *q, const void *k_pages,
+                                      const void *v_pages, const int32_t *page_table,
+                                      const int64_t *head_page_off, const int32_t *head_kv_len,
+                                      const int32_t *group_of_head, float scale, void *out,
+                                      float *lse, tg_stream stream) {
+    return decode_bf16(p, q, k_pages, v_pages, page_table, head_page_off, head_kv_len,
+                       group_of_head, scale, out, lse, nullptr, stream);
+}
+
+extern "C" int tg_ragged_paged_decode_scores(tg_plan *p, const void *q, const void *k_pages,
+                                             const void *v_pages, const int32_t *page_table,
+                                             const int64_t *head_page_off,
+                                             const int32_t *head_kv_len,
+                                             const int32_t *group_of_head, float scale,
+                                             void *out, float *lse, float *token_scores,
+                                             tg_stream stream) {
+    if (!token_scores || (reinterpret_cast<uintptr_t>(token_scores) & 3u)) return TG_EINVAL;
+    return decode_bf16(p, q, k_pages, v_pages, page_table, head_page_off, head_kv_len,
+                       group_of_head, scale, out, lse, token_scores, stream);
 }
 
 extern "C" int tg_tiered_decode(tg_plan *p, const void *q, const int8_t *k_q8,

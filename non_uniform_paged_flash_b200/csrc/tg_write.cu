@@ -1,0 +1,286 @@
+// Decode-step write path: append one token per (sequence, KV head) into a head whose footprint
+// is fixed, and the H2O score bookkeeping that chooses which retained token a full head gives up.
+//
+// Sources: "Tangram" explainer, 三大机制 1 (Budget Reservation: a head's post-compression
+// footprint is fixed when the request starts; no page is reclaimed or added at run time) and
+// 落地形态 (compression rules such as H2O run on top unchanged); CAP survey §2.4.1 (3)
+// (LM-Infinite / StreamingLLM keep the first tokens and the last L tokens) and (4) (H2O keeps
+// the last L tokens plus the tokens with the largest attention accumulated at run time).
+//
+// Both kernels are small and memory-bound: the append moves 4·D bytes per head; the H2O update
+// reads 8 + 4·G bytes and writes 4 per retained token.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <cstdio>
+
+#include "tg.h"
+#include "tg_internal.h"
+
+namespace tg {
+
+namespace {
+
+constexpr int kAppendWarps = 8;     // heads per CTA of the append kernel
+constexpr int kUpdateThreads = 512;  // threads per head of the H2O update kernel
+
+// Append: one warp per (b, h). Lane 0 picks the slot; the warp copies the K and V rows with
+// 16-byte stores (D*2 bytes each); lane 0 updates the head's counters.
+//   POLICY 0: sink + recent (head_cursor in/out); POLICY 1: H2O (head_victim in).
+template <int POLICY>
+__global__ void __launch_bounds__(kAppendWarps * 32)
+    append_kernel(int32_t BH, int32_t Hkv, int32_t D, int64_t num_pages, int32_t sink,
+                  const uint4 *k_new, const uint4 *v_new, uint4 *k_pages, uint4 *v_pages,
+                  const int32_t *table, const int64_t *head_off, const int32_t *budget,
+                  int32_t *kv_len, int32_t *cursor, const int32_t *victim, int32_t *slot_pos,
+                  float *slot_score, const int32_t *new_pos, int32_t *slot_out) {
+    const int32_t bh = blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (bh >= BH) return;
+    int32_t slot = -1;
+    int64_t pid = -1;
+    if (lane == 0) {
+        const int32_t bud = budget[bh], n = kv_len[bh];
+        if (bud >= 1) {
+            if (n < bud) {
+                slot = n < 0 ? 0 : n;
+            } else if (POLICY == 0) {
+                const int32_t s = max(0, min(sink, bud - 1));
+                const int32_t R = bud - s;
+                int32_t c = cursor[bh] % R;
+                if (c < 0) c += R;
+                slot = s + c;
+            } else {
+                const int32_t v = victim[bh];
+                slot = (v >= 0 && v < bud) ? v : -1;
+            }
+        }
+        if (slot >= 0) {
+            pid = table[head_off[bh] + slot / 16];
+            if (pid < 0 || pid >= num_pages) slot = -1;
+        }
+    }
+    slot = __shfl_sync(0xffffffffu, slot, 0);
+    pid = __shfl_sync(0xffffffffu, pid, 0);
+    if (slot >= 0) {
+        const int nvec = D / 8;  // 16-byte vectors per row
+        const int64_t dst = (pid * 16 + slot % 16) * nvec;
+        const int64_t src = static_cast<int64_t>(bh) * nvec;
+        for (int i = lane; i < 2 * nvec; i += 32) {
+            if (i < nvec) k_pages[dst + i] = k_new[src + i];
+            else v_pages[dst + i - nvec] = v_new[src + i - nvec];
+        }
+    }
+    if (lane == 0) {
+        slot_out[bh] = slot;
+        if (slot >= 0) {
+            const int32_t bud = budget[bh], n = kv_len[bh];
+            if (n < bud) {
+                kv_len[bh] = slot + 1;
+            } else if (POLICY == 0) {
+                const int32_t s = max(0, min(sink, bud - 1));
+                const int32_t R = bud - s;
+                cursor[bh] = (slot - s + 1) % R;
+            }
+            if (POLICY == 1) {
+                const int64_t e = head_off[bh] * 16 + slot;
+                slot_pos[e] = new_pos[bh / Hkv];
+                slot_score[e] = 0.f;
+            }
+        }
+    }
+}
+
+// H2O update: one CTA per (b, h). Adds this step's attention to every retained token's score
+// and picks the slot the next token takes: with a free slot, kv_len; else the lowest score among
+// tokens older than the last `recent` positions (ties: lowest slot), else the oldest token.
+// Each thread takes kUnroll slots per round and issues all their loads before using any, so a
+// long head (up to thousands of slots) costs a few dependent rounds, not one per slot.
+constexpr int kUnroll = 4;
+
+struct MinPair {
+    float s;     // candidate: lowest score ...
+    int32_t i;   // ... at the lowest slot
+    int32_t p;   // oldest: lowest position ...
+    int32_t o;   // ... at the lowest slot
+};
+
+__device__ __forceinline__ void take(MinPair &m, float s, int32_t i, int32_t p, int32_t o) {
+    if (s < m.s || (s == m.s && i < m.i)) {
+        m.s = s;
+        m.i = i;
+    }
+    if (p < m.p || (p == m.p && o < m.o)) {
+        m.p = p;
+        m.o = o;
+    }
+}
+
+template <int G4>  // 1: G == 4, token scores read as one 16-byte vector
+__global__ void __launch_bounds__(kUpdateThreads)
+    h2o_update_kernel(int32_t Hq, int32_t Hkv, int32_t recent, const float *token_scores,
+                      const float *lse, const int64_t *head_off, const int32_t *budget,
+                      const int32_t *kv_len, const int32_t *slot_pos, float *slot_score,
+                      const int32_t *next_pos, int32_t *victim) {
+    const int32_t bh = blockIdx.x;
+    const int32_t b = bh / Hkv, h = bh - b * Hkv;
+    const int32_t G = Hq / Hkv;
+    const int32_t n = max(0, kv_len[bh]);
+    const int64_t base = head_off[bh] * 16;
+    const float *lrow = lse + static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * G;
+    const int64_t limit = static_cast<int64_t>(next_pos[b]) - recent;
+    float l4[4] = {0.f, 0.f, 0.f, 0.f};
+    if (G4 && token_scores) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) l4[g] = lrow[g];
+    }
+
+    MinPair m{INFINITY, 0x7fffffff, 0x7fffffff, 0x7fffffff};
+    for (int32_t t0 = threadIdx.x; t0 < n; t0 += kUpdateThreads * kUnroll) {
+        float sc[kUnroll];
+        int32_t ps[kUnroll];
+        float4 tv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int32_t t = t0 + u * kUpdateThreads;
+            sc[u] = 0.f;
+            ps[u] = 0x7fffffff;
+            tv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t < n) {
+                sc[u] = slot_score[base + t];
+                ps[u] = slot_pos[base + t];
+                if (G4 && token_scores) tv[u] = reinterpret_cast<const float4 *>(token_scores)[base + t];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int32_t t = t0 + u * kUpdateThreads;
+            if (t >= n) continue;
+            float s = sc[u];
+            if (token_scores) {
+                if (G4) {
+                    s += expf(tv[u].x - l4[0]);
+                    s += expf(tv[u].y - l4[1]);
+                    s += expf(tv[u].z - l4[2]);
+                    s += expf(tv[u].w - l4[3]);
+                } else {
+                    const float *ts = token_scores + (base + t) * G;
+                    for (int32_t g = 0; g < G; ++g) s += expf(ts[g] - lrow[g]);
+                }
+                slot_score[base + t] = s;
+            }
+            const bool cand = static_cast<int64_t>(ps[u]) < limit;
+            take(m, cand ? s : INFINITY, cand ? t : 0x7fffffff, ps[u], t);
+        }
+    }
+    // (score, slot) and (position, slot) minima: warp shuffles, then one value per warp.
+    for (int off = 16; off > 0; off >>= 1) {
+        const float os = __shfl_xor_sync(0xffffffffu, m.s, off);
+        const int32_t oi = __shfl_xor_sync(0xffffffffu, m.i, off);
+        const int32_t op = __shfl_xor_sync(0xffffffffu, m.p, off);
+        const int32_t oo = __shfl_xor_sync(0xffffffffu, m.o, off);
+        take(m, os, oi, op, oo);
+    }
+    __shared__ MinPair wm[kUpdateThreads / 32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) wm[warp] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kUpdateThreads / 32; ++w) take(m, wm[w].s, wm[w].i, wm[w].p, wm[w].o);
+        const int32_t bud = budget[bh];
+        int32_t v;
+        if (bud < 1) v = -1;
+        else if (n < bud) v = n;
+        else if (m.i != 0x7fffffff) v = m.i;
+        else v = (m.o != 0x7fffffff) ? m.o : -1;
+        victim[bh] = v;
+    }
+}
+
+bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(const tg_shape *s) {
+    if (!s || s->B < 0 || s->Hkv < 1 || s->Hq < s->Hkv || s->Hq % s->Hkv != 0 || s->page != 16 ||
+        s->D < 8 || s->D % 8 != 0 || s->num_pages < 0)
+        return TG_EINVAL;
+    return TG_OK;
+}
+
+int launch_status(const char *what) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        set_cuda_error(what, static_cast<int>(e));
+        return TG_ECUDA;
+    }
+    return TG_OK;
+}
+
+}  // namespace
+
+}  // namespace tg
+
+using namespace tg;
+
+extern "C" int tg_append_sink_recent(const tg_shape *shape, int32_t sink, const void *k_new,
+                                     const void *v_new, void *k_pages, void *v_pages,
+                                     const int32_t *page_table, const int64_t *head_page_off,
+                                     const int32_t *head_budget, int32_t *head_kv_len,
+                                     int32_t *head_cursor, int32_t *slot_out, tg_stream stream) {
+    if (check_shape(shape) != TG_OK || sink < 0) return TG_EINVAL;
+    const int32_t BH = shape->B * shape->Hkv;
+    if (BH == 0) return TG_OK;
+    if (!k_new || !v_new || !k_pages || !v_pages || !page_table || !head_page_off ||
+        !head_budget || !head_kv_len || !head_cursor || !slot_out || !al16(k_new) ||
+        !al16(v_new) || !al16(k_pages) || !al16(v_pages))
+        return TG_EINVAL;
+    const unsigned grid = static_cast<unsigned>((BH + kAppendWarps - 1) / kAppendWarps);
+    append_kernel<0><<<grid, kAppendWarps * 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        BH, shape->Hkv, shape->D, shape->num_pages, sink, static_cast<const uint4 *>(k_new),
+        static_cast<const uint4 *>(v_new), static_cast<uint4 *>(k_pages),
+        static_cast<uint4 *>(v_pages), page_table, head_page_off, head_budget, head_kv_len,
+        head_cursor, nullptr, nullptr, nullptr, nullptr, slot_out);
+    return launch_status("append_kernel<sink+recent>");
+}
+
+extern "C" int tg_append_h2o(const tg_shape *shape, const void *k_new, const void *v_new,
+                             void *k_pages, void *v_pages, const int32_t *page_table,
+                             const int64_t *head_page_off, const int32_t *head_budget,
+                             int32_t *head_kv_len, const int32_t *head_victim, int32_t *slot_pos,
+                             float *slot_score, const int32_t *new_pos, int32_t *slot_out,
+                             tg_stream stream) {
+    if (check_shape(shape) != TG_OK) return TG_EINVAL;
+    const int32_t BH = shape->B * shape->Hkv;
+    if (BH == 0) return TG_OK;
+    if (!k_new || !v_new || !k_pages || !v_pages || !page_table || !head_page_off ||
+        !head_budget || !head_kv_len || !head_victim || !slot_pos || !slot_score || !new_pos ||
+        !slot_out || !al16(k_new) || !al16(v_new) || !al16(k_pages) || !al16(v_pages))
+        return TG_EINVAL;
+    const unsigned grid = static_cast<unsigned>((BH + kAppendWarps - 1) / kAppendWarps);
+    append_kernel<1><<<grid, kAppendWarps * 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        BH, shape->Hkv, shape->D, shape->num_pages, 0, static_cast<const uint4 *>(k_new),
+        static_cast<const uint4 *>(v_new), static_cast<uint4 *>(k_pages),
+        static_cast<uint4 *>(v_pages), page_table, head_page_off, head_budget, head_kv_len,
+        nullptr, head_victim, slot_pos, slot_score, new_pos, slot_out);
+    return launch_status("append_kernel<h2o>");
+}
+
+extern "C" int tg_h2o_update(const tg_shape *shape, int32_t recent, const float *token_scores,
+                             const float *lse, const int64_t *head_page_off,
+                             const int32_t *head_budget, const int32_t *head_kv_len,
+                             const int32_t *slot_pos, float *slot_score, const int32_t *next_pos,
+                             int32_t *head_victim, tg_stream stream) {
+    if (check_shape(shape) != TG_OK || recent < 0) return TG_EINVAL;
+    const int32_t BH = shape->B * shape->Hkv;
+    if (BH == 0) return TG_OK;
+    if ((token_scores && !lse) || !head_page_off || !head_budget || !head_kv_len || !slot_pos ||
+        !slot_score || !next_pos || !head_victim)
+        return TG_EINVAL;
+    const bool g4 = shape->Hq / shape->Hkv == 4 &&
+                    (reinterpret_cast<uintptr_t>(token_scores) & 15u) == 0;
+    auto kern = g4 ? h2o_update_kernel<1> : h2o_update_kernel<0>;
+    kern<<<static_cast<unsigned>(BH), kUpdateThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        shape->Hq, shape->Hkv, recent, token_scores, lse, head_page_off, head_budget, head_kv_len,
+        slot_pos, slot_score, next_pos, head_victim);
+    return launch_status("h2o_update_kernel");
+}

@@ -70,7 +70,9 @@ def _plan_kw(cfg):
     elif cfg == 3:
         kw.update(static_permille=900, dyn_chunk_pages=32)
     elif cfg == 4:
-        kw.update(static_permille=1000)        # shared prefix pages: L2 locality wins
+        # shared prefix pages: the cascade reads each shared run once per step for all its
+        # readers; the private pages stay on the split-K items
+        kw.update(static_permille=1000, cascade=True)
     elif cfg == 5:
         kw.update(min_splits=64, max_chunk_pages=128, static_permille=900, dyn_chunk_pages=32)
     return kw
@@ -403,7 +405,9 @@ def run_ours(args):
             "kv_bytes_per_step": int(kv_total),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": _traffic(cfg) if world == 1 else None,
-                         "peak_kind": peak_kind, "kernel": "decode_kernel",
+                         "peak_kind": peak_kind,
+                         "kernel": "cascade_kernel + decode_kernel" if info["n_cascade"] > 0
+                         else "decode_kernel",
                          "algorithmic_bytes_per_launch": alg["total"],
                          "avg_launch_ms": dec_avg, "merge_avg_ms": mrg_ms / max(n_rec, 1),
                          "launches_timed": n_rec},
@@ -412,9 +416,10 @@ def run_ours(args):
                     "d2h_bytes_per_step": int(db.out.numel() * db.out.element_size() +
                                               db.lse.numel() * db.lse.element_size()),
                     "steps": k_e2e},
-            "gpu_launches": args.steps * (1 + (1 if info["n_merge"] > 0 else 0)),
+            "gpu_launches": args.steps * (1 + (1 if info["n_merge"] > 0 else 0) +
+                                          (1 if info["n_cascade"] > 0 else 0)),
             "plan": {k: info[k] for k in ("n_items", "n_partials", "n_merge", "n_workers",
-                                          "grid", "stages", "smem_bytes")},
+                                          "grid", "stages", "smem_bytes", "n_cascade")},
             "device_status": "ok" if not bad else "error word set",
             "clocks": clocks,
         }

@@ -207,11 +207,34 @@ typedef struct tg_plan_info {
     int32_t block;            /* threads per CTA */
     int32_t smem_bytes;       /* dynamic shared memory per CTA */
     int32_t stages;           /* pipeline stages per worker */
-    int32_t reserved;
+    int32_t n_cascade;        /* prefix-cascade units (tg_plan_create_cascade), else 0 */
     int64_t device_bytes;     /* bytes of the plan's device allocation */
     int64_t kv_bytes;         /* retained K/V bytes one step reads (scales included) */
 } tg_plan_info;
 int tg_plan_get_info(const tg_plan *p, tg_plan_info *info);
+
+/* Prefix-aware cascade plan for shared pages ("RadixAttention and KV reuse": a radix tree over
+ * token sequences, each node owning the KV blocks of its range, reused by every request whose
+ * prefix passes through it). As tg_plan_create (bf16, no tiers), and from the HOST copies of the
+ * page table and head offsets (page_table int32 [table_len], head_page_off int64 [B*Hkv]) it
+ * recovers, per KV head, the runs of full pages that >= min_readers (at least 2) heads' rows
+ * share at the same positions: rows are grouped by their page id at a position, a group runs
+ * as far as all its rows keep the same page ids, then splits again below. Every run is read
+ * once per step by cascade units of up to 64 query rows (64/G readers with their G query
+ * heads each: a dense tile for the tensor cores) instead of once per reader; each reader's
+ * private pages (after its deepest run) go through the ordinary split-K items; every head with
+ * a run is merged from its run partials (in run order) and its items'. Results equal those of
+ * tg_ragged_paged_decode up to rounding; the plan stays valid while the device table and
+ * lengths are the ones given here. TG_EINVAL on a row outside the table. */
+int tg_plan_create_cascade(const tg_shape *shape, const int32_t *kv_len,
+                           const int32_t *group_of_head, const int64_t *group_off,
+                           int32_t n_groups, const int32_t *page_table,
+                           const int64_t *head_page_off, int64_t table_len, int32_t min_readers,
+                           const tg_plan_opts *opts, tg_plan **out);
+/* Inspection: per cascade unit (tg_plan_info.n_cascade of them), 4 + 2*64 ints: KV head, first
+ * page position, end page position, readers, then 64 reader sequences and 64 partial slots
+ * (-1 past the readers). */
+int tg_plan_cascade_units(const tg_plan *p, int32_t *units);
 
 /* Work list export for inspection: items (host, n_items x 8 int32): per item
  * {b*Hkv + h, page_begin, page_end, tier_tokens, partial slot (-1 = final), INT8 tier (0/1),

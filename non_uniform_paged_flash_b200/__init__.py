@@ -55,7 +55,7 @@ class tg_plan_info(ctypes.Structure):
                 ("n_workers", ctypes.c_int32),
                 ("grid", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("smem_bytes", ctypes.c_int32), ("stages", ctypes.c_int32),
-                ("reserved", ctypes.c_int32), ("device_bytes", ctypes.c_int64),
+                ("n_cascade", ctypes.c_int32), ("device_bytes", ctypes.c_int64),
                 ("kv_bytes", ctypes.c_int64)]
 
 
@@ -103,6 +103,10 @@ _SIGS = [
                                      _P, _P, _P, _P, _P, _P]),
     ("tg_h2o_update", ctypes.c_int, [ctypes.POINTER(tg_shape), _I32, _P, _P, _P, _P, _P, _P, _P,
                                      _P, _P, _P]),
+    ("tg_plan_create_cascade", ctypes.c_int, [ctypes.POINTER(tg_shape), _P, _P, _P, _I32, _P, _P,
+                                              _I64, _I32, ctypes.POINTER(tg_plan_opts),
+                                              ctypes.POINTER(_P)]),
+    ("tg_plan_cascade_units", ctypes.c_int, [_P, _P]),
 ]
 
 #: Symbols the C ABI exports (include/tg.h).
@@ -300,6 +304,38 @@ def tg_plan_create(shape: tg_shape, kv_len, group_of_head, group_off, fast_len=N
     return Plan(h, shape, fl is not None)
 
 
+def tg_plan_create_cascade(shape: tg_shape, kv_len, group_of_head, group_off, page_table,
+                           head_page_off, min_readers: int = 2, num_workers: int = 0,
+                           min_splits: int = 1, max_chunk_pages: int = 0, host_only: bool = False,
+                           device: int = -1, static_permille: int = 0, dyn_chunk_pages: int = 0,
+                           early_prologue: bool = False, wait_limit_us: int = 0) -> Plan:
+    """Prefix-aware cascade plan from the host page table (see include/tg.h)."""
+    kv = _h(kv_len, np.int32).reshape(-1)
+    goh = _h(group_of_head, np.int32).reshape(-1)
+    goff = _h(group_off, np.int64).reshape(-1)
+    tbl = _h(page_table, np.int32).reshape(-1)
+    hoff = _h(head_page_off, np.int64).reshape(-1)
+    opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
+                        static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us, 0)
+    h = ctypes.c_void_p()
+    _check(_lib().tg_plan_create_cascade(ctypes.byref(shape), _hp(kv), _hp(goh), _hp(goff),
+                                         goff.size - 1, _hp(tbl), _hp(hoff), tbl.size,
+                                         int(min_readers), ctypes.byref(opts), ctypes.byref(h)),
+           "tg_plan_create_cascade")
+    return Plan(h, shape, False)
+
+
+def tg_plan_cascade_units(plan: Plan):
+    """Cascade units: (meta int32[n, 4] = KV head, first page position, end position, readers;
+    readers int32[n, 64]; slots int32[n, 64]), -1 past each unit's readers."""
+    n = tg_plan_get_info(plan)["n_cascade"]
+    w = 4 + 2 * 64
+    out = np.empty((max(n, 1), w), dtype=np.int32)
+    _check(_lib().tg_plan_cascade_units(plan.handle, _hp(out)), "tg_plan_cascade_units")
+    out = out[:n]
+    return out[:, :4], out[:, 4:68], out[:, 68:]
+
+
 def tg_plan_destroy(plan: Plan):
     plan.destroy()
 
@@ -307,7 +343,7 @@ def tg_plan_destroy(plan: Plan):
 def tg_plan_get_info(plan: Plan) -> dict:
     info = tg_plan_info()
     _check(_lib().tg_plan_get_info(plan.handle, ctypes.byref(info)), "tg_plan_get_info")
-    return {f: getattr(info, f) for f, _ in tg_plan_info._fields_ if f != "reserved"}
+    return {f: getattr(info, f) for f, _ in tg_plan_info._fields_}
 
 
 def tg_plan_items(plan: Plan) -> np.ndarray:

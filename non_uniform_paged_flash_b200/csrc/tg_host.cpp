@@ -299,7 +299,8 @@ namespace tg {
 
 int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
                     int32_t num_workers, int32_t min_splits, int32_t max_chunk_pages,
-                    int32_t static_permille, int32_t dyn_chunk_pages) {
+                    int32_t static_permille, int32_t dyn_chunk_pages, const int32_t *pstart,
+                    const int32_t *casc_cnt) {
     const tg_shape &s = p->shape;
     const int64_t BH = static_cast<int64_t>(s.B) * s.Hkv;
     const int32_t page = s.page;
@@ -331,16 +332,19 @@ int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
             runs[nr++] = {n, 0, bf16_page_cost};
             kv_bytes += static_cast<int64_t>(n) * 2 * s.D * 2;
         }
+        // pages [0, p0) of a cascade plan's head are read by its cascade units
+        const int32_t p0 = pstart ? pstart[bh] : 0;
         int64_t head_pages = 0;
         for (int r = 0; r < nr; ++r) head_pages += (runs[r].tokens + page - 1) / page;
+        head_pages -= p0;
         int64_t cap = max_chunk_pages > 0 ? max_chunk_pages : INT32_MAX;
         if (min_splits > 1 && head_pages > 0)
             cap = std::min<int64_t>(cap, std::max<int64_t>(1, head_pages / min_splits));
         for (int r = 0; r < nr; ++r) {
-            const int32_t pages = (runs[r].tokens + page - 1) / page;
-            if (pages == 0) continue;
+            const int32_t pages = (runs[r].tokens + page - 1) / page - p0;
+            if (pages <= 0) continue;
             const int64_t k = (pages + cap - 1) / cap;
-            int32_t at = 0;
+            int32_t at = p0;
             for (int64_t c = 0; c < k; ++c) {
                 const int32_t sz = static_cast<int32_t>(pages / k + (c < pages % k ? 1 : 0));
                 chunks.push_back({static_cast<int32_t>(bh), at, at + sz, runs[r].tokens,
@@ -462,6 +466,8 @@ int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
     }
 
     // Partial slots and the merge list: a head's items are consecutive in the list.
+    // A cascade head's partials come first (slots first_slot .. first_slot + casc_cnt - 1, in
+    // the order of its cascade runs), then its items'.
     std::vector<int32_t> cnt(static_cast<size_t>(BH), 0), first(static_cast<size_t>(BH), -1);
     for (size_t i = 0; i < p->items.size(); ++i) {
         const int32_t bh = p->items[i].bh;
@@ -473,18 +479,21 @@ int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
     p->merge_warps = 1;
     int64_t slot = 0;
     for (int64_t bh = 0; bh < BH; ++bh) {
-        if (cnt[bh] == 0) {
+        const int32_t cc = casc_cnt ? casc_cnt[bh] : 0;
+        const int32_t total = cnt[bh] + cc;
+        if (total == 0) {
             p->empties.push_back(static_cast<int32_t>(bh));
-        } else if (cnt[bh] > 1) {
+        } else if (total > 1 || cc > 0) {
             const int32_t mi = static_cast<int32_t>(p->merge.size());
-            p->merge.push_back({static_cast<int32_t>(bh), static_cast<int32_t>(slot), cnt[bh], 0});
+            p->merge.push_back({static_cast<int32_t>(bh), static_cast<int32_t>(slot), total, 0});
+            slot += cc;
             for (int32_t j = 0; j < cnt[bh]; ++j) {
                 Item &it = p->items[first[bh] + j];
                 it.slot = static_cast<int32_t>(slot++);
                 it.flags |= mi << 1;
             }
             // warps per merge CTA: up to 8 splits per warp, at most 32 warps
-            p->merge_warps = std::max(p->merge_warps, std::min(32, (cnt[bh] + 7) / 8));
+            p->merge_warps = std::max(p->merge_warps, std::min(32, (total + 7) / 8));
         }
     }
     p->n_partials = slot;
@@ -496,11 +505,71 @@ int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
 // ------------------------------------------------------------------------------------------
 // Plan creation (host part) and inspection.
 // ------------------------------------------------------------------------------------------
-extern "C" int tg_plan_create(const tg_shape *shape, const int32_t *kv_len,
-                              const int32_t *fast_len, const int32_t *group_of_head,
-                              const int64_t *group_off, int32_t n_groups,
-                              int64_t slow_table_len, const tg_plan_opts *opts,
-                              tg_plan **out) {
+namespace {
+
+// Shared-prefix runs of one KV head ("RadixAttention and KV reuse": a radix tree over token
+// sequences whose nodes own the KV blocks of their range, reused by every request whose prefix
+// passes through the node). Here the tree is recovered from the page tables themselves: the
+// rows of head h are grouped by their page id at a position; a group of >= min_readers rows
+// that agree on the page forms a node, which runs as far as all of them keep agreeing (full
+// pages only); the group is then split again below the node. Each row's private part starts
+// where its deepest node ends. Nodes are emitted parent first, groups in order of their first
+// row, so the result is deterministic.
+struct Node {
+    int32_t h, pos_begin, pos_end;
+    std::vector<int32_t> readers;
+};
+
+void shared_runs(int32_t h, const std::vector<int32_t> &rows, int32_t Hkv, const int32_t *kv_len,
+                 const int32_t *table, const int64_t *head_off, int32_t min_readers,
+                 std::vector<Node> &nodes, std::vector<int32_t> &pstart) {
+    struct Task { std::vector<int32_t> readers; int32_t depth; };
+    std::vector<Task> stack;
+    stack.push_back({rows, 0});
+    auto full = [&](int32_t b) { return kv_len[static_cast<int64_t>(b) * Hkv + h] / 16; };
+    auto pid = [&](int32_t b, int32_t pos) {
+        return table[head_off[static_cast<int64_t>(b) * Hkv + h] + pos];
+    };
+    while (!stack.empty()) {
+        Task t = std::move(stack.back());
+        stack.pop_back();
+        std::vector<int32_t> keys;                  // page ids in order of first appearance
+        std::vector<std::vector<int32_t>> groups;
+        for (int32_t b : t.readers) {
+            if (t.depth >= full(b)) continue;
+            const int32_t k = pid(b, t.depth);
+            size_t gi = 0;
+            while (gi < keys.size() && keys[gi] != k) ++gi;
+            if (gi == keys.size()) {
+                keys.push_back(k);
+                groups.emplace_back();
+            }
+            groups[gi].push_back(b);
+        }
+        std::vector<Task> children;
+        for (size_t gi = 0; gi < groups.size(); ++gi) {
+            const std::vector<int32_t> &g = groups[gi];
+            if (static_cast<int32_t>(g.size()) < std::max(2, min_readers)) continue;
+            int32_t end = t.depth + 1;
+            for (;;) {
+                bool ok = true;
+                for (int32_t b : g)
+                    if (end >= full(b) || pid(b, end) != pid(g[0], end)) { ok = false; break; }
+                if (!ok) break;
+                ++end;
+            }
+            nodes.push_back({h, t.depth, end, g});
+            for (int32_t b : g) pstart[static_cast<int64_t>(b) * Hkv + h] = end;
+            children.push_back({g, end});
+        }
+        for (size_t c = children.size(); c-- > 0;) stack.push_back(std::move(children[c]));
+    }
+}
+
+int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,
+                const int32_t *group_of_head, const int64_t *group_off, int32_t n_groups,
+                int64_t slow_table_len, const tg_plan_opts *opts, const int32_t *table,
+                const int64_t *head_off, int64_t table_len, int32_t min_readers, tg_plan **out) {
     if (!shape || !kv_len || !out || !group_of_head || !group_off || n_groups < 1) return TG_EINVAL;
     const tg_shape &s = *shape;
     if (s.B < 0 || s.Hkv < 1 || s.Hq < 1 || s.Hq % s.Hkv != 0 || s.D < 1 || s.page < 1 ||
@@ -534,6 +603,43 @@ extern "C" int tg_plan_create(const tg_shape *shape, const int32_t *kv_len,
     if (o.wait_limit_us > 0) p->wait_ns = static_cast<uint64_t>(o.wait_limit_us) * 1000ull;
     p->withhold = o.test_withhold_page > 0 ? o.test_withhold_page : 0;
 
+    // Prefix cascade: shared runs per KV head, cut into units of kCascadeRows query rows.
+    std::vector<int32_t> casc_cnt;
+    if (table) {
+        const int64_t BH = static_cast<int64_t>(s.B) * s.Hkv;
+        for (int64_t bh = 0; bh < BH; ++bh) {
+            const int64_t npages = (kv_len[bh] + 15) / 16;
+            if (kv_len[bh] < 0 || head_off[bh] < 0 || head_off[bh] + npages > table_len) {
+                delete p;
+                return TG_EINVAL;
+            }
+        }
+        p->pstart.assign(static_cast<size_t>(BH), 0);
+        std::vector<Node> nodes;
+        std::vector<int32_t> rows(static_cast<size_t>(s.B));
+        for (int32_t b = 0; b < s.B; ++b) rows[b] = b;
+        for (int32_t h = 0; h < s.Hkv; ++h)
+            shared_runs(h, rows, s.Hkv, kv_len, table, head_off, min_readers, nodes, p->pstart);
+        casc_cnt.assign(static_cast<size_t>(BH), 0);
+        for (const Node &n : nodes)
+            for (int32_t b : n.readers) ++casc_cnt[static_cast<int64_t>(b) * s.Hkv + n.h];
+        const int32_t per = tg::kCascadeRows / G;
+        for (const Node &n : nodes) {
+            for (size_t r0 = 0; r0 < n.readers.size(); r0 += per) {
+                tg::CascadeUnit u{};
+                u.h = n.h;
+                u.pos_begin = n.pos_begin;
+                u.pos_end = n.pos_end;
+                u.n_readers = static_cast<int32_t>(std::min<size_t>(per, n.readers.size() - r0));
+                for (int32_t r = 0; r < u.n_readers; ++r) {
+                    u.reader[r] = n.readers[r0 + r];
+                    u.slot[r] = -1;
+                }
+                p->cunits.push_back(u);
+            }
+        }
+    }
+
     int32_t workers = o.num_workers;
     if (!p->host_only) {
         int rc = tg::device_num_sms(o.device, &p->num_sms);
@@ -544,8 +650,18 @@ extern "C" int tg_plan_create(const tg_shape *shape, const int32_t *kv_len,
     }
     const int32_t sp = o.static_permille <= 0 ? 800 : std::min(1000, o.static_permille);
     const int32_t dc = o.dyn_chunk_pages <= 0 ? 16 : o.dyn_chunk_pages;
-    int rc = tg::build_work_list(p, kv_len, fast_len, workers, o.min_splits, o.max_chunk_pages, sp, dc);
+    int rc = tg::build_work_list(p, kv_len, fast_len, workers, o.min_splits, o.max_chunk_pages, sp,
+                                 dc, table ? p->pstart.data() : nullptr,
+                                 table ? casc_cnt.data() : nullptr);
     if (rc != TG_OK) { delete p; return rc; }
+    if (table) {
+        // Cascade partial slots: a head's merge list starts with its runs, in unit order.
+        std::vector<int32_t> next(static_cast<size_t>(s.B) * s.Hkv, -1);
+        for (const tg::MergeHead &m : p->merge) next[m.bh] = m.first_slot;
+        for (tg::CascadeUnit &u : p->cunits)
+            for (int32_t r = 0; r < u.n_readers; ++r)
+                u.slot[r] = next[static_cast<int64_t>(u.reader[r]) * s.Hkv + u.h]++;
+    }
     p->grid = (p->n_workers + p->pairs - 1) / p->pairs;
     if (p->n_dyn > 0 && p->grid == 0) p->grid = 1;
     if (p->grid == 0 && !p->empties.empty()) p->grid = 1;  // the kernel also writes empty heads
@@ -555,6 +671,28 @@ extern "C" int tg_plan_create(const tg_shape *shape, const int32_t *kv_len,
     }
     *out = p;
     return TG_OK;
+}
+
+}  // namespace
+
+extern "C" int tg_plan_create(const tg_shape *shape, const int32_t *kv_len,
+                              const int32_t *fast_len, const int32_t *group_of_head,
+                              const int64_t *group_off, int32_t n_groups,
+                              int64_t slow_table_len, const tg_plan_opts *opts,
+                              tg_plan **out) {
+    return plan_create(shape, kv_len, fast_len, group_of_head, group_off, n_groups,
+                       slow_table_len, opts, nullptr, nullptr, 0, 0, out);
+}
+
+extern "C" int tg_plan_create_cascade(const tg_shape *shape, const int32_t *kv_len,
+                                      const int32_t *group_of_head, const int64_t *group_off,
+                                      int32_t n_groups, const int32_t *page_table,
+                                      const int64_t *head_page_off, int64_t table_len,
+                                      int32_t min_readers, const tg_plan_opts *opts,
+                                      tg_plan **out) {
+    if (!page_table || !head_page_off || table_len < 0) return TG_EINVAL;
+    return plan_create(shape, kv_len, nullptr, group_of_head, group_off, n_groups, 0, opts,
+                       page_table, head_page_off, table_len, min_readers, out);
 }
 
 extern "C" void tg_plan_destroy(tg_plan *p) {
@@ -578,6 +716,22 @@ extern "C" int tg_plan_get_info(const tg_plan *p, tg_plan_info *info) {
     info->stages = p->stages;
     info->device_bytes = p->dev_bytes;
     info->kv_bytes = p->kv_bytes;
+    info->n_cascade = static_cast<int32_t>(p->cunits.size());
+    return TG_OK;
+}
+
+extern "C" int tg_plan_cascade_units(const tg_plan *p, int32_t *units) {
+    if (!p || !units) return TG_EINVAL;
+    const int32_t w = 4 + 2 * tg::kCascadeRows;
+    for (size_t i = 0; i < p->cunits.size(); ++i) {
+        const tg::CascadeUnit &u = p->cunits[i];
+        int32_t *o = units + static_cast<int64_t>(w) * static_cast<int64_t>(i);
+        o[0] = u.h; o[1] = u.pos_begin; o[2] = u.pos_end; o[3] = u.n_readers;
+        for (int32_t r = 0; r < tg::kCascadeRows; ++r) {
+            o[4 + r] = r < u.n_readers ? u.reader[r] : -1;
+            o[4 + tg::kCascadeRows + r] = r < u.n_readers ? u.slot[r] : -1;
+        }
+    }
     return TG_OK;
 }
 

@@ -32,6 +32,20 @@ struct MergeHead {
     int32_t pad;
 };
 
+// Prefix cascade: one unit = up to 64 query rows (kCascadeRows / G readers, each with its G
+// query heads) that read the same run of shared pages [pos_begin, pos_end) of KV head h: the
+// pages are identical in every reader's table row. Each reader gets one partial result.
+constexpr int kCascadeRows = 64;
+struct CascadeUnit {
+    int32_t h;
+    int32_t pos_begin;  // first page position (index within every reader's row)
+    int32_t pos_end;    // one past the last
+    int32_t n_readers;
+    int32_t reader[kCascadeRows];  // sequence b of each reader
+    int32_t slot[kCascadeRows];    // partial-result slot of (b, h) for this run
+};
+static_assert(sizeof(CascadeUnit) == 16 + 8 * kCascadeRows, "CascadeUnit layout");
+
 // Device error-word bits.
 constexpr uint32_t kErrBadPage = 1u;   // page id outside the pool
 constexpr uint32_t kErrBadRow = 2u;    // row outside its group table / table
@@ -39,8 +53,8 @@ constexpr uint32_t kErrPlan = 4u;      // device lengths differ from the plan
 constexpr uint32_t kErrTimeout = 8u;   // a bounded wait gave up
 
 // Launch geometry of the decode kernels (see tg_kernels.cu): (producer warp, consumer warp)
-// pairs per CTA. (8 pairs for the tiered kernel were tried: at 128 registers per thread its
-// consumer spills, and ptxas does not raise the consumer's budget past a register split.)
+// pairs per CTA. The tiered kernel's INT8 consumer is latency-bound, so it trades ring depth
+// for consumers (measured: 6 pairs with 4 stages beat 4 x 6, 7 x 3 and 8 x 3).
 constexpr int kPairs = 4;              // bf16 decode kernel
 constexpr int kPairsTiered = 6;        // tiered decode kernel (12 warps; 4 ring stages at D = 128)
 constexpr int kThreads = kPairs * 64;  // threads per CTA of the bf16 decode kernel
@@ -68,6 +82,8 @@ struct tg_plan {
     std::vector<int32_t> empties;     // heads with no retained token
     std::vector<int64_t> group_off;   // [n_groups + 1]
     std::vector<int32_t> planned_kv;  // [B*Hkv]
+    std::vector<tg::CascadeUnit> cunits;  // prefix cascade units (cascade plans only)
+    std::vector<int32_t> pstart;          // [B*Hkv] first page of the head's private part
     int64_t n_partials = 0;
     int32_t merge_warps = 1;          // warps per (split head, row) CTA of the merge kernel
     int32_t pairs = tg::kPairs;       // worker pairs per CTA of this plan's decode kernel
@@ -94,6 +110,7 @@ struct tg_plan {
     float *d_part_lse = nullptr;  // [n_partials][G]
     int32_t *d_empties = nullptr;   // [n_empty]
     uint32_t *d_dyn = nullptr;      // [2] dynamic ticket, producers done
+    tg::CascadeUnit *d_cunits = nullptr;
     uint32_t *d_err = nullptr;
 
     // kernel timing: 2 events per recorded call (cudaEvent_t stored as void*)
@@ -109,9 +126,12 @@ struct tg_plan {
 
 namespace tg {
 // Host planner (tg_host.cpp): fills items / worker_off / merge / n_partials / kv_bytes.
+// pstart (nullable): first page of each head's private part (earlier pages are covered by
+// cascade units); casc_cnt (nullable): the head's cascade partials, merged before its items.
 int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
                     int32_t num_workers, int32_t min_splits, int32_t max_chunk_pages,
-                    int32_t static_permille, int32_t dyn_chunk_pages);
+                    int32_t static_permille, int32_t dyn_chunk_pages,
+                    const int32_t *pstart = nullptr, const int32_t *casc_cnt = nullptr);
 // Device side (tg_kernels.cu).
 int device_init_plan(tg_plan *p);
 void device_free_plan(tg_plan *p);

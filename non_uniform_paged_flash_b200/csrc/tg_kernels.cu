@@ -1046,6 +1046,281 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
 }
 
 // ------------------------------------------------------------------------------------------
+// Prefix cascade kernel: one CTA per cascade unit (a run of pages shared by up to 64 query
+// rows). Warp kCasConsumers is the producer: it reads the run's page ids from the first
+// reader's row 32 at a time, and one lane issues 2-D TMA loads of K and V into a ring of
+// kCasStages stages. Warps 0..3 each own 16 query rows and compute, per 16-token page,
+// S = Q K^T (rows on M, tokens on N, mma.m16n8k16; K fragments by ldmatrix from the swizzled
+// page; even and odd k-steps in separate accumulators to halve the dependent chain), the online
+// softmax of their rows, and O += P V with P taken from the S accumulators as the A operand
+// (tokens on K) and V fragments by ldmatrix.trans. Every run is whole pages (the planner takes
+// full pages only), so no token mask. Each reader's rows end as a normalised partial (o, lse)
+// in its slot, merged with the head's other partials by the merge kernel.
+// ------------------------------------------------------------------------------------------
+constexpr int kCasConsumers = 4;
+constexpr int kCasThreads = (kCasConsumers + 1) * 32;
+constexpr int kCasStages = 6;
+
+struct CascadeArgs {
+    const CascadeUnit *units;
+    int32_t G, Hq, Hkv;
+    float scale_log2;
+    const __nv_bfloat16 *q;
+    const int32_t *table;
+    const int64_t *head_off;
+    const int32_t *kv_len_dev;
+    int64_t num_pages;
+    float *part_o;
+    float *part_lse;
+    uint32_t *err;
+    uint64_t wait_ns;
+};
+
+template <int D>
+constexpr int cascade_smem_bytes() {
+    return 1024 + kCasStages * 2 * Layout<D>::KB + kCasStages * 16 + kCasStages * 4 + 16;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kCasThreads)
+    cascade_kernel(const __grid_constant__ CascadeArgs a, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v) {
+    using L = Layout<D>;
+    constexpr int KS = D / 16;  // k-steps of S = Q K^T
+    constexpr int NT = D / 8;   // n-tiles of O
+    constexpr unsigned FULL = 0xffffffffu;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kCasStages * 2 * L::KB);
+    volatile int32_t *skip = reinterpret_cast<volatile int32_t *>(bars + 2 * kCasStages);
+    volatile int32_t *abort_flag = skip + kCasStages;
+    const uint32_t full0 = dev::smem_addr(bars), empty0 = dev::smem_addr(bars + kCasStages);
+
+    const CascadeUnit *u = a.units + blockIdx.x;
+    const int32_t h = u->h, pb = u->pos_begin, pe = u->pos_end, nr = u->n_readers;
+    const int32_t npages = pe - pb;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kCasStages; ++st) {
+            dev::mbar_init(full0 + 8 * st, 1);
+            dev::mbar_init(empty0 + 8 * st, kCasConsumers);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    // The previous kernel in the stream (a merge reading the partial slots, a writer of q or of
+    // the pages) completes first; then the decode kernel that follows may launch.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    if (warp == kCasConsumers) {
+        // ================================ producer warp ================================
+        // Page ids are read 32 at a time (lane k: page k of the block), one block ahead, so
+        // the copies are never held up by an id load; lane 0 waits for the stages and issues.
+        if (lane == 0)
+            for (int32_t r = 0; r < nr; ++r)
+                if (a.kv_len_dev[static_cast<int64_t>(u->reader[r]) * a.Hkv + h] < pe * 16)
+                    atomicOr(a.err, kErrPlan);
+        const int32_t *row = a.table + a.head_off[static_cast<int64_t>(u->reader[0]) * a.Hkv + h] + pb;
+        int32_t ids = lane < npages ? __ldg(row + lane) : -1;
+        int32_t ids_next = 32 + lane < npages ? __ldg(row + 32 + lane) : -1;
+        int32_t issued = 0;
+        for (int32_t i = 0; i < npages; ++i) {
+            if (i > 0 && (i & 31) == 0) {
+                ids = ids_next;
+                ids_next = i + 32 + lane < npages ? __ldg(row + i + 32 + lane) : -1;
+            }
+            const int64_t pid = __shfl_sync(FULL, ids, i & 31);
+            int32_t stop = 0;
+            if (lane == 0) {
+                const int st = i % kCasStages;
+                const uint32_t ph = static_cast<uint32_t>(i / kCasStages) & 1u;
+                if (!dev::mbar_wait(empty0 + 8 * st, ph ^ 1u, a.wait_ns) || *abort_flag) {
+                    atomicOr(a.err, kErrTimeout);
+                    *abort_flag = 1;
+                    stop = 1;
+                } else {
+                    const uint32_t fb = full0 + 8 * st;
+                    if (pid < 0 || pid >= a.num_pages) {
+                        atomicOr(a.err, kErrBadPage);
+                        skip[st] = 1;
+                        dev::mbar_arrive(fb);
+                    } else {
+                        skip[st] = 0;
+                        const uint32_t sa = dev::smem_addr(smem + st * 2 * L::KB);
+                        const int32_t y = static_cast<int32_t>(pid * 16);
+                        dev::mbar_arrive_expect_tx(fb, 2u * L::KB);
+#pragma unroll
+                        for (int bx = 0; bx < D / 64; ++bx) {
+                            dev::tma_load_2d(sa + bx * 2048, &tm_k, bx * 64, y, fb);
+                            dev::tma_load_2d(sa + L::KB + bx * 2048, &tm_v, bx * 64, y, fb);
+                        }
+                    }
+                }
+            }
+            if (__shfl_sync(FULL, stop, 0)) break;
+            issued = i + 1;
+        }
+        // No copy may be in flight when the CTA exits: wait for the last page of every stage.
+        if (lane == 0)
+            for (int32_t i = issued - kCasStages < 0 ? 0 : issued - kCasStages; i < issued; ++i)
+                dev::mbar_wait(full0 + 8 * (i % kCasStages), static_cast<uint32_t>(i / kCasStages) & 1u,
+                               a.wait_ns < dev::kDrainNs ? a.wait_ns : dev::kDrainNs);
+        return;
+    }
+
+    // ================================ consumer warps ================================
+    const int g = lane >> 2, t = lane & 3;
+    const int G = a.G;
+    const int r0 = warp * 16 + g, r1 = r0 + 8;          // this lane's two query rows
+    const bool ok0 = r0 / G < nr, ok1 = r1 / G < nr;
+    // query fragments (A operand: rows on M, d on K), straight from global memory
+    uint32_t qa[KS][4];
+    {
+        const __nv_bfloat16 *q0 = ok0 ? a.q + ((static_cast<int64_t>(u->reader[r0 / G]) * a.Hq + h * G + r0 % G) * D) : nullptr;
+        const __nv_bfloat16 *q1 = ok1 ? a.q + ((static_cast<int64_t>(u->reader[r1 / G]) * a.Hq + h * G + r1 % G) * D) : nullptr;
+#pragma unroll
+        for (int j = 0; j < KS; ++j) {
+            qa[j][0] = q0 ? *reinterpret_cast<const uint32_t *>(q0 + 16 * j + 2 * t) : 0u;
+            qa[j][1] = q1 ? *reinterpret_cast<const uint32_t *>(q1 + 16 * j + 2 * t) : 0u;
+            qa[j][2] = q0 ? *reinterpret_cast<const uint32_t *>(q0 + 16 * j + 2 * t + 8) : 0u;
+            qa[j][3] = q1 ? *reinterpret_cast<const uint32_t *>(q1 + 16 * j + 2 * t + 8) : 0u;
+        }
+    }
+    // ldmatrix row offsets: K (B operand of S; matrices (tokens 0-7 | 8-15) x (chunk 2j | 2j+1))
+    // and V (B operand of O, transposed; matrices (tokens 0-7 | 8-15) x (chunk 2i | 2i+1)).
+    uint32_t offK[KS], offV[NT / 2];
+#pragma unroll
+    for (int j = 0; j < KS; ++j) {
+        const uint32_t tok = (lane & 7) + 8 * (lane >> 4), ch = 2 * j + ((lane >> 3) & 1);
+        offK[j] = (ch >> 3) * 2048 + dev::swz(tok, ch & 7);
+    }
+#pragma unroll
+    for (int i = 0; i < NT / 2; ++i) {
+        const uint32_t tok = (lane & 7) + 8 * ((lane >> 3) & 1), ch = 2 * i + (lane >> 4);
+        offV[i] = L::KB + (ch >> 3) * 2048 + dev::swz(tok, ch & 7);
+    }
+    float o[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, le0 = 0.f, le1 = 0.f, lr0 = 0.f, lr1 = 0.f;
+
+    for (int32_t i = 0; i < npages; ++i) {
+        const int st = i % kCasStages;
+        const uint32_t ph = static_cast<uint32_t>(i / kCasStages) & 1u;
+        if (!dev::mbar_wait(full0 + 8 * st, ph, a.wait_ns) || *abort_flag) {
+            if (lane == 0) {
+                atomicOr(a.err, kErrTimeout);
+                *abort_flag = 1;
+            }
+            return;
+        }
+        if (!skip[st]) {
+            const uint32_t sa = dev::smem_addr(smem + st * 2 * L::KB);
+            float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int j = 0; j < KS; ++j) {
+                uint32_t b0, b1, b2, b3;
+                dev::ldsm_x4(sa + offK[j], b0, b1, b2, b3);
+                float (&acc)[2][4] = (j & 1) ? s2 : s;
+                dev::mma_bf16(acc[0], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b0, b1);
+                dev::mma_bf16(acc[1], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b2, b3);
+            }
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) s[n][c] += s2[n][c];
+            // s[n][0..1]: row g, tokens 8n + 2t, +1; s[n][2..3]: row g + 8
+            float x[2][4];
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) x[n][c] = s[n][c] * a.scale_log2;
+            float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+            float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 1));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 1));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 2));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 2));
+            // lazy rescale: the running max moves only when a page exceeds it by more than 2^8
+            const bool up0 = mx0 > m0 + 8.f, up1 = mx1 > m1 + 8.f;
+            if (__any_sync(FULL, up0 || up1)) {
+                const float n0 = up0 ? mx0 : m0, n1 = up1 ? mx1 : m1;
+                const float c0 = m0 == -INFINITY ? 0.f : dev::ex2(m0 - n0);
+                const float c1 = m1 == -INFINITY ? 0.f : dev::ex2(m1 - n1);
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    o[n][0] *= c0;
+                    o[n][1] *= c0;
+                    o[n][2] *= c1;
+                    o[n][3] *= c1;
+                }
+                le0 *= c0;
+                lr0 *= c0;
+                le1 *= c1;
+                lr1 *= c1;
+                m0 = n0;
+                m1 = n1;
+            }
+            float p[2][4];
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                p[n][0] = dev::ex2(x[n][0] - m0);
+                p[n][1] = dev::ex2(x[n][1] - m0);
+                p[n][2] = dev::ex2(x[n][2] - m1);
+                p[n][3] = dev::ex2(x[n][3] - m1);
+            }
+            le0 += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+            le1 += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
+            // P as the A operand of O += P V (rows on M, tokens on K)
+            const uint32_t pa0 = dev::pack_bf16(p[0][0], p[0][1]), pa1 = dev::pack_bf16(p[0][2], p[0][3]);
+            const uint32_t pa2 = dev::pack_bf16(p[1][0], p[1][1]), pa3 = dev::pack_bf16(p[1][2], p[1][3]);
+            lr0 += (dev::bf16_lo(pa0) + dev::bf16_hi(pa0)) + (dev::bf16_lo(pa2) + dev::bf16_hi(pa2));
+            lr1 += (dev::bf16_lo(pa1) + dev::bf16_hi(pa1)) + (dev::bf16_lo(pa3) + dev::bf16_hi(pa3));
+#pragma unroll
+            for (int i2 = 0; i2 < NT / 2; ++i2) {
+                uint32_t v0, v1, v2, v3;
+                dev::ldsm_x4_t(sa + offV[i2], v0, v1, v2, v3);
+                dev::mma_bf16(o[2 * i2], pa0, pa1, pa2, pa3, v0, v1);
+                dev::mma_bf16(o[2 * i2 + 1], pa0, pa1, pa2, pa3, v2, v3);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(empty0 + 8 * st);
+    }
+
+    // Row sums over the 4 lanes of a row, then the partials of valid rows.
+    le0 += __shfl_xor_sync(FULL, le0, 1);
+    le0 += __shfl_xor_sync(FULL, le0, 2);
+    le1 += __shfl_xor_sync(FULL, le1, 1);
+    le1 += __shfl_xor_sync(FULL, le1, 2);
+    lr0 += __shfl_xor_sync(FULL, lr0, 1);
+    lr0 += __shfl_xor_sync(FULL, lr0, 2);
+    lr1 += __shfl_xor_sync(FULL, lr1, 1);
+    lr1 += __shfl_xor_sync(FULL, lr1, 2);
+    constexpr float kLn2 = 0.69314718055994530942f;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int r = half ? r1 : r0;
+        if (!(half ? ok1 : ok0)) continue;
+        const float le = half ? le1 : le0, lr = half ? lr1 : lr0, m = half ? m1 : m0;
+        const float inv = lr > 0.f ? 1.f / lr : 0.f;
+        const int64_t slot = u->slot[r / G];
+        float *po = a.part_o + (slot * G + r % G) * D;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const float2 v = half ? make_float2(o[n][2] * inv, o[n][3] * inv)
+                                  : make_float2(o[n][0] * inv, o[n][1] * inv);
+            *reinterpret_cast<float2 *>(po + 8 * n + 2 * t) = v;
+        }
+        if (t == 0) a.part_lse[slot * G + r % G] = le > 0.f ? (m + dev::lg2(le)) * kLn2 : -INFINITY;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
 // Merge of split heads (log-sum-exp): one CTA per (split head, query row). Warp w owns the
 // contiguous splits [w*k, (w+1)*k); it loads them 4 at a time (all loads in flight), keeps a
 // running maximum and sum, and the warps' results are combined through shared memory in warp
@@ -1286,6 +1561,17 @@ int device_init_plan(tg_plan *p) {
     else if (s.D == 128 && p->tiered) rc = set_smem_attr<128, true, kPairsTiered>(p->smem_bytes);
     else if (s.D == 64 && !p->tiered) rc = set_smem_attr<64, false, kPairs>(p->smem_bytes);
     else rc = TG_EUNSUPPORTED;
+    if (rc == TG_OK && !p->cunits.empty()) {
+        cudaError_t ce = s.D == 128
+            ? cudaFuncSetAttribute(cascade_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   cascade_smem_bytes<128>())
+            : cudaFuncSetAttribute(cascade_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   cascade_smem_bytes<64>());
+        if (ce != cudaSuccess) {
+            set_cuda_error("cudaFuncSetAttribute(cascade_kernel)", static_cast<int>(ce));
+            rc = TG_ECUDA;
+        }
+    }
     if (rc != TG_OK) {
         if (p->device != cur) cudaSetDevice(cur);
         return rc;
@@ -1302,7 +1588,8 @@ int device_init_plan(tg_plan *p) {
     const int64_t b_pl = al(p->n_partials * p->G * 4LL);
     const int64_t b_emp = al(static_cast<int64_t>(p->empties.size()) * 4LL);
     const int64_t b_err = 256;  // error word + dynamic ticket counters
-    p->dev_bytes = b_items + b_woff + b_merge + b_goff + b_po + b_pl + b_emp + b_err;
+    const int64_t b_cu = al(static_cast<int64_t>(p->cunits.size()) * static_cast<int64_t>(sizeof(CascadeUnit)));
+    p->dev_bytes = b_items + b_woff + b_merge + b_goff + b_po + b_pl + b_emp + b_err + b_cu;
     cudaError_t e = cudaMalloc(&p->dev_base, static_cast<size_t>(p->dev_bytes));
     if (e != cudaSuccess) {
         set_cuda_error("cudaMalloc(plan)", static_cast<int>(e));
@@ -1327,6 +1614,8 @@ int device_init_plan(tg_plan *p) {
     base += b_emp;
     p->d_err = reinterpret_cast<uint32_t *>(base);
     p->d_dyn = p->d_err + 16;
+    base += b_err;
+    p->d_cunits = p->cunits.empty() ? nullptr : reinterpret_cast<CascadeUnit *>(base);
 
     rc = TG_OK;
     auto up = [&](void *dst, const void *src, int64_t bytes) {
@@ -1337,6 +1626,7 @@ int device_init_plan(tg_plan *p) {
             rc = TG_ECUDA;
         }
     };
+    up(p->d_cunits, p->cunits.data(), static_cast<int64_t>(p->cunits.size()) * static_cast<int64_t>(sizeof(CascadeUnit)));
     up(p->d_items, p->items.data(), n_items * static_cast<int64_t>(sizeof(Item)));
     up(p->d_worker_off, p->worker_off.data(), (p->n_workers + 1) * 4LL);
     up(p->d_merge, p->merge.data(), static_cast<int64_t>(p->merge.size()) * static_cast<int64_t>(sizeof(MergeHead)));
@@ -1504,12 +1794,56 @@ static int decode_bf16(tg_plan *p, const void *q, const void *k_pages, const voi
     int rc = check_device(p);
     if (rc != TG_OK) return rc;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    const bool cascade = !p->cunits.empty();
+    if (cascade && (!k_pages || !v_pages || !page_table || !head_page_off ||
+                    !aligned16(k_pages) || !aligned16(v_pages) || p->shape.num_pages < 1))
+        return TG_EINVAL;
+    if (cascade) {
+        // Shared runs first (the decode kernel that follows waits for them before it starts).
+        rc = get_map(p, 0, k_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
+        if (rc == TG_OK) rc = get_map(p, 1, v_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
+        if (rc != TG_OK) return rc;
+        CascadeArgs c{};
+        c.units = p->d_cunits;
+        c.G = p->G;
+        c.Hq = p->shape.Hq;
+        c.Hkv = p->shape.Hkv;
+        c.scale_log2 = scale * 1.44269504088896340736f;
+        c.q = static_cast<const __nv_bfloat16 *>(q);
+        c.table = page_table;
+        c.head_off = head_page_off;
+        c.kv_len_dev = head_kv_len;
+        c.num_pages = p->shape.num_pages;
+        c.part_o = p->d_part_o;
+        c.part_lse = p->d_part_lse;
+        c.err = p->d_err;
+        c.wait_ns = p->wait_ns;
+        timing_mark(p, 0, stream);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(p->cunits.size()));
+        cfg.blockDim = dim3(kCasThreads);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const CUtensorMap &tk = *reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
+        const CUtensorMap &tv = *reinterpret_cast<const CUtensorMap *>(p->tmaps[1]);
+        if (p->shape.D == 128) {
+            cfg.dynamicSmemBytes = cascade_smem_bytes<128>();
+            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, cascade_kernel<128>, c, tk, tv));
+        } else {
+            cfg.dynamicSmemBytes = cascade_smem_bytes<64>();
+            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, cascade_kernel<64>, c, tk, tv));
+        }
+    }
     if (launch) {
         if (any_items) rc = get_map(p, 0, k_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
         if (rc == TG_OK && any_items) rc = get_map(p, 1, v_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
         if (rc != TG_OK) return rc;
         DecodeArgs a = base_args(p, q, head_kv_len, scale, out, lse);
-        timing_mark(p, 0, stream);
+        if (!cascade) timing_mark(p, 0, stream);
         a.table = page_table;
         a.head_off = head_page_off;
         a.group_of_head = group_of_head;
@@ -1521,7 +1855,7 @@ static int decode_bf16(tg_plan *p, const void *q, const void *k_pages, const voi
         else
             rc = launch_decode(p, decode_kernel<64, false, kPairs>, a, tk, tv, tk, tv, stream);
         if (rc != TG_OK) return rc;
-    } else {
+    } else if (!cascade) {
         timing_mark(p, 0, stream);
     }
     return finish_call(p, out, lse, stream);
@@ -1773,6 +2107,7 @@ extern "C" int tg_ragged_paged_decode_noalloc(tg_plan *p, const void *q, const v
                                               const int32_t *group_of_head, float scale,
                                               void *out, float *lse, tg_stream stream_) {
     if (!p || p->tiered) return TG_EINVAL;
+    if (!p->cunits.empty()) return TG_EUNSUPPORTED;  // cascade units live in the plan's memory
     if (!q || !out || !lse || !head_kv_len || !aligned16(q) || !aligned16(out) || !aligned16(lse))
         return TG_EINVAL;
     const bool any_items = !p->items.empty();

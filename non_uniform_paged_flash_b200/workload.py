@@ -202,19 +202,30 @@ def _pool_to_device(sp, which, n, layer, device, chunk_pages=1 << 16):
 def to_device(sp: synth.Spec, lay: Layout, layer: int = 0, device="cuda", num_workers: int = 0,
               min_splits: int = 1, max_chunk_pages: int = 0, seqs=None, static_permille: int = 0,
               dyn_chunk_pages: int = 0, early_prologue: bool = False, wait_limit_us: int = 0,
-              test_withhold_page: int = 0) -> DeviceBatch:
+              test_withhold_page: int = 0, cascade: bool = False,
+              min_readers: int = 2) -> DeviceBatch:
     import torch
     dev = torch.device(device)
     B = lay.kv_len.shape[0]
     shape = make_shape(B, sp.Hq, sp.Hkv, sp.D, lay.num_pages, lay.num_slow_pages, sp.page)
-    plan = tg_plan_create(shape, lay.kv_len, lay.group_of_head, lay.group_off,
-                          fast_len=lay.fast_len,
-                          slow_table_len=0 if lay.slow_table is None else lay.slow_table.size,
-                          num_workers=num_workers, min_splits=min_splits,
-                          max_chunk_pages=max_chunk_pages, static_permille=static_permille,
-                          dyn_chunk_pages=dyn_chunk_pages, early_prologue=early_prologue,
-                          wait_limit_us=wait_limit_us, test_withhold_page=test_withhold_page,
-                          device=dev.index if dev.index is not None else -1)
+    if cascade:
+        from . import tg_plan_create_cascade
+        plan = tg_plan_create_cascade(
+            shape, lay.kv_len, lay.group_of_head, lay.group_off,
+            lay.table if lay.table.size else np.full(1, -1), lay.head_off,
+            min_readers=min_readers, num_workers=num_workers, min_splits=min_splits,
+            max_chunk_pages=max_chunk_pages, static_permille=static_permille,
+            dyn_chunk_pages=dyn_chunk_pages, early_prologue=early_prologue,
+            wait_limit_us=wait_limit_us, device=dev.index if dev.index is not None else -1)
+    else:
+        plan = tg_plan_create(shape, lay.kv_len, lay.group_of_head, lay.group_off,
+                              fast_len=lay.fast_len,
+                              slow_table_len=0 if lay.slow_table is None else lay.slow_table.size,
+                              num_workers=num_workers, min_splits=min_splits,
+                              max_chunk_pages=max_chunk_pages, static_permille=static_permille,
+                              dyn_chunk_pages=dyn_chunk_pages, early_prologue=early_prologue,
+                              wait_limit_us=wait_limit_us, test_withhold_page=test_withhold_page,
+                              device=dev.index if dev.index is not None else -1)
     qb = synth.q_bits(sp, layer)
     q = _bf16_tensor(qb if seqs is None else np.ascontiguousarray(qb[seqs]), dev)
     out = torch.empty((B, sp.Hq, sp.D), dtype=torch.bfloat16, device=dev)

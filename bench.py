@@ -72,7 +72,7 @@ def _plan_kw(cfg):
     elif cfg == 4:
         # shared prefix pages: the cascade reads each shared run once per step for all its
         # readers; the private pages stay on the split-K items
-        kw.update(static_permille=1000, cascade=True)
+        kw.update(static_permille=850, dyn_chunk_pages=16, cascade=True)
     elif cfg == 5:
         kw.update(min_splits=64, max_chunk_pages=128, static_permille=900, dyn_chunk_pages=32)
     return kw

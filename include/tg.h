@@ -220,8 +220,9 @@ int tg_plan_get_info(const tg_plan *p, tg_plan_info *info);
  * recovers, per KV head, the runs of full pages that >= min_readers (at least 2) heads' rows
  * share at the same positions: rows are grouped by their page id at a position, a group runs
  * as far as all its rows keep the same page ids, then splits again below. Every run is read
- * once per step by cascade units of up to 64 query rows (64/G readers with their G query
- * heads each: a dense tile for the tensor cores) instead of once per reader; each reader's
+ * once per step by cascade units of up to 256 query rows (256/G readers with their G query
+ * heads each: two 128-row tiles for tcgen05.mma, S and O in tensor memory) instead of once per
+ * reader; each reader's
  * private pages (after its deepest run) go through the ordinary split-K items; every head with
  * a run is merged from its run partials (in run order) and its items'. Results equal those of
  * tg_ragged_paged_decode up to rounding; the plan stays valid while the device table and
@@ -231,8 +232,8 @@ int tg_plan_create_cascade(const tg_shape *shape, const int32_t *kv_len,
                            int32_t n_groups, const int32_t *page_table,
                            const int64_t *head_page_off, int64_t table_len, int32_t min_readers,
                            const tg_plan_opts *opts, tg_plan **out);
-/* Inspection: per cascade unit (tg_plan_info.n_cascade of them), 4 + 2*64 ints: KV head, first
- * page position, end page position, readers, then 64 reader sequences and 64 partial slots
+/* Inspection: per cascade unit (tg_plan_info.n_cascade of them), 4 + 2*256 ints: KV head, first
+ * page position, end page position, readers, then 256 reader sequences and 256 partial slots
  * (-1 past the readers). */
 int tg_plan_cascade_units(const tg_plan *p, int32_t *units);
 

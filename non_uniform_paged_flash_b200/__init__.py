@@ -61,6 +61,9 @@ class tg_plan_info(ctypes.Structure):
 
 _L = None
 
+#: Query rows of one prefix-cascade unit (two tensor-core tiles of 128 rows).
+CASCADE_ROWS = 256
+
 # (name, restype, argtypes)
 _P, _I32, _I64, _F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
 _SIGS = [
@@ -327,13 +330,13 @@ def tg_plan_create_cascade(shape: tg_shape, kv_len, group_of_head, group_off, pa
 
 def tg_plan_cascade_units(plan: Plan):
     """Cascade units: (meta int32[n, 4] = KV head, first page position, end position, readers;
-    readers int32[n, 64]; slots int32[n, 64]), -1 past each unit's readers."""
+    readers int32[n, 256]; slots int32[n, 256]), -1 past each unit's readers."""
     n = tg_plan_get_info(plan)["n_cascade"]
-    w = 4 + 2 * 64
-    out = np.empty((max(n, 1), w), dtype=np.int32)
+    R = CASCADE_ROWS
+    out = np.empty((max(n, 1), 4 + 2 * R), dtype=np.int32)
     _check(_lib().tg_plan_cascade_units(plan.handle, _hp(out)), "tg_plan_cascade_units")
     out = out[:n]
-    return out[:, :4], out[:, 4:68], out[:, 68:]
+    return out[:, :4], out[:, 4:4 + R], out[:, 4 + R:]
 
 
 def tg_plan_destroy(plan: Plan):

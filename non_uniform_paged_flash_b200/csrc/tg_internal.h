@@ -32,10 +32,11 @@ struct MergeHead {
     int32_t pad;
 };
 
-// Prefix cascade: one unit = up to 64 query rows (kCascadeRows / G readers, each with its G
-// query heads) that read the same run of shared pages [pos_begin, pos_end) of KV head h: the
-// pages are identical in every reader's table row. Each reader gets one partial result.
-constexpr int kCascadeRows = 64;
+// Prefix cascade: one unit = up to 256 query rows (two tensor-core tiles of 128; kCascadeRows / G
+// readers, each with its G query heads) that read the same run of shared pages
+// [pos_begin, pos_end) of KV head h: the pages are identical in every reader's table row. Each
+// reader gets one partial result.
+constexpr int kCascadeRows = 256;
 struct CascadeUnit {
     int32_t h;
     int32_t pos_begin;  // first page position (index within every reader's row)

@@ -255,6 +255,8 @@ struct DecodeArgs {
     uint32_t *err;
     uint64_t *trace;                 // worker timeline (n_workers x kTraceWords) or null
     float *token_scores;             // bf16 kernel: per-token scores [table_len*16][G], or null
+    int32_t late_wait;               // wait for the preceding grid only before exiting (cascade
+                                     // plans: that grid is the cascade kernel, independent work)
 };
 
 // Per-stage header written by the producer before it arrives on the stage's full barrier.
@@ -547,7 +549,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
     // tables first and wait just before their first copy (queries, K/V and every write come
     // after the wait).
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (!a.early_prologue || !producer) asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!a.late_wait && (!a.early_prologue || !producer)) asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // Heads with no retained token: out = 0, lse = -inf (consumer warps).
     if (a.n_empty > 0 && !producer) {
@@ -584,7 +586,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
         int pstage = 0;        // seq % stages
         uint32_t pphase = 0;   // (seq / stages) & 1
         bool aborted = false;
-        bool waited = !a.early_prologue;
+        bool waited = !a.early_prologue || a.late_wait;
         auto wait_predecessor = [&]() {
             if (!waited) {
                 asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -790,6 +792,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                 }
             }
         }
+        if (a.late_wait) asm volatile("griddepcontrol.wait;" ::: "memory");
         return;
     }
 
@@ -839,6 +842,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
         for (uint32_t s = seq; s < issued; ++s)
             dev::mbar_wait(full0 + 8 * (s % stages), (s / stages) & 1u,
                            a.wait_ns < dev::kDrainNs ? a.wait_ns : dev::kDrainNs);
+        if (a.late_wait) asm volatile("griddepcontrol.wait;" ::: "memory");
     };
 
     while (true) {
@@ -1043,24 +1047,28 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
         }
     }
     if (trace && lane == 0) trace[4] = dev::global_timer();
+    if (a.late_wait) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ------------------------------------------------------------------------------------------
-// Prefix cascade kernel: one CTA per cascade unit (a run of pages shared by up to 64 query
-// rows). Warp kCasConsumers is the producer: it reads the run's page ids from the first
-// reader's row 32 at a time, and one lane issues 2-D TMA loads of K and V into a ring of
-// kCasStages stages. Warps 0..3 each own 16 query rows and compute, per 16-token page,
-// S = Q K^T (rows on M, tokens on N, mma.m16n8k16; K fragments by ldmatrix from the swizzled
-// page; even and odd k-steps in separate accumulators to halve the dependent chain), the online
-// softmax of their rows, and O += P V with P taken from the S accumulators as the A operand
-// (tokens on K) and V fragments by ldmatrix.trans. Every run is whole pages (the planner takes
-// full pages only), so no token mask. Each reader's rows end as a normalised partial (o, lse)
-// in its slot, merged with the head's other partials by the merge kernel.
+// Prefix cascade kernel (5th-generation tensor cores): one CTA per cascade unit, a run of pages
+// shared by up to two tiles of 128 query rows (each row one (reader, query head) pair).
+//   warps 0-3 / 4-7: softmax of tile 0 / 1; thread i of a warpgroup owns query row i, which is
+//                    lane i of tensor memory, so a row's max and sums need no shuffles
+//   warp 8:          allocates tensor memory; lane 0 issues every tcgen05.mma
+//   warp 9:          producer: page ids 32 at a time, 2-D TMA loads of K and V, 4 pages (64
+//                    tokens) per block, into a ring of kTcStages blocks
+// Per block and tile: S = Q K^T (M = 128 rows, N = 64 tokens, K = D; both operands K-major,
+// 128-byte swizzled, S in tensor memory); the softmax reads S with tcgen05.ld, keeps the
+// running max (lazy rescale: the max moves only when a block exceeds it by 2^8; then O is
+// read, scaled and written back in tensor memory), writes P as bf16 into a swizzled tile;
+// O += P V (M = 128, N = D, K = 16 tokens per page; V is the MN-major operand, as stored).
+// The two tiles alternate, so one tile's softmax overlaps the other's MMAs. Each reader's
+// rows end as a normalised partial (o, lse) in its slot, merged with the head's other
+// partials by the merge kernel.
+// Tensor memory (512 columns): tile t holds S in columns [256t, 256t + 64) and O in
+// [256t + 128, 256t + 128 + D).
 // ------------------------------------------------------------------------------------------
-constexpr int kCasConsumers = 4;
-constexpr int kCasThreads = (kCasConsumers + 1) * 32;
-constexpr int kCasStages = 6;
-
 struct CascadeArgs {
     const CascadeUnit *units;
     int32_t G, Hq, Hkv;
@@ -1076,248 +1084,412 @@ struct CascadeArgs {
     uint64_t wait_ns;
 };
 
+namespace tc {
+
+// 32 lanes x 64 consecutive columns of fp32 from tensor memory (lane = the warp's quarter).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+                 :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Shared-memory matrix descriptor of a 128-byte-swizzled operand (atoms of 8 rows x 128 bytes,
+// 1024-byte aligned): start address, leading byte offset, stride byte offset (8-row groups),
+// the descriptor version of this architecture (1) and the swizzle mode (2 = 128 bytes).
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
+           (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, A K-major, B K-major
+// (b_mn = 0) or MN-major (b_mn = 1), N and M.
+__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t n, uint32_t m, uint32_t b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn << 16) | ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                    uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        :: "r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives on the mbarrier once every tcgen05.mma issued so far by this thread has completed.
+__device__ __forceinline__ void commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(bar) : "memory");
+}
+
+}  // namespace tc
+
+constexpr int kTcRows = 128;               // rows per tile = tensor-memory lanes
+constexpr int kTcThreads = 11 * 32;        // 8 softmax warps, 2 MMA warps, 1 producer warp
+constexpr int kTcStages = 3;               // K/V blocks in flight
+constexpr uint32_t kTcCols = 512;          // tensor-memory columns of the CTA
+
+template <int D>
+struct TcLayout {
+    static constexpr int kHalves = D / 64;                  // 64-element (128-byte) column halves
+    static constexpr int kQTile = kTcRows * D * 2;          // one tile of Q
+    static constexpr int kPTile = kTcRows * 64 * 2;         // one buffer of P (64 tokens)
+    static constexpr int kKBlock = 64 * D * 2;              // 64 tokens of K
+    static constexpr int kStage = 2 * kKBlock;              // K then V
+    static constexpr int kQ = 0;
+    static constexpr int kP = kQ + 2 * kQTile;              // [tile][buffer]
+    static constexpr int kKV = kP + 4 * kPTile;
+    static constexpr int kBars = kKV + kTcStages * kStage;  // mbarriers, then the TMEM address
+    static constexpr int kBytes = kBars + 256;
+};
+
 template <int D>
 constexpr int cascade_smem_bytes() {
-    return 1024 + kCasStages * 2 * Layout<D>::KB + kCasStages * 16 + kCasStages * 4 + 16;
+    return 1024 + TcLayout<D>::kBytes;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kCasThreads)
+__global__ void __launch_bounds__(kTcThreads, 1)
     cascade_kernel(const __grid_constant__ CascadeArgs a, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v) {
-    using L = Layout<D>;
+    using TL = TcLayout<D>;
     constexpr int KS = D / 16;  // k-steps of S = Q K^T
-    constexpr int NT = D / 8;   // n-tiles of O
     constexpr unsigned FULL = 0xffffffffu;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kCasStages * 2 * L::KB);
-    volatile int32_t *skip = reinterpret_cast<volatile int32_t *>(bars + 2 * kCasStages);
-    volatile int32_t *abort_flag = skip + kCasStages;
-    const uint32_t full0 = dev::smem_addr(bars), empty0 = dev::smem_addr(bars + kCasStages);
+    const uint32_t sbase = dev::smem_addr(smem);
+    // mbarriers: kv_full[S], kv_empty[S], q_full, then per tile t and buffer b (index 2t + b):
+    // s_full[4], p_full[4], o_done[4]; then drain[2]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TL::kBars);
+    const uint32_t bar0 = dev::smem_addr(bars);
+    const uint32_t kv_full = bar0, kv_empty = bar0 + 8 * kTcStages, q_full = bar0 + 16 * kTcStages;
+    const uint32_t s_full = q_full + 8, p_full = s_full + 32, o_done = p_full + 32, drain = o_done + 32;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + TL::kBars + 8 * (2 * kTcStages + 15));
+    volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
 
     const CascadeUnit *u = a.units + blockIdx.x;
     const int32_t h = u->h, pb = u->pos_begin, pe = u->pos_end, nr = u->n_readers;
+    const int32_t G = a.G;
     const int32_t npages = pe - pb;
+    const int32_t nblocks = (npages + 3) / 4;
+    const int32_t ntiles = nr * G > kTcRows ? 2 : 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
     if (threadIdx.x == 0) {
-        for (int st = 0; st < kCasStages; ++st) {
-            dev::mbar_init(full0 + 8 * st, 1);
-            dev::mbar_init(empty0 + 8 * st, kCasConsumers);
+        for (int st = 0; st < kTcStages; ++st) {
+            dev::mbar_init(kv_full + 8 * st, 1);
+            dev::mbar_init(kv_empty + 8 * st, ntiles);
         }
+        dev::mbar_init(q_full, 4 * ntiles);
+        for (int k = 0; k < 4; ++k) {
+            dev::mbar_init(s_full + 8 * k, 1);
+            dev::mbar_init(p_full + 8 * k, 4);
+            dev::mbar_init(o_done + 8 * k, 1);
+        }
+        dev::mbar_init(drain, 1);
+        dev::mbar_init(drain + 8, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    if (warp == 8) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(dev::smem_addr(tmem_slot)), "r"(kTcCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc::fence_before();
     __syncthreads();
-    // The previous kernel in the stream (a merge reading the partial slots, a writer of q or of
-    // the pages) completes first; then the decode kernel that follows may launch.
+    tc::fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // The previous kernel in the stream completes first; then the next one may launch.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    auto timed_out = [&]() {
+        atomicOr(a.err, kErrTimeout);
+        *abort_flag = 1;
+    };
 
-    if (warp == kCasConsumers) {
+    if (warp == 10) {
         // ================================ producer warp ================================
-        // Page ids are read 32 at a time (lane k: page k of the block), one block ahead, so
-        // the copies are never held up by an id load; lane 0 waits for the stages and issues.
-        if (lane == 0)
-            for (int32_t r = 0; r < nr; ++r)
-                if (a.kv_len_dev[static_cast<int64_t>(u->reader[r]) * a.Hkv + h] < pe * 16)
-                    atomicOr(a.err, kErrPlan);
         const int32_t *row = a.table + a.head_off[static_cast<int64_t>(u->reader[0]) * a.Hkv + h] + pb;
         int32_t ids = lane < npages ? __ldg(row + lane) : -1;
         int32_t ids_next = 32 + lane < npages ? __ldg(row + 32 + lane) : -1;
         int32_t issued = 0;
-        for (int32_t i = 0; i < npages; ++i) {
-            if (i > 0 && (i & 31) == 0) {
-                ids = ids_next;
-                ids_next = i + 32 + lane < npages ? __ldg(row + i + 32 + lane) : -1;
+        for (int32_t blk = 0; blk < nblocks; ++blk) {
+            if (blk == 1) {
+                // every reader's length still covers the run (checked once the copies are going)
+                bool bad = false;
+                for (int32_t r = lane; r < nr; r += 32)
+                    bad |= a.kv_len_dev[static_cast<int64_t>(u->reader[r]) * a.Hkv + h] < pe * 16;
+                if (__any_sync(FULL, bad) && lane == 0) atomicOr(a.err, kErrPlan);
             }
-            const int64_t pid = __shfl_sync(FULL, ids, i & 31);
+            const int st = blk % kTcStages;
+            const uint32_t ph = static_cast<uint32_t>(blk / kTcStages) & 1u;
             int32_t stop = 0;
-            if (lane == 0) {
-                const int st = i % kCasStages;
-                const uint32_t ph = static_cast<uint32_t>(i / kCasStages) & 1u;
-                if (!dev::mbar_wait(empty0 + 8 * st, ph ^ 1u, a.wait_ns) || *abort_flag) {
-                    atomicOr(a.err, kErrTimeout);
-                    *abort_flag = 1;
-                    stop = 1;
-                } else {
-                    const uint32_t fb = full0 + 8 * st;
-                    if (pid < 0 || pid >= a.num_pages) {
-                        atomicOr(a.err, kErrBadPage);
-                        skip[st] = 1;
-                        dev::mbar_arrive(fb);
-                    } else {
-                        skip[st] = 0;
-                        const uint32_t sa = dev::smem_addr(smem + st * 2 * L::KB);
-                        const int32_t y = static_cast<int32_t>(pid * 16);
-                        dev::mbar_arrive_expect_tx(fb, 2u * L::KB);
-#pragma unroll
-                        for (int bx = 0; bx < D / 64; ++bx) {
-                            dev::tma_load_2d(sa + bx * 2048, &tm_k, bx * 64, y, fb);
-                            dev::tma_load_2d(sa + L::KB + bx * 2048, &tm_v, bx * 64, y, fb);
-                        }
-                    }
-                }
+            if (lane == 0 && (!dev::mbar_wait(kv_empty + 8 * st, ph ^ 1u, a.wait_ns) || *abort_flag)) {
+                timed_out();
+                stop = 1;
             }
             if (__shfl_sync(FULL, stop, 0)) break;
-            issued = i + 1;
+            const int32_t np = min(4, npages - 4 * blk);
+            const uint32_t kv = sbase + TL::kKV + st * TL::kStage;
+            if (lane == 0) dev::mbar_arrive_expect_tx(kv_full + 8 * st, static_cast<uint32_t>(np) * 2u * 16u * D * 2u);
+            // lane k < np loads page 4 blk + k (its ids block starts at a multiple of 32 pages,
+            // and 4 blk .. 4 blk + 3 never straddle one)
+            if (blk > 0 && ((4 * blk) & 31) == 0) {
+                ids = ids_next;
+                ids_next = 4 * blk + 32 + lane < npages ? __ldg(row + 4 * blk + 32 + lane) : -1;
+            }
+            int64_t pid = __shfl_sync(FULL, ids, (4 * blk + (lane & 3)) & 31);
+            __syncwarp();
+            if (lane < np) {
+                if (pid < 0 || pid >= a.num_pages) {
+                    atomicOr(a.err, kErrBadPage);
+                    pid = 0;  // a page of the pool; the result is flagged as wrong
+                }
+                const int32_t y = static_cast<int32_t>(pid * 16);
+#pragma unroll
+                for (int hf = 0; hf < TL::kHalves; ++hf) {
+                    dev::tma_load_2d(kv + hf * (TL::kKBlock / TL::kHalves) + lane * 2048, &tm_k, hf * 64, y, kv_full + 8 * st);
+                    dev::tma_load_2d(kv + TL::kKBlock + hf * (TL::kKBlock / TL::kHalves) + lane * 2048, &tm_v, hf * 64, y,
+                                     kv_full + 8 * st);
+                }
+            }
+            __syncwarp();
+            issued = blk + 1;
         }
-        // No copy may be in flight when the CTA exits: wait for the last page of every stage.
+        if (nblocks <= 1) {
+            bool bad = false;
+            for (int32_t r = lane; r < nr; r += 32)
+                bad |= a.kv_len_dev[static_cast<int64_t>(u->reader[r]) * a.Hkv + h] < pe * 16;
+            if (__any_sync(FULL, bad) && lane == 0) atomicOr(a.err, kErrPlan);
+        }
+        // No copy may be in flight when the CTA exits: wait for the last block of every stage.
         if (lane == 0)
-            for (int32_t i = issued - kCasStages < 0 ? 0 : issued - kCasStages; i < issued; ++i)
-                dev::mbar_wait(full0 + 8 * (i % kCasStages), static_cast<uint32_t>(i / kCasStages) & 1u,
+            for (int32_t b = issued - kTcStages < 0 ? 0 : issued - kTcStages; b < issued; ++b)
+                dev::mbar_wait(kv_full + 8 * (b % kTcStages), static_cast<uint32_t>(b / kTcStages) & 1u,
                                a.wait_ns < dev::kDrainNs ? a.wait_ns : dev::kDrainNs);
         return;
     }
 
-    // ================================ consumer warps ================================
-    const int g = lane >> 2, t = lane & 3;
-    const int G = a.G;
-    const int r0 = warp * 16 + g, r1 = r0 + 8;          // this lane's two query rows
-    const bool ok0 = r0 / G < nr, ok1 = r1 / G < nr;
-    // query fragments (A operand: rows on M, d on K), straight from global memory
-    uint32_t qa[KS][4];
-    {
-        const __nv_bfloat16 *q0 = ok0 ? a.q + ((static_cast<int64_t>(u->reader[r0 / G]) * a.Hq + h * G + r0 % G) * D) : nullptr;
-        const __nv_bfloat16 *q1 = ok1 ? a.q + ((static_cast<int64_t>(u->reader[r1 / G]) * a.Hq + h * G + r1 % G) * D) : nullptr;
+    if (warp == 8 || warp == 9) {
+        // ========================= MMA warps (tile 0: warp 8, tile 1: warp 9) =========================
+        // S(blk) goes to buffer blk & 1 and is issued before PV(blk - 1), so the next block's
+        // scores are ready when the softmax finishes a block.
+        const int t = warp - 8;
+        if (lane == 0 && t < ntiles) {
+            const uint32_t id_s = tc::idesc_bf16(64, kTcRows, 0);
+            const uint32_t id_o = tc::idesc_bf16(D, kTcRows, 1);
+            const uint32_t q = sbase + TL::kQ + t * TL::kQTile;
+            bool ok = dev::mbar_wait(q_full, 0, a.wait_ns);
+            tc::fence_after();
+            auto issue_o = [&](int32_t blk) {
+                const uint32_t kv = sbase + TL::kKV + (blk % kTcStages) * TL::kStage + TL::kKBlock;
+                const uint32_t pt = sbase + TL::kP + (2 * t + (blk & 1)) * TL::kPTile;
+                const int32_t np = min(4, npages - 4 * blk);
+                for (int32_t k = 0; k < np; ++k)
+                    tc::mma(tmem + 256 * t + 128, tc::sdesc(pt + k * 32, 16, 1024),
+                            tc::sdesc(kv + k * 2048, TL::kKBlock / TL::kHalves, 1024), id_o, blk > 0 || k > 0);
+                tc::commit(o_done + 8 * (2 * t + (blk & 1)));
+                tc::commit(kv_empty + 8 * (blk % kTcStages));
+            };
+            for (int32_t blk = 0; ok && blk <= nblocks; ++blk) {
+                if (blk < nblocks) {
+                    const int st = blk % kTcStages;
+                    ok = dev::mbar_wait(kv_full + 8 * st, static_cast<uint32_t>(blk / kTcStages) & 1u, a.wait_ns) &&
+                         !*abort_flag;
+                    tc::fence_after();
+                    if (!ok) break;
+                    const uint32_t kv = sbase + TL::kKV + st * TL::kStage;
 #pragma unroll
-        for (int j = 0; j < KS; ++j) {
-            qa[j][0] = q0 ? *reinterpret_cast<const uint32_t *>(q0 + 16 * j + 2 * t) : 0u;
-            qa[j][1] = q1 ? *reinterpret_cast<const uint32_t *>(q1 + 16 * j + 2 * t) : 0u;
-            qa[j][2] = q0 ? *reinterpret_cast<const uint32_t *>(q0 + 16 * j + 2 * t + 8) : 0u;
-            qa[j][3] = q1 ? *reinterpret_cast<const uint32_t *>(q1 + 16 * j + 2 * t + 8) : 0u;
-        }
-    }
-    // ldmatrix row offsets: K (B operand of S; matrices (tokens 0-7 | 8-15) x (chunk 2j | 2j+1))
-    // and V (B operand of O, transposed; matrices (tokens 0-7 | 8-15) x (chunk 2i | 2i+1)).
-    uint32_t offK[KS], offV[NT / 2];
-#pragma unroll
-    for (int j = 0; j < KS; ++j) {
-        const uint32_t tok = (lane & 7) + 8 * (lane >> 4), ch = 2 * j + ((lane >> 3) & 1);
-        offK[j] = (ch >> 3) * 2048 + dev::swz(tok, ch & 7);
-    }
-#pragma unroll
-    for (int i = 0; i < NT / 2; ++i) {
-        const uint32_t tok = (lane & 7) + 8 * ((lane >> 3) & 1), ch = 2 * i + (lane >> 4);
-        offV[i] = L::KB + (ch >> 3) * 2048 + dev::swz(tok, ch & 7);
-    }
-    float o[NT][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, le0 = 0.f, le1 = 0.f, lr0 = 0.f, lr1 = 0.f;
-
-    for (int32_t i = 0; i < npages; ++i) {
-        const int st = i % kCasStages;
-        const uint32_t ph = static_cast<uint32_t>(i / kCasStages) & 1u;
-        if (!dev::mbar_wait(full0 + 8 * st, ph, a.wait_ns) || *abort_flag) {
-            if (lane == 0) {
-                atomicOr(a.err, kErrTimeout);
-                *abort_flag = 1;
-            }
-            return;
-        }
-        if (!skip[st]) {
-            const uint32_t sa = dev::smem_addr(smem + st * 2 * L::KB);
-            float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int j = 0; j < KS; ++j) {
-                uint32_t b0, b1, b2, b3;
-                dev::ldsm_x4(sa + offK[j], b0, b1, b2, b3);
-                float (&acc)[2][4] = (j & 1) ? s2 : s;
-                dev::mma_bf16(acc[0], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b0, b1);
-                dev::mma_bf16(acc[1], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b2, b3);
-            }
-#pragma unroll
-            for (int n = 0; n < 2; ++n)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) s[n][c] += s2[n][c];
-            // s[n][0..1]: row g, tokens 8n + 2t, +1; s[n][2..3]: row g + 8
-            float x[2][4];
-#pragma unroll
-            for (int n = 0; n < 2; ++n)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) x[n][c] = s[n][c] * a.scale_log2;
-            float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
-            float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
-            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 1));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 1));
-            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 2));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 2));
-            // lazy rescale: the running max moves only when a page exceeds it by more than 2^8
-            const bool up0 = mx0 > m0 + 8.f, up1 = mx1 > m1 + 8.f;
-            if (__any_sync(FULL, up0 || up1)) {
-                const float n0 = up0 ? mx0 : m0, n1 = up1 ? mx1 : m1;
-                const float c0 = m0 == -INFINITY ? 0.f : dev::ex2(m0 - n0);
-                const float c1 = m1 == -INFINITY ? 0.f : dev::ex2(m1 - n1);
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    o[n][0] *= c0;
-                    o[n][1] *= c0;
-                    o[n][2] *= c1;
-                    o[n][3] *= c1;
+                    for (int k = 0; k < KS; ++k) {
+                        const uint32_t hf = k / 4, off = (k % 4) * 32;
+                        tc::mma(tmem + 256 * t + 64 * (blk & 1),
+                                tc::sdesc(q + hf * (kTcRows * 128) + off, 16, 1024),
+                                tc::sdesc(kv + hf * (TL::kKBlock / TL::kHalves) + off, 16, 1024), id_s, k > 0);
+                    }
+                    tc::commit(s_full + 8 * (2 * t + (blk & 1)));
                 }
-                le0 *= c0;
-                lr0 *= c0;
-                le1 *= c1;
-                lr1 *= c1;
-                m0 = n0;
-                m1 = n1;
+                if (blk >= 1) {
+                    const int32_t pbk = blk - 1;
+                    ok = dev::mbar_wait(p_full + 8 * (2 * t + (pbk & 1)), static_cast<uint32_t>(pbk >> 1) & 1u, a.wait_ns) &&
+                         !*abort_flag;
+                    tc::fence_after();
+                    if (!ok) break;
+                    issue_o(pbk);
+                }
             }
-            float p[2][4];
-#pragma unroll
-            for (int n = 0; n < 2; ++n) {
-                p[n][0] = dev::ex2(x[n][0] - m0);
-                p[n][1] = dev::ex2(x[n][1] - m0);
-                p[n][2] = dev::ex2(x[n][2] - m1);
-                p[n][3] = dev::ex2(x[n][3] - m1);
-            }
-            le0 += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
-            le1 += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
-            // P as the A operand of O += P V (rows on M, tokens on K)
-            const uint32_t pa0 = dev::pack_bf16(p[0][0], p[0][1]), pa1 = dev::pack_bf16(p[0][2], p[0][3]);
-            const uint32_t pa2 = dev::pack_bf16(p[1][0], p[1][1]), pa3 = dev::pack_bf16(p[1][2], p[1][3]);
-            lr0 += (dev::bf16_lo(pa0) + dev::bf16_hi(pa0)) + (dev::bf16_lo(pa2) + dev::bf16_hi(pa2));
-            lr1 += (dev::bf16_lo(pa1) + dev::bf16_hi(pa1)) + (dev::bf16_lo(pa3) + dev::bf16_hi(pa3));
-#pragma unroll
-            for (int i2 = 0; i2 < NT / 2; ++i2) {
-                uint32_t v0, v1, v2, v3;
-                dev::ldsm_x4_t(sa + offV[i2], v0, v1, v2, v3);
-                dev::mma_bf16(o[2 * i2], pa0, pa1, pa2, pa3, v0, v1);
-                dev::mma_bf16(o[2 * i2 + 1], pa0, pa1, pa2, pa3, v2, v3);
-            }
+            if (!ok) timed_out();
+            // every MMA this thread issued has finished before tensor memory is released
+            tc::commit(drain + 8 * t);
+            dev::mbar_wait(drain + 8 * t, 0, a.wait_ns < dev::kDrainNs ? a.wait_ns : dev::kDrainNs);
         }
         __syncwarp();
-        if (lane == 0) dev::mbar_arrive(empty0 + 8 * st);
-    }
+    } else {
+        // ================================ softmax warpgroups ================================
+        const int t = warp >> 2, qd = warp & 3;
+        const int i = 32 * qd + lane;                 // row of the tile = tensor-memory lane
+        const int r = kTcRows * t + i;                // row of the unit
+        const bool active = t < ntiles;
+        const bool valid = r < nr * G;
+        const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
+        const uint32_t t_s = tmem + lanes + 256 * t, t_o = t_s + 128;
+        float m = -INFINITY, le = 0.f;
+        if (active) {
+            // Q row -> the tile's swizzled K-major layout (zeros for rows past the readers)
+            const uint32_t qrow = sbase + TL::kQ + t * TL::kQTile + i * 128;
+            const uint4 *src = valid ? reinterpret_cast<const uint4 *>(
+                                           a.q + (static_cast<int64_t>(u->reader[r / G]) * a.Hq + h * G + r % G) * D)
+                                     : nullptr;
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) {
+                const uint4 v = src ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t addr = qrow + (c / 8) * (kTcRows * 128) + (((c % 8) ^ (i & 7)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                             :: "r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+            }
+            tc::fence_async_smem();
+            __syncwarp();
+            if (lane == 0) dev::mbar_arrive(q_full);
 
-    // Row sums over the 4 lanes of a row, then the partials of valid rows.
-    le0 += __shfl_xor_sync(FULL, le0, 1);
-    le0 += __shfl_xor_sync(FULL, le0, 2);
-    le1 += __shfl_xor_sync(FULL, le1, 1);
-    le1 += __shfl_xor_sync(FULL, le1, 2);
-    lr0 += __shfl_xor_sync(FULL, lr0, 1);
-    lr0 += __shfl_xor_sync(FULL, lr0, 2);
-    lr1 += __shfl_xor_sync(FULL, lr1, 1);
-    lr1 += __shfl_xor_sync(FULL, lr1, 2);
-    constexpr float kLn2 = 0.69314718055994530942f;
+            bool ok = true;
+            for (int32_t blk = 0; blk < nblocks; ++blk) {
+                const int bf = blk & 1;
+                const uint32_t ph = static_cast<uint32_t>(blk >> 1) & 1u;   // phase of buffer bf's barriers
+                ok = dev::mbar_wait(s_full + 8 * (2 * t + bf), ph, a.wait_ns) && !*abort_flag;
+                if (!__all_sync(FULL, ok)) { ok = false; break; }
+                tc::fence_after();
+                uint32_t sr[64];
+                tc::tmem_ld64(t_s + 64 * bf, sr);
+                tc::tmem_wait_ld();
+                const int32_t nv = 16 * min(4, npages - 4 * blk);    // valid tokens of the block
+                // row max of the raw scores (the scale is positive), 8 independent chains
+                float mr[8];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        const int r = half ? r1 : r0;
-        if (!(half ? ok1 : ok0)) continue;
-        const float le = half ? le1 : le0, lr = half ? lr1 : lr0, m = half ? m1 : m0;
-        const float inv = lr > 0.f ? 1.f / lr : 0.f;
-        const int64_t slot = u->slot[r / G];
-        float *po = a.part_o + (slot * G + r % G) * D;
+                for (int c = 0; c < 8; ++c) mr[c] = -INFINITY;
+                if (nv == 64) {
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const float2 v = half ? make_float2(o[n][2] * inv, o[n][3] * inv)
-                                  : make_float2(o[n][0] * inv, o[n][1] * inv);
-            *reinterpret_cast<float2 *>(po + 8 * n + 2 * t) = v;
+                    for (int c = 0; c < 64; ++c) mr[c & 7] = fmaxf(mr[c & 7], __uint_as_float(sr[c]));
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (c < nv) mr[c & 7] = fmaxf(mr[c & 7], __uint_as_float(sr[c]));
+                }
+                const float mx = fmaxf(fmaxf(fmaxf(mr[0], mr[1]), fmaxf(mr[2], mr[3])),
+                                       fmaxf(fmaxf(mr[4], mr[5]), fmaxf(mr[6], mr[7]))) * a.scale_log2;
+                // P buffer bf was last read by PV(blk - 2)
+                if (blk >= 2) {
+                    ok = dev::mbar_wait(o_done + 8 * (2 * t + bf), ph ^ 1u, a.wait_ns) && !*abort_flag;
+                    if (!__all_sync(FULL, ok)) { ok = false; break; }
+                }
+                const bool up = mx > m + 8.f;
+                if (__any_sync(FULL, up)) {
+                    const float mn = up ? mx : m;
+                    const float c0 = !up ? 1.f : (m == -INFINITY ? 0.f : dev::ex2(m - mn));
+                    if (blk > 0) {
+                        // O holds PV(0 .. blk - 1): wait for PV(blk - 1), then scale it in place
+                        ok = dev::mbar_wait(o_done + 8 * (2 * t + (bf ^ 1)), static_cast<uint32_t>((blk - 1) >> 1) & 1u,
+                                            a.wait_ns) && !*abort_flag;
+                        if (!__all_sync(FULL, ok)) { ok = false; break; }
+                        tc::fence_after();
+#pragma unroll 1
+                        for (int ch = 0; ch < D / 32; ++ch) {
+                            uint32_t o[32];
+                            tc::tmem_ld32(t_o + 32 * ch, o);
+                            tc::tmem_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * c0);
+                            tc::tmem_st32(t_o + 32 * ch, o);
+                        }
+                        tc::tmem_wait_st();
+                    }
+                    le *= c0;
+                    m = mn;
+                }
+                // p = 2^(s * scale - m): one FFMA and one ex2 per score; 8 partial sums
+                const uint32_t prow = sbase + TL::kP + (2 * t + bf) * TL::kPTile + i * 128;
+                float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                const float nm = -m;
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = 8 * c8 + 2 * e;
+                        float p0 = dev::ex2(fmaf(__uint_as_float(sr[c]), a.scale_log2, nm));
+                        float p1 = dev::ex2(fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, nm));
+                        if (nv < 64) {
+                            p0 = c < nv ? p0 : 0.f;
+                            p1 = c + 1 < nv ? p1 : 0.f;
+                        }
+                        ls[e] += p0;
+                        ls[4 + e] += p1;
+                        w[e] = dev::pack_bf16(p0, p1);
+                    }
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                 :: "r"(prow + ((c8 ^ (i & 7)) << 4)), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                                 : "memory");
+                }
+                le += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+                tc::fence_async_smem();
+                tc::fence_before();
+                __syncwarp();
+                if (lane == 0) dev::mbar_arrive(p_full + 8 * (2 * t + bf));
+            }
+            // all of PV(0 .. nblocks - 1) are done: wait for the last two
+            for (int32_t b = nblocks - 2 < 0 ? 0 : nblocks - 2; ok && b < nblocks; ++b) {
+                ok = dev::mbar_wait(o_done + 8 * (2 * t + (b & 1)), static_cast<uint32_t>(b >> 1) & 1u, a.wait_ns);
+                ok = __all_sync(FULL, ok);
+            }
+            tc::fence_after();
+            if (!ok) {
+                if (lane == 0) timed_out();
+            } else {
+                // out row = O / le (partial), lse = (m + log2 le) ln 2
+                const float inv = le > 0.f ? 1.f / le : 0.f;
+                float *po = valid ? a.part_o + (static_cast<int64_t>(u->slot[r / G]) * G + r % G) * D : nullptr;
+#pragma unroll 1
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t o[32];
+                    tc::tmem_ld32(t_o + 32 * ch, o);
+                    tc::tmem_wait_ld();
+                    if (po) {
+#pragma unroll
+                        for (int c = 0; c < 32; c += 4)
+                            *reinterpret_cast<float4 *>(po + 32 * ch + c) =
+                                make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
+                                            __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
+                    }
+                }
+                if (valid) {
+                    constexpr float kLn2 = 0.69314718055994530942f;
+                    a.part_lse[static_cast<int64_t>(u->slot[r / G]) * G + r % G] =
+                        le > 0.f ? (m + dev::lg2(le)) * kLn2 : -INFINITY;
+                }
+            }
         }
-        if (t == 0) a.part_lse[slot * G + r % G] = le > 0.f ? (m + dev::lg2(le)) * kLn2 : -INFINITY;
     }
+    // Warps 0-9 meet before tensor memory is released (the producer may have left already).
+    tc::fence_before();
+    asm volatile("bar.sync 1, %0;" :: "r"(10 * 32) : "memory");
+    tc::fence_after();
+    if (warp == 8) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTcCols) : "memory");
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1327,9 +1499,10 @@ __global__ void __launch_bounds__(kCasThreads)
 // order, so the result does not depend on timing. Launched as a programmatic dependent of
 // the decode kernel: it waits for that grid before reading.
 // ------------------------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(1024) split_merge_kernel(const MergeHead *mh, int32_t G, int32_t Hq,
-                                                           int32_t Hkv, const float *part_o,
+template <int D, bool ROWS>
+__global__ void __launch_bounds__(1024) split_merge_kernel(const MergeHead *mh, int64_t n_rows,
+                                                           int32_t G, int32_t Hq, int32_t Hkv,
+                                                           const float *part_o,
                                                            const float *part_lse,
                                                            __nv_bfloat16 *out, float *lse) {
     constexpr int VEC = D / 32;
@@ -1338,14 +1511,19 @@ __global__ void __launch_bounds__(1024) split_merge_kernel(const MergeHead *mh, 
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // Every CTA of this grid has started: the next kernel may be scheduled.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    const MergeHead h = mh[blockIdx.x / G];
-    const int n = blockIdx.x % G;
+    // ROWS: one warp per (split head, query row), several rows per CTA (heads of few splits);
+    // else one CTA per row, its warps splitting the head's splits.
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nw = ROWS ? 1 : blockDim.x >> 5;
+    const int64_t rid = ROWS ? static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp : blockIdx.x;
+    if (rid >= n_rows) return;
+    const MergeHead h = mh[rid / G];
+    const int n = static_cast<int>(rid % G);
     const float *pl = part_lse + static_cast<int64_t>(h.first_slot) * G + n;
     const float *po = part_o + (static_cast<int64_t>(h.first_slot) * G + n) * D + lane * VEC;
     const int64_t pstride = static_cast<int64_t>(G) * D;
     const int k = (h.nsplit + nw - 1) / nw;
-    const int j0 = warp * k, j1 = min(h.nsplit, j0 + k);
+    const int j0 = (ROWS ? 0 : warp) * k, j1 = min(h.nsplit, j0 + k);
 
     float m = -INFINITY, sum = 0.f, acc[VEC];
 #pragma unroll
@@ -1378,7 +1556,7 @@ __global__ void __launch_bounds__(1024) split_merge_kernel(const MergeHead *mh, 
     }
     const int32_t b = h.bh / Hkv, hh = h.bh - b * Hkv;
     const int64_t row = static_cast<int64_t>(b) * Hq + static_cast<int64_t>(hh) * G + n;
-    if (nw > 1) {
+    if (!ROWS && nw > 1) {
         float *s_m = s_dyn, *s_s = s_dyn + nw;
         float(*s_acc)[D] = reinterpret_cast<float(*)[D]>(s_dyn + 2 * nw);
         if (lane == 0) {
@@ -1707,28 +1885,42 @@ static int launch_decode(tg_plan *p, DecodeFn fn, const DecodeArgs &a, const CUt
     return TG_OK;
 }
 
+// Merge kernel of the split heads (optionally a programmatic dependent launch). Heads of at
+// most 8 splits (merge_warps == 1) get one warp per query row, 8 rows per CTA.
+static int launch_merge(const tg_plan *p, const MergeHead *d_merge, const float *po, const float *pl,
+                        void *out, float *lse, cudaStream_t stream, bool pdl) {
+    constexpr int kRowsPerCta = 8;
+    const int64_t n_rows = static_cast<int64_t>(p->merge.size()) * p->G;
+    const bool rows = p->merge_warps == 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(rows ? (n_rows + kRowsPerCta - 1) / kRowsPerCta : n_rows));
+    cfg.blockDim = dim3(static_cast<unsigned>(rows ? 32 * kRowsPerCta : 32 * p->merge_warps));
+    cfg.dynamicSmemBytes = !rows ? static_cast<size_t>(p->merge_warps) * (2 + p->shape.D) * 4 : 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const int32_t G = p->G, Hq = p->shape.Hq, Hkv = p->shape.Hkv;
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
+    if (p->shape.D == 128) {
+        if (rows) TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<128, true>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, lse));
+        else TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<128, false>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, lse));
+    } else {
+        if (rows) TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<64, true>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, lse));
+        else TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<64, false>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, lse));
+    }
+    return TG_OK;
+}
+
 // Merge kernel of the split heads, as a programmatic dependent launch of the decode kernel;
 // then close the call's timing record.
 static int finish_call(tg_plan *p, void *out, float *lse, cudaStream_t stream) {
     timing_mark(p, 1, stream);
     if (!p->merge.empty()) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(p->merge.size() * p->G));
-        cfg.blockDim = dim3(static_cast<unsigned>(32 * p->merge_warps));
-        cfg.dynamicSmemBytes = p->merge_warps > 1 ? static_cast<size_t>(p->merge_warps) * (2 + p->shape.D) * 4 : 0;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const int32_t G = p->G, Hq = p->shape.Hq, Hkv = p->shape.Hkv;
-        const float *po = p->d_part_o, *pl = p->d_part_lse;
-        __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
-        if (p->shape.D == 128)
-            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<128>, (const MergeHead *)p->d_merge, G, Hq, Hkv, po, pl, o, lse));
-        else
-            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<64>, (const MergeHead *)p->d_merge, G, Hq, Hkv, po, pl, o, lse));
+        const int rc = launch_merge(p, p->d_merge, p->d_part_o, p->d_part_lse, out, lse, stream, true);
+        if (rc != TG_OK) return rc;
     }
     timing_mark(p, 2, stream);
     return TG_OK;
@@ -1821,7 +2013,7 @@ static int decode_bf16(tg_plan *p, const void *q, const void *k_pages, const voi
         timing_mark(p, 0, stream);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(p->cunits.size()));
-        cfg.blockDim = dim3(kCasThreads);
+        cfg.blockDim = dim3(kTcThreads);
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1848,6 +2040,10 @@ static int decode_bf16(tg_plan *p, const void *q, const void *k_pages, const voi
         a.head_off = head_page_off;
         a.group_of_head = group_of_head;
         a.token_scores = token_scores;
+        // The cascade kernel before this one waited for the previous step's merge before it let
+        // this grid launch, and writes other partial slots: the decode overlaps it and waits for
+        // it only before exiting (so the merge that follows sees both).
+        a.late_wait = cascade ? 1 : 0;
         const CUtensorMap &tk = *reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
         const CUtensorMap &tv = *reinterpret_cast<const CUtensorMap *>(p->tmaps[1]);
         if (p->shape.D == 128)
@@ -2239,19 +2435,8 @@ extern "C" int tg_ragged_paged_decode_noalloc(tg_plan *p, const void *q, const v
         else
             TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel<64, false, tg::kPairs>, a, tk, tv, tk, tv));
     }
-    if (!p->merge.empty()) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(p->merge.size() * p->G));
-        cfg.blockDim = dim3(static_cast<unsigned>(32 * p->merge_warps));
-        cfg.dynamicSmemBytes = p->merge_warps > 1 ? static_cast<size_t>(p->merge_warps) * (2 + s.D) * 4 : 0;
-        cfg.stream = stream;
-        __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
-        if (s.D == 128)
-            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<128>, (const MergeHead *)d_merge,
-                                           p->G, s.Hq, s.Hkv, (const float *)d_po, (const float *)d_pl, o, lse));
-        else
-            TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<64>, (const MergeHead *)d_merge,
-                                           p->G, s.Hq, s.Hkv, (const float *)d_po, (const float *)d_pl, o, lse));
-    }
+    if (!p->merge.empty())
+        return launch_merge(p, reinterpret_cast<const MergeHead *>(d_merge), reinterpret_cast<const float *>(d_po),
+                            reinterpret_cast<const float *>(d_pl), out, lse, stream, false);
     return TG_OK;
 }

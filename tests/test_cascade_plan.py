@@ -29,7 +29,7 @@ def check_cascade(plan, B, Hq, Hkv, kv_len, table, head_off, min_readers=2):
     partials = {}
     runs = {}
     for (h, pb, pe, nr), rd, sl in zip(meta, readers, slots):
-        assert 0 <= pb < pe and 1 <= nr <= 64 // G
+        assert 0 <= pb < pe and 1 <= nr <= tg.CASCADE_ROWS // G
         assert (rd[nr:] == -1).all() and (sl[nr:] == -1).all()
         rows = rd[:nr]
         for b in rows:
@@ -84,7 +84,7 @@ def test_prefix_config_runs(full):
     sys_pages = sp.sys_tokens // 16
     doc_pages = sp.doc_tokens // 16
     doc, _ = synth.prefix_layout(sp)
-    per = 64 // (sp.Hq // sp.Hkv)
+    per = tg.CASCADE_ROWS // (sp.Hq // sp.Hkv)
     for h in range(sp.Hkv):
         m = meta[meta[:, 0] == h]
         sysu = m[(m[:, 1] == 0) & (m[:, 2] == sys_pages)]

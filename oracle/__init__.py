@@ -61,6 +61,8 @@ def _L():
         lib.or_token_scores.argtypes = [i32, i32, i32, i32, i32, p, p, i64, p, p, p, f64, p]
         lib.or_token_scores.restype = ctypes.c_int
         lib.or_h2o_accumulate.argtypes = [i32, i32, p, p, p, p]
+        lib.or_tier_step.argtypes = [i32, i32, i32, i32, p, p]
+        lib.or_tier_step.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -269,3 +271,12 @@ def h2o_accumulate(s, lse, score):
     out = np.empty(n, dtype=np.float32)
     _L().or_h2o_accumulate(n, G, _ptr(s_), _ptr(l_), _ptr(sc), _ptr(out))
     return out
+
+
+def tier_step(n: int, f: int, cap: int, slow_cap: int):
+    """(fast slot, slow index) of appending position n to a head with f fast tokens out of n;
+    slow index -1 when nothing moves; (-1, -1) when the state is outside the rules."""
+    fs = np.zeros(1, np.int32)
+    si = np.zeros(1, np.int32)
+    rc = _L().or_tier_step(int(n), int(f), int(cap), int(slow_cap), _ptr(fs), _ptr(si))
+    return (int(fs[0]), int(si[0])) if rc == 0 else (-1, -1)

@@ -572,3 +572,31 @@ void or_h2o_accumulate(int32_t n, int32_t G, const double *s, const double *lse,
         score_out[t] = (float)acc;
     }
 }
+
+/* ---------------------------------------------------------------------------------------
+ * Tier migration. [TTKV] 核心方法 1 (Tier Layout: recent tokens in the fast high-precision
+ * tier, older ones in the slow quantised tier) and 2 (Tier Content: the most recent tokens, as
+ * many as the fast tier holds, are fast; the rest slow). Readings used: the fast tier of a head
+ * holds the last f <= cap tokens, the token at position p in fast slot p mod cap; the slow tier
+ * holds positions [0, n - f) at slow index = position. Appending position n: with f < cap (only
+ * when every token is fast, n == f) it takes fast slot n and nothing moves; with f == cap the
+ * oldest fast token (position n - cap) moves to slow index n - cap (quantised by
+ * or_quantize_int8) and the new token takes its slot. Returns 0 with the slots, or -1 when the
+ * state is outside these rules or the slow tier has no reserved slot left.
+ * ------------------------------------------------------------------------------------- */
+int or_tier_step(int32_t n, int32_t f, int32_t cap, int32_t slow_cap, int32_t *fast_slot,
+                 int32_t *slow_index) {
+    *fast_slot = -1;
+    *slow_index = -1;
+    if (cap < 1 || f < 0 || f > cap || f > n) return -1;
+    if (f < cap) {
+        if (n != f) return -1;
+        *fast_slot = n;
+        return 0;
+    }
+    int32_t old = n - cap;
+    if (old >= slow_cap) return -1;
+    *slow_index = old;
+    *fast_slot = old % cap;
+    return 0;
+}

@@ -533,3 +533,42 @@ def test_h2o_accumulate_adds_one_per_query_head():
         assert (sc1 >= sc0).all()
         inc = sc1.astype(np.float64) - sc0.astype(np.float64)
         assert inc.sum() == pytest.approx(G, abs=n * 4 * 2.0 ** -23)
+
+
+# ---------------------------------------------------------------------------------------
+# Tier migration (fast window -> INT8 tier): hand-worked steps and the tier invariants.
+# ---------------------------------------------------------------------------------------
+
+def test_tier_step_hand_worked():
+    """cap 3: positions 0, 1, 2 fill fast slots 0, 1, 2; position 3 moves position 0 to slow
+    index 0 and takes slot 0; position 4 moves 1 (slot 1); position 5 moves 2 (slot 2); 6 moves
+    3 (slot 0)."""
+    n, f = 0, 0
+    got = []
+    for _ in range(7):
+        got.append(oracle.tier_step(n, f, 3, 100))
+        n, f = n + 1, min(f + 1, 3)
+    assert got == [(0, -1), (1, -1), (2, -1), (0, 0), (1, 1), (2, 2), (0, 3)]
+    assert oracle.tier_step(10, 2, 3, 100) == (-1, -1)     # not full, yet older tokens exist
+    assert oracle.tier_step(10, 3, 3, 7) == (-1, -1)       # no reserved slow slot for position 7
+    assert oracle.tier_step(10, 3, 3, 8) == (1, 7)
+
+
+def test_tier_step_keeps_recent_fast_and_older_slow():
+    rng = np.random.default_rng(45)
+    for _ in range(60):
+        cap = int(rng.integers(1, 40))
+        fast = {}
+        slow = []
+        n, f = 0, 0
+        for _ in range(int(rng.integers(1, 200))):
+            fs, si = oracle.tier_step(n, f, cap, 10**6)
+            assert fs >= 0
+            if si >= 0:
+                assert fast[fs] == si                   # the oldest fast token leaves
+                slow.append(si)
+            fast[fs] = n
+            n, f = n + 1, min(f + 1, cap)
+        assert sorted(fast.values()) == list(range(n - f, n))
+        assert all(s_ == p % cap for s_, p in fast.items())
+        assert slow == list(range(n - f))

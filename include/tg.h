@@ -174,6 +174,14 @@ typedef struct tg_plan_opts {
     int32_t test_withhold_page; /* testing only (0 = off): worker 0's producer never signals
                                  its page number test_withhold_page (1-based), so a bounded
                                  wait runs out on purpose; no copy is issued for that page */
+    int32_t capacity;         /* tiered plans only ("TTKV" tiers that grow every step): 1 = the
+                                 kv_len / fast_len given to tg_plan_create are capacities, the
+                                 reserved slots of each head (fast tier: fast_len; INT8 tier:
+                                 kv_len - fast_len); each decode call reads the current lengths
+                                 from head_kv_len / head_fast_len (which must fit them, else
+                                 TG_EBADPAGE) and skips reserved pages that hold no token yet,
+                                 so appends (tg_tiered_append) never need a new plan. 0: the
+                                 lengths are exact, as for bf16 plans */
 } tg_plan_opts;
 
 /* Build a plan. kv_len[B*Hkv] (host): retained tokens per (sequence, KV head); the decode
@@ -418,6 +426,31 @@ int tg_h2o_update(const tg_shape *shape, int32_t recent, const float *token_scor
                   const float *lse, const int64_t *head_page_off, const int32_t *head_budget,
                   const int32_t *head_kv_len, const int32_t *slot_pos, float *slot_score,
                   const int32_t *next_pos, int32_t *head_victim, tg_stream stream);
+
+/* Tier migration ("TTKV" 核心方法 1 Tier Layout, 2 Tier Content: the most recent tokens stay in
+ * the high-precision fast tier, older ones move to the quantised slow tier). Per (sequence, KV
+ * head): the fast tier holds the last f = head_fast_len tokens of the n = head_kv_len, at most
+ * head_fast_cap of them, token at position p in fast slot p mod head_fast_cap of its fast row
+ * (fast_page_table / fast_head_off, as for tg_tiered_decode); the INT8 tier holds positions
+ * [0, n - f) at slow index = position (slow_page_table / slow_head_off; head_slow_cap reserved
+ * slots). Appending position n: with f < cap (then n == f: every token is still fast) it takes
+ * fast slot n; with a full window the oldest fast token (position n - cap) is quantised into
+ * slow index n - cap with the rule of tg_quantize_int8 (codes and scale bit-exact with it) and
+ * the new token takes its fast slot. head_kv_len grows by one, head_fast_len up to the cap.
+ *   k_new, v_new  device bf16 [B][Hkv][D] (16-byte aligned); k_fast, v_fast the bf16 pools;
+ *   k_q8, v_q8, k_scale, v_scale the INT8 pools and scales (written); shape.num_pages and
+ *   shape.num_slow_pages bound the page ids; D % 32 == 0, D <= 128.
+ *   moved_out (int32 [B*Hkv]): slow index written, or -1; slot_out: fast slot written, or -1
+ *   when nothing was appended (a state outside the rules above, no reserved slow slot left, or
+ *   a page id outside its pool).
+ * One launch, one warp per head. A tiered plan made with tg_plan_opts.capacity = 1 for the
+ * reserved sizes decodes every later state without a new plan. */
+int tg_tiered_append(const tg_shape *shape, const void *k_new, const void *v_new, void *k_fast,
+                     void *v_fast, const int32_t *fast_page_table, const int64_t *fast_head_off,
+                     const int32_t *head_fast_cap, int8_t *k_q8, int8_t *v_q8, float *k_scale,
+                     float *v_scale, const int32_t *slow_page_table, const int64_t *slow_head_off,
+                     const int32_t *head_slow_cap, int32_t *head_kv_len, int32_t *head_fast_len,
+                     int32_t *moved_out, int32_t *slot_out, tg_stream stream);
 
 #ifdef __cplusplus
 }

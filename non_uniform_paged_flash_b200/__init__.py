@@ -45,7 +45,8 @@ class tg_plan_opts(ctypes.Structure):
                 ("max_chunk_pages", ctypes.c_int32), ("host_only", ctypes.c_int32),
                 ("device", ctypes.c_int32), ("static_permille", ctypes.c_int32),
                 ("dyn_chunk_pages", ctypes.c_int32), ("early_prologue", ctypes.c_int32),
-                ("wait_limit_us", ctypes.c_int32), ("test_withhold_page", ctypes.c_int32)]
+                ("wait_limit_us", ctypes.c_int32), ("test_withhold_page", ctypes.c_int32),
+                ("capacity", ctypes.c_int32)]
 
 
 class tg_plan_info(ctypes.Structure):
@@ -110,6 +111,8 @@ _SIGS = [
                                               _I64, _I32, ctypes.POINTER(tg_plan_opts),
                                               ctypes.POINTER(_P)]),
     ("tg_plan_cascade_units", ctypes.c_int, [_P, _P]),
+    ("tg_tiered_append", ctypes.c_int, [ctypes.POINTER(tg_shape), _P, _P, _P, _P, _P, _P, _P, _P,
+                                        _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
 ]
 
 #: Symbols the C ABI exports (include/tg.h).
@@ -292,14 +295,14 @@ def tg_plan_create(shape: tg_shape, kv_len, group_of_head, group_off, fast_len=N
                    max_chunk_pages: int = 0, host_only: bool = False, device: int = -1,
                    static_permille: int = 0, dyn_chunk_pages: int = 0,
                    early_prologue: bool = False, wait_limit_us: int = 0,
-                   test_withhold_page: int = 0) -> Plan:
+                   test_withhold_page: int = 0, capacity: bool = False) -> Plan:
     kv = _h(kv_len, np.int32).reshape(-1)
     fl = None if fast_len is None else _h(fast_len, np.int32).reshape(-1)
     goh = _h(group_of_head, np.int32).reshape(-1)
     goff = _h(group_off, np.int64).reshape(-1)
     opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
                         static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us,
-                        test_withhold_page)
+                        test_withhold_page, int(capacity))
     h = ctypes.c_void_p()
     _check(_lib().tg_plan_create(ctypes.byref(shape), _hp(kv), _hp(fl), _hp(goh), _hp(goff),
                                  goff.size - 1, slow_table_len, ctypes.byref(opts),
@@ -319,7 +322,7 @@ def tg_plan_create_cascade(shape: tg_shape, kv_len, group_of_head, group_off, pa
     tbl = _h(page_table, np.int32).reshape(-1)
     hoff = _h(head_page_off, np.int64).reshape(-1)
     opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
-                        static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us, 0)
+                        static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us, 0, 0)
     h = ctypes.c_void_p()
     _check(_lib().tg_plan_create_cascade(ctypes.byref(shape), _hp(kv), _hp(goh), _hp(goff),
                                          goff.size - 1, _hp(tbl), _hp(hoff), tbl.size,
@@ -453,6 +456,20 @@ def tg_h2o_update(shape: tg_shape, recent: int, token_scores, lse, head_page_off
         ctypes.byref(shape), int(recent), _dp(token_scores), _dp(lse), _dp(head_page_off),
         _dp(head_budget), _dp(head_kv_len), _dp(slot_pos), _dp(slot_score), _dp(next_pos),
         _dp(head_victim), _stream(stream)), "tg_h2o_update")
+
+
+def tg_tiered_append(shape: tg_shape, k_new, v_new, k_fast, v_fast, fast_page_table,
+                     fast_head_off, head_fast_cap, k_q8, v_q8, k_scale, v_scale, slow_page_table,
+                     slow_head_off, head_slow_cap, head_kv_len, head_fast_len, moved_out,
+                     slot_out, stream=None):
+    """Append one token per (sequence, KV head) to the fast tier, migrating the oldest fast
+    token of a full window into the INT8 tier (see include/tg.h)."""
+    _check(_lib().tg_tiered_append(
+        ctypes.byref(shape), _dp(k_new), _dp(v_new), _dp(k_fast), _dp(v_fast),
+        _dp(fast_page_table), _dp(fast_head_off), _dp(head_fast_cap), _dp(k_q8), _dp(v_q8),
+        _dp(k_scale), _dp(v_scale), _dp(slow_page_table), _dp(slow_head_off),
+        _dp(head_slow_cap), _dp(head_kv_len), _dp(head_fast_len), _dp(moved_out),
+        _dp(slot_out), _stream(stream)), "tg_tiered_append")
 
 
 def tg_tiered_decode(plan: Plan, q, k_q8, v_q8, k_scale, v_scale, slow_page_table,

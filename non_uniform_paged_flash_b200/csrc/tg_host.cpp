@@ -602,6 +602,8 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
     p->early_prologue = o.early_prologue != 0;
     if (o.wait_limit_us > 0) p->wait_ns = static_cast<uint64_t>(o.wait_limit_us) * 1000ull;
     p->withhold = o.test_withhold_page > 0 ? o.test_withhold_page : 0;
+    if (o.capacity && !fast_len) { delete p; return TG_EINVAL; }
+    p->capacity = o.capacity != 0;
 
     // Prefix cascade: shared runs per KV head, cut into units of kCascadeRows query rows.
     std::vector<int32_t> casc_cnt;

@@ -91,6 +91,7 @@ struct tg_plan {
     bool early_prologue = false;      // see tg_plan_opts.early_prologue
     uint64_t wait_ns = 4000000000ull; // bound of any single wait in the decode kernel
     int32_t withhold = 0;             // see tg_plan_opts.test_withhold_page
+    bool capacity = false;            // see tg_plan_opts.capacity
     int32_t n_workers = 0;
     int64_t kv_bytes = 0;
 

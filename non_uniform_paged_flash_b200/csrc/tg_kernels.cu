@@ -257,6 +257,8 @@ struct DecodeArgs {
     float *token_scores;             // bf16 kernel: per-token scores [table_len*16][G], or null
     int32_t late_wait;               // wait for the preceding grid only before exiting (cascade
                                      // plans: that grid is the cascade kernel, independent work)
+    int32_t capacity;                // tiered: planned lengths are capacities; tier token counts
+                                     // come from the device lengths of each call
 };
 
 // Per-stage header written by the producer before it arrives on the stage's full barrier.
@@ -597,6 +599,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
             Item mi{};
             int64_t mrow = 0;
             int32_t mok = 0;
+            int32_t mtt = 0;  // tokens of the item's tier in its head (this call's)
             if (lane < nc) {
                 mi = a.items[c0 + lane];
                 const bool slow = TIERED && (mi.flags & kItemSlow);
@@ -622,8 +625,17 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                 }
                 mok = (mrow >= lo && mrow + row_pages <= hi) ? 1 : 0;
                 if (!mok) atomicOr(a.err, kErrBadRow);
-                bool plan_ok = a.kv_len_dev[mi.bh] == mi.kv_len;
-                if (TIERED) plan_ok = plan_ok && a.fast_len_dev[mi.bh] == mi.fast_len;
+                mtt = mi.tier_tokens;
+                bool plan_ok;
+                if (TIERED && a.capacity) {
+                    // the plan reserved mi.fast_len fast and mi.kv_len - mi.fast_len slow slots
+                    const int32_t n = a.kv_len_dev[mi.bh], f = a.fast_len_dev[mi.bh];
+                    plan_ok = f >= 0 && f <= n && f <= mi.fast_len && n - f <= mi.kv_len - mi.fast_len;
+                    mtt = !plan_ok ? 0 : (slow ? n - f : f);
+                } else {
+                    plan_ok = a.kv_len_dev[mi.bh] == mi.kv_len;
+                    if (TIERED) plan_ok = plan_ok && a.fast_len_dev[mi.bh] == mi.fast_len;
+                }
                 if (!plan_ok) atomicOr(a.err, kErrPlan);
             }
             // Page ids of block (item j, pages p0 .. p0+31): lane k gets page p0 + k. The value
@@ -660,7 +672,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                 const int64_t row_j = __shfl_sync(FULL, mrow, j);
                 const int32_t pb = __shfl_sync(FULL, mi.page_begin, j);
                 const int32_t pe = __shfl_sync(FULL, mi.page_end, j);
-                const int32_t tt = __shfl_sync(FULL, mi.tier_tokens, j);
+                const int32_t tt = __shfl_sync(FULL, mtt, j);
                 const int32_t slot = __shfl_sync(FULL, mi.slot, j);
                 const int32_t fl = __shfl_sync(FULL, mi.flags, j);
                 const bool slow = TIERED && (fl & kItemSlow);
@@ -682,8 +694,11 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         return;
                     }
                     if (lane == 0) {
-                        if (page_id != kNoLoad &&
-                            (page_id < 0 || page_id >= (slow ? a.num_slow_pages : a.num_pages))) {
+                        const int32_t vtok = max(0, min(16, tt - pg * 16));
+                        if (vtok == 0) {
+                            page_id = kNoLoad;  // a reserved page holding no token yet
+                        } else if (page_id != kNoLoad &&
+                                   (page_id < 0 || page_id >= (slow ? a.num_slow_pages : a.num_pages))) {
                             atomicOr(a.err, kErrBadPage);
                             page_id = kNoLoad;
                         }
@@ -692,7 +707,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         // pages (pb, pb+1), (pb+2, pb+3), ... of an item are consumed together
                         const bool pair = ((pg - pb) & 1) == 0 && pg + 1 < pe;
                         StageHdr hd;
-                        hd.valid = page_id >= 0 ? min(16, tt - pg * 16) : 0;
+                        hd.valid = page_id >= 0 ? vtok : 0;
                         hd.flags = (slow ? kHdrSlow : 0) | (first ? kHdrFirst : 0) |
                                    (last ? kHdrLast : 0) | (pair ? kHdrPair : 0);
                         hd.bh = bh;
@@ -1959,6 +1974,7 @@ static DecodeArgs base_args(const tg_plan *p, const void *q, const int32_t *kv, 
     a.early_prologue = p->early_prologue ? 1 : 0;
     a.wait_ns = p->wait_ns;
     a.withhold = p->withhold;
+    a.capacity = p->capacity ? 1 : 0;
     return a;
 }
 

@@ -9,6 +9,7 @@
 //
 // Both kernels are small and memory-bound: the append moves 4·D bytes per head; the H2O update
 // reads 8 + 4·G bytes and writes 4 per retained token.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -198,6 +199,98 @@ __global__ void __launch_bounds__(kUpdateThreads)
     }
 }
 
+// Tier migration ("TTKV" 核心方法 1 Tier Layout, 2 Tier Content): one warp per (b, h). The fast
+// tier holds the most recent f <= cap tokens, token at position p in fast slot p mod cap; the
+// slow tier holds tokens [0, n - f) at slow index = position. A step appends position n: with
+// a free fast slot (f < cap, then all tokens are fast: n == f) it takes slot n; with a full
+// window the oldest fast token (position n - cap) is quantised (symmetric absmax INT8 per
+// token, the rule of tg_quantize_int8) into slow index n - cap, and the new token takes its slot.
+__global__ void __launch_bounds__(kAppendWarps * 32)
+    tier_append_kernel(int32_t BH, int32_t D, int64_t num_pages, int64_t num_slow_pages,
+                       const __nv_bfloat16 *k_new, const __nv_bfloat16 *v_new,
+                       __nv_bfloat16 *k_fast, __nv_bfloat16 *v_fast, const int32_t *fast_table,
+                       const int64_t *fast_off, const int32_t *fast_cap, int8_t *k_q8,
+                       int8_t *v_q8, float *k_scale, float *v_scale, const int32_t *slow_table,
+                       const int64_t *slow_off, const int32_t *slow_cap, int32_t *kv_len,
+                       int32_t *fast_len, int32_t *moved_out, int32_t *slot_out) {
+    const int32_t bh = blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (bh >= BH) return;
+    int32_t fslot = -1, sidx = -1;
+    int64_t fpid = -1, spid = -1;
+    if (lane == 0) {
+        const int32_t n = kv_len[bh], f = fast_len[bh], cap = fast_cap[bh];
+        const bool ok = cap >= 1 && f >= 0 && f <= cap && f <= n && (f == cap || n == f);
+        if (ok) {
+            if (f < cap) {
+                fslot = n;
+            } else {
+                sidx = n - cap;
+                fslot = sidx % cap;
+                if (sidx >= slow_cap[bh]) fslot = sidx = -1;  // no reserved slow slot left
+            }
+        }
+        if (fslot >= 0) {
+            fpid = fast_table[fast_off[bh] + fslot / 16];
+            if (fpid < 0 || fpid >= num_pages) fslot = sidx = -1;
+        }
+        if (sidx >= 0) {
+            spid = slow_table[slow_off[bh] + sidx / 16];
+            if (spid < 0 || spid >= num_slow_pages) fslot = sidx = -1;
+        }
+    }
+    fslot = __shfl_sync(0xffffffffu, fslot, 0);
+    sidx = __shfl_sync(0xffffffffu, sidx, 0);
+    fpid = __shfl_sync(0xffffffffu, fpid, 0);
+    spid = __shfl_sync(0xffffffffu, spid, 0);
+    if (fslot >= 0) {
+        const int64_t frow = (fpid * 16 + fslot % 16) * D;
+        if (sidx >= 0) {
+            // the leaving token's K and V rows -> INT8 codes + fp32 scale (read before overwrite)
+            const int64_t srow = spid * 16 + sidx % 16;
+            for (int t = 0; t < 2; ++t) {
+                const __nv_bfloat16 *src = (t == 0 ? k_fast : v_fast) + frow;
+                float x[4];
+                float amax = 0.f;
+                const int per = D / 32;  // 1..4
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    x[k] = k < per ? __bfloat162float(src[lane * per + k]) : 0.f;
+                    amax = fmaxf(amax, fabsf(x[k]));
+                }
+                for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+                const float sc = __fdiv_rn(amax, 127.f);
+                int8_t *codes = (t == 0 ? k_q8 : v_q8) + srow * D;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    int v = 0;
+                    if (amax != 0.f) v = max(-127, min(127, __float2int_rn(__fdiv_rn(x[k], sc))));
+                    if (k < per) codes[lane * per + k] = static_cast<int8_t>(v);
+                }
+                if (lane == 0) (t == 0 ? k_scale : v_scale)[srow] = sc;
+            }
+        }
+        __syncwarp();
+        const int nvec = D / 8;
+        const uint4 *kn = reinterpret_cast<const uint4 *>(k_new) + static_cast<int64_t>(bh) * nvec;
+        const uint4 *vn = reinterpret_cast<const uint4 *>(v_new) + static_cast<int64_t>(bh) * nvec;
+        uint4 *kd = reinterpret_cast<uint4 *>(k_fast + frow), *vd = reinterpret_cast<uint4 *>(v_fast + frow);
+        for (int i = lane; i < 2 * nvec; i += 32) {
+            if (i < nvec) kd[i] = kn[i];
+            else vd[i - nvec] = vn[i - nvec];
+        }
+    }
+    if (lane == 0) {
+        slot_out[bh] = fslot;
+        moved_out[bh] = sidx;
+        if (fslot >= 0) {
+            const int32_t f = fast_len[bh], cap = fast_cap[bh];
+            kv_len[bh] = kv_len[bh] + 1;
+            fast_len[bh] = f < cap ? f + 1 : cap;
+        }
+    }
+}
+
 bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_shape(const tg_shape *s) {
@@ -283,4 +376,32 @@ extern "C" int tg_h2o_update(const tg_shape *shape, int32_t recent, const float 
         shape->Hq, shape->Hkv, recent, token_scores, lse, head_page_off, head_budget, head_kv_len,
         slot_pos, slot_score, next_pos, head_victim);
     return launch_status("h2o_update_kernel");
+}
+
+extern "C" int tg_tiered_append(const tg_shape *shape, const void *k_new, const void *v_new,
+                                void *k_fast, void *v_fast, const int32_t *fast_page_table,
+                                const int64_t *fast_head_off, const int32_t *head_fast_cap,
+                                int8_t *k_q8, int8_t *v_q8, float *k_scale, float *v_scale,
+                                const int32_t *slow_page_table, const int64_t *slow_head_off,
+                                const int32_t *head_slow_cap, int32_t *head_kv_len,
+                                int32_t *head_fast_len, int32_t *moved_out, int32_t *slot_out,
+                                tg_stream stream) {
+    if (check_shape(shape) != TG_OK || shape->D % 32 != 0 || shape->D > 128 ||
+        shape->num_slow_pages < 0)
+        return TG_EINVAL;
+    const int32_t BH = shape->B * shape->Hkv;
+    if (BH == 0) return TG_OK;
+    if (!k_new || !v_new || !k_fast || !v_fast || !fast_page_table || !fast_head_off ||
+        !head_fast_cap || !k_q8 || !v_q8 || !k_scale || !v_scale || !slow_page_table ||
+        !slow_head_off || !head_slow_cap || !head_kv_len || !head_fast_len || !moved_out ||
+        !slot_out || !al16(k_new) || !al16(v_new) || !al16(k_fast) || !al16(v_fast))
+        return TG_EINVAL;
+    const unsigned grid = static_cast<unsigned>((BH + kAppendWarps - 1) / kAppendWarps);
+    tier_append_kernel<<<grid, kAppendWarps * 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        BH, shape->D, shape->num_pages, shape->num_slow_pages,
+        static_cast<const __nv_bfloat16 *>(k_new), static_cast<const __nv_bfloat16 *>(v_new),
+        static_cast<__nv_bfloat16 *>(k_fast), static_cast<__nv_bfloat16 *>(v_fast), fast_page_table,
+        fast_head_off, head_fast_cap, k_q8, v_q8, k_scale, v_scale, slow_page_table, slow_head_off,
+        head_slow_cap, head_kv_len, head_fast_len, moved_out, slot_out);
+    return launch_status("tier_append_kernel");
 }

@@ -466,10 +466,12 @@ def run_write_path(args):
     import non_uniform_paged_flash_b200 as tg
     from non_uniform_paged_flash_b200 import workload
 
+    if args.path == "ttkv":
+        return run_tier_path(args)
     cfg = args.config
     sp = synth.preset(cfg)
     if sp.kind == "tiered":
-        raise SystemExit("the write path is built for the bf16 tier")
+        raise SystemExit("--path sink|h2o is built for the bf16 tier; use --path ttkv")
     lay = workload.layout(sp, 0)
     db = workload.to_device(sp, lay, 0, **_plan_kw(cfg))
     B, Hkv = lay.kv_len.shape
@@ -570,6 +572,114 @@ def run_write_path(args):
     return 0
 
 
+def run_tier_path(args):
+    """Tiered decode step with the tier write path on one GPU (config 5 shape): every step
+    appends one token per (sequence, KV head) to the fast window, which moves its oldest token
+    into the INT8 tier (quantised in the same launch), then the tiered decode (+ merge) runs
+    from one capacity plan made for the reserved sizes. Prints one JSON line."""
+    import torch
+    import non_uniform_paged_flash_b200 as tg
+    from non_uniform_paged_flash_b200 import workload
+
+    cfg = 5
+    sp = synth.preset(cfg)
+    lay = workload.layout(sp, 0)
+    kw = _plan_kw(cfg)
+    db = workload.to_device(sp, lay, 0, **kw)
+    B, Hkv = lay.kv_len.shape
+    BH = B * Hkv
+    dev = db.q.device
+    stream = torch.cuda.current_stream()
+    n0 = lay.kv_len.reshape(-1).astype(np.int64)
+    f0 = lay.fast_len.reshape(-1).astype(np.int64)
+    n_ev = min(args.steps, 256)
+    extra = args.warmup + args.steps + n_ev + 1           # tokens every head gains in this run
+    # INT8 tier with room to grow: each head's row keeps its pages and gets hp new ones
+    old_rows = -(-(n0 - f0) // 16)
+    hp = -(-int(((n0 - f0) % 16).max() + extra) // 16) + 1
+    P_old = lay.num_slow_pages
+    table, off = [], np.zeros(BH, np.int64)
+    for bh in range(BH):
+        o = int(lay.slow_off.reshape(-1)[bh])
+        off[bh] = len(table)
+        table += lay.slow_table[o:o + int(old_rows[bh])].tolist()
+        table += list(range(P_old + bh * hp, P_old + (bh + 1) * hp))
+    P_new = P_old + BH * hp
+    it = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).to(dev)
+    stab, soff = it(table, np.int32), it(off.reshape(B, Hkv), np.int64)
+
+    def grow(t, tail):
+        g = torch.zeros((P_new,) + tuple(t.shape[1:]), dtype=t.dtype, device=dev)
+        g[:P_old].copy_(t)
+        return g
+    kq, vq = grow(db.k_q8, 16), grow(db.v_q8, 16)
+    ks, vs = grow(db.k_scale, 16), grow(db.v_scale, 16)
+    db.k_q8 = db.v_q8 = db.k_scale = db.v_scale = None
+    S = (old_rows + hp) * 16                               # reserved INT8 slots per head
+    shape = tg.make_shape(B, sp.Hq, sp.Hkv, sp.D, lay.num_pages, P_new)
+    plan = tg.tg_plan_create(shape, (f0 + S).reshape(B, Hkv), lay.group_of_head, lay.group_off,
+                             fast_len=f0.reshape(B, Hkv), slow_table_len=len(table),
+                             capacity=True, **kw)
+    fcap = it(f0, np.int32)
+    scap = it(S, np.int32)
+    kv_dev, fl_dev = it(n0, np.int32), it(f0, np.int32)
+    moved = torch.empty(BH, dtype=torch.int32, device=dev)
+    slot = torch.empty(BH, dtype=torch.int32, device=dev)
+    k_new = workload._bf16_tensor(synth.new_kv_bits(sp, 0, "k"), dev)
+    v_new = workload._bf16_tensor(synth.new_kv_bits(sp, 0, "v"), dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    marks = [[ev() for _ in range(3)] for _ in range(n_ev)]
+
+    def step(m=None):
+        if m: m[0].record(stream)
+        tg.tg_tiered_append(shape, k_new, v_new, db.k, db.v, db.table, db.head_off, fcap, kq, vq,
+                            ks, vs, stab, soff, scap, kv_dev, fl_dev, moved, slot, stream)
+        if m: m[1].record(stream)
+        tg.tg_tiered_decode(plan, db.q, kq, vq, ks, vs, stab, soff, db.k, db.v, db.table,
+                            db.head_off, kv_dev, fl_dev, sp.scale, db.out, db.lse, stream)
+        if m: m[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert tg.tg_plan_status(plan) == tg.TG_OK
+    assert (slot.cpu().numpy() >= 0).all() and (moved.cpu().numpy() >= 0).all()
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms_step = e0.elapsed_time(e1) / args.steps
+    for m in marks:
+        step(m)
+    torch.cuda.synchronize()
+    assert tg.tg_plan_status(plan) == tg.TG_OK
+    assert (moved.cpu().numpy() >= 0).all()
+    t_app = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
+    t_dec = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
+    kv_bytes = float(((kv_dev.cpu().numpy() - fl_dev.cpu().numpy()).astype(np.int64) * 2 * (sp.D + 4)).sum()
+                     + fl_dev.cpu().numpy().astype(np.int64).sum() * 2 * sp.D * 2)
+    peak, peak_kind = _measured_peak()
+    line = {
+        "metric": "tiered decode step with tier migration: step time", "value": ms_step * 1e3,
+        "unit": "us", "higher_is_better": False, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup,
+        "config": {"workload": WORKLOAD_NAMES[cfg], "config_id": cfg, "plan": "capacity"},
+        "kernels_us": {"tier_append": t_app * 1e3, "decode+merge": t_dec * 1e3},
+        "kv_bytes_per_step": int(kv_bytes),
+        "step_kv_gbs": kv_bytes / (ms_step * 1e-3) / 1e9, "peak_gbs": peak, "peak_kind": peak_kind,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -578,9 +688,10 @@ def main():
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", default="decode", choices=["decode", "sink", "h2o"],
+    ap.add_argument("--path", default="decode", choices=["decode", "sink", "h2o", "ttkv"],
                     help="decode: the decode step (default); sink / h2o: the decode step with "
-                         "the write path (one GPU, separate JSON line)")
+                         "the write path; ttkv: the tiered step with tier migration (config 5); "
+                         "one GPU, separate JSON line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

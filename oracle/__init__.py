@@ -63,6 +63,10 @@ def _L():
         lib.or_h2o_accumulate.argtypes = [i32, i32, p, p, p, p]
         lib.or_tier_step.argtypes = [i32, i32, i32, i32, p, p]
         lib.or_tier_step.restype = ctypes.c_int
+        lib.or_splitzip_codebook.argtypes = [i64, p, p]
+        lib.or_splitzip_encode.argtypes = [i64, p, p, p, p, p, p]
+        lib.or_splitzip_encode.restype = i64
+        lib.or_splitzip_decode.argtypes = [i64, p, p, p, i64, p, p, p]
         _lib = lib
     return _lib
 
@@ -280,3 +284,26 @@ def tier_step(n: int, f: int, cap: int, slow_cap: int):
     si = np.zeros(1, np.int32)
     rc = _L().or_tier_step(int(n), int(f), int(cap), int(slow_cap), _ptr(fs), _ptr(si))
     return (int(fs[0]), int(si[0])) if rc == 0 else (-1, -1)
+
+
+def splitzip_encode(x_bits):
+    """bf16 bits -> (codebook uint8[16], sm uint8[n], codes uint8[(n+1)//2], esc_pos int64[k],
+    esc_exp uint8[k])."""
+    x = _c(x_bits, np.uint16).reshape(-1)
+    n = x.size
+    cb = np.empty(16, np.uint8)
+    _L().or_splitzip_codebook(n, _ptr(x), _ptr(cb))
+    sm = np.empty(max(n, 1), np.uint8)
+    codes = np.empty(max((n + 1) // 2, 1), np.uint8)
+    pos = np.empty(max(n, 1), np.int64)
+    exp = np.empty(max(n, 1), np.uint8)
+    k = int(_L().or_splitzip_encode(n, _ptr(x), _ptr(cb), _ptr(sm), _ptr(codes), _ptr(pos), _ptr(exp)))
+    return cb, sm[:n], codes[:(n + 1) // 2], pos[:k], exp[:k]
+
+
+def splitzip_decode(n, codebook, sm, codes, esc_pos, esc_exp):
+    out = np.empty(max(int(n), 1), np.uint16)
+    cb, s_, c_ = _c(codebook, np.uint8), _c(sm, np.uint8), _c(codes, np.uint8)
+    p_, e_ = _c(esc_pos, np.int64), _c(esc_exp, np.uint8)
+    _L().or_splitzip_decode(int(n), _ptr(cb), _ptr(s_), _ptr(c_), p_.size, _ptr(p_), _ptr(e_), _ptr(out))
+    return out[:int(n)]

@@ -600,3 +600,65 @@ int or_tier_step(int32_t n, int32_t f, int32_t cap, int32_t slow_cap, int32_t *f
     *fast_slot = old % cap;
     return 0;
 }
+
+/* ---------------------------------------------------------------------------------------
+ * SplitZip: lossless BF16 codec for KV transfer. [SplitZip] explainer (arXiv 2605.01708),
+ * "Die SplitZip-Strategie" and "Warum es schnell ist": a bf16 value is sign, 8-bit exponent and
+ * 7-bit mantissa; exponents repeat, so the 16 most frequent get 4-bit codes (two per byte), the
+ * rare ones go to an escape stream (position, exponent) that decoding applies as overwrites.
+ * Readings used: the codebook lists 16 exponents by count descending, ties by exponent
+ * ascending, over all 256 exponent values (so it always holds 16 distinct entries); sign and
+ * mantissa are stored as one byte per element, (sign << 7) | mantissa; the 4-bit code of
+ * element i sits in byte i/2, low nibble for even i; an escaped element carries code 0; escapes
+ * are listed in ascending position.
+ * ------------------------------------------------------------------------------------- */
+void or_splitzip_codebook(int64_t n, const uint16_t *x, uint8_t *codebook) {
+    int64_t count[256];
+    for (int e = 0; e < 256; ++e) count[e] = 0;
+    for (int64_t i = 0; i < n; ++i) ++count[(x[i] >> 7) & 0xFF];
+    int taken[256];
+    for (int e = 0; e < 256; ++e) taken[e] = 0;
+    for (int k = 0; k < 16; ++k) {
+        int best = -1;
+        for (int e = 0; e < 256; ++e) {
+            if (taken[e]) continue;
+            if (best < 0 || count[e] > count[best]) best = e;  /* ties keep the smaller exponent */
+        }
+        taken[best] = 1;
+        codebook[k] = (uint8_t)best;
+    }
+}
+
+int64_t or_splitzip_encode(int64_t n, const uint16_t *x, const uint8_t *codebook, uint8_t *sm,
+                           uint8_t *codes, int64_t *esc_pos, uint8_t *esc_exp) {
+    int64_t n_esc = 0;
+    for (int64_t i = 0; i < (n + 1) / 2; ++i) codes[i] = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        int sign = (x[i] >> 15) & 1, e = (x[i] >> 7) & 0xFF, m = x[i] & 0x7F;
+        sm[i] = (uint8_t)((sign << 7) | m);
+        int code = -1;
+        for (int k = 0; k < 16; ++k)
+            if (codebook[k] == e) code = k;
+        if (code < 0) {
+            esc_pos[n_esc] = i;
+            esc_exp[n_esc] = (uint8_t)e;
+            ++n_esc;
+            code = 0;
+        }
+        codes[i / 2] |= (uint8_t)(code << (4 * (i % 2)));
+    }
+    return n_esc;
+}
+
+void or_splitzip_decode(int64_t n, const uint8_t *codebook, const uint8_t *sm, const uint8_t *codes,
+                        int64_t n_esc, const int64_t *esc_pos, const uint8_t *esc_exp, uint16_t *x) {
+    for (int64_t i = 0; i < n; ++i) {
+        int code = (codes[i / 2] >> (4 * (i % 2))) & 0xF;
+        int e = codebook[code];
+        x[i] = (uint16_t)(((sm[i] >> 7) << 15) | (e << 7) | (sm[i] & 0x7F));
+    }
+    for (int64_t j = 0; j < n_esc; ++j) {
+        int64_t i = esc_pos[j];
+        x[i] = (uint16_t)((x[i] & 0x807F) | (esc_exp[j] << 7));
+    }
+}

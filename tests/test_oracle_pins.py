@@ -572,3 +572,50 @@ def test_tier_step_keeps_recent_fast_and_older_slow():
         assert sorted(fast.values()) == list(range(n - f, n))
         assert all(s_ == p % cap for s_, p in fast.items())
         assert slow == list(range(n - f))
+
+
+# ---------------------------------------------------------------------------------------
+# SplitZip codec: hand-worked streams, lossless round trip, codebook and escapes by brute force.
+# ---------------------------------------------------------------------------------------
+
+def _bf16_specials(rng, n):
+    x = rng.integers(0, 1 << 16, n).astype(np.uint16)               # any bit pattern
+    special = np.array([0x0000, 0x8000, 0x7F80, 0xFF80, 0x7FC0, 0xFFC1, 0x0001, 0x807F,
+                        0x3F80, 0x7F7F], np.uint16)
+    x[rng.integers(0, n, min(n, 40))] = rng.choice(special, min(n, 40))
+    return x
+
+
+def test_splitzip_golden():
+    for c in gold("splitzip.json")["cases"]:
+        x = np.array(c["x"], np.uint16)
+        cb, sm, codes, pos, exp = oracle.splitzip_encode(x)
+        assert cb[:len(c["codebook_head"])].tolist() == c["codebook_head"], c["work"]
+        assert sm.tolist() == c["sm"] and codes.tolist() == c["codes"], c["work"]
+        assert pos.tolist() == c["esc_pos"] and exp.tolist() == c["esc_exp"], c["work"]
+        np.testing.assert_array_equal(oracle.splitzip_decode(x.size, cb, sm, codes, pos, exp), x)
+
+
+@pytest.mark.parametrize("n", [0, 1, 2, 7, 1000, 65537])
+def test_splitzip_round_trip_is_lossless(n):
+    rng = np.random.default_rng(47 + n)
+    for x in (_bf16_specials(rng, n), bf16(rng.normal(size=n) * 3) if n else np.zeros(0, np.uint16)):
+        cb, sm, codes, pos, exp = oracle.splitzip_encode(x)
+        np.testing.assert_array_equal(oracle.splitzip_decode(x.size, cb, sm, codes, pos, exp), x)
+
+
+def test_splitzip_codebook_and_escapes_by_brute_force():
+    rng = np.random.default_rng(48)
+    for x in (bf16(rng.normal(size=5000)), _bf16_specials(rng, 3000), bf16(rng.standard_cauchy(4000))):
+        cb, sm, codes, pos, exp = oracle.splitzip_encode(x)
+        e = (x >> 7) & 0xFF
+        counts = np.bincount(e, minlength=256)
+        order = np.lexsort((np.arange(256), -counts))               # count desc, exponent asc
+        np.testing.assert_array_equal(cb, order[:16])
+        esc = np.flatnonzero(~np.isin(e, cb))
+        np.testing.assert_array_equal(pos, esc)
+        np.testing.assert_array_equal(exp, e[esc])
+        assert (sm == (((x >> 15) << 7) | (x & 0x7F))).all()
+        # normal data: the top 16 exponents cover almost everything (the page's premise)
+    xn = bf16(rng.normal(size=100000))
+    assert oracle.splitzip_encode(xn)[3].size < 0.01 * xn.size

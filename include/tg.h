@@ -452,6 +452,39 @@ int tg_tiered_append(const tg_shape *shape, const void *k_new, const void *v_new
                      const int32_t *head_slow_cap, int32_t *head_kv_len, int32_t *head_fast_len,
                      int32_t *moved_out, int32_t *slot_out, tg_stream stream);
 
+/* =====================================================================================
+ * SplitZip: lossless BF16 codec for KV transfer ("SplitZip" explainer, arXiv 2605.01708, "Die
+ * SplitZip-Strategie", "Warum es schnell ist"). A bf16 value is sign, 8-bit exponent and 7-bit
+ * mantissa; the 16 most frequent exponents get 4-bit codes, two per byte; rare exponents go to
+ * an escape stream (position, exponent) applied as overwrites on decode. Stream layout:
+ *   codebook uint8[16]: exponents by count descending, ties by exponent ascending (over all
+ *            256, so always 16 distinct entries);
+ *   sm       uint8[n]: (sign << 7) | mantissa;  (16-byte aligned)
+ *   codes    uint8[(n+1)/2]: element i's code in byte i/2, low nibble for even i; an escaped
+ *            element carries code 0;  (8-byte aligned)
+ *   esc_pos  int64[esc_cap], esc_exp uint8[esc_cap]: escapes in ascending position; n_esc (one
+ *            device int64) their number — if it exceeds esc_cap the stream is incomplete.
+ * All pointers device; calls are stream-ordered and allocate nothing.
+ * ===================================================================================== */
+
+/* Bytes of device workspace tg_splitzip_encode needs for n elements: about n/8 + 12 KB. The
+ * workspace must be 256-byte aligned. Returns -1 for n < 0. */
+int64_t tg_splitzip_workspace_bytes(int64_t n);
+
+/* Encode n bf16 values (src, 16-byte aligned). Kernels: exponent histogram, codebook, a
+ * 4096-element tile per CTA writing sm and codes (and, in tiles that hold escapes, which
+ * elements escape), and one escape pass that places each tile's escapes at its offset.
+ * Errors: TG_EINVAL for negative sizes, null or misaligned pointers; TG_ECUDA on a launch
+ * failure (tg_last_cuda_error() has the text). */
+int tg_splitzip_encode(int64_t n, const void *src, uint8_t *codebook, uint8_t *sm,
+                       uint8_t *codes, int64_t *esc_pos, uint8_t *esc_exp, int64_t esc_cap,
+                       int64_t *n_esc, void *workspace, tg_stream stream);
+
+/* Decode into dst (bf16 [n], 16-byte aligned): codes through the codebook, then the escapes. */
+int tg_splitzip_decode(int64_t n, const uint8_t *codebook, const uint8_t *sm,
+                       const uint8_t *codes, const int64_t *esc_pos, const uint8_t *esc_exp,
+                       const int64_t *n_esc, int64_t esc_cap, void *dst, tg_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -113,6 +113,9 @@ _SIGS = [
     ("tg_plan_cascade_units", ctypes.c_int, [_P, _P]),
     ("tg_tiered_append", ctypes.c_int, [ctypes.POINTER(tg_shape), _P, _P, _P, _P, _P, _P, _P, _P,
                                         _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    ("tg_splitzip_workspace_bytes", _I64, [_I64]),
+    ("tg_splitzip_encode", ctypes.c_int, [_I64, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _P]),
+    ("tg_splitzip_decode", ctypes.c_int, [_I64, _P, _P, _P, _P, _P, _P, _I64, _P, _P]),
 ]
 
 #: Symbols the C ABI exports (include/tg.h).
@@ -494,3 +497,27 @@ def tg_quantize_int8(src, codes, scale, stream=None):
     n_rows = src.numel() // D
     _check(_lib().tg_quantize_int8(n_rows, D, _dp(src), _dp(codes), _dp(scale), _stream(stream)),
            "tg_quantize_int8")
+
+
+# ---------------------------------------------------------------------------------------
+# SplitZip codec (see include/tg.h).
+# ---------------------------------------------------------------------------------------
+
+def tg_splitzip_workspace_bytes(n: int) -> int:
+    return int(_lib().tg_splitzip_workspace_bytes(int(n)))
+
+
+def tg_splitzip_encode(n: int, src, codebook, sm, codes, esc_pos, esc_exp, n_esc, workspace,
+                       stream=None):
+    """Encode n bf16 values of src (device); esc_cap = esc_pos.numel()."""
+    cap = 0 if esc_pos is None else esc_pos.numel()
+    _check(_lib().tg_splitzip_encode(int(n), _dp(src), _dp(codebook), _dp(sm), _dp(codes),
+                                     _dp(esc_pos), _dp(esc_exp), cap, _dp(n_esc),
+                                     _dp(workspace), _stream(stream)), "tg_splitzip_encode")
+
+
+def tg_splitzip_decode(n: int, codebook, sm, codes, esc_pos, esc_exp, n_esc, dst, stream=None):
+    cap = 0 if esc_pos is None else esc_pos.numel()
+    _check(_lib().tg_splitzip_decode(int(n), _dp(codebook), _dp(sm), _dp(codes), _dp(esc_pos),
+                                     _dp(esc_exp), _dp(n_esc), cap, _dp(dst), _stream(stream)),
+           "tg_splitzip_decode")

@@ -356,6 +356,52 @@ int tg_tiered_decode(tg_plan *plan, const void *q, const int8_t *k_q8, const int
                      const int32_t *head_kv_len, const int32_t *head_fast_len, float scale,
                      void *out, float *lse, tg_stream stream);
 
+/* =====================================================================================
+ * Host-buffer decode pipeline (no counterpart on the pages: the decode step as a serving loop
+ * calls it, queries arriving in and outputs leaving through host memory). A pipe owns two
+ * device staging sets (q, out, lse of a plan's shape) and two copy streams (host->device,
+ * device->host). Call i uses set i % 2: its input copy waits until call i-2's decode has read
+ * that set; its decode runs on `stream` after that copy and after call i-2's output copy; its
+ * output copy follows its decode. So the copies of neighbouring calls overlap this call's
+ * decode, and calls return at once. Host buffers must be page-locked (cudaHostAlloc or
+ * cudaHostRegister; pageable memory makes the copies synchronous); q_host must stay unchanged
+ * and out_host / lse_host unread until tg_host_pipe_wait (or a tg_host_pipe_join'd stream)
+ * says the call is done.
+ * ===================================================================================== */
+typedef struct tg_host_pipe tg_host_pipe;
+
+/* Create a pipe for calls on plans of `plan`'s shape (B, Hq, D) and device. Allocates
+ * 2 x (2 B*Hq*D*2 + B*Hq*4) bytes of device memory, two streams and six events.
+ * TG_EINVAL for a host-only plan; TG_ENOMEM; TG_ECUDA. */
+int tg_host_pipe_create(const tg_plan *plan, tg_host_pipe **out);
+/* Wait for the pipe's copies, then free it. NULL is ignored. */
+void tg_host_pipe_destroy(tg_host_pipe *p);
+/* Block the host until every copy issued on the pipe has finished (all out / lse delivered). */
+int tg_host_pipe_wait(tg_host_pipe *p);
+/* Device-side ordering with another stream: tg_host_pipe_after makes the pipe's copy streams
+ * wait for the work queued on `stream` so far; tg_host_pipe_join makes `stream` wait for every
+ * copy issued on the pipe so far (e.g. to bracket a run of calls between two events). */
+int tg_host_pipe_after(tg_host_pipe *p, tg_stream stream);
+int tg_host_pipe_join(tg_host_pipe *p, tg_stream stream);
+
+/* tg_ragged_paged_decode / tg_tiered_decode with q_host (bf16 [B][Hq][D]) read from host
+ * memory and out_host (bf16 [B][Hq][D]) / lse_host (fp32 [B][Hq]) written to host memory
+ * through the pipe; every other argument as in those calls. TG_EINVAL if the plan's shape or
+ * device differs from the pipe's or a host pointer is NULL; otherwise the decode call's
+ * status. */
+int tg_ragged_paged_decode_host(tg_host_pipe *p, tg_plan *plan, const void *q_host,
+                                const void *k_pages, const void *v_pages,
+                                const int32_t *page_table, const int64_t *head_page_off,
+                                const int32_t *head_kv_len, const int32_t *group_of_head,
+                                float scale, void *out_host, float *lse_host, tg_stream stream);
+int tg_tiered_decode_host(tg_host_pipe *p, tg_plan *plan, const void *q_host,
+                          const int8_t *k_q8, const int8_t *v_q8, const float *k_scale,
+                          const float *v_scale, const int32_t *slow_page_table,
+                          const int64_t *slow_head_off, const void *k_fast, const void *v_fast,
+                          const int32_t *fast_page_table, const int64_t *fast_head_off,
+                          const int32_t *head_kv_len, const int32_t *head_fast_len, float scale,
+                          void *out_host, float *lse_host, tg_stream stream);
+
 /* Log-sum-exp merge of split results (CAP §2.4.3 online normaliser; Fig. 5 Dist Attention):
  * for each of n_rows rows, its splits j = row_split_off[r] .. row_split_off[r+1]-1 hold a
  * normalised partial part_o[j][D] (fp32) and part_lse[j] (fp32, natural log):

@@ -116,6 +116,15 @@ _SIGS = [
     ("tg_splitzip_workspace_bytes", _I64, [_I64]),
     ("tg_splitzip_encode", ctypes.c_int, [_I64, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _P]),
     ("tg_splitzip_decode", ctypes.c_int, [_I64, _P, _P, _P, _P, _P, _P, _I64, _P, _P]),
+    ("tg_host_pipe_create", ctypes.c_int, [_P, ctypes.POINTER(_P)]),
+    ("tg_host_pipe_destroy", None, [_P]),
+    ("tg_host_pipe_wait", ctypes.c_int, [_P]),
+    ("tg_host_pipe_after", ctypes.c_int, [_P, _P]),
+    ("tg_host_pipe_join", ctypes.c_int, [_P, _P]),
+    ("tg_ragged_paged_decode_host", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _F32, _P,
+                                                   _P, _P]),
+    ("tg_tiered_decode_host", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                             _P, _P, _F32, _P, _P, _P]),
 ]
 
 #: Symbols the C ABI exports (include/tg.h).
@@ -483,6 +492,78 @@ def tg_tiered_decode(plan: Plan, q, k_q8, v_q8, k_scale, v_scale, slow_page_tabl
         _dp(slow_page_table), _dp(slow_head_off), _dp(k_fast), _dp(v_fast),
         _dp(fast_page_table), _dp(fast_head_off), _dp(head_kv_len), _dp(head_fast_len),
         float(scale), _dp(out), _dp(lse), _stream(stream)), "tg_tiered_decode")
+
+
+# ------------------------------------------------------------------------------------------
+# Host-buffer decode pipeline
+# ------------------------------------------------------------------------------------------
+
+def _hostp(t):
+    """Host pointer of a page-locked CPU tensor."""
+    if t is None or getattr(t, "is_cuda", True):
+        raise ValueError("expected a CPU tensor for a host argument")
+    if not t.is_pinned():
+        raise ValueError("host buffers of the pipe must be page-locked (pin_memory())")
+    if not t.is_contiguous():
+        raise ValueError("host buffers must be contiguous")
+    return t.data_ptr()
+
+
+class HostPipe:
+    """Owns a tg_host_pipe handle (two device staging sets, two copy streams)."""
+
+    def __init__(self, plan: Plan):
+        h = ctypes.c_void_p()
+        _check(_lib().tg_host_pipe_create(plan.handle, ctypes.byref(h)), "tg_host_pipe_create")
+        self.handle = h
+
+    def wait(self):
+        _check(_lib().tg_host_pipe_wait(self.handle), "tg_host_pipe_wait")
+
+    def after(self, stream=None):
+        _check(_lib().tg_host_pipe_after(self.handle, _stream(stream)), "tg_host_pipe_after")
+
+    def join(self, stream=None):
+        _check(_lib().tg_host_pipe_join(self.handle, _stream(stream)), "tg_host_pipe_join")
+
+    def destroy(self):
+        if self.handle:
+            _lib().tg_host_pipe_destroy(self.handle)
+            self.handle = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def tg_host_pipe_create(plan: Plan) -> HostPipe:
+    return HostPipe(plan)
+
+
+def tg_ragged_paged_decode_host(pipe: HostPipe, plan: Plan, q_host, k_pages, v_pages, page_table,
+                                head_page_off, head_kv_len, group_of_head, scale: float,
+                                out_host, lse_host, stream=None):
+    """tg_ragged_paged_decode with q read from, and out / lse written to, pinned host tensors
+    (asynchronous: read the outputs after pipe.wait())."""
+    _check(_lib().tg_ragged_paged_decode_host(
+        pipe.handle, plan.handle, _hostp(q_host), _dp(k_pages), _dp(v_pages), _dp(page_table),
+        _dp(head_page_off), _dp(head_kv_len), _dp(group_of_head), float(scale),
+        _hostp(out_host), _hostp(lse_host), _stream(stream)), "tg_ragged_paged_decode_host")
+
+
+def tg_tiered_decode_host(pipe: HostPipe, plan: Plan, q_host, k_q8, v_q8, k_scale, v_scale,
+                          slow_page_table, slow_head_off, k_fast, v_fast, fast_page_table,
+                          fast_head_off, head_kv_len, head_fast_len, scale: float, out_host,
+                          lse_host, stream=None):
+    """tg_tiered_decode with pinned host q / out / lse (see tg_ragged_paged_decode_host)."""
+    _check(_lib().tg_tiered_decode_host(
+        pipe.handle, plan.handle, _hostp(q_host), _dp(k_q8), _dp(v_q8), _dp(k_scale),
+        _dp(v_scale), _dp(slow_page_table), _dp(slow_head_off), _dp(k_fast), _dp(v_fast),
+        _dp(fast_page_table), _dp(fast_head_off), _dp(head_kv_len), _dp(head_fast_len),
+        float(scale), _hostp(out_host), _hostp(lse_host), _stream(stream)),
+        "tg_tiered_decode_host")
 
 
 def tg_lse_merge(row_split_off, part_o, part_lse, out, lse, stream=None):

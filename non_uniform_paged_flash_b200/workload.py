@@ -178,6 +178,20 @@ class DeviceBatch:
                              self.out, self.lse, stream)
 
 
+    def run_host(self, pipe, q_host, out_host, lse_host, stream=None):
+        """One decode step through the host-buffer pipe (pinned q in, out / lse back)."""
+        from . import tg_ragged_paged_decode_host, tg_tiered_decode_host
+        if self.lay.fast_len is None:
+            tg_ragged_paged_decode_host(pipe, self.plan, q_host, self.k, self.v, self.table,
+                                        self.head_off, self.kv_len, self.group_of_head,
+                                        self.spec.scale, out_host, lse_host, stream)
+        else:
+            tg_tiered_decode_host(pipe, self.plan, q_host, self.k_q8, self.v_q8, self.k_scale,
+                                  self.v_scale, self.slow_table, self.slow_off, self.k, self.v,
+                                  self.table, self.head_off, self.kv_len, self.fast_len,
+                                  self.spec.scale, out_host, lse_host, stream)
+
+
 def _bf16_tensor(bits: np.ndarray, device):
     import torch
     return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)

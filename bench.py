@@ -460,6 +460,8 @@ def run_ours(args):
             "device_status": "ok" if not bad else "error word set",
             "clocks": clocks,
         }
+        if world == 1 and cfg == 1:
+            line["graph_replay"] = graph_replay(db, alg)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg)
         print(json.dumps(line), flush=True)
@@ -467,6 +469,57 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def graph_replay(db, alg, copies=1024, reps=5):
+    """The tiny ragged MHA step is launch-bound and L2-resident on its own. Here `copies`
+    distinct copies of its inputs (q, K and V pools, outputs; together above L2) are decoded by
+    one CUDA graph of `copies` decode calls on the same plan, replayed `reps` times; the
+    figure is K/V bytes of all copies / replay time."""
+    import torch
+    import non_uniform_paged_flash_b200 as tg
+    dev = db.q.device
+    k = db.k.unsqueeze(0).repeat(copies, *([1] * db.k.dim()))
+    v = db.v.unsqueeze(0).repeat(copies, *([1] * db.v.dim()))
+    q = db.q.unsqueeze(0).repeat(copies, *([1] * db.q.dim()))
+    out = torch.empty((copies,) + tuple(db.out.shape), dtype=db.out.dtype, device=dev)
+    lse = torch.empty((copies,) + tuple(db.lse.shape), dtype=db.lse.dtype, device=dev)
+    held = (k.numel() + v.numel() + q.numel() + out.numel()) * 2 + lse.numel() * 4
+    s = torch.cuda.Stream(device=dev)
+
+    def calls():
+        for i in range(copies):
+            tg.tg_ragged_paged_decode(db.plan, q[i], k[i], v[i], db.table, db.head_off, db.kv_len,
+                                      db.group_of_head, db.spec.scale, out[i], lse[i], s)
+    try:
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            calls()
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            calls()
+        for _ in range(2):
+            g.replay()
+        s.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for _ in range(reps):
+                g.replay()
+            e1.record(s)
+        s.synchronize()
+        ms = e0.elapsed_time(e1) / (reps * copies)
+        db.run()
+        torch.cuda.synchronize()
+        same = bool(torch.equal(out[0], db.out) and torch.equal(out[copies - 1], db.out))
+        del g
+    except Exception as e:   # reported, never silently replaced by another number
+        return {"error": str(e).splitlines()[0][:200]}
+    return {"copies": copies, "replays": reps, "bytes_held": int(held),
+            "us_per_step": ms * 1e3, "kv_gbs": alg["kv"] / (ms * 1e-3) / 1e9,
+            "launches_per_step": 1 + (1 if tg.tg_plan_get_info(db.plan)["n_merge"] > 0 else 0),
+            "outputs_equal_single_call": same}
 
 
 def run_write_path(args):
@@ -692,6 +745,81 @@ def run_tier_path(args):
     return 0
 
 
+def run_tier_host(args):
+    """Tiered decode step with the INT8 tier in page-locked host memory (config 5 shape),
+    streamed block-wise into an HBM ring while earlier blocks are decoded (TTKV's DRAM slow
+    tier). The bound is the host link: the figure is INT8-tier bytes per step / step time,
+    against a plain pinned host-to-device copy of the same size measured in the same run.
+    Prints one JSON line."""
+    import torch
+    import non_uniform_paged_flash_b200 as tg
+    from non_uniform_paged_flash_b200 import workload
+
+    cfg = 5
+    sp = synth.preset(cfg)
+    lay = workload.layout(sp, 0)
+    kw = _plan_kw(cfg)
+    db = workload.to_device(sp, lay, 0, **kw)
+    stream = torch.cuda.current_stream()
+    db.run(stream)
+    torch.cuda.synchronize()
+    ref_out, ref_lse = db.out.clone(), db.lse.clone()
+    host = db.host_slow_tier()
+    slow_bytes = sum(t.numel() * t.element_size() for t in host)
+    block_pages = args.block_pages
+    ss = db.slow_stream(block_pages, 3, **{k: v for k, v in kw.items() if k != "early_prologue"})
+    n_blocks = len(ss.blocks()[0])
+    for _ in range(args.warmup):
+        db.run_streamed(ss, host, stream)
+    torch.cuda.synchronize()
+    assert ss.status() == tg.TG_OK
+    e_out = (db.out.float() - ref_out.float()).abs().max().item()
+    e_lse = (db.lse - ref_lse).abs().max().item()
+    # the host link alone: one pinned copy of the same bytes
+    dst = torch.empty(slow_bytes, dtype=torch.uint8, device=db.q.device)
+    src = torch.empty(slow_bytes, dtype=torch.uint8).pin_memory()
+    link = []
+    for _ in range(3):
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        dst.copy_(src, non_blocking=True)
+        b_.record(stream)
+        torch.cuda.synchronize()
+        link.append(slow_bytes / (a_.elapsed_time(b_) * 1e-3) / 1e9)
+    del dst, src
+    reps = max(1, min(args.steps, 20))
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        db.run_streamed(ss, host, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / reps
+    peak_link = max(link)
+    achieved = slow_bytes / (ms * 1e-3) / 1e9
+    alg = workload.algorithmic_bytes(sp, lay)
+    line = {
+        "metric": "tiered decode step, INT8 tier streamed from host memory (GB/s of INT8 tier)",
+        "value": achieved, "unit": "GB/s", "higher_is_better": True, "n_gpus": 1, "steps": reps,
+        "warmup": args.warmup, "ms_per_step": ms, "dtype": "bf16+int8", "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAMES[cfg] + "; INT8 tier in pinned host memory",
+                   "block_pages": block_pages, "ring_blocks": 3, "blocks_per_step": n_blocks},
+        "host_tier_bytes_per_step": slow_bytes, "kv_bytes_per_step": int(alg["kv"]),
+        "roofline": {"bound": "host link", "achieved": achieved, "peak": peak_link,
+                     "unit": "GB/s", "frac": achieved / peak_link,
+                     "peak_kind": "pinned host-to-device copy of the same bytes, this run"},
+        "vs_hbm_tiered_step": {"max_abs_out": e_out, "max_abs_lse": e_lse},
+        "gpu_launches": reps * (n_blocks * 2 + 3), "vs_baseline": None, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    ss.destroy()
+    return 0
+
+
 def run_splitzip(args):
     """SplitZip codec throughput on one GPU: the K and V pools of the GQA decode workload
     (config 2 shape, bf16) encoded and decoded back, each timed with CUDA events over
@@ -769,10 +897,14 @@ def main():
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", default="decode", choices=["decode", "sink", "h2o", "ttkv", "splitzip"],
+    ap.add_argument("--block-pages", type=int, default=8192,
+                    help="--path ttkv-host: INT8-tier pages per streamed block")
+    ap.add_argument("--path", default="decode",
+                    choices=["decode", "sink", "h2o", "ttkv", "ttkv-host", "splitzip"],
                     help="decode: the decode step (default); sink / h2o: the decode step with "
                          "the write path; ttkv: the tiered step with tier migration (config 5); "
-                         "one GPU, separate JSON line")
+                         "ttkv-host: the tiered step with the INT8 tier streamed from host "
+                         "memory (config 5); splitzip: the KV codec; one GPU, separate JSON line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -780,6 +912,8 @@ def main():
         return run_reference(args)
     if args.path == "splitzip":
         return run_splitzip(args)
+    if args.path == "ttkv-host":
+        return run_tier_host(args)
     if args.path != "decode":
         return run_write_path(args)
     return run_ours(args)

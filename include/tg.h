@@ -182,6 +182,9 @@ typedef struct tg_plan_opts {
                                  TG_EBADPAGE) and skips reserved pages that hold no token yet,
                                  so appends (tg_tiered_append) never need a new plan. 0: the
                                  lengths are exact, as for bf16 plans */
+    int32_t out_f32;          /* 1: the decode calls' out is fp32 [B][Hq][D] (the normalised
+                                 output before bf16 rounding, e.g. a partial result to be merged
+                                 with others by tg_lse_merge); 0 (default): bf16 */
 } tg_plan_opts;
 
 /* Build a plan. kv_len[B*Hkv] (host): retained tokens per (sequence, KV head); the decode
@@ -401,6 +404,58 @@ int tg_tiered_decode_host(tg_host_pipe *p, tg_plan *plan, const void *q_host,
                           const int32_t *fast_page_table, const int64_t *fast_head_off,
                           const int32_t *head_kv_len, const int32_t *head_fast_len, float scale,
                           void *out_host, float *lse_host, tg_stream stream);
+
+/* =====================================================================================
+ * TTKV slow tier in host memory, streamed block-wise ("TTKV" 核心方法 1 Tier Layout: the slow
+ * tier in DRAM, the fast tier in HBM; 3 Tier Interaction: Block-wise Streaming Attention, the
+ * DRAM data fetched in blocks with the fetch overlapping the computation). The INT8 pool (codes
+ * int8 [num_slow_pages][16][D] for K and V, scales fp32 [num_slow_pages][16]) stays in
+ * page-locked host memory. Its pages are cut into blocks of block_pages consecutive page ids;
+ * each block that holds a retained token is copied per step into one of ring_blocks HBM slots
+ * (copy stream) and decoded when it lands (compute stream) while the next block copies. Each
+ * block and the bf16 fast tier give an fp32 partial per query row; one merge kernel combines
+ * them by log-sum-exp (fast tier first, then blocks in page order). Results equal
+ * tg_tiered_decode's up to rounding.
+ * ===================================================================================== */
+typedef struct tg_slow_stream tg_slow_stream;
+
+/* Build the per-block tables and plans (host) and, unless opts->host_only, the device state:
+ * the ring (ring_blocks x block_pages pages of codes and scales), the block tables, partials
+ * fp32 [1 + blocks][B*Hq][D + 1], a copy stream and 2 x ring_blocks events. Arguments as
+ * tg_plan_create for a tiered plan (kv_len, fast_len, group_of_head, group_off, n_groups over
+ * the fast tier's group tables) plus the INT8 tier's HOST table (slow_page_table int32
+ * [slow_table_len], slow_head_off int64 [B*Hkv]); shape->num_slow_pages = pages of the host pool.
+ * opts as for tg_plan_create (out_f32 and capacity are set by the stream). TG_EINVAL on a bad
+ * argument or a page id outside the pool. */
+int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,
+                          const int32_t *group_of_head, const int64_t *group_off,
+                          int32_t n_groups, const int32_t *slow_page_table,
+                          const int64_t *slow_head_off, int64_t slow_table_len,
+                          int32_t block_pages, int32_t ring_blocks, const tg_plan_opts *opts,
+                          tg_slow_stream **out);
+/* Wait for the stream's copies, then free it. NULL is ignored. */
+void tg_slow_stream_destroy(tg_slow_stream *s);
+/* Inspection: returns the number of streamed blocks J (blocks with no retained token are
+ * skipped) and, for non-NULL arrays, each block's first page id (int64 [J]), its page count
+ * (int32 [J]) and the tokens of every (sequence, KV head) in it (int32 [J][B*Hkv]). */
+int tg_slow_stream_blocks(const tg_slow_stream *s, int64_t *first_page, int32_t *pages,
+                          int32_t *tokens);
+/* The worst device status over the stream's plans (as tg_plan_status; synchronises). */
+int tg_slow_stream_status(tg_slow_stream *s, tg_stream stream);
+
+/* One tiered decode step with the INT8 tier read from page-locked HOST memory (k_q8_host,
+ * v_q8_host, k_scale_host, v_scale_host; pageable memory is rejected with TG_EINVAL). q, the
+ * fast tier (k_fast, v_fast bf16 pools, fast_page_table, fast_head_off, group_of_head) and
+ * out (bf16 [B][Hq][D]) / lse (fp32 [B][Hq]) are device buffers, as for tg_tiered_decode; the
+ * lengths are the ones given to tg_slow_stream_create. Stream-ordered: the copies start after
+ * the work already queued on `stream`, and out / lse are complete when `stream` reaches the
+ * end of the call. */
+int tg_tiered_decode_streamed(tg_slow_stream *s, const void *q, const int8_t *k_q8_host,
+                              const int8_t *v_q8_host, const float *k_scale_host,
+                              const float *v_scale_host, const void *k_fast, const void *v_fast,
+                              const int32_t *fast_page_table, const int64_t *fast_head_off,
+                              const int32_t *group_of_head, float scale, void *out, float *lse,
+                              tg_stream stream);
 
 /* Log-sum-exp merge of split results (CAP §2.4.3 online normaliser; Fig. 5 Dist Attention):
  * for each of n_rows rows, its splits j = row_split_off[r] .. row_split_off[r+1]-1 hold a

@@ -46,7 +46,8 @@ class tg_plan_opts(ctypes.Structure):
                 ("device", ctypes.c_int32), ("static_permille", ctypes.c_int32),
                 ("dyn_chunk_pages", ctypes.c_int32), ("early_prologue", ctypes.c_int32),
                 ("wait_limit_us", ctypes.c_int32), ("test_withhold_page", ctypes.c_int32),
-                ("capacity", ctypes.c_int32)]
+                ("capacity", ctypes.c_int32),
+                ("out_f32", ctypes.c_int32)]
 
 
 class tg_plan_info(ctypes.Structure):
@@ -125,6 +126,14 @@ _SIGS = [
                                                    _P, _P]),
     ("tg_tiered_decode_host", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                              _P, _P, _F32, _P, _P, _P]),
+    ("tg_slow_stream_create", ctypes.c_int, [ctypes.POINTER(tg_shape), _P, _P, _P, _P, _I32, _P, _P,
+                                             _I64, _I32, _I32, ctypes.POINTER(tg_plan_opts),
+                                             ctypes.POINTER(_P)]),
+    ("tg_slow_stream_destroy", None, [_P]),
+    ("tg_slow_stream_blocks", ctypes.c_int, [_P, _P, _P, _P]),
+    ("tg_slow_stream_status", ctypes.c_int, [_P, _P]),
+    ("tg_tiered_decode_streamed", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F32,
+                                                 _P, _P, _P]),
 ]
 
 #: Symbols the C ABI exports (include/tg.h).
@@ -307,14 +316,15 @@ def tg_plan_create(shape: tg_shape, kv_len, group_of_head, group_off, fast_len=N
                    max_chunk_pages: int = 0, host_only: bool = False, device: int = -1,
                    static_permille: int = 0, dyn_chunk_pages: int = 0,
                    early_prologue: bool = False, wait_limit_us: int = 0,
-                   test_withhold_page: int = 0, capacity: bool = False) -> Plan:
+                   test_withhold_page: int = 0, capacity: bool = False,
+                   out_f32: bool = False) -> Plan:
     kv = _h(kv_len, np.int32).reshape(-1)
     fl = None if fast_len is None else _h(fast_len, np.int32).reshape(-1)
     goh = _h(group_of_head, np.int32).reshape(-1)
     goff = _h(group_off, np.int64).reshape(-1)
     opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
                         static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us,
-                        test_withhold_page, int(capacity))
+                        test_withhold_page, int(capacity), int(out_f32))
     h = ctypes.c_void_p()
     _check(_lib().tg_plan_create(ctypes.byref(shape), _hp(kv), _hp(fl), _hp(goh), _hp(goff),
                                  goff.size - 1, slow_table_len, ctypes.byref(opts),
@@ -326,7 +336,8 @@ def tg_plan_create_cascade(shape: tg_shape, kv_len, group_of_head, group_off, pa
                            head_page_off, min_readers: int = 2, num_workers: int = 0,
                            min_splits: int = 1, max_chunk_pages: int = 0, host_only: bool = False,
                            device: int = -1, static_permille: int = 0, dyn_chunk_pages: int = 0,
-                           early_prologue: bool = False, wait_limit_us: int = 0) -> Plan:
+                           early_prologue: bool = False, wait_limit_us: int = 0,
+                           out_f32: bool = False) -> Plan:
     """Prefix-aware cascade plan from the host page table (see include/tg.h)."""
     kv = _h(kv_len, np.int32).reshape(-1)
     goh = _h(group_of_head, np.int32).reshape(-1)
@@ -334,7 +345,8 @@ def tg_plan_create_cascade(shape: tg_shape, kv_len, group_of_head, group_off, pa
     tbl = _h(page_table, np.int32).reshape(-1)
     hoff = _h(head_page_off, np.int64).reshape(-1)
     opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
-                        static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us, 0, 0)
+                        static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us, 0, 0,
+                        int(out_f32))
     h = ctypes.c_void_p()
     _check(_lib().tg_plan_create_cascade(ctypes.byref(shape), _hp(kv), _hp(goh), _hp(goff),
                                          goff.size - 1, _hp(tbl), _hp(hoff), tbl.size,
@@ -564,6 +576,71 @@ def tg_tiered_decode_host(pipe: HostPipe, plan: Plan, q_host, k_q8, v_q8, k_scal
         _dp(fast_page_table), _dp(fast_head_off), _dp(head_kv_len), _dp(head_fast_len),
         float(scale), _hostp(out_host), _hostp(lse_host), _stream(stream)),
         "tg_tiered_decode_host")
+
+
+# ------------------------------------------------------------------------------------------
+# TTKV slow tier in host memory, streamed block-wise
+# ------------------------------------------------------------------------------------------
+
+class SlowStream:
+    """Owns a tg_slow_stream handle (per-block plans, HBM ring, copy stream)."""
+
+    def __init__(self, shape: tg_shape, kv_len, fast_len, group_of_head, group_off,
+                 slow_page_table, slow_head_off, block_pages: int, ring_blocks: int = 3,
+                 num_workers: int = 0, min_splits: int = 1, max_chunk_pages: int = 0,
+                 host_only: bool = False, device: int = -1, static_permille: int = 0,
+                 dyn_chunk_pages: int = 0, early_prologue: bool = False):
+        self.shape = shape
+        kv = _h(kv_len, np.int32).reshape(-1)
+        fl = _h(fast_len, np.int32).reshape(-1)
+        goh = _h(group_of_head, np.int32).reshape(-1)
+        goff = _h(group_off, np.int64).reshape(-1)
+        tbl = _h(slow_page_table, np.int32).reshape(-1)
+        off = _h(slow_head_off, np.int64).reshape(-1)
+        opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
+                            static_permille, dyn_chunk_pages, int(early_prologue), 0, 0, 0, 0)
+        h = ctypes.c_void_p()
+        _check(_lib().tg_slow_stream_create(ctypes.byref(shape), _hp(kv), _hp(fl), _hp(goh),
+                                            _hp(goff), goff.size - 1, _hp(tbl) if tbl.size else None,
+                                            _hp(off), tbl.size, int(block_pages), int(ring_blocks),
+                                            ctypes.byref(opts), ctypes.byref(h)),
+               "tg_slow_stream_create")
+        self.handle = h
+
+    def blocks(self):
+        """(first_page int64 [J], pages int32 [J], tokens int32 [J][B*Hkv])."""
+        J = _lib().tg_slow_stream_blocks(self.handle, None, None, None)
+        BH = self.shape.B * self.shape.Hkv
+        first = np.empty(J, np.int64)
+        pages = np.empty(J, np.int32)
+        tokens = np.empty((J, BH), np.int32)
+        _lib().tg_slow_stream_blocks(self.handle, _hp(first), _hp(pages), _hp(tokens))
+        return first, pages, tokens
+
+    def status(self, stream=None) -> int:
+        return _lib().tg_slow_stream_status(self.handle, _stream(stream))
+
+    def destroy(self):
+        if self.handle:
+            _lib().tg_slow_stream_destroy(self.handle)
+            self.handle = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def tg_tiered_decode_streamed(ss: SlowStream, q, k_q8_host, v_q8_host, k_scale_host,
+                              v_scale_host, k_fast, v_fast, fast_page_table, fast_head_off,
+                              group_of_head, scale: float, out, lse, stream=None):
+    """Tiered decode with the INT8 tier in pinned host memory, streamed block-wise."""
+    _check(_lib().tg_tiered_decode_streamed(
+        ss.handle, _dp(q), _hostp(k_q8_host), _hostp(v_q8_host), _hostp(k_scale_host),
+        _hostp(v_scale_host), _dp(k_fast), _dp(v_fast), _dp(fast_page_table), _dp(fast_head_off),
+        _dp(group_of_head), float(scale), _dp(out), _dp(lse), _stream(stream)),
+        "tg_tiered_decode_streamed")
 
 
 def tg_lse_merge(row_split_off, part_o, part_lse, out, lse, stream=None):

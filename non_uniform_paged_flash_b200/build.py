@@ -11,7 +11,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libtg.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("tg_host.cpp", "tg_pipe.cpp", "tg_kernels.cu", "tg_write.cu",
-                                               "tg_splitzip.cu")]
+                                               "tg_splitzip.cu", "tg_slowstream.cu")]
 HEADERS = [os.path.join(CSRC, "tg_internal.h"), os.path.join(INCLUDE, "tg.h")]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",

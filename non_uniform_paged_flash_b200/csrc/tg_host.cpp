@@ -604,6 +604,7 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
     p->withhold = o.test_withhold_page > 0 ? o.test_withhold_page : 0;
     if (o.capacity && !fast_len) { delete p; return TG_EINVAL; }
     p->capacity = o.capacity != 0;
+    p->out_f32 = o.out_f32 != 0;
 
     // Prefix cascade: shared runs per KV head, cut into units of kCascadeRows query rows.
     std::vector<int32_t> casc_cnt;

@@ -242,6 +242,7 @@ struct DecodeArgs {
     const int32_t *fast_len_dev;     // [B*Hkv] (tiered) or null
     int64_t num_pages, num_slow_pages;
     __nv_bfloat16 *out;              // [B][Hq][D]
+    float *out_f32;                  // [B][Hq][D] instead of out (plans with out_f32), else null
     float *lse;                      // [B][Hq]
     float *part_o;                   // [n_partials][G][D]
     float *part_lse;                 // [n_partials][G]
@@ -563,7 +564,10 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
             const int32_t b = bh / a.Hkv, h = bh - b * a.Hkv;
             const int64_t r = i % per;
             const int64_t row = static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * a.G + r / D;
-            a.out[row * D + r % D] = __float2bfloat16_rn(0.f);
+            if (a.out_f32)
+                a.out_f32[row * D + r % D] = 0.f;
+            else
+                a.out[row * D + r % D] = __float2bfloat16_rn(0.f);
             if (r % D == 0) a.lse[row] = -INFINITY;
         }
     }
@@ -1007,7 +1011,9 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
             const int32_t b = hd.bh / a.Hkv, h = hd.bh - b * a.Hkv;
             const int n0 = 2 * t, n1 = 2 * t + 1;
             if (hd.slot < 0) {
-                __nv_bfloat16 *ob = a.out + (static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * a.G) * D;
+                const int64_t obase = (static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * a.G) * D;
+                __nv_bfloat16 *ob = a.out_f32 ? nullptr : a.out + obase;
+                float *of = a.out_f32 ? a.out_f32 + obase : nullptr;
 #pragma unroll
                 for (int i = 0; i < KSTEPS; ++i) {
                     int dlo, dhi;
@@ -1018,13 +1024,24 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         dlo = 16 * i + 2 * g;
                         dhi = dlo + 1;
                     }
-                    if (n0 < a.G) {
-                        ob[n0 * D + dlo] = __float2bfloat16_rn(o[i][0] * inv0);
-                        ob[n0 * D + dhi] = __float2bfloat16_rn(o[i][2] * inv0);
-                    }
-                    if (n1 < a.G) {
-                        ob[n1 * D + dlo] = __float2bfloat16_rn(o[i][1] * inv1);
-                        ob[n1 * D + dhi] = __float2bfloat16_rn(o[i][3] * inv1);
+                    if (of) {
+                        if (n0 < a.G) {
+                            of[n0 * D + dlo] = o[i][0] * inv0;
+                            of[n0 * D + dhi] = o[i][2] * inv0;
+                        }
+                        if (n1 < a.G) {
+                            of[n1 * D + dlo] = o[i][1] * inv1;
+                            of[n1 * D + dhi] = o[i][3] * inv1;
+                        }
+                    } else {
+                        if (n0 < a.G) {
+                            ob[n0 * D + dlo] = __float2bfloat16_rn(o[i][0] * inv0);
+                            ob[n0 * D + dhi] = __float2bfloat16_rn(o[i][2] * inv0);
+                        }
+                        if (n1 < a.G) {
+                            ob[n1 * D + dlo] = __float2bfloat16_rn(o[i][1] * inv1);
+                            ob[n1 * D + dhi] = __float2bfloat16_rn(o[i][3] * inv1);
+                        }
                     }
                 }
                 if (g == 0) {
@@ -1519,7 +1536,8 @@ __global__ void __launch_bounds__(1024) split_merge_kernel(const MergeHead *mh, 
                                                            int32_t G, int32_t Hq, int32_t Hkv,
                                                            const float *part_o,
                                                            const float *part_lse,
-                                                           __nv_bfloat16 *out, float *lse) {
+                                                           __nv_bfloat16 *out, float *out_f32,
+                                                           float *lse) {
     constexpr int VEC = D / 32;
     constexpr int U = 4;
     extern __shared__ float s_dyn[];  // [nw] maxima, [nw] sums, [nw][D] sums of V (nw > 1)
@@ -1598,16 +1616,15 @@ __global__ void __launch_bounds__(1024) split_merge_kernel(const MergeHead *mh, 
         }
         m = M;
     }
-    if (m == -INFINITY) {
+    const float inv = m == -INFINITY ? 0.f : 1.f / sum;
 #pragma unroll
-        for (int c = 0; c < VEC; ++c) out[row * D + lane * VEC + c] = __float2bfloat16_rn(0.f);
-        if (lane == 0) lse[row] = -INFINITY;
-        return;
+    for (int c = 0; c < VEC; ++c) {
+        if (out_f32)
+            out_f32[row * D + lane * VEC + c] = acc[c] * inv;
+        else
+            out[row * D + lane * VEC + c] = __float2bfloat16_rn(acc[c] * inv);
     }
-    const float inv = 1.f / sum;
-#pragma unroll
-    for (int c = 0; c < VEC; ++c) out[row * D + lane * VEC + c] = __float2bfloat16_rn(acc[c] * inv);
-    if (lane == 0) lse[row] = m + logf(sum);
+    if (lane == 0) lse[row] = m == -INFINITY ? -INFINITY : m + logf(sum);
 }
 
 // Generic merge (exported as tg_lse_merge): rows with contiguous split ranges.
@@ -1918,13 +1935,14 @@ static int launch_merge(const tg_plan *p, const MergeHead *d_merge, const float 
     cfg.attrs = pdl ? attr : nullptr;
     cfg.numAttrs = pdl ? 1 : 0;
     const int32_t G = p->G, Hq = p->shape.Hq, Hkv = p->shape.Hkv;
-    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
+    __nv_bfloat16 *o = p->out_f32 ? nullptr : static_cast<__nv_bfloat16 *>(out);
+    float *of = p->out_f32 ? static_cast<float *>(out) : nullptr;
     if (p->shape.D == 128) {
-        if (rows) TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<128, true>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, lse));
-        else TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<128, false>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, lse));
+        if (rows) TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<128, true>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, of, lse));
+        else TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<128, false>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, of, lse));
     } else {
-        if (rows) TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<64, true>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, lse));
-        else TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<64, false>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, lse));
+        if (rows) TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<64, true>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, of, lse));
+        else TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<64, false>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, of, lse));
     }
     return TG_OK;
 }
@@ -1960,7 +1978,8 @@ static DecodeArgs base_args(const tg_plan *p, const void *q, const int32_t *kv, 
     a.kv_len_dev = kv;
     a.num_pages = p->shape.num_pages;
     a.num_slow_pages = p->shape.num_slow_pages;
-    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.out = p->out_f32 ? nullptr : static_cast<__nv_bfloat16 *>(out);
+    a.out_f32 = p->out_f32 ? static_cast<float *>(out) : nullptr;
     a.lse = lse;
     a.part_o = p->d_part_o;
     a.part_lse = p->d_part_lse;
@@ -2425,7 +2444,8 @@ extern "C" int tg_ragged_paged_decode_noalloc(tg_plan *p, const void *q, const v
         a.kv_len_dev = head_kv_len;
         a.num_pages = s.num_pages;
         a.num_slow_pages = s.num_slow_pages;
-        a.out = static_cast<__nv_bfloat16 *>(out);
+        a.out = p->out_f32 ? nullptr : static_cast<__nv_bfloat16 *>(out);
+        a.out_f32 = p->out_f32 ? static_cast<float *>(out) : nullptr;
         a.lse = lse;
         a.part_o = d_po;
         a.part_lse = d_pl;

@@ -192,6 +192,27 @@ class DeviceBatch:
                                   self.spec.scale, out_host, lse_host, stream)
 
 
+    def host_slow_tier(self):
+        """Page-locked host copies of the INT8 tier: (k codes, v codes, k scales, v scales)."""
+        return tuple(t.cpu().pin_memory() for t in (self.k_q8, self.v_q8, self.k_scale, self.v_scale))
+
+    def slow_stream(self, block_pages: int, ring_blocks: int = 3, **kw):
+        """A tg_slow_stream over this batch's tiers (the INT8 tier to be read from host)."""
+        from . import SlowStream
+        lay = self.lay
+        dev = self.q.device.index
+        return SlowStream(self.plan.shape, lay.kv_len, lay.fast_len, lay.group_of_head,
+                          lay.group_off, lay.slow_table if lay.slow_table.size else np.full(1, -1),
+                          lay.slow_off, block_pages, ring_blocks,
+                          device=dev if dev is not None else -1, **kw)
+
+    def run_streamed(self, ss, host, stream=None):
+        """One tiered step with the INT8 tier streamed from the pinned host copies `host`."""
+        from . import tg_tiered_decode_streamed
+        tg_tiered_decode_streamed(ss, self.q, *host, self.k, self.v, self.table, self.head_off,
+                                  self.group_of_head, self.spec.scale, self.out, self.lse, stream)
+
+
 def _bf16_tensor(bits: np.ndarray, device):
     import torch
     return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)

@@ -52,6 +52,8 @@ def _L():
         lib.or_tiered_decode.argtypes = [i32, i32, i32, i32, i32, p, p, p, p, p, i64, p, p,
                                          p, p, i64, p, p, p, p, f64, i64, p, p, p]
         lib.or_quantize_int8.argtypes = [i64, i32, p, p, p]
+        lib.or_quantize_int4.argtypes = [i64, i32, p, p, p]
+        lib.or_unpack_int4.argtypes = [i64, i32, p, p]
         lib.or_lse_merge.argtypes = [i32, i64, i32, p, p, p, p]
         lib.or_place_sequences.argtypes = [i32, p, i32, p]
         lib.or_sink_recent_slot.argtypes = [i32, i32, i32, p]
@@ -210,6 +212,31 @@ def quantize_int8(src_bits):
     scale = np.empty(a.shape[:-1], dtype=np.float32)
     _L().or_quantize_int8(rows, D, _ptr(a), _ptr(codes), _ptr(scale))
     return codes, scale
+
+
+def quantize_int4(src_bits):
+    """Per-row symmetric absmax INT4 of bf16 rows, packed two codes per byte (byte i: d = i low
+    nibble, d = i + D/2 high nibble, offset-binary code + 8). src uint16[..., D] ->
+    (packed uint8[..., D/2], scale float32[...])."""
+    a = _c(src_bits, np.uint16)
+    D = a.shape[-1]
+    if D % 2:
+        raise ValueError("INT4 rows need an even D")
+    rows = a.size // D
+    packed = np.empty(a.shape[:-1] + (D // 2,), dtype=np.uint8)
+    scale = np.empty(a.shape[:-1], dtype=np.float32)
+    _L().or_quantize_int4(rows, D, _ptr(a), _ptr(packed), _ptr(scale))
+    return packed, scale
+
+
+def unpack_int4(packed):
+    """Codes int8[..., D] of packed INT4 rows uint8[..., D/2]."""
+    a = _c(packed, np.uint8)
+    D = 2 * a.shape[-1]
+    rows = a.size // (D // 2)
+    codes = np.empty(a.shape[:-1] + (D,), dtype=np.int8)
+    _L().or_unpack_int4(rows, D, _ptr(a), _ptr(codes))
+    return codes
 
 
 def lse_merge(parts_o, parts_lse):

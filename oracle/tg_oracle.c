@@ -423,6 +423,48 @@ void or_quantize_int8(int64_t rows, int32_t D, const uint16_t *src, int8_t *code
 }
 
 /* ---------------------------------------------------------------------------------------
+ * Slow-tier INT4 quantisation. [TTKV] 核心方法 1 Tier Layout names INT8/INT4 for the slow
+ * tier and leaves the scheme open. Reading used, the INT8 rule with 7 levels a side:
+ *     amax = max_d |x_d|,  scale = amax / 7  (fp32),
+ *     code_d = clamp(nearbyint(x_d / scale), -7, 7)  (fp32 quotient, ties to even),
+ * amax = 0 gives scale = 0 and all codes 0. Storage: two codes per byte as offset-binary
+ * nibbles u = code + 8; byte i (i < D/2) of a row holds d = i in its low nibble and
+ * d = i + D/2 in its high nibble. packed: uint8 [rows][D/2].
+ * ------------------------------------------------------------------------------------- */
+void or_quantize_int4(int64_t rows, int32_t D, const uint16_t *src, uint8_t *packed, float *scale) {
+    int8_t *c = (int8_t *)malloc((size_t)D);
+    for (int64_t r = 0; r < rows; ++r) {
+        float amax = 0.0f;
+        for (int32_t d = 0; d < D; ++d) {
+            float a = fabsf((float)or_bf16(src[r * D + d]));
+            if (a > amax) amax = a;
+        }
+        float sc = amax / 7.0f;
+        scale[r] = sc;
+        for (int32_t d = 0; d < D; ++d) {
+            if (amax == 0.0f) { c[d] = 0; continue; }
+            float v = nearbyintf((float)or_bf16(src[r * D + d]) / sc);
+            if (v > 7.0f) v = 7.0f;
+            if (v < -7.0f) v = -7.0f;
+            c[d] = (int8_t)v;
+        }
+        for (int32_t i = 0; i < D / 2; ++i)
+            packed[r * (D / 2) + i] = (uint8_t)((c[i] + 8) | ((c[i + D / 2] + 8) << 4));
+    }
+    free(c);
+}
+
+/* The codes of packed INT4 rows (layout of or_quantize_int4): codes int8 [rows][D]. */
+void or_unpack_int4(int64_t rows, int32_t D, const uint8_t *packed, int8_t *codes) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int32_t i = 0; i < D / 2; ++i) {
+            uint8_t b = packed[r * (D / 2) + i];
+            codes[r * D + i] = (int8_t)((b & 0xF) - 8);
+            codes[r * D + i + D / 2] = (int8_t)((b >> 4) - 8);
+        }
+}
+
+/* ---------------------------------------------------------------------------------------
  * Merge of split results. [CAP] §2.4.3 (online normaliser) and Fig. 5 (Dist Attention: the
  * decode query is one token and the partial results over disjoint KV ranges are combined).
  * For splits j = 0..S-1 with normalised partials o_j and log-sum-exp lse_j:

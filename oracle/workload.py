@@ -141,11 +141,24 @@ def reference(sp, o: OLayout, layer=0, sel=None, seqs=None):
         return _sampled(sp, o, q, layer, sel)
     k = synth.pool_bits(sp, "k", o.num_pages, layer)
     v = synth.pool_bits(sp, "v", o.num_pages, layer)
-    kq, ks = oracle.quantize_int8(synth.pool_bits(sp, "kslow", o.num_slow_pages, layer))
-    vq, vs = oracle.quantize_int8(synth.pool_bits(sp, "vslow", o.num_slow_pages, layer))
+    kq, ks, vq, vs = slow_tier(sp, o, layer)
     st = o.slow_table if o.slow_table.size else np.zeros(1, np.int32)
     return oracle.tiered_decode(q, kq, vq, ks, vs, st, o.slow_off, k, v, o.table, o.head_off,
                                 o.kv_len, o.fast_len, sp.scale, sel=sel)
+
+
+def slow_tier(sp, o: OLayout, layer=0):
+    """The quantised slow tier as the oracle stores it: (k codes, k scales, v codes, v scales),
+    codes int8 [Ps][page][D] (INT4 tiers unpacked from their packed form)."""
+    kb = synth.pool_bits(sp, "kslow", o.num_slow_pages, layer)
+    vb = synth.pool_bits(sp, "vslow", o.num_slow_pages, layer)
+    if getattr(sp, "slow_bits", 8) == 4:
+        kp, ks = oracle.quantize_int4(kb)
+        vp, vs = oracle.quantize_int4(vb)
+        return oracle.unpack_int4(kp), ks, oracle.unpack_int4(vp), vs
+    kq, ks = oracle.quantize_int8(kb)
+    vq, vs = oracle.quantize_int8(vb)
+    return kq, ks, vq, vs
 
 
 def _sampled(sp, o, q, layer, sel):

@@ -161,6 +161,7 @@ class Spec:
     suffix_hi: int = 0
     fast_tokens: int = 0
     seed: int = 0x7A4E0000
+    slow_bits: int = 8          # tiered: code width of the slow tier (8 or 4)
 
     @property
     def G(self) -> int:

@@ -416,6 +416,81 @@ def test_tiered_equals_untiered_on_exact_values():
 
 
 # ---------------------------------------------------------------------------------------
+# The INT4 slow-tier quantiser: hand-worked rows and packed bytes, bounds, symmetry, and the
+# exact dequantisation of values c * 2^-e (|c| <= 7) through the tiered decode.
+# ---------------------------------------------------------------------------------------
+
+def test_quantize_int4_golden():
+    for c in gold("quantize_int4.json")["cases"]:
+        packed, scale = oracle.quantize_int4(bf16([c["x"]]))
+        np.testing.assert_array_equal(packed[0], c["packed"])
+        np.testing.assert_array_equal(oracle.unpack_int4(packed)[0], c["codes"])
+        assert float(scale[0]) == c["scale"]
+
+
+def test_quantize_int4_bounds_and_symmetry():
+    x = bf16(np.random.default_rng(23).normal(size=(500, 128)) * 2)
+    packed, scale = oracle.quantize_int4(x)
+    assert packed.shape == (500, 64)
+    codes = oracle.unpack_int4(packed).astype(int)
+    xf = widen(x)
+    assert (np.abs(codes) <= 7).all()
+    assert (np.abs(codes).max(1) == 7).all()                            # the max maps to ±7
+    err = np.abs(xf - codes * scale[:, None].astype(np.float64))
+    assert (err <= scale[:, None] * (0.5 + 1e-5)).all()                 # half a step
+    assert ((packed & 0xF) != 0).all() and ((packed >> 4) != 0).all()   # nibble 0 (= -8) unused
+    nc = oracle.unpack_int4(oracle.quantize_int4(synth.f64_to_bf16_bits(-xf))[0])
+    np.testing.assert_array_equal(nc, -codes)
+
+
+def test_int4_tier_equals_untiered_on_exact_values():
+    """Rows c * 2^-e with |c| <= 7 and a 7 in every row quantise exactly (scale 2^-e): the
+    INT4 quantiser returns c, and the tiered decode of the unpacked INT4 tier equals the
+    untiered decode of the bf16 rows."""
+    rng = np.random.default_rng(24)
+    B, Hq, Hkv, D, page = 1, 4, 2, 64, 16
+    kv = np.array([[50, 37]], np.int32)
+    fast = np.array([[18, 5]], np.int32)
+    q = bf16(rng.normal(size=(B, Hq, D)))
+    rows_k, rows_v = [], []
+    for n in kv.reshape(-1):
+        for rows in (rows_k, rows_v):
+            c = rng.integers(-7, 8, (int(n), D))
+            c[np.arange(int(n)), rng.integers(0, D, int(n))] = rng.choice([-7, 7], int(n))
+            e = rng.integers(2, 9, int(n))
+            rows.append(bf16(c * 2.0 ** -e[:, None]))
+    need = int(((kv + page - 1) // page).sum())
+    order = rng.permutation(need)
+    kp, ids, cnt = scatter_rows(rows_k, page, order, D, num_pages=need)
+    vp, _, _ = scatter_rows(rows_v, page, order, D, num_pages=need)
+    t, off = flat_table(ids, cnt)
+    ref, rlse = oracle.decode(q, kp, vp, t, off.reshape(B, Hkv), kv, 0.125)
+    # slow tier = the first n - f tokens of each head, quantised to INT4 page by page
+    slow_k = [r[:n - f] for r, n, f in zip(rows_k, kv.reshape(-1), fast.reshape(-1))]
+    slow_v = [r[:n - f] for r, n, f in zip(rows_v, kv.reshape(-1), fast.reshape(-1))]
+    fast_k = [r[n - f:] for r, n, f in zip(rows_k, kv.reshape(-1), fast.reshape(-1))]
+    fast_v = [r[n - f:] for r, n, f in zip(rows_v, kv.reshape(-1), fast.reshape(-1))]
+    ns = sum(-(-r.shape[0] // page) for r in slow_k)
+    so = rng.permutation(ns)
+    kb, sids, scnt = scatter_rows(slow_k, page, so, D, num_pages=ns)
+    vb, _, _ = scatter_rows(slow_v, page, so, D, num_pages=ns)
+    kpk, ks = oracle.quantize_int4(kb)
+    vpk, vs = oracle.quantize_int4(vb)
+    kq, vq = oracle.unpack_int4(kpk), oracle.unpack_int4(vpk)
+    np.testing.assert_array_equal(kq * ks[..., None].astype(np.float64), widen(kb))   # exact
+    nf = sum(-(-r.shape[0] // page) for r in fast_k)
+    fo = rng.permutation(nf)
+    kf, fids, fcnt = scatter_rows(fast_k, page, fo, D, num_pages=nf)
+    vf, _, _ = scatter_rows(fast_v, page, fo, D, num_pages=nf)
+    st, soff = flat_table(sids, scnt)
+    ft, foff = flat_table(fids, fcnt)
+    out, lse = oracle.tiered_decode(q, kq, vq, ks, vs, st, soff.reshape(B, Hkv), kf, vf, ft,
+                                    foff.reshape(B, Hkv), kv, fast, 0.125)
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+    np.testing.assert_allclose(lse, rlse, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------
 # Decode-step write path (sink + recent, H2O): hand-worked cases, closed forms, invariants.
 # ---------------------------------------------------------------------------------------
 

@@ -78,8 +78,18 @@ def _plan_kw(cfg):
     return kw
 
 
-def _global_spec(cfg, world):
+SLOW_BITS = 8   # code width of the tiered workloads' slow tier (--slow-bits)
+
+
+def _preset(cfg):
+    """The named workload; tiered ones with the slow tier at SLOW_BITS."""
+    from dataclasses import replace
     sp = synth.preset(cfg)
+    return replace(sp, slow_bits=SLOW_BITS) if sp.kind == "tiered" else sp
+
+
+def _global_spec(cfg, world):
+    sp = _preset(cfg)
     if world > 1:
         from dataclasses import replace
         sp = replace(sp, B=sp.B * world)
@@ -427,8 +437,10 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if lay.fast_len is None else "bf16+int8", "data": "synthetic",
-            "config": {"workload": WORKLOAD_NAMES[cfg], "config_id": cfg,
+            "dtype": "bf16" if lay.fast_len is None else "bf16+int%d" % sp.slow_bits,
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAMES[cfg] + ("" if sp.slow_bits == 8 or lay.fast_len is None
+                                                          else " (INT4 slow tier)"), "config_id": cfg,
                        "global_batch": int(b_total), "parallelism":
                        "sequence shards by AOT byte placement, no collective" if world > 1
                        else "single GPU",
@@ -756,7 +768,7 @@ def run_tier_host(args):
     from non_uniform_paged_flash_b200 import workload
 
     cfg = 5
-    sp = synth.preset(cfg)
+    sp = _preset(cfg)
     lay = workload.layout(sp, 0)
     kw = _plan_kw(cfg)
     db = workload.to_device(sp, lay, 0, **kw)
@@ -803,10 +815,11 @@ def run_tier_host(args):
     achieved = slow_bytes / (ms * 1e-3) / 1e9
     alg = workload.algorithmic_bytes(sp, lay)
     line = {
-        "metric": "tiered decode step, INT8 tier streamed from host memory (GB/s of INT8 tier)",
+        "metric": "tiered decode step, slow tier streamed from host memory (GB/s of slow tier)",
         "value": achieved, "unit": "GB/s", "higher_is_better": True, "n_gpus": 1, "steps": reps,
-        "warmup": args.warmup, "ms_per_step": ms, "dtype": "bf16+int8", "data": "synthetic",
-        "config": {"workload": WORKLOAD_NAMES[cfg] + "; INT8 tier in pinned host memory",
+        "warmup": args.warmup, "ms_per_step": ms, "dtype": "bf16+int%d" % sp.slow_bits,
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAMES[cfg] + "; INT%d tier in pinned host memory" % sp.slow_bits,
                    "block_pages": block_pages, "ring_blocks": 3, "blocks_per_step": n_blocks},
         "host_tier_bytes_per_step": slow_bytes, "kv_bytes_per_step": int(alg["kv"]),
         "roofline": {"bound": "host link", "achieved": achieved, "peak": peak_link,
@@ -897,6 +910,8 @@ def main():
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--slow-bits", type=int, default=8, choices=[8, 4],
+                    help="code width of the tiered workloads' slow tier (config 5, ttkv-host)")
     ap.add_argument("--block-pages", type=int, default=8192,
                     help="--path ttkv-host: INT8-tier pages per streamed block")
     ap.add_argument("--path", default="decode",
@@ -906,6 +921,10 @@ def main():
                          "ttkv-host: the tiered step with the INT8 tier streamed from host "
                          "memory (config 5); splitzip: the KV codec; one GPU, separate JSON line")
     args = ap.parse_args()
+    global SLOW_BITS
+    SLOW_BITS = args.slow_bits
+    if args.slow_bits == 4 and args.path == "ttkv":
+        ap.error("--path ttkv migrates into the INT8 tier; INT4 runs with the decode and ttkv-host paths")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -185,6 +185,10 @@ typedef struct tg_plan_opts {
     int32_t out_f32;          /* 1: the decode calls' out is fp32 [B][Hq][D] (the normalised
                                  output before bf16 rounding, e.g. a partial result to be merged
                                  with others by tg_lse_merge); 0 (default): bf16 */
+    int32_t slow_bits;        /* tiered plans: code width of the slow tier, 8 (0 = default) or
+                                 4 (D = 128 only): INT4 pools are uint8 [num_slow_pages][16][D/2]
+                                 as tg_quantize_int4 writes them, passed where the INT8 calls
+                                 take k_q8 / v_q8 */
 } tg_plan_opts;
 
 /* Build a plan. kv_len[B*Hkv] (host): retained tokens per (sequence, KV head); the decode
@@ -473,6 +477,15 @@ int tg_lse_merge(int64_t n_rows, int32_t D, const int64_t *row_split_off, const 
  * src device bf16 [n_rows][D]; codes device int8 [n_rows][D]; scale device fp32 [n_rows].
  * A page of the INT8 pool is 16 consecutive rows. */
 int tg_quantize_int8(int64_t n_rows, int32_t D, const void *src, int8_t *codes, float *scale,
+                     tg_stream stream);
+
+/* INT4 slow-tier quantisation ("TTKV" 核心方法 1 Tier Layout names INT8 or INT4 for the slow
+ * tier; the scheme is left open): the INT8 rule with 7 levels a side,
+ *   scale = amax / 7 (fp32), code = clamp(rint(x / scale), -7, 7),
+ * packed two codes per byte as offset-binary nibbles: byte i (i < D/2) of a row is
+ * (code_i + 8) | (code_{i+D/2} + 8) << 4. src device bf16 [n_rows][D]; packed device uint8
+ * [n_rows][D/2]; scale device fp32 [n_rows]. Tiered plans with slow_bits = 4 read this layout. */
+int tg_quantize_int4(int64_t n_rows, int32_t D, const void *src, uint8_t *packed, float *scale,
                      tg_stream stream);
 
 /* =====================================================================================

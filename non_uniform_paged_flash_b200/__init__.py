@@ -47,7 +47,7 @@ class tg_plan_opts(ctypes.Structure):
                 ("dyn_chunk_pages", ctypes.c_int32), ("early_prologue", ctypes.c_int32),
                 ("wait_limit_us", ctypes.c_int32), ("test_withhold_page", ctypes.c_int32),
                 ("capacity", ctypes.c_int32),
-                ("out_f32", ctypes.c_int32)]
+                ("out_f32", ctypes.c_int32), ("slow_bits", ctypes.c_int32)]
 
 
 class tg_plan_info(ctypes.Structure):
@@ -100,6 +100,7 @@ _SIGS = [
                                         _F32, _P, _P, _P]),
     ("tg_lse_merge", ctypes.c_int, [_I64, _I32, _P, _P, _P, _P, _P, _P]),
     ("tg_quantize_int8", ctypes.c_int, [_I64, _I32, _P, _P, _P, _P]),
+    ("tg_quantize_int4", ctypes.c_int, [_I64, _I32, _P, _P, _P, _P]),
     ("tg_ragged_paged_decode_scores", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _F32, _P,
                                                      _P, _P, _P]),
     ("tg_append_sink_recent", ctypes.c_int, [ctypes.POINTER(tg_shape), _I32, _P, _P, _P, _P, _P,
@@ -317,14 +318,14 @@ def tg_plan_create(shape: tg_shape, kv_len, group_of_head, group_off, fast_len=N
                    static_permille: int = 0, dyn_chunk_pages: int = 0,
                    early_prologue: bool = False, wait_limit_us: int = 0,
                    test_withhold_page: int = 0, capacity: bool = False,
-                   out_f32: bool = False) -> Plan:
+                   out_f32: bool = False, slow_bits: int = 8) -> Plan:
     kv = _h(kv_len, np.int32).reshape(-1)
     fl = None if fast_len is None else _h(fast_len, np.int32).reshape(-1)
     goh = _h(group_of_head, np.int32).reshape(-1)
     goff = _h(group_off, np.int64).reshape(-1)
     opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
                         static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us,
-                        test_withhold_page, int(capacity), int(out_f32))
+                        test_withhold_page, int(capacity), int(out_f32), int(slow_bits))
     h = ctypes.c_void_p()
     _check(_lib().tg_plan_create(ctypes.byref(shape), _hp(kv), _hp(fl), _hp(goh), _hp(goff),
                                  goff.size - 1, slow_table_len, ctypes.byref(opts),
@@ -346,7 +347,7 @@ def tg_plan_create_cascade(shape: tg_shape, kv_len, group_of_head, group_off, pa
     hoff = _h(head_page_off, np.int64).reshape(-1)
     opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
                         static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us, 0, 0,
-                        int(out_f32))
+                        int(out_f32), 8)
     h = ctypes.c_void_p()
     _check(_lib().tg_plan_create_cascade(ctypes.byref(shape), _hp(kv), _hp(goh), _hp(goff),
                                          goff.size - 1, _hp(tbl), _hp(hoff), tbl.size,
@@ -589,7 +590,7 @@ class SlowStream:
                  slow_page_table, slow_head_off, block_pages: int, ring_blocks: int = 3,
                  num_workers: int = 0, min_splits: int = 1, max_chunk_pages: int = 0,
                  host_only: bool = False, device: int = -1, static_permille: int = 0,
-                 dyn_chunk_pages: int = 0, early_prologue: bool = False):
+                 dyn_chunk_pages: int = 0, early_prologue: bool = False, slow_bits: int = 8):
         self.shape = shape
         kv = _h(kv_len, np.int32).reshape(-1)
         fl = _h(fast_len, np.int32).reshape(-1)
@@ -598,7 +599,8 @@ class SlowStream:
         tbl = _h(slow_page_table, np.int32).reshape(-1)
         off = _h(slow_head_off, np.int64).reshape(-1)
         opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
-                            static_permille, dyn_chunk_pages, int(early_prologue), 0, 0, 0, 0)
+                            static_permille, dyn_chunk_pages, int(early_prologue), 0, 0, 0, 0,
+                            int(slow_bits))
         h = ctypes.c_void_p()
         _check(_lib().tg_slow_stream_create(ctypes.byref(shape), _hp(kv), _hp(fl), _hp(goh),
                                             _hp(goff), goff.size - 1, _hp(tbl) if tbl.size else None,
@@ -655,6 +657,13 @@ def tg_quantize_int8(src, codes, scale, stream=None):
     n_rows = src.numel() // D
     _check(_lib().tg_quantize_int8(n_rows, D, _dp(src), _dp(codes), _dp(scale), _stream(stream)),
            "tg_quantize_int8")
+
+
+def tg_quantize_int4(src, packed, scale, stream=None):
+    D = src.shape[-1]
+    n_rows = src.numel() // D
+    _check(_lib().tg_quantize_int4(n_rows, D, _dp(src), _dp(packed), _dp(scale), _stream(stream)),
+           "tg_quantize_int4")
 
 
 # ---------------------------------------------------------------------------------------

@@ -305,7 +305,8 @@ int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
     const int64_t BH = static_cast<int64_t>(s.B) * s.Hkv;
     const int32_t page = s.page;
     const int64_t bf16_page_cost = 2LL * page * s.D * 2;            // K + V bytes of a page
-    const int64_t i8_page_cost = 2LL * (page * s.D + page * 4);     // codes + fp32 scales
+    const int64_t slow_row = p->slow_bits == 4 ? s.D / 2 : s.D;       // code bytes per token
+    const int64_t i8_page_cost = 2LL * (page * slow_row + page * 4);  // codes + fp32 scales
     const int64_t item_cost = static_cast<int64_t>(p->G) * s.D * 6; // q in + partial out
 
     struct Chunk {
@@ -327,7 +328,7 @@ int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
         if (fast_len) {
             runs[nr++] = {n - f, kItemSlow, i8_page_cost};
             runs[nr++] = {f, 0, bf16_page_cost};
-            kv_bytes += static_cast<int64_t>(n - f) * 2 * (s.D + 4) + static_cast<int64_t>(f) * 2 * s.D * 2;
+            kv_bytes += static_cast<int64_t>(n - f) * 2 * (slow_row + 4) + static_cast<int64_t>(f) * 2 * s.D * 2;
         } else {
             runs[nr++] = {n, 0, bf16_page_cost};
             kv_bytes += static_cast<int64_t>(n) * 2 * s.D * 2;
@@ -605,6 +606,11 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
     if (o.capacity && !fast_len) { delete p; return TG_EINVAL; }
     p->capacity = o.capacity != 0;
     p->out_f32 = o.out_f32 != 0;
+    p->slow_bits = o.slow_bits == 0 ? 8 : o.slow_bits;
+    if ((p->slow_bits != 8 && p->slow_bits != 4) || (p->slow_bits == 4 && (!fast_len || shape->D != 128))) {
+        delete p;
+        return TG_EINVAL;
+    }
 
     // Prefix cascade: shared runs per KV head, cut into units of kCascadeRows query rows.
     std::vector<int32_t> casc_cnt;

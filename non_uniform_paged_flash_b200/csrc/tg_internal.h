@@ -93,6 +93,7 @@ struct tg_plan {
     int32_t withhold = 0;             // see tg_plan_opts.test_withhold_page
     bool capacity = false;            // see tg_plan_opts.capacity
     bool out_f32 = false;             // see tg_plan_opts.out_f32
+    int32_t slow_bits = 8;            // see tg_plan_opts.slow_bits
     int32_t n_workers = 0;
     int64_t kv_bytes = 0;
 

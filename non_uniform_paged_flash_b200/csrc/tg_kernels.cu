@@ -159,6 +159,15 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Unsigned A (INT4 codes widened to offset-binary bytes 0..15) against signed B.
+__device__ __forceinline__ void mma_u8s8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                        uint32_t a3, uint32_t b0, uint32_t b1) {
     asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
@@ -209,6 +218,30 @@ __device__ __forceinline__ void i8pair_to_f16(uint32_t v, uint32_t &lo, uint32_t
     __half2 hb = __hsub2(*reinterpret_cast<__half2 *>(&b), bias);
     lo = *reinterpret_cast<uint32_t *>(&ha);
     hi = *reinterpret_cast<uint32_t *>(&hb);
+}
+
+// One ldmatrix.trans register of INT4 V (offset-binary nibbles; bits 0-7 token t byte b,
+// 8-15 token t byte b+1, 16-23 token t+1 byte b, 24-31 token t+1 byte b+1) -> fp16x2 (t, t+1)
+// of its four d: `lo` takes the low nibbles of bytes b (shift 0) or b+1 (shift 8), exactly as
+// 1024 + u - 1032; `hi` the high nibbles, as (1024 + 16u) / 16 - 72.
+__device__ __forceinline__ uint32_t nib_lo_f16(uint32_t v) {
+    uint32_t h = (v & 0x000F000Fu) | 0x64006400u;
+    const __half2 bias = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032
+    __half2 r = __hsub2(*reinterpret_cast<__half2 *>(&h), bias);
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+__device__ __forceinline__ uint32_t nib_hi_f16(uint32_t v) {
+    uint32_t h = (v & 0x00F000F0u) | 0x64006400u;
+    const __half2 k = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));     // 1/16
+    const __half2 c = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));     // -72
+    __half2 r = __hfma2(*reinterpret_cast<__half2 *>(&h), k, c);
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a box of 64-byte rows written by TMA
+// with 64-byte swizzle (chunk bits XOR address bits 7-8; the box base is 512-byte aligned).
+__device__ __forceinline__ uint32_t swz64(uint32_t row, uint32_t chunk) {
+    return row * 64u + (((chunk ^ (row >> 1)) & 3u) << 4);
 }
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a box of 128-byte rows written by TMA
@@ -277,17 +310,21 @@ constexpr int32_t kNoLoad = -2;  // page id placeholder of a row that failed its
 // Shared-memory stage layout (offsets within a stage; D = 128 shown, D = 64 halves the bf16
 // regions): K bf16 [0, KB) as D/64 boxes of 16 rows x 128 B; V bf16 [KB, 2KB); q [2KB, +QB).
 // INT8 pages reuse it: K codes [0, 2048), K scales [2048, 2112), V scales [2112, 2176),
-// V codes [KB, KB + 2048).
+// V codes [KB, KB + 2048). INT4 pages: packed K [KB + 2048, KB + 3072), packed V
+// [KB + 3072, KB + 4096) (16 rows x 64 B each, 64-byte swizzle), scales as INT8.
 template <int D>
 struct Layout {
     static constexpr int KB = 16 * D * 2;
     static constexpr int kI8 = 16 * D;  // one INT8 page of one tensor
+    static constexpr int kI4 = 8 * D;   // one INT4 page of one tensor
     static constexpr int kKScale = 2048, kVScale = 2112;
+    static constexpr int kK4 = KB + kI8, kV4 = KB + kI8 + kI4;
 };
 
 // Online-softmax state of the two query heads (2t, 2t+1) a consumer lane accumulates.
 struct PageState {
     float sq0, sq1;  // INT8 tier: s_q * scale * log2(e) / 254 of heads 2t, 2t+1
+    int32_t k0, k1;  // INT4 tier: 8 (254 sum q1 + sum q2) of heads 2t, 2t+1 (offset-binary K)
     float m0, m1;    // running maxima, log2 units
     float le0, le1;  // sums of fp32 probabilities (for the lse)
     float lr0, lr1;  // sums of the probabilities multiplied into V
@@ -301,8 +338,10 @@ struct PageState {
 // 8 heads, tokens on M), one max reduction and rescale check for all NP pages, then O^T +=
 // V^T P^T per page. With NP = 2 the two pages' instruction streams interleave (independent
 // chains). SLOW: INT8 pages (K codes on the s8 tensor path against two int8 digits of q, V codes
-// widened to fp16 in registers, per-token scales).
-template <int D, int NP, bool SLOW>
+// widened to fp16 in registers, per-token scales); with SB = 4 the pages hold INT4 codes (byte
+// i of a row: d = i low nibble, d = i + D/2 high nibble, offset-binary), and off8[0..1] are the
+// ldmatrix offsets of the two 32-byte halves of the 64-byte rows.
+template <int D, int NP, bool SLOW, int SB = 8>
 __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const int (&valid)[NP],
                                               const uint32_t (&qf)[D / 16][2],
                                               float (&o)[D / 16][4], PageState &ps,
@@ -331,6 +370,48 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
                 dev::ldsm_x4(sa[p] + offK[j], a0, a1, a2, a3);
                 dev::mma_bf16(s[p], a0, a1, a2, a3, qf[j][0], qf[j][1]);
             }
+        }
+    } else if (SB == 4) {
+        // INT4 K: one ldmatrix of a 32-byte half gives, per register, four bytes of one token;
+        // their low nibbles are the u8 A fragment of d chunk jj and their high nibbles that of
+        // chunk jj + 2 (d + 64). S = s_q (K.q1 + K.q2 / 254) with K = u - 8: the 8 (254 sum q1
+        // + sum q2) of the offset is subtracted in int32 (ps.k0 / ps.k1).
+        int32_t s1[NP][4], s2[NP][4];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) s1[p][0] = s1[p][1] = s1[p][2] = s1[p][3] = s2[p][0] = s2[p][1] = s2[p][2] = s2[p][3] = 0;
+#pragma unroll
+        for (int jj = 0; jj < D / 64; ++jj) {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                uint32_t r0, r1, r2, r3;
+                dev::ldsm_x4(sa[p] + L::kK4 + off8[jj], r0, r1, r2, r3);
+                const uint32_t m = 0x0F0F0F0Fu;
+                dev::mma_u8s8(s1[p], r0 & m, r1 & m, r2 & m, r3 & m, qf[jj][0], qf[jj][1]);
+                dev::mma_u8s8(s2[p], r0 & m, r1 & m, r2 & m, r3 & m, qf[KS / 2 + jj][0], qf[KS / 2 + jj][1]);
+                dev::mma_u8s8(s1[p], (r0 >> 4) & m, (r1 >> 4) & m, (r2 >> 4) & m, (r3 >> 4) & m,
+                              qf[jj + D / 64][0], qf[jj + D / 64][1]);
+                dev::mma_u8s8(s2[p], (r0 >> 4) & m, (r1 >> 4) & m, (r2 >> 4) & m, (r3 >> 4) & m,
+                              qf[KS / 2 + jj + D / 64][0], qf[KS / 2 + jj + D / 64][1]);
+            }
+        }
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            s[p][0] = static_cast<float>(s1[p][0] * 254 + s2[p][0] - ps.k0);
+            s[p][1] = static_cast<float>(s1[p][1] * 254 + s2[p][1] - ps.k1);
+            s[p][2] = static_cast<float>(s1[p][2] * 254 + s2[p][2] - ps.k0);
+            s[p][3] = static_cast<float>(s1[p][3] * 254 + s2[p][3] - ps.k1);
+        }
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            float k0, k1, v0, v1;
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(k0) : "r"(sa[p] + L::kKScale + 4 * g));
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(k1) : "r"(sa[p] + L::kKScale + 4 * (g + 8)));
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v0) : "r"(sa[p] + L::kVScale + 4 * g));
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v1) : "r"(sa[p] + L::kVScale + 4 * (g + 8)));
+            ks[p][0] = k0;
+            ks[p][1] = k1;
+            vs[p][0] = v0;
+            vs[p][1] = v1;
         }
     } else {
         // INT8 codes straight into the integer tensor-core path: K (tokens x 32 d, as stored)
@@ -480,6 +561,28 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
             b0[p] = dev::movm_t(dev::pack_f16(q0, q1));
             b1[p] = dev::movm_t(dev::pack_f16(q2, q3));
         }
+        if (SB == 4) {
+            // INT4 V: ldmatrix.trans of a 32-byte half jj (chunks 2jj, 2jj+1): r0 / r1 tokens
+            // (2t, 2t+1) / (8+2t, 9+2t) at bytes 32jj + 2g, +1, r2 / r3 the same 16 bytes on.
+            // Low nibbles: d tiles 2jj and 2jj+1; high nibbles: the tiles D/32 further (d + D/2);
+            // row g -> d 16i + 2g (byte b), row g+8 -> d + 1 (byte b+1), as on the INT8 path.
+#pragma unroll
+            for (int jj = 0; jj < D / 64; ++jj) {
+#pragma unroll
+                for (int p = 0; p < NP; ++p) {
+                    uint32_t r0, r1, r2, r3;
+                    dev::ldsm_x4_t(sa[p] + L::kV4 + off8[jj], r0, r1, r2, r3);
+                    dev::mma_f16(o[2 * jj], dev::nib_lo_f16(r0), dev::nib_lo_f16(r0 >> 8), dev::nib_lo_f16(r1),
+                                 dev::nib_lo_f16(r1 >> 8), b0[p], b1[p]);
+                    dev::mma_f16(o[2 * jj + D / 32], dev::nib_hi_f16(r0), dev::nib_hi_f16(r0 >> 8),
+                                 dev::nib_hi_f16(r1), dev::nib_hi_f16(r1 >> 8), b0[p], b1[p]);
+                    dev::mma_f16(o[2 * jj + 1], dev::nib_lo_f16(r2), dev::nib_lo_f16(r2 >> 8), dev::nib_lo_f16(r3),
+                                 dev::nib_lo_f16(r3 >> 8), b0[p], b1[p]);
+                    dev::mma_f16(o[2 * jj + 1 + D / 32], dev::nib_hi_f16(r2), dev::nib_hi_f16(r2 >> 8),
+                                 dev::nib_hi_f16(r3), dev::nib_hi_f16(r3 >> 8), b0[p], b1[p]);
+                }
+            }
+        } else {
 #pragma unroll
         for (int ii = 0; ii < KS / 2; ++ii) {
 #pragma unroll
@@ -497,13 +600,14 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
                 dev::mma_f16(o[2 * ii + 1], a0, a1, a2, a3, b0[p], b1[p]);
             }
         }
+        }
     }
 }
 
 // ------------------------------------------------------------------------------------------
 // Decode kernel
 // ------------------------------------------------------------------------------------------
-template <int D, bool TIERED, int NPAIRS>
+template <int D, bool TIERED, int NPAIRS, int SB = 8>
 __global__ void __launch_bounds__(NPAIRS * 64, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v,
@@ -723,7 +827,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         const uint32_t fb = full0 + 8 * stage;
                         const uint32_t qbytes = static_cast<uint32_t>(a.G * D * 2);
                         uint32_t bytes = first ? qbytes : 0u;
-                        if (page_id >= 0) bytes += slow ? 2u * (L::kI8 + 64u) : 2u * L::KB;
+                        if (page_id >= 0) bytes += slow ? 2u * ((SB == 4 ? L::kI4 : L::kI8) + 64u) : 2u * L::KB;
                         if (a.withhold && worker == 0 && seq + 1 == static_cast<uint32_t>(a.withhold)) {
                             // testing: this stage is never signalled; the consumer's bounded
                             // wait runs out and the call reports a timeout
@@ -737,7 +841,12 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                                                qbytes, fb);
                             if (page_id >= 0) {
                                 const int32_t y = page_id * 16;
-                                if (slow) {
+                                if (slow && SB == 4) {
+                                    dev::tma_load_2d(st + L::kK4, &tm_kq, 0, y, fb);
+                                    dev::tma_load_2d(st + L::kV4, &tm_vq, 0, y, fb);
+                                    dev::bulk_load(st + L::kKScale, a.k_scale + static_cast<int64_t>(page_id) * 16, 64, fb);
+                                    dev::bulk_load(st + L::kVScale, a.v_scale + static_cast<int64_t>(page_id) * 16, 64, fb);
+                                } else if (slow) {
                                     dev::tma_load_2d(st, &tm_kq, 0, y, fb);
                                     dev::tma_load_2d(st + L::KB, &tm_vq, 0, y, fb);
                                     dev::bulk_load(st + L::kKScale, a.k_scale + static_cast<int64_t>(page_id) * 16, 64, fb);
@@ -832,7 +941,8 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
         }
 #pragma unroll
         for (int j = 0; j < KSTEPS / 2; ++j)
-            off8[j] = dev::swz((lm & 1) * 8 + (lane & 7), 2 * j + (lm >> 1));
+            off8[j] = SB == 4 ? dev::swz64((lm & 1) * 8 + (lane & 7), 2 * j + (lm >> 1))
+                              : dev::swz((lm & 1) * 8 + (lane & 7), 2 * j + (lm >> 1));
     }
     uint32_t qf[KSTEPS][2];
     float o[KSTEPS][4];
@@ -938,6 +1048,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                 amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
                 const float inv = amax > 0.f ? 127.f / amax : 0.f;
                 const float sq = amax / 127.f;
+                int32_t sum1 = 0, sum2 = 0;  // this lane's digit sums (INT4 offset correction)
 #pragma unroll
                 for (int jj = 0; jj < KSTEPS / 2; ++jj) {
                     uint32_t d1[2] = {0u, 0u}, d2[2] = {0u, 0u};
@@ -946,6 +1057,8 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         const float y = qv[jj][e] * inv;
                         const int c1 = max(-127, min(127, __float2int_rn(y)));
                         const int c2 = max(-127, min(127, __float2int_rn((y - static_cast<float>(c1)) * 254.f)));
+                        sum1 += c1;
+                        sum2 += c2;
                         d1[e >> 2] |= (static_cast<uint32_t>(c1) & 0xFFu) << (8 * (e & 3));
                         d2[e >> 2] |= (static_cast<uint32_t>(c2) & 0xFFu) << (8 * (e & 3));
                     }
@@ -958,6 +1071,16 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                 const float sqf = sq * (a.scale_log2 * (1.f / 254.f));
                 ps.sq0 = __shfl_sync(FULL, sqf, 8 * t);      // head 2t lives in lanes 4 * 2t + ...
                 ps.sq1 = __shfl_sync(FULL, sqf, 8 * t + 4);  // head 2t+1
+                if (SB == 4) {
+                    // the four lanes of head g hold all D of its digits
+                    sum1 += __shfl_xor_sync(FULL, sum1, 1);
+                    sum1 += __shfl_xor_sync(FULL, sum1, 2);
+                    sum2 += __shfl_xor_sync(FULL, sum2, 1);
+                    sum2 += __shfl_xor_sync(FULL, sum2, 2);
+                    const int32_t corr = 8 * (254 * sum1 + sum2);
+                    ps.k0 = __shfl_sync(FULL, corr, 8 * t);
+                    ps.k1 = __shfl_sync(FULL, corr, 8 * t + 4);
+                }
             }
 #pragma unroll
             for (int i = 0; i < KSTEPS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
@@ -981,11 +1104,11 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
             if (pair) {
                 const uint32_t sa[2] = {aA, aB};
                 const int va[2] = {hd.valid, validB};
-                consume_pages<D, 2, true>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
+                consume_pages<D, 2, true, SB>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
             } else {
                 const uint32_t sa[1] = {aA};
                 const int va[1] = {hd.valid};
-                consume_pages<D, 1, true>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
+                consume_pages<D, 1, true, SB>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
             }
         }
         __syncwarp();
@@ -1685,6 +1808,39 @@ __global__ void quantize_kernel(int64_t n_rows, const __nv_bfloat16 *src, int8_t
     }
 }
 
+// INT4 quantiser: one warp per row; scale = amax / 7, code = clamp(rint(x / scale), -7, 7)
+// (fp32 quotient, ties to even); byte i of the packed row = (code_i + 8) | (code_{i+D/2} + 8) << 4.
+template <int D>
+__global__ void quantize4_kernel(int64_t n_rows, const __nv_bfloat16 *src, uint8_t *packed,
+                                 float *scale) {
+    constexpr int PB = D / 64;  // packed bytes per lane
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < n_rows; r += warps) {
+        float lo[PB], hi[PB];
+        float amax = 0.f;
+#pragma unroll
+        for (int k = 0; k < PB; ++k) {
+            lo[k] = __bfloat162float(src[r * D + lane * PB + k]);
+            hi[k] = __bfloat162float(src[r * D + D / 2 + lane * PB + k]);
+            amax = fmaxf(amax, fmaxf(fabsf(lo[k]), fabsf(hi[k])));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        const float sc = __fdiv_rn(amax, 7.f);
+#pragma unroll
+        for (int k = 0; k < PB; ++k) {
+            int cl = 0, ch = 0;
+            if (amax != 0.f) {
+                cl = max(-7, min(7, __float2int_rn(__fdiv_rn(lo[k], sc))));
+                ch = max(-7, min(7, __float2int_rn(__fdiv_rn(hi[k], sc))));
+            }
+            packed[r * (D / 2) + lane * PB + k] = static_cast<uint8_t>((cl + 8) | ((ch + 8) << 4));
+        }
+        if (lane == 0) scale[r] = sc;
+    }
+}
+
 // ------------------------------------------------------------------------------------------
 // Host: tensor maps, plan device state, launchers
 // ------------------------------------------------------------------------------------------
@@ -1705,10 +1861,11 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Tensor map over a pool of pages [rows = pages * 16][inner] with 128-byte swizzled boxes of
-// box_inner elements x 16 rows.
+// Tensor map over a pool of pages [rows = pages * 16][inner] with swizzled boxes of box_inner
+// elements x 16 rows (128-byte swizzle, or 64-byte for the 64-byte rows of INT4 pages).
 static int make_pool_map(CUtensorMap *tm, const void *base, CUtensorMapDataType dt, int elem,
-                         uint64_t inner, uint64_t rows, uint32_t box_inner) {
+                         uint64_t inner, uint64_t rows, uint32_t box_inner,
+                         CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) {
         set_cuda_error("cuTensorMapEncodeTiled unavailable", 0);
@@ -1719,7 +1876,7 @@ static int make_pool_map(CUtensorMap *tm, const void *base, CUtensorMapDataType 
     cuuint32_t box[2] = {box_inner, 16};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(tm, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         std::snprintf(g_cuda_msg, sizeof(g_cuda_msg), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -1737,9 +1894,9 @@ int device_num_sms(int device, int *num_sms) {
 
 static constexpr int kSmemBudget = 232448;  // 227 KB opt-in dynamic shared memory per CTA
 
-template <int D, bool TIERED, int NPAIRS>
+template <int D, bool TIERED, int NPAIRS, int SB = 8>
 static int set_smem_attr(int bytes) {
-    TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<D, TIERED, NPAIRS>,
+    TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<D, TIERED, NPAIRS, SB>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
     return TG_OK;
 }
@@ -1768,6 +1925,7 @@ int device_init_plan(tg_plan *p) {
 
     int rc = TG_OK;
     if (s.D == 128 && !p->tiered) rc = set_smem_attr<128, false, kPairs>(p->smem_bytes);
+    else if (s.D == 128 && p->tiered && p->slow_bits == 4) rc = set_smem_attr<128, true, kPairsTiered, 4>(p->smem_bytes);
     else if (s.D == 128 && p->tiered) rc = set_smem_attr<128, true, kPairsTiered>(p->smem_bytes);
     else if (s.D == 64 && !p->tiered) rc = set_smem_attr<64, false, kPairs>(p->smem_bytes);
     else rc = TG_EUNSUPPORTED;
@@ -1876,10 +2034,11 @@ void device_free_plan(tg_plan *p) {
 static bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 static int get_map(tg_plan *p, int idx, const void *base, CUtensorMapDataType dt, int elem,
-                   uint64_t pages, uint32_t box_inner) {
+                   uint64_t pages, uint32_t box_inner, bool int4 = false) {
     if (p->tm_key[idx] == base) return TG_OK;
     int rc = make_pool_map(reinterpret_cast<CUtensorMap *>(p->tmaps[idx]), base, dt, elem,
-                           static_cast<uint64_t>(p->shape.D), pages * 16, box_inner);
+                           static_cast<uint64_t>(int4 ? p->shape.D / 2 : p->shape.D), pages * 16, box_inner,
+                           int4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc == TG_OK) p->tm_key[idx] = base;
     return rc;
 }
@@ -2142,8 +2301,10 @@ extern "C" int tg_tiered_decode(tg_plan *p, const void *q, const int8_t *k_q8,
             if (rc == TG_OK) rc = get_map(p, 1, v_fast, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);
         }
         if (rc == TG_OK && has_slow) {
-            rc = get_map(p, 2, k_q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p->shape.num_slow_pages, 128);
-            if (rc == TG_OK) rc = get_map(p, 3, v_q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p->shape.num_slow_pages, 128);
+            const bool i4 = p->slow_bits == 4;
+            const uint32_t box = i4 ? static_cast<uint32_t>(p->shape.D / 2) : 128u;
+            rc = get_map(p, 2, k_q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p->shape.num_slow_pages, box, i4);
+            if (rc == TG_OK) rc = get_map(p, 3, v_q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p->shape.num_slow_pages, box, i4);
         }
         if (rc != TG_OK) return rc;
         DecodeArgs a = base_args(p, q, head_kv_len, scale, out, lse);
@@ -2159,8 +2320,12 @@ extern "C" int tg_tiered_decode(tg_plan *p, const void *q, const int8_t *k_q8,
         a.fast_len_dev = head_fast_len;
         // The fast tier's rows are bounded by its whole table [group_off[0], group_off[n]).
         const CUtensorMap *maps = reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
-        rc = launch_decode(p, decode_kernel<128, true, kPairsTiered>, a, maps[has_fast ? 0 : 2], maps[has_fast ? 1 : 3],
-                           maps[has_slow ? 2 : 0], maps[has_slow ? 3 : 1], stream);
+        if (p->slow_bits == 4)
+            rc = launch_decode(p, decode_kernel<128, true, kPairsTiered, 4>, a, maps[has_fast ? 0 : 2],
+                               maps[has_fast ? 1 : 3], maps[has_slow ? 2 : 0], maps[has_slow ? 3 : 1], stream);
+        else
+            rc = launch_decode(p, decode_kernel<128, true, kPairsTiered>, a, maps[has_fast ? 0 : 2],
+                               maps[has_fast ? 1 : 3], maps[has_slow ? 2 : 0], maps[has_slow ? 3 : 1], stream);
         if (rc != TG_OK) return rc;
     } else {
         timing_mark(p, 0, stream);
@@ -2216,6 +2381,28 @@ extern "C" int tg_quantize_int8(int64_t n_rows, int32_t D, const void *src, int8
     else
         quantize_kernel<64><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
             n_rows, static_cast<const __nv_bfloat16 *>(src), codes, scale);
+    TG_CUDA_TRY(cudaGetLastError());
+    return TG_OK;
+}
+
+extern "C" int tg_quantize_int4(int64_t n_rows, int32_t D, const void *src, uint8_t *packed,
+                                float *scale, tg_stream stream_) {
+    if (n_rows < 0 || (D != 64 && D != 128)) return n_rows < 0 ? TG_EINVAL : TG_EUNSUPPORTED;
+    if (n_rows == 0) return TG_OK;
+    if (!src || !packed || !scale) return TG_EINVAL;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int threads = 256;
+    int64_t blocks = (n_rows * 32 + threads - 1) / threads;
+    if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
+    if (D == 128)
+        quantize4_kernel<128><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+            n_rows, static_cast<const __nv_bfloat16 *>(src), packed, scale);
+    else
+        quantize4_kernel<64><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+            n_rows, static_cast<const __nv_bfloat16 *>(src), packed, scale);
     TG_CUDA_TRY(cudaGetLastError());
     return TG_OK;
 }

@@ -23,6 +23,7 @@ struct tg_slow_stream {
     int device = 0;
     int32_t G = 0;
     int32_t block_pages = 0, ring = 0;
+    int32_t row_bytes = 0;                  // code bytes per token and tensor: D (INT8) or D/2 (INT4)
     bool host_only = true;
     tg_plan *fast = nullptr;                // bf16 plan over the fast tier (fp32 out)
     std::vector<tg_plan *> blk;             // one tiered plan per streamed block (fp32 out)
@@ -156,6 +157,7 @@ extern "C" int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_le
     s->G = S.Hq / S.Hkv;
     s->block_pages = block_pages;
     s->ring = ring_blocks;
+    s->row_bytes = o.slow_bits == 4 ? S.D / 2 : S.D;
     s->host_only = o.host_only != 0;
     for (int64_t j = 0; j < n_all_blocks; ++j) {
         bool used = false;
@@ -188,7 +190,9 @@ extern "C" int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_le
     po.capacity = 0;
     tg_shape fs = S;
     fs.num_slow_pages = 0;
-    int rc = tg_plan_create(&fs, fl.data(), nullptr, group_of_head, group_off, n_groups, 0, &po, &s->fast);
+    tg_plan_opts fo = po;
+    fo.slow_bits = 0;
+    int rc = tg_plan_create(&fs, fl.data(), nullptr, group_of_head, group_off, n_groups, 0, &fo, &s->fast);
     std::vector<int32_t> zeros(static_cast<size_t>(BH), 0);
     tg_shape bs = S;
     bs.num_slow_pages = block_pages;
@@ -213,7 +217,7 @@ extern "C" int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_le
     cudaGetDevice(&prev);
     cudaSetDevice(s->device);
     const size_t D = static_cast<size_t>(S.D);
-    const size_t slot_codes = static_cast<size_t>(block_pages) * 16 * D;
+    const size_t slot_codes = static_cast<size_t>(block_pages) * 16 * static_cast<size_t>(s->row_bytes);
     const size_t slot_scales = static_cast<size_t>(block_pages) * 16 * sizeof(float);
     const size_t rows_q = static_cast<size_t>(S.B) * static_cast<size_t>(S.Hq);
     const size_t parts = static_cast<size_t>(1 + J);
@@ -327,7 +331,8 @@ extern "C" int tg_tiered_decode_streamed(tg_slow_stream *s, const void *q, const
     const int64_t BH = static_cast<int64_t>(S.B) * S.Hkv;
     const size_t D = static_cast<size_t>(S.D);
     const int64_t rows = static_cast<int64_t>(S.B) * S.Hq;
-    const size_t slot_codes = static_cast<size_t>(s->block_pages) * 16 * D;
+    const size_t R = static_cast<size_t>(s->row_bytes);
+    const size_t slot_codes = static_cast<size_t>(s->block_pages) * 16 * R;
     const size_t slot_scales = static_cast<size_t>(s->block_pages) * 16;
     // Copies never start before the work already queued on `stream` (this call's inputs).
     if ((e = cudaEventRecord(s->start, stream)) != cudaSuccess || (e = cudaStreamWaitEvent(s->copy, s->start, 0)) != cudaSuccess)
@@ -345,8 +350,8 @@ extern "C" int tg_tiered_decode_streamed(tg_slow_stream *s, const void *q, const
         int8_t *rk = s->ring_k + r * slot_codes, *rv = s->ring_v + r * slot_codes;
         float *rks = s->ring_ks + r * slot_scales, *rvs = s->ring_vs + r * slot_scales;
         if ((e = cudaStreamWaitEvent(s->copy, s->freed[r], 0)) != cudaSuccess ||
-            (e = cudaMemcpyAsync(rk, k_q8_host + first * 16 * D, pages * 16 * D, cudaMemcpyHostToDevice, s->copy)) != cudaSuccess ||
-            (e = cudaMemcpyAsync(rv, v_q8_host + first * 16 * D, pages * 16 * D, cudaMemcpyHostToDevice, s->copy)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(rk, k_q8_host + first * 16 * R, pages * 16 * R, cudaMemcpyHostToDevice, s->copy)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(rv, v_q8_host + first * 16 * R, pages * 16 * R, cudaMemcpyHostToDevice, s->copy)) != cudaSuccess ||
             (e = cudaMemcpyAsync(rks, k_scale_host + first * 16, pages * 16 * 4, cudaMemcpyHostToDevice, s->copy)) != cudaSuccess ||
             (e = cudaMemcpyAsync(rvs, v_scale_host + first * 16, pages * 16 * 4, cudaMemcpyHostToDevice, s->copy)) != cudaSuccess ||
             (e = cudaEventRecord(s->landed[r], s->copy)) != cudaSuccess)

@@ -16,7 +16,7 @@ import numpy as np
 import synth
 from . import (make_shape, tg_alloc_create, tg_alloc_destroy, tg_alloc_reserve,
                tg_alloc_share_segment, tg_budget_groups, tg_group_tables, tg_plan_create,
-               tg_quantize_int8, tg_retained_lengths)
+               tg_quantize_int4, tg_quantize_int8, tg_retained_lengths)
 
 
 @dataclass
@@ -204,7 +204,8 @@ class DeviceBatch:
         return SlowStream(self.plan.shape, lay.kv_len, lay.fast_len, lay.group_of_head,
                           lay.group_off, lay.slow_table if lay.slow_table.size else np.full(1, -1),
                           lay.slow_off, block_pages, ring_blocks,
-                          device=dev if dev is not None else -1, **kw)
+                          device=dev if dev is not None else -1, slow_bits=self.spec.slow_bits,
+                          **kw)
 
     def run_streamed(self, ss, host, stream=None):
         """One tiered step with the INT8 tier streamed from the pinned host copies `host`."""
@@ -260,7 +261,8 @@ def to_device(sp: synth.Spec, lay: Layout, layer: int = 0, device="cuda", num_wo
                               max_chunk_pages=max_chunk_pages, static_permille=static_permille,
                               dyn_chunk_pages=dyn_chunk_pages, early_prologue=early_prologue,
                               wait_limit_us=wait_limit_us, test_withhold_page=test_withhold_page,
-                              device=dev.index if dev.index is not None else -1)
+                              device=dev.index if dev.index is not None else -1,
+                              slow_bits=sp.slow_bits if lay.fast_len is not None else 8)
     qb = synth.q_bits(sp, layer)
     q = _bf16_tensor(qb if seqs is None else np.ascontiguousarray(qb[seqs]), dev)
     out = torch.empty((B, sp.Hq, sp.D), dtype=torch.bfloat16, device=dev)
@@ -278,13 +280,16 @@ def to_device(sp: synth.Spec, lay: Layout, layer: int = 0, device="cuda", num_wo
         db.fast_len = it(lay.fast_len, np.int32)
         db.slow_table = it(lay.slow_table if lay.slow_table.size else np.full(1, -1), np.int32)
         db.slow_off = it(lay.slow_off, np.int64)
-        db.k_q8 = torch.empty((ns, sp.page, sp.D), dtype=torch.int8, device=dev)
-        db.v_q8 = torch.empty((ns, sp.page, sp.D), dtype=torch.int8, device=dev)
+        # INT8 pools int8 [ns][page][D]; INT4 pools packed uint8 [ns][page][D/2]
+        i4 = sp.slow_bits == 4
+        cshape, cdt = ((ns, sp.page, sp.D // 2), torch.uint8) if i4 else ((ns, sp.page, sp.D), torch.int8)
+        db.k_q8 = torch.empty(cshape, dtype=cdt, device=dev)
+        db.v_q8 = torch.empty(cshape, dtype=cdt, device=dev)
         db.k_scale = torch.empty((ns, sp.page), dtype=torch.float32, device=dev)
         db.v_scale = torch.empty((ns, sp.page), dtype=torch.float32, device=dev)
         for which, codes, scale in (("kslow", db.k_q8, db.k_scale), ("vslow", db.v_q8, db.v_scale)):
             src = _pool_to_device(sp, which, ns, layer, dev)
-            tg_quantize_int8(src, codes, scale)
+            (tg_quantize_int4 if i4 else tg_quantize_int8)(src, codes, scale)
             del src
         torch.cuda.synchronize(dev)
     return db
@@ -295,15 +300,16 @@ def admit(sp: synth.Spec, layer: int = 0, device="cuda", seqs=None, **plan_kw) -
 
 
 def algorithmic_bytes(sp: synth.Spec, lay: Layout) -> dict:
-    """Bytes one decode step must move: retained K/V (INT8 scales included), the page-table
+    """Bytes one decode step must move: retained K/V (INT8 / INT4 scales included), the page-table
     entries and per-head table words read, q in, out + lse written."""
     kv = lay.kv_len.astype(np.int64)
     if lay.fast_len is None:
         kvb = int(kv.sum()) * 2 * sp.D * 2
         tab = int(pages_of(kv, sp.page).sum()) * 4
     else:
-        f = lay.fast_len.astype(np.int64)
-        kvb = int((kv - f).sum()) * 2 * (sp.D + 4) + int(f.sum()) * 2 * sp.D * 2
+        f = np.minimum(lay.fast_len.astype(np.int64), kv)
+        row = sp.D // 2 if sp.slow_bits == 4 else sp.D   # code bytes per slow token and tensor
+        kvb = int((kv - f).sum()) * 2 * (row + 4) + int(f.sum()) * 2 * sp.D * 2
         tab = int((pages_of(kv - f, sp.page) + pages_of(f, sp.page)).sum()) * 4
     B = lay.kv_len.shape[0]
     BH = B * sp.Hkv

@@ -330,3 +330,25 @@ def test_plan_balances_bytes_across_workers(cfg):
     # equal-cost contiguous ranges: every worker within a few bf16 pages of the mean
     assert work.max() - work.mean() <= 4 * 2 * 16 * sp.D * 2
     assert work.mean() - work.min() <= 4 * 2 * 16 * sp.D * 2
+
+
+def test_plan_slow_bits_validation():
+    """slow_bits: 8 (default) or 4 for tiered D = 128 plans; INT4 halves the code bytes."""
+    import synth
+    from non_uniform_paged_flash_b200 import workload
+    sp = synth.small(5)
+    lay = workload.layout(sp, 0)
+    B = lay.kv_len.shape[0]
+    shape = tg.make_shape(B, sp.Hq, sp.Hkv, sp.D, lay.num_pages, lay.num_slow_pages, sp.page)
+    kw = dict(fast_len=lay.fast_len, slow_table_len=lay.slow_table.size, num_workers=64,
+              host_only=True)
+    i8 = tg.tg_plan_get_info(tg.tg_plan_create(shape, lay.kv_len, lay.group_of_head,
+                                               lay.group_off, **kw))["kv_bytes"]
+    i4 = tg.tg_plan_get_info(tg.tg_plan_create(shape, lay.kv_len, lay.group_of_head,
+                                               lay.group_off, slow_bits=4, **kw))["kv_bytes"]
+    ns = int((lay.kv_len - np.minimum(lay.fast_len, lay.kv_len)).sum())
+    assert i8 - i4 == ns * 2 * (sp.D // 2)
+    for bad in (dict(kw, slow_bits=5), dict(num_workers=64, host_only=True, slow_bits=4)):
+        with pytest.raises(tg.TGError) as ei:
+            tg.tg_plan_create(shape, lay.kv_len, lay.group_of_head, lay.group_off, **bad)
+        assert ei.value.status == tg.TG_EINVAL

@@ -58,24 +58,9 @@ def _env_int(name, default):
 
 
 def _plan_kw(cfg):
-    """Plan options per workload (chosen by measurement on B200): the static share of the
-    bytes, the largest dynamic item, and early prologue (this bench runs only this library's
-    kernels back to back, so the decode may read its plan and tables before the previous
-    step's merge kernel has finished)."""
-    kw = dict(early_prologue=True)
-    if cfg == 1:
-        kw.update(static_permille=1000)
-    elif cfg == 2:
-        kw.update(static_permille=850, dyn_chunk_pages=16)
-    elif cfg == 3:
-        kw.update(static_permille=900, dyn_chunk_pages=32)
-    elif cfg == 4:
-        # shared prefix pages: the cascade reads each shared run once per step for all its
-        # readers; the private pages stay on the split-K items
-        kw.update(static_permille=850, dyn_chunk_pages=16, cascade=True)
-    elif cfg == 5:
-        kw.update(min_splits=64, max_chunk_pages=128, static_permille=900, dyn_chunk_pages=32)
-    return kw
+    """Plan options per workload (chosen by measurement on B200; see workload.timed_plan_options)."""
+    from non_uniform_paged_flash_b200 import workload
+    return workload.timed_plan_options(cfg)
 
 
 SLOW_BITS = 8   # code width of the tiered workloads' slow tier (--slow-bits)
@@ -258,31 +243,50 @@ def run_reference(args):
 # Our arm
 # ------------------------------------------------------------------------------------------
 
-def cpu_baseline(cfg, budget_s=20.0):
+def cpu_baseline(cfg, budget_s=20.0, min_s=10.0):
     """The oracle as it stands on a bounded sample of this workload (rank 0, N = 1)."""
     import oracle
     from oracle import workload as ow
-    sp = synth.preset(cfg)
+    sp = _preset(cfg)
     o = ow.layout(sp, 0)
     q = ow.q_bits(sp)
     cores = oracle.num_threads()
-    if o.fast_len is not None:
-        return None
     k = synth.pool_bits(sp, "k", o.num_pages)
     v = synth.pool_bits(sp, "v", o.num_pages)
-    done, nbytes, t_used = 0, 0, 0.0
+    kv = o.kv_len.astype(np.int64)
+    if o.fast_len is None:
+        row_bytes = kv * 2 * sp.D * 2
+
+        def rows(sel):
+            oracle.decode(q, k, v, o.table, o.head_off, o.kv_len, sp.scale, sel=sel)
+    else:
+        kq, ks, vq, vs = ow.slow_tier(sp, o)
+        st = o.slow_table if o.slow_table.size else np.zeros(1, np.int32)
+        f = np.minimum(o.fast_len.astype(np.int64), kv)
+        cb = sp.D // 2 if sp.slow_bits == 4 else sp.D
+        row_bytes = (kv - f) * 2 * (cb + 4) + f * 2 * sp.D * 2
+
+        def rows(sel):
+            oracle.tiered_decode(q, kq, vq, ks, vs, st, o.slow_off, k, v, o.table, o.head_off,
+                                 o.kv_len, o.fast_len, sp.scale, sel=sel)
+    # passes over the batch, a few sequences at a time, until min_s of oracle time (or the
+    # budget) is spent
+    done, nbytes, t_used, passes = 0, 0, 0.0, 0
     chunk = max(1, sp.B // 16)
-    while done < sp.B and t_used < budget_s:
+    while t_used < min_s and t_used < budget_s:
         b1 = min(sp.B, done + chunk)
         sel = np.arange(done * sp.Hq, b1 * sp.Hq)
         t0 = time.perf_counter()
-        oracle.decode(q, k, v, o.table, o.head_off, o.kv_len, sp.scale, sel=sel)
+        rows(sel)
         t_used += time.perf_counter() - t0
-        nbytes += int(o.kv_len[done:b1].astype(np.int64).sum()) * 2 * sp.D * 2
+        nbytes += int(row_bytes[done:b1].sum())
         done = b1
+        if done == sp.B:
+            done, passes = 0, passes + 1
+    seqs = f"{passes} passes over all {sp.B} sequences" + (f" + sequences 0..{done - 1}" if done else "")
     return {"value": nbytes / t_used / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"sequences 0..{done - 1} of the batch (all their query rows), "
-                      f"{t_used:.1f} s of fp64 oracle time on {cores} host threads"}
+            "sample": f"{seqs} (all their query rows), {t_used:.1f} s of fp64 oracle time on "
+                      f"{cores} host threads"}
 
 
 def run_ours(args):

@@ -214,6 +214,27 @@ class DeviceBatch:
                                   self.group_of_head, self.spec.scale, self.out, self.lse, stream)
 
 
+def timed_plan_options(cfg: int) -> dict:
+    """Plan options per workload, chosen by measurement on B200, the ones bench.py times: the
+    static share of the bytes, the largest dynamic item, the cascade for shared prefixes, and
+    early prologue (only this library's kernels run back to back, so the decode may read its
+    plan and tables before the previous step's merge kernel has finished)."""
+    kw = dict(early_prologue=True)
+    if cfg == 1:
+        kw.update(static_permille=1000)
+    elif cfg == 2:
+        kw.update(static_permille=850, dyn_chunk_pages=16)
+    elif cfg == 3:
+        kw.update(static_permille=900, dyn_chunk_pages=32)
+    elif cfg == 4:
+        # shared prefix pages: the cascade reads each shared run once per step for all its
+        # readers; the private pages stay on the split-K items
+        kw.update(static_permille=850, dyn_chunk_pages=16, cascade=True)
+    elif cfg == 5:
+        kw.update(min_splits=64, max_chunk_pages=128, static_permille=900, dyn_chunk_pages=32)
+    return kw
+
+
 def _bf16_tensor(bits: np.ndarray, device):
     import torch
     return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)

@@ -241,24 +241,52 @@ def _sample_rows(sp, n, seed):
 
 
 def test_full_config1_all_rows():
-    _run(synth.preset(1))
+    _run(synth.preset(1), **workload.timed_plan_options(1))
 
 
 def test_full_config2_all_rows():
+    _run(synth.preset(2), **workload.timed_plan_options(2))
+
+
+def test_full_config2_default_plan_all_rows():
     _run(synth.preset(2))
 
 
 def test_full_config3_sampled_rows_two_layers():
     sp = synth.preset(3)
     for layer in (0, 17):
-        _run(sp, layer, sel=_sample_rows(sp, 96, layer))
+        _run(sp, layer, sel=_sample_rows(sp, 96, layer), **workload.timed_plan_options(3))
 
 
 def test_full_config4_sampled_rows():
+    """The prefix-cascade plan the bench times (tcgen05 cascade + split-K items + merge)."""
     sp = synth.preset(4)
-    _run(sp, sel=_sample_rows(sp, 256, 4))
+    db, _ = _run(sp, sel=_sample_rows(sp, 256, 4), **workload.timed_plan_options(4))
+    assert tg.tg_plan_get_info(db.plan)["n_cascade"] > 0
 
 
 def test_full_config5_sampled_rows():
     sp = synth.preset(5)
-    _run(sp, sel=_sample_rows(sp, 24, 5), min_splits=64, max_chunk_pages=128)
+    _run(sp, sel=_sample_rows(sp, 24, 5), **workload.timed_plan_options(5))
+
+
+def test_full_config5_int4_sampled_rows():
+    sp = replace(synth.preset(5), slow_bits=4)
+    _run(sp, sel=_sample_rows(sp, 24, 6), **workload.timed_plan_options(5))
+
+
+def test_full_config5_host_streamed_sampled_rows():
+    """The INT8 tier streamed from pinned host memory in 8192-page blocks through a ring of 3
+    (the bench's ttkv-host configuration), sampled rows against the oracle."""
+    sp = synth.preset(5)
+    lay = workload.layout(sp, 0)
+    kw = {k: v for k, v in workload.timed_plan_options(5).items() if k != "early_prologue"}
+    db = workload.to_device(sp, lay, 0, **kw)
+    ss = db.slow_stream(8192, 3, **kw)
+    db.run_streamed(ss, db.host_slow_tier())
+    torch.cuda.synchronize()
+    assert ss.status() == tg.TG_OK
+    sel = _sample_rows(sp, 24, 7)
+    ol = ors.layout(sp, 0)
+    ref_out, ref_lse = ors.reference(sp, ol, 0, sel=sel)
+    _compare(db, ref_out, ref_lse, sel)

@@ -463,11 +463,6 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
         mx0 = fmaxf(mx0, fmaxf(x[p][0], x[p][2]));
         mx1 = fmaxf(mx1, fmaxf(x[p][1], x[p][3]));
     }
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
-    }
     if (!SLOW && ts != nullptr) {
         // Per-token scores s = x * ln 2 of the valid tokens, entry (tpos * 16 + token) * G + head.
         constexpr float kLn2f = 0.69314718055994530942f;
@@ -487,10 +482,17 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
         }
     }
     // Lazy rescale: the running max moves only when a tile exceeds it by more than the
-    // threshold (2^8 for bf16 probabilities; exact for the fp16 INT8 path).
+    // threshold (2^8 for bf16 probabilities; exact for the fp16 INT8 path). A lane's own
+    // maxima decide whether any head's tile maximum does (the running max is the same across
+    // a head's lanes), so the cross-lane reduction runs only when it will be used.
     const float thr = SLOW ? 0.f : 8.f;
-    const bool up0 = mx0 > ps.m0 + thr, up1 = mx1 > ps.m1 + thr;
-    if (__any_sync(FULL, up0 || up1)) {
+    if (__any_sync(FULL, mx0 > ps.m0 + thr || mx1 > ps.m1 + thr)) {
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
+        }
+        const bool up0 = mx0 > ps.m0 + thr, up1 = mx1 > ps.m1 + thr;
         const float n0 = up0 ? mx0 : ps.m0, n1 = up1 ? mx1 : ps.m1;
         const float c0 = (ps.m0 == -INFINITY) ? 0.f : dev::ex2(ps.m0 - n0);
         const float c1 = (ps.m1 == -INFINITY) ? 0.f : dev::ex2(ps.m1 - n1);

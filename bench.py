@@ -663,7 +663,7 @@ def run_tier_path(args):
     from non_uniform_paged_flash_b200 import workload
 
     cfg = 5
-    sp = synth.preset(cfg)
+    sp = _preset(cfg)
     lay = workload.layout(sp, 0)
     kw = _plan_kw(cfg)
     db = workload.to_device(sp, lay, 0, **kw)
@@ -700,7 +700,8 @@ def run_tier_path(args):
     shape = tg.make_shape(B, sp.Hq, sp.Hkv, sp.D, lay.num_pages, P_new)
     plan = tg.tg_plan_create(shape, (f0 + S).reshape(B, Hkv), lay.group_of_head, lay.group_off,
                              fast_len=f0.reshape(B, Hkv), slow_table_len=len(table),
-                             capacity=True, **kw)
+                             capacity=True, slow_bits=sp.slow_bits, **kw)
+    append = tg.tg_tiered_append_int4 if sp.slow_bits == 4 else tg.tg_tiered_append
     fcap = it(f0, np.int32)
     scap = it(S, np.int32)
     kv_dev, fl_dev = it(n0, np.int32), it(f0, np.int32)
@@ -713,8 +714,8 @@ def run_tier_path(args):
 
     def step(m=None):
         if m: m[0].record(stream)
-        tg.tg_tiered_append(shape, k_new, v_new, db.k, db.v, db.table, db.head_off, fcap, kq, vq,
-                            ks, vs, stab, soff, scap, kv_dev, fl_dev, moved, slot, stream)
+        append(shape, k_new, v_new, db.k, db.v, db.table, db.head_off, fcap, kq, vq,
+               ks, vs, stab, soff, scap, kv_dev, fl_dev, moved, slot, stream)
         if m: m[1].record(stream)
         tg.tg_tiered_decode(plan, db.q, kq, vq, ks, vs, stab, soff, db.k, db.v, db.table,
                             db.head_off, kv_dev, fl_dev, sp.scale, db.out, db.lse, stream)
@@ -744,14 +745,17 @@ def run_tier_path(args):
     assert (moved.cpu().numpy() >= 0).all()
     t_app = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
     t_dec = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
-    kv_bytes = float(((kv_dev.cpu().numpy() - fl_dev.cpu().numpy()).astype(np.int64) * 2 * (sp.D + 4)).sum()
+    row = sp.D // 2 if sp.slow_bits == 4 else sp.D      # code bytes per slow token and tensor
+    kv_bytes = float(((kv_dev.cpu().numpy() - fl_dev.cpu().numpy()).astype(np.int64) * 2 * (row + 4)).sum()
                      + fl_dev.cpu().numpy().astype(np.int64).sum() * 2 * sp.D * 2)
     peak, peak_kind = _measured_peak()
     line = {
         "metric": "tiered decode step with tier migration: step time", "value": ms_step * 1e3,
         "unit": "us", "higher_is_better": False, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup,
-        "config": {"workload": WORKLOAD_NAMES[cfg], "config_id": cfg, "plan": "capacity"},
+        "config": {"workload": WORKLOAD_NAMES[cfg], "config_id": cfg, "plan": "capacity",
+                   "slow_tier": "INT%d" % sp.slow_bits},
+        "dtype": "bf16+int%d" % sp.slow_bits, "data": "synthetic",
         "kernels_us": {"tier_append": t_app * 1e3, "decode+merge": t_dec * 1e3},
         "kv_bytes_per_step": int(kv_bytes),
         "step_kv_gbs": kv_bytes / (ms_step * 1e-3) / 1e9, "peak_gbs": peak, "peak_kind": peak_kind,
@@ -927,8 +931,6 @@ def main():
     args = ap.parse_args()
     global SLOW_BITS
     SLOW_BITS = args.slow_bits
-    if args.slow_bits == 4 and args.path == "ttkv":
-        ap.error("--path ttkv migrates into the INT8 tier; INT4 runs with the decode and ttkv-host paths")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -566,6 +566,20 @@ int tg_tiered_append(const tg_shape *shape, const void *k_new, const void *v_new
                      const int32_t *head_slow_cap, int32_t *head_kv_len, int32_t *head_fast_len,
                      int32_t *moved_out, int32_t *slot_out, tg_stream stream);
 
+/* tg_tiered_append into an INT4 slow tier: the leaving token is quantised with the rule of
+ * tg_quantize_int4 (scale = amax / 7; codes and scale bit-exact with it) into the packed
+ * pools k_q4, v_q4 (uint8 [num_slow_pages][16][D/2], byte i = d i low nibble and d i + D/2
+ * high nibble, offset-binary); everything else as tg_tiered_append. Tiered plans with
+ * tg_plan_opts.slow_bits = 4 (and capacity = 1) decode the result. */
+int tg_tiered_append_int4(const tg_shape *shape, const void *k_new, const void *v_new,
+                          void *k_fast, void *v_fast, const int32_t *fast_page_table,
+                          const int64_t *fast_head_off, const int32_t *head_fast_cap,
+                          uint8_t *k_q4, uint8_t *v_q4, float *k_scale, float *v_scale,
+                          const int32_t *slow_page_table, const int64_t *slow_head_off,
+                          const int32_t *head_slow_cap, int32_t *head_kv_len,
+                          int32_t *head_fast_len, int32_t *moved_out, int32_t *slot_out,
+                          tg_stream stream);
+
 /* =====================================================================================
  * SplitZip: lossless BF16 codec for KV transfer ("SplitZip" explainer, arXiv 2605.01708, "Die
  * SplitZip-Strategie", "Warum es schnell ist"). A bf16 value is sign, 8-bit exponent and 7-bit

@@ -115,6 +115,8 @@ _SIGS = [
     ("tg_plan_cascade_units", ctypes.c_int, [_P, _P]),
     ("tg_tiered_append", ctypes.c_int, [ctypes.POINTER(tg_shape), _P, _P, _P, _P, _P, _P, _P, _P,
                                         _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    ("tg_tiered_append_int4", ctypes.c_int, [ctypes.POINTER(tg_shape), _P, _P, _P, _P, _P, _P, _P,
+                                             _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     ("tg_splitzip_workspace_bytes", _I64, [_I64]),
     ("tg_splitzip_encode", ctypes.c_int, [_I64, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _P]),
     ("tg_splitzip_decode", ctypes.c_int, [_I64, _P, _P, _P, _P, _P, _P, _I64, _P, _P]),
@@ -495,6 +497,19 @@ def tg_tiered_append(shape: tg_shape, k_new, v_new, k_fast, v_fast, fast_page_ta
         _dp(k_scale), _dp(v_scale), _dp(slow_page_table), _dp(slow_head_off),
         _dp(head_slow_cap), _dp(head_kv_len), _dp(head_fast_len), _dp(moved_out),
         _dp(slot_out), _stream(stream)), "tg_tiered_append")
+
+
+def tg_tiered_append_int4(shape: tg_shape, k_new, v_new, k_fast, v_fast, fast_page_table,
+                          fast_head_off, head_fast_cap, k_q4, v_q4, k_scale, v_scale,
+                          slow_page_table, slow_head_off, head_slow_cap, head_kv_len,
+                          head_fast_len, moved_out, slot_out, stream=None):
+    """tg_tiered_append into packed INT4 pools (see include/tg.h)."""
+    _check(_lib().tg_tiered_append_int4(
+        ctypes.byref(shape), _dp(k_new), _dp(v_new), _dp(k_fast), _dp(v_fast),
+        _dp(fast_page_table), _dp(fast_head_off), _dp(head_fast_cap), _dp(k_q4), _dp(v_q4),
+        _dp(k_scale), _dp(v_scale), _dp(slow_page_table), _dp(slow_head_off),
+        _dp(head_slow_cap), _dp(head_kv_len), _dp(head_fast_len), _dp(moved_out),
+        _dp(slot_out), _stream(stream)), "tg_tiered_append_int4")
 
 
 def tg_tiered_decode(plan: Plan, q, k_q8, v_q8, k_scale, v_scale, slow_page_table,

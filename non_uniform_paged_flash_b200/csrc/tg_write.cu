@@ -205,12 +205,15 @@ __global__ void __launch_bounds__(kUpdateThreads)
 // a free fast slot (f < cap, then all tokens are fast: n == f) it takes slot n; with a full
 // window the oldest fast token (position n - cap) is quantised (symmetric absmax INT8 per
 // token, the rule of tg_quantize_int8) into slow index n - cap, and the new token takes its slot.
+// BITS = 8: INT8 codes int8 [row][D]; BITS = 4: INT4 codes packed uint8 [row][D/2], byte i =
+// (code_i + 8) | (code_{i+D/2} + 8) << 4 (lane l < 16 packs its values with lane l + 16's).
+template <int BITS>
 __global__ void __launch_bounds__(kAppendWarps * 32)
     tier_append_kernel(int32_t BH, int32_t D, int64_t num_pages, int64_t num_slow_pages,
                        const __nv_bfloat16 *k_new, const __nv_bfloat16 *v_new,
                        __nv_bfloat16 *k_fast, __nv_bfloat16 *v_fast, const int32_t *fast_table,
-                       const int64_t *fast_off, const int32_t *fast_cap, int8_t *k_q8,
-                       int8_t *v_q8, float *k_scale, float *v_scale, const int32_t *slow_table,
+                       const int64_t *fast_off, const int32_t *fast_cap, void *k_q8,
+                       void *v_q8, float *k_scale, float *v_scale, const int32_t *slow_table,
                        const int64_t *slow_off, const int32_t *slow_cap, int32_t *kv_len,
                        int32_t *fast_len, int32_t *moved_out, int32_t *slot_out) {
     const int32_t bh = blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
@@ -246,8 +249,11 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
     if (fslot >= 0) {
         const int64_t frow = (fpid * 16 + fslot % 16) * D;
         if (sidx >= 0) {
-            // the leaving token's K and V rows -> INT8 codes + fp32 scale (read before overwrite)
+            // the leaving token's K and V rows -> INT8 / INT4 codes + fp32 scale (read before
+            // overwrite)
             const int64_t srow = spid * 16 + sidx % 16;
+            constexpr float kLevels = BITS == 4 ? 7.f : 127.f;
+            constexpr int kMax = BITS == 4 ? 7 : 127;
             for (int t = 0; t < 2; ++t) {
                 const __nv_bfloat16 *src = (t == 0 ? k_fast : v_fast) + frow;
                 float x[4];
@@ -259,13 +265,27 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
                     amax = fmaxf(amax, fabsf(x[k]));
                 }
                 for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-                const float sc = __fdiv_rn(amax, 127.f);
-                int8_t *codes = (t == 0 ? k_q8 : v_q8) + srow * D;
+                const float sc = __fdiv_rn(amax, kLevels);
+                int c[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    int v = 0;
-                    if (amax != 0.f) v = max(-127, min(127, __float2int_rn(__fdiv_rn(x[k], sc))));
-                    if (k < per) codes[lane * per + k] = static_cast<int8_t>(v);
+                    c[k] = 0;
+                    if (amax != 0.f) c[k] = max(-kMax, min(kMax, __float2int_rn(__fdiv_rn(x[k], sc))));
+                }
+                if (BITS == 8) {
+                    int8_t *codes = static_cast<int8_t *>(t == 0 ? k_q8 : v_q8) + srow * D;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (k < per) codes[lane * per + k] = static_cast<int8_t>(c[k]);
+                } else {
+                    // d = lane * per + k (< D/2) pairs with d + D/2, held by lane + 16
+                    uint8_t *packed = static_cast<uint8_t *>(t == 0 ? k_q8 : v_q8) + srow * (D / 2);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int hi = __shfl_down_sync(0xffffffffu, c[k], 16);
+                        if (lane < 16 && k < per)
+                            packed[lane * per + k] = static_cast<uint8_t>((c[k] + 8) | ((hi + 8) << 4));
+                    }
                 }
                 if (lane == 0) (t == 0 ? k_scale : v_scale)[srow] = sc;
             }
@@ -378,6 +398,38 @@ extern "C" int tg_h2o_update(const tg_shape *shape, int32_t recent, const float 
     return launch_status("h2o_update_kernel");
 }
 
+namespace tg {
+namespace {
+
+template <int BITS>
+int tiered_append(const tg_shape *shape, const void *k_new, const void *v_new, void *k_fast, void *v_fast,
+                  const int32_t *fast_page_table, const int64_t *fast_head_off, const int32_t *head_fast_cap,
+                  void *k_codes, void *v_codes, float *k_scale, float *v_scale, const int32_t *slow_page_table,
+                  const int64_t *slow_head_off, const int32_t *head_slow_cap, int32_t *head_kv_len,
+                  int32_t *head_fast_len, int32_t *moved_out, int32_t *slot_out, tg_stream stream) {
+    if (check_shape(shape) != TG_OK || shape->D % 32 != 0 || shape->D > 128 ||
+        shape->num_slow_pages < 0)
+        return TG_EINVAL;
+    const int32_t BH = shape->B * shape->Hkv;
+    if (BH == 0) return TG_OK;
+    if (!k_new || !v_new || !k_fast || !v_fast || !fast_page_table || !fast_head_off ||
+        !head_fast_cap || !k_codes || !v_codes || !k_scale || !v_scale || !slow_page_table ||
+        !slow_head_off || !head_slow_cap || !head_kv_len || !head_fast_len || !moved_out ||
+        !slot_out || !al16(k_new) || !al16(v_new) || !al16(k_fast) || !al16(v_fast))
+        return TG_EINVAL;
+    const unsigned grid = static_cast<unsigned>((BH + kAppendWarps - 1) / kAppendWarps);
+    tier_append_kernel<BITS><<<grid, kAppendWarps * 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        BH, shape->D, shape->num_pages, shape->num_slow_pages,
+        static_cast<const __nv_bfloat16 *>(k_new), static_cast<const __nv_bfloat16 *>(v_new),
+        static_cast<__nv_bfloat16 *>(k_fast), static_cast<__nv_bfloat16 *>(v_fast), fast_page_table,
+        fast_head_off, head_fast_cap, k_codes, v_codes, k_scale, v_scale, slow_page_table, slow_head_off,
+        head_slow_cap, head_kv_len, head_fast_len, moved_out, slot_out);
+    return launch_status("tier_append_kernel");
+}
+
+}  // namespace
+}  // namespace tg
+
 extern "C" int tg_tiered_append(const tg_shape *shape, const void *k_new, const void *v_new,
                                 void *k_fast, void *v_fast, const int32_t *fast_page_table,
                                 const int64_t *fast_head_off, const int32_t *head_fast_cap,
@@ -386,22 +438,20 @@ extern "C" int tg_tiered_append(const tg_shape *shape, const void *k_new, const 
                                 const int32_t *head_slow_cap, int32_t *head_kv_len,
                                 int32_t *head_fast_len, int32_t *moved_out, int32_t *slot_out,
                                 tg_stream stream) {
-    if (check_shape(shape) != TG_OK || shape->D % 32 != 0 || shape->D > 128 ||
-        shape->num_slow_pages < 0)
-        return TG_EINVAL;
-    const int32_t BH = shape->B * shape->Hkv;
-    if (BH == 0) return TG_OK;
-    if (!k_new || !v_new || !k_fast || !v_fast || !fast_page_table || !fast_head_off ||
-        !head_fast_cap || !k_q8 || !v_q8 || !k_scale || !v_scale || !slow_page_table ||
-        !slow_head_off || !head_slow_cap || !head_kv_len || !head_fast_len || !moved_out ||
-        !slot_out || !al16(k_new) || !al16(v_new) || !al16(k_fast) || !al16(v_fast))
-        return TG_EINVAL;
-    const unsigned grid = static_cast<unsigned>((BH + kAppendWarps - 1) / kAppendWarps);
-    tier_append_kernel<<<grid, kAppendWarps * 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        BH, shape->D, shape->num_pages, shape->num_slow_pages,
-        static_cast<const __nv_bfloat16 *>(k_new), static_cast<const __nv_bfloat16 *>(v_new),
-        static_cast<__nv_bfloat16 *>(k_fast), static_cast<__nv_bfloat16 *>(v_fast), fast_page_table,
-        fast_head_off, head_fast_cap, k_q8, v_q8, k_scale, v_scale, slow_page_table, slow_head_off,
-        head_slow_cap, head_kv_len, head_fast_len, moved_out, slot_out);
-    return launch_status("tier_append_kernel");
+    return tg::tiered_append<8>(shape, k_new, v_new, k_fast, v_fast, fast_page_table, fast_head_off,
+                                head_fast_cap, k_q8, v_q8, k_scale, v_scale, slow_page_table, slow_head_off,
+                                head_slow_cap, head_kv_len, head_fast_len, moved_out, slot_out, stream);
+}
+
+extern "C" int tg_tiered_append_int4(const tg_shape *shape, const void *k_new, const void *v_new,
+                                     void *k_fast, void *v_fast, const int32_t *fast_page_table,
+                                     const int64_t *fast_head_off, const int32_t *head_fast_cap,
+                                     uint8_t *k_q4, uint8_t *v_q4, float *k_scale, float *v_scale,
+                                     const int32_t *slow_page_table, const int64_t *slow_head_off,
+                                     const int32_t *head_slow_cap, int32_t *head_kv_len,
+                                     int32_t *head_fast_len, int32_t *moved_out, int32_t *slot_out,
+                                     tg_stream stream) {
+    return tg::tiered_append<4>(shape, k_new, v_new, k_fast, v_fast, fast_page_table, fast_head_off,
+                                head_fast_cap, k_q4, v_q4, k_scale, v_scale, slow_page_table, slow_head_off,
+                                head_slow_cap, head_kv_len, head_fast_len, moved_out, slot_out, stream);
 }

@@ -1,4 +1,4 @@
-"""GPU parity of the tier migration (fast window -> INT8 tier) and of the tiered decode of a
+"""GPU parity of the tier migration (fast window -> INT8 or INT4 tier) and of the tiered decode of a
 capacity plan (made once for the reserved sizes, valid as the tiers grow) against the oracle:
 slot choices, lengths and both tiers' pools bit for bit (the moved rows quantised by the pinned
 quantiser), the decode within 2e-2 / 1e-3 at several points of the growth.
@@ -31,7 +31,8 @@ def _bits(t):
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def test_tiered_append_and_capacity_decode():
+@pytest.mark.parametrize("bits", [8, 4])
+def test_tiered_append_and_capacity_decode(bits):
     sp = synth.small(5)                     # 2 sequences, 2100 tokens, 300 in the fast tier
     lay = workload.layout(sp, 0)
     ol = ors.layout(sp, 0)
@@ -52,14 +53,18 @@ def test_tiered_append_and_capacity_decode():
     # INT8 tier contents: seeded bf16 rows quantised by the library / by the oracle
     ks_bits = synth.pool_bits(sp, "kslow", Ps)
     vs_bits = synth.pool_bits(sp, "vslow", Ps)
-    kq_exp, ksc_exp = oracle.quantize_int8(ks_bits)
-    vq_exp, vsc_exp = oracle.quantize_int8(vs_bits)
-    kq = torch.empty((Ps, 16, sp.D), dtype=torch.int8, device="cuda")
+    quant = oracle.quantize_int4 if bits == 4 else oracle.quantize_int8
+    kq_exp, ksc_exp = quant(ks_bits)        # INT4: packed bytes
+    vq_exp, vsc_exp = quant(vs_bits)
+    codes = oracle.unpack_int4 if bits == 4 else (lambda x: x)
+    kq = torch.empty((Ps, 16, sp.D // 2 if bits == 4 else sp.D),
+                     dtype=torch.uint8 if bits == 4 else torch.int8, device="cuda")
     vq = torch.empty_like(kq)
     ksc = torch.empty((Ps, 16), dtype=torch.float32, device="cuda")
     vsc = torch.empty_like(ksc)
-    tg.tg_quantize_int8(_bf(ks_bits), kq, ksc)
-    tg.tg_quantize_int8(_bf(vs_bits), vq, vsc)
+    (tg.tg_quantize_int4 if bits == 4 else tg.tg_quantize_int8)(_bf(ks_bits), kq, ksc)
+    (tg.tg_quantize_int4 if bits == 4 else tg.tg_quantize_int8)(_bf(vs_bits), vq, vsc)
+    append = tg.tg_tiered_append_int4 if bits == 4 else tg.tg_tiered_append
     kf_exp = synth.pool_bits(sp, "k", ol.num_pages)
     vf_exp = synth.pool_bits(sp, "v", ol.num_pages)
     kf, vf = _bf(kf_exp), _bf(vf_exp)
@@ -75,7 +80,7 @@ def test_tiered_append_and_capacity_decode():
     # one capacity plan for the whole growth
     plan = tg.tg_plan_create(shape, f0 + S, lay.group_of_head, lay.group_off, fast_len=f0,
                              slow_table_len=Ps, num_workers=23, min_splits=8,
-                             max_chunk_pages=16, capacity=True)
+                             max_chunk_pages=16, capacity=True, slow_bits=bits)
     q_bits = synth.q_bits(sp)
     q = _bf(q_bits)
     out = torch.empty((B, sp.Hq, sp.D), dtype=torch.bfloat16, device="cuda")
@@ -89,7 +94,8 @@ def test_tiered_append_and_capacity_decode():
                             fl_dev, sp.scale, out, lse)
         torch.cuda.synchronize()
         assert tg.tg_plan_status(plan) == tg.TG_OK
-        ro, rl = oracle.tiered_decode(q_bits, kq_exp, vq_exp, ksc_exp, vsc_exp, slow_table,
+        ro, rl = oracle.tiered_decode(q_bits, codes(kq_exp), codes(vq_exp), ksc_exp, vsc_exp,
+                                      slow_table,
                                       slow_off, kf_exp, vf_exp, ol.table, ol.head_off,
                                       n.reshape(B, Hkv).astype(np.int32),
                                       f.reshape(B, Hkv).astype(np.int32), sp.scale)
@@ -101,8 +107,8 @@ def test_tiered_append_and_capacity_decode():
     check_decode()
     for step in range(T):
         kn, vn = synth.new_kv_bits(sp, step, "k"), synth.new_kv_bits(sp, step, "v")
-        tg.tg_tiered_append(shape, _bf(kn), _bf(vn), kf, vf, ftab, foff, fcap, kq, vq, ksc, vsc,
-                            stab, soff, scap, kv_dev, fl_dev, moved, slot)
+        append(shape, _bf(kn), _bf(vn), kf, vf, ftab, foff, fcap, kq, vq, ksc, vsc,
+               stab, soff, scap, kv_dev, fl_dev, moved, slot)
         want_fs, want_si = np.empty(B * Hkv, np.int32), np.empty(B * Hkv, np.int32)
         for bh in range(B * Hkv):
             fs, si = oracle.tier_step(int(n[bh]), int(f[bh]), cap, S)
@@ -113,7 +119,7 @@ def test_tiered_append_and_capacity_decode():
             if si >= 0:
                 spid = slow_table[soff_h[bh] + si // 16]
                 for src, q8, sc in ((kf_exp, kq_exp, ksc_exp), (vf_exp, vq_exp, vsc_exp)):
-                    c, s_ = oracle.quantize_int8(src[fpid, fs % 16][None, :])
+                    c, s_ = quant(src[fpid, fs % 16][None, :])
                     q8[spid, si % 16] = c[0]
                     sc[spid, si % 16] = s_[0]
             kf_exp[fpid, fs % 16] = kn[b, h]

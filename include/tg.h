@@ -8,7 +8,8 @@
  *     2 Ragged Paging, 3 Ahead-of-Time Load Balancing);
  *   - prefix pages shared across sequences through their page tables (RadixAttention lesson,
  *     Phase 17 · 06: the radix tree as KV index and its worked example);
- *   - a recent bf16 tier and an older INT8 tier dequantised inside the attention loop
+ *   - a recent bf16 tier and an older INT8 or INT4 tier dequantised inside the attention loop
+ *     (HBM-resident, or streamed block-wise from host memory)
  *     ("TTKV" explainer, arXiv 2604.19769: 核心方法 1 Tier Layout, 2 Tier Content,
  *     3 Tier Interaction);
  *   - split-K over each head's tokens merged by log-sum-exp (CAP survey, arXiv 2405.11299,
@@ -61,7 +62,7 @@ typedef struct tg_shape {
     int32_t page;           /* tokens per page (16) */
     int32_t reserved;       /* 0 */
     int64_t num_pages;      /* pages in the bf16 pools (k_pages, v_pages / k_fast, v_fast) */
-    int64_t num_slow_pages; /* pages in the INT8 pools (tiered decode only; else 0) */
+    int64_t num_slow_pages; /* pages in the INT8 / INT4 pools (tiered decode only; else 0) */
 } tg_shape;
 
 /* Human-readable text of a status code (static storage). */
@@ -355,7 +356,10 @@ int tg_ragged_paged_decode_noalloc(tg_plan *plan, const void *q, const void *k_p
  * digits, q = s_q (q1 + q2/254) (|error| <= max|q| / 64516 per element), exact in int32; INT8
  * V codes are converted exactly to fp16 in registers; the K scale multiplies the score and the
  * V scale multiplies the probability before P.V (both in fp32). plan from tg_plan_create with
- * this fast_len. D must be 128. */
+ * this fast_len. D must be 128. Plans with tg_plan_opts.slow_bits = 4 read an INT4 tier here
+ * instead (k_q8 / v_q8 then point to packed uint8 [num_slow_pages][16][D/2] pools of
+ * tg_quantize_int4): its K nibbles enter the same product (unsigned, offset corrected in
+ * int32), its V nibbles are widened exactly to fp16. */
 int tg_tiered_decode(tg_plan *plan, const void *q, const int8_t *k_q8, const int8_t *v_q8,
                      const float *k_scale, const float *v_scale, const int32_t *slow_page_table,
                      const int64_t *slow_head_off, const void *k_fast, const void *v_fast,

@@ -190,6 +190,12 @@ typedef struct tg_plan_opts {
                                  4 (D = 128 only): INT4 pools are uint8 [num_slow_pages][16][D/2]
                                  as tg_quantize_int4 writes them, passed where the INT8 calls
                                  take k_q8 / v_q8 */
+    int32_t whole_heads;      /* bf16 plans without a cascade: 1 = every head is one item (no
+                                 split heads, so no partials and no merge kernel), whole heads
+                                 placed on up to num_workers workers longest first; for small
+                                 batches, where a step is launch-bound. Ignored for tiered and
+                                 cascade plans; static_permille, min_splits and max_chunk_pages
+                                 do not apply */
 } tg_plan_opts;
 
 /* Build a plan. kv_len[B*Hkv] (host): retained tokens per (sequence, KV head); the decode

@@ -47,7 +47,8 @@ class tg_plan_opts(ctypes.Structure):
                 ("dyn_chunk_pages", ctypes.c_int32), ("early_prologue", ctypes.c_int32),
                 ("wait_limit_us", ctypes.c_int32), ("test_withhold_page", ctypes.c_int32),
                 ("capacity", ctypes.c_int32),
-                ("out_f32", ctypes.c_int32), ("slow_bits", ctypes.c_int32)]
+                ("out_f32", ctypes.c_int32), ("slow_bits", ctypes.c_int32),
+                ("whole_heads", ctypes.c_int32)]
 
 
 class tg_plan_info(ctypes.Structure):
@@ -320,14 +321,15 @@ def tg_plan_create(shape: tg_shape, kv_len, group_of_head, group_off, fast_len=N
                    static_permille: int = 0, dyn_chunk_pages: int = 0,
                    early_prologue: bool = False, wait_limit_us: int = 0,
                    test_withhold_page: int = 0, capacity: bool = False,
-                   out_f32: bool = False, slow_bits: int = 8) -> Plan:
+                   out_f32: bool = False, slow_bits: int = 8, whole_heads: bool = False) -> Plan:
     kv = _h(kv_len, np.int32).reshape(-1)
     fl = None if fast_len is None else _h(fast_len, np.int32).reshape(-1)
     goh = _h(group_of_head, np.int32).reshape(-1)
     goff = _h(group_off, np.int64).reshape(-1)
     opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
                         static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us,
-                        test_withhold_page, int(capacity), int(out_f32), int(slow_bits))
+                        test_withhold_page, int(capacity), int(out_f32), int(slow_bits),
+                        int(whole_heads))
     h = ctypes.c_void_p()
     _check(_lib().tg_plan_create(ctypes.byref(shape), _hp(kv), _hp(fl), _hp(goh), _hp(goff),
                                  goff.size - 1, slow_table_len, ctypes.byref(opts),

@@ -297,6 +297,43 @@ extern "C" int tg_place_sequences(int32_t n_seq, const int64_t *seq_bytes, int32
 // ------------------------------------------------------------------------------------------
 namespace tg {
 
+// Partial slots and the merge list: a head's items are consecutive in the list.
+// A cascade head's partials come first (slots first_slot .. first_slot + casc_cnt - 1, in
+// the order of its cascade runs), then its items'.
+static int finish_slots(tg_plan *p, const int32_t *casc_cnt) {
+    const int64_t BH = static_cast<int64_t>(p->shape.B) * p->shape.Hkv;
+    std::vector<int32_t> cnt(static_cast<size_t>(BH), 0), first(static_cast<size_t>(BH), -1);
+    for (size_t i = 0; i < p->items.size(); ++i) {
+        const int32_t bh = p->items[i].bh;
+        if (first[bh] < 0) first[bh] = static_cast<int32_t>(i);
+        ++cnt[bh];
+    }
+    p->merge.clear();
+    p->empties.clear();
+    p->merge_warps = 1;
+    int64_t slot = 0;
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        const int32_t cc = casc_cnt ? casc_cnt[bh] : 0;
+        const int32_t total = cnt[bh] + cc;
+        if (total == 0) {
+            p->empties.push_back(static_cast<int32_t>(bh));
+        } else if (total > 1 || cc > 0) {
+            const int32_t mi = static_cast<int32_t>(p->merge.size());
+            p->merge.push_back({static_cast<int32_t>(bh), static_cast<int32_t>(slot), total, 0});
+            slot += cc;
+            for (int32_t j = 0; j < cnt[bh]; ++j) {
+                Item &it = p->items[first[bh] + j];
+                it.slot = static_cast<int32_t>(slot++);
+                it.flags |= mi << 1;
+            }
+            // warps per merge CTA: up to 8 splits per warp, at most 32 warps
+            p->merge_warps = std::max(p->merge_warps, std::min(32, (total + 7) / 8));
+        }
+    }
+    p->n_partials = slot;
+    return TG_OK;
+}
+
 int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
                     int32_t num_workers, int32_t min_splits, int32_t max_chunk_pages,
                     int32_t static_permille, int32_t dyn_chunk_pages, const int32_t *pstart,
@@ -368,6 +405,49 @@ int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
         const Chunk &c = chunks[i];
         total_cost += static_cast<long double>(c.pe - c.pb) * c.page_cost;
         if (i == 0 || chunks[i - 1].bh != c.bh || chunks[i - 1].flags != c.flags) total_cost += item_cost;
+    }
+
+    if (p->whole_heads && !fast_len && !pstart) {
+        // Small bf16 batches: every head is one item (no split, so no partials and no merge
+        // kernel); heads go to workers longest first, each to the least loaded worker (ties:
+        // the lower index), one worker per head at most.
+        std::vector<int64_t> heads;
+        for (int64_t bh = 0; bh < BH; ++bh)
+            if (kv_len[bh] > 0) heads.push_back(bh);
+        std::stable_sort(heads.begin(), heads.end(), [&](int64_t x, int64_t y) { return kv_len[x] > kv_len[y]; });
+        const int64_t Wh = std::max<int64_t>(1, std::min<int64_t>(std::max(1, num_workers), static_cast<int64_t>(heads.size())));
+        std::vector<int64_t> load(static_cast<size_t>(Wh), 0);
+        std::vector<std::vector<int64_t>> of(static_cast<size_t>(Wh));
+        for (int64_t bh : heads) {
+            int64_t w = 0;
+            for (int64_t k = 1; k < Wh; ++k)
+                if (load[k] < load[w]) w = k;
+            load[w] += (kv_len[bh] + page - 1) / page;
+            of[w].push_back(bh);
+        }
+        p->items.clear();
+        p->worker_of_item.clear();
+        for (int64_t w = 0; w < Wh; ++w)
+            for (int64_t bh : of[w]) {
+                Item it{};
+                it.bh = static_cast<int32_t>(bh);
+                it.page_begin = 0;
+                it.page_end = (kv_len[bh] + page - 1) / page;
+                it.tier_tokens = kv_len[bh];
+                it.slot = -1;
+                it.flags = 0;
+                it.kv_len = kv_len[bh];
+                it.fast_len = 0;
+                p->items.push_back(it);
+                p->worker_of_item.push_back(static_cast<int32_t>(w));
+            }
+        p->n_workers = p->items.empty() ? 0 : static_cast<int32_t>(Wh);
+        p->worker_off.assign(static_cast<size_t>(p->n_workers) + 1, 0);
+        for (size_t i = 0; i < p->items.size(); ++i) p->worker_off[p->worker_of_item[i] + 1] = static_cast<int32_t>(i + 1);
+        for (int32_t i = 1; i <= p->n_workers; ++i) p->worker_off[i] = std::max(p->worker_off[i], p->worker_off[i - 1]);
+        p->dyn_first = static_cast<int32_t>(p->items.size());
+        p->n_dyn = 0;
+        return finish_slots(p, casc_cnt);
     }
 
     const bool hybrid = static_permille < 1000;
@@ -466,39 +546,7 @@ int build_work_list(tg_plan *p, const int32_t *kv_len, const int32_t *fast_len,
         p->worker_of_item.push_back(-1);
     }
 
-    // Partial slots and the merge list: a head's items are consecutive in the list.
-    // A cascade head's partials come first (slots first_slot .. first_slot + casc_cnt - 1, in
-    // the order of its cascade runs), then its items'.
-    std::vector<int32_t> cnt(static_cast<size_t>(BH), 0), first(static_cast<size_t>(BH), -1);
-    for (size_t i = 0; i < p->items.size(); ++i) {
-        const int32_t bh = p->items[i].bh;
-        if (first[bh] < 0) first[bh] = static_cast<int32_t>(i);
-        ++cnt[bh];
-    }
-    p->merge.clear();
-    p->empties.clear();
-    p->merge_warps = 1;
-    int64_t slot = 0;
-    for (int64_t bh = 0; bh < BH; ++bh) {
-        const int32_t cc = casc_cnt ? casc_cnt[bh] : 0;
-        const int32_t total = cnt[bh] + cc;
-        if (total == 0) {
-            p->empties.push_back(static_cast<int32_t>(bh));
-        } else if (total > 1 || cc > 0) {
-            const int32_t mi = static_cast<int32_t>(p->merge.size());
-            p->merge.push_back({static_cast<int32_t>(bh), static_cast<int32_t>(slot), total, 0});
-            slot += cc;
-            for (int32_t j = 0; j < cnt[bh]; ++j) {
-                Item &it = p->items[first[bh] + j];
-                it.slot = static_cast<int32_t>(slot++);
-                it.flags |= mi << 1;
-            }
-            // warps per merge CTA: up to 8 splits per warp, at most 32 warps
-            p->merge_warps = std::max(p->merge_warps, std::min(32, (total + 7) / 8));
-        }
-    }
-    p->n_partials = slot;
-    return TG_OK;
+    return finish_slots(p, casc_cnt);
 }
 
 }  // namespace tg
@@ -606,6 +654,7 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
     if (o.capacity && !fast_len) { delete p; return TG_EINVAL; }
     p->capacity = o.capacity != 0;
     p->out_f32 = o.out_f32 != 0;
+    p->whole_heads = o.whole_heads != 0;
     p->slow_bits = o.slow_bits == 0 ? 8 : o.slow_bits;
     if ((p->slow_bits != 8 && p->slow_bits != 4) || (p->slow_bits == 4 && (!fast_len || shape->D != 128))) {
         delete p;

@@ -94,6 +94,7 @@ struct tg_plan {
     bool capacity = false;            // see tg_plan_opts.capacity
     bool out_f32 = false;             // see tg_plan_opts.out_f32
     int32_t slow_bits = 8;            // see tg_plan_opts.slow_bits
+    bool whole_heads = false;         // see tg_plan_opts.whole_heads
     int32_t n_workers = 0;
     int64_t kv_bytes = 0;
 

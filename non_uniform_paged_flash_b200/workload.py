@@ -221,7 +221,8 @@ def timed_plan_options(cfg: int) -> dict:
     plan and tables before the previous step's merge kernel has finished)."""
     kw = dict(early_prologue=True)
     if cfg == 1:
-        kw.update(static_permille=1000)
+        # one tiny batch: whole heads, so a step is one launch (no split head, no merge)
+        kw.update(whole_heads=True)
     elif cfg == 2:
         kw.update(static_permille=850, dyn_chunk_pages=16)
     elif cfg == 3:
@@ -260,7 +261,7 @@ def to_device(sp: synth.Spec, lay: Layout, layer: int = 0, device="cuda", num_wo
               min_splits: int = 1, max_chunk_pages: int = 0, seqs=None, static_permille: int = 0,
               dyn_chunk_pages: int = 0, early_prologue: bool = False, wait_limit_us: int = 0,
               test_withhold_page: int = 0, cascade: bool = False,
-              min_readers: int = 2) -> DeviceBatch:
+              min_readers: int = 2, whole_heads: bool = False) -> DeviceBatch:
     import torch
     dev = torch.device(device)
     B = lay.kv_len.shape[0]
@@ -283,7 +284,8 @@ def to_device(sp: synth.Spec, lay: Layout, layer: int = 0, device="cuda", num_wo
                               dyn_chunk_pages=dyn_chunk_pages, early_prologue=early_prologue,
                               wait_limit_us=wait_limit_us, test_withhold_page=test_withhold_page,
                               device=dev.index if dev.index is not None else -1,
-                              slow_bits=sp.slow_bits if lay.fast_len is not None else 8)
+                              slow_bits=sp.slow_bits if lay.fast_len is not None else 8,
+                              whole_heads=whole_heads)
     qb = synth.q_bits(sp, layer)
     q = _bf16_tensor(qb if seqs is None else np.ascontiguousarray(qb[seqs]), dev)
     out = torch.empty((B, sp.Hq, sp.D), dtype=torch.bfloat16, device=dev)

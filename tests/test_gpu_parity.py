@@ -61,6 +61,15 @@ def test_small_configs_match_oracle(cfg, workers, static_permille):
         _run(sp, layer, **kw)
 
 
+@pytest.mark.parametrize("cfg", [1, 2])
+@pytest.mark.parametrize("workers", [0, 3])
+def test_whole_head_plans_match_oracle(cfg, workers):
+    """whole_heads plans: one item per head, no merge kernel."""
+    sp = synth.small(cfg)
+    db, _ = _run(sp, num_workers=workers, whole_heads=True)
+    assert tg.tg_plan_get_info(db.plan)["n_merge"] == 0
+
+
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 @pytest.mark.parametrize("D", [64, 128])
 def test_gqa_and_head_dims(G, D):

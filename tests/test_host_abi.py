@@ -352,3 +352,38 @@ def test_plan_slow_bits_validation():
         with pytest.raises(tg.TGError) as ei:
             tg.tg_plan_create(shape, lay.kv_len, lay.group_of_head, lay.group_off, **bad)
         assert ei.value.status == tg.TG_EINVAL
+
+
+def test_whole_heads_plan():
+    """whole_heads: one item per non-empty head (every page once, no partials, no merge),
+    heads placed longest first on the least-loaded worker; tiered plans ignore it."""
+    rng = np.random.default_rng(61)
+    B, Hq, Hkv, D = 3, 8, 4, 128
+    kv = rng.integers(0, 300, (B, Hkv)).astype(np.int32)
+    kv[1, 2] = 0
+    goh = np.zeros(Hkv, np.int32)
+    pages = -(-kv // 16)
+    goff = np.array([0, int(pages.max()) * B * Hkv], np.int64)
+    shape = tg.make_shape(B, Hq, Hkv, D, int(pages.sum()) + 1)
+    for W in (1, 3, 64):
+        p = tg.tg_plan_create(shape, kv, goh, goff, host_only=True, num_workers=W, whole_heads=True)
+        info = tg.tg_plan_get_info(p)
+        items = tg.tg_plan_items(p)
+        nonempty = int((kv > 0).sum())
+        assert info["n_items"] == nonempty and info["n_merge"] == 0 and info["n_partials"] == 0
+        assert info["n_empty"] == B * Hkv - nonempty and info["n_dynamic"] == 0
+        assert info["n_workers"] == min(W, nonempty)
+        assert sorted(items[:, 0].tolist()) == sorted(np.nonzero(kv.reshape(-1))[0].tolist())
+        for it in items:
+            assert it[1] == 0 and it[2] == pages.reshape(-1)[it[0]] and it[4] == -1
+        # LPT: no worker could take a head from the most-loaded one and end below it
+        load = np.zeros(info["n_workers"], np.int64)
+        for it in items:
+            load[it[6]] += it[2]
+        assert load.max() - load.min() <= pages.max()
+    # tiered plans: the option is ignored (the usual split-K list)
+    fl = np.minimum(kv, 40).astype(np.int32)
+    shape_t = tg.make_shape(B, Hq, Hkv, D, int(pages.sum()) + 1, int(pages.sum()) + 1)
+    pt = tg.tg_plan_create(shape_t, kv, goh, goff, fast_len=fl, slow_table_len=int(goff[1]),
+                           host_only=True, num_workers=64, min_splits=4, whole_heads=True)
+    assert tg.tg_plan_get_info(pt)["n_merge"] > 0

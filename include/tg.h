@@ -209,8 +209,9 @@ typedef struct tg_plan_opts {
  * num_workers equal contiguous ranges assigned ahead of time (at least ~8 pages per worker;
  * fewer workers for tiny batches); the rest is cut into dynamic items of at most
  * dyn_chunk_pages pages that workers take from a shared ticket when their own range is done
- * (absorbing per-SM bandwidth differences). A head cut into several items is merged
- * by log-sum-exp inside the decode kernel.
+ * (absorbing per-SM bandwidth differences). A head cut into several items is merged by
+ * log-sum-exp in split order by a second kernel that the decode call launches as a
+ * programmatic dependent (its launch overlaps the decode's tail).
  * The plan owns one device allocation (work list, merge list, partial results, error word),
  * made here; nothing is allocated per call. */
 int tg_plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,

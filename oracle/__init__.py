@@ -1,7 +1,7 @@
 """CPU oracle for ragged / prefix-shared / tiered paged decode attention.
 
 TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU
-baseline leg may import this package. The product (``non_uniform_paged_flash_b200``) never
+baseline leg and reference arm may import this package. The product (``non_uniform_paged_flash_b200``) never
 imports it, and the two share no code.
 
 The arithmetic lives in ``tg_oracle.c`` (plain loops, fp64 attention); this module only

@@ -2,7 +2,7 @@
  * CPU ORACLE for ragged / prefix-shared / tiered paged decode attention.
  *
  * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the bench's CPU-baseline leg
- * may load this library. The product path (the CUDA library and its Python binding) never
+ * and reference arm may load this library. The product path (the CUDA library and its Python binding) never
  * calls it, and the two share no code: no headers, helpers, tables or constants.
  *
  * Plain, slow and written to be checked by eye: straight loops in the order the sources
@@ -20,6 +20,8 @@
  *             §2.4.3 分布式加速, "加速单个请求" (online normaliser) and Fig. 5 (Dist Attention).
  *  [Radix]    "RadixAttention and KV reuse" lesson (Phase 17 · 06), section on the radix tree
  *             as KV index and its worked example tree.
+ *  [SplitZip] "SplitZip: Ultra Fast Lossless KV Compression for Disaggregated LLM Serving"
+ *             (explainer of arXiv 2605.01708), "Die SplitZip-Strategie", "Warum es schnell ist".
  *
  * Functions whose parity is pinned, and by what, are listed in the test suite
  * (tests/test_oracle_pins.py); none of the functions here is unpinned.

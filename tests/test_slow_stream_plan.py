@@ -70,3 +70,30 @@ def test_bad_page_id_is_rejected():
     with pytest.raises(tg.TGError) as ei:
         _stream(replace(lay, slow_table=bad), sp, 4)
     assert ei.value.status == tg.TG_EINVAL
+
+
+def test_blocks_do_not_depend_on_code_width():
+    """INT4 and INT8 slow tiers stream the same blocks and tokens (only the bytes differ)."""
+    sp = synth.small(5)
+    lay = workload.layout(sp, 0)
+    B = lay.kv_len.shape[0]
+    shape = tg.make_shape(B, sp.Hq, sp.Hkv, sp.D, lay.num_pages, lay.num_slow_pages, sp.page)
+    got = []
+    for bits in (8, 4):
+        ss = tg.SlowStream(shape, lay.kv_len, lay.fast_len, lay.group_of_head, lay.group_off,
+                           lay.slow_table, lay.slow_off, 7, 2, num_workers=64, host_only=True,
+                           slow_bits=bits)
+        got.append(ss.blocks())
+    for a, b in zip(*got):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_algorithmic_bytes_int4_closed_form():
+    """Per slow token-head 2 (D/2 + 4) bytes for INT4 and 2 (D + 4) for INT8; fast 4 D."""
+    sp = synth.small(5)
+    lay = workload.layout(sp, 0)
+    kv = lay.kv_len.astype(np.int64)
+    f = np.minimum(lay.fast_len.astype(np.int64), kv)
+    for bits, row in ((8, sp.D), (4, sp.D // 2)):
+        alg = workload.algorithmic_bytes(replace(sp, slow_bits=bits), lay)
+        assert alg["kv"] == int((kv - f).sum()) * 2 * (row + 4) + int(f.sum()) * 4 * sp.D

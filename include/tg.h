@@ -390,7 +390,8 @@ typedef struct tg_host_pipe tg_host_pipe;
 
 /* Create a pipe for calls on plans of `plan`'s shape (B, Hq, D) and device. Allocates
  * 2 x (2 B*Hq*D*2 + B*Hq*4) bytes of device memory, two streams and six events.
- * TG_EINVAL for a host-only plan; TG_ENOMEM; TG_ECUDA. */
+ * TG_EINVAL for a host-only plan or one with tg_plan_opts.out_f32 (the pipe carries bf16
+ * outputs; calls with such a plan are rejected too); TG_ENOMEM; TG_ECUDA. */
 int tg_host_pipe_create(const tg_plan *plan, tg_host_pipe **out);
 /* Wait for the pipe's copies, then free it. NULL is ignored. */
 void tg_host_pipe_destroy(tg_host_pipe *p);

@@ -47,9 +47,10 @@ void release(tg_host_pipe *p) {
     delete p;
 }
 
+// The staging sets hold bf16 outputs: plans that write fp32 outputs are not served.
 bool same_shape(const tg_host_pipe *p, const tg_plan *plan) {
     return plan->shape.B == p->B && plan->shape.Hq == p->Hq && plan->shape.D == p->D &&
-           plan->device == p->device;
+           plan->device == p->device && !plan->out_f32;
 }
 
 // Steps before the decode of one call: returns the staging set, or -1 after a CUDA error.
@@ -84,7 +85,7 @@ int stage_out(tg_host_pipe *p, int s, void *out_host, float *lse_host, cudaStrea
 extern "C" int tg_host_pipe_create(const tg_plan *plan, tg_host_pipe **out) {
     if (!plan || !out) return TG_EINVAL;
     *out = nullptr;
-    if (plan->host_only) return TG_EINVAL;
+    if (plan->host_only || plan->out_f32) return TG_EINVAL;
     tg_host_pipe *p = new (std::nothrow) tg_host_pipe();
     if (!p) return TG_ENOMEM;
     p->device = plan->device;

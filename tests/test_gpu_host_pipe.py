@@ -89,6 +89,16 @@ def test_pipe_rejects_mismatch_and_pageable():
                                        other.head_off, other.kv_len, other.group_of_head,
                                        other.spec.scale, out, lse)
     assert ei.value.status == tg.TG_EINVAL
+    B = db.lay.kv_len.shape[0]
+    shape = tg.make_shape(B, sp.Hq, sp.Hkv, sp.D, db.lay.num_pages)
+    p32 = tg.tg_plan_create(shape, db.lay.kv_len, db.lay.group_of_head, db.lay.group_off,
+                            out_f32=True)
+    with pytest.raises(tg.TGError) as e32:       # fp32 outputs do not fit the bf16 staging
+        tg.tg_ragged_paged_decode_host(pipe, p32, q, db.k, db.v, db.table, db.head_off,
+                                       db.kv_len, db.group_of_head, sp.scale, out, lse)
+    assert e32.value.status == tg.TG_EINVAL
+    with pytest.raises(tg.TGError):
+        tg.HostPipe(p32)
     with pytest.raises(ValueError):
         db.run_host(pipe, db.q.cpu(), out, lse)   # pageable q
     with pytest.raises(ValueError):

@@ -187,6 +187,29 @@ def _dp(t):
     return t.data_ptr()
 
 
+def _need(t, n, dtype, what):
+    """A tensor argument holds at least n elements of dtype (the C ABI takes bare pointers)."""
+    import torch
+    if t is None:
+        raise ValueError(f"{what}: missing")
+    if t.dtype != dtype:
+        raise ValueError(f"{what}: expected {dtype}, got {t.dtype}")
+    if t.numel() < n:
+        raise ValueError(f"{what}: {t.numel()} elements, the plan needs {n}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what}: must be contiguous")
+
+
+def _check_io(plan, q, out, lse):
+    """q bf16 [B][Hq][D]; out bf16 (fp32 for out_f32 plans) [B][Hq][D]; lse fp32 [B][Hq]."""
+    import torch
+    s = plan.shape
+    rows = s.B * s.Hq
+    _need(q, rows * s.D, torch.bfloat16, "q")
+    _need(out, rows * s.D, torch.float32 if plan.out_f32 else torch.bfloat16, "out")
+    _need(lse, rows, torch.float32, "lse")
+
+
 def _stream(stream):
     if stream is not None:
         return stream if isinstance(stream, int) else stream.cuda_stream
@@ -298,6 +321,7 @@ class Plan:
     handle: ctypes.c_void_p
     shape: tg_shape
     tiered: bool
+    out_f32: bool = False
 
     def destroy(self):
         if self.handle:
@@ -334,7 +358,7 @@ def tg_plan_create(shape: tg_shape, kv_len, group_of_head, group_off, fast_len=N
     _check(_lib().tg_plan_create(ctypes.byref(shape), _hp(kv), _hp(fl), _hp(goh), _hp(goff),
                                  goff.size - 1, slow_table_len, ctypes.byref(opts),
                                  ctypes.byref(h)), "tg_plan_create")
-    return Plan(h, shape, fl is not None)
+    return Plan(h, shape, fl is not None, bool(out_f32))
 
 
 def tg_plan_create_cascade(shape: tg_shape, kv_len, group_of_head, group_off, page_table,
@@ -357,7 +381,7 @@ def tg_plan_create_cascade(shape: tg_shape, kv_len, group_of_head, group_off, pa
                                          goff.size - 1, _hp(tbl), _hp(hoff), tbl.size,
                                          int(min_readers), ctypes.byref(opts), ctypes.byref(h)),
            "tg_plan_create_cascade")
-    return Plan(h, shape, False)
+    return Plan(h, shape, False, bool(out_f32))
 
 
 def tg_plan_cascade_units(plan: Plan):
@@ -429,6 +453,7 @@ def tg_plan_trace_read(plan: Plan, stream=None) -> np.ndarray:
 
 def tg_ragged_paged_decode(plan: Plan, q, k_pages, v_pages, page_table, head_page_off,
                            head_kv_len, group_of_head, scale: float, out, lse, stream=None):
+    _check_io(plan, q, out, lse)
     _check(_lib().tg_ragged_paged_decode(
         plan.handle, _dp(q), _dp(k_pages), _dp(v_pages), _dp(page_table), _dp(head_page_off),
         _dp(head_kv_len), _dp(group_of_head), float(scale), _dp(out), _dp(lse),
@@ -440,6 +465,7 @@ def tg_ragged_paged_decode_noalloc(plan: Plan, q, k_pages, v_pages, page_table, 
                                    stream=None):
     """As tg_ragged_paged_decode, for callers that cannot allocate device memory: the plan may
     be host-only; the scratch is the library's fixed 16 MiB device array."""
+    _check_io(plan, q, out, lse)
     _check(_lib().tg_ragged_paged_decode_noalloc(
         plan.handle, _dp(q), _dp(k_pages), _dp(v_pages), _dp(page_table), _dp(head_page_off),
         _dp(head_kv_len), _dp(group_of_head), float(scale), _dp(out), _dp(lse),
@@ -451,6 +477,7 @@ def tg_ragged_paged_decode_scores(plan: Plan, q, k_pages, v_pages, page_table, h
                                   token_scores, stream=None):
     """As tg_ragged_paged_decode, also writing every retained token's scores
     s = scale * q . K_t to token_scores (fp32 [table_len * 16, G])."""
+    _check_io(plan, q, out, lse)
     _check(_lib().tg_ragged_paged_decode_scores(
         plan.handle, _dp(q), _dp(k_pages), _dp(v_pages), _dp(page_table), _dp(head_page_off),
         _dp(head_kv_len), _dp(group_of_head), float(scale), _dp(out), _dp(lse),
@@ -517,6 +544,7 @@ def tg_tiered_append_int4(shape: tg_shape, k_new, v_new, k_fast, v_fast, fast_pa
 def tg_tiered_decode(plan: Plan, q, k_q8, v_q8, k_scale, v_scale, slow_page_table,
                      slow_head_off, k_fast, v_fast, fast_page_table, fast_head_off, head_kv_len,
                      head_fast_len, scale: float, out, lse, stream=None):
+    _check_io(plan, q, out, lse)
     _check(_lib().tg_tiered_decode(
         plan.handle, _dp(q), _dp(k_q8), _dp(v_q8), _dp(k_scale), _dp(v_scale),
         _dp(slow_page_table), _dp(slow_head_off), _dp(k_fast), _dp(v_fast),

@@ -231,10 +231,14 @@ def test_bounded_wait_runs_out_and_context_survives():
 def test_argument_validation():
     sp = synth.small(1)
     db = workload.admit(sp)
+    big = torch.empty(db.out.numel() + 8, dtype=db.out.dtype, device=db.out.device)
     with pytest.raises(tg.TGError) as e:
         tg.tg_ragged_paged_decode(db.plan, db.q, db.k, db.v, db.table, db.head_off, db.kv_len,
+                                  db.group_of_head, sp.scale, big[1:1 + db.out.numel()], db.lse)
+    assert e.value.status == tg.TG_EINVAL          # misaligned output (the C ABI's check)
+    with pytest.raises(ValueError):                 # too small (the binding's check)
+        tg.tg_ragged_paged_decode(db.plan, db.q, db.k, db.v, db.table, db.head_off, db.kv_len,
                                   db.group_of_head, sp.scale, db.out.view(-1)[1:], db.lse)
-    assert e.value.status == tg.TG_EINVAL          # misaligned output
     with pytest.raises(tg.TGError):
         tg.tg_tiered_decode(db.plan, db.q, None, None, None, None, None, None, db.k, db.v,
                             db.table, db.head_off, db.kv_len, db.kv_len, sp.scale, db.out, db.lse)

@@ -387,3 +387,26 @@ def test_whole_heads_plan():
     pt = tg.tg_plan_create(shape_t, kv, goh, goff, fast_len=fl, slow_table_len=int(goff[1]),
                            host_only=True, num_workers=64, min_splits=4, whole_heads=True)
     assert tg.tg_plan_get_info(pt)["n_merge"] > 0
+
+
+def test_decode_wrappers_check_sizes_and_dtypes():
+    """The binding checks q / out / lse against the plan before any pointer crosses the ABI."""
+    import torch
+    sp = synth.small(2)
+    lay = workload.layout(sp, 0)
+    B = lay.kv_len.shape[0]
+    shape = tg.make_shape(B, sp.Hq, sp.Hkv, sp.D, lay.num_pages)
+    p = tg.tg_plan_create(shape, lay.kv_len, lay.group_of_head, lay.group_off, host_only=True,
+                          num_workers=64)
+    rows = B * sp.Hq
+    q = torch.zeros(rows * sp.D, dtype=torch.bfloat16)
+    out = torch.zeros(rows * sp.D, dtype=torch.bfloat16)
+    lse = torch.zeros(rows, dtype=torch.float32)
+    args = (None, None, None, None, None, None, sp.scale)
+    for bad in ((q[1:], out, lse), (q, out.float(), lse), (q, out, lse[1:]), (q.float(), out, lse)):
+        with pytest.raises(ValueError):
+            tg.tg_ragged_paged_decode(p, bad[0], *args[:6], args[6], bad[1], bad[2])
+    p32 = tg.tg_plan_create(shape, lay.kv_len, lay.group_of_head, lay.group_off, host_only=True,
+                            num_workers=64, out_f32=True)
+    with pytest.raises(ValueError):                   # an fp32-output plan takes fp32 out
+        tg.tg_ragged_paged_decode(p32, q, *args[:6], args[6], out, lse)

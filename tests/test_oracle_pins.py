@@ -500,6 +500,7 @@ def _run_sink_recent(budget, sink, kv_len, slot_pos, new_positions):
     slots = []
     for p in new_positions:
         s = oracle.sink_recent_slot(budget, sink, n, np.array(pos[:max(n, 1)], np.int32))
+        assert 0 <= s < budget, (budget, sink, n)    # a head with budget >= 1 always takes a slot
         slots.append(s)
         pos[s] = p
         n = max(n, s + 1)
@@ -511,6 +512,15 @@ def test_sink_recent_golden():
         slots, final = _run_sink_recent(c["budget"], c["sink"], c["kv_len"], c["slot_pos"], c["new_pos"])
         assert slots == c["slots"], c["work"]
         assert final == c["final_pos"], c["work"]
+
+
+def test_sink_recent_sinks_never_fill_the_budget():
+    """At most budget - 1 sinks: with sink >= budget one slot still turns over (hand-worked:
+    budget 3, sink 5, positions 0, 1, 2 in slots 0-2; sinks are positions 0 and 1, so the new
+    position 3 replaces position 2 in slot 2, then position 4 replaces 3 in slot 2)."""
+    slots, final = _run_sink_recent(3, 5, 3, [0, 1, 2], [3, 4])
+    assert slots == [2, 2] and final == [0, 1, 4]
+    assert oracle.sink_recent_slot(1, 3, 1, np.array([7], np.int32)) == 0   # budget 1: no sink
 
 
 def test_sink_recent_keeps_first_and_last_tokens():

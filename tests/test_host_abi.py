@@ -410,3 +410,31 @@ def test_decode_wrappers_check_sizes_and_dtypes():
                             num_workers=64, out_f32=True)
     with pytest.raises(ValueError):                   # an fp32-output plan takes fp32 out
         tg.tg_ragged_paged_decode(p32, q, *args[:6], args[6], out, lse)
+
+
+def test_new_entries_reject_bad_arguments_without_a_gpu():
+    """Argument checks that run before any device work: slow stream geometry, SplitZip sizes,
+    host pipe on a host-only plan, INT4 append shape."""
+    sp = synth.small(5)
+    lay = workload.layout(sp, 0)
+    B = lay.kv_len.shape[0]
+    shape = tg.make_shape(B, sp.Hq, sp.Hkv, sp.D, lay.num_pages, lay.num_slow_pages, sp.page)
+    ok = dict(num_workers=64, host_only=True)
+    for block_pages, ring in ((0, 2), (4, 0)):
+        with pytest.raises(tg.TGError) as e:
+            tg.SlowStream(shape, lay.kv_len, lay.fast_len, lay.group_of_head, lay.group_off,
+                          lay.slow_table, lay.slow_off, block_pages, ring, **ok)
+        assert e.value.status == tg.TG_EINVAL
+    bad_fl = lay.fast_len.copy()
+    bad_fl[0, 0] = -1
+    with pytest.raises(tg.TGError):
+        tg.SlowStream(shape, lay.kv_len, bad_fl, lay.group_of_head, lay.group_off,
+                      lay.slow_table, lay.slow_off, 4, 2, **ok)
+    assert tg.tg_splitzip_workspace_bytes(-1) == -1
+    assert tg.tg_splitzip_workspace_bytes(0) > 0
+    assert tg.tg_splitzip_workspace_bytes(1 << 20) >= (1 << 20) // 8
+    hp = tg.tg_plan_create(tg.make_shape(B, sp.Hq, sp.Hkv, sp.D, lay.num_pages), lay.kv_len,
+                           lay.group_of_head, lay.group_off, **ok)
+    with pytest.raises(tg.TGError) as e:
+        tg.HostPipe(hp)
+    assert e.value.status == tg.TG_EINVAL

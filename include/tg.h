@@ -213,7 +213,10 @@ typedef struct tg_plan_opts {
  * log-sum-exp in split order by a second kernel that the decode call launches as a
  * programmatic dependent (its launch overlaps the decode's tail).
  * The plan owns one device allocation (work list, merge list, partial results, error word),
- * made here; nothing is allocated per call. */
+ * made here; nothing is allocated per call. Returns TG_EINVAL for bad arguments,
+ * TG_EUNSUPPORTED for a shape the kernels do not serve (page != 16, D not 64 or 128, Hq/Hkv
+ * not 1, 2, 4 or 8, a tiered plan with D != 128); on any error *out is NULL and nothing is
+ * left allocated. */
 int tg_plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,
                    const int32_t *group_of_head, const int64_t *group_off, int32_t n_groups,
                    int64_t slow_table_len, const tg_plan_opts *opts, tg_plan **out);

@@ -135,7 +135,7 @@ extern "C" int tg_alloc_share_segment(tg_alloc *a, int32_t n_tokens, int32_t n_h
         a->refs[p] = 1;  // the segment's own reference
         s.pages.push_back(p);
     }
-    if (page_ids) std::memcpy(page_ids, s.pages.data(), sizeof(int32_t) * static_cast<size_t>(need));
+    if (page_ids && need > 0) std::memcpy(page_ids, s.pages.data(), sizeof(int32_t) * static_cast<size_t>(need));
     *seg_id = static_cast<int32_t>(a->segs.size());
     a->segs.push_back(std::move(s));
     return TG_OK;
@@ -619,7 +619,9 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
                 const int32_t *group_of_head, const int64_t *group_off, int32_t n_groups,
                 int64_t slow_table_len, const tg_plan_opts *opts, const int32_t *table,
                 const int64_t *head_off, int64_t table_len, int32_t min_readers, tg_plan **out) {
-    if (!shape || !kv_len || !out || !group_of_head || !group_off || n_groups < 1) return TG_EINVAL;
+    if (!out) return TG_EINVAL;
+    *out = nullptr;
+    if (!shape || !kv_len || !group_of_head || !group_off || n_groups < 1) return TG_EINVAL;
     const tg_shape &s = *shape;
     if (s.B < 0 || s.Hkv < 1 || s.Hq < 1 || s.Hq % s.Hkv != 0 || s.D < 1 || s.page < 1 ||
         s.num_pages < 0 || s.num_slow_pages < 0)

@@ -1,0 +1,30 @@
+"""The library's host code (allocator, group tables, planner, placement) built with
+AddressSanitizer and UndefinedBehaviorSanitizer and driven on seeded random inputs
+(tests/native/host_fuzz.cpp); no GPU involved."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
+def test_host_code_is_clean_under_asan_and_ubsan():
+    out_dir = os.path.join(ROOT, "tests", "native", "_build")   # git-ignored
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "host_fuzz")
+    cmd = ["g++", "-std=c++17", "-O1", "-g", "-fsanitize=address,undefined",
+           "-fno-sanitize-recover=undefined", "-fno-omit-frame-pointer",
+           "-I", os.path.join(ROOT, "include"),
+           "-I", os.path.join(ROOT, "non_uniform_paged_flash_b200", "csrc"),
+           os.path.join(ROOT, "tests", "native", "host_fuzz.cpp"),
+           os.path.join(ROOT, "non_uniform_paged_flash_b200", "csrc", "tg_host.cpp"),
+           "-o", str(exe)]
+    subprocess.check_call(cmd)
+    env = dict(os.environ, ASAN_OPTIONS="detect_leaks=1:abort_on_error=0",
+               UBSAN_OPTIONS="print_stacktrace=1")
+    r = subprocess.run([str(exe), "200"], capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, (r.stdout + r.stderr)[-4000:]
+    assert "rounds clean" in r.stdout

@@ -4,7 +4,7 @@
 #include <algorithm>
 #include <climits>
 #include <cstring>
-#include <deque>
+#include <memory>
 #include <new>
 #include <numeric>
 #include <unordered_map>
@@ -53,14 +53,16 @@ extern "C" int tg_retained_lengths(int64_t n, const int32_t *full_len, const int
 // ------------------------------------------------------------------------------------------
 extern "C" int tg_budget_groups(int32_t n, const int32_t *budget_ppm, int32_t n_groups,
                                 int32_t *group_of_head) {
-    if (n <= 0 || !budget_ppm || !group_of_head || n_groups < 1 || n_groups > n) return TG_EINVAL;
-    std::vector<int32_t> order(n);
-    std::iota(order.begin(), order.end(), 0);
-    std::stable_sort(order.begin(), order.end(),
-                     [&](int32_t a, int32_t b) { return budget_ppm[a] < budget_ppm[b]; });
-    for (int32_t pos = 0; pos < n; ++pos)
-        group_of_head[order[pos]] = static_cast<int32_t>(static_cast<int64_t>(pos) * n_groups / n);
-    return TG_OK;
+    return tg::no_throw([&] {
+        if (n <= 0 || !budget_ppm || !group_of_head || n_groups < 1 || n_groups > n) return TG_EINVAL;
+        std::vector<int32_t> order(n);
+        std::iota(order.begin(), order.end(), 0);
+        std::stable_sort(order.begin(), order.end(),
+                         [&](int32_t a, int32_t b) { return budget_ppm[a] < budget_ppm[b]; });
+        for (int32_t pos = 0; pos < n; ++pos)
+            group_of_head[order[pos]] = static_cast<int32_t>(static_cast<int64_t>(pos) * n_groups / n);
+        return TG_OK;
+    });
 }
 
 // ------------------------------------------------------------------------------------------
@@ -69,7 +71,10 @@ extern "C" int tg_budget_groups(int32_t n, const int32_t *budget_ppm, int32_t n_
 struct tg_alloc {
     int64_t num_pages = 0;
     int32_t page = 16;
-    std::deque<int32_t> free_list;
+    // Free pages in FIFO order: a ring of num_pages entries (a page is in it at most once), so
+    // that returning a page never allocates.
+    std::vector<int32_t> ring;
+    int64_t head = 0, n_free = 0;
     std::vector<int32_t> refs;
     struct Segment {
         int32_t n_heads = 0, full = 0;
@@ -83,68 +88,69 @@ struct tg_alloc {
     };
     std::unordered_map<int32_t, Seq> seqs;
 
+    int32_t take() {
+        const int32_t p = ring[head];
+        head = head + 1 == num_pages ? 0 : head + 1;
+        --n_free;
+        return p;
+    }
+    void give(int32_t p) {
+        int64_t at = head + n_free;
+        if (at >= num_pages) at -= num_pages;
+        ring[at] = p;
+        ++n_free;
+    }
     void unref(int32_t p) {
-        if (--refs[p] == 0) free_list.push_back(p);
+        if (--refs[p] == 0) give(p);
     }
 };
 
-extern "C" int tg_alloc_create(int64_t num_pages, int32_t page, const int32_t *free_order,
-                               tg_alloc **out) {
+namespace {
+
+int alloc_create(int64_t num_pages, int32_t page, const int32_t *free_order, tg_alloc **out) {
     if (!out || num_pages < 1 || num_pages > INT32_MAX || page < 1) return TG_EINVAL;
-    tg_alloc *a = new (std::nothrow) tg_alloc;
-    if (!a) return TG_ENOMEM;
+    std::unique_ptr<tg_alloc> a(new tg_alloc);
     a->num_pages = num_pages;
     a->page = page;
     a->refs.assign(static_cast<size_t>(num_pages), 0);
+    a->ring.assign(static_cast<size_t>(num_pages), 0);
     std::vector<char> seen(static_cast<size_t>(num_pages), 0);
     for (int64_t i = 0; i < num_pages; ++i) {
         const int32_t p = free_order ? free_order[i] : static_cast<int32_t>(i);
-        if (p < 0 || p >= num_pages || seen[p]) { delete a; return TG_EINVAL; }
+        if (p < 0 || p >= num_pages || seen[p]) return TG_EINVAL;
         seen[p] = 1;
-        a->free_list.push_back(p);
+        a->give(p);
     }
-    *out = a;
+    *out = a.release();
     return TG_OK;
 }
 
-extern "C" void tg_alloc_destroy(tg_alloc *a) { delete a; }
-
-extern "C" int64_t tg_alloc_free_pages(const tg_alloc *a) {
-    return a ? static_cast<int64_t>(a->free_list.size()) : -1;
-}
-
-extern "C" int32_t tg_alloc_refcount(const tg_alloc *a, int32_t page_id) {
-    if (!a || page_id < 0 || page_id >= a->num_pages) return -1;
-    return a->refs[page_id];
-}
-
-extern "C" int tg_alloc_share_segment(tg_alloc *a, int32_t n_tokens, int32_t n_heads,
-                                      int32_t *seg_id, int32_t *page_ids) {
+int alloc_share_segment(tg_alloc *a, int32_t n_tokens, int32_t n_heads, int32_t *seg_id,
+                        int32_t *page_ids) {
     if (!a || !seg_id || n_tokens < 0 || n_heads < 1) return TG_EINVAL;
     const int32_t full = n_tokens / a->page;
     const int64_t need = static_cast<int64_t>(full) * n_heads;
-    if (need > static_cast<int64_t>(a->free_list.size())) return TG_ENOSPC;
-    tg_alloc::Segment s;
+    if (need > a->n_free) return TG_ENOSPC;
+    std::vector<int32_t> pages;
+    pages.reserve(static_cast<size_t>(need));  // the fallible steps come first
+    a->segs.emplace_back();
+    tg_alloc::Segment &s = a->segs.back();
     s.n_heads = n_heads;
     s.full = full;
     s.alive = true;
-    s.pages.reserve(static_cast<size_t>(need));
     for (int64_t i = 0; i < need; ++i) {
-        const int32_t p = a->free_list.front();
-        a->free_list.pop_front();
+        const int32_t p = a->take();
         a->refs[p] = 1;  // the segment's own reference
-        s.pages.push_back(p);
+        pages.push_back(p);
     }
-    if (page_ids && need > 0) std::memcpy(page_ids, s.pages.data(), sizeof(int32_t) * static_cast<size_t>(need));
-    *seg_id = static_cast<int32_t>(a->segs.size());
-    a->segs.push_back(std::move(s));
+    if (page_ids && need > 0) std::memcpy(page_ids, pages.data(), sizeof(int32_t) * static_cast<size_t>(need));
+    s.pages = std::move(pages);
+    *seg_id = static_cast<int32_t>(a->segs.size() - 1);
     return TG_OK;
 }
 
-extern "C" int tg_alloc_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads,
-                                const int32_t *kv_len, int32_t n_prefix,
-                                const int32_t *prefix_segs, int32_t *page_ids, int64_t capacity,
-                                int64_t *n_written) {
+int alloc_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads, const int32_t *kv_len, int32_t n_prefix,
+                  const int32_t *prefix_segs, int32_t *page_ids, int64_t capacity, int64_t *n_written) {
     if (!a || n_heads < 1 || !kv_len || n_prefix < 0 || (n_prefix > 0 && !prefix_segs) ||
         (capacity > 0 && !page_ids) || capacity < 0)
         return TG_EINVAL;
@@ -166,9 +172,17 @@ extern "C" int tg_alloc_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads,
         total += shared_pages + priv;
     }
     if (total > capacity) return TG_EINVAL;
-    if (priv_total > static_cast<int64_t>(a->free_list.size())) return TG_ENOSPC;
+    if (priv_total > a->n_free) return TG_ENOSPC;
 
-    tg_alloc::Seq sq;
+    // The fallible steps (the sequence's record and its page lists) before any page moves.
+    tg_alloc::Seq &sq = a->seqs[seq_id];
+    try {
+        sq.shared.reserve(static_cast<size_t>(shared_pages) * static_cast<size_t>(n_heads));
+        sq.priv.reserve(static_cast<size_t>(priv_total));
+    } catch (...) {
+        a->seqs.erase(seq_id);
+        throw;
+    }
     int64_t w = 0;
     for (int32_t h = 0; h < n_heads; ++h) {
         for (int32_t c = 0; c < n_prefix; ++c) {
@@ -184,16 +198,44 @@ extern "C" int tg_alloc_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads,
         }
         const int64_t priv = (kv_len[h] - shared_tokens + a->page - 1) / a->page;
         for (int64_t p = 0; p < priv; ++p) {
-            const int32_t id = a->free_list.front();
-            a->free_list.pop_front();
+            const int32_t id = a->take();
             a->refs[id] = 1;
             sq.priv.push_back(id);
             page_ids[w++] = id;
         }
     }
     if (n_written) *n_written = w;
-    a->seqs.emplace(seq_id, std::move(sq));
     return TG_OK;
+}
+
+}  // namespace
+
+extern "C" int tg_alloc_create(int64_t num_pages, int32_t page, const int32_t *free_order,
+                               tg_alloc **out) {
+    return tg::no_throw([&] { return alloc_create(num_pages, page, free_order, out); });
+}
+
+extern "C" void tg_alloc_destroy(tg_alloc *a) { delete a; }
+
+extern "C" int64_t tg_alloc_free_pages(const tg_alloc *a) { return a ? a->n_free : -1; }
+
+extern "C" int32_t tg_alloc_refcount(const tg_alloc *a, int32_t page_id) {
+    if (!a || page_id < 0 || page_id >= a->num_pages) return -1;
+    return a->refs[page_id];
+}
+
+extern "C" int tg_alloc_share_segment(tg_alloc *a, int32_t n_tokens, int32_t n_heads,
+                                      int32_t *seg_id, int32_t *page_ids) {
+    return tg::no_throw([&] { return alloc_share_segment(a, n_tokens, n_heads, seg_id, page_ids); });
+}
+
+extern "C" int tg_alloc_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads,
+                                const int32_t *kv_len, int32_t n_prefix,
+                                const int32_t *prefix_segs, int32_t *page_ids, int64_t capacity,
+                                int64_t *n_written) {
+    return tg::no_throw([&] {
+        return alloc_reserve(a, seq_id, n_heads, kv_len, n_prefix, prefix_segs, page_ids, capacity, n_written);
+    });
 }
 
 extern "C" int tg_alloc_release(tg_alloc *a, int32_t seq_id) {
@@ -223,49 +265,51 @@ extern "C" int tg_group_tables(int32_t B, int32_t Hkv, const int32_t *head_count
                                const int32_t *group_of_head, int32_t n_groups,
                                const int32_t *page_ids, int32_t *table, int64_t *head_off,
                                int64_t *group_off) {
-    if (B < 0 || Hkv < 1 || !head_count || !group_of_head || n_groups < 1 || !group_off)
-        return TG_EINVAL;
-    for (int32_t h = 0; h < Hkv; ++h)
-        if (group_of_head[h] < 0 || group_of_head[h] >= n_groups) return TG_EINVAL;
-    const int64_t BH = static_cast<int64_t>(B) * Hkv;
-    std::vector<int64_t> src(static_cast<size_t>(BH) + 1, 0);
-    for (int64_t i = 0; i < BH; ++i) {
-        if (head_count[i] < 0) return TG_EINVAL;
-        src[i + 1] = src[i] + head_count[i];
-    }
-    if (table && (!page_ids || !head_off)) return TG_EINVAL;
-    int64_t pos = 0;
-    for (int32_t g = 0; g < n_groups; ++g) {
-        group_off[g] = pos;
-        std::vector<int32_t> heads;
-        int64_t Pg = 0;
-        for (int32_t h = 0; h < Hkv; ++h) {
-            if (group_of_head[h] != g) continue;
-            heads.push_back(h);
-            for (int32_t b = 0; b < B; ++b)
-                Pg = std::max<int64_t>(Pg, head_count[static_cast<int64_t>(b) * Hkv + h]);
+    return tg::no_throw([&] {
+        if (B < 0 || Hkv < 1 || !head_count || !group_of_head || n_groups < 1 || !group_off)
+            return TG_EINVAL;
+        for (int32_t h = 0; h < Hkv; ++h)
+            if (group_of_head[h] < 0 || group_of_head[h] >= n_groups) return TG_EINVAL;
+        const int64_t BH = static_cast<int64_t>(B) * Hkv;
+        std::vector<int64_t> src(static_cast<size_t>(BH) + 1, 0);
+        for (int64_t i = 0; i < BH; ++i) {
+            if (head_count[i] < 0) return TG_EINVAL;
+            src[i + 1] = src[i] + head_count[i];
         }
-        const int64_t Hg = static_cast<int64_t>(heads.size());
-        if (table) {
-            for (int32_t b = 0; b < B; ++b)
-                for (int64_t j = 0; j < Hg; ++j) {
-                    const int64_t bh = static_cast<int64_t>(b) * Hkv + heads[j];
-                    const int64_t row = pos + (static_cast<int64_t>(b) * Hg + j) * Pg;
-                    head_off[bh] = row;
-                    const int64_t cnt = head_count[bh];
-                    for (int64_t p = 0; p < Pg; ++p)
-                        table[row + p] = p < cnt ? page_ids[src[bh] + p] : -1;
-                }
-        } else if (head_off) {
-            for (int32_t b = 0; b < B; ++b)
-                for (int64_t j = 0; j < Hg; ++j)
-                    head_off[static_cast<int64_t>(b) * Hkv + heads[j]] =
-                        pos + (static_cast<int64_t>(b) * Hg + j) * Pg;
+        if (table && (!page_ids || !head_off)) return TG_EINVAL;
+        int64_t pos = 0;
+        for (int32_t g = 0; g < n_groups; ++g) {
+            group_off[g] = pos;
+            std::vector<int32_t> heads;
+            int64_t Pg = 0;
+            for (int32_t h = 0; h < Hkv; ++h) {
+                if (group_of_head[h] != g) continue;
+                heads.push_back(h);
+                for (int32_t b = 0; b < B; ++b)
+                    Pg = std::max<int64_t>(Pg, head_count[static_cast<int64_t>(b) * Hkv + h]);
+            }
+            const int64_t Hg = static_cast<int64_t>(heads.size());
+            if (table) {
+                for (int32_t b = 0; b < B; ++b)
+                    for (int64_t j = 0; j < Hg; ++j) {
+                        const int64_t bh = static_cast<int64_t>(b) * Hkv + heads[j];
+                        const int64_t row = pos + (static_cast<int64_t>(b) * Hg + j) * Pg;
+                        head_off[bh] = row;
+                        const int64_t cnt = head_count[bh];
+                        for (int64_t p = 0; p < Pg; ++p)
+                            table[row + p] = p < cnt ? page_ids[src[bh] + p] : -1;
+                    }
+            } else if (head_off) {
+                for (int32_t b = 0; b < B; ++b)
+                    for (int64_t j = 0; j < Hg; ++j)
+                        head_off[static_cast<int64_t>(b) * Hkv + heads[j]] =
+                            pos + (static_cast<int64_t>(b) * Hg + j) * Pg;
+            }
+            pos += static_cast<int64_t>(B) * Hg * Pg;
         }
-        pos += static_cast<int64_t>(B) * Hg * Pg;
-    }
-    group_off[n_groups] = pos;
-    return TG_OK;
+        group_off[n_groups] = pos;
+        return TG_OK;
+    });
 }
 
 // ------------------------------------------------------------------------------------------
@@ -273,18 +317,20 @@ extern "C" int tg_group_tables(int32_t B, int32_t Hkv, const int32_t *head_count
 // ------------------------------------------------------------------------------------------
 extern "C" int tg_place_sequences(int32_t n_seq, const int64_t *seq_bytes, int32_t n_gpus,
                                   int32_t *gpu_of_seq) {
-    if (n_seq < 0 || n_gpus < 1 || (n_seq > 0 && (!seq_bytes || !gpu_of_seq))) return TG_EINVAL;
-    std::vector<int32_t> order(n_seq);
-    std::iota(order.begin(), order.end(), 0);
-    std::stable_sort(order.begin(), order.end(),
-                     [&](int32_t a, int32_t b) { return seq_bytes[a] > seq_bytes[b]; });
-    std::vector<int64_t> load(n_gpus, 0);
-    for (int32_t s : order) {
-        const int32_t g = static_cast<int32_t>(std::min_element(load.begin(), load.end()) - load.begin());
-        gpu_of_seq[s] = g;
-        load[g] += seq_bytes[s];
-    }
-    return TG_OK;
+    return tg::no_throw([&] {
+        if (n_seq < 0 || n_gpus < 1 || (n_seq > 0 && (!seq_bytes || !gpu_of_seq))) return TG_EINVAL;
+        std::vector<int32_t> order(n_seq);
+        std::iota(order.begin(), order.end(), 0);
+        std::stable_sort(order.begin(), order.end(),
+                         [&](int32_t a, int32_t b) { return seq_bytes[a] > seq_bytes[b]; });
+        std::vector<int64_t> load(n_gpus, 0);
+        for (int32_t s : order) {
+            const int32_t g = static_cast<int32_t>(std::min_element(load.begin(), load.end()) - load.begin());
+            gpu_of_seq[s] = g;
+            load[g] += seq_bytes[s];
+        }
+        return TG_OK;
+    });
 }
 
 // ------------------------------------------------------------------------------------------
@@ -615,6 +661,12 @@ void shared_runs(int32_t h, const std::vector<int32_t> &rows, int32_t Hkv, const
     }
 }
 
+// Frees a plan under construction the way tg_plan_destroy does (no CUDA call for a plan that
+// holds no device state yet).
+struct PlanFree {
+    void operator()(tg_plan *p) const { tg_plan_destroy(p); }
+};
+
 int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,
                 const int32_t *group_of_head, const int64_t *group_off, int32_t n_groups,
                 int64_t slow_table_len, const tg_plan_opts *opts, const int32_t *table,
@@ -639,8 +691,8 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
     if (opts) o = *opts;
     if (o.min_splits < 1) o.min_splits = 1;
 
-    tg_plan *p = new (std::nothrow) tg_plan;
-    if (!p) return TG_ENOMEM;
+    std::unique_ptr<tg_plan, PlanFree> hold(new tg_plan);  // freed on every early return
+    tg_plan *p = hold.get();
     p->shape = s;
     p->G = G;
     p->tiered = fast_len != nullptr;
@@ -653,15 +705,13 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
     p->early_prologue = o.early_prologue != 0;
     if (o.wait_limit_us > 0) p->wait_ns = static_cast<uint64_t>(o.wait_limit_us) * 1000ull;
     p->withhold = o.test_withhold_page > 0 ? o.test_withhold_page : 0;
-    if (o.capacity && !fast_len) { delete p; return TG_EINVAL; }
+    if (o.capacity && !fast_len) return TG_EINVAL;
     p->capacity = o.capacity != 0;
     p->out_f32 = o.out_f32 != 0;
     p->whole_heads = o.whole_heads != 0;
     p->slow_bits = o.slow_bits == 0 ? 8 : o.slow_bits;
-    if ((p->slow_bits != 8 && p->slow_bits != 4) || (p->slow_bits == 4 && (!fast_len || shape->D != 128))) {
-        delete p;
+    if ((p->slow_bits != 8 && p->slow_bits != 4) || (p->slow_bits == 4 && (!fast_len || shape->D != 128)))
         return TG_EINVAL;
-    }
 
     // Prefix cascade: shared runs per KV head, cut into units of kCascadeRows query rows.
     std::vector<int32_t> casc_cnt;
@@ -669,10 +719,7 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
         const int64_t BH = static_cast<int64_t>(s.B) * s.Hkv;
         for (int64_t bh = 0; bh < BH; ++bh) {
             const int64_t npages = (kv_len[bh] + 15) / 16;
-            if (kv_len[bh] < 0 || head_off[bh] < 0 || head_off[bh] + npages > table_len) {
-                delete p;
-                return TG_EINVAL;
-            }
+            if (kv_len[bh] < 0 || head_off[bh] < 0 || head_off[bh] + npages > table_len) return TG_EINVAL;
         }
         p->pstart.assign(static_cast<size_t>(BH), 0);
         std::vector<Node> nodes;
@@ -703,7 +750,7 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
     int32_t workers = o.num_workers;
     if (!p->host_only) {
         int rc = tg::device_num_sms(o.device, &p->num_sms);
-        if (rc != TG_OK) { delete p; return rc; }
+        if (rc != TG_OK) return rc;
         if (workers <= 0) workers = p->num_sms * p->pairs;
     } else if (workers <= 0) {
         workers = 148 * p->pairs;
@@ -713,7 +760,7 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
     int rc = tg::build_work_list(p, kv_len, fast_len, workers, o.min_splits, o.max_chunk_pages, sp,
                                  dc, table ? p->pstart.data() : nullptr,
                                  table ? casc_cnt.data() : nullptr);
-    if (rc != TG_OK) { delete p; return rc; }
+    if (rc != TG_OK) return rc;
     if (table) {
         // Cascade partial slots: a head's merge list starts with its runs, in unit order.
         std::vector<int32_t> next(static_cast<size_t>(s.B) * s.Hkv, -1);
@@ -727,9 +774,9 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
     if (p->grid == 0 && !p->empties.empty()) p->grid = 1;  // the kernel also writes empty heads
     if (!p->host_only) {
         rc = tg::device_init_plan(p);
-        if (rc != TG_OK) { tg::device_free_plan(p); delete p; return rc; }
+        if (rc != TG_OK) return rc;
     }
-    *out = p;
+    *out = hold.release();
     return TG_OK;
 }
 
@@ -740,8 +787,10 @@ extern "C" int tg_plan_create(const tg_shape *shape, const int32_t *kv_len,
                               const int64_t *group_off, int32_t n_groups,
                               int64_t slow_table_len, const tg_plan_opts *opts,
                               tg_plan **out) {
-    return plan_create(shape, kv_len, fast_len, group_of_head, group_off, n_groups,
-                       slow_table_len, opts, nullptr, nullptr, 0, 0, out);
+    return tg::no_throw([&] {
+        return plan_create(shape, kv_len, fast_len, group_of_head, group_off, n_groups, slow_table_len, opts,
+                           nullptr, nullptr, 0, 0, out);
+    });
 }
 
 extern "C" int tg_plan_create_cascade(const tg_shape *shape, const int32_t *kv_len,
@@ -750,9 +799,12 @@ extern "C" int tg_plan_create_cascade(const tg_shape *shape, const int32_t *kv_l
                                       const int64_t *head_page_off, int64_t table_len,
                                       int32_t min_readers, const tg_plan_opts *opts,
                                       tg_plan **out) {
+    if (out) *out = nullptr;
     if (!page_table || !head_page_off || table_len < 0) return TG_EINVAL;
-    return plan_create(shape, kv_len, nullptr, group_of_head, group_off, n_groups, 0, opts,
-                       page_table, head_page_off, table_len, min_readers, out);
+    return tg::no_throw([&] {
+        return plan_create(shape, kv_len, nullptr, group_of_head, group_off, n_groups, 0, opts, page_table,
+                           head_page_off, table_len, min_readers, out);
+    });
 }
 
 extern "C" void tg_plan_destroy(tg_plan *p) {

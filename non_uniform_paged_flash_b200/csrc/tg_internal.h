@@ -3,12 +3,29 @@
 #pragma once
 
 #include <cstdint>
+#include <new>
+#include <stdexcept>
 #include <string>
 #include <vector>
 
 #include "tg.h"
 
 namespace tg {
+
+// The host code builds std containers. A C entry point runs its body through no_throw so that
+// a container that cannot grow (std::bad_alloc, or a length past its limit) returns TG_ENOMEM
+// instead of unwinding through the C ABI. Bodies make their fallible allocations before they
+// change any state that outlives the call.
+template <class F>
+int no_throw(F &&body) noexcept {
+    try {
+        return body();
+    } catch (const std::bad_alloc &) {
+        return TG_ENOMEM;
+    } catch (const std::length_error &) {
+        return TG_ENOMEM;
+    }
+}
 
 // One work item: a contiguous page range of one (sequence, KV head) row in one tier.
 struct Item {

@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <memory>
 #include <new>
 #include <vector>
 
@@ -110,17 +111,23 @@ bool pinned(const void *p) {
 
 using namespace tg;
 
-extern "C" int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,
-                                     const int32_t *group_of_head, const int64_t *group_off, int32_t n_groups,
-                                     const int32_t *slow_page_table, const int64_t *slow_head_off,
-                                     int64_t slow_table_len, int32_t block_pages, int32_t ring_blocks,
-                                     const tg_plan_opts *opts, tg_slow_stream **out) {
-    if (!shape || !kv_len || !fast_len || !group_of_head || !group_off || !slow_head_off || !out ||
+namespace {
+
+struct Release {
+    void operator()(tg_slow_stream *s) const { release(s); }
+};
+
+int slow_stream_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,
+                       const int32_t *group_of_head, const int64_t *group_off, int32_t n_groups,
+                       const int32_t *slow_page_table, const int64_t *slow_head_off, int64_t slow_table_len,
+                       int32_t block_pages, int32_t ring_blocks, const tg_plan_opts *opts, tg_slow_stream **out) {
+    if (!out) return TG_EINVAL;
+    *out = nullptr;
+    if (!shape || !kv_len || !fast_len || !group_of_head || !group_off || !slow_head_off ||
         block_pages < 1 || ring_blocks < 1 || slow_table_len < 0 || shape->B < 1 || shape->Hkv < 1 ||
         shape->Hq < shape->Hkv || shape->Hq % shape->Hkv || shape->page != 16 ||
         (shape->D != 64 && shape->D != 128) || shape->num_slow_pages < 0 || (slow_table_len > 0 && !slow_page_table))
         return TG_EINVAL;
-    *out = nullptr;
     tg_plan_opts o{};
     if (opts) o = *opts;
     const tg_shape &S = *shape;
@@ -140,7 +147,7 @@ extern "C" int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_le
         fl[bh] = f;
         const int32_t ns = n - f;
         const int32_t np = (ns + 15) / 16;
-        if (np > 0 && (slow_head_off[bh] < 0 || slow_head_off[bh] + np > slow_table_len)) return TG_EINVAL;
+        if (np > 0 && (slow_head_off[bh] < 0 || slow_head_off[bh] > slow_table_len - np)) return TG_EINVAL;
         for (int32_t t = 0; t < np; ++t) {
             const int32_t id = slow_page_table[slow_head_off[bh] + t];
             if (id < 0 || id >= nsp) return TG_EINVAL;
@@ -151,8 +158,8 @@ extern "C" int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_le
             else rows[j * BH + bh].push_back(local);
         }
     }
-    tg_slow_stream *s = new (std::nothrow) tg_slow_stream();
-    if (!s) return TG_ENOMEM;
+    std::unique_ptr<tg_slow_stream, Release> hold(new tg_slow_stream());  // released on every early return
+    tg_slow_stream *s = hold.get();
     s->shape = S;
     s->G = S.Hq / S.Hkv;
     s->block_pages = block_pages;
@@ -192,6 +199,7 @@ extern "C" int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_le
     fs.num_slow_pages = 0;
     tg_plan_opts fo = po;
     fo.slow_bits = 0;
+    s->blk.reserve(static_cast<size_t>(J));  // so that keeping a made plan never throws
     int rc = tg_plan_create(&fs, fl.data(), nullptr, group_of_head, group_off, n_groups, 0, &fo, &s->fast);
     std::vector<int32_t> zeros(static_cast<size_t>(BH), 0);
     tg_shape bs = S;
@@ -202,16 +210,18 @@ extern "C" int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_le
                             std::max<int64_t>(1, s->blk_table_len[j]), &po, &p);
         if (rc == TG_OK) s->blk.push_back(p);
     }
-    if (rc != TG_OK || s->host_only) {
-        if (rc != TG_OK) {
-            release(s);
-            return rc;
-        }
-        *out = s;
+    if (rc != TG_OK) return rc;
+    if (s->host_only) {
+        *out = hold.release();
         return TG_OK;
     }
 
     // Device state: ring | tables | offsets | lengths | zeros | fast lengths | partials.
+    std::vector<int32_t> lens(s->blk_len);
+    lens.insert(lens.end(), zeros.begin(), zeros.end());
+    lens.insert(lens.end(), fl.begin(), fl.end());
+    s->landed.reserve(static_cast<size_t>(ring_blocks));
+    s->freed.reserve(static_cast<size_t>(ring_blocks));
     s->device = s->fast->device;
     int prev = 0;
     cudaGetDevice(&prev);
@@ -235,7 +245,6 @@ extern "C" int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_le
     cudaError_t e = cudaMalloc(&s->dev, at);
     if (e != cudaSuccess) {
         cudaSetDevice(prev);
-        release(s);
         return e == cudaErrorMemoryAllocation ? TG_ENOMEM : fail("cudaMalloc(slow stream)", e);
     }
     char *b = static_cast<char *>(s->dev);
@@ -250,9 +259,6 @@ extern "C" int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_le
     s->d_fast_len = s->d_zero + BH;
     s->part_o = reinterpret_cast<float *>(b + off[7]);
     s->part_lse = reinterpret_cast<float *>(b + off[8]);
-    std::vector<int32_t> lens(s->blk_len);
-    lens.insert(lens.end(), zeros.begin(), zeros.end());
-    lens.insert(lens.end(), fl.begin(), fl.end());
     if ((!s->h_table.empty() &&
          (e = cudaMemcpy(s->d_table, s->h_table.data(), s->h_table.size() * 4, cudaMemcpyHostToDevice)) != cudaSuccess) ||
         (!s->h_off.empty() &&
@@ -270,12 +276,22 @@ extern "C" int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_le
         if (f) s->freed.push_back(f);
     }
     cudaSetDevice(prev);
-    if (rc != TG_OK) {
-        release(s);
-        return rc;
-    }
-    *out = s;
+    if (rc != TG_OK) return rc;
+    *out = hold.release();
     return TG_OK;
+}
+
+}  // namespace
+
+extern "C" int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,
+                                     const int32_t *group_of_head, const int64_t *group_off, int32_t n_groups,
+                                     const int32_t *slow_page_table, const int64_t *slow_head_off,
+                                     int64_t slow_table_len, int32_t block_pages, int32_t ring_blocks,
+                                     const tg_plan_opts *opts, tg_slow_stream **out) {
+    return no_throw([&] {
+        return slow_stream_create(shape, kv_len, fast_len, group_of_head, group_off, n_groups, slow_page_table,
+                                  slow_head_off, slow_table_len, block_pages, ring_blocks, opts, out);
+    });
 }
 
 extern "C" void tg_slow_stream_destroy(tg_slow_stream *s) {

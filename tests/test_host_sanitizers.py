@@ -1,6 +1,8 @@
 """The library's host code (allocator, group tables, planner, placement) built with
 AddressSanitizer and UndefinedBehaviorSanitizer and driven on seeded random inputs
-(tests/native/host_fuzz.cpp); no GPU involved."""
+(tests/native/host_fuzz.cpp), then with allocation failures injected into every allocation of
+every call in turn: each such call returns TG_ENOMEM (or falls back to the same result), leaves
+the allocator unchanged, hands back no object and leaks nothing. No GPU involved."""
 import os
 import shutil
 import subprocess
@@ -25,6 +27,8 @@ def test_host_code_is_clean_under_asan_and_ubsan():
     subprocess.check_call(cmd)
     env = dict(os.environ, ASAN_OPTIONS="detect_leaks=1:abort_on_error=0",
                UBSAN_OPTIONS="print_stacktrace=1")
-    r = subprocess.run([str(exe), "200"], capture_output=True, text=True, env=env, timeout=600)
+    r = subprocess.run([str(exe), "200", "20261202", "20"], capture_output=True, text=True, env=env,
+                       timeout=600)
     assert r.returncode == 0, (r.stdout + r.stderr)[-4000:]
-    assert "rounds clean" in r.stdout
+    assert "200 rounds clean" in r.stdout
+    assert "allocation failures: 20 rounds" in r.stdout

@@ -51,6 +51,10 @@ extern "C" {
 #define TG_EUNSUPPORTED 8  /* shape outside what the kernels support */
 #define TG_EEXIST 9        /* sequence id already holds a reservation */
 
+/* Longest retained length of one (sequence, KV head) that plans accept (2^30 tokens, 2^26
+ * pages): every token and page index of a head then fits 32-bit arithmetic with room to spare. */
+#define TG_MAX_HEAD_TOKENS (1 << 30)
+
 typedef struct CUstream_st *tg_stream; /* == cudaStream_t */
 
 /* Shape of one decode step over one layer. */
@@ -213,10 +217,11 @@ typedef struct tg_plan_opts {
  * log-sum-exp in split order by a second kernel that the decode call launches as a
  * programmatic dependent (its launch overlaps the decode's tail).
  * The plan owns one device allocation (work list, merge list, partial results, error word),
- * made here; nothing is allocated per call. Returns TG_EINVAL for bad arguments,
- * TG_EUNSUPPORTED for a shape the kernels do not serve (page != 16, D not 64 or 128, Hq/Hkv
- * not 1, 2, 4 or 8, a tiered plan with D != 128); on any error *out is NULL and nothing is
- * left allocated. */
+ * made here; nothing is allocated per call. Returns TG_EINVAL for bad arguments (a negative
+ * length among them), TG_EUNSUPPORTED for a shape the kernels do not serve (page != 16, D not
+ * 64 or 128, Hq/Hkv not 1, 2, 4 or 8, a tiered plan with D != 128, a kv_len above
+ * TG_MAX_HEAD_TOKENS), TG_ENOMEM when host or device memory runs out; on any error *out is
+ * NULL and nothing is left allocated. */
 int tg_plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,
                    const int32_t *group_of_head, const int64_t *group_off, int32_t n_groups,
                    int64_t slow_table_len, const tg_plan_opts *opts, tg_plan **out);

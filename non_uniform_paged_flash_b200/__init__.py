@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(_PKG, "libtg.so")
 
 TG_OK, TG_EINVAL, TG_ENOSPC, TG_EBADPAGE, TG_ECUDA, TG_ETIMEOUT = 0, 1, 2, 3, 4, 5
 TG_ENOMEM, TG_ENOTFOUND, TG_EUNSUPPORTED, TG_EEXIST = 6, 7, 8, 9
+TG_MAX_HEAD_TOKENS = 1 << 30   # longest retained length of one (sequence, KV head) a plan accepts
 
 
 class TGError(RuntimeError):

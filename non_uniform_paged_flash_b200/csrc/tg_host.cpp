@@ -685,6 +685,11 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
     if (s.num_pages > (INT64_C(1) << 28) || s.num_slow_pages > (INT64_C(1) << 28)) return TG_EUNSUPPORTED;
     for (int32_t h = 0; h < s.Hkv; ++h)
         if (group_of_head[h] < 0 || group_of_head[h] >= n_groups) return TG_EINVAL;
+    const int64_t n_heads = static_cast<int64_t>(s.B) * s.Hkv;
+    for (int64_t bh = 0; bh < n_heads; ++bh) {
+        if (kv_len[bh] < 0 || (fast_len && fast_len[bh] < 0)) return TG_EINVAL;
+        if (kv_len[bh] > TG_MAX_HEAD_TOKENS) return TG_EUNSUPPORTED;
+    }
     tg_plan_opts o{};
     o.min_splits = 1;
     o.device = -1;

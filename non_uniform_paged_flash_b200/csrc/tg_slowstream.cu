@@ -143,6 +143,7 @@ int slow_stream_create(const tg_shape *shape, const int32_t *kv_len, const int32
     for (int64_t bh = 0; bh < BH; ++bh) {
         const int32_t n = kv_len[bh];
         if (n < 0 || fast_len[bh] < 0) return TG_EINVAL;
+        if (n > TG_MAX_HEAD_TOKENS) return TG_EUNSUPPORTED;
         const int32_t f = std::min(fast_len[bh], n);
         fl[bh] = f;
         const int32_t ns = n - f;

@@ -438,3 +438,28 @@ def test_new_entries_reject_bad_arguments_without_a_gpu():
     with pytest.raises(tg.TGError) as e:
         tg.HostPipe(hp)
     assert e.value.status == tg.TG_EINVAL
+
+
+def test_plan_rejects_unsupported_shapes_and_lengths():
+    """Shapes the kernels do not serve and lengths past TG_MAX_HEAD_TOKENS are refused with
+    TG_EUNSUPPORTED (a negative length with TG_EINVAL); a head of exactly the maximum plans."""
+    goh = np.zeros(2, np.int32)
+    goff = np.array([0, 1 << 27], np.int64)
+    kv = np.array([[100, 37]], np.int32)
+    ok = dict(host_only=True, num_workers=16, whole_heads=True)
+    for shape in (tg.make_shape(1, 6, 2, 128, 1 << 20),      # 3 query heads per KV head
+                  tg.make_shape(1, 8, 2, 96, 1 << 20),       # head dim 96
+                  tg.make_shape(1, 8, 2, 128, 1 << 20, page=32)):
+        with pytest.raises(tg.TGError) as e:
+            tg.tg_plan_create(shape, kv, goh, goff, **ok)
+        assert e.value.status == tg.TG_EUNSUPPORTED
+    shape = tg.make_shape(1, 8, 2, 128, 1 << 26)
+    for bad, status in ((tg.TG_MAX_HEAD_TOKENS + 1, tg.TG_EUNSUPPORTED),
+                        (2**31 - 1, tg.TG_EUNSUPPORTED), (-1, tg.TG_EINVAL)):
+        with pytest.raises(tg.TGError) as e:
+            tg.tg_plan_create(shape, np.array([[100, bad]], np.int32), goh, goff, **ok)
+        assert e.value.status == status
+    p = tg.tg_plan_create(shape, np.array([[100, tg.TG_MAX_HEAD_TOKENS]], np.int32), goh, goff, **ok)
+    info = tg.tg_plan_get_info(p)
+    assert info["n_items"] == 2
+    assert info["kv_bytes"] == (100 + tg.TG_MAX_HEAD_TOKENS) * 2 * 128 * 2

@@ -220,7 +220,7 @@ typedef struct tg_plan_opts {
  * made here; nothing is allocated per call. Returns TG_EINVAL for bad arguments (a negative
  * length among them), TG_EUNSUPPORTED for a shape the kernels do not serve (page != 16, D not
  * 64 or 128, Hq/Hkv not 1, 2, 4 or 8, a tiered plan with D != 128, a kv_len above
- * TG_MAX_HEAD_TOKENS), TG_ENOMEM when host or device memory runs out; on any error *out is
+ * TG_MAX_HEAD_TOKENS, B*Hq above INT32_MAX), TG_ENOMEM when host or device memory runs out; on any error *out is
  * NULL and nothing is left allocated. */
 int tg_plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,
                    const int32_t *group_of_head, const int64_t *group_off, int32_t n_groups,

@@ -683,6 +683,7 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
         return TG_EUNSUPPORTED;
     if (fast_len && s.D != 128) return TG_EUNSUPPORTED;
     if (s.num_pages > (INT64_C(1) << 28) || s.num_slow_pages > (INT64_C(1) << 28)) return TG_EUNSUPPORTED;
+    if (static_cast<int64_t>(s.B) * s.Hq > INT32_MAX) return TG_EUNSUPPORTED;  // query rows index in 32 bits
     for (int32_t h = 0; h < s.Hkv; ++h)
         if (group_of_head[h] < 0 || group_of_head[h] >= n_groups) return TG_EINVAL;
     const int64_t n_heads = static_cast<int64_t>(s.B) * s.Hkv;

@@ -315,7 +315,7 @@ bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_shape(const tg_shape *s) {
     if (!s || s->B < 0 || s->Hkv < 1 || s->Hq < s->Hkv || s->Hq % s->Hkv != 0 || s->page != 16 ||
-        s->D < 8 || s->D % 8 != 0 || s->num_pages < 0)
+        s->D < 8 || s->D % 8 != 0 || s->num_pages < 0 || static_cast<int64_t>(s->B) * s->Hkv > INT32_MAX)
         return TG_EINVAL;
     return TG_OK;
 }

@@ -449,7 +449,8 @@ def test_plan_rejects_unsupported_shapes_and_lengths():
     ok = dict(host_only=True, num_workers=16, whole_heads=True)
     for shape in (tg.make_shape(1, 6, 2, 128, 1 << 20),      # 3 query heads per KV head
                   tg.make_shape(1, 8, 2, 96, 1 << 20),       # head dim 96
-                  tg.make_shape(1, 8, 2, 128, 1 << 20, page=32)):
+                  tg.make_shape(1, 8, 2, 128, 1 << 20, page=32),
+                  tg.make_shape(2**28, 8, 2, 128, 1 << 20)):    # 2^31 query rows
         with pytest.raises(tg.TGError) as e:
             tg.tg_plan_create(shape, kv, goh, goff, **ok)
         assert e.value.status == tg.TG_EUNSUPPORTED

@@ -7,6 +7,7 @@ batch's KV cache, page tables and plan are resident in HBM before timing (admiss
 once, as in serving); the step's inputs are the queries.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+    python bench.py --path sink|h2o|ttkv|ttkv-host|splitzip|layers ...   (one GPU, other lines)
 
 N > 1 runs under torch.distributed.run, one rank per GPU. The batch is sharded by sequence with
 the library's ahead-of-time placement (per-GPU work fixed: weak scaling); the decode has no
@@ -845,6 +846,79 @@ def run_tier_host(args):
     return 0
 
 
+def run_layers(args):
+    """The multi-turn serving step (config 3) over its layers, one GPU. The 32 layers' pools
+    (about 189 GB at the workload's occupancy) do not fit one GPU, so each layer's tables, plan
+    and pools are made resident in turn (outside any timed region) and its decode step timed
+    with CUDA events over args.steps steps (each layer's 5.5 GB of K/V is far above L2). Prints
+    one JSON line: each layer's step time and K/V bytes, the mean step, and value = all the
+    layers' K/V bytes / the sum of their step times."""
+    import torch
+    import non_uniform_paged_flash_b200 as tg
+    from non_uniform_paged_flash_b200 import workload
+
+    if _env_int("WORLD_SIZE", 1) != 1:
+        raise SystemExit("--path layers runs on one GPU")
+    cfg = 3
+    sp = _preset(cfg)
+    n_layers = min(args.layers, sp.layers)
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(0)
+    per_layer, bad = [], False
+    for layer in range(n_layers):
+        lay = workload.layout(sp, layer)
+        db = workload.to_device(sp, lay, layer, **_plan_kw(cfg))
+        alg = workload.algorithmic_bytes(sp, lay)
+        for _ in range(args.warmup):
+            db.run(stream)
+        torch.cuda.synchronize()
+        n_timed = min(args.steps, 256)
+        tg.tg_plan_timing_enable(db.plan, n_timed)
+        if layer == 0:
+            sampler.start()
+            time.sleep(0.3)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            db.run(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        n_rec, dec_ms, _ = tg.tg_plan_timing_read(db.plan)
+        bad = bad or tg.tg_plan_status(db.plan) != tg.TG_OK
+        info = tg.tg_plan_get_info(db.plan)
+        per_layer.append({"layer": layer, "ms_per_step": e0.elapsed_time(e1) / args.steps,
+                          "kv_bytes": int(alg["kv"]), "algorithmic_bytes": int(alg["total"]),
+                          "decode_avg_ms": dec_ms / max(n_rec, 1), "batch": int(lay.kv_len.shape[0]),
+                          "launches": args.steps * (1 + (1 if info["n_merge"] > 0 else 0))})
+        db.plan.destroy()
+        del db
+        torch.cuda.empty_cache()
+    clocks = sampler.stop()
+    ms_sum = sum(r["ms_per_step"] for r in per_layer)
+    kv_sum = sum(r["kv_bytes"] for r in per_layer)
+    peak, peak_kind = _measured_peak()
+    achieved = sum(r["algorithmic_bytes"] for r in per_layer) / (
+        sum(r["decode_avg_ms"] for r in per_layer) * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": kv_sum / (ms_sum * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_sum / n_layers,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAMES[cfg] + "; layers %d of %d, one resident at a time"
+                   % (n_layers, sp.layers), "config_id": cfg, "layers": n_layers,
+                   "l2": "inputs larger than L2 (K/V per layer-step above 5 GB vs 126 MB)"},
+        "tokens_per_s_per_layer": per_layer[0]["batch"] / (ms_sum / n_layers * 1e-3),
+        "per_layer": per_layer,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                     "kernel": "decode_kernel (mean over the layers)"},
+        "gpu_launches": sum(r["launches"] for r in per_layer),
+        "device_status": "ok" if not bad else "error word set", "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_splitzip(args):
     """SplitZip codec throughput on one GPU: the K and V pools of the GQA decode workload
     (config 2 shape, bf16) encoded and decoded back, each timed with CUDA events over
@@ -926,12 +1000,15 @@ def main():
                     help="code width of the tiered workloads' slow tier (config 5, ttkv-host)")
     ap.add_argument("--block-pages", type=int, default=8192,
                     help="--path ttkv-host: INT8-tier pages per streamed block")
+    ap.add_argument("--layers", type=int, default=32,
+                    help="--path layers: how many of config 3's layers to time, one at a time")
     ap.add_argument("--path", default="decode",
-                    choices=["decode", "sink", "h2o", "ttkv", "ttkv-host", "splitzip"],
+                    choices=["decode", "sink", "h2o", "ttkv", "ttkv-host", "splitzip", "layers"],
                     help="decode: the decode step (default); sink / h2o: the decode step with "
                          "the write path; ttkv: the tiered step with tier migration (config 5); "
                          "ttkv-host: the tiered step with the INT8 tier streamed from host "
-                         "memory (config 5); splitzip: the KV codec; one GPU, separate JSON line")
+                         "memory (config 5); splitzip: the KV codec; layers: config 3's step on "
+                         "each of its layers in turn; one GPU, separate JSON line")
     args = ap.parse_args()
     global SLOW_BITS
     SLOW_BITS = args.slow_bits
@@ -943,6 +1020,10 @@ def main():
         return run_splitzip(args)
     if args.path == "ttkv-host":
         return run_tier_host(args)
+    if args.path == "layers":
+        if args.layers < 1:
+            ap.error("--layers must be >= 1")
+        return run_layers(args)
     if args.path != "decode":
         return run_write_path(args)
     return run_ours(args)

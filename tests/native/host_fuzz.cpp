@@ -2,7 +2,7 @@
 // on seeded random inputs, built with AddressSanitizer and UndefinedBehaviorSanitizer by
 // tests/test_host_sanitizers.py. Plans are host-only; the device hooks the planner references
 // are stubbed below, so no GPU and no CUDA runtime are involved. Any sanitizer report aborts
-// with a non-zero status; the driver itself checks only what the host API promises (status
+// with a non-zero status; this program itself checks only what the host API promises (status
 // codes, exact page accounting).
 // A second drive injects allocation failures: this file replaces the global operator new, and
 // while a library call is armed the k-th allocation throws std::bad_alloc, for k = 0, 1, ...

@@ -262,11 +262,13 @@ def _multi_head_workload(rng, B=3, Hq=8, Hkv=2, D=64, maxn=120, page=16):
                 rows_v=rows_v, D=D, B=B, Hq=Hq, Hkv=Hkv, order=order, page=page)
 
 
-def test_gqa_mapping_against_per_row_sdpa():
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (8, 8), (8, 1)])
+def test_gqa_mapping_against_per_row_sdpa(Hq, Hkv):
     """Every query row against the library routine on its own KV head's rows: pins the
-    contiguous GQA mapping hq -> hq // (Hq/Hkv) and the per-(b, h) table offsets."""
-    rng = np.random.default_rng(9)
-    w = _multi_head_workload(rng)
+    contiguous GQA mapping hq -> hq // (Hq/Hkv) and the per-(b, h) table offsets; Hq = Hkv is
+    plain multi-head attention (G = 1), Hkv = 1 multi-query."""
+    rng = np.random.default_rng(9 + Hkv)
+    w = _multi_head_workload(rng, Hq=Hq, Hkv=Hkv)
     out, lse = oracle.decode(w["q"], w["kp"], w["vp"], w["table"], w["off"], w["kv"], 0.125)
     G = w["Hq"] // w["Hkv"]
     for b in range(w["B"]):

@@ -180,6 +180,25 @@ def test_full_size_layout_matches_oracle(cfg):
     ors.assert_same_layout(workload.layout(sp, 0), ors.layout(sp, 0))
 
 
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_pool_occupancy_as_specified(cfg):
+    """Pool sizes against the workloads' own statement, not against the shared formula: the tiny
+    workload's pool is exactly the used pages; the GQA layer's and the serving step's pools are
+    floor(used * 10 / 9) pages, so at least 90 % occupied, and one page more would not be."""
+    sp = synth.preset(cfg)
+    lay = workload.layout(sp, 0)
+    used = int(lay.head_count.sum())
+    assert used == int(((lay.kv_len.astype(np.int64) + 15) // 16).sum())
+    if cfg == 1:
+        assert lay.num_pages == used
+    else:
+        assert lay.num_pages == used * 10 // 9
+        assert used / lay.num_pages >= 0.9
+        assert used / (lay.num_pages + 1) < 0.9
+    ids = np.asarray(lay.page_ids)
+    assert len(np.unique(ids)) == used and ids.min() >= 0 and ids.max() < lay.num_pages
+
+
 def test_full_size_layout_matches_oracle_multi_layer():
     sp = synth.preset(3)
     for layer in (0, 31):

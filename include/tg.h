@@ -204,10 +204,10 @@ typedef struct tg_plan_opts {
 
 /* Build a plan. kv_len[B*Hkv] (host): retained tokens per (sequence, KV head); the decode
  * calls check the device copy against it. fast_len[B*Hkv] (host) or NULL: tiered plan whose
- * last min(fast_len, kv_len) tokens of each head are in the bf16 tier and the rest in the INT8
- * tier. group_of_head[Hkv] and group_off[n_groups+1] (host; from tg_budget_groups /
+ * last min(fast_len, kv_len) tokens of each head are in the bf16 tier and the rest in the slow
+ * tier (INT8, or INT4 with opts->slow_bits = 4). group_of_head[Hkv] and group_off[n_groups+1] (host; from tg_budget_groups /
  * tg_group_tables) bound every row of the bf16 (fast) table to its group table; for a tiered
- * plan slow_table_len bounds the INT8 tier's table (ignored otherwise).
+ * plan slow_table_len bounds the slow tier's table (ignored otherwise).
  * Each head's tokens are cut into chunks (min_splits, max_chunk_pages; chunks never cross a
  * tier boundary). The first static_permille of the chunks' byte cost is partitioned into
  * num_workers equal contiguous ranges assigned ahead of time (at least ~8 pages per worker;
@@ -449,8 +449,11 @@ typedef struct tg_slow_stream tg_slow_stream;
  * tg_plan_create for a tiered plan (kv_len, fast_len, group_of_head, group_off, n_groups over
  * the fast tier's group tables) plus the INT8 tier's HOST table (slow_page_table int32
  * [slow_table_len], slow_head_off int64 [B*Hkv]); shape->num_slow_pages = pages of the host pool.
- * opts as for tg_plan_create (out_f32 and capacity are set by the stream). TG_EINVAL on a bad
- * argument or a page id outside the pool. */
+ * opts as for tg_plan_create (out_f32 and capacity are set by the stream); with
+ * opts->slow_bits = 4 the host pool holds packed INT4 codes, uint8 [num_slow_pages][16][D/2]
+ * as tg_quantize_int4 writes them, and the ring is sized for them. Returns TG_EINVAL on a bad
+ * argument or a page id outside the pool, TG_EUNSUPPORTED for a kv_len above
+ * TG_MAX_HEAD_TOKENS, TG_ENOMEM when host or device memory runs out; *out is NULL on error. */
 int tg_slow_stream_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fast_len,
                           const int32_t *group_of_head, const int64_t *group_off,
                           int32_t n_groups, const int32_t *slow_page_table,

@@ -16,7 +16,9 @@
  *     §2.4.3 "加速单个请求": the online normaliser; Fig. 5 Dist Attention).
  *
  * Conventions for every function:
- *   - Return value: TG_OK (0) or one of the TG_E* codes below. Nothing throws across the ABI.
+ *   - Return value: TG_OK (0) or one of the TG_E* codes below. Nothing throws across the ABI
+ *     (one exception, stated at tg_plan_timing_enable); host allocation failures return
+ *     TG_ENOMEM and leave the objects as they were.
  *   - Host pointers are read during the call only. Device pointers are caller-owned device
  *     memory (allocate them with any allocator); the library never frees them.
  *   - Device calls are stream-ordered and asynchronous on the given stream; they allocate
@@ -285,7 +287,9 @@ int tg_plan_status(tg_plan *p, tg_stream stream);
  * overlap); later calls record nothing. The events are created here (no device memory);
  * max_calls = 0 destroys them. tg_plan_timing_read waits for the last recorded event, returns
  * the number of calls recorded and the summed decode-kernel and merge-kernel times in
- * milliseconds, and restarts the count. */
+ * milliseconds, and restarts the count. The host table of 3 * max_calls events is the one
+ * allocation in this library whose failure is not turned into TG_ENOMEM (std::bad_alloc
+ * propagates): keep max_calls to what the caller means to time (the bench uses <= 256). */
 int tg_plan_timing_enable(tg_plan *p, int32_t max_calls);
 int tg_plan_timing_read(tg_plan *p, int32_t *n_calls, double *decode_ms, double *merge_ms);
 

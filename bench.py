@@ -90,10 +90,22 @@ def _my_sequences(sp, rank, world, kv_len, fast_len):
     if fast_len is None:
         per_seq = kv_len.astype(np.int64).sum(1) * 2 * sp.D * 2
     else:
-        f = fast_len.astype(np.int64)
-        per_seq = ((kv_len - f) * 2 * (sp.D + 4) + f * 2 * sp.D * 2).sum(1)
+        f = np.minimum(fast_len, kv_len).astype(np.int64)
+        slow_row = sp.D if sp.slow_bits == 8 else sp.D // 2     # code bytes per slow token-head
+        per_seq = ((kv_len - f) * 2 * (slow_row + 4) + f * 2 * sp.D * 2).sum(1)
     gpu = tg.tg_place_sequences(per_seq, world)
     return np.nonzero(gpu == rank)[0]
+
+
+def _over_ranks(dist, vals, n_max):
+    """The first n_max entries of vals (times, error flags) as their maximum over ranks, the
+    rest (work done) as their sum; vals is a float64 tensor on the process group's device."""
+    if dist is None:
+        return vals.tolist()
+    mx, sm = vals.clone(), vals.clone()
+    dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+    dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+    return mx[:n_max].tolist() + sm[n_max:].tolist()
 
 
 def _measured_peak():
@@ -420,20 +432,11 @@ def run_ours(args):
     pipe.destroy()
     barrier()
 
-    # Max over ranks (time) and sums (work).
-    vals = torch.tensor([ms_total, e2e_ms, dec_ms / max(n_rec, 1), float(alg["kv"]),
-                         float(B_local), float(status != tg.TG_OK)], dtype=torch.float64,
+    # Max over ranks (time, error flag) and sums (work).
+    vals = torch.tensor([ms_total, e2e_ms, dec_ms / max(n_rec, 1), float(status != tg.TG_OK),
+                         float(alg["kv"]), float(B_local)], dtype=torch.float64,
                         device=f"cuda:{local}")
-    if dist is not None:
-        mx = vals.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        sm = vals.clone()
-        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
-        ms_total, e2e_ms, dec_avg = mx[0].item(), mx[1].item(), mx[2].item()
-        kv_total, b_total, bad = sm[3].item(), sm[4].item(), mx[5].item()
-    else:
-        dec_avg = vals[2].item()
-        kv_total, b_total, bad = float(alg["kv"]), float(B_local), float(status != tg.TG_OK)
+    ms_total, e2e_ms, dec_avg, bad, kv_total, b_total = _over_ranks(dist, vals, 4)
 
     ms_step = ms_total / args.steps
     value = kv_total / (ms_step * 1e-3) / 1e9

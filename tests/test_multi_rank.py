@@ -28,76 +28,91 @@ def _init(rank, world, port, timeout_s=30):
                             world_size=world, timeout=datetime.timedelta(seconds=timeout_s))
 
 
-def _shard_worker(rank, world, port, cfg, q):
+def _shard_worker(rank, world, port, cfg, slow_bits, q):
+    """One rank of `bench.py --gpus N`'s set-up, on the bench's own functions and full-size
+    workloads: the global spec, this rank's sequences by ahead-of-time placement, its layout
+    (checked against the oracle's) and plan, and the max / sum reduction over ranks."""
     try:
         sys.path.insert(0, ROOT)
         import torch
+        import bench
         import non_uniform_paged_flash_b200 as tg
-        import synth
-        from dataclasses import replace
         from non_uniform_paged_flash_b200 import workload
         from oracle import workload as ow
 
         _init(rank, world, port)
-        sp = replace(synth.small(cfg), B=synth.small(cfg).B * world)
+        bench.SLOW_BITS = slow_bits
+        sp = bench._global_spec(cfg, world)
         kv, fast = workload.retained(sp, 0)
-        per_seq = kv.astype(np.int64).sum(1) * 2 * sp.D * 2 if fast is None else \
-            ((kv - fast) * 2 * (sp.D + 4) + fast * 2 * sp.D * 2).sum(1)
-        gpu = tg.tg_place_sequences(per_seq, world)
-        mine = np.nonzero(gpu == rank)[0]
+        mine = bench._my_sequences(sp, rank, world, kv, fast)
         lay = workload.layout(sp, 0, mine)
         ow.assert_same_layout(lay, ow.layout(sp, 0, mine))
         shape = tg.make_shape(len(mine), sp.Hq, sp.Hkv, sp.D, lay.num_pages, lay.num_slow_pages)
         plan = tg.tg_plan_create(shape, lay.kv_len, lay.group_of_head, lay.group_off,
                                  fast_len=lay.fast_len,
                                  slow_table_len=0 if lay.slow_table is None else lay.slow_table.size,
-                                 host_only=True, num_workers=64)
+                                 host_only=True, num_workers=64, slow_bits=slow_bits if fast is not None else 0)
         items = tg.tg_plan_items(plan)
         pages_local = int((items[:, 2] - items[:, 1]).sum())
-        # gather: sequences and page counts of every rank
-        t = torch.tensor([len(mine), pages_local, int(per_seq[mine].sum())], dtype=torch.int64)
-        allt = [torch.zeros_like(t) for _ in range(world)]
-        dist.all_gather(allt, t)
+        # the bench's reduction: times / flags as the max over ranks, work as the sum
+        vals = torch.tensor([float(rank + 1), 10.0 * (rank + 1), float(len(mine)), float(pages_local)],
+                            dtype=torch.float64)
+        reduced = bench._over_ranks(dist, vals, 2)
         seqs = torch.from_numpy(np.pad(mine, (0, sp.B - len(mine)), constant_values=-1))
         alls = [torch.zeros_like(seqs) for _ in range(world)]
         dist.all_gather(alls, seqs)
         dist.barrier()
         dist.destroy_process_group()
-        q.put((rank, [x.tolist() for x in allt], [x.numpy() for x in alls], per_seq.tolist(),
-               None))
+        q.put((rank, reduced, [x.numpy() for x in alls], sp.B, None))
     except Exception:
         q.put((rank, None, None, None, traceback.format_exc()))
 
 
-@pytest.mark.parametrize("cfg", [2, 4, 5])
-def test_two_rank_shards_cover_batch_once_and_balance(cfg):
+def _seq_bytes(sp, kv, fast, slow_bits):
+    """Retained K/V bytes per sequence, written out from the tier layouts (bf16 K + V: 4 D per
+    token-head; a slow token-head: codes of K and V plus two fp32 scales)."""
+    if fast is None:
+        return kv.astype(np.int64).sum(1) * 4 * sp.D
+    f = np.minimum(fast, kv).astype(np.int64)
+    code = sp.D if slow_bits == 8 else sp.D // 2
+    return ((kv - f) * (2 * code + 8) + f * 4 * sp.D).sum(1)
+
+
+@pytest.mark.parametrize("cfg,slow_bits", [(2, 8), (4, 8), (5, 8), (5, 4)])
+def test_two_rank_shards_cover_batch_once_and_balance(cfg, slow_bits):
     world, port = 2, _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, cfg, q)) for r in range(world)]
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, cfg, slow_bits, q))
+             for r in range(world)]
     for p in procs:
         p.start()
     res = [q.get(timeout=180) for _ in range(world)]
     for p in procs:
         p.join(timeout=60)
-    for rank, allt, alls, per_seq, err in res:
+    for rank, reduced, alls, B, err in res:
         assert err is None, err
-    _, allt, alls, per_seq, _ = res[0]
-    seqs = np.concatenate([a[a >= 0] for a in alls])
-    assert sorted(seqs.tolist()) == list(range(len(per_seq)))           # each exactly once
-    loads = [x[2] for x in allt]
-    assert max(loads) <= sum(per_seq) / world + max(per_seq)            # LPT bound
-    # pages of the shards add up to the pages of the whole batch
     import synth
     from dataclasses import replace
     from oracle import workload as ow
-    sp = replace(synth.small(cfg), B=synth.small(cfg).B * world)
+    _, reduced, alls, B, _ = res[0]
+    seqs = np.concatenate([a[a >= 0] for a in alls])
+    assert sorted(seqs.tolist()) == list(range(B))                     # each exactly once
+    sp = replace(synth.preset(cfg), B=B)
+    if sp.kind == "tiered":
+        sp = replace(sp, slow_bits=slow_bits)
     kv, fast = ow.retained(sp, 0)
+    per_seq = _seq_bytes(sp, kv, fast, slow_bits)
+    loads = [int(per_seq[a[a >= 0]].sum()) for a in alls]
+    assert max(loads) <= per_seq.sum() / world + per_seq.max()        # LPT bound
+    # every rank sees the same reduction: max of the times, sums of the work
     if fast is None:
-        want = int(((kv.astype(np.int64) + 15) // 16).sum())
+        want_pages = int(((kv.astype(np.int64) + 15) // 16).sum())
     else:
-        want = int((((kv - fast).astype(np.int64) + 15) // 16 + (fast.astype(np.int64) + 15) // 16).sum())
-    assert sum(x[1] for x in allt) == want
+        f = np.minimum(fast, kv).astype(np.int64)
+        want_pages = int((((kv - f) + 15) // 16 + (f + 15) // 16).sum())
+    for _, r, _, _, _ in res:
+        assert r == [float(world), 10.0 * world, float(B), float(want_pages)]
 
 
 def _dying_worker(rank, world, port, q):

@@ -32,3 +32,23 @@ def test_host_code_is_clean_under_asan_and_ubsan():
     assert r.returncode == 0, (r.stdout + r.stderr)[-4000:]
     assert "200 rounds clean" in r.stdout
     assert "allocation failures: 20 rounds" in r.stdout
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+def test_oracle_is_clean_under_asan_and_ubsan():
+    """The CPU oracle's C code (oracle/tg_oracle.c) under the same sanitizers, every exported
+    function on seeded random cases (tests/native/oracle_fuzz.c; OpenMP off, so one thread)."""
+    out_dir = os.path.join(ROOT, "tests", "native", "_build")   # git-ignored
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "oracle_fuzz")
+    cmd = ["gcc", "-std=c11", "-O1", "-g", "-fsanitize=address,undefined,float-cast-overflow",
+           "-fno-sanitize-recover=all", "-fno-omit-frame-pointer", "-Wno-unknown-pragmas",
+           os.path.join(ROOT, "tests", "native", "oracle_fuzz.c"),
+           os.path.join(ROOT, "oracle", "tg_oracle.c"), "-lm", "-o", str(exe)]
+    subprocess.check_call(cmd)
+    env = dict(os.environ, ASAN_OPTIONS="detect_leaks=1:abort_on_error=0",
+               UBSAN_OPTIONS="print_stacktrace=1")
+    r = subprocess.run([str(exe), "300", "20261202"], capture_output=True, text=True, env=env,
+                       timeout=600)
+    assert r.returncode == 0, (r.stdout + r.stderr)[-4000:]
+    assert "300 rounds clean" in r.stdout

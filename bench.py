@@ -260,8 +260,10 @@ def run_reference(args):
 # Our arm
 # ------------------------------------------------------------------------------------------
 
-def cpu_baseline(cfg, budget_s=20.0, min_s=10.0):
-    """The oracle as it stands on a bounded sample of this workload (rank 0, N = 1)."""
+def cpu_baseline(cfg, budget_s=20.0, min_s=10.0, sample=None):
+    """The oracle as it stands on a bounded sample of this workload (rank 0, N = 1). With a
+    list `sample`, the first chunk's (row ids, (out, lse)) is appended to it, for the parity
+    check of the bench line."""
     import oracle
     from oracle import workload as ow
     sp = _preset(cfg)
@@ -275,7 +277,7 @@ def cpu_baseline(cfg, budget_s=20.0, min_s=10.0):
         row_bytes = kv * 2 * sp.D * 2
 
         def rows(sel):
-            oracle.decode(q, k, v, o.table, o.head_off, o.kv_len, sp.scale, sel=sel)
+            return oracle.decode(q, k, v, o.table, o.head_off, o.kv_len, sp.scale, sel=sel)
     else:
         kq, ks, vq, vs = ow.slow_tier(sp, o)
         st = o.slow_table if o.slow_table.size else np.zeros(1, np.int32)
@@ -284,8 +286,8 @@ def cpu_baseline(cfg, budget_s=20.0, min_s=10.0):
         row_bytes = (kv - f) * 2 * (cb + 4) + f * 2 * sp.D * 2
 
         def rows(sel):
-            oracle.tiered_decode(q, kq, vq, ks, vs, st, o.slow_off, k, v, o.table, o.head_off,
-                                 o.kv_len, o.fast_len, sp.scale, sel=sel)
+            return oracle.tiered_decode(q, kq, vq, ks, vs, st, o.slow_off, k, v, o.table,
+                                        o.head_off, o.kv_len, o.fast_len, sp.scale, sel=sel)
     # passes over the batch, a few sequences at a time, until min_s of oracle time (or the
     # budget) is spent
     done, nbytes, t_used, passes = 0, 0, 0.0, 0
@@ -294,8 +296,10 @@ def cpu_baseline(cfg, budget_s=20.0, min_s=10.0):
         b1 = min(sp.B, done + chunk)
         sel = np.arange(done * sp.Hq, b1 * sp.Hq)
         t0 = time.perf_counter()
-        rows(sel)
+        res = rows(sel)
         t_used += time.perf_counter() - t0
+        if sample is not None and not sample:
+            sample.append((sel, res))
         nbytes += int(row_bytes[done:b1].sum())
         done = b1
         if done == sp.B:
@@ -304,6 +308,22 @@ def cpu_baseline(cfg, budget_s=20.0, min_s=10.0):
     return {"value": nbytes / t_used / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"{seqs} (all their query rows), {t_used:.1f} s of fp64 oracle time on "
                       f"{cores} host threads"}
+
+
+def _parity_sample(first, db, D):
+    """Max-abs differences of the timed step's outputs from the fp64 oracle on the rows the
+    CPU baseline computed (its first chunk of sequences, every query row of them)."""
+    try:
+        sel, (o_ref, l_ref) = first[0]
+        out = db.out.float().reshape(-1, D).cpu().numpy()[sel]
+        lse = db.lse.reshape(-1).cpu().numpy()[sel]
+        fin = np.isfinite(l_ref)
+        assert np.array_equal(fin, np.isfinite(lse)), "empty heads differ"
+        return {"rows": int(len(sel)), "max_abs_out": float(np.abs(out - o_ref).max()),
+                "max_abs_lse": float(np.abs(lse[fin] - l_ref[fin]).max()) if fin.any() else 0.0,
+                "tolerance": {"out": 2e-2, "lse": 1e-3}}
+    except Exception as e:   # the line is still printed; the failure is recorded in it
+        return {"error": (type(e).__name__ + ": " + str(e))[:200]}
 
 
 def run_ours(args):
@@ -487,7 +507,9 @@ def run_ours(args):
         if world == 1 and cfg == 1:
             line["graph_replay"] = graph_replay(db, alg)
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(cfg)
+            first = []
+            line["cpu_baseline"] = cpu_baseline(cfg, sample=first)
+            line["parity_sample"] = _parity_sample(first, db, sp.D)
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

@@ -65,6 +65,7 @@ def _plan_kw(cfg):
 
 
 SLOW_BITS = 8   # code width of the tiered workloads' slow tier (--slow-bits)
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e nominal bandwidth (context beside the measured peak)
 
 
 def _preset(cfg):
@@ -484,6 +485,8 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": _traffic(cfg) if world == 1 else None,
                          "peak_kind": peak_kind,
+                         "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
+                         "nominal_gbs": NOMINAL_HBM_GBS,
                          "kernel": "cascade_kernel + decode_kernel" if info["n_cascade"] > 0
                          else "decode_kernel",
                          "algorithmic_bytes_per_launch": alg["total"],

@@ -569,15 +569,23 @@ def _hostp(t):
 
 
 class HostPipe:
-    """Owns a tg_host_pipe handle (two device staging sets, two copy streams)."""
+    """Owns a tg_host_pipe handle (two device staging sets, two copy streams). The host tensors
+    of every call are kept alive here until wait() or destroy(), since the pipe's copies read
+    and write them after the call returns."""
 
     def __init__(self, plan: Plan):
         h = ctypes.c_void_p()
+        self._held = {}
         _check(_lib().tg_host_pipe_create(plan.handle, ctypes.byref(h)), "tg_host_pipe_create")
         self.handle = h
 
+    def _hold(self, *tensors):
+        for t in tensors:
+            self._held[id(t)] = t
+
     def wait(self):
         _check(_lib().tg_host_pipe_wait(self.handle), "tg_host_pipe_wait")
+        self._held.clear()
 
     def after(self, stream=None):
         _check(_lib().tg_host_pipe_after(self.handle, _stream(stream)), "tg_host_pipe_after")
@@ -587,8 +595,9 @@ class HostPipe:
 
     def destroy(self):
         if self.handle:
-            _lib().tg_host_pipe_destroy(self.handle)
+            _lib().tg_host_pipe_destroy(self.handle)   # waits for the pipe's copies
             self.handle = ctypes.c_void_p()
+        self._held.clear()
 
     def __del__(self):
         try:
@@ -606,6 +615,7 @@ def tg_ragged_paged_decode_host(pipe: HostPipe, plan: Plan, q_host, k_pages, v_p
                                 out_host, lse_host, stream=None):
     """tg_ragged_paged_decode with q read from, and out / lse written to, pinned host tensors
     (asynchronous: read the outputs after pipe.wait())."""
+    pipe._hold(q_host, out_host, lse_host)
     _check(_lib().tg_ragged_paged_decode_host(
         pipe.handle, plan.handle, _hostp(q_host), _dp(k_pages), _dp(v_pages), _dp(page_table),
         _dp(head_page_off), _dp(head_kv_len), _dp(group_of_head), float(scale),
@@ -617,6 +627,7 @@ def tg_tiered_decode_host(pipe: HostPipe, plan: Plan, q_host, k_q8, v_q8, k_scal
                           fast_head_off, head_kv_len, head_fast_len, scale: float, out_host,
                           lse_host, stream=None):
     """tg_tiered_decode with pinned host q / out / lse (see tg_ragged_paged_decode_host)."""
+    pipe._hold(q_host, out_host, lse_host)
     _check(_lib().tg_tiered_decode_host(
         pipe.handle, plan.handle, _hostp(q_host), _dp(k_q8), _dp(v_q8), _dp(k_scale),
         _dp(v_scale), _dp(slow_page_table), _dp(slow_head_off), _dp(k_fast), _dp(v_fast),

@@ -641,7 +641,9 @@ def tg_tiered_decode_host(pipe: HostPipe, plan: Plan, q_host, k_q8, v_q8, k_scal
 # ------------------------------------------------------------------------------------------
 
 class SlowStream:
-    """Owns a tg_slow_stream handle (per-block plans, HBM ring, copy stream)."""
+    """Owns a tg_slow_stream handle (per-block plans, HBM ring, copy stream). The host pools
+    of its calls are kept alive here until destroy(), since the copy stream reads them after
+    a call returns."""
 
     def __init__(self, shape: tg_shape, kv_len, fast_len, group_of_head, group_off,
                  slow_page_table, slow_head_off, block_pages: int, ring_blocks: int = 3,
@@ -649,6 +651,7 @@ class SlowStream:
                  host_only: bool = False, device: int = -1, static_permille: int = 0,
                  dyn_chunk_pages: int = 0, early_prologue: bool = False, slow_bits: int = 8):
         self.shape = shape
+        self._held = {}
         kv = _h(kv_len, np.int32).reshape(-1)
         fl = _h(fast_len, np.int32).reshape(-1)
         goh = _h(group_of_head, np.int32).reshape(-1)
@@ -681,8 +684,9 @@ class SlowStream:
 
     def destroy(self):
         if self.handle:
-            _lib().tg_slow_stream_destroy(self.handle)
+            _lib().tg_slow_stream_destroy(self.handle)   # waits for the stream's copies
             self.handle = ctypes.c_void_p()
+        self._held.clear()
 
     def __del__(self):
         try:
@@ -695,6 +699,8 @@ def tg_tiered_decode_streamed(ss: SlowStream, q, k_q8_host, v_q8_host, k_scale_h
                               v_scale_host, k_fast, v_fast, fast_page_table, fast_head_off,
                               group_of_head, scale: float, out, lse, stream=None):
     """Tiered decode with the INT8 tier in pinned host memory, streamed block-wise."""
+    for t in (k_q8_host, v_q8_host, k_scale_host, v_scale_host):
+        ss._held[id(t)] = t
     _check(_lib().tg_tiered_decode_streamed(
         ss.handle, _dp(q), _hostp(k_q8_host), _hostp(v_q8_host), _hostp(k_scale_host),
         _hostp(v_scale_host), _dp(k_fast), _dp(v_fast), _dp(fast_page_table), _dp(fast_head_off),

@@ -126,7 +126,8 @@ extern "C" int tg_host_pipe_create(const tg_plan *plan, tg_host_pipe **out) {
                 (e = cudaEventCreateWithFlags(&p->ev_d2h[s], cudaEventDisableTiming)) != cudaSuccess)
                 status = fail("cudaEventCreateWithFlags", e);
     }
-    cudaSetDevice(prev);
+    // The caller's device comes back, or the pipe is not made (its calls would run elsewhere).
+    if ((e = cudaSetDevice(prev)) != cudaSuccess && status == TG_OK) status = fail("cudaSetDevice", e);
     if (status != TG_OK) {
         release(p);
         return status;

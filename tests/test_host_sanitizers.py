@@ -52,3 +52,30 @@ def test_oracle_is_clean_under_asan_and_ubsan():
                        timeout=600)
     assert r.returncode == 0, (r.stdout + r.stderr)[-4000:]
     assert "300 rounds clean" in r.stdout
+
+
+CUDA_INCLUDE = "/usr/local/cuda/include"
+
+
+@pytest.mark.skipif(shutil.which("g++") is None or not os.path.exists(
+    os.path.join(CUDA_INCLUDE, "cuda_runtime.h")), reason="needs g++ and the CUDA headers")
+def test_host_pipe_failure_paths_with_a_fake_runtime():
+    """The host-buffer pipe (csrc/tg_pipe.cpp) against stubs of the CUDA runtime calls it makes
+    (tests/native/pipe_faults.cpp): each runtime call failing in turn is reported, creation
+    hands back nothing and leaks nothing, the pipe serves the next call; under ASan/UBSan."""
+    out_dir = os.path.join(ROOT, "tests", "native", "_build")   # git-ignored
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "pipe_faults")
+    cmd = ["g++", "-std=c++17", "-O1", "-g", "-fsanitize=address,undefined",
+           "-fno-sanitize-recover=undefined", "-fno-omit-frame-pointer",
+           "-I", os.path.join(ROOT, "include"),
+           "-I", os.path.join(ROOT, "non_uniform_paged_flash_b200", "csrc"), "-I", CUDA_INCLUDE,
+           os.path.join(ROOT, "tests", "native", "pipe_faults.cpp"),
+           os.path.join(ROOT, "non_uniform_paged_flash_b200", "csrc", "tg_pipe.cpp"),
+           "-o", str(exe)]
+    subprocess.check_call(cmd)
+    env = dict(os.environ, ASAN_OPTIONS="detect_leaks=1:abort_on_error=0",
+               UBSAN_OPTIONS="print_stacktrace=1")
+    r = subprocess.run([str(exe)], capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0, (r.stdout + r.stderr)[-4000:]
+    assert "every one reported, nothing leaked" in r.stdout

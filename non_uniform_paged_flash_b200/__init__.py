@@ -14,7 +14,6 @@ from __future__ import annotations
 import ctypes
 import os
 from dataclasses import dataclass
-from typing import Optional
 
 import numpy as np
 

@@ -13,7 +13,7 @@ from __future__ import annotations
 import ctypes
 import os
 import subprocess
-from dataclasses import dataclass, field, replace
+from dataclasses import dataclass, replace
 from typing import Optional
 
 import numpy as np

@@ -3,7 +3,6 @@ random retained lengths, shared segments, per-sequence segment chains (with abse
 shuffled free orders and page sizes; the library's page ids and segment pages must equal the
 oracle's bit for bit, and a pool one page short must be refused with nothing taken."""
 import numpy as np
-import pytest
 from hypothesis import given, settings, strategies as st
 
 import non_uniform_paged_flash_b200 as tg

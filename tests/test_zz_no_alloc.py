@@ -4,7 +4,6 @@ framework owns every device allocation). It must give the results of the plan-ba
 point, call after call, with its scratch in the library's fixed device array.
 
 Kept in a file of its own, collected last: if it fails, every other test has already run."""
-import numpy as np
 import pytest
 import torch
 

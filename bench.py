@@ -68,6 +68,14 @@ SLOW_BITS = 8   # code width of the tiered workloads' slow tier (--slow-bits)
 NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e nominal bandwidth (context beside the measured peak)
 
 
+def _workload_name(cfg, sp):
+    """The workload's name, with the slow tier's code width where it is not the named INT8."""
+    name = WORKLOAD_NAMES[cfg]
+    if sp.kind == "tiered" and sp.slow_bits == 4:
+        name = name.replace("older INT8", "older INT4") if "older INT8" in name else name + " (INT4 slow tier)"
+    return name
+
+
 def _preset(cfg):
     """The named workload; tiered ones with the slow tier at SLOW_BITS."""
     from dataclasses import replace
@@ -204,7 +212,7 @@ def run_reference(args):
     import oracle
     from oracle import workload as ow
     cfg = args.config
-    sp = synth.preset(cfg)
+    sp = _preset(cfg)
     o = ow.layout(sp, 0)
     q = ow.q_bits(sp)
     G = sp.Hq // sp.Hkv
@@ -220,8 +228,8 @@ def run_reference(args):
     else:
         k = synth.pool_bits(sp, "k", o.num_pages)
         v = synth.pool_bits(sp, "v", o.num_pages)
-        kq, ks = oracle.quantize_int8(synth.pool_bits(sp, "kslow", o.num_slow_pages))
-        vq, vs = oracle.quantize_int8(synth.pool_bits(sp, "vslow", o.num_slow_pages))
+        kq, ks, vq, vs = ow.slow_tier(sp, o)            # INT8, or INT4 codes widened to int8
+        cb = sp.D // 2 if sp.slow_bits == 4 else sp.D  # stored code bytes per slow token-head
 
         def step(b):
             # one KV head of one sequence per step (bounded: the heads are 131072 tokens)
@@ -230,8 +238,9 @@ def run_reference(args):
             sel = np.arange(bb * sp.Hq + h * G, bb * sp.Hq + (h + 1) * G)
             oracle.tiered_decode(q, kq, vq, ks, vs, o.slow_table, o.slow_off, k, v, o.table,
                                  o.head_off, o.kv_len, o.fast_len, sp.scale, sel=sel)
-            n, f = int(o.kv_len[bb, h]), int(o.fast_len[bb, h])
-            return (n - f) * 2 * (sp.D + 4) + f * 2 * sp.D * 2
+            n = int(o.kv_len[bb, h])
+            f = min(int(o.fast_len[bb, h]), n)
+            return (n - f) * 2 * (cb + 4) + f * 2 * sp.D * 2
     for i in range(args.warmup):
         step(i % sp.B)
     t0 = time.perf_counter()
@@ -248,7 +257,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD_NAMES[cfg], "config_id": cfg},
+            "config": {"workload": _workload_name(cfg, sp), "config_id": cfg},
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -472,8 +481,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if lay.fast_len is None else "bf16+int%d" % sp.slow_bits,
             "data": "synthetic",
-            "config": {"workload": WORKLOAD_NAMES[cfg] + ("" if sp.slow_bits == 8 or lay.fast_len is None
-                                                          else " (INT4 slow tier)"), "config_id": cfg,
+            "config": {"workload": _workload_name(cfg, sp), "config_id": cfg,
                        "global_batch": int(b_total), "parallelism":
                        "sequence shards by AOT byte placement, no collective" if world > 1
                        else "single GPU",
@@ -786,7 +794,7 @@ def run_tier_path(args):
         "metric": "tiered decode step with tier migration: step time", "value": ms_step * 1e3,
         "unit": "us", "higher_is_better": False, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup,
-        "config": {"workload": WORKLOAD_NAMES[cfg], "config_id": cfg, "plan": "capacity",
+        "config": {"workload": _workload_name(cfg, sp), "config_id": cfg, "plan": "capacity",
                    "slow_tier": "INT%d" % sp.slow_bits},
         "dtype": "bf16+int%d" % sp.slow_bits, "data": "synthetic",
         "kernels_us": {"tier_append": t_app * 1e3, "decode+merge": t_dec * 1e3},

@@ -135,7 +135,7 @@ def group_tables(group_of_head, n_groups, page_ids, head_count):
     cap = 0
     for g in range(n_groups):
         hs = [h for h in range(Hkv) if goh[h] == g]
-        if hs:
+        if hs and B > 0:
             cap += B * len(hs) * int(cnt[:, hs].max())
     table = np.empty(max(cap, 1), dtype=np.int32)
     off = np.empty((B, Hkv), dtype=np.int64)

@@ -97,3 +97,40 @@ def test_pool_one_page_short_is_refused_without_taking_pages(case):
         assert refused
     finally:
         tg.tg_alloc_destroy(a)
+
+
+@settings(max_examples=200, deadline=None)
+@given(st.integers(0, 7), st.integers(1, 9), st.integers(1, 9), st.integers(0, 12), st.integers(0, 2**32 - 1))
+def test_group_tables_equal_oracle(B, H, G, max_pages, seed):
+    """Group page tables (any group map, empty groups included) against the oracle's."""
+    G = min(G, H)
+    rng = np.random.default_rng(seed)
+    cnt = rng.integers(0, max_pages + 1, (B, H)).astype(np.int32)
+    goh = rng.integers(0, G, H).astype(np.int32)
+    ids = rng.permutation(int(cnt.sum()) + 2)[: int(cnt.sum())].astype(np.int32)
+    t, off, goff = tg.tg_group_tables(cnt, goh, G, ids)
+    ot, ooff, ogoff = oracle.group_tables(goh, G, ids, cnt)
+    np.testing.assert_array_equal(t, ot)
+    np.testing.assert_array_equal(goff, ogoff)
+    np.testing.assert_array_equal(off, ooff)
+
+
+@settings(max_examples=200, deadline=None)
+@given(st.lists(st.integers(0, 10**9), min_size=0, max_size=60), st.integers(1, 9))
+def test_placement_equals_oracle(seq_bytes, n_gpus):
+    """Ahead-of-time placement (ties included) against the oracle's LPT."""
+    b = np.asarray(seq_bytes, dtype=np.int64)
+    np.testing.assert_array_equal(tg.tg_place_sequences(b, n_gpus), oracle.place_sequences(b, n_gpus))
+
+
+@settings(max_examples=200, deadline=None)
+@given(st.lists(st.tuples(st.integers(0, 2**31 - 1), st.integers(0, 1_000_000)), min_size=1, max_size=40),
+       st.integers(1, 8))
+def test_lengths_and_groups_equal_oracle(pairs, n_groups):
+    """Retained lengths (full int32 range of lengths) and budget groups against the oracle's."""
+    full = np.array([p[0] for p in pairs], dtype=np.int32)
+    ratio = np.array([p[1] for p in pairs], dtype=np.int32)
+    np.testing.assert_array_equal(tg.tg_retained_lengths(full, ratio),
+                                  oracle.retained_lengths(full, ratio))
+    G = min(n_groups, len(pairs))
+    np.testing.assert_array_equal(tg.tg_budget_groups(ratio, G), oracle.budget_groups(ratio, G))

@@ -178,6 +178,14 @@ def _hp(a):
     return None if a is None else a.ctypes.data
 
 
+def _count(a, n, what, at_least=False):
+    """A host array holds n entries (at least n with at_least): the C side reads that many."""
+    if a is None:
+        return
+    if (a.size < n) if at_least else (a.size != n):
+        raise ValueError(f"{what}: {a.size} entries, {'at least ' if at_least else ''}{n} expected")
+
+
 def _dp(t):
     """Device pointer of a CUDA tensor (None -> NULL)."""
     if t is None:
@@ -239,7 +247,8 @@ def tg_budget_groups(budget_ppm, n_groups: int) -> np.ndarray:
 
 
 def tg_alloc_create(num_pages: int, page: int = 16, free_order=None):
-    fo = None if free_order is None else _h(free_order, np.int32)
+    fo = None if free_order is None else _h(free_order, np.int32).reshape(-1)
+    _count(fo, num_pages, "free_order")
     h = ctypes.c_void_p()
     _check(_lib().tg_alloc_create(num_pages, page, _hp(fo), ctypes.byref(h)), "tg_alloc_create")
     return h
@@ -292,8 +301,10 @@ def tg_group_tables(head_count, group_of_head, n_groups: int, page_ids):
     """Returns (table int32[len], head_off int64[B, Hkv], group_off int64[n_groups + 1])."""
     hc = _h(head_count, np.int32)
     B, Hkv = hc.shape
-    goh = _h(group_of_head, np.int32)
-    ids = _h(page_ids, np.int32)
+    goh = _h(group_of_head, np.int32).reshape(-1)
+    ids = _h(page_ids, np.int32).reshape(-1)
+    _count(goh, Hkv, "group_of_head")
+    _count(ids, int(np.maximum(hc, 0).astype(np.int64).sum()), "page_ids", at_least=True)
     goff = np.empty(n_groups + 1, dtype=np.int64)
     _check(_lib().tg_group_tables(B, Hkv, _hp(hc), _hp(goh), n_groups, None, None, None,
                                   _hp(goff)), "tg_group_tables")
@@ -350,6 +361,10 @@ def tg_plan_create(shape: tg_shape, kv_len, group_of_head, group_off, fast_len=N
     fl = None if fast_len is None else _h(fast_len, np.int32).reshape(-1)
     goh = _h(group_of_head, np.int32).reshape(-1)
     goff = _h(group_off, np.int64).reshape(-1)
+    _count(kv, shape.B * shape.Hkv, "kv_len")
+    _count(fl, shape.B * shape.Hkv, "fast_len")
+    _count(goh, shape.Hkv, "group_of_head")
+    _count(goff, 2, "group_off", at_least=True)
     opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
                         static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us,
                         test_withhold_page, int(capacity), int(out_f32), int(slow_bits),
@@ -373,6 +388,10 @@ def tg_plan_create_cascade(shape: tg_shape, kv_len, group_of_head, group_off, pa
     goff = _h(group_off, np.int64).reshape(-1)
     tbl = _h(page_table, np.int32).reshape(-1)
     hoff = _h(head_page_off, np.int64).reshape(-1)
+    _count(kv, shape.B * shape.Hkv, "kv_len")
+    _count(goh, shape.Hkv, "group_of_head")
+    _count(goff, 2, "group_off", at_least=True)
+    _count(hoff, shape.B * shape.Hkv, "head_page_off")
     opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
                         static_permille, dyn_chunk_pages, int(early_prologue), wait_limit_us, 0, 0,
                         int(out_f32), 8)
@@ -657,6 +676,12 @@ class SlowStream:
         goff = _h(group_off, np.int64).reshape(-1)
         tbl = _h(slow_page_table, np.int32).reshape(-1)
         off = _h(slow_head_off, np.int64).reshape(-1)
+        BH = shape.B * shape.Hkv
+        _count(kv, BH, "kv_len")
+        _count(fl, BH, "fast_len")
+        _count(goh, shape.Hkv, "group_of_head")
+        _count(goff, 2, "group_off", at_least=True)
+        _count(off, BH, "slow_head_off")
         opts = tg_plan_opts(num_workers, min_splits, max_chunk_pages, int(host_only), device,
                             static_permille, dyn_chunk_pages, int(early_prologue), 0, 0, 0, 0,
                             int(slow_bits))

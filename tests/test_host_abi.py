@@ -1,6 +1,7 @@
 """CPU tests of the C ABI: the library loads and exports every declared symbol, and its host
 steps (retained lengths, groups, reservation, group tables, placement, the planner) agree bit
 for bit with the oracle's own derivation. No device calls."""
+import ctypes
 import os
 import re
 
@@ -468,11 +469,23 @@ def test_plan_rejects_unsupported_shapes_and_lengths():
     ok = dict(host_only=True, num_workers=16, whole_heads=True)
     for shape in (tg.make_shape(1, 6, 2, 128, 1 << 20),      # 3 query heads per KV head
                   tg.make_shape(1, 8, 2, 96, 1 << 20),       # head dim 96
-                  tg.make_shape(1, 8, 2, 128, 1 << 20, page=32),
-                  tg.make_shape(2**28, 8, 2, 128, 1 << 20)):    # 2^31 query rows
+                  tg.make_shape(1, 8, 2, 128, 1 << 20, page=32)):
         with pytest.raises(tg.TGError) as e:
             tg.tg_plan_create(shape, kv, goh, goff, **ok)
         assert e.value.status == tg.TG_EUNSUPPORTED
+    # 2^31 query rows: refused before any length is read (through the C entry itself; the
+    # binding would first insist on B * Hkv lengths)
+    big = tg.make_shape(2**28, 8, 2, 128, 1 << 20)
+    opts = tg.tg_plan_opts(16, 1, 0, 1, -1, 0, 0, 0, 0, 0, 0, 0, 8, 1)
+    h = ctypes.c_void_p()
+    kvc, gohc, goffc = (np.ascontiguousarray(kv), np.ascontiguousarray(goh),
+                        np.ascontiguousarray(goff))
+    assert tg._lib().tg_plan_create(ctypes.byref(big), kvc.ctypes.data, None, gohc.ctypes.data,
+                                    goffc.ctypes.data, 1, 0, ctypes.byref(opts),
+                                    ctypes.byref(h)) == tg.TG_EUNSUPPORTED
+    assert not h.value
+    with pytest.raises(ValueError):                  # the binding's own size check
+        tg.tg_plan_create(big, kv, goh, goff, **ok)
     shape = tg.make_shape(1, 8, 2, 128, 1 << 26)
     for bad, status in ((tg.TG_MAX_HEAD_TOKENS + 1, tg.TG_EUNSUPPORTED),
                         (2**31 - 1, tg.TG_EUNSUPPORTED), (-1, tg.TG_EINVAL)):
@@ -483,3 +496,33 @@ def test_plan_rejects_unsupported_shapes_and_lengths():
     info = tg.tg_plan_get_info(p)
     assert info["n_items"] == 2
     assert info["kv_bytes"] == (100 + tg.TG_MAX_HEAD_TOKENS) * 2 * 128 * 2
+
+
+def test_binding_checks_host_array_sizes():
+    """Host arrays whose size the C side infers from the shape are checked before the call
+    (a short array would otherwise be read past its end)."""
+    shape = tg.make_shape(2, 8, 2, 128, 1024)
+    kv = np.array([[40, 17], [3, 90]], np.int32)
+    goh = np.zeros(2, np.int32)
+    goff = np.array([0, 64], np.int64)
+    ok = dict(host_only=True, num_workers=8)
+    tg.tg_plan_destroy(tg.tg_plan_create(shape, kv, goh, goff, **ok))
+    for bad in (dict(kv_len=kv[:1]), dict(group_of_head=goh[:1]), dict(group_off=goff[:1]),
+                dict(fast_len=np.zeros(3, np.int32))):
+        args = dict(kv_len=kv, group_of_head=goh, group_off=goff)
+        args.update(bad)
+        with pytest.raises(ValueError):
+            tg.tg_plan_create(shape, args["kv_len"], args["group_of_head"], args["group_off"],
+                              fast_len=args.get("fast_len"), **ok)
+    table = np.arange(16, dtype=np.int32)
+    with pytest.raises(ValueError):
+        tg.tg_plan_create_cascade(shape, kv, goh, goff, table, np.zeros(3, np.int64), **ok)
+    with pytest.raises(ValueError):
+        tg.tg_alloc_create(10, 16, np.arange(9))
+    cnt = np.array([[2, 1], [0, 3]], np.int32)
+    with pytest.raises(ValueError):
+        tg.tg_group_tables(cnt, np.zeros(3, np.int32), 1, np.arange(6))
+    with pytest.raises(ValueError):
+        tg.tg_group_tables(cnt, np.zeros(2, np.int32), 1, np.arange(5))   # 6 page ids needed
+    t, off, g = tg.tg_group_tables(cnt, np.zeros(2, np.int32), 1, np.arange(6))
+    assert g[-1] == 2 * 2 * 3

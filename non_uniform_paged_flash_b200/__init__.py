@@ -251,7 +251,18 @@ def tg_alloc_create(num_pages: int, page: int = 16, free_order=None):
     _count(fo, num_pages, "free_order")
     h = ctypes.c_void_p()
     _check(_lib().tg_alloc_create(num_pages, page, _hp(fo), ctypes.byref(h)), "tg_alloc_create")
+    h.page = page   # output buffers of the calls below are sized with the allocator's page
     return h
+
+
+def _alloc_page(a, page):
+    """The allocator's page size (a page argument that disagrees with it is refused)."""
+    own = getattr(a, "page", None)
+    if own is None:
+        return page
+    if page is not None and page != own:
+        raise ValueError(f"page {page} given, the allocator's page is {own}")
+    return own
 
 
 def tg_alloc_destroy(a):
@@ -266,8 +277,11 @@ def tg_alloc_refcount(a, page_id: int) -> int:
     return int(_lib().tg_alloc_refcount(a, page_id))
 
 
-def tg_alloc_share_segment(a, n_tokens: int, n_heads: int, page: int = 16):
+def tg_alloc_share_segment(a, n_tokens: int, n_heads: int, page: int = None):
     """Returns (seg_id, page_ids int32[n_heads, n_tokens // page])."""
+    page = _alloc_page(a, page)
+    if page is None:
+        raise ValueError("page size unknown: pass the allocator's page")
     full = n_tokens // page
     ids = np.empty((n_heads, full), dtype=np.int32)
     sid = ctypes.c_int32()
@@ -276,8 +290,9 @@ def tg_alloc_share_segment(a, n_tokens: int, n_heads: int, page: int = 16):
     return sid.value, ids
 
 
-def tg_alloc_reserve(a, seq_id: int, kv_len, prefix_segs=(), page: int = 16) -> np.ndarray:
+def tg_alloc_reserve(a, seq_id: int, kv_len, prefix_segs=(), page: int = None) -> np.ndarray:
     """Reserve all heads of one sequence; returns its page ids (flat, head after head)."""
+    page = _alloc_page(a, page) or 1   # page 1 sizes the buffer for any allocator
     kv = _h(kv_len, np.int32).reshape(-1)
     segs = _h(np.asarray(prefix_segs, dtype=np.int32).reshape(-1), np.int32)
     cap = int(kv.astype(np.int64).sum() // page + kv.size * (1 + max(1, segs.size)))

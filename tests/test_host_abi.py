@@ -526,3 +526,20 @@ def test_binding_checks_host_array_sizes():
         tg.tg_group_tables(cnt, np.zeros(2, np.int32), 1, np.arange(5))   # 6 page ids needed
     t, off, g = tg.tg_group_tables(cnt, np.zeros(2, np.int32), 1, np.arange(6))
     assert g[-1] == 2 * 2 * 3
+
+
+def test_allocator_outputs_sized_with_its_own_page():
+    """The binding sizes segment and reservation outputs with the allocator's page (a larger
+    page argument would under-size them); a page argument that disagrees is refused."""
+    a = tg.tg_alloc_create(64, 8)
+    try:
+        sid, ids = tg.tg_alloc_share_segment(a, 40, 2)               # 5 full 8-token pages per head
+        assert ids.shape == (2, 5) and len(np.unique(ids)) == 10
+        with pytest.raises(ValueError):
+            tg.tg_alloc_share_segment(a, 40, 2, 16)
+        r = tg.tg_alloc_reserve(a, 0, [41, 40], [sid])               # 40 shared + 1 private token
+        assert r.size == 5 + 1 + 5 and tg.tg_alloc_free_pages(a) == 64 - 10 - 1
+        with pytest.raises(ValueError):
+            tg.tg_alloc_reserve(a, 1, [8], (), 16)
+    finally:
+        tg.tg_alloc_destroy(a)

@@ -776,17 +776,47 @@ def tg_splitzip_workspace_bytes(n: int) -> int:
     return int(_lib().tg_splitzip_workspace_bytes(int(n)))
 
 
+def _bytes(t, n, what):
+    """A device buffer holds at least n bytes and is contiguous (the kernels index it by n)."""
+    if t is None:
+        raise ValueError(f"{what}: missing")
+    if t.numel() * t.element_size() < n:
+        raise ValueError(f"{what}: {t.numel() * t.element_size()} bytes, {n} needed")
+    if not t.is_contiguous():
+        raise ValueError(f"{what}: must be contiguous")
+
+
+def _zip_buffers(n, codebook, sm, codes, esc_pos, esc_exp, n_esc):
+    cap = 0 if esc_pos is None else esc_pos.numel()
+    _bytes(codebook, 16, "codebook")
+    _bytes(n_esc, 8, "n_esc")
+    if n > 0:
+        _bytes(sm, n, "sm")
+        _bytes(codes, (n + 1) // 2, "codes")
+    if cap > 0:
+        _bytes(esc_pos, 8 * cap, "esc_pos")
+        _bytes(esc_exp, cap, "esc_exp")
+    return cap
+
+
 def tg_splitzip_encode(n: int, src, codebook, sm, codes, esc_pos, esc_exp, n_esc, workspace,
                        stream=None):
     """Encode n bf16 values of src (device); esc_cap = esc_pos.numel()."""
-    cap = 0 if esc_pos is None else esc_pos.numel()
+    n = int(n)
+    cap = _zip_buffers(n, codebook, sm, codes, esc_pos, esc_exp, n_esc)
+    if n > 0:
+        _bytes(src, 2 * n, "src")
+    _bytes(workspace, max(0, tg_splitzip_workspace_bytes(n)), "workspace")
     _check(_lib().tg_splitzip_encode(int(n), _dp(src), _dp(codebook), _dp(sm), _dp(codes),
                                      _dp(esc_pos), _dp(esc_exp), cap, _dp(n_esc),
                                      _dp(workspace), _stream(stream)), "tg_splitzip_encode")
 
 
 def tg_splitzip_decode(n: int, codebook, sm, codes, esc_pos, esc_exp, n_esc, dst, stream=None):
-    cap = 0 if esc_pos is None else esc_pos.numel()
+    n = int(n)
+    cap = _zip_buffers(n, codebook, sm, codes, esc_pos, esc_exp, n_esc)
+    if n > 0:
+        _bytes(dst, 2 * n, "dst")
     _check(_lib().tg_splitzip_decode(int(n), _dp(codebook), _dp(sm), _dp(codes), _dp(esc_pos),
                                      _dp(esc_exp), _dp(n_esc), cap, _dp(dst), _stream(stream)),
            "tg_splitzip_decode")

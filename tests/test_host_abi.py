@@ -543,3 +543,28 @@ def test_allocator_outputs_sized_with_its_own_page():
             tg.tg_alloc_reserve(a, 1, [8], (), 16)
     finally:
         tg.tg_alloc_destroy(a)
+
+
+def test_splitzip_buffers_are_size_checked():
+    """Every SplitZip buffer is checked against n before a kernel could index past its end."""
+    import torch
+    n, cap = 100, 10
+    ok = dict(src=torch.zeros(n, dtype=torch.int16), codebook=torch.zeros(16, dtype=torch.uint8),
+              sm=torch.zeros(n, dtype=torch.uint8), codes=torch.zeros(50, dtype=torch.uint8),
+              esc_pos=torch.zeros(cap, dtype=torch.int64), esc_exp=torch.zeros(cap, dtype=torch.uint8),
+              n_esc=torch.zeros(1, dtype=torch.int64),
+              workspace=torch.zeros(tg.tg_splitzip_workspace_bytes(n), dtype=torch.uint8))
+    short = dict(src=ok["src"][:n - 1], codebook=ok["codebook"][:15], sm=ok["sm"][:n - 1],
+                 codes=ok["codes"][:49], esc_exp=ok["esc_exp"][:cap - 1], n_esc=torch.zeros(0, dtype=torch.int64),
+                 workspace=ok["workspace"][:-1])
+    for name, t in short.items():
+        args = dict(ok, **{name: t})
+        with pytest.raises(ValueError, match=name):
+            tg.tg_splitzip_encode(n, args["src"], args["codebook"], args["sm"], args["codes"],
+                                  args["esc_pos"], args["esc_exp"], args["n_esc"], args["workspace"])
+    with pytest.raises(ValueError, match="dst"):
+        tg.tg_splitzip_decode(n, ok["codebook"], ok["sm"], ok["codes"], ok["esc_pos"], ok["esc_exp"],
+                              ok["n_esc"], torch.zeros(n - 1, dtype=torch.int16))
+    with pytest.raises(ValueError, match="sm"):
+        tg.tg_splitzip_decode(n, ok["codebook"], short["sm"], ok["codes"], ok["esc_pos"], ok["esc_exp"],
+                              ok["n_esc"], torch.zeros(n, dtype=torch.int16))

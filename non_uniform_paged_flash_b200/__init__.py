@@ -738,6 +738,11 @@ def tg_tiered_decode_streamed(ss: SlowStream, q, k_q8_host, v_q8_host, k_scale_h
                               v_scale_host, k_fast, v_fast, fast_page_table, fast_head_off,
                               group_of_head, scale: float, out, lse, stream=None):
     """Tiered decode with the INT8 tier in pinned host memory, streamed block-wise."""
+    rows = ss.shape.B * ss.shape.Hq
+    if rows > 0:
+        _bytes(q, 2 * rows * ss.shape.D, "q")
+        _bytes(out, 2 * rows * ss.shape.D, "out")
+        _bytes(lse, 4 * rows, "lse")
     for t in (k_q8_host, v_q8_host, k_scale_host, v_scale_host):
         ss._held[id(t)] = t
     _check(_lib().tg_tiered_decode_streamed(
@@ -750,6 +755,9 @@ def tg_tiered_decode_streamed(ss: SlowStream, q, k_q8_host, v_q8_host, k_scale_h
 def tg_lse_merge(row_split_off, part_o, part_lse, out, lse, stream=None):
     n_rows = row_split_off.numel() - 1
     D = part_o.shape[-1]
+    if n_rows > 0:
+        _bytes(out, 2 * n_rows * D, "out")
+        _bytes(lse, 4 * n_rows, "lse")
     _check(_lib().tg_lse_merge(n_rows, D, _dp(row_split_off), _dp(part_o), _dp(part_lse),
                                _dp(out), _dp(lse), _stream(stream)), "tg_lse_merge")
 
@@ -757,6 +765,9 @@ def tg_lse_merge(row_split_off, part_o, part_lse, out, lse, stream=None):
 def tg_quantize_int8(src, codes, scale, stream=None):
     D = src.shape[-1]
     n_rows = src.numel() // D
+    if n_rows > 0:
+        _bytes(codes, n_rows * D, "codes")
+        _bytes(scale, 4 * n_rows, "scale")
     _check(_lib().tg_quantize_int8(n_rows, D, _dp(src), _dp(codes), _dp(scale), _stream(stream)),
            "tg_quantize_int8")
 
@@ -764,6 +775,9 @@ def tg_quantize_int8(src, codes, scale, stream=None):
 def tg_quantize_int4(src, packed, scale, stream=None):
     D = src.shape[-1]
     n_rows = src.numel() // D
+    if n_rows > 0:
+        _bytes(packed, n_rows * D // 2, "packed")
+        _bytes(scale, 4 * n_rows, "scale")
     _check(_lib().tg_quantize_int4(n_rows, D, _dp(src), _dp(packed), _dp(scale), _stream(stream)),
            "tg_quantize_int4")
 

@@ -568,3 +568,20 @@ def test_splitzip_buffers_are_size_checked():
     with pytest.raises(ValueError, match="sm"):
         tg.tg_splitzip_decode(n, ok["codebook"], short["sm"], ok["codes"], ok["esc_pos"], ok["esc_exp"],
                               ok["n_esc"], torch.zeros(n, dtype=torch.int16))
+
+
+def test_quantizer_and_merge_outputs_are_size_checked():
+    import torch
+    src = torch.zeros((10, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="codes"):
+        tg.tg_quantize_int8(src, torch.zeros(10 * 128 - 1, dtype=torch.int8), torch.zeros(10))
+    with pytest.raises(ValueError, match="scale"):
+        tg.tg_quantize_int8(src, torch.zeros(10 * 128, dtype=torch.int8), torch.zeros(9))
+    with pytest.raises(ValueError, match="packed"):
+        tg.tg_quantize_int4(src, torch.zeros(10 * 64 - 1, dtype=torch.uint8), torch.zeros(10))
+    off = torch.tensor([0, 2, 3], dtype=torch.int64)
+    po, pl = torch.zeros((3, 128)), torch.zeros(3)
+    with pytest.raises(ValueError, match="out"):
+        tg.tg_lse_merge(off, po, pl, torch.zeros((1, 128), dtype=torch.bfloat16), torch.zeros(2))
+    with pytest.raises(ValueError, match="lse"):
+        tg.tg_lse_merge(off, po, pl, torch.zeros((2, 128), dtype=torch.bfloat16), torch.zeros(1))

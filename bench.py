@@ -6,8 +6,16 @@ the log-sum-exp merge, through the C ABI (tg_ragged_paged_decode / tg_tiered_dec
 batch's KV cache, page tables and plan are resident in HBM before timing (admission happens
 once, as in serving); the step's inputs are the queries.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
-    python bench.py --path sink|h2o|ttkv|ttkv-host|splitzip|layers ...   (one GPU, other lines)
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--layers L]
+                    [--impl ours|reference]
+    python bench.py --path sink|h2o|ttkv|ttkv-host|splitzip ...   (one GPU, other lines)
+
+The default workload is the multi-turn serving step (config 3): its 32 layers are made resident
+one at a time (all 32 layers' pools exceed one GPU) and each layer's step is timed; the line
+reports all layers' K/V bytes over the summed step time, per-layer figures and the worst layer.
+Per layer: W warm-up steps, K timed steps with nothing instrumented, then a separate pass with
+the library's kernel events on (per-kernel times for the roofline), then K end-to-end steps
+through the host-buffer call.
 
 N > 1 runs under torch.distributed.run, one rank per GPU. The batch is sharded by sequence with
 the library's ahead-of-time placement (per-GPU work fixed: weak scaling); the decode has no
@@ -146,10 +154,11 @@ def _traffic(cfg):
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples of SM clock and throttle reasons while the timed regions run."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "utilization.gpu")
 
     def __init__(self, gpu_index):
         self.gpu = str(gpu_index)
@@ -171,7 +180,19 @@ class ClockSampler:
         self.reader = threading.Thread(target=lambda: self.lines.extend(self.proc.stdout), daemon=True)
         self.reader.start()
 
-    def stop(self):
+    @staticmethod
+    def _when(stamp):
+        """nvidia-smi's local timestamp ("YYYY/MM/DD HH:MM:SS.mmm") as seconds since the epoch."""
+        import datetime
+        try:
+            return datetime.datetime.strptime(stamp.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
+
+    def stop(self, windows=()):
+        """Summary of the samples. With windows [(t0, t1), ...] (time.time() around the timed
+        regions), the SM clock median is taken over the samples inside them, else over the
+        samples that saw the GPU busy, else over all; throttle reasons over the same set."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -181,24 +202,29 @@ class ClockSampler:
             self.proc.kill()
         if self.reader is not None:
             self.reader.join(timeout=5)
-        sm, mx, reasons = [], None, set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in list(self.lines):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 11:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                rows.append({"t": self._when(parts[0]), "sm": float(parts[2]), "max": float(parts[3]),
+                             "reasons": {n for n, v in zip(names, parts[6:10]) if v.lower() == "active"},
+                             "util": float(parts[10]) if parts[10].replace(".", "", 1).isdigit() else 0.0})
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        if not rows:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        inside = [r for r in rows if r["t"] is not None and
+                  any(t0 - 0.05 <= r["t"] <= t1 + 0.05 for t0, t1 in windows)]
+        busy = [r for r in rows if r["util"] >= 50.0]
+        used, basis = (inside, "samples inside the timed regions") if inside else (
+            (busy, "samples with the GPU busy") if busy else (rows, "all samples"))
+        reasons = set().union(*(r["reasons"] for r in used))
+        return {"sm_mhz": statistics.median(r["sm"] for r in used), "sm_max_mhz": rows[-1]["max"],
+                "reasons": sorted(reasons), "samples": len(used), "samples_total": len(rows),
+                "basis": basis}
 
 
 # ------------------------------------------------------------------------------------------
@@ -252,12 +278,13 @@ def run_reference(args):
     cores = oracle.num_threads()
     sample = ("per step: all query rows of one sequence" if o.fast_len is None else
               "per step: the query rows of one (sequence, KV head)") + \
-        f"; fp64 oracle over {cores} threads"
+        (" of layer 0" if sp.layers > 1 else "") + f"; fp64 oracle over {cores} threads"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": _workload_name(cfg, sp), "config_id": cfg},
+            "config": _config(cfg, _global_spec(cfg, _env_int("WORLD_SIZE", 1)),
+                              _env_int("WORLD_SIZE", 1), min(args.layers, sp.layers)),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -320,13 +347,13 @@ def cpu_baseline(cfg, budget_s=20.0, min_s=10.0, sample=None):
                       f"{cores} host threads"}
 
 
-def _parity_sample(first, db, D):
-    """Max-abs differences of the timed step's outputs from the fp64 oracle on the rows the
-    CPU baseline computed (its first chunk of sequences, every query row of them)."""
+def _parity_sample(first, out, lse):
+    """Max-abs differences of the timed step's outputs (layer 0; host copies out [rows, D],
+    lse [rows]) from the fp64 oracle on the rows the CPU baseline computed (its first chunk of
+    sequences, every query row of them)."""
     try:
         sel, (o_ref, l_ref) = first[0]
-        out = db.out.float().reshape(-1, D).cpu().numpy()[sel]
-        lse = db.lse.reshape(-1).cpu().numpy()[sel]
+        out, lse = out[sel], lse[sel]
         fin = np.isfinite(l_ref)
         assert np.array_equal(fin, np.isfinite(lse)), "empty heads differ"
         return {"rows": int(len(sel)), "max_abs_out": float(np.abs(out - o_ref).max()),
@@ -336,9 +363,183 @@ def _parity_sample(first, db, D):
         return {"error": (type(e).__name__ + ": " + str(e))[:200]}
 
 
-def run_ours(args):
+def _config(cfg, sp, world, n_layers):
+    """The line's config dict (the same for both arms); sp is the global spec."""
+    name = _workload_name(cfg, sp)
+    c = {"workload": name, "config_id": cfg, "global_batch": int(sp.B),
+         "parallelism": "sequence shards by AOT byte placement, no collective" if world > 1
+         else "single GPU",
+         "l2": "L2 flushed (252 MB written) between steps, outside the timed step" if cfg == 1
+         else "inputs larger than L2 (K/V per step > 0.5 GB vs 126 MB L2); no flush"}
+    if sp.layers > 1:
+        c["workload"] = name + "; layers %d of %d, one resident at a time" % (n_layers, sp.layers)
+        c["layers"] = n_layers
+    return c
+
+
+def _unique_kv_bytes(sp, lay):
+    """K/V bytes of the distinct pages one step reads: a page referenced from r rows (a shared
+    prefix page; always full) counts once instead of r times."""
+    t = lay.table[lay.table >= 0]
+    _, cnt = np.unique(t, return_counts=True)
+    dup_tokens = int((cnt[cnt > 1].astype(np.int64) - 1).sum()) * sp.page
+    return (int(lay.kv_len.astype(np.int64).sum()) - dup_tokens) * 2 * sp.D * 2
+
+
+def _l2_profile(cfg):
+    """L2 hit rate of the cascade kernel from a committed ncu capture, while the kernel source
+    is unchanged since the capture; else None."""
+    src = os.path.join(ROOT, "non_uniform_paged_flash_b200", "csrc", "tg_kernels.cu")
+    path = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+    try:
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        with open(path) as f:
+            e = json.load(f).get(f"config{cfg}")
+        if e and e.get("kernel_sha") == sha and "l2_hit_rate" in e:
+            return float(e["l2_hit_rate"])
+    except Exception:
+        pass
+    return None
+
+
+def _measure_layer(args, cfg, sp, layer, rank, world, dist, local, stream, pools, keep):
+    """One layer of the workload made resident and measured: warm-up, then the timed steps
+    (nothing instrumented), then a separate pass with the library's kernel events on (the
+    per-kernel times of the roofline), then the end-to-end steps through the host-buffer call.
+    Returns the layer's figures (host numbers only; device memory is released)."""
     import torch
     import non_uniform_paged_flash_b200 as tg
+    from non_uniform_paged_flash_b200 import workload
+
+    kv_all, fast_all = workload.retained(sp, layer)
+    seqs = _my_sequences(sp, rank, world, kv_all, fast_all)
+    lay = workload.layout(sp, layer, seqs)
+    db = workload.to_device(sp, lay, layer, device=f"cuda:{local}", seqs=seqs, pools=pools,
+                            **_plan_kw(cfg))
+    info = tg.tg_plan_get_info(db.plan)
+    alg = workload.algorithmic_bytes(sp, lay)
+
+    # L2: inputs larger than L2 need no flush; smaller ones get a flush between steps.
+    flush = None
+    if alg["kv"] < 2 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=f"cuda:{local}")
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def timed_steps(n, one):
+        """Device time (ms) of n steps `one()` on the stream; with a flush, each step has its
+        own event pair and the flush runs outside it."""
+        if flush is None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                one()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for e0, e1 in evs:
+            flush.zero_()
+            e0.record(stream)
+            one()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return sum(e0.elapsed_time(e1) for e0, e1 in evs)
+
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
+        db.run(stream)
+    torch.cuda.synchronize()
+    assert tg.tg_plan_status(db.plan) == tg.TG_OK, "device error word set during warm-up"
+
+    # 1. the timed steps: the product path, nothing recorded inside it
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    ms_total = timed_steps(args.steps, lambda: db.run(stream))
+    window = (t0, time.time())
+    barrier()
+
+    # 2. per-kernel times: the library's own events around the decode and merge launches, in a
+    # separate pass (a recorded call gives up the merge kernel's launch overlap)
+    n_ev = min(args.steps, 256)
+    tg.tg_plan_timing_enable(db.plan, n_ev)
+    for _ in range(n_ev):
+        if flush is not None:
+            flush.zero_()
+        db.run(stream)
+    n_rec, dec_ms, mrg_ms = tg.tg_plan_timing_read(db.plan)
+    tg.tg_plan_timing_enable(db.plan, 0)
+    status = tg.tg_plan_status(db.plan)
+
+    # 3. end to end through the C-ABI host-buffer call: every step copies its pinned host q in
+    # and its out + lse back to pinned host memory. The library's pipe double-buffers the device
+    # staging, so a step's copies overlap its neighbours' decodes; the timed region runs from
+    # before the first input copy to after the last output copy.
+    q_host = db.q.cpu().pin_memory()
+    out_host = torch.empty(db.out.shape, dtype=db.out.dtype).pin_memory()
+    lse_host = torch.empty(db.lse.shape, dtype=db.lse.dtype).pin_memory()
+    pipe = tg.HostPipe(db.plan)
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
+        db.run_host(pipe, q_host, out_host, lse_host, stream)
+    pipe.wait()
+    barrier()
+    torch.cuda.synchronize()
+
+    def e2e_one():
+        pipe.after(stream)
+        db.run_host(pipe, q_host, out_host, lse_host, stream)
+        pipe.join(stream)
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        pipe.after(stream)
+        for _ in range(args.steps):
+            db.run_host(pipe, q_host, out_host, lse_host, stream)
+        pipe.join(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+    else:
+        e2e_ms = timed_steps(args.steps, e2e_one)   # no overlap: the flush sits between steps
+    pipe.wait()
+    assert torch.equal(out_host, db.out.cpu()), "host-buffer call differs from the device call"
+    pipe.destroy()
+    barrier()
+
+    r = {"layer": layer, "ms_per_step": ms_total / args.steps, "e2e_ms_per_step": e2e_ms / args.steps,
+         "decode_avg_ms": dec_ms / max(n_rec, 1), "merge_avg_ms": mrg_ms / max(n_rec, 1),
+         "launches_timed": n_rec, "ok": status == tg.TG_OK, "kv_bytes": int(alg["kv"]),
+         "algorithmic_bytes": int(alg["total"]), "batch": int(lay.kv_len.shape[0]),
+         "launches_per_step": 1 + (1 if info["n_merge"] > 0 else 0) + (1 if info["n_cascade"] > 0 else 0),
+         "plan": {k: info[k] for k in ("n_items", "n_partials", "n_merge", "n_workers", "grid",
+                                       "stages", "smem_bytes", "n_cascade")},
+         "h2d_bytes": int(db.q.numel() * db.q.element_size()),
+         "d2h_bytes": int(db.out.numel() * db.out.element_size() + db.lse.numel() * db.lse.element_size()),
+         "window": window}
+    if info["n_cascade"] > 0:
+        r["unique_kv_bytes"] = _unique_kv_bytes(sp, lay)
+    if keep:
+        r["out"] = db.out.float().reshape(-1, sp.D).cpu().numpy()
+        r["lse"] = db.lse.reshape(-1).cpu().numpy()
+    if keep and cfg == 1:
+        r["db"] = db        # the tiny workload also replays a CUDA graph of many copies
+    else:
+        db.plan.destroy()
+        del db
+        torch.cuda.empty_cache()
+    return r
+
+
+def run_ours(args):
+    import torch
     from non_uniform_paged_flash_b200 import workload
 
     rank, world = _env_int("RANK", 0), _env_int("WORLD_SIZE", 1)
@@ -353,174 +554,117 @@ def run_ours(args):
 
     cfg = args.config
     sp = _global_spec(cfg, world)
-    kv_all, fast_all = workload.retained(sp, 0)
-    seqs = _my_sequences(sp, rank, world, kv_all, fast_all)
-    lay = workload.layout(sp, 0, seqs)
-    db = workload.to_device(sp, lay, 0, device=f"cuda:{local}", seqs=seqs, **_plan_kw(cfg))
-    info = tg.tg_plan_get_info(db.plan)
-    alg = workload.algorithmic_bytes(sp, lay)
-    B_local = lay.kv_len.shape[0]
+    n_layers = min(args.layers, sp.layers)
     stream = torch.cuda.current_stream()
 
-    # L2: inputs larger than L2 need no flush; smaller ones get a flush between steps.
-    flush = None
-    if alg["kv"] < 2 * L2_BYTES:
-        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=f"cuda:{local}")
+    # A multi-layer workload keeps one pair of bf16 pools for all its layers (the pool bytes do
+    # not depend on the layer; each layer's own tables decide what its heads read): sized for the
+    # largest layer, uploaded once, outside any timed region.
+    pools = None
+    if n_layers > 1:
+        most = 0
+        for layer in range(n_layers):
+            kv_all, fast_all = workload.retained(sp, layer)
+            seqs = _my_sequences(sp, rank, world, kv_all, fast_all)
+            most = max(most, workload.layout(sp, layer, seqs).num_pages)
+        pools = workload.pools_to_device(sp, most, device=f"cuda:{local}")
 
-    def step():
-        if flush is not None:
-            flush.zero_()
-        db.run(stream)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    assert tg.tg_plan_status(db.plan) == tg.TG_OK, "device error word set during warm-up"
-
-    n_timed = min(args.steps, 256)   # kernel events on the first calls of the timed region
-    tg.tg_plan_timing_enable(db.plan, n_timed)
     sampler = ClockSampler(local) if rank == 0 else None
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
-    if flush is None:
-        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        ms_total = ev0.elapsed_time(ev1)
-    else:
-        # the L2 flush runs between steps, outside each step's event pair
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        for e0_, e1_ in evs:
-            flush.zero_()
-            e0_.record(stream)
-            db.run(stream)
-            e1_.record(stream)
-        torch.cuda.synchronize()
-        ms_total = sum(e0_.elapsed_time(e1_) for e0_, e1_ in evs)
-    barrier()
-    clocks = sampler.stop() if sampler else None
-    n_rec, dec_ms, mrg_ms = tg.tg_plan_timing_read(db.plan)
-    tg.tg_plan_timing_enable(db.plan, 0)
-    status = tg.tg_plan_status(db.plan)
+    layers = [_measure_layer(args, cfg, sp, layer, rank, world, dist, local, stream, pools,
+                             keep=(layer == 0 and rank == 0))
+              for layer in range(n_layers)]
+    clocks = sampler.stop([r["window"] for r in layers]) if sampler else None
+    del pools
 
-    # End to end through the C-ABI host-buffer call: every step copies its pinned host q in and
-    # its out + lse back to pinned host memory. The library's pipe double-buffers the device
-    # staging, so a step's copies overlap its neighbours' decodes; the timed region runs from
-    # before the first input copy to after the last output copy.
-    q_host = db.q.cpu().pin_memory()
-    out_host = torch.empty(db.out.shape, dtype=db.out.dtype).pin_memory()
-    lse_host = torch.empty(db.lse.shape, dtype=db.lse.dtype).pin_memory()
-    pipe = tg.HostPipe(db.plan)
-    k_e2e = min(args.steps, 2000)
-
-    def e2e_step():
-        db.run_host(pipe, q_host, out_host, lse_host, stream)
-
-    for _ in range(args.warmup):
-        if flush is not None:
-            flush.zero_()
-        e2e_step()
-    pipe.wait()
-    barrier()
-    torch.cuda.synchronize()
-    if flush is None:
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        pipe.after(stream)
-        for _ in range(k_e2e):
-            e2e_step()
-        pipe.join(stream)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-    else:
-        # the L2 flush runs between steps, outside each step's event pair (no overlap then)
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(k_e2e)]
-        for a_, b_ in evs:
-            flush.zero_()
-            a_.record(stream)
-            pipe.after(stream)
-            e2e_step()
-            pipe.join(stream)
-            b_.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = sum(a_.elapsed_time(b_) for a_, b_ in evs)
-    pipe.wait()
-    assert torch.equal(out_host, db.out.cpu()), "host-buffer call differs from the device call"
-    pipe.destroy()
-    barrier()
-
-    # Max over ranks (time, error flag) and sums (work).
-    vals = torch.tensor([ms_total, e2e_ms, dec_ms / max(n_rec, 1), float(status != tg.TG_OK),
-                         float(alg["kv"]), float(B_local)], dtype=torch.float64,
-                        device=f"cuda:{local}")
-    ms_total, e2e_ms, dec_avg, bad, kv_total, b_total = _over_ranks(dist, vals, 4)
-
-    ms_step = ms_total / args.steps
-    value = kv_total / (ms_step * 1e-3) / 1e9
-    e2e_value = kv_total / (e2e_ms / k_e2e * 1e-3) / 1e9
+    # Max over ranks (times, error flag) and sums (work), per layer.
+    vals = []
+    for r in layers:
+        vals += [r["ms_per_step"], r["e2e_ms_per_step"], r["decode_avg_ms"], r["merge_avg_ms"],
+                 float(not r["ok"])]
+    n_max = len(vals)
+    for r in layers:
+        vals += [float(r["kv_bytes"]), float(r["algorithmic_bytes"]), float(r["batch"])]
+    vals = torch.tensor(vals, dtype=torch.float64, device=f"cuda:{local}")
+    red = _over_ranks(dist, vals, n_max)
+    mx, sm = red[:n_max], red[n_max:]
+    per_layer = []
+    for i, r in enumerate(layers):
+        ms, e2e, dec, mrg, bad = mx[5 * i:5 * i + 5]
+        kv, algb, b = sm[3 * i:3 * i + 3]
+        per_layer.append({"layer": r["layer"], "ms_per_step": ms, "e2e_ms_per_step": e2e,
+                          "decode_avg_ms": dec, "merge_avg_ms": mrg, "bad": bad > 0,
+                          "kv_bytes": kv, "algorithmic_bytes": algb, "batch": b,
+                          "frac_of_peak": None})
 
     if rank == 0:
         peak, peak_kind = _measured_peak()
-        achieved = alg["total"] / (dec_avg * 1e-3) / 1e9
+        ms_sum = sum(r["ms_per_step"] for r in per_layer)
+        e2e_sum = sum(r["e2e_ms_per_step"] for r in per_layer)
+        kv_sum = sum(r["kv_bytes"] for r in per_layer)
+        alg_sum = sum(r["algorithmic_bytes"] for r in per_layer)
+        dec_sum = sum(r["decode_avg_ms"] for r in per_layer)
+        for r in per_layer:
+            r["frac_of_peak"] = r["algorithmic_bytes"] / (r["decode_avg_ms"] * 1e-3) / 1e9 / peak
+        worst = min(per_layer, key=lambda r: r["frac_of_peak"])
+        ms_step = ms_sum / n_layers
+        achieved = alg_sum / (dec_sum * 1e-3) / 1e9
+        b_total = per_layer[0]["batch"]
+        first = layers[0]
+        cascade = first["plan"]["n_cascade"] > 0
+        launches = sum(args.steps * r["launches_per_step"] for r in layers)
         line = {
-            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "metric": METRIC, "value": kv_sum / (ms_sum * 1e-3) / 1e9, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if lay.fast_len is None else "bf16+int%d" % sp.slow_bits,
+            "dtype": "bf16" if sp.kind != "tiered" else "bf16+int%d" % sp.slow_bits,
             "data": "synthetic",
-            "config": {"workload": _workload_name(cfg, sp), "config_id": cfg,
-                       "global_batch": int(b_total), "parallelism":
-                       "sequence shards by AOT byte placement, no collective" if world > 1
-                       else "single GPU",
-                       "l2": ("inputs larger than L2 (%.2f GB K/V per step vs 126 MB)" %
-                              (alg["kv"] / 1e9)) if flush is None else
-                       "L2 flushed (252 MB written) between steps, outside the timed step"},
+            "config": _config(cfg, sp, world, n_layers),
             "tokens_per_s_per_layer": b_total / (ms_step * 1e-3),
-            "kv_bytes_per_step": int(kv_total),
+            "kv_bytes_per_step": int(kv_sum / n_layers),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": _traffic(cfg) if world == 1 else None,
+                         "frac": achieved / peak,
+                         "traffic": _traffic(cfg) if world == 1 and n_layers == 1 else None,
                          "peak_kind": peak_kind,
                          "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
                          "nominal_gbs": NOMINAL_HBM_GBS,
-                         "kernel": "cascade_kernel + decode_kernel" if info["n_cascade"] > 0
-                         else "decode_kernel",
-                         "algorithmic_bytes_per_launch": alg["total"],
-                         "avg_launch_ms": dec_avg, "merge_avg_ms": mrg_ms / max(n_rec, 1),
-                         "launches_timed": n_rec},
-            "e2e": {"value": e2e_value, "unit": "GB/s",
-                    "h2d_bytes_per_step": int(db.q.numel() * db.q.element_size()),
-                    "d2h_bytes_per_step": int(db.out.numel() * db.out.element_size() +
-                                              db.lse.numel() * db.lse.element_size()),
-                    "steps": k_e2e, "call": "tg_ragged_paged_decode_host" if lay.fast_len is None
+                         "kernel": "cascade_kernel + decode_kernel" if cascade else "decode_kernel",
+                         "algorithmic_bytes_per_launch": alg_sum / n_layers,
+                         "avg_launch_ms": dec_sum / n_layers,
+                         "merge_avg_ms": sum(r["merge_avg_ms"] for r in per_layer) / n_layers,
+                         "launches_timed": first["launches_timed"],
+                         "timing": "decode-kernel events in a separate pass after the timed steps"},
+            "e2e": {"value": kv_sum / (e2e_sum * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": first["h2d_bytes"] * world,
+                    "d2h_bytes_per_step": first["d2h_bytes"] * world,
+                    "steps": args.steps,
+                    "call": "tg_ragged_paged_decode_host" if sp.kind != "tiered"
                     else "tg_tiered_decode_host",
                     "overlap": "double-buffered staging; copies of neighbouring steps overlap"
-                    if flush is None else "none (L2 flush between steps)"},
-            "gpu_launches": args.steps * (1 + (1 if info["n_merge"] > 0 else 0) +
-                                          (1 if info["n_cascade"] > 0 else 0)),
-            "plan": {k: info[k] for k in ("n_items", "n_partials", "n_merge", "n_workers",
-                                          "grid", "stages", "smem_bytes", "n_cascade")},
-            "device_status": "ok" if not bad else "error word set",
+                    if cfg != 1 else "none (L2 flush between steps)"},
+            "gpu_launches": launches,
+            "plan": first["plan"],
+            "device_status": "ok" if not any(r["bad"] for r in per_layer) else "error word set",
             "clocks": clocks,
         }
+        if n_layers > 1:
+            line["roofline"]["worst_layer"] = {"layer": worst["layer"], "frac": worst["frac_of_peak"]}
+            line["per_layer"] = [{k: (round(v, 6) if isinstance(v, float) else v)
+                                  for k, v in r.items() if k != "bad"} for r in per_layer]
+        if cascade:
+            uniq = first["unique_kv_bytes"] * world
+            line["roofline"]["unique_kv_bytes_per_step"] = uniq
+            line["roofline"]["frac_unique"] = uniq / (ms_step * 1e-3) / 1e9 / peak
+            line["roofline"]["frac_logical"] = kv_sum / (ms_sum * 1e-3) / 1e9 / peak
+            line["roofline"]["l2_hit_rate"] = _l2_profile(cfg)
         if world == 1 and cfg == 1:
-            line["graph_replay"] = graph_replay(db, alg)
+            line["graph_replay"] = graph_replay(first["db"], workload.algorithmic_bytes(sp, first["db"].lay))
         if world == 1 and not args.no_cpu_baseline:
-            first = []
-            line["cpu_baseline"] = cpu_baseline(cfg, sample=first)
-            line["parity_sample"] = _parity_sample(first, db, sp.D)
+            sample = []
+            line["cpu_baseline"] = cpu_baseline(cfg, sample=sample)
+            line["parity_sample"] = _parity_sample(sample, first["out"], first["lse"])
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
@@ -882,79 +1026,6 @@ def run_tier_host(args):
     return 0
 
 
-def run_layers(args):
-    """The multi-turn serving step (config 3) over its layers, one GPU. The 32 layers' pools
-    (about 189 GB at the workload's occupancy) do not fit one GPU, so each layer's tables, plan
-    and pools are made resident in turn (outside any timed region) and its decode step timed
-    with CUDA events over args.steps steps (each layer's 5.5 GB of K/V is far above L2). Prints
-    one JSON line: each layer's step time and K/V bytes, the mean step, and value = all the
-    layers' K/V bytes / the sum of their step times."""
-    import torch
-    import non_uniform_paged_flash_b200 as tg
-    from non_uniform_paged_flash_b200 import workload
-
-    if _env_int("WORLD_SIZE", 1) != 1:
-        raise SystemExit("--path layers runs on one GPU")
-    cfg = 3
-    sp = _preset(cfg)
-    n_layers = min(args.layers, sp.layers)
-    stream = torch.cuda.current_stream()
-    sampler = ClockSampler(0)
-    per_layer, bad = [], False
-    for layer in range(n_layers):
-        lay = workload.layout(sp, layer)
-        db = workload.to_device(sp, lay, layer, **_plan_kw(cfg))
-        alg = workload.algorithmic_bytes(sp, lay)
-        for _ in range(args.warmup):
-            db.run(stream)
-        torch.cuda.synchronize()
-        n_timed = min(args.steps, 256)
-        tg.tg_plan_timing_enable(db.plan, n_timed)
-        if layer == 0:
-            sampler.start()
-            time.sleep(0.3)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            db.run(stream)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        n_rec, dec_ms, _ = tg.tg_plan_timing_read(db.plan)
-        bad = bad or tg.tg_plan_status(db.plan) != tg.TG_OK
-        info = tg.tg_plan_get_info(db.plan)
-        per_layer.append({"layer": layer, "ms_per_step": e0.elapsed_time(e1) / args.steps,
-                          "kv_bytes": int(alg["kv"]), "algorithmic_bytes": int(alg["total"]),
-                          "decode_avg_ms": dec_ms / max(n_rec, 1), "batch": int(lay.kv_len.shape[0]),
-                          "launches": args.steps * (1 + (1 if info["n_merge"] > 0 else 0))})
-        db.plan.destroy()
-        del db
-        torch.cuda.empty_cache()
-    clocks = sampler.stop()
-    ms_sum = sum(r["ms_per_step"] for r in per_layer)
-    kv_sum = sum(r["kv_bytes"] for r in per_layer)
-    peak, peak_kind = _measured_peak()
-    achieved = sum(r["algorithmic_bytes"] for r in per_layer) / (
-        sum(r["decode_avg_ms"] for r in per_layer) * 1e-3) / 1e9
-    line = {
-        "metric": METRIC, "value": kv_sum / (ms_sum * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_sum / n_layers,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": WORKLOAD_NAMES[cfg] + "; layers %d of %d, one resident at a time"
-                   % (n_layers, sp.layers), "config_id": cfg, "layers": n_layers,
-                   "l2": "inputs larger than L2 (K/V per layer-step above 5 GB vs 126 MB)"},
-        "tokens_per_s_per_layer": per_layer[0]["batch"] / (ms_sum / n_layers * 1e-3),
-        "per_layer": per_layer,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
-                     "kernel": "decode_kernel (mean over the layers)"},
-        "gpu_launches": sum(r["launches"] for r in per_layer),
-        "device_status": "ok" if not bad else "error word set", "clocks": clocks,
-    }
-    print(json.dumps(line), flush=True)
-    return 0
-
-
 def run_splitzip(args):
     """SplitZip codec throughput on one GPU: the K and V pools of the GQA decode workload
     (config 2 shape, bf16) encoded and decoded back, each timed with CUDA events over
@@ -967,7 +1038,7 @@ def run_splitzip(args):
     sp = synth.preset(cfg)
     lay = workload.layout(sp, 0)
     dev = torch.device("cuda:0")
-    src = torch.cat([workload._pool_to_device(sp, w, lay.num_pages, 0, dev).view(torch.int16).reshape(-1)
+    src = torch.cat([workload._pool_to_device(sp, w, lay.num_pages, dev).view(torch.int16).reshape(-1)
                      for w in ("k", "v")])
     n = src.numel()
     cb = torch.empty(16, dtype=torch.uint8, device=dev)
@@ -1027,9 +1098,9 @@ def run_splitzip(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", type=int, default=3, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--slow-bits", type=int, default=8, choices=[8, 4],
@@ -1037,14 +1108,14 @@ def main():
     ap.add_argument("--block-pages", type=int, default=8192,
                     help="--path ttkv-host: INT8-tier pages per streamed block")
     ap.add_argument("--layers", type=int, default=32,
-                    help="--path layers: how many of config 3's layers to time, one at a time")
+                    help="multi-layer workload (config 3): how many of its layers to measure, "
+                         "each made resident in turn (default: all 32)")
     ap.add_argument("--path", default="decode",
-                    choices=["decode", "sink", "h2o", "ttkv", "ttkv-host", "splitzip", "layers"],
+                    choices=["decode", "sink", "h2o", "ttkv", "ttkv-host", "splitzip"],
                     help="decode: the decode step (default); sink / h2o: the decode step with "
                          "the write path; ttkv: the tiered step with tier migration (config 5); "
                          "ttkv-host: the tiered step with the INT8 tier streamed from host "
-                         "memory (config 5); splitzip: the KV codec; layers: config 3's step on "
-                         "each of its layers in turn; one GPU, separate JSON line")
+                         "memory (config 5); splitzip: the KV codec; one GPU, separate JSON line")
     args = ap.parse_args()
     global SLOW_BITS
     SLOW_BITS = args.slow_bits
@@ -1056,10 +1127,8 @@ def main():
         return run_splitzip(args)
     if args.path == "ttkv-host":
         return run_tier_host(args)
-    if args.path == "layers":
-        if args.layers < 1:
-            ap.error("--layers must be >= 1")
-        return run_layers(args)
+    if args.layers < 1:
+        ap.error("--layers must be >= 1")
     if args.path != "decode":
         return run_write_path(args)
     return run_ours(args)

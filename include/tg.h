@@ -160,8 +160,9 @@ typedef struct tg_plan_opts {
     int32_t num_workers;      /* 0: (SM count) x (workers per CTA) of the device */
     int32_t min_splits;       /* cut every head into at least this many chunks (>= 1) */
     int32_t max_chunk_pages;  /* 0: no cap; else chunks hold at most this many pages */
-    int32_t host_only;        /* 1: build the work list on the host only (inspection; decode
-                                 calls reject such a plan); 0: also create device state */
+    int32_t host_only;        /* 1: build the work list on the host only (inspection, or
+                                 tg_ragged_paged_decode_noalloc; the other decode calls reject
+                                 such a plan); 0: also create device state */
     int32_t device;           /* CUDA device ordinal, -1 = current */
     int32_t static_permille;  /* share of the bytes assigned to workers ahead of time, in
                                  1/1000 (0 = default 800; 1000 = all static); the rest is
@@ -331,22 +332,6 @@ int tg_ragged_paged_decode(tg_plan *plan, const void *q, const void *k_pages,
                            const int32_t *group_of_head, float scale, void *out, float *lse,
                            tg_stream stream);
 
-/* Ragged paged decode that allocates no device memory. The source pages have no counterpart:
- * this entry exists for callers that cannot allocate device memory after start-up — an engine
- * that reserves the whole device for its KV pool and treats any later cudaMalloc as a failure,
- * a plug-in whose host framework owns every device allocation, a runtime that permits
- * allocation only during initialisation. Arguments and results are those of
- * tg_ragged_paged_decode; plan may be a host-only plan (tg_plan_opts.host_only = 1), which holds
- * no device memory. The kernels' scratch (the plan's work list, copied in by plain host-to-
- * device copies on the stream, and the split heads' partial results) lives in one fixed
- * 16 MiB device array inside this library, which every GPU that loads the library holds
- * until the process exits; a plan that needs more returns TG_ENOMEM (the message says how
- * much it needs) without launching anything. The first call on a device also looks up the
- * array's device address and sets the kernels' shared-memory limit on that device; make that
- * first call before any stream capture. All calls share the array and each call overwrites
- * it: calls whose work overlaps on the GPU (other streams, other host threads) race and must
- * be serialised by the caller. Kernel-side range errors are skipped as in the plan-based
- * entry but are not reported. Calls no cudaMalloc, cudaFree or allocating library routine. */
 /* tg_ragged_paged_decode that also writes every retained token's scores for the H2O rule
  * below: token_scores (device fp32, 4-byte aligned, [table_len*16][G]) gets, at entry
  * (head_page_off[b*Hkv+h]*16 + t)*G + g, s = scale * q[b][h*G+g] . K_t (natural-log units, as
@@ -358,11 +343,37 @@ int tg_ragged_paged_decode_scores(tg_plan *plan, const void *q, const void *k_pa
                                   const int32_t *group_of_head, float scale, void *out, float *lse,
                                   float *token_scores, tg_stream stream);
 
+/* Ragged paged decode that allocates no device memory. The source pages have no counterpart:
+ * this entry exists for callers that cannot allocate device memory after start-up — an engine
+ * that reserves the whole device for its KV pool and treats any later cudaMalloc as a failure,
+ * a plug-in whose host framework owns every device allocation, a runtime that permits
+ * allocation only during initialisation. Arguments and results are those of
+ * tg_ragged_paged_decode; plan may be a host-only plan (tg_plan_opts.host_only = 1), which holds
+ * no device memory (the one case where a decode call accepts a host-only plan; cascade plans
+ * return TG_EUNSUPPORTED). A plan made for a device (tg_plan_opts.device >= 0) runs only on
+ * that device (TG_EINVAL when another one is current); a host-only plan made with device -1
+ * runs on the current device. The kernels' scratch (the plan's work list, copied in by plain
+ * host-to-device copies on the stream, and the split heads' partial results) lives in one
+ * fixed 16 MiB device array inside this library, which every GPU that loads the library holds
+ * until the process exits; a plan that needs more returns TG_ENOMEM (the message says how much
+ * it needs) without launching anything. The first call on a device also looks up the array's
+ * device address, clears its error word and sets the kernels' shared-memory limit on that
+ * device; make that first call before any stream capture. All calls share the array and each
+ * call overwrites it: calls whose work overlaps on the GPU (other streams, other host threads)
+ * race and must be serialised by the caller. The plan's wait bound (wait_limit_us) applies.
+ * Kernel-side range errors are skipped as in the plan-based entry and, with timeouts, are
+ * recorded in the array's error word, read by tg_ragged_paged_decode_noalloc_status. Calls no
+ * cudaMalloc, cudaFree or allocating library routine. */
 int tg_ragged_paged_decode_noalloc(tg_plan *plan, const void *q, const void *k_pages,
                                    const void *v_pages, const int32_t *page_table,
                                    const int64_t *head_page_off, const int32_t *head_kv_len,
                                    const int32_t *group_of_head, float scale, void *out,
                                    float *lse, tg_stream stream);
+/* Read and clear the error word of tg_ragged_paged_decode_noalloc's array on the current device,
+ * after the work queued on stream: TG_OK, TG_EBADPAGE or TG_ETIMEOUT for the no-alloc calls
+ * since the last read (TG_OK if no such call has run on this device). Synchronises the stream;
+ * allocates nothing. */
+int tg_ragged_paged_decode_noalloc_status(tg_stream stream);
 
 /* Tiered decode ("TTKV" 核心方法 1-3): as tg_ragged_paged_decode over the union of two tiers.
  * Per head, f = min(head_fast_len, n): tokens [0, n - f) are in the INT8 tier (row starts at

@@ -97,6 +97,7 @@ _SIGS = [
     ("tg_ragged_paged_decode", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _F32, _P, _P, _P]),
     ("tg_ragged_paged_decode_noalloc", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _F32, _P,
                                                       _P, _P]),
+    ("tg_ragged_paged_decode_noalloc_status", ctypes.c_int, [_P]),
     ("tg_tiered_decode", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                         _F32, _P, _P, _P]),
     ("tg_lse_merge", ctypes.c_int, [_I64, _I32, _P, _P, _P, _P, _P, _P]),
@@ -504,6 +505,12 @@ def tg_ragged_paged_decode_noalloc(plan: Plan, q, k_pages, v_pages, page_table, 
         plan.handle, _dp(q), _dp(k_pages), _dp(v_pages), _dp(page_table), _dp(head_page_off),
         _dp(head_kv_len), _dp(group_of_head), float(scale), _dp(out), _dp(lse),
         _stream(stream)), "tg_ragged_paged_decode_noalloc")
+
+
+def tg_ragged_paged_decode_noalloc_status(stream=None) -> int:
+    """Read and clear the no-alloc entry's error word on the current device (after the work
+    queued on stream): TG_OK, TG_EBADPAGE or TG_ETIMEOUT."""
+    return int(_lib().tg_ragged_paged_decode_noalloc_status(_stream(stream)))
 
 
 def tg_ragged_paged_decode_scores(plan: Plan, q, k_pages, v_pages, page_table, head_page_off,

@@ -56,7 +56,6 @@ void set_cuda_error(const char *what, int code) {
 // ------------------------------------------------------------------------------------------
 namespace dev {
 
-constexpr uint64_t kWaitNs = 4000000000ull;  // default bound of any single wait: 4 s
 constexpr uint64_t kDrainNs = 200000000ull;  // bound of the drain after a timeout: 0.2 s
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
@@ -2498,8 +2497,8 @@ constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
 
-// One-time set-up on the current device: the array's device address, and the decode
-// kernels' shared-memory limit.
+// One-time set-up on the current device: the array's device address, a cleared error word,
+// and the decode kernels' shared-memory limit.
 int noalloc_setup(int dev, void **ptr) {
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
     if (!g_noalloc_ptr[dev]) {
@@ -2509,6 +2508,7 @@ int noalloc_setup(int dev, void **ptr) {
             set_cuda_error("cudaGetSymbolAddress(scratch)", static_cast<int>(e));
             return TG_ECUDA;
         }
+        TG_CUDA_TRY(cudaMemset(p, 0, 256));
         TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<128, false, tg::kPairs>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget));
         TG_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<64, false, tg::kPairs>,
@@ -2528,6 +2528,10 @@ extern "C" int tg_ragged_paged_decode_noalloc(tg_plan *p, const void *q, const v
                                               void *out, float *lse, tg_stream stream_) {
     if (!p || p->tiered) return TG_EINVAL;
     if (!p->cunits.empty()) return TG_EUNSUPPORTED;  // cascade units live in the plan's memory
+    int dev = 0;
+    TG_CUDA_TRY(cudaGetDevice(&dev));
+    // A plan made for one device (host-only plans may name none: device -1) runs only there.
+    if (p->device >= 0 && p->device != dev) return TG_EINVAL;
     if (!q || !out || !lse || !head_kv_len || !aligned16(q) || !aligned16(out) || !aligned16(lse))
         return TG_EINVAL;
     const bool any_items = !p->items.empty();
@@ -2564,8 +2568,6 @@ extern "C" int tg_ragged_paged_decode_noalloc(tg_plan *p, const void *q, const v
     if (stages < 2) return TG_EUNSUPPORTED;
     const int smem_bytes = 1024 + tg::kPairs * stages * (stage_bytes + per_stage_extra) + tg::kPairs * 8;
 
-    int dev = 0;
-    TG_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= kNoAllocMaxDevices) return TG_EUNSUPPORTED;
     void *base_v = nullptr;
     int rc = noalloc_setup(dev, &base_v);
@@ -2590,9 +2592,11 @@ extern "C" int tg_ragged_paged_decode_noalloc(tg_plan *p, const void *q, const v
     at += b_po;
     float *d_pl = reinterpret_cast<float *>(at);
 
-    // The scratch keeps the previous call's contents: the error word and the dynamic tickets
-    // must start at zero; the work list is written afresh (plain copies, no allocation).
-    TG_CUDA_TRY(cudaMemsetAsync(base, 0, 256, stream));
+    // The scratch keeps the previous call's contents: the dynamic tickets must start at zero
+    // (a call that timed out leaves them part-counted); the error word collects the calls'
+    // range errors and timeouts until tg_ragged_paged_decode_noalloc_status reads and clears
+    // it; the work list is written afresh (plain copies, no allocation).
+    TG_CUDA_TRY(cudaMemsetAsync(d_dyn, 0, 8, stream));
     if (!p->items.empty())
         TG_CUDA_TRY(cudaMemcpyAsync(d_items, p->items.data(), p->items.size() * sizeof(Item),
                                     cudaMemcpyHostToDevice, stream));
@@ -2646,8 +2650,8 @@ extern "C" int tg_ragged_paged_decode_noalloc(tg_plan *p, const void *q, const v
         a.n_dyn = p->n_dyn;
         a.dyn_next = d_dyn;
         a.early_prologue = 0;
-        a.wait_ns = dev::kWaitNs;
-        a.withhold = 0;
+        a.wait_ns = p->wait_ns;
+        a.withhold = p->withhold;
         const CUtensorMap &tk = *reinterpret_cast<const CUtensorMap *>(p->tmaps[0]);
         const CUtensorMap &tv = *reinterpret_cast<const CUtensorMap *>(p->tmaps[1]);
         cudaLaunchConfig_t cfg = {};
@@ -2663,5 +2667,26 @@ extern "C" int tg_ragged_paged_decode_noalloc(tg_plan *p, const void *q, const v
     if (!p->merge.empty())
         return launch_merge(p, reinterpret_cast<const MergeHead *>(d_merge), reinterpret_cast<const float *>(d_po),
                             reinterpret_cast<const float *>(d_pl), out, lse, stream, false);
+    return TG_OK;
+}
+
+extern "C" int tg_ragged_paged_decode_noalloc_status(tg_stream stream_) {
+    int dev = 0;
+    TG_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return TG_EUNSUPPORTED;
+    void *base = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        base = g_noalloc_ptr[dev];
+    }
+    if (!base) return TG_OK;  // no call has run on this device yet
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    uint32_t err = 0;
+    TG_CUDA_TRY(cudaMemcpyAsync(&err, base, 4, cudaMemcpyDeviceToHost, stream));
+    TG_CUDA_TRY(cudaStreamSynchronize(stream));
+    TG_CUDA_TRY(cudaMemsetAsync(base, 0, 4, stream));
+    TG_CUDA_TRY(cudaStreamSynchronize(stream));
+    if (err & kErrTimeout) return TG_ETIMEOUT;
+    if (err & (kErrBadPage | kErrBadRow | kErrPlan)) return TG_EBADPAGE;
     return TG_OK;
 }

@@ -241,8 +241,9 @@ def _bf16_tensor(bits: np.ndarray, device):
     return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)
 
 
-def _pool_to_device(sp, which, n, layer, device, chunk_pages=1 << 16):
-    """Generate a pool on the host in chunks and copy it to the device."""
+def _pool_to_device(sp, which, n, device, chunk_pages=1 << 16):
+    """Generate a pool on the host in chunks and copy it to the device. The contents do not
+    depend on the layer (see synth.pool_bits)."""
     import torch
     out = torch.empty((n, sp.page, sp.D), dtype=torch.bfloat16, device=device)
     per = sp.page * sp.D
@@ -250,18 +251,28 @@ def _pool_to_device(sp, which, n, layer, device, chunk_pages=1 << 16):
     buf = np.empty(min(n, chunk_pages) * per, dtype=np.uint16)
     for p0 in range(0, n, chunk_pages):
         c = min(chunk_pages, n - p0)
-        synth.normal_bf16(sp.seed, synth.stream_id(kind, layer), c * per, i0=p0 * per,
+        synth.normal_bf16(sp.seed, synth.stream_id(kind), c * per, i0=p0 * per,
                           out=buf[:c * per])
         out[p0:p0 + c].copy_(torch.from_numpy(buf[:c * per].view(np.int16)).view(torch.bfloat16)
                              .view(c, sp.page, sp.D), non_blocking=False)
     return out
 
 
+def pools_to_device(sp: synth.Spec, num_pages: int, device="cuda"):
+    """The bf16 K and V pools of num_pages pages on the device. A layer whose pool has n <=
+    num_pages pages reads the first n of them (the same bytes its own pool would hold), so one
+    upload serves every layer of a multi-layer workload."""
+    return (_pool_to_device(sp, "k", num_pages, device), _pool_to_device(sp, "v", num_pages, device))
+
+
 def to_device(sp: synth.Spec, lay: Layout, layer: int = 0, device="cuda", num_workers: int = 0,
               min_splits: int = 1, max_chunk_pages: int = 0, seqs=None, static_permille: int = 0,
               dyn_chunk_pages: int = 0, early_prologue: bool = False, wait_limit_us: int = 0,
               test_withhold_page: int = 0, cascade: bool = False,
-              min_readers: int = 2, whole_heads: bool = False) -> DeviceBatch:
+              min_readers: int = 2, whole_heads: bool = False, pools=None) -> DeviceBatch:
+    """Upload one layer's tables, lengths and queries, make its plan, and upload (or, with
+    pools = (k, v) from pools_to_device holding at least lay.num_pages pages, reuse) its bf16
+    K and V pools."""
     import torch
     dev = torch.device(device)
     B = lay.kv_len.shape[0]
@@ -292,8 +303,12 @@ def to_device(sp: synth.Spec, lay: Layout, layer: int = 0, device="cuda", num_wo
     lse = torch.empty((B, sp.Hq), dtype=torch.float32, device=dev)
     it = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).to(dev)
     db = DeviceBatch(sp, lay, plan, q, out, lse)
-    db.k = _pool_to_device(sp, "k", lay.num_pages, layer, dev)
-    db.v = _pool_to_device(sp, "v", lay.num_pages, layer, dev)
+    if pools is not None:
+        assert pools[0].shape[0] >= lay.num_pages and pools[1].shape[0] >= lay.num_pages
+        db.k, db.v = pools[0][:lay.num_pages], pools[1][:lay.num_pages]
+    else:
+        db.k = _pool_to_device(sp, "k", lay.num_pages, dev)
+        db.v = _pool_to_device(sp, "v", lay.num_pages, dev)
     db.table = it(lay.table if lay.table.size else np.full(1, -1), np.int32)
     db.head_off = it(lay.head_off, np.int64)
     db.kv_len = it(lay.kv_len, np.int32)
@@ -311,7 +326,7 @@ def to_device(sp: synth.Spec, lay: Layout, layer: int = 0, device="cuda", num_wo
         db.k_scale = torch.empty((ns, sp.page), dtype=torch.float32, device=dev)
         db.v_scale = torch.empty((ns, sp.page), dtype=torch.float32, device=dev)
         for which, codes, scale in (("kslow", db.k_q8, db.k_scale), ("vslow", db.v_q8, db.v_scale)):
-            src = _pool_to_device(sp, which, ns, layer, dev)
+            src = _pool_to_device(sp, which, ns, dev)
             (tg_quantize_int4 if i4 else tg_quantize_int8)(src, codes, scale)
             del src
         torch.cuda.synchronize(dev)

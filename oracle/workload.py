@@ -135,12 +135,12 @@ def reference(sp, o: OLayout, layer=0, sel=None, seqs=None):
     q = q_bits(sp, layer, seqs)
     if o.fast_len is None:
         if sel is None:
-            k = synth.pool_bits(sp, "k", o.num_pages, layer)
-            v = synth.pool_bits(sp, "v", o.num_pages, layer)
+            k = synth.pool_bits(sp, "k", o.num_pages)
+            v = synth.pool_bits(sp, "v", o.num_pages)
             return oracle.decode(q, k, v, o.table, o.head_off, o.kv_len, sp.scale)
         return _sampled(sp, o, q, layer, sel)
-    k = synth.pool_bits(sp, "k", o.num_pages, layer)
-    v = synth.pool_bits(sp, "v", o.num_pages, layer)
+    k = synth.pool_bits(sp, "k", o.num_pages)
+    v = synth.pool_bits(sp, "v", o.num_pages)
     kq, ks, vq, vs = slow_tier(sp, o, layer)
     st = o.slow_table if o.slow_table.size else np.zeros(1, np.int32)
     return oracle.tiered_decode(q, kq, vq, ks, vs, st, o.slow_off, k, v, o.table, o.head_off,
@@ -150,8 +150,8 @@ def reference(sp, o: OLayout, layer=0, sel=None, seqs=None):
 def slow_tier(sp, o: OLayout, layer=0):
     """The quantised slow tier as the oracle stores it: (k codes, k scales, v codes, v scales),
     codes int8 [Ps][page][D] (INT4 tiers unpacked from their packed form)."""
-    kb = synth.pool_bits(sp, "kslow", o.num_slow_pages, layer)
-    vb = synth.pool_bits(sp, "vslow", o.num_slow_pages, layer)
+    kb = synth.pool_bits(sp, "kslow", o.num_slow_pages)
+    vb = synth.pool_bits(sp, "vslow", o.num_slow_pages)
     if getattr(sp, "slow_bits", 8) == 4:
         kp, ks = oracle.quantize_int4(kb)
         vp, vs = oracle.quantize_int4(vb)
@@ -173,8 +173,8 @@ def _sampled(sp, o, q, layer, sel):
         off = int(o.head_off.reshape(-1)[x])
         pages.append(o.table[off:off + n])
     uniq = np.unique(np.concatenate(pages))
-    k = synth.pool_page_bits(sp, "k", uniq, layer)
-    v = synth.pool_page_bits(sp, "v", uniq, layer)
+    k = synth.pool_page_bits(sp, "k", uniq)
+    v = synth.pool_page_bits(sp, "v", uniq)
     table = _remap(o.table, uniq)
     return oracle.decode(q, k, v, table, o.head_off, o.kv_len, sp.scale, sel=sel)
 

@@ -283,25 +283,27 @@ def q_bits(sp: Spec, layer: int = 0) -> np.ndarray:
     return normal_bf16(sp.seed, stream_id(S_Q, layer), n).reshape(sp.B, sp.Hq, sp.D)
 
 
-def pool_bits(sp: Spec, which: str, num_pages: int, layer: int = 0,
+def pool_bits(sp: Spec, which: str, num_pages: int,
               out: Optional[np.ndarray] = None) -> np.ndarray:
     """Page-pool contents as bf16 bits uint16[num_pages, page, D], N(0, 1) per element,
-    a pure function of (physical page, slot, dim). which in {"k", "v", "kslow", "vslow"}."""
+    a pure function of (physical page, slot, dim). which in {"k", "v", "kslow", "vslow"}.
+    The contents do not depend on the layer: every layer's pool holds the same bytes, and
+    the layer's own tables decide which pages (and so which values) its heads read."""
     kind = {"k": S_K, "v": S_V, "kslow": S_KSLOW, "vslow": S_VSLOW}[which]
     n = num_pages * sp.page * sp.D
     flat = None if out is None else out.reshape(-1)
-    return normal_bf16(sp.seed, stream_id(kind, layer), n, out=flat).reshape(
+    return normal_bf16(sp.seed, stream_id(kind), n, out=flat).reshape(
         num_pages, sp.page, sp.D)
 
 
-def pool_page_bits(sp: Spec, which: str, pages: np.ndarray, layer: int = 0) -> np.ndarray:
+def pool_page_bits(sp: Spec, which: str, pages: np.ndarray) -> np.ndarray:
     """Contents of selected physical pages only (same values as pool_bits), for sampled
     checks at full size: uint16[len(pages), page, D]."""
     kind = {"k": S_K, "v": S_V, "kslow": S_KSLOW, "vslow": S_VSLOW}[which]
     per = sp.page * sp.D
     out = np.empty((len(pages), sp.page, sp.D), dtype=np.uint16)
     for i, p in enumerate(np.asarray(pages, dtype=np.int64)):
-        normal_bf16(sp.seed, stream_id(kind, layer), per, i0=int(p) * per,
+        normal_bf16(sp.seed, stream_id(kind), per, i0=int(p) * per,
                     out=out[i].reshape(-1))
     return out
 

@@ -2,7 +2,6 @@
 oracle rows, and `_parity_sample` compares a step's outputs with them row by row (here the
 "step" outputs are the oracle's own rows rounded to the device dtypes, so the differences are
 rounding only, and a planted error shows up)."""
-import types
 from dataclasses import replace
 
 import numpy as np
@@ -32,19 +31,19 @@ def test_parity_sample_against_oracle_rows(monkeypatch, cfg, bits):
     lse = torch.full((rows,), float("-inf"), dtype=torch.float64)
     out[torch.from_numpy(sel)] = torch.from_numpy(o_ref)
     lse[torch.from_numpy(sel)] = torch.from_numpy(l_ref)
-    db = types.SimpleNamespace(out=out.to(torch.bfloat16).reshape(sp.B, sp.Hq, sp.D),
-                               lse=lse.to(torch.float32).reshape(sp.B, sp.Hq))
-    rep = bench._parity_sample(first, db, sp.D)
+    out_d = out.to(torch.bfloat16).float().numpy()      # the step's outputs in device dtypes
+    lse_d = lse.to(torch.float32).numpy()
+    rep = bench._parity_sample(first, out_d, lse_d)
     assert "error" not in rep, rep
     assert rep["rows"] == len(sel)
     assert rep["max_abs_out"] <= 2 ** -8 * max(1.0, float(np.abs(o_ref).max()))   # bf16 rounding
     assert rep["max_abs_lse"] <= 1e-5 * max(1.0, float(np.abs(l_ref[np.isfinite(l_ref)]).max()))
     # a planted error in one sampled row is reported as it is
     r0 = int(sel[len(sel) // 2])
-    db.out.reshape(rows, sp.D)[r0, 3] += 0.5
-    assert bench._parity_sample(first, db, sp.D)["max_abs_out"] >= 0.4
+    out_d[r0, 3] += 0.5
+    assert bench._parity_sample(first, out_d, lse_d)["max_abs_out"] >= 0.4
 
 
 def test_parity_sample_records_a_failure_instead_of_raising():
-    rep = bench._parity_sample([], types.SimpleNamespace(out=None, lse=None), 128)
+    rep = bench._parity_sample([], None, None)
     assert set(rep) == {"error"}

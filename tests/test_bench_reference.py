@@ -8,10 +8,10 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _run(env_extra):
+def _run(env_extra, extra=("--config", "2")):
     env = dict(os.environ, **env_extra)
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "3",
-                        "--warmup", "3"], cwd=ROOT, env=env, capture_output=True, text=True,
+                        "--warmup", "3", *extra], cwd=ROOT, env=env, capture_output=True, text=True,
                        timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     return [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
@@ -34,3 +34,17 @@ def test_reference_arm_json_line():
 
 def test_reference_arm_other_ranks_print_nothing():
     assert _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+def test_both_arms_name_the_same_config():
+    """The two arms build their config dicts with one helper: for the default multi-layer
+    workload it names every layer, and a multi-rank run names the global batch."""
+    sys.path.insert(0, ROOT)
+    import bench
+    for world in (1, 2):
+        sp = bench._global_spec(3, world)
+        c = bench._config(3, sp, world, 32)
+        assert c["layers"] == 32 and c["global_batch"] == 256 * world and c["config_id"] == 3
+        assert "layers 32 of 32" in c["workload"]
+    c1 = bench._config(1, bench._global_spec(1, 1), 1, 1)
+    assert "layers" not in c1 and "flushed" in c1["l2"]

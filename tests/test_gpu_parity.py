@@ -78,6 +78,21 @@ def test_gqa_and_head_dims(G, D):
     _run(sp, num_workers=37)
 
 
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("workers", [0, 37])
+def test_tiered_gqa_sweep(G, bits, workers):
+    """The tiered kernel at every group size it accepts (G = 8 runs a shallower ring: its
+    stages hold 8 query rows), INT8 and INT4 slow tiers, ragged tail pages in both tiers
+    (1300 slow = 81 pages + 4 tokens, 200 fast = 12 pages + 8 tokens), heads split into
+    several items and merged."""
+    sp = synth.Spec("tiered gqa sweep", "tiered", B=2, Hq=2 * G, Hkv=2, D=128, len_lo=1500,
+                    len_hi=1500, fast_tokens=200, seed=0x7A4E1100 + 10 * G + bits,
+                    slow_bits=bits)
+    db, _ = _run(sp, num_workers=workers, min_splits=4, max_chunk_pages=16)
+    assert tg.tg_plan_get_info(db.plan)["n_merge"] > 0
+
+
 def test_empty_and_single_token_heads():
     sp = synth.Spec("edges", "direct", B=4, Hq=8, Hkv=4, D=128, len_lo=0, len_hi=2,
                     seed=0x7A4E2000)
@@ -248,11 +263,6 @@ def test_argument_validation():
 # Full sizes, in the launch configuration the bench times (default plan options).
 # ---------------------------------------------------------------------------------------
 
-def _sample_rows(sp, n, seed):
-    rng = np.random.default_rng(seed)
-    return np.sort(rng.choice(sp.B * sp.Hq, size=min(n, sp.B * sp.Hq), replace=False))
-
-
 def test_full_config1_all_rows():
     _run(synth.preset(1), **workload.timed_plan_options(1))
 
@@ -265,33 +275,37 @@ def test_full_config2_default_plan_all_rows():
     _run(synth.preset(2))
 
 
-def test_full_config3_sampled_rows_two_layers():
+def test_full_config3_all_rows_two_layers():
+    """Every query row of two layers of the serving step (8192 rows each), in the plan options
+    the bench times; the layers share the bench's one pool upload."""
     sp = synth.preset(3)
     for layer in (0, 17):
-        _run(sp, layer, sel=_sample_rows(sp, 96, layer), **workload.timed_plan_options(3))
+        _run(sp, layer, **workload.timed_plan_options(3))
 
 
-def test_full_config4_sampled_rows():
-    """The prefix-cascade plan the bench times (tcgen05 cascade + split-K items + merge)."""
+def test_full_config4_all_rows():
+    """The prefix-cascade plan the bench times (tcgen05 cascade + split-K items + merge), every
+    one of the 16384 query rows."""
     sp = synth.preset(4)
-    db, _ = _run(sp, sel=_sample_rows(sp, 256, 4), **workload.timed_plan_options(4))
+    db, _ = _run(sp, **workload.timed_plan_options(4))
     assert tg.tg_plan_get_info(db.plan)["n_cascade"] > 0
 
 
-def test_full_config5_sampled_rows():
+def test_full_config5_all_rows():
     sp = synth.preset(5)
-    _run(sp, sel=_sample_rows(sp, 24, 5), **workload.timed_plan_options(5))
+    _run(sp, **workload.timed_plan_options(5))
 
 
-def test_full_config5_int4_sampled_rows():
+def test_full_config5_int4_all_rows():
     sp = replace(synth.preset(5), slow_bits=4)
-    _run(sp, sel=_sample_rows(sp, 24, 6), **workload.timed_plan_options(5))
+    _run(sp, **workload.timed_plan_options(5))
 
 
-def test_full_config5_host_streamed_sampled_rows():
-    """The INT8 tier streamed from pinned host memory in 8192-page blocks through a ring of 3
-    (the bench's ttkv-host configuration), sampled rows against the oracle."""
-    sp = synth.preset(5)
+@pytest.mark.parametrize("bits", [8, 4])
+def test_full_config5_host_streamed_all_rows(bits):
+    """The slow tier streamed from pinned host memory in 8192-page blocks through a ring of 3
+    (the bench's ttkv-host configuration), every row against the oracle."""
+    sp = replace(synth.preset(5), slow_bits=bits)
     lay = workload.layout(sp, 0)
     kw = {k: v for k, v in workload.timed_plan_options(5).items() if k != "early_prologue"}
     db = workload.to_device(sp, lay, 0, **kw)
@@ -299,7 +313,6 @@ def test_full_config5_host_streamed_sampled_rows():
     db.run_streamed(ss, db.host_slow_tier())
     torch.cuda.synchronize()
     assert ss.status() == tg.TG_OK
-    sel = _sample_rows(sp, 24, 7)
     ol = ors.layout(sp, 0)
-    ref_out, ref_lse = ors.reference(sp, ol, 0, sel=sel)
-    _compare(db, ref_out, ref_lse, sel)
+    ref_out, ref_lse = ors.reference(sp, ol, 0)
+    _compare(db, ref_out, ref_lse)

@@ -85,7 +85,7 @@ def test_full_pool_round_trip():
     sp = synth.preset(2)
     from non_uniform_paged_flash_b200 import workload
     lay = workload.layout(sp, 0)
-    k = workload._pool_to_device(sp, "k", lay.num_pages, 0, "cuda")
+    k = workload._pool_to_device(sp, "k", lay.num_pages, "cuda")
     n = k.numel()
     flat = k.view(torch.int16).reshape(-1)
     cb = torch.empty(16, dtype=torch.uint8, device="cuda")

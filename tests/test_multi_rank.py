@@ -43,10 +43,13 @@ def _shard_worker(rank, world, port, cfg, slow_bits, q):
         _init(rank, world, port)
         bench.SLOW_BITS = slow_bits
         sp = bench._global_spec(cfg, world)
-        kv, fast = workload.retained(sp, 0)
-        mine = bench._my_sequences(sp, rank, world, kv, fast)
-        lay = workload.layout(sp, 0, mine)
-        ow.assert_same_layout(lay, ow.layout(sp, 0, mine))
+        # the multi-layer workload places each layer's sequences by that layer's bytes; the
+        # rest of the check runs on its last layer here
+        for layer in ((0, 17) if sp.layers > 1 else (0,)):
+            kv, fast = workload.retained(sp, layer)
+            mine = bench._my_sequences(sp, rank, world, kv, fast)
+            lay = workload.layout(sp, layer, mine)
+            ow.assert_same_layout(lay, ow.layout(sp, layer, mine))
         shape = tg.make_shape(len(mine), sp.Hq, sp.Hkv, sp.D, lay.num_pages, lay.num_slow_pages)
         plan = tg.tg_plan_create(shape, lay.kv_len, lay.group_of_head, lay.group_off,
                                  fast_len=lay.fast_len,
@@ -78,7 +81,7 @@ def _seq_bytes(sp, kv, fast, slow_bits):
     return ((kv - f) * (2 * code + 8) + f * 4 * sp.D).sum(1)
 
 
-@pytest.mark.parametrize("cfg,slow_bits", [(2, 8), (4, 8), (5, 8), (5, 4)])
+@pytest.mark.parametrize("cfg,slow_bits", [(2, 8), (3, 8), (4, 8), (5, 8), (5, 4)])
 def test_two_rank_shards_cover_batch_once_and_balance(cfg, slow_bits):
     world, port = 2, _free_port()
     ctx = mp.get_context("spawn")
@@ -101,7 +104,7 @@ def test_two_rank_shards_cover_batch_once_and_balance(cfg, slow_bits):
     sp = replace(synth.preset(cfg), B=B)
     if sp.kind == "tiered":
         sp = replace(sp, slow_bits=slow_bits)
-    kv, fast = ow.retained(sp, 0)
+    kv, fast = ow.retained(sp, 17 if sp.layers > 1 else 0)     # the worker's last layer
     per_seq = _seq_bytes(sp, kv, fast, slow_bits)
     loads = [int(per_seq[a[a >= 0]].sum()) for a in alls]
     assert max(loads) <= per_seq.sum() / world + per_seq.max()        # LPT bound

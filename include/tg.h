@@ -101,10 +101,17 @@ int tg_budget_groups(int32_t n_heads, const int32_t *budget_ppm, int32_t n_group
  * memory. */
 typedef struct tg_alloc tg_alloc;
 
-/* num_pages >= 1; page = tokens per page (>= 1). free_order: a permutation of
- * 0..num_pages-1 giving the initial free-list order (NULL = ascending). A non-permutation
- * returns TG_EINVAL. */
-int tg_alloc_create(int64_t num_pages, int32_t page, const int32_t *free_order, tg_alloc **out);
+/* Allocator over a pool of num_pages pages (>= 1) of `page` tokens each (>= 1) whose initial
+ * free list is a seeded shuffle of the page ids (the pool's pages in no particular order, as a
+ * long-running server's pool): the Fisher-Yates (Durstenfeld) shuffle of 0..num_pages-1 that
+ * for i = num_pages-1 down to 1 swaps entries i and (x_k mod (i+1)), where x_0, x_1, ... is the
+ * SplitMix64 sequence seeded with `seed` (Steele, Lea & Flood 2014: state += 0x9E3779B97F4A7C15,
+ * output = its 64-bit finaliser) and k counts the swaps from 0. */
+int tg_alloc_create(int64_t num_pages, int32_t page, uint64_t seed, tg_alloc **out);
+/* As tg_alloc_create with the initial free-list order given: free_order is a permutation of
+ * 0..num_pages-1 (NULL = ascending). A non-permutation returns TG_EINVAL. */
+int tg_alloc_create_ordered(int64_t num_pages, int32_t page, const int32_t *free_order,
+                            tg_alloc **out);
 void tg_alloc_destroy(tg_alloc *a);
 int64_t tg_alloc_free_pages(const tg_alloc *a);   /* pages currently on the free list */
 /* References held on a page (0 = free; a shared page counts its segment plus each reader). */
@@ -114,35 +121,38 @@ int32_t tg_alloc_refcount(const tg_alloc *a, int32_t page_id);
  * head, taken head ascending, page ascending. Only full pages are shared; a partial tail goes
  * into each reader's private pages. *seg_id receives the segment id; page_ids (may be NULL)
  * receives [n_heads][floor(n_tokens/page)]. All-or-nothing: TG_ENOSPC leaves state unchanged. */
-int tg_alloc_share_segment(tg_alloc *a, int32_t n_tokens, int32_t n_heads, int32_t *seg_id,
-                           int32_t *page_ids);
+int tg_share_segment(tg_alloc *a, int32_t n_tokens, int32_t n_heads, int32_t *seg_id,
+                     int32_t *page_ids);
 
 /* Reservation of sequence seq_id at admission: for each KV head h (ascending), its page list
  * is the full pages of each segment in prefix_segs[0..n_prefix) (in order; a negative id is
  * skipped), followed by ceil((kv_len[h] - shared tokens)/page) private pages from the free
  * list. kv_len[h] must be >= the shared tokens (TG_EINVAL otherwise). All-or-nothing:
  * TG_ENOSPC leaves state unchanged. page_ids (host, capacity entries) receives the lists
- * head after head; *n_written the total. Each head's count is ceil(kv_len[h]/page) when every
+ * head after head; head_count (host, n_heads entries, may be NULL) each head's page count
+ * (its shared pages plus its private ones), the head_count rows tg_build_group_tables takes;
+ * *n_written (may be NULL) the total. Each head's count is ceil(kv_len[h]/page) when every
  * shared segment holds whole pages. seq_id must be new (TG_EEXIST). */
-int tg_alloc_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads, const int32_t *kv_len,
-                     int32_t n_prefix, const int32_t *prefix_segs, int32_t *page_ids,
-                     int64_t capacity, int64_t *n_written);
+int tg_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads, const int32_t *kv_len,
+               int32_t n_prefix, const int32_t *prefix_segs, int32_t *page_ids,
+               int64_t capacity, int32_t *head_count, int64_t *n_written);
 /* Release a sequence: private pages return to the free list, shared pages drop one reference. */
-int tg_alloc_release(tg_alloc *a, int32_t seq_id);
+int tg_release(tg_alloc *a, int32_t seq_id);
 /* Drop a segment's own reference; its pages return once no sequence reads them. */
-int tg_alloc_release_segment(tg_alloc *a, int32_t seg_id);
+int tg_release_segment(tg_alloc *a, int32_t seg_id);
 
 /* Group page tables ("Tangram" 三大机制 2). For B sequences x Hkv heads with head_count[b][h]
  * pages whose ids are listed in page_ids (flat: b ascending, h ascending, page ascending —
- * the order tg_alloc_reserve writes them for b = 0, 1, ...): group g's table is dense
+ * the order tg_reserve writes them for b = 0, 1, ...): group g's table is dense
  * [B][H_g][P_g] (heads of g ascending, P_g = max page count in g, unused slots -1); tables
  * concatenated in group order. Writes head_off[B*Hkv] (start of each row) and
  * group_off[n_groups+1] (start of each group table; group_off[n_groups] = total length).
  * table may be NULL to query the length (head_off then may be NULL too); otherwise it must
  * hold group_off[n_groups] entries. All arrays host. */
-int tg_group_tables(int32_t B, int32_t Hkv, const int32_t *head_count,
-                    const int32_t *group_of_head, int32_t n_groups, const int32_t *page_ids,
-                    int32_t *table, int64_t *head_off, int64_t *group_off);
+int tg_build_group_tables(int32_t B, int32_t Hkv, const int32_t *head_count,
+                          const int32_t *group_of_head, int32_t n_groups,
+                          const int32_t *page_ids, int32_t *table, int64_t *head_off,
+                          int64_t *group_off);
 
 /* Ahead-of-time placement of sequences on GPUs ("Tangram" 三大机制 3): longest-processing-
  * time greedy over seq_bytes (descending, ties by index) onto the least-loaded GPU (ties by
@@ -209,7 +219,7 @@ typedef struct tg_plan_opts {
  * calls check the device copy against it. fast_len[B*Hkv] (host) or NULL: tiered plan whose
  * last min(fast_len, kv_len) tokens of each head are in the bf16 tier and the rest in the slow
  * tier (INT8, or INT4 with opts->slow_bits = 4). group_of_head[Hkv] and group_off[n_groups+1] (host; from tg_budget_groups /
- * tg_group_tables) bound every row of the bf16 (fast) table to its group table; for a tiered
+ * tg_build_group_tables) bound every row of the bf16 (fast) table to its group table; for a tiered
  * plan slow_table_len bounds the slow tier's table (ignored otherwise).
  * Each head's tokens are cut into chunks (min_splits, max_chunk_pages; chunks never cross a
  * tier boundary). The first static_permille of the chunks' byte cost is partitioned into
@@ -316,7 +326,7 @@ int tg_plan_trace_read(tg_plan *p, uint64_t *trace, tg_stream stream);
  *   plan        from tg_plan_create with fast_len = NULL and this shape.
  *   q           device bf16 [B][Hq][D]
  *   k_pages     device bf16 [num_pages][16][D];   v_pages likewise
- *   page_table  device int32, the concatenated group tables (tg_group_tables)
+ *   page_table  device int32, the concatenated group tables (tg_build_group_tables)
  *   head_page_off device int64 [B*Hkv];  head_kv_len device int32 [B*Hkv] (must equal the
  *               plan's kv_len); group_of_head device int32 [Hkv]
  *   scale       softmax scale applied in fp32 (e.g. 1/sqrt(D))

@@ -74,15 +74,16 @@ _SIGS = [
     ("tg_last_cuda_error", ctypes.c_char_p, []),
     ("tg_retained_lengths", ctypes.c_int, [_I64, _P, _P, _P]),
     ("tg_budget_groups", ctypes.c_int, [_I32, _P, _I32, _P]),
-    ("tg_alloc_create", ctypes.c_int, [_I64, _I32, _P, ctypes.POINTER(_P)]),
+    ("tg_alloc_create", ctypes.c_int, [_I64, _I32, ctypes.c_uint64, ctypes.POINTER(_P)]),
+    ("tg_alloc_create_ordered", ctypes.c_int, [_I64, _I32, _P, ctypes.POINTER(_P)]),
     ("tg_alloc_destroy", None, [_P]),
     ("tg_alloc_free_pages", _I64, [_P]),
     ("tg_alloc_refcount", _I32, [_P, _I32]),
-    ("tg_alloc_share_segment", ctypes.c_int, [_P, _I32, _I32, _P, _P]),
-    ("tg_alloc_reserve", ctypes.c_int, [_P, _I32, _I32, _P, _I32, _P, _P, _I64, _P]),
-    ("tg_alloc_release", ctypes.c_int, [_P, _I32]),
-    ("tg_alloc_release_segment", ctypes.c_int, [_P, _I32]),
-    ("tg_group_tables", ctypes.c_int, [_I32, _I32, _P, _P, _I32, _P, _P, _P, _P]),
+    ("tg_share_segment", ctypes.c_int, [_P, _I32, _I32, _P, _P]),
+    ("tg_reserve", ctypes.c_int, [_P, _I32, _I32, _P, _I32, _P, _P, _I64, _P, _P]),
+    ("tg_release", ctypes.c_int, [_P, _I32]),
+    ("tg_release_segment", ctypes.c_int, [_P, _I32]),
+    ("tg_build_group_tables", ctypes.c_int, [_I32, _I32, _P, _P, _I32, _P, _P, _P, _P]),
     ("tg_place_sequences", ctypes.c_int, [_I32, _P, _I32, _P]),
     ("tg_plan_create", ctypes.c_int, [ctypes.POINTER(tg_shape), _P, _P, _P, _P, _I32, _I64,
                                       ctypes.POINTER(tg_plan_opts), ctypes.POINTER(_P)]),
@@ -247,11 +248,21 @@ def tg_budget_groups(budget_ppm, n_groups: int) -> np.ndarray:
     return out
 
 
-def tg_alloc_create(num_pages: int, page: int = 16, free_order=None):
+def tg_alloc_create(num_pages: int, page: int = 16, seed: int = 0):
+    """Allocator whose initial free list is the library's seeded shuffle of the page ids."""
+    h = ctypes.c_void_p()
+    _check(_lib().tg_alloc_create(num_pages, page, ctypes.c_uint64(int(seed) & (2**64 - 1)),
+                                  ctypes.byref(h)), "tg_alloc_create")
+    h.page = page   # output buffers of the calls below are sized with the allocator's page
+    return h
+
+
+def tg_alloc_create_ordered(num_pages: int, page: int = 16, free_order=None):
     fo = None if free_order is None else _h(free_order, np.int32).reshape(-1)
     _count(fo, num_pages, "free_order")
     h = ctypes.c_void_p()
-    _check(_lib().tg_alloc_create(num_pages, page, _hp(fo), ctypes.byref(h)), "tg_alloc_create")
+    _check(_lib().tg_alloc_create_ordered(num_pages, page, _hp(fo), ctypes.byref(h)),
+           "tg_alloc_create_ordered")
     h.page = page   # output buffers of the calls below are sized with the allocator's page
     return h
 
@@ -278,7 +289,7 @@ def tg_alloc_refcount(a, page_id: int) -> int:
     return int(_lib().tg_alloc_refcount(a, page_id))
 
 
-def tg_alloc_share_segment(a, n_tokens: int, n_heads: int, page: int = None):
+def tg_share_segment(a, n_tokens: int, n_heads: int, page: int = None):
     """Returns (seg_id, page_ids int32[n_heads, n_tokens // page])."""
     page = _alloc_page(a, page)
     if page is None:
@@ -286,34 +297,38 @@ def tg_alloc_share_segment(a, n_tokens: int, n_heads: int, page: int = None):
     full = n_tokens // page
     ids = np.empty((n_heads, full), dtype=np.int32)
     sid = ctypes.c_int32()
-    _check(_lib().tg_alloc_share_segment(a, n_tokens, n_heads, ctypes.byref(sid), _hp(ids)),
-           "tg_alloc_share_segment")
+    _check(_lib().tg_share_segment(a, n_tokens, n_heads, ctypes.byref(sid), _hp(ids)),
+           "tg_share_segment")
     return sid.value, ids
 
 
-def tg_alloc_reserve(a, seq_id: int, kv_len, prefix_segs=(), page: int = None) -> np.ndarray:
-    """Reserve all heads of one sequence; returns its page ids (flat, head after head)."""
+def tg_reserve(a, seq_id: int, kv_len, prefix_segs=(), page: int = None,
+               with_counts: bool = False):
+    """Reserve all heads of one sequence; returns its page ids (flat, head after head), and
+    with with_counts also each head's page count (int32[n_heads])."""
     page = _alloc_page(a, page) or 1   # page 1 sizes the buffer for any allocator
     kv = _h(kv_len, np.int32).reshape(-1)
     segs = _h(np.asarray(prefix_segs, dtype=np.int32).reshape(-1), np.int32)
     cap = int(kv.astype(np.int64).sum() // page + kv.size * (1 + max(1, segs.size)))
     ids = np.empty(cap, dtype=np.int32)
+    counts = np.empty(kv.size, dtype=np.int32)
     n = ctypes.c_int64()
-    _check(_lib().tg_alloc_reserve(a, seq_id, kv.size, _hp(kv), segs.size,
-                                   _hp(segs) if segs.size else None, _hp(ids), cap,
-                                   ctypes.byref(n)), "tg_alloc_reserve")
-    return ids[:n.value].copy()
+    _check(_lib().tg_reserve(a, seq_id, kv.size, _hp(kv), segs.size,
+                             _hp(segs) if segs.size else None, _hp(ids), cap, _hp(counts),
+                             ctypes.byref(n)), "tg_reserve")
+    ids = ids[:n.value].copy()
+    return (ids, counts) if with_counts else ids
 
 
-def tg_alloc_release(a, seq_id: int):
-    _check(_lib().tg_alloc_release(a, seq_id), "tg_alloc_release")
+def tg_release(a, seq_id: int):
+    _check(_lib().tg_release(a, seq_id), "tg_release")
 
 
-def tg_alloc_release_segment(a, seg_id: int):
-    _check(_lib().tg_alloc_release_segment(a, seg_id), "tg_alloc_release_segment")
+def tg_release_segment(a, seg_id: int):
+    _check(_lib().tg_release_segment(a, seg_id), "tg_release_segment")
 
 
-def tg_group_tables(head_count, group_of_head, n_groups: int, page_ids):
+def tg_build_group_tables(head_count, group_of_head, n_groups: int, page_ids):
     """Returns (table int32[len], head_off int64[B, Hkv], group_off int64[n_groups + 1])."""
     hc = _h(head_count, np.int32)
     B, Hkv = hc.shape
@@ -322,12 +337,12 @@ def tg_group_tables(head_count, group_of_head, n_groups: int, page_ids):
     _count(goh, Hkv, "group_of_head")
     _count(ids, int(np.maximum(hc, 0).astype(np.int64).sum()), "page_ids", at_least=True)
     goff = np.empty(n_groups + 1, dtype=np.int64)
-    _check(_lib().tg_group_tables(B, Hkv, _hp(hc), _hp(goh), n_groups, None, None, None,
-                                  _hp(goff)), "tg_group_tables")
+    _check(_lib().tg_build_group_tables(B, Hkv, _hp(hc), _hp(goh), n_groups, None, None, None,
+                                        _hp(goff)), "tg_build_group_tables")
     table = np.empty(max(1, int(goff[-1])), dtype=np.int32)
     off = np.empty((B, Hkv), dtype=np.int64)
-    _check(_lib().tg_group_tables(B, Hkv, _hp(hc), _hp(goh), n_groups, _hp(ids), _hp(table),
-                                  _hp(off), _hp(goff)), "tg_group_tables")
+    _check(_lib().tg_build_group_tables(B, Hkv, _hp(hc), _hp(goh), n_groups, _hp(ids),
+                                        _hp(table), _hp(off), _hp(goff)), "tg_build_group_tables")
     return table[:int(goff[-1])].copy(), off, goff
 
 

@@ -150,7 +150,8 @@ int alloc_share_segment(tg_alloc *a, int32_t n_tokens, int32_t n_heads, int32_t 
 }
 
 int alloc_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads, const int32_t *kv_len, int32_t n_prefix,
-                  const int32_t *prefix_segs, int32_t *page_ids, int64_t capacity, int64_t *n_written) {
+                  const int32_t *prefix_segs, int32_t *page_ids, int64_t capacity, int32_t *head_count,
+                  int64_t *n_written) {
     if (!a || n_heads < 1 || !kv_len || n_prefix < 0 || (n_prefix > 0 && !prefix_segs) ||
         (capacity > 0 && !page_ids) || capacity < 0)
         return TG_EINVAL;
@@ -203,6 +204,7 @@ int alloc_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads, const int32_t *k
             sq.priv.push_back(id);
             page_ids[w++] = id;
         }
+        if (head_count) head_count[h] = static_cast<int32_t>(shared_pages + priv);
     }
     if (n_written) *n_written = w;
     return TG_OK;
@@ -210,9 +212,34 @@ int alloc_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads, const int32_t *k
 
 }  // namespace
 
-extern "C" int tg_alloc_create(int64_t num_pages, int32_t page, const int32_t *free_order,
-                               tg_alloc **out) {
+extern "C" int tg_alloc_create_ordered(int64_t num_pages, int32_t page, const int32_t *free_order,
+                                       tg_alloc **out) {
     return tg::no_throw([&] { return alloc_create(num_pages, page, free_order, out); });
+}
+
+// SplitMix64 (Steele, Lea & Flood, "Fast splittable pseudorandom number generators", 2014):
+// the state advances by the golden-ratio increment and each output is the state's 64-bit
+// finaliser (two xor-shift-multiply rounds and a final xor-shift).
+static uint64_t splitmix64_next(uint64_t &state) {
+    uint64_t z = (state += 0x9E3779B97F4A7C15ULL);
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+    return z ^ (z >> 31);
+}
+
+extern "C" int tg_alloc_create(int64_t num_pages, int32_t page, uint64_t seed, tg_alloc **out) {
+    return tg::no_throw([&] {
+        if (!out || num_pages < 1 || num_pages > INT32_MAX || page < 1) return TG_EINVAL;
+        // Durstenfeld's in-place Fisher-Yates shuffle, the k-th swap drawing the k-th output.
+        std::vector<int32_t> order(static_cast<size_t>(num_pages));
+        for (int64_t i = 0; i < num_pages; ++i) order[static_cast<size_t>(i)] = static_cast<int32_t>(i);
+        uint64_t state = seed;
+        for (int64_t i = num_pages - 1; i >= 1; --i) {
+            const int64_t j = static_cast<int64_t>(splitmix64_next(state) % static_cast<uint64_t>(i + 1));
+            std::swap(order[static_cast<size_t>(i)], order[static_cast<size_t>(j)]);
+        }
+        return alloc_create(num_pages, page, order.data(), out);
+    });
 }
 
 extern "C" void tg_alloc_destroy(tg_alloc *a) { delete a; }
@@ -224,21 +251,21 @@ extern "C" int32_t tg_alloc_refcount(const tg_alloc *a, int32_t page_id) {
     return a->refs[page_id];
 }
 
-extern "C" int tg_alloc_share_segment(tg_alloc *a, int32_t n_tokens, int32_t n_heads,
-                                      int32_t *seg_id, int32_t *page_ids) {
+extern "C" int tg_share_segment(tg_alloc *a, int32_t n_tokens, int32_t n_heads, int32_t *seg_id,
+                                int32_t *page_ids) {
     return tg::no_throw([&] { return alloc_share_segment(a, n_tokens, n_heads, seg_id, page_ids); });
 }
 
-extern "C" int tg_alloc_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads,
-                                const int32_t *kv_len, int32_t n_prefix,
-                                const int32_t *prefix_segs, int32_t *page_ids, int64_t capacity,
-                                int64_t *n_written) {
+extern "C" int tg_reserve(tg_alloc *a, int32_t seq_id, int32_t n_heads, const int32_t *kv_len,
+                          int32_t n_prefix, const int32_t *prefix_segs, int32_t *page_ids,
+                          int64_t capacity, int32_t *head_count, int64_t *n_written) {
     return tg::no_throw([&] {
-        return alloc_reserve(a, seq_id, n_heads, kv_len, n_prefix, prefix_segs, page_ids, capacity, n_written);
+        return alloc_reserve(a, seq_id, n_heads, kv_len, n_prefix, prefix_segs, page_ids, capacity,
+                             head_count, n_written);
     });
 }
 
-extern "C" int tg_alloc_release(tg_alloc *a, int32_t seq_id) {
+extern "C" int tg_release(tg_alloc *a, int32_t seq_id) {
     if (!a) return TG_EINVAL;
     auto it = a->seqs.find(seq_id);
     if (it == a->seqs.end()) return TG_ENOTFOUND;
@@ -248,7 +275,7 @@ extern "C" int tg_alloc_release(tg_alloc *a, int32_t seq_id) {
     return TG_OK;
 }
 
-extern "C" int tg_alloc_release_segment(tg_alloc *a, int32_t seg_id) {
+extern "C" int tg_release_segment(tg_alloc *a, int32_t seg_id) {
     if (!a) return TG_EINVAL;
     if (seg_id < 0 || seg_id >= static_cast<int32_t>(a->segs.size()) || !a->segs[seg_id].alive)
         return TG_ENOTFOUND;
@@ -261,10 +288,10 @@ extern "C" int tg_alloc_release_segment(tg_alloc *a, int32_t seg_id) {
 // ------------------------------------------------------------------------------------------
 // Group page tables (Ragged Paging).
 // ------------------------------------------------------------------------------------------
-extern "C" int tg_group_tables(int32_t B, int32_t Hkv, const int32_t *head_count,
-                               const int32_t *group_of_head, int32_t n_groups,
-                               const int32_t *page_ids, int32_t *table, int64_t *head_off,
-                               int64_t *group_off) {
+extern "C" int tg_build_group_tables(int32_t B, int32_t Hkv, const int32_t *head_count,
+                                     const int32_t *group_of_head, int32_t n_groups,
+                                     const int32_t *page_ids, int32_t *table, int64_t *head_off,
+                                     int64_t *group_off) {
     return tg::no_throw([&] {
         if (B < 0 || Hkv < 1 || !head_count || !group_of_head || n_groups < 1 || !group_off)
             return TG_EINVAL;

@@ -14,8 +14,8 @@ from typing import Optional
 import numpy as np
 
 import synth
-from . import (make_shape, tg_alloc_create, tg_alloc_destroy, tg_alloc_reserve,
-               tg_alloc_share_segment, tg_budget_groups, tg_group_tables, tg_plan_create,
+from . import (make_shape, tg_alloc_create, tg_alloc_destroy, tg_alloc_free_pages, tg_reserve,
+               tg_share_segment, tg_budget_groups, tg_build_group_tables, tg_plan_create,
                tg_quantize_int4, tg_quantize_int8, tg_retained_lengths)
 
 
@@ -83,24 +83,43 @@ def groups(sp: synth.Spec, layer: int = 0):
     return tg_budget_groups(table[layer], sp.groups), sp.groups
 
 
-def _reserve(sp, num_pages, order, kv, segs=(), chain=None):
-    """Budget Reservation of every sequence (shared segments first; chain[b] lists the
-    segments sequence b extends). Returns page ids flat and the shared segments' pages."""
+def _reserve(sp, num_pages, seed, kv, segs=(), chain=None):
+    """Budget Reservation of every sequence from a pool the library shuffles with `seed`
+    (shared segments first; chain[b] lists the segments sequence b extends). Returns the page
+    ids flat, each head's page count int32[B, Hkv] and the shared segments' pages."""
     B, H = kv.shape
-    a = tg_alloc_create(num_pages, sp.page, order)
+    a = tg_alloc_create(num_pages, sp.page, seed)
     try:
         seg_ids, seg_pages = [], []
         for n_tok in segs:
-            sid, ids = tg_alloc_share_segment(a, int(n_tok), H, sp.page)
+            sid, ids = tg_share_segment(a, int(n_tok), H, sp.page)
             seg_ids.append(sid)
             seg_pages.append(ids.reshape(-1))
-        out = []
+        out, counts = [], np.zeros((B, H), np.int32)
         for b in range(B):
             pre = () if chain is None else [seg_ids[c] for c in chain[b]]
-            out.append(tg_alloc_reserve(a, b, kv[b], pre, sp.page))
+            ids, counts[b] = tg_reserve(a, b, kv[b], pre, sp.page, with_counts=True)
+            out.append(ids)
         ids = np.concatenate(out) if out else np.zeros(0, np.int32)
         sp_all = np.concatenate(seg_pages) if seg_pages else np.zeros(0, np.int32)
-        return ids.astype(np.int32), sp_all.astype(np.int32)
+        return ids.astype(np.int32), counts, sp_all.astype(np.int32)
+    finally:
+        tg_alloc_destroy(a)
+
+
+def _pages_used(sp, kv, segs=(), chain=None) -> int:
+    """Pages a reservation of these heads takes (each shared segment's pages once, then every
+    head's private pages), as the allocator counts them: its free pages before minus after, in
+    a pool with room for any reservation of these lengths."""
+    H = kv.shape[1]
+    room = int(kv.astype(np.int64).sum()) // sp.page + kv.size + H * sum(int(t) // sp.page for t in segs) + 1
+    a = tg_alloc_create(room, sp.page, 0)
+    try:
+        before = tg_alloc_free_pages(a)
+        seg_ids = [tg_share_segment(a, int(t), H, sp.page)[0] for t in segs]
+        for b in range(kv.shape[0]):
+            tg_reserve(a, b, kv[b], () if chain is None else [seg_ids[c] for c in chain[b]], sp.page)
+        return int(before - tg_alloc_free_pages(a))
     finally:
         tg_alloc_destroy(a)
 
@@ -117,25 +136,21 @@ def layout(sp: synth.Spec, layer: int = 0, seqs=None) -> Layout:
             doc = doc[seqs]
         chain = np.stack([np.zeros(B, np.int32), 1 + doc], axis=1)
     if fast is None:
-        # a head's pages: the full pages of its shared segments, then its private pages
-        shared_pages = (sp.sys_tokens // sp.page + sp.doc_tokens // sp.page) if segs else 0
-        private = pages_of(kv.astype(np.int64) - shared_pages * sp.page, sp.page)
-        count = (shared_pages + private).astype(np.int32)
-        used = int(private.sum()) + sum(H * (s // sp.page) for s in segs)
+        # the pool is sized from the pages the workload uses (its occupancy): the reservation
+        # is made once in a pool with room for every page, which gives the pages in use, then
+        # in the pool of the workload's size
+        used = _pages_used(sp, kv, segs, chain)
         num_pages = _occupied(sp, used)
-        order = synth.free_order(sp, num_pages, layer)
-        ids, segp = _reserve(sp, num_pages, order, kv, segs, chain)
-        table, off, goff = tg_group_tables(count, goh, G, ids)
+        ids, count, segp = _reserve(sp, num_pages, synth.free_order_seed(sp, layer), kv, segs, chain)
+        table, off, goff = tg_build_group_tables(count, goh, G, ids)
         return Layout(kv, None, goh, G, num_pages, ids, count, table, off, goff, seg_pages=segp)
     slow_n = kv - fast
-    fcount = pages_of(fast, sp.page).astype(np.int32)
-    scount = pages_of(slow_n, sp.page).astype(np.int32)
-    nf = _occupied(sp, int(fcount.sum()))
-    ns = _occupied(sp, int(scount.sum()))
-    fids, _ = _reserve(sp, nf, synth.free_order(sp, nf, layer), fast)
-    sids, _ = _reserve(sp, ns, synth.free_order(sp, ns, layer, slow=True), slow_n)
-    ft, foff, fgoff = tg_group_tables(fcount, goh, G, fids)
-    st, soff, sgoff = tg_group_tables(scount, np.zeros(H, np.int32), 1, sids)
+    nf = _occupied(sp, _pages_used(sp, fast))
+    ns = _occupied(sp, _pages_used(sp, slow_n))
+    fids, fcount, _ = _reserve(sp, nf, synth.free_order_seed(sp, layer), fast)
+    sids, scount, _ = _reserve(sp, ns, synth.free_order_seed(sp, layer, slow=True), slow_n)
+    ft, foff, fgoff = tg_build_group_tables(fcount, goh, G, fids)
+    st, soff, sgoff = tg_build_group_tables(scount, np.zeros(H, np.int32), 1, sids)
     return Layout(kv, fast, goh, G, nf, fids, fcount, ft, foff, fgoff, num_slow_pages=ns,
                   slow_ids=sids, slow_count=scount, slow_table=st, slow_off=soff)
 

@@ -62,6 +62,8 @@ def _L():
         build()
         lib = ctypes.CDLL(_LIB_PATH)
         u64, i64, p = ctypes.c_uint64, ctypes.c_int64, ctypes.c_void_p
+        lib.synth_stream_key.restype = u64
+        lib.synth_stream_key.argtypes = [u64, u64]
         lib.synth_draw.restype = u64
         lib.synth_draw.argtypes = [u64, u64, u64]
         lib.synth_draws.argtypes = [u64, u64, u64, i64, p]
@@ -71,6 +73,12 @@ def _L():
         lib.synth_permutation.argtypes = [u64, u64, i64, p]
         _lib = lib
     return _lib
+
+
+def stream_key(seed: int, stream: int) -> int:
+    """The SplitMix64 seed of a stream: its draw i is the (i+1)-th output of SplitMix64 seeded
+    with this value (so a consumer holding its own SplitMix64 can replay the stream)."""
+    return int(_L().synth_stream_key(seed, stream))
 
 
 def draws(seed: int, stream: int, n: int, i0: int = 0) -> np.ndarray:
@@ -275,6 +283,12 @@ def prefix_layout(sp: Spec):
 def free_order(sp: Spec, num_pages: int, layer: int = 0, slow: bool = False) -> np.ndarray:
     """Initial free-list order of a pool of num_pages pages (a seeded shuffle)."""
     return permutation(sp.seed, stream_id(S_FREE_SLOW if slow else S_FREE, layer), num_pages)
+
+
+def free_order_seed(sp: Spec, layer: int = 0, slow: bool = False) -> int:
+    """SplitMix64 seed of the free-order stream: an allocator that shuffles its pool itself
+    (Fisher-Yates driven by SplitMix64 from this seed) reproduces free_order."""
+    return stream_key(sp.seed, stream_id(S_FREE_SLOW if slow else S_FREE, layer))
 
 
 def q_bits(sp: Spec, layer: int = 0) -> np.ndarray:

@@ -27,6 +27,10 @@ static uint64_t stream_key(uint64_t seed, uint64_t stream) {
     return mix64(seed ^ mix64(stream * SYNTH_GAMMA + 0x632BE59BD9B4E019ULL));
 }
 
+/* The SplitMix64 state from which stream s of seed k starts: draw i of the stream is the
+ * (i+1)-th output of SplitMix64 seeded with this value. */
+uint64_t synth_stream_key(uint64_t seed, uint64_t stream) { return stream_key(seed, stream); }
+
 uint64_t synth_draw(uint64_t seed, uint64_t stream, uint64_t i) {
     return mix64(stream_key(seed, stream) + (i + 1) * SYNTH_GAMMA);
 }

@@ -113,11 +113,11 @@ static void admission_round() {
     for (int64_t i = 0; i < num_pages; ++i) order[i] = static_cast<int32_t>(i);
     std::shuffle(order.begin(), order.end(), rng);
     tg_alloc *a = nullptr;
-    CHECK(tg_alloc_create(num_pages, 16, order.data(), &a) == TG_OK);
+    CHECK(tg_alloc_create_ordered(num_pages, 16, order.data(), &a) == TG_OK);
     int32_t seg = -1;
     const int32_t seg_tokens = static_cast<int32_t>(uni(0, 600));
     std::vector<int32_t> seg_pages(static_cast<size_t>(Hkv) * (seg_tokens / 16) + 1);
-    CHECK(tg_alloc_share_segment(a, seg_tokens, Hkv, &seg, seg_pages.data()) == TG_OK);
+    CHECK(tg_share_segment(a, seg_tokens, Hkv, &seg, seg_pages.data()) == TG_OK);
     std::vector<int32_t> ids;
     std::vector<int32_t> head_count(BH);
     for (int32_t b = 0; b < B; ++b) {
@@ -129,7 +129,9 @@ static void admission_round() {
         for (int32_t x : kvb) cap += (x + 15) / 16;
         std::vector<int32_t> out(static_cast<size_t>(cap) + 1);
         int64_t written = -1;
-        const int rc = tg_alloc_reserve(a, b, Hkv, kvb.data(), prefixed ? 1 : 0, &seg, out.data(), cap, &written);
+        std::vector<int32_t> counts(static_cast<size_t>(Hkv), -1);
+        const int rc = tg_reserve(a, b, Hkv, kvb.data(), prefixed ? 1 : 0, &seg, out.data(), cap,
+                                  counts.data(), &written);
         CHECK(rc == TG_OK || rc == TG_ENOSPC);
         if (rc == TG_ENOSPC) {
             for (int32_t h = 0; h < Hkv; ++h) head_count[static_cast<int64_t>(b) * Hkv + h] = 0;
@@ -137,7 +139,8 @@ static void admission_round() {
         }
         CHECK(written == cap);
         for (int32_t h = 0; h < Hkv; ++h) {
-            head_count[static_cast<int64_t>(b) * Hkv + h] = (kvb[h] + 15) / 16;
+            CHECK(counts[h] == (kvb[h] + 15) / 16);  // the segment holds whole pages
+            head_count[static_cast<int64_t>(b) * Hkv + h] = counts[h];
             kv[static_cast<int64_t>(b) * Hkv + h] = kvb[h];
         }
         ids.insert(ids.end(), out.begin(), out.begin() + cap);
@@ -146,7 +149,7 @@ static void admission_round() {
     std::vector<int32_t> huge(Hkv, static_cast<int32_t>(16 * (num_pages + 1)));
     int64_t w2 = 0;
     std::vector<int32_t> sink(1);
-    CHECK(tg_alloc_reserve(a, 1000, Hkv, huge.data(), 0, nullptr, sink.data(), 0, &w2) != TG_OK);
+    CHECK(tg_reserve(a, 1000, Hkv, huge.data(), 0, nullptr, sink.data(), 0, nullptr, &w2) != TG_OK);
 
     // group tables over what was reserved
     std::vector<int64_t> goff(static_cast<size_t>(n_groups) + 1);
@@ -162,7 +165,7 @@ static void admission_round() {
     }
     std::vector<int32_t> table(static_cast<size_t>(tsize) + 1);
     std::vector<int64_t> hoff(BH);
-    CHECK(tg_group_tables(B, Hkv, head_count.data(), goh.data(), n_groups, ids.data(), table.data(), hoff.data(),
+    CHECK(tg_build_group_tables(B, Hkv, head_count.data(), goh.data(), n_groups, ids.data(), table.data(), hoff.data(),
                           goff.data()) == TG_OK);
 
     // plans: bf16 (static, hybrid, whole heads), tiered INT8 / INT4, cascade
@@ -243,8 +246,8 @@ static void admission_round() {
     }
 
     // release everything; every page returns to the free list
-    for (int32_t b = 0; b < B; ++b) tg_alloc_release(a, b);
-    CHECK(tg_alloc_release_segment(a, seg) == TG_OK);
+    for (int32_t b = 0; b < B; ++b) tg_release(a, b);
+    CHECK(tg_release_segment(a, seg) == TG_OK);
     CHECK(tg_alloc_free_pages(a) == num_pages);
     tg_alloc_destroy(a);
 
@@ -297,7 +300,12 @@ static void fault_round(long *runs) {
     const int64_t BH = static_cast<int64_t>(B) * Hkv;
     const int64_t num_pages = 300 + uni(0, 100);
     tg_alloc *a = nullptr;
-    CHECK(under_failures([&] { return tg_alloc_create(num_pages, 16, nullptr, &a); }, [&](int) { CHECK(!a); }, runs) ==
+    // the seeded form (it shuffles in a temporary order vector first), then the ordered form
+    CHECK(under_failures([&] { return tg_alloc_create(num_pages, 16, static_cast<uint64_t>(num_pages), &a); },
+                         [&](int) { CHECK(!a); }, runs) == TG_OK);
+    tg_alloc_destroy(a);
+    a = nullptr;
+    CHECK(under_failures([&] { return tg_alloc_create_ordered(num_pages, 16, nullptr, &a); }, [&](int) { CHECK(!a); }, runs) ==
           TG_OK);
     auto refs = [&] {
         std::vector<int32_t> r(static_cast<size_t>(num_pages));
@@ -315,7 +323,7 @@ static void fault_round(long *runs) {
     const int32_t seg_tokens = 64 + static_cast<int32_t>(uni(0, 15));
     int32_t seg = -1;
     std::vector<int32_t> seg_pages(static_cast<size_t>(Hkv) * 4);
-    CHECK(under_failures([&] { return tg_alloc_share_segment(a, seg_tokens, Hkv, &seg, seg_pages.data()); },
+    CHECK(under_failures([&] { return tg_share_segment(a, seg_tokens, Hkv, &seg, seg_pages.data()); },
                          [&](int) { CHECK(refs() == before && tg_alloc_free_pages(a) == free_before); }, runs) ==
           TG_OK);
     consistent();
@@ -331,10 +339,10 @@ static void fault_round(long *runs) {
         before = refs();
         free_before = tg_alloc_free_pages(a);
         CHECK(under_failures(
-                  [&] { return tg_alloc_reserve(a, b, Hkv, kvb.data(), 1, segs, out.data(), cap, &written); },
+                  [&] { return tg_reserve(a, b, Hkv, kvb.data(), 1, segs, out.data(), cap, nullptr, &written); },
                   [&](int) {
                       CHECK(refs() == before && tg_alloc_free_pages(a) == free_before);
-                      CHECK(tg_alloc_release(a, b) == TG_ENOTFOUND);
+                      CHECK(tg_release(a, b) == TG_ENOTFOUND);
                   },
                   runs) == TG_OK);
         CHECK(written == cap);
@@ -355,12 +363,12 @@ static void fault_round(long *runs) {
                          [&](int rc) { CHECK(rc != TG_OK || goh == goh_expect); }, runs) == TG_OK);
     CHECK(goh == goh_expect);
     std::vector<int64_t> goff(static_cast<size_t>(n_groups) + 1), hoff(static_cast<size_t>(BH));
-    CHECK(tg_group_tables(B, Hkv, head_count.data(), goh.data(), n_groups, ids.data(), nullptr, hoff.data(),
+    CHECK(tg_build_group_tables(B, Hkv, head_count.data(), goh.data(), n_groups, ids.data(), nullptr, hoff.data(),
                           goff.data()) == TG_OK);
     const int64_t tsize = goff[n_groups];
     std::vector<int32_t> table(static_cast<size_t>(tsize) + 1);
     CHECK(under_failures([&] {
-              return tg_group_tables(B, Hkv, head_count.data(), goh.data(), n_groups, ids.data(), table.data(),
+              return tg_build_group_tables(B, Hkv, head_count.data(), goh.data(), n_groups, ids.data(), table.data(),
                                      hoff.data(), goff.data());
           },
           [](int rc) { CHECK(rc == TG_ENOMEM); }, runs) == TG_OK);
@@ -419,8 +427,8 @@ static void fault_round(long *runs) {
         tg_plan_destroy(p);
     }
 
-    for (int32_t b = 0; b < B; ++b) CHECK(tg_alloc_release(a, b) == TG_OK);
-    CHECK(tg_alloc_release_segment(a, seg) == TG_OK);
+    for (int32_t b = 0; b < B; ++b) CHECK(tg_release(a, b) == TG_OK);
+    CHECK(tg_release_segment(a, seg) == TG_OK);
     CHECK(tg_alloc_free_pages(a) == num_pages);
     tg_alloc_destroy(a);
 }

@@ -32,17 +32,17 @@ def batches(draw):
 
 
 def _lib_layout(num_pages, order, kv, segs, chain, page):
-    a = tg.tg_alloc_create(num_pages, page, order)
+    a = tg.tg_alloc_create_ordered(num_pages, page, order)
     try:
         seg_ids, seg_pages = [], []
         for s in segs:
-            sid, ids = tg.tg_alloc_share_segment(a, s, kv.shape[1], page)
+            sid, ids = tg.tg_share_segment(a, s, kv.shape[1], page)
             seg_ids.append(sid)
             seg_pages.append(ids.reshape(-1))
         out = []
         for b in range(kv.shape[0]):
             pre = [seg_ids[c] if c >= 0 else -1 for c in chain[b]]
-            out.append(tg.tg_alloc_reserve(a, b, kv[b], pre, page))
+            out.append(tg.tg_reserve(a, b, kv[b], pre, page))
         free_left = tg.tg_alloc_free_pages(a)
         return (np.concatenate(out) if out else np.zeros(0, np.int32),
                 np.concatenate(seg_pages) if seg_pages else np.zeros(0, np.int32), free_left)
@@ -73,12 +73,12 @@ def test_pool_one_page_short_is_refused_without_taking_pages(case):
         return
     num_pages = exact - 1
     order = np.random.default_rng(seed).permutation(num_pages).astype(np.int32)
-    a = tg.tg_alloc_create(num_pages, page, order)
+    a = tg.tg_alloc_create_ordered(num_pages, page, order)
     try:
         seg_ids = []
         for s in segs:
             try:
-                sid, _ = tg.tg_alloc_share_segment(a, s, kv.shape[1], page)
+                sid, _ = tg.tg_share_segment(a, s, kv.shape[1], page)
             except tg.TGError as e:
                 assert e.status == tg.TG_ENOSPC
                 return                                   # the segments alone do not fit
@@ -88,7 +88,7 @@ def test_pool_one_page_short_is_refused_without_taking_pages(case):
             before = tg.tg_alloc_free_pages(a)
             pre = [seg_ids[c] if c >= 0 else -1 for c in chain[b]]
             try:
-                tg.tg_alloc_reserve(a, b, kv[b], pre, page)
+                tg.tg_reserve(a, b, kv[b], pre, page)
             except tg.TGError as e:
                 assert e.status == tg.TG_ENOSPC
                 assert tg.tg_alloc_free_pages(a) == before   # nothing taken
@@ -108,7 +108,7 @@ def test_group_tables_equal_oracle(B, H, G, max_pages, seed):
     cnt = rng.integers(0, max_pages + 1, (B, H)).astype(np.int32)
     goh = rng.integers(0, G, H).astype(np.int32)
     ids = rng.permutation(int(cnt.sum()) + 2)[: int(cnt.sum())].astype(np.int32)
-    t, off, goff = tg.tg_group_tables(cnt, goh, G, ids)
+    t, off, goff = tg.tg_build_group_tables(cnt, goh, G, ids)
     ot, ooff, ogoff = oracle.group_tables(goh, G, ids, cnt)
     np.testing.assert_array_equal(t, ot)
     np.testing.assert_array_equal(goff, ogoff)

@@ -28,6 +28,29 @@ def test_library_exports_every_declared_symbol():
     assert declared == set(tg.ABI_SYMBOLS), declared ^ set(tg.ABI_SYMBOLS)
 
 
+# The calls the hot path's boundary names (the scope table's C-ABI sketch), by name.
+BOUNDARY_CALLS = ("tg_alloc_create", "tg_reserve", "tg_share_segment", "tg_release",
+                  "tg_alloc_destroy", "tg_build_group_tables", "tg_plan_create",
+                  "tg_ragged_paged_decode", "tg_tiered_decode", "tg_plan_destroy", "tg_strerror")
+
+
+def test_boundary_calls_are_exported_under_their_names():
+    hdr = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "tg.h")).read(), flags=re.S)
+    lib = tg.load()
+    for name in BOUNDARY_CALLS:
+        assert re.search(r"\b%s\s*\(" % name, hdr), f"tg.h does not declare {name}"
+        assert hasattr(lib, name), f"libtg.so does not export {name}"
+    # and the host ones run through the C ABI here (the device ones need a GPU)
+    a = tg.tg_alloc_create(64, 16, 9)
+    sid, _ = tg.tg_share_segment(a, 32, 2, 16)
+    ids, counts = tg.tg_reserve(a, 0, [40, 33], (sid,), 16, with_counts=True)
+    table, off, goff = tg.tg_build_group_tables(counts.reshape(1, 2), [0, 0], 1, ids)
+    assert table.tolist() == ids.tolist() and counts.tolist() == [3, 3]
+    tg.tg_release(a, 0)
+    tg.tg_alloc_destroy(a)
+    assert tg.load().tg_strerror(0).decode() == "ok"
+
+
 def test_strerror_covers_codes():
     for code in range(10):
         assert tg.load().tg_strerror(code).decode() != "unknown status"
@@ -52,18 +75,18 @@ def test_budget_groups_match_oracle():
 
 
 def _lib_reservation(num_pages, order, kv, segs=(), chain=None, page=16):
-    a = tg.tg_alloc_create(num_pages, page, order)
+    a = tg.tg_alloc_create_ordered(num_pages, page, order)
     try:
         seg_ids = []
         seg_pages = []
         for s in segs:
-            sid, ids = tg.tg_alloc_share_segment(a, s, kv.shape[1], page)
+            sid, ids = tg.tg_share_segment(a, s, kv.shape[1], page)
             seg_ids.append(sid)
             seg_pages.append(ids.reshape(-1))
         out = []
         for b in range(kv.shape[0]):
             pre = [] if chain is None else [seg_ids[c] if c >= 0 else -1 for c in chain[b]]
-            out.append(tg.tg_alloc_reserve(a, b, kv[b], pre, page))
+            out.append(tg.tg_reserve(a, b, kv[b], pre, page))
         return np.concatenate(out), (np.concatenate(seg_pages) if seg_pages else np.zeros(0, np.int32))
     finally:
         tg.tg_alloc_destroy(a)
@@ -90,21 +113,21 @@ def test_reservation_matches_oracle_plain_and_prefix():
 
 
 def test_reservation_is_all_or_nothing():
-    a = tg.tg_alloc_create(10, 16, np.arange(10)[::-1])
+    a = tg.tg_alloc_create_ordered(10, 16, np.arange(10)[::-1])
     try:
-        tg.tg_alloc_reserve(a, 0, [40, 16])                       # 3 + 1 pages
+        tg.tg_reserve(a, 0, [40, 16])                       # 3 + 1 pages
         assert tg.tg_alloc_free_pages(a) == 6
         with pytest.raises(tg.TGError) as e:
-            tg.tg_alloc_reserve(a, 1, [64, 64])                   # needs 8 > 6
+            tg.tg_reserve(a, 1, [64, 64])                   # needs 8 > 6
         assert e.value.status == tg.TG_ENOSPC
         assert tg.tg_alloc_free_pages(a) == 6                     # unchanged
-        ids = tg.tg_alloc_reserve(a, 1, [32, 1])                  # same as if no failure
+        ids = tg.tg_reserve(a, 1, [32, 1])                  # same as if no failure
         np.testing.assert_array_equal(ids, [5, 4, 3])
         with pytest.raises(tg.TGError) as e:
-            tg.tg_alloc_reserve(a, 1, [1])
+            tg.tg_reserve(a, 1, [1])
         assert e.value.status == tg.TG_EEXIST
         with pytest.raises(tg.TGError) as e:
-            tg.tg_alloc_release(a, 7)
+            tg.tg_release(a, 7)
         assert e.value.status == tg.TG_ENOTFOUND
     finally:
         tg.tg_alloc_destroy(a)
@@ -112,36 +135,36 @@ def test_reservation_is_all_or_nothing():
 
 def test_free_order_must_be_a_permutation():
     with pytest.raises(tg.TGError):
-        tg.tg_alloc_create(4, 16, [0, 1, 1, 2])
+        tg.tg_alloc_create_ordered(4, 16, [0, 1, 1, 2])
     with pytest.raises(tg.TGError):
-        tg.tg_alloc_create(3, 16, [0, 1, 3])
+        tg.tg_alloc_create_ordered(3, 16, [0, 1, 3])
 
 
 def test_shared_segment_refcounts_and_release_order():
-    a = tg.tg_alloc_create(40, 16)
+    a = tg.tg_alloc_create_ordered(40, 16)
     try:
-        sid, sp = tg.tg_alloc_share_segment(a, 40, 2, 16)         # 2 full pages per head
+        sid, sp = tg.tg_share_segment(a, 40, 2, 16)         # 2 full pages per head
         np.testing.assert_array_equal(sp, [[0, 1], [2, 3]])
-        r0 = tg.tg_alloc_reserve(a, 0, [50, 33], [sid])          # shared 32 tokens
-        r1 = tg.tg_alloc_reserve(a, 1, [32, 40], [sid])
+        r0 = tg.tg_reserve(a, 0, [50, 33], [sid])          # shared 32 tokens
+        r1 = tg.tg_reserve(a, 1, [32, 40], [sid])
         np.testing.assert_array_equal(r0, [0, 1, 4, 5, 2, 3, 6])
         np.testing.assert_array_equal(r1, [0, 1, 2, 3, 7])
         for p in (0, 1, 2, 3):
             assert tg.tg_alloc_refcount(a, p) == 3                # segment + 2 readers
         assert tg.tg_alloc_refcount(a, 4) == 1
-        tg.tg_alloc_release(a, 0)
+        tg.tg_release(a, 0)
         assert tg.tg_alloc_refcount(a, 0) == 2 and tg.tg_alloc_refcount(a, 4) == 0
         free_before = tg.tg_alloc_free_pages(a)
-        tg.tg_alloc_release_segment(a, sid)
+        tg.tg_release_segment(a, sid)
         assert tg.tg_alloc_free_pages(a) == free_before           # reader 1 still holds them
-        tg.tg_alloc_release(a, 1)
+        tg.tg_release(a, 1)
         assert all(tg.tg_alloc_refcount(a, p) == 0 for p in range(8))
         assert tg.tg_alloc_free_pages(a) == 40
         # released pages are appended at the back, in release order: the front is unchanged
-        ids = tg.tg_alloc_reserve(a, 2, [16])
+        ids = tg.tg_reserve(a, 2, [16])
         np.testing.assert_array_equal(ids, [8])
         with pytest.raises(tg.TGError):
-            tg.tg_alloc_reserve(a, 3, [16], [sid])               # dead segment
+            tg.tg_reserve(a, 3, [16], [sid])               # dead segment
     finally:
         tg.tg_alloc_destroy(a)
 
@@ -152,7 +175,7 @@ def test_group_tables_match_oracle():
         cnt = rng.integers(0, 9, (B, H)).astype(np.int32)
         goh = rng.integers(0, G, H).astype(np.int32)
         ids = rng.permutation(int(cnt.sum()) + 3)[: int(cnt.sum())].astype(np.int32)
-        t, off, goff = tg.tg_group_tables(cnt, goh, G, ids)
+        t, off, goff = tg.tg_build_group_tables(cnt, goh, G, ids)
         ot, ooff, ogoff = oracle.group_tables(goh, G, ids, cnt)
         np.testing.assert_array_equal(t, ot)
         np.testing.assert_array_equal(goff, ogoff)
@@ -518,29 +541,29 @@ def test_binding_checks_host_array_sizes():
     with pytest.raises(ValueError):
         tg.tg_plan_create_cascade(shape, kv, goh, goff, table, np.zeros(3, np.int64), **ok)
     with pytest.raises(ValueError):
-        tg.tg_alloc_create(10, 16, np.arange(9))
+        tg.tg_alloc_create_ordered(10, 16, np.arange(9))
     cnt = np.array([[2, 1], [0, 3]], np.int32)
     with pytest.raises(ValueError):
-        tg.tg_group_tables(cnt, np.zeros(3, np.int32), 1, np.arange(6))
+        tg.tg_build_group_tables(cnt, np.zeros(3, np.int32), 1, np.arange(6))
     with pytest.raises(ValueError):
-        tg.tg_group_tables(cnt, np.zeros(2, np.int32), 1, np.arange(5))   # 6 page ids needed
-    t, off, g = tg.tg_group_tables(cnt, np.zeros(2, np.int32), 1, np.arange(6))
+        tg.tg_build_group_tables(cnt, np.zeros(2, np.int32), 1, np.arange(5))   # 6 page ids needed
+    t, off, g = tg.tg_build_group_tables(cnt, np.zeros(2, np.int32), 1, np.arange(6))
     assert g[-1] == 2 * 2 * 3
 
 
 def test_allocator_outputs_sized_with_its_own_page():
     """The binding sizes segment and reservation outputs with the allocator's page (a larger
     page argument would under-size them); a page argument that disagrees is refused."""
-    a = tg.tg_alloc_create(64, 8)
+    a = tg.tg_alloc_create_ordered(64, 8)
     try:
-        sid, ids = tg.tg_alloc_share_segment(a, 40, 2)               # 5 full 8-token pages per head
+        sid, ids = tg.tg_share_segment(a, 40, 2)               # 5 full 8-token pages per head
         assert ids.shape == (2, 5) and len(np.unique(ids)) == 10
         with pytest.raises(ValueError):
-            tg.tg_alloc_share_segment(a, 40, 2, 16)
-        r = tg.tg_alloc_reserve(a, 0, [41, 40], [sid])               # 40 shared + 1 private token
+            tg.tg_share_segment(a, 40, 2, 16)
+        r = tg.tg_reserve(a, 0, [41, 40], [sid])               # 40 shared + 1 private token
         assert r.size == 5 + 1 + 5 and tg.tg_alloc_free_pages(a) == 64 - 10 - 1
         with pytest.raises(ValueError):
-            tg.tg_alloc_reserve(a, 1, [8], (), 16)
+            tg.tg_reserve(a, 1, [8], (), 16)
     finally:
         tg.tg_alloc_destroy(a)
 

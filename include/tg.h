@@ -208,9 +208,15 @@ typedef struct tg_plan_opts {
                                  as tg_quantize_int4 writes them, passed where the INT8 calls
                                  take k_q8 / v_q8 */
     int32_t whole_heads;      /* bf16 plans without a cascade: 1 = every head is one item (no
-                                 split heads, so no partials and no merge kernel), whole heads
-                                 placed on up to num_workers workers longest first; for small
-                                 batches, where a step is launch-bound. Ignored for tiered and
+                                 split heads, so no partials and no merge kernel), for small
+                                 batches, where a step is launch-bound. When no head holds more
+                                 than 64 pages the plan runs the lean kernel: one CTA per
+                                 (sequence, KV head) reading its pages with plain 16-byte loads
+                                 (no copy pipeline, no tensor map, no shared-memory ring), fp32
+                                 scores and probabilities, one launch per call (the H2O scores
+                                 call keeps the pipelined kernel; the lean kernel records no
+                                 worker timeline). Otherwise whole heads are placed on up to
+                                 num_workers workers longest first. Ignored for tiered and
                                  cascade plans; static_permille, min_splits and max_chunk_pages
                                  do not apply */
 } tg_plan_opts;

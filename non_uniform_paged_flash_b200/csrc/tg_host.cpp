@@ -802,6 +802,14 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
             for (int32_t r = 0; r < u.n_readers; ++r)
                 u.slot[r] = next[static_cast<int64_t>(u.reader[r]) * s.Hkv + u.h]++;
     }
+    // Whole-head bf16 plans whose longest head holds at most kLeanMaxPages pages run the lean
+    // kernel (one CTA per (sequence, KV head), no copy pipeline to set up): a tiny batch's step
+    // is one launch's latency, not bandwidth.
+    if (p->whole_heads && !p->tiered && p->cunits.empty()) {
+        int64_t most = 0;
+        for (const tg::Item &it : p->items) most = std::max<int64_t>(most, it.page_end - it.page_begin);
+        p->lean = most <= tg::kLeanMaxPages;
+    }
     p->grid = (p->n_workers + p->pairs - 1) / p->pairs;
     if (p->n_dyn > 0 && p->grid == 0) p->grid = 1;
     if (p->grid == 0 && !p->empties.empty()) p->grid = 1;  // the kernel also writes empty heads
@@ -855,10 +863,10 @@ extern "C" int tg_plan_get_info(const tg_plan *p, tg_plan_info *info) {
     info->n_empty = static_cast<int64_t>(p->empties.size());
     info->n_dynamic = p->n_dyn;
     info->n_workers = p->n_workers;
-    info->grid = p->grid;
-    info->block = p->pairs * 64;
-    info->smem_bytes = p->smem_bytes;
-    info->stages = p->stages;
+    info->grid = p->lean ? static_cast<int32_t>(static_cast<int64_t>(p->shape.B) * p->shape.Hkv) : p->grid;
+    info->block = p->lean ? tg::kLeanWarps * 32 : p->pairs * 64;
+    info->smem_bytes = p->lean ? 0 : p->smem_bytes;
+    info->stages = p->lean ? 0 : p->stages;
     info->device_bytes = p->dev_bytes;
     info->kv_bytes = p->kv_bytes;
     info->n_cascade = static_cast<int32_t>(p->cunits.size());

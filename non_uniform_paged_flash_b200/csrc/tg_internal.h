@@ -77,6 +77,11 @@ constexpr int kPairs = 4;              // bf16 decode kernel
 constexpr int kPairsTiered = 6;        // tiered decode kernel (12 warps; 4 ring stages at D = 128)
 constexpr int kThreads = kPairs * 64;  // threads per CTA of the bf16 decode kernel
 constexpr int kTraceWords = 8;         // worker timeline words (see tg_plan_trace_enable)
+// Lean decode kernel (whole-head bf16 plans of short heads: tiny batches where a step is one
+// launch's latency): one CTA of kLeanWarps warps per (sequence, KV head), for heads of at most
+// kLeanMaxPages pages.
+constexpr int kLeanWarps = 8;
+constexpr int kLeanMaxPages = 64;
 
 }  // namespace tg
 
@@ -112,6 +117,7 @@ struct tg_plan {
     bool out_f32 = false;             // see tg_plan_opts.out_f32
     int32_t slow_bits = 8;            // see tg_plan_opts.slow_bits
     bool whole_heads = false;         // see tg_plan_opts.whole_heads
+    bool lean = false;                // whole-head plan run by the lean kernel (short heads)
     int32_t n_workers = 0;
     int64_t kv_bytes = 0;
 
@@ -133,6 +139,7 @@ struct tg_plan {
     int32_t *d_empties = nullptr;   // [n_empty]
     uint32_t *d_dyn = nullptr;      // [2] dynamic ticket, producers done
     tg::CascadeUnit *d_cunits = nullptr;
+    int32_t *d_planned = nullptr;   // [B*Hkv] planned lengths (lean plans)
     uint32_t *d_err = nullptr;
 
     // kernel timing: 2 events per recorded call (cudaEvent_t stored as void*)

@@ -93,6 +93,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test: has the phase of the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase of the given parity; false after `limit` ns.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -608,6 +621,8 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
 // ------------------------------------------------------------------------------------------
 // Decode kernel
 // ------------------------------------------------------------------------------------------
+constexpr int kIssueLanes = 8;  // most pages one producer batch issues (lane l: page k + l)
+
 template <int D, bool TIERED, int NPAIRS, int SB = 8>
 __global__ void __launch_bounds__(NPAIRS * 64, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
@@ -787,13 +802,14 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                 const bool slow = TIERED && (fl & kItemSlow);
                 const int32_t b = bh / a.Hkv, h = bh - b * a.Hkv;
                 const int32_t cnt = min(32, pe - p0);
-                for (int32_t k = 0; k < cnt; ++k) {
-                    int32_t page_id = __shfl_sync(FULL, ids, k);
-                    const int32_t pg = p0 + k;
-                    const int stage = pstage;
-                    const uint32_t phase = pphase;
+                // Pages are issued in batches: the first free stage is waited for, the stages
+                // after it that the consumer has already released (it releases a page pair at
+                // once) are tested without waiting, and lane l issues page k + l of the block
+                // into stage pstage + l, so the copies of up to kIssueLanes pages are issued
+                // side by side instead of one after another from one lane.
+                for (int32_t k = 0; k < cnt;) {
                     wait_predecessor();
-                    const bool ok = dev::mbar_wait(empty0 + 8 * stage, phase ^ 1u, a.wait_ns);
+                    const bool ok = dev::mbar_wait(empty0 + 8 * pstage, pphase ^ 1u, a.wait_ns);
                     if (!ok || ctl[1]) {
                         if (lane == 0) {
                             atomicOr(a.err, kErrTimeout);
@@ -802,7 +818,21 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         aborted = true;
                         return;
                     }
-                    if (lane == 0) {
+                    const int nmax = min(cnt - k, min(stages, kIssueLanes));
+                    int stage = pstage + lane;
+                    uint32_t phase = pphase;
+                    if (stage >= stages) {
+                        stage -= stages;
+                        phase ^= 1u;
+                    }
+                    const bool is_free = lane == 0 ||
+                                         (lane < nmax && dev::mbar_test(empty0 + 8 * stage, phase ^ 1u));
+                    const uint32_t freed = __ballot_sync(FULL, is_free);
+                    const int n = __ffs(~freed) - 1;  // released stages from pstage on, <= nmax
+                    int32_t page_id = __shfl_sync(FULL, ids, (k + lane) & 31);
+                    if (lane < n) {
+                        const int32_t pg = p0 + k + lane;
+                        const uint32_t sq = seq + static_cast<uint32_t>(lane);
                         const int32_t vtok = max(0, min(16, tt - pg * 16));
                         if (vtok == 0) {
                             page_id = kNoLoad;  // a reserved page holding no token yet
@@ -829,7 +859,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         const uint32_t qbytes = static_cast<uint32_t>(a.G * D * 2);
                         uint32_t bytes = first ? qbytes : 0u;
                         if (page_id >= 0) bytes += slow ? 2u * ((SB == 4 ? L::kI4 : L::kI8) + 64u) : 2u * L::KB;
-                        if (a.withhold && worker == 0 && seq + 1 == static_cast<uint32_t>(a.withhold)) {
+                        if (a.withhold && worker == 0 && sq + 1 == static_cast<uint32_t>(a.withhold)) {
                             // testing: this stage is never signalled; the consumer's bounded
                             // wait runs out and the call reports a timeout
                         } else if (bytes == 0) {
@@ -861,15 +891,17 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                                 }
                             }
                         }
-                        ctl[0] = static_cast<int32_t>(seq + 1);
-                        if (trace && seq == 0) trace[1] = dev::global_timer();
+                        if (trace && sq == 0) trace[1] = dev::global_timer();
                     }
                     __syncwarp();
-                    ++seq;
-                    if (++pstage == stages) {
-                        pstage = 0;
+                    if (lane == 0) ctl[0] = static_cast<int32_t>(seq + static_cast<uint32_t>(n));
+                    seq += static_cast<uint32_t>(n);
+                    pstage += n;
+                    if (pstage >= stages) {
+                        pstage -= stages;
                         pphase ^= 1u;
                     }
+                    k += n;
                 }
                 j = jn;
                 p0 = pn;
@@ -1649,6 +1681,245 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------
+// Lean decode kernel: whole-head plans of short heads (a tiny batch, where a step is the latency
+// of one launch and a few dependent memory reads, not bandwidth). CTA i < B*Hkv handles
+// (sequence, KV head) i with all its G query heads; no copy pipeline, tensor map or
+// shared-memory ring to set up, so the critical path is: lengths and row offset, page ids,
+// K/V rows (all of a chunk's loads in flight at once), arithmetic, one merge through shared
+// memory, the output.
+//   Lanes: a token row of D bf16 is D/8 16-byte slices; LPT = D/8 lanes hold one token (lane
+//   sub = lane % LPT has dims [8 sub, 8 sub + 8)), so a warp covers TPW = 32/LPT tokens per
+//   round; R rounds per chunk (fewer for larger G: the per-lane state grows with G).
+//   Scores: fp32 dot products of the 8-dim slices summed over the LPT lanes by xor-shuffles,
+//   in log2 units; each lane keeps its own running max, sum and output slice over its tokens
+//   (the online-normaliser identity), rescaled once per chunk.
+//   Merge: the TPW token groups of a warp by xor-shuffles, then the warps through shared memory
+//   (fixed order, so results are deterministic); out = O / L, lse = ln 2 (M + log2 L).
+// ------------------------------------------------------------------------------------------
+struct LeanArgs {
+    int32_t Hq, Hkv;
+    float scale_log2;
+    const __nv_bfloat16 *q;
+    const __nv_bfloat16 *k_pages, *v_pages;
+    const int32_t *table;
+    const int64_t *head_off;
+    const int32_t *group_of_head;
+    const int64_t *group_off;
+    int32_t n_groups;
+    const int32_t *kv_len_dev;
+    const int32_t *planned;          // [B*Hkv] the plan's lengths
+    int64_t num_pages;
+    __nv_bfloat16 *out;
+    float *out_f32;
+    float *lse;
+    uint32_t *err;
+    int32_t early_prologue;
+};
+
+template <int D, int G>
+__global__ void __launch_bounds__(kLeanWarps * 32) lean_decode_kernel(const __grid_constant__ LeanArgs a) {
+    constexpr int LPT = D / 8;
+    constexpr int TPW = 32 / LPT;
+    constexpr int R = G <= 2 ? 8 : (G == 4 ? 4 : 2);
+    constexpr int CHUNK = kLeanWarps * TPW * R;
+    constexpr unsigned FULL = 0xffffffffu;
+    __shared__ float red_o[kLeanWarps][G][D];
+    __shared__ float red_m[kLeanWarps][G];
+    __shared__ float red_l[kLeanWarps][G];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane % LPT, tig = lane / LPT;
+    const int32_t bh = blockIdx.x;
+    const int32_t b = bh / a.Hkv, h = bh - b * a.Hkv;
+
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (!a.early_prologue) asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    // Metadata: planned and current length, row offset, the row's bounds in its group table.
+    const int32_t n = a.planned[bh];
+    const int32_t n_dev = a.kv_len_dev[bh];
+    const int64_t row = a.head_off[bh];
+    int64_t lo = a.group_off[0], hi = a.group_off[a.n_groups];
+    if (a.group_of_head) {
+        const int32_t g = a.group_of_head[h];
+        if (g >= 0 && g < a.n_groups) {
+            lo = a.group_off[g];
+            hi = a.group_off[g + 1];
+        } else {
+            hi = lo - 1;
+        }
+    }
+    const int32_t npages = (n + 15) >> 4;
+    const bool row_ok = n == 0 || (row >= lo && row + npages <= hi);
+    if (threadIdx.x == 0) {
+        if (n_dev != n) atomicOr(a.err, kErrPlan);
+        if (!row_ok) atomicOr(a.err, kErrBadRow);
+    }
+    const int32_t n_eff = row_ok ? n : 0;
+
+    // Page ids of this lane's tokens of the first chunk (before the predecessor's wait: tables
+    // only; queries and K/V after it).
+    auto token_of = [&](int32_t c0, int r) { return c0 + (r * kLeanWarps + warp) * TPW + tig; };
+    int32_t pid[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int32_t t = token_of(0, r);
+        pid[r] = t < n_eff ? __ldg(a.table + row + (t >> 4)) : -1;
+    }
+    if (a.early_prologue) asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    float qf[G][8];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
+            a.q + (static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * G + g) * D + 8 * sub));
+        qf[g][0] = dev::bf16_lo(v.x); qf[g][1] = dev::bf16_hi(v.x);
+        qf[g][2] = dev::bf16_lo(v.y); qf[g][3] = dev::bf16_hi(v.y);
+        qf[g][4] = dev::bf16_lo(v.z); qf[g][5] = dev::bf16_hi(v.z);
+        qf[g][6] = dev::bf16_lo(v.w); qf[g][7] = dev::bf16_hi(v.w);
+    }
+    float m[G], l[G], o[G][8];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        m[g] = -INFINITY;
+        l[g] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[g][i] = 0.f;
+    }
+
+    for (int32_t c0 = 0; c0 < n_eff; c0 += CHUNK) {
+        if (c0 > 0) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int32_t t = token_of(c0, r);
+                pid[r] = t < n_eff ? __ldg(a.table + row + (t >> 4)) : -1;
+            }
+        }
+        // every K and V slice of the chunk in flight before any arithmetic
+        uint4 kr[R], vr[R];
+        bool valid[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int32_t t = token_of(c0, r);
+            valid[r] = false;
+            kr[r] = make_uint4(0u, 0u, 0u, 0u);
+            vr[r] = kr[r];
+            if (t < n_eff) {
+                if (pid[r] < 0 || pid[r] >= a.num_pages) {
+                    if (sub == 0) atomicOr(a.err, kErrBadPage);  // skipped, never read
+                } else {
+                    const int64_t off = (static_cast<int64_t>(pid[r]) * 16 + (t & 15)) * D + 8 * sub;
+                    kr[r] = __ldg(reinterpret_cast<const uint4 *>(a.k_pages + off));
+                    vr[r] = __ldg(reinterpret_cast<const uint4 *>(a.v_pages + off));
+                    valid[r] = true;
+                }
+            }
+        }
+        float sc[R][G];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            float kf[8];
+            kf[0] = dev::bf16_lo(kr[r].x); kf[1] = dev::bf16_hi(kr[r].x);
+            kf[2] = dev::bf16_lo(kr[r].y); kf[3] = dev::bf16_hi(kr[r].y);
+            kf[4] = dev::bf16_lo(kr[r].z); kf[5] = dev::bf16_hi(kr[r].z);
+            kf[6] = dev::bf16_lo(kr[r].w); kf[7] = dev::bf16_hi(kr[r].w);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float acc = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc = fmaf(qf[g][i], kf[i], acc);
+#pragma unroll
+                for (int off = 1; off < LPT; off <<= 1) acc += __shfl_xor_sync(FULL, acc, off);
+                sc[r][g] = valid[r] ? acc * a.scale_log2 : -INFINITY;
+            }
+        }
+        // one rescale per chunk and head
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float mc = m[g];
+#pragma unroll
+            for (int r = 0; r < R; ++r) mc = fmaxf(mc, sc[r][g]);
+            if (mc > m[g]) {
+                const float al = m[g] == -INFINITY ? 0.f : dev::ex2(m[g] - mc);
+                l[g] *= al;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) o[g][i] *= al;
+                m[g] = mc;
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            float vf[8];
+            vf[0] = dev::bf16_lo(vr[r].x); vf[1] = dev::bf16_hi(vr[r].x);
+            vf[2] = dev::bf16_lo(vr[r].y); vf[3] = dev::bf16_hi(vr[r].y);
+            vf[4] = dev::bf16_lo(vr[r].z); vf[5] = dev::bf16_hi(vr[r].z);
+            vf[6] = dev::bf16_lo(vr[r].w); vf[7] = dev::bf16_hi(vr[r].w);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float pr = valid[r] ? dev::ex2(sc[r][g] - m[g]) : 0.f;
+                l[g] += pr;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) o[g][i] = fmaf(pr, vf[i], o[g][i]);
+            }
+        }
+    }
+
+    // Merge the warp's token groups (lanes that hold the same dims), then the warps.
+#pragma unroll
+    for (int off = LPT; off < 32; off <<= 1) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float mo = __shfl_xor_sync(FULL, m[g], off);
+            const float lo2 = __shfl_xor_sync(FULL, l[g], off);
+            const float M = fmaxf(m[g], mo);
+            const float fa = m[g] == -INFINITY ? 0.f : dev::ex2(m[g] - M);
+            const float fb = mo == -INFINITY ? 0.f : dev::ex2(mo - M);
+            l[g] = l[g] * fa + lo2 * fb;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[g][i] = o[g][i] * fa + __shfl_xor_sync(FULL, o[g][i], off) * fb;
+            m[g] = M;
+        }
+    }
+    if (tig == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) red_o[warp][g][8 * sub + i] = o[g][i];
+            if (sub == 0) {
+                red_m[warp][g] = m[g];
+                red_l[warp][g] = l[g];
+            }
+        }
+    }
+    __syncthreads();
+    constexpr float kLn2 = 0.69314718055994530942f;
+    const int64_t obase = (static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * G) * D;
+    for (int idx = threadIdx.x; idx < G * D; idx += kLeanWarps * 32) {
+        const int g = idx / D, d = idx - g * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kLeanWarps; ++w) M = fmaxf(M, red_m[w][g]);
+        float L = 0.f, O = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kLeanWarps; ++w) {
+                const float f = red_m[w][g] == -INFINITY ? 0.f : dev::ex2(red_m[w][g] - M);
+                L = fmaf(red_l[w][g], f, L);
+                O = fmaf(red_o[w][g][d], f, O);
+            }
+        }
+        const float val = L > 0.f ? O / L : 0.f;
+        if (a.out_f32)
+            a.out_f32[obase + idx] = val;
+        else
+            a.out[obase + idx] = __float2bfloat16_rn(val);
+        if (d == 0)
+            a.lse[static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * G + g] =
+                L > 0.f ? (M + dev::lg2(L)) * kLn2 : -INFINITY;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
 // Merge of split heads (log-sum-exp): one CTA per (split head, query row). Warp w owns the
 // contiguous splits [w*k, (w+1)*k); it loads them 4 at a time (all loads in flight), keeps a
 // running maximum and sum, and the warps' results are combined through shared memory in warp
@@ -1958,7 +2229,8 @@ int device_init_plan(tg_plan *p) {
     const int64_t b_emp = al(static_cast<int64_t>(p->empties.size()) * 4LL);
     const int64_t b_err = 256;  // error word + dynamic ticket counters
     const int64_t b_cu = al(static_cast<int64_t>(p->cunits.size()) * static_cast<int64_t>(sizeof(CascadeUnit)));
-    p->dev_bytes = b_items + b_woff + b_merge + b_goff + b_po + b_pl + b_emp + b_err + b_cu;
+    const int64_t b_plan = p->lean ? al(static_cast<int64_t>(p->planned_kv.size()) * 4LL) : 0;
+    p->dev_bytes = b_items + b_woff + b_merge + b_goff + b_po + b_pl + b_emp + b_err + b_cu + b_plan;
     cudaError_t e = cudaMalloc(&p->dev_base, static_cast<size_t>(p->dev_bytes));
     if (e != cudaSuccess) {
         set_cuda_error("cudaMalloc(plan)", static_cast<int>(e));
@@ -1985,6 +2257,8 @@ int device_init_plan(tg_plan *p) {
     p->d_dyn = p->d_err + 16;
     base += b_err;
     p->d_cunits = p->cunits.empty() ? nullptr : reinterpret_cast<CascadeUnit *>(base);
+    base += b_cu;
+    p->d_planned = p->lean ? reinterpret_cast<int32_t *>(base) : nullptr;
 
     rc = TG_OK;
     auto up = [&](void *dst, const void *src, int64_t bytes) {
@@ -2001,6 +2275,7 @@ int device_init_plan(tg_plan *p) {
     up(p->d_merge, p->merge.data(), static_cast<int64_t>(p->merge.size()) * static_cast<int64_t>(sizeof(MergeHead)));
     up(p->d_group_off, p->group_off.data(), (p->n_groups + 1) * 8LL);
     up(p->d_empties, p->empties.data(), static_cast<int64_t>(p->empties.size()) * 4LL);
+    if (p->lean) up(p->d_planned, p->planned_kv.data(), static_cast<int64_t>(p->planned_kv.size()) * 4LL);
     if (rc == TG_OK) {
         cudaError_t ee = cudaMemset(p->d_err, 0, 256);
         if (ee != cudaSuccess) { set_cuda_error("cudaMemset(plan)", static_cast<int>(ee)); rc = TG_ECUDA; }
@@ -2119,6 +2394,60 @@ static int finish_call(tg_plan *p, void *out, float *lse, cudaStream_t stream) {
     return TG_OK;
 }
 
+// Lean kernel launch (whole-head plans of short heads), as a programmatic dependent of whatever
+// precedes it in the stream.
+template <int D, int G>
+static int launch_lean_t(const tg_plan *p, const LeanArgs &a, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(static_cast<int64_t>(p->shape.B) * p->shape.Hkv));
+    cfg.blockDim = dim3(kLeanWarps * 32);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, lean_decode_kernel<D, G>, a));
+    return TG_OK;
+}
+
+static int launch_lean(const tg_plan *p, const void *q, const void *k_pages, const void *v_pages,
+                       const int32_t *page_table, const int64_t *head_page_off,
+                       const int32_t *head_kv_len, const int32_t *group_of_head, float scale,
+                       void *out, float *lse, cudaStream_t stream) {
+    LeanArgs a{};
+    a.Hq = p->shape.Hq;
+    a.Hkv = p->shape.Hkv;
+    a.scale_log2 = scale * 1.44269504088896340736f;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.k_pages = static_cast<const __nv_bfloat16 *>(k_pages);
+    a.v_pages = static_cast<const __nv_bfloat16 *>(v_pages);
+    a.table = page_table;
+    a.head_off = head_page_off;
+    a.group_of_head = group_of_head;
+    a.group_off = p->d_group_off;
+    a.n_groups = p->n_groups;
+    a.kv_len_dev = head_kv_len;
+    a.planned = p->d_planned;
+    a.num_pages = p->shape.num_pages;
+    a.out = p->out_f32 ? nullptr : static_cast<__nv_bfloat16 *>(out);
+    a.out_f32 = p->out_f32 ? static_cast<float *>(out) : nullptr;
+    a.lse = lse;
+    a.err = p->d_err;
+    a.early_prologue = p->early_prologue ? 1 : 0;
+    const int G = p->G;
+    if (p->shape.D == 128) {
+        if (G == 1) return launch_lean_t<128, 1>(p, a, stream);
+        if (G == 2) return launch_lean_t<128, 2>(p, a, stream);
+        if (G == 4) return launch_lean_t<128, 4>(p, a, stream);
+        return launch_lean_t<128, 8>(p, a, stream);
+    }
+    if (G == 1) return launch_lean_t<64, 1>(p, a, stream);
+    if (G == 2) return launch_lean_t<64, 2>(p, a, stream);
+    if (G == 4) return launch_lean_t<64, 4>(p, a, stream);
+    return launch_lean_t<64, 8>(p, a, stream);
+}
+
 static DecodeArgs base_args(const tg_plan *p, const void *q, const int32_t *kv, float scale,
                             void *out, float *lse) {
     DecodeArgs a{};
@@ -2185,6 +2514,20 @@ static int decode_bf16(tg_plan *p, const void *q, const void *k_pages, const voi
     if (cascade && (!k_pages || !v_pages || !page_table || !head_page_off ||
                     !aligned16(k_pages) || !aligned16(v_pages) || p->shape.num_pages < 1))
         return TG_EINVAL;
+    if (p->lean && !token_scores) {
+        // Whole-head plan of short heads: the lean kernel, one CTA per (sequence, KV head).
+        const int64_t heads = static_cast<int64_t>(p->shape.B) * p->shape.Hkv;
+        timing_mark(p, 0, stream);
+        if (heads > 0) {
+            if (!k_pages || !v_pages || !page_table || !head_page_off || !aligned16(k_pages) ||
+                !aligned16(v_pages))
+                return TG_EINVAL;
+            rc = launch_lean(p, q, k_pages, v_pages, page_table, head_page_off, head_kv_len,
+                             group_of_head, scale, out, lse, stream);
+            if (rc != TG_OK) return rc;
+        }
+        return finish_call(p, out, lse, stream);
+    }
     if (cascade) {
         // Shared runs first (the decode kernel that follows waits for them before it starts).
         rc = get_map(p, 0, k_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->shape.num_pages, 64);

@@ -244,8 +244,9 @@ def timed_plan_options(cfg: int) -> dict:
         kw.update(static_permille=900, dyn_chunk_pages=32)
     elif cfg == 4:
         # shared prefix pages: the cascade reads each shared run once per step for all its
-        # readers; the private pages stay on the split-K items
-        kw.update(static_permille=850, dyn_chunk_pages=16, cascade=True)
+        # readers; the private pages stay on the split-K items. The decode kernel's CTAs start
+        # as the cascade's finish, so less of its work is placed ahead of time
+        kw.update(static_permille=400, dyn_chunk_pages=16, cascade=True)
     elif cfg == 5:
         kw.update(min_splits=64, max_chunk_pages=128, static_permille=900, dyn_chunk_pages=32)
     return kw

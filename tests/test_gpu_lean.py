@@ -36,15 +36,16 @@ def _check(db, sp, lay, layer=0):
     return ref_out, ref_lse
 
 
+@pytest.mark.parametrize("span", [(0, 1024), (0, 20)])
 @pytest.mark.parametrize("early", [False, True])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 @pytest.mark.parametrize("D", [64, 128])
-def test_lean_matches_oracle(G, D, early):
-    # lengths 0 .. 1024 tokens: empty heads, single tokens, ragged tails, exactly 64 pages
-    sp = synth.Spec("lean sweep", "direct", B=5, Hq=3 * G, Hkv=3, D=D, len_lo=0, len_hi=1024,
-                    seed=0x7A4E4000 + 10 * G + D)
+def test_lean_matches_oracle(G, D, early, span):
+    # lengths drawn in [0, 1024] (several chunks, ragged tails, up to 64 pages) or [0, 20]
+    # (empty heads, single tokens, one or two pages)
+    sp = synth.Spec("lean sweep", "direct", B=5, Hq=3 * G, Hkv=3, D=D, len_lo=span[0],
+                    len_hi=span[1], seed=0x7A4E4000 + 10 * G + D + span[1])
     lay = workload.layout(sp, 0)
-    assert (lay.kv_len == 0).any() or lay.kv_len.min() < 16
     db = workload.to_device(sp, lay, 0, whole_heads=True, early_prologue=early)
     assert _is_lean(db.plan)
     db.run()

@@ -86,3 +86,31 @@ def test_plan_invariants(case):
         assert dyn[int(np.argmax(dyn)):].all()
     if opts["whole_heads"]:
         assert info["n_merge"] == 0 and len(items) == int((kv > 0).sum())
+
+
+def test_whole_head_plans_of_short_heads_take_the_lean_kernel():
+    """Whole-head bf16 plans whose heads hold at most 64 pages report the lean kernel's launch
+    (one CTA of 256 threads per (sequence, KV head), no ring, no shared-memory carve-out); longer
+    heads, split plans and tiered plans keep the pipelined kernel."""
+    import non_uniform_paged_flash_b200 as tg
+
+    def info(kv, **kw):
+        kv = np.asarray(kv, np.int32)
+        B, H = kv.shape
+        shape = tg.make_shape(B, 4 * H, H, 128, 1 << 16, 1 << 12 if "fast_len" in kw else 0)
+        plan = tg.tg_plan_create(shape, kv, np.zeros(H, np.int32), np.array([0, 1 << 20], np.int64),
+                                 host_only=True, **kw)
+        return tg.tg_plan_get_info(plan)
+
+    # lean: one CTA per (sequence, KV head), the empty head included
+    lean = info([[1024, 0, 17], [1, 999, 64]], whole_heads=True)
+    assert (lean["grid"], lean["block"], lean["stages"], lean["smem_bytes"]) == (6, 256, 0, 0)
+    assert lean["n_merge"] == 0 and lean["n_empty"] == 1
+    # a head of 65 pages: the pipelined kernel, its 2 whole heads on one CTA of 4 workers
+    long_ = info([[1025, 10]], whole_heads=True)
+    assert long_["grid"] == 1 and long_["n_workers"] == 2
+    split = info([[1024, 10]])
+    assert split["block"] == 4 * 64 and split["grid"] == -(-split["n_workers"] // 4)
+    tiered = info([[1024, 10]], whole_heads=True, fast_len=np.array([[100, 10]], np.int32),
+                  slow_table_len=1 << 10)
+    assert tiered["block"] == 6 * 64

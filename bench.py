@@ -135,9 +135,11 @@ def _measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def _traffic(cfg):
+def _traffic(cfg, alg_per_launch=None):
     """DRAM bytes per launch of the decode kernel from a committed ncu capture, if the kernel
-    source is unchanged since the capture; else None."""
+    source is unchanged since the capture; else None. A capture of one layer of a multi-layer
+    workload is stored as its traffic / algorithmic-bytes ratio and scaled to alg_per_launch
+    (the traffic grows with the pages a launch reads)."""
     src = os.path.join(ROOT, "non_uniform_paged_flash_b200", "csrc", "tg_kernels.cu")
     path = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
     try:
@@ -147,7 +149,10 @@ def _traffic(cfg):
             j = json.load(f)
         e = j.get(f"config{cfg}")
         if e and e.get("kernel_sha") == sha:
-            return float(e["traffic_bytes_per_launch"])
+            if "traffic_over_algorithmic" in e and alg_per_launch is not None:
+                return float(e["traffic_over_algorithmic"]) * float(alg_per_launch)
+            if "traffic_bytes_per_launch" in e:
+                return float(e["traffic_bytes_per_launch"])
     except Exception:
         pass
     return None
@@ -630,7 +635,7 @@ def run_ours(args):
             "kv_bytes_per_step": int(kv_sum / n_layers),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak,
-                         "traffic": _traffic(cfg) if world == 1 and n_layers == 1 else None,
+                         "traffic": (_traffic(cfg, alg_sum / n_layers) if world == 1 else None),
                          "peak_kind": peak_kind,
                          "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
                          "nominal_gbs": NOMINAL_HBM_GBS,

@@ -27,7 +27,6 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
-#include <type_traits>
 
 #include "tg_internal.h"
 
@@ -318,48 +317,21 @@ struct alignas(16) StageHdr {
     int64_t pad;
 };
 constexpr int32_t kHdrSlow = 1, kHdrFirst = 2, kHdrLast = 4, kHdrStop = 8, kHdrPair = 16;
-constexpr int32_t kHdrTwo = 32;  // the page's V is in the next stage (tiered kernel's bf16 pages)
 constexpr int32_t kNoLoad = -2;  // page id placeholder of a row that failed its bounds check
 
-// Shared-memory stage layout of the bf16 decode kernel (offsets within a stage; D = 128 shown,
-// D = 64 halves the bf16 regions): K bf16 [0, KB) as D/64 boxes of 16 rows x 128 B; V bf16
-// [KB, 2KB); q [2KB, +QB). One page per stage.
+// Shared-memory stage layout (offsets within a stage; D = 128 shown, D = 64 halves the bf16
+// regions): K bf16 [0, KB) as D/64 boxes of 16 rows x 128 B; V bf16 [KB, 2KB); q [2KB, +QB).
+// INT8 pages reuse it: K codes [0, 2048), K scales [2048, 2112), V scales [2112, 2176),
+// V codes [KB, KB + 2048). INT4 pages: packed K [KB + 2048, KB + 3072), packed V
+// [KB + 3072, KB + 4096) (16 rows x 64 B each, 64-byte swizzle), scales as INT8.
 template <int D>
 struct Layout {
-    static constexpr bool kTwo = false;  // a bf16 page spans two stages
     static constexpr int KB = 16 * D * 2;
-    static constexpr int kI8 = 16 * D;   // one INT8 page of one tensor
-    static constexpr int kI4 = 8 * D;    // one INT4 page of one tensor
-    static constexpr int kVbf = KB;      // bf16 V, within the page's stage
-    static constexpr int kQ = 2 * KB;
-    // (slow-tier offsets: unused by this kernel)
-    static constexpr int kV8 = KB, kK4 = KB + kI8, kV4 = KB + kI8 + kI4;
+    static constexpr int kI8 = 16 * D;  // one INT8 page of one tensor
+    static constexpr int kI4 = 8 * D;   // one INT4 page of one tensor
     static constexpr int kKScale = 2048, kVScale = 2112;
+    static constexpr int kK4 = KB + kI8, kV4 = KB + kI8 + kI4;
 };
-
-// Stage layout of the tiered decode kernel (D = 128): a stage is sized for one slow-tier page,
-// so the ring holds as many pages as its shared memory allows (pages in flight per worker, not
-// bytes, bound the tiered step). INT8: K codes [0, 2048), V codes [2048, 4096) (16 rows x 128 B
-// each, 128-byte swizzle); INT4: packed K [0, 1024), packed V [1024, 2048) (16 rows x 64 B,
-// 64-byte swizzle); K scales [4096, 4160), V scales [4160, 4224); the item's q rows at 4224. A
-// bf16 page takes two consecutive stages: K [0, 4096) and q in the first, V [0, 4096) in the
-// second.
-template <int D>
-struct TierLayout {
-    static constexpr bool kTwo = true;
-    static constexpr int KB = 16 * D * 2;
-    static constexpr int kI8 = 16 * D;
-    static constexpr int kI4 = 8 * D;
-    static constexpr int kVbf = 0;       // bf16 V, within the page's second stage
-    static constexpr int kV8 = 2048;
-    static constexpr int kK4 = 0, kV4 = 1024;
-    static constexpr int kKScale = 4096, kVScale = 4160;
-    static constexpr int kQ = 4224;
-    static_assert(D == 128, "the tiered kernel serves D = 128");
-};
-// Stage bytes of the tiered kernel: one slow-tier page, its scales and G query rows, rounded to
-// the 1024-byte alignment of 128-byte-swizzled boxes.
-constexpr int tier_stage_bytes(int G, int D) { return (4224 + G * D * 2 + 1023) / 1024 * 1024; }
 
 // Online-softmax state of the two query heads (2t, 2t+1) a consumer lane accumulates.
 struct PageState {
@@ -381,9 +353,8 @@ struct PageState {
 // widened to fp16 in registers, per-token scales); with SB = 4 the pages hold INT4 codes (byte
 // i of a row: d = i low nibble, d = i + D/2 high nibble, offset-binary), and off8[0..1] are the
 // ldmatrix offsets of the two 32-byte halves of the 64-byte rows.
-template <int D, int NP, bool SLOW, int SB, class L>
-__device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const uint32_t (&sv)[NP],
-                                              const int (&valid)[NP],
+template <int D, int NP, bool SLOW, int SB = 8>
+__device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const int (&valid)[NP],
                                               const uint32_t (&qf)[D / 16][2],
                                               float (&o)[D / 16][4], PageState &ps,
                                               const uint32_t (&offK)[D / 16],
@@ -391,6 +362,7 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const ui
                                               const uint32_t (&off8)[D / 32], float scale_log2,
                                               int lane, float *ts = nullptr, int64_t tpos = 0,
                                               int32_t G = 0) {
+    using L = Layout<D>;
     constexpr int KS = D / 16;
     constexpr unsigned FULL = 0xffffffffu;
     const int g = lane >> 2, t = lane & 3;
@@ -580,7 +552,7 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const ui
 #pragma unroll
             for (int p = 0; p < NP; ++p) {
                 uint32_t a0, a1, a2, a3;
-                dev::ldsm_x4_t(sv[p] + offV[i], a0, a1, a2, a3);
+                dev::ldsm_x4_t(sa[p] + offV[i], a0, a1, a2, a3);
                 if (tail[p]) {
                     a0 &= mk01[p];
                     a1 &= mk01[p];
@@ -630,7 +602,7 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const ui
 #pragma unroll
             for (int p = 0; p < NP; ++p) {
                 uint32_t r0, r1, r2, r3;
-                dev::ldsm_x4_t(sa[p] + L::kV8 + off8[ii], r0, r1, r2, r3);
+                dev::ldsm_x4_t(sa[p] + L::KB + off8[ii], r0, r1, r2, r3);
                 // r0/r1: tokens (2t, 2t+1) / (8+2t, 9+2t) at d = 32ii + 2g, +1 (chunk 2ii);
                 // r2/r3: the same for chunk 2ii+1. Tile i rows: g -> d 16i + 2g, g+8 -> +1.
                 uint32_t a0, a1, a2, a3;
@@ -657,7 +629,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                   const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ CUtensorMap tm_kq,
                   const __grid_constant__ CUtensorMap tm_vq) {
-    using L = std::conditional_t<TIERED, TierLayout<D>, Layout<D>>;
+    using L = Layout<D>;
     constexpr unsigned FULL = 0xffffffffu;
 
     extern __shared__ unsigned char smem_raw[];
@@ -830,28 +802,14 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                 const bool slow = TIERED && (fl & kItemSlow);
                 const int32_t b = bh / a.Hkv, h = bh - b * a.Hkv;
                 const int32_t cnt = min(32, pe - p0);
-                // Pages are issued in batches: the first page's stages are waited for, the
-                // stages of the following pages that the consumer has already released (it
-                // releases a page pair at once) are tested without waiting, and lane l issues
-                // page k + l, so the copies of up to kIssueLanes pages are issued side by side
-                // instead of one after another from one lane. A page takes spp stages (two for
-                // a bf16 page in the tiered kernel's compact ring); stages are released in
-                // order, so a page's stages are free once its last one is.
-                const int spp = (L::kTwo && !slow) ? 2 : 1;
-                auto stage_of = [&](int x, uint32_t &ph) {
-                    int st_ = pstage + x;
-                    ph = pphase;
-                    if (st_ >= stages) {
-                        st_ -= stages;
-                        ph ^= 1u;
-                    }
-                    return st_;
-                };
+                // Pages are issued in batches: the first free stage is waited for, the stages
+                // after it that the consumer has already released (it releases a page pair at
+                // once) are tested without waiting, and lane l issues page k + l of the block
+                // into stage pstage + l, so the copies of up to kIssueLanes pages are issued
+                // side by side instead of one after another from one lane.
                 for (int32_t k = 0; k < cnt;) {
                     wait_predecessor();
-                    uint32_t ph0;
-                    const int last0 = stage_of(spp - 1, ph0);
-                    const bool ok = dev::mbar_wait(empty0 + 8 * last0, ph0 ^ 1u, a.wait_ns);
+                    const bool ok = dev::mbar_wait(empty0 + 8 * pstage, pphase ^ 1u, a.wait_ns);
                     if (!ok || ctl[1]) {
                         if (lane == 0) {
                             atomicOr(a.err, kErrTimeout);
@@ -860,22 +818,21 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         aborted = true;
                         return;
                     }
-                    const int nmax = min(cnt - k, min(stages / spp, kIssueLanes));
-                    bool is_free = lane == 0;
-                    if (lane > 0 && lane < nmax) {
-                        uint32_t phl;
-                        const int lastl = stage_of((lane + 1) * spp - 1, phl);
-                        is_free = dev::mbar_test(empty0 + 8 * lastl, phl ^ 1u);
+                    const int nmax = min(cnt - k, min(stages, kIssueLanes));
+                    int stage = pstage + lane;
+                    uint32_t phase = pphase;
+                    if (stage >= stages) {
+                        stage -= stages;
+                        phase ^= 1u;
                     }
+                    const bool is_free = lane == 0 ||
+                                         (lane < nmax && dev::mbar_test(empty0 + 8 * stage, phase ^ 1u));
                     const uint32_t freed = __ballot_sync(FULL, is_free);
-                    const int n = __ffs(~freed) - 1;  // pages whose stages are released, <= nmax
+                    const int n = __ffs(~freed) - 1;  // released stages from pstage on, <= nmax
                     int32_t page_id = __shfl_sync(FULL, ids, (k + lane) & 31);
                     if (lane < n) {
-                        uint32_t phase_unused;
-                        const int stage = stage_of(lane * spp, phase_unused);
-                        const int stage2 = spp == 2 ? (stage + 1 == stages ? 0 : stage + 1) : stage;
                         const int32_t pg = p0 + k + lane;
-                        const uint32_t sq = seq + static_cast<uint32_t>(lane * spp);
+                        const uint32_t sq = seq + static_cast<uint32_t>(lane);
                         const int32_t vtok = max(0, min(16, tt - pg * 16));
                         if (vtok == 0) {
                             page_id = kNoLoad;  // a reserved page holding no token yet
@@ -891,8 +848,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         StageHdr hd;
                         hd.valid = page_id >= 0 ? vtok : 0;
                         hd.flags = (slow ? kHdrSlow : 0) | (first ? kHdrFirst : 0) |
-                                   (last ? kHdrLast : 0) | (pair ? kHdrPair : 0) |
-                                   (spp == 2 ? kHdrTwo : 0);
+                                   (last ? kHdrLast : 0) | (pair ? kHdrPair : 0);
                         hd.bh = bh;
                         hd.slot = slot;
                         hd.tpos = row_j + pg;
@@ -902,10 +858,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         const uint32_t fb = full0 + 8 * stage;
                         const uint32_t qbytes = static_cast<uint32_t>(a.G * D * 2);
                         uint32_t bytes = first ? qbytes : 0u;
-                        if (page_id >= 0) {
-                            if (slow) bytes += 2u * ((SB == 4 ? L::kI4 : L::kI8) + 64u);
-                            else bytes += spp == 2 ? static_cast<uint32_t>(L::KB) : 2u * L::KB;
-                        }
+                        if (page_id >= 0) bytes += slow ? 2u * ((SB == 4 ? L::kI4 : L::kI8) + 64u) : 2u * L::KB;
                         if (a.withhold && worker == 0 && sq + 1 == static_cast<uint32_t>(a.withhold)) {
                             // testing: this stage is never signalled; the consumer's bounded
                             // wait runs out and the call reports a timeout
@@ -914,7 +867,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                         } else {
                             dev::mbar_arrive_expect_tx(fb, bytes);
                             if (first)
-                                dev::bulk_load(st + L::kQ,
+                                dev::bulk_load(st + 2 * L::KB,
                                                a.q + (static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * a.G) * D,
                                                qbytes, fb);
                             if (page_id >= 0) {
@@ -926,41 +879,24 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                                     dev::bulk_load(st + L::kVScale, a.v_scale + static_cast<int64_t>(page_id) * 16, 64, fb);
                                 } else if (slow) {
                                     dev::tma_load_2d(st, &tm_kq, 0, y, fb);
-                                    dev::tma_load_2d(st + L::kV8, &tm_vq, 0, y, fb);
+                                    dev::tma_load_2d(st + L::KB, &tm_vq, 0, y, fb);
                                     dev::bulk_load(st + L::kKScale, a.k_scale + static_cast<int64_t>(page_id) * 16, 64, fb);
                                     dev::bulk_load(st + L::kVScale, a.v_scale + static_cast<int64_t>(page_id) * 16, 64, fb);
                                 } else {
 #pragma unroll
-                                    for (int bx = 0; bx < D / 64; ++bx)
+                                    for (int bx = 0; bx < D / 64; ++bx) {
                                         dev::tma_load_2d(st + bx * 2048, &tm_k, bx * 64, y, fb);
-                                    if (spp == 1) {
-#pragma unroll
-                                        for (int bx = 0; bx < D / 64; ++bx)
-                                            dev::tma_load_2d(st + L::kVbf + bx * 2048, &tm_v, bx * 64, y, fb);
+                                        dev::tma_load_2d(st + L::KB + bx * 2048, &tm_v, bx * 64, y, fb);
                                     }
                                 }
-                            }
-                        }
-                        if (spp == 2) {
-                            // the page's V in the next stage
-                            const uint32_t st2 = dev::smem_addr(ring + static_cast<size_t>(stage2) * a.stage_bytes);
-                            const uint32_t fb2 = full0 + 8 * stage2;
-                            if (page_id >= 0) {
-                                dev::mbar_arrive_expect_tx(fb2, static_cast<uint32_t>(L::KB));
-#pragma unroll
-                                for (int bx = 0; bx < D / 64; ++bx)
-                                    dev::tma_load_2d(st2 + L::kVbf + bx * 2048, &tm_v, bx * 64, page_id * 16, fb2);
-                            } else {
-                                dev::mbar_arrive(fb2);
                             }
                         }
                         if (trace && sq == 0) trace[1] = dev::global_timer();
                     }
                     __syncwarp();
-                    const int used = n * spp;
-                    if (lane == 0) ctl[0] = static_cast<int32_t>(seq + static_cast<uint32_t>(used));
-                    seq += static_cast<uint32_t>(used);
-                    pstage += used;
+                    if (lane == 0) ctl[0] = static_cast<int32_t>(seq + static_cast<uint32_t>(n));
+                    seq += static_cast<uint32_t>(n);
+                    pstage += n;
                     if (pstage >= stages) {
                         pstage -= stages;
                         pphase ^= 1u;
@@ -1034,7 +970,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
             const uint32_t rk = (lm & 1) * 8 + (lane & 7), ck = 2 * j + (lm >> 1);
             offK[j] = (ck >> 3) * 2048 + dev::swz(rk, ck & 7);
             const uint32_t rv = (lm >> 1) * 8 + (lane & 7), cv = 2 * j + (lm & 1);
-            offV[j] = L::kVbf + (cv >> 3) * 2048 + dev::swz(rv, cv & 7);
+            offV[j] = L::KB + (cv >> 3) * 2048 + dev::swz(rv, cv & 7);
         }
 #pragma unroll
         for (int j = 0; j < KSTEPS / 2; ++j)
@@ -1082,20 +1018,9 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
             if (trace && lane == 0) trace[3] = dev::global_timer();
             break;
         }
-        // A page's stages: one, or (kHdrTwo: a bf16 page of the tiered kernel) K in the first
-        // and V in the next; with kHdrPair the next page is consumed in the same step.
         const int sA = cstage;
         advance();
-        int sAv = sA;
-        if (hd.flags & kHdrTwo) {
-            if (!dev::mbar_wait(full0 + 8 * cstage, cphase, a.wait_ns)) {
-                timed_out();
-                return;
-            }
-            sAv = cstage;
-            advance();
-        }
-        int sB = sA, sBv = sA;
+        int sB = sA;
         int validB = 0;
         int32_t last_flags = hd.flags;
         const bool pair = (hd.flags & kHdrPair) != 0;
@@ -1106,18 +1031,9 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
             }
             const StageHdr hb = hdr[cstage];
             sB = cstage;
-            sBv = sB;
             validB = hb.valid;
             last_flags = hb.flags;
             advance();
-            if (hb.flags & kHdrTwo) {
-                if (!dev::mbar_wait(full0 + 8 * cstage, cphase, a.wait_ns)) {
-                    timed_out();
-                    return;
-                }
-                sBv = cstage;
-                advance();
-            }
         }
         const unsigned char *stA = ring + static_cast<size_t>(sA) * a.stage_bytes;
         const unsigned char *stB = ring + static_cast<size_t>(sB) * a.stage_bytes;
@@ -1126,7 +1042,7 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
         if (hd.flags & kHdrFirst) {
             // New item: query fragments (B operand, N = head g of this KV head) and state.
             item_slow = slow;
-            const unsigned char *qs = stA + L::kQ;
+            const unsigned char *qs = stA + 2 * L::KB;
 #pragma unroll
             for (int j = 0; j < KSTEPS; ++j) {
                 if (g < a.G) {
@@ -1205,41 +1121,33 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
         }
 
         const uint32_t aA = dev::smem_addr(stA), aB = dev::smem_addr(stB);
-        // bf16 V: in the page's own stage (bf16 kernel) or the one after it (tiered kernel)
-        const uint32_t vA = dev::smem_addr(ring + static_cast<size_t>(sAv) * a.stage_bytes);
-        const uint32_t vB = dev::smem_addr(ring + static_cast<size_t>(sBv) * a.stage_bytes);
         if (!slow) {
             if (pair) {
-                const uint32_t sa[2] = {aA, aB}, sv[2] = {vA, vB};
+                const uint32_t sa[2] = {aA, aB};
                 const int va[2] = {hd.valid, validB};
-                consume_pages<D, 2, false, 8, L>(sa, sv, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane,
-                                                 a.token_scores, hd.tpos, a.G);
+                consume_pages<D, 2, false>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane,
+                                           a.token_scores, hd.tpos, a.G);
             } else {
-                const uint32_t sa[1] = {aA}, sv[1] = {vA};
+                const uint32_t sa[1] = {aA};
                 const int va[1] = {hd.valid};
-                consume_pages<D, 1, false, 8, L>(sa, sv, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane,
-                                                 a.token_scores, hd.tpos, a.G);
+                consume_pages<D, 1, false>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane,
+                                           a.token_scores, hd.tpos, a.G);
             }
         } else if (TIERED) {
             if (pair) {
                 const uint32_t sa[2] = {aA, aB};
                 const int va[2] = {hd.valid, validB};
-                consume_pages<D, 2, true, SB, L>(sa, sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
+                consume_pages<D, 2, true, SB>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
             } else {
                 const uint32_t sa[1] = {aA};
                 const int va[1] = {hd.valid};
-                consume_pages<D, 1, true, SB, L>(sa, sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
+                consume_pages<D, 1, true, SB>(sa, va, qf, o, ps, offK, offV, off8, a.scale_log2, lane);
             }
         }
         __syncwarp();
         if (lane == 0) {
-            // in stage order
             dev::mbar_arrive(empty0 + 8 * sA);
-            if (sAv != sA) dev::mbar_arrive(empty0 + 8 * sAv);
-            if (pair) {
-                dev::mbar_arrive(empty0 + 8 * sB);
-                if (sBv != sB) dev::mbar_arrive(empty0 + 8 * sBv);
-            }
+            if (pair) dev::mbar_arrive(empty0 + 8 * sB);
         }
 
         if (last_flags & kHdrLast) {
@@ -1637,12 +1545,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint4 *src = valid ? reinterpret_cast<const uint4 *>(
                                            a.q + (static_cast<int64_t>(u->reader[r / G]) * a.Hq + h * G + r % G) * D)
                                      : nullptr;
+            // every load of the row in flight before the first store (an asm store with a
+            // memory clobber would otherwise hold each next load back: D/8 serial round trips)
+            uint4 qv[D / 8];
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) qv[c] = src ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
             for (int c = 0; c < D / 8; ++c) {
-                const uint4 v = src ? src[c] : make_uint4(0u, 0u, 0u, 0u);
                 const uint32_t addr = qrow + (c / 8) * (kTcRows * 128) + (((c % 8) ^ (i & 7)) << 4);
                 asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                             :: "r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+                             :: "r"(addr), "r"(qv[c].x), "r"(qv[c].y), "r"(qv[c].z), "r"(qv[c].w) : "memory");
             }
             tc::fence_async_smem();
             __syncwarp();
@@ -2274,17 +2186,15 @@ int device_init_plan(tg_plan *p) {
     if (p->device < 0) p->device = cur;
     if (p->device != cur) TG_CUDA_TRY(cudaSetDevice(p->device));
 
-    // Stage geometry: the bf16 kernel's stage holds a page and q; the tiered kernel's holds one
-    // slow-tier page and q (a bf16 page takes two stages).
+    // Stage geometry.
     const int KB = 16 * s.D * 2;
     const int QB = ((p->G * s.D * 2) + 1023) / 1024 * 1024;
-    p->stage_bytes = p->tiered ? tier_stage_bytes(p->G, s.D) : 2 * KB + QB;
+    p->stage_bytes = 2 * KB + QB;
     const int per_stage_extra = static_cast<int>(sizeof(StageHdr)) + 16;  // header + 2 barriers
     const int np = p->pairs;
     int stages = (kSmemBudget - 1024 - np * 8) / (np * (p->stage_bytes + per_stage_extra));
     stages = stages > 8 ? 8 : stages;
-    // a page pair plus one page in flight (a tiered bf16 pair takes four stages)
-    if (stages < (p->tiered ? 5 : 3)) {
+    if (stages < 3) {  // a page pair plus one page in flight
         if (p->device != cur) cudaSetDevice(cur);
         return TG_EUNSUPPORTED;
     }

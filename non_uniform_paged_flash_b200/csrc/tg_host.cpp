@@ -760,45 +760,19 @@ int plan_create(const tg_shape *shape, const int32_t *kv_len, const int32_t *fas
         for (int32_t b = 0; b < s.B; ++b) rows[b] = b;
         for (int32_t h = 0; h < s.Hkv; ++h)
             shared_runs(h, rows, s.Hkv, kv_len, table, head_off, min_readers, nodes, p->pstart);
-        // Long runs are cut into segments of at most `cap` pages, so that the cascade CTAs (one
-        // per unit, two tensor-core tiles of query rows each) are of similar length: the
-        // kernel's time is its longest CTA. cap: four pages per block, at least the blocks one
-        // SM would run if all the runs' blocks were spread evenly (at least 8 blocks).
-        int nsm = 148;
-        if (!p->host_only && tg::device_num_sms(o.device, &nsm) != TG_OK) nsm = 148;
-        const int32_t per = tg::kCascadeRows / G;
-        int64_t total_blocks = 0;
-        for (const Node &n : nodes)
-            total_blocks += (static_cast<int64_t>(n.readers.size()) + per - 1) / per * ((n.pos_end - n.pos_begin + 3) / 4);
-        const int64_t target = std::max<int64_t>(8, (total_blocks + nsm - 1) / std::max(1, nsm));
-        const int32_t cap = static_cast<int32_t>(4 * target);
-        struct Seg { int32_t h, pb, pe; const Node *n; };
-        std::vector<Seg> segs;
-        for (const Node &n : nodes) {
-            const int32_t len = n.pos_end - n.pos_begin;
-            const int32_t k = (len + cap - 1) / cap;
-            for (int32_t c = 0, at = n.pos_begin; c < k; ++c) {
-                const int32_t sz = len / k + (c < len % k ? 1 : 0);
-                segs.push_back({n.h, at, at + sz, &n});
-                at += sz;
-            }
-        }
-        // longest segments first: CTAs are dispatched in index order
-        std::stable_sort(segs.begin(), segs.end(),
-                         [](const Seg &x, const Seg &y) { return x.pe - x.pb > y.pe - y.pb; });
         casc_cnt.assign(static_cast<size_t>(BH), 0);
-        for (const Seg &sg : segs)
-            for (int32_t b : sg.n->readers) ++casc_cnt[static_cast<int64_t>(b) * s.Hkv + sg.h];
-        for (const Seg &sg : segs) {
-            const std::vector<int32_t> &rd = sg.n->readers;
-            for (size_t r0 = 0; r0 < rd.size(); r0 += per) {
+        for (const Node &n : nodes)
+            for (int32_t b : n.readers) ++casc_cnt[static_cast<int64_t>(b) * s.Hkv + n.h];
+        const int32_t per = tg::kCascadeRows / G;
+        for (const Node &n : nodes) {
+            for (size_t r0 = 0; r0 < n.readers.size(); r0 += per) {
                 tg::CascadeUnit u{};
-                u.h = sg.h;
-                u.pos_begin = sg.pb;
-                u.pos_end = sg.pe;
-                u.n_readers = static_cast<int32_t>(std::min<size_t>(per, rd.size() - r0));
+                u.h = n.h;
+                u.pos_begin = n.pos_begin;
+                u.pos_end = n.pos_end;
+                u.n_readers = static_cast<int32_t>(std::min<size_t>(per, n.readers.size() - r0));
                 for (int32_t r = 0; r < u.n_readers; ++r) {
-                    u.reader[r] = rd[r0 + r];
+                    u.reader[r] = n.readers[r0 + r];
                     u.slot[r] = -1;
                 }
                 p->cunits.push_back(u);

@@ -74,8 +74,7 @@ def check_cascade(plan, B, Hq, Hkv, kv_len, table, head_off, min_readers=2):
 @pytest.mark.parametrize("full", [False, True])
 def test_prefix_config_runs(full):
     """Config 4: per KV head one run of the system pages read by every sequence, and one run
-    of each document's full pages read by the sequences on it; a run may be cut into
-    consecutive page segments (balanced cascade CTAs), each read by all the run's readers."""
+    of each document's full pages read by the sequences on it."""
     sp = synth.preset(4) if full else synth.small(4)
     lay = workload.layout(sp, 0)
     B = lay.kv_len.shape[0]
@@ -86,25 +85,13 @@ def test_prefix_config_runs(full):
     doc_pages = sp.doc_tokens // 16
     doc, _ = synth.prefix_layout(sp)
     per = tg.CASCADE_ROWS // (sp.Hq // sp.Hkv)
-    def segments(m, lo, hi):
-        """The units of [lo, hi) by segment: the segments tile [lo, hi) in order."""
-        sel = m[(m[:, 1] >= lo) & (m[:, 2] <= hi)]
-        segs = sorted({(int(a), int(b)) for a, b in sel[:, 1:3]})
-        assert segs and segs[0][0] == lo and segs[-1][1] == hi
-        assert all(x[1] == y[0] for x, y in zip(segs, segs[1:]))
-        return segs, sel
-
-    readers = np.bincount(doc, minlength=sp.n_docs)
     for h in range(sp.Hkv):
         m = meta[meta[:, 0] == h]
-        segs, sel = segments(m, 0, sys_pages)
-        for a, b in segs:
-            u = sel[(sel[:, 1] == a) & (sel[:, 2] == b)]
-            assert u[:, 3].sum() == B and len(u) == -(-B // per)
-        segs, sel = segments(m, sys_pages, sys_pages + doc_pages)
-        for a, b in segs:
-            u = sel[(sel[:, 1] == a) & (sel[:, 2] == b)]
-            assert u[:, 3].sum() == readers[readers >= 2].sum()
+        sysu = m[(m[:, 1] == 0) & (m[:, 2] == sys_pages)]
+        assert sysu[:, 3].sum() == B and len(sysu) == -(-B // per)
+        docu = m[(m[:, 1] == sys_pages) & (m[:, 2] == sys_pages + doc_pages)]
+        readers = sorted(np.bincount(doc, minlength=sp.n_docs)[np.bincount(doc, minlength=sp.n_docs) >= 2])
+        assert docu[:, 3].sum() == sum(readers)
     # the private items start after the deepest run of each row
     assert (items[:, 1] >= sys_pages + doc_pages).all()
 

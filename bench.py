@@ -1021,7 +1021,7 @@ def run_tier_host(args):
         "value": achieved, "unit": "GB/s", "higher_is_better": True, "n_gpus": 1, "steps": reps,
         "warmup": args.warmup, "ms_per_step": ms, "dtype": "bf16+int%d" % sp.slow_bits,
         "data": "synthetic",
-        "config": {"workload": WORKLOAD_NAMES[cfg] + "; INT%d tier in pinned host memory" % sp.slow_bits,
+        "config": {"workload": _workload_name(cfg, sp) + "; INT%d tier in pinned host memory" % sp.slow_bits,
                    "block_pages": block_pages, "ring_blocks": 3, "blocks_per_step": n_blocks},
         "host_tier_bytes_per_step": slow_bytes, "kv_bytes_per_step": int(alg["kv"]),
         "roofline": {"bound": "host link", "achieved": achieved, "peak": peak_link,

@@ -218,37 +218,26 @@ __device__ __forceinline__ float f16_hi(uint32_t v) {
 }
 
 // One ldmatrix.trans register of INT8 V codes, bytes (x[t][d], x[t][d+1], x[t+1][d], x[t+1][d+1]),
-// -> two fp16x2 registers (x[t][d], x[t+1][d]) and (x[t][d+1], x[t+1][d+1]), exactly: bias each
-// byte to x + 128, place it in the low mantissa byte of fp16 1024 (0x6400), subtract 1152.
+// -> two fp16x2 registers (x[t][d], x[t+1][d]) and (x[t][d+1], x[t+1][d+1]) holding x + 1152,
+// exactly: bias each byte to x + 128 and place it in the low mantissa byte of fp16 1024 (0x6400).
+// The constant 1152 is not subtracted here: the P V product carries 1152 sum(p') per head, which
+// the item's end removes once (kV8Offset).
 __device__ __forceinline__ void i8pair_to_f16(uint32_t v, uint32_t &lo, uint32_t &hi) {
     const uint32_t u = v ^ 0x80808080u;
-    uint32_t a, b;
-    asm("prmt.b32 %0, %1, %2, 0x4240;" : "=r"(a) : "r"(u), "r"(0x64646464u));
-    asm("prmt.b32 %0, %1, %2, 0x4341;" : "=r"(b) : "r"(u), "r"(0x64646464u));
-    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
-    __half2 ha = __hsub2(*reinterpret_cast<__half2 *>(&a), bias);
-    __half2 hb = __hsub2(*reinterpret_cast<__half2 *>(&b), bias);
-    lo = *reinterpret_cast<uint32_t *>(&ha);
-    hi = *reinterpret_cast<uint32_t *>(&hb);
+    asm("prmt.b32 %0, %1, %2, 0x4240;" : "=r"(lo) : "r"(u), "r"(0x64646464u));
+    asm("prmt.b32 %0, %1, %2, 0x4341;" : "=r"(hi) : "r"(u), "r"(0x64646464u));
 }
+constexpr float kV8Offset = 1152.f;
 
-// One ldmatrix.trans register of INT4 V (offset-binary nibbles; bits 0-7 token t byte b,
-// 8-15 token t byte b+1, 16-23 token t+1 byte b, 24-31 token t+1 byte b+1) -> fp16x2 (t, t+1)
-// of its four d: `lo` takes the low nibbles of bytes b (shift 0) or b+1 (shift 8), exactly as
-// 1024 + u - 1032; `hi` the high nibbles, as (1024 + 16u) / 16 - 72.
-__device__ __forceinline__ uint32_t nib_lo_f16(uint32_t v) {
-    uint32_t h = (v & 0x000F000Fu) | 0x64006400u;
-    const __half2 bias = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032
-    __half2 r = __hsub2(*reinterpret_cast<__half2 *>(&h), bias);
-    return *reinterpret_cast<uint32_t *>(&r);
-}
-__device__ __forceinline__ uint32_t nib_hi_f16(uint32_t v) {
-    uint32_t h = (v & 0x00F000F0u) | 0x64006400u;
-    const __half2 k = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));     // 1/16
-    const __half2 c = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));     // -72
-    __half2 r = __hfma2(*reinterpret_cast<__half2 *>(&h), k, c);
-    return *reinterpret_cast<uint32_t *>(&r);
-}
+// One ldmatrix.trans register of INT4 V (offset-binary nibbles u = x + 8; bits 0-7 token t byte
+// b, 8-15 token t byte b+1, 16-23 token t+1 byte b, 24-31 token t+1 byte b+1) -> fp16x2 (t, t+1)
+// of its four d, exactly and with the offsets left in: `lo` takes the low nibbles of bytes b
+// (shift 0) or b+1 (shift 8) as 1024 + u = x + 1032; `hi` the high nibbles as 1024 + 16 u =
+// 16 x + 1152, i.e. 16 (x + 72). The item's end scales the high-nibble tiles by 1/16 and removes
+// 1032 or 72 times sum(p') per head.
+__device__ __forceinline__ uint32_t nib_lo_f16(uint32_t v) { return (v & 0x000F000Fu) | 0x64006400u; }
+__device__ __forceinline__ uint32_t nib_hi_f16(uint32_t v) { return (v & 0x00F000F0u) | 0x64006400u; }
+constexpr float kV4LoOffset = 1032.f, kV4HiOffset = 72.f;
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a box of 64-byte rows written by TMA
 // with 64-byte swizzle (chunk bits XOR address bits 7-8; the box base is 512-byte aligned).
@@ -340,9 +329,10 @@ struct PageState {
     float m0, m1;    // running maxima, log2 units
     float le0, le1;  // sums of fp32 probabilities (for the lse)
     float lr0, lr1;  // sums of the probabilities multiplied into V
+    float w0, w1;    // slow tiers: sums of the fp16 p' = p * v_scale that met the offset V codes
     __device__ __forceinline__ void reset() {
         m0 = m1 = -INFINITY;
-        le0 = le1 = lr0 = lr1 = 0.f;
+        le0 = le1 = lr0 = lr1 = w0 = w1 = 0.f;
     }
 };
 
@@ -519,6 +509,10 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
         ps.le1 *= c1;
         ps.lr0 *= c0;
         ps.lr1 *= c1;
+        if (SLOW) {
+            ps.w0 *= c0;
+            ps.w1 *= c1;
+        }
         ps.m0 = n0;
         ps.m1 = n1;
     }
@@ -572,8 +566,11 @@ __device__ __forceinline__ void consume_pages(const uint32_t (&sa)[NP], const in
             const bool v0 = g < valid[p], v1 = g + 8 < valid[p];
             const float q0 = v0 ? pv[p][0] * vs[p][0] : 0.f, q1 = v0 ? pv[p][1] * vs[p][0] : 0.f;
             const float q2 = v1 ? pv[p][2] * vs[p][1] : 0.f, q3 = v1 ? pv[p][3] * vs[p][1] : 0.f;
-            b0[p] = dev::movm_t(dev::pack_f16(q0, q1));
-            b1[p] = dev::movm_t(dev::pack_f16(q2, q3));
+            const uint32_t h01 = dev::pack_f16(q0, q1), h23 = dev::pack_f16(q2, q3);
+            ps.w0 += dev::f16_lo(h01) + dev::f16_lo(h23);
+            ps.w1 += dev::f16_hi(h01) + dev::f16_hi(h23);
+            b0[p] = dev::movm_t(h01);
+            b1[p] = dev::movm_t(h23);
         }
         if (SB == 4) {
             // INT4 V: ldmatrix.trans of a 32-byte half jj (chunks 2jj, 2jj+1): r0 / r1 tokens
@@ -1159,6 +1156,26 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
                 E1 += __shfl_xor_sync(FULL, E1, off);
                 R0 += __shfl_xor_sync(FULL, R0, off);
                 R1 += __shfl_xor_sync(FULL, R1, off);
+            }
+            if (TIERED && item_slow) {
+                // the V codes entered P V with their offsets (see i8pair_to_f16, nib_lo_f16):
+                // remove offset * sum(p') per head, and the x16 of the INT4 high-nibble tiles
+                float W0 = ps.w0, W1 = ps.w1;
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    W0 += __shfl_xor_sync(FULL, W0, off);
+                    W1 += __shfl_xor_sync(FULL, W1, off);
+                }
+#pragma unroll
+                for (int i = 0; i < KSTEPS; ++i) {
+                    const bool hi4 = SB == 4 && i >= KSTEPS / 2;
+                    const float f = hi4 ? 1.f / 16.f : 1.f;
+                    const float off = SB == 4 ? (hi4 ? dev::kV4HiOffset : dev::kV4LoOffset) : dev::kV8Offset;
+                    o[i][0] = o[i][0] * f - off * W0;
+                    o[i][2] = o[i][2] * f - off * W0;
+                    o[i][1] = o[i][1] * f - off * W1;
+                    o[i][3] = o[i][3] * f - off * W1;
+                }
             }
             const float inv0 = R0 > 0.f ? 1.f / R0 : 0.f, inv1 = R1 > 0.f ? 1.f / R1 : 0.f;
             constexpr float kLn2 = 0.69314718055994530942f;

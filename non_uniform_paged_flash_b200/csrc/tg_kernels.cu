@@ -1260,19 +1260,20 @@ __global__ void __launch_bounds__(NPAIRS * 64, 1)
 // shared by up to two tiles of 128 query rows (each row one (reader, query head) pair).
 //   warps 0-3 / 4-7: softmax of tile 0 / 1; thread i of a warpgroup owns query row i, which is
 //                    lane i of tensor memory, so a row's max and sums need no shuffles
-//   warp 8:          allocates tensor memory; lane 0 issues every tcgen05.mma
-//   warp 9:          producer: page ids 32 at a time, 2-D TMA loads of K and V, 4 pages (64
+//   warps 8 / 9:     MMA issue of tile 0 / 1 (lane 0); warp 8 also allocates tensor memory
+//   warp 10:         producer: page ids 32 at a time, 2-D TMA loads of K and V, 4 pages (64
 //                    tokens) per block, into a ring of kTcStages blocks
 // Per block and tile: S = Q K^T (M = 128 rows, N = 64 tokens, K = D; both operands K-major,
 // 128-byte swizzled, S in tensor memory); the softmax reads S with tcgen05.ld, keeps the
 // running max (lazy rescale: the max moves only when a block exceeds it by 2^8; then O is
-// read, scaled and written back in tensor memory), writes P as bf16 into a swizzled tile;
-// O += P V (M = 128, N = D, K = 16 tokens per page; V is the MN-major operand, as stored).
+// read, scaled and written back in tensor memory) and writes P as bf16 pairs back over the
+// first 32 columns of the same S buffer with tcgen05.st; O += P V (M = 128, N = D, K = 16
+// tokens per page; A = P from tensor memory, V the MN-major shared-memory operand, as stored).
 // The two tiles alternate, so one tile's softmax overlaps the other's MMAs. Each reader's
 // rows end as a normalised partial (o, lse) in its slot, merged with the head's other
 // partials by the merge kernel.
-// Tensor memory (512 columns): tile t holds S in columns [256t, 256t + 64) and O in
-// [256t + 128, 256t + 128 + D).
+// Tensor memory (512 columns): tile t holds two S / P buffers in columns [256t, 256t + 128)
+// and O in [256t + 128, 256t + 128 + D). Shared memory: the two Q tiles, then the K/V ring.
 // ------------------------------------------------------------------------------------------
 struct CascadeArgs {
     const CascadeUnit *units;
@@ -1337,6 +1338,17 @@ __device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a, uint64_t b, uin
         : "memory");
 }
 
+// As mma, with the A operand in tensor memory at a_tmem (M rows on the lanes, K along the
+// columns, two 16-bit elements per 32-bit column).
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        :: "r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrives on the mbarrier once every tcgen05.mma issued so far by this thread has completed.
 __device__ __forceinline__ void commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -1347,19 +1359,17 @@ __device__ __forceinline__ void commit(uint32_t bar) {
 
 constexpr int kTcRows = 128;               // rows per tile = tensor-memory lanes
 constexpr int kTcThreads = 11 * 32;        // 8 softmax warps, 2 MMA warps, 1 producer warp
-constexpr int kTcStages = 3;               // K/V blocks in flight
+constexpr int kTcStages = 5;               // K/V blocks in flight
 constexpr uint32_t kTcCols = 512;          // tensor-memory columns of the CTA
 
 template <int D>
 struct TcLayout {
     static constexpr int kHalves = D / 64;                  // 64-element (128-byte) column halves
     static constexpr int kQTile = kTcRows * D * 2;          // one tile of Q
-    static constexpr int kPTile = kTcRows * 64 * 2;         // one buffer of P (64 tokens)
     static constexpr int kKBlock = 64 * D * 2;              // 64 tokens of K
     static constexpr int kStage = 2 * kKBlock;              // K then V
     static constexpr int kQ = 0;
-    static constexpr int kP = kQ + 2 * kQTile;              // [tile][buffer]
-    static constexpr int kKV = kP + 4 * kPTile;
+    static constexpr int kKV = kQ + 2 * kQTile;
     static constexpr int kBars = kKV + kTcStages * kStage;  // mbarriers, then the TMEM address
     static constexpr int kBytes = kBars + 256;
 };
@@ -1495,8 +1505,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == 8 || warp == 9) {
         // ========================= MMA warps (tile 0: warp 8, tile 1: warp 9) =========================
-        // S(blk) goes to buffer blk & 1 and is issued before PV(blk - 1), so the next block's
-        // scores are ready when the softmax finishes a block.
+        // S(blk) goes to tensor-memory buffer blk & 1 and is issued before PV(blk - 1), so the
+        // next block's scores are ready when the softmax finishes a block. The softmax writes
+        // P(blk) as bf16 pairs over the first 32 columns of S(blk)'s buffer, and PV(blk) takes it
+        // from there as its A operand; S(blk + 2), which reuses the buffer, is issued by this
+        // thread after PV(blk), and the MMAs of one thread run in issue order.
         const int t = warp - 8;
         if (lane == 0 && t < ntiles) {
             const uint32_t id_s = tc::idesc_bf16(64, kTcRows, 0);
@@ -1506,11 +1519,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc::fence_after();
             auto issue_o = [&](int32_t blk) {
                 const uint32_t kv = sbase + TL::kKV + (blk % kTcStages) * TL::kStage + TL::kKBlock;
-                const uint32_t pt = sbase + TL::kP + (2 * t + (blk & 1)) * TL::kPTile;
+                const uint32_t pt = tmem + 256 * t + 64 * (blk & 1);  // P(blk): 8 columns per 16 tokens
                 const int32_t np = min(4, npages - 4 * blk);
                 for (int32_t k = 0; k < np; ++k)
-                    tc::mma(tmem + 256 * t + 128, tc::sdesc(pt + k * 32, 16, 1024),
-                            tc::sdesc(kv + k * 2048, TL::kKBlock / TL::kHalves, 1024), id_o, blk > 0 || k > 0);
+                    tc::mma_ts(tmem + 256 * t + 128, pt + 8 * k,
+                               tc::sdesc(kv + k * 2048, TL::kKBlock / TL::kHalves, 1024), id_o, blk > 0 || k > 0);
                 tc::commit(o_done + 8 * (2 * t + (blk & 1)));
                 tc::commit(kv_empty + 8 * (blk % kTcStages));
             };
@@ -1602,11 +1615,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 const float mx = fmaxf(fmaxf(fmaxf(mr[0], mr[1]), fmaxf(mr[2], mr[3])),
                                        fmaxf(fmaxf(mr[4], mr[5]), fmaxf(mr[6], mr[7]))) * a.scale_log2;
-                // P buffer bf was last read by PV(blk - 2)
-                if (blk >= 2) {
-                    ok = dev::mbar_wait(o_done + 8 * (2 * t + bf), ph ^ 1u, a.wait_ns) && !*abort_flag;
-                    if (!__all_sync(FULL, ok)) { ok = false; break; }
-                }
                 const bool up = mx > m + 8.f;
                 if (__any_sync(FULL, up)) {
                     const float mn = up ? mx : m;
@@ -1631,32 +1639,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     le *= c0;
                     m = mn;
                 }
-                // p = 2^(s * scale - m): one FFMA and one ex2 per score; 8 partial sums
-                const uint32_t prow = sbase + TL::kP + (2 * t + bf) * TL::kPTile + i * 128;
+                // p = 2^(s * scale - m): one FFMA and one ex2 per score; 8 partial sums. P goes
+                // to the first 32 columns of this S buffer (bf16 pairs; the scores are in
+                // registers), the A operand of PV(blk).
                 float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                 const float nm = -m;
+                uint32_t pw[32];
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = 8 * c8 + 2 * e;
-                        float p0 = dev::ex2(fmaf(__uint_as_float(sr[c]), a.scale_log2, nm));
-                        float p1 = dev::ex2(fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, nm));
-                        if (nv < 64) {
-                            p0 = c < nv ? p0 : 0.f;
-                            p1 = c + 1 < nv ? p1 : 0.f;
-                        }
-                        ls[e] += p0;
-                        ls[4 + e] += p1;
-                        w[e] = dev::pack_bf16(p0, p1);
+                for (int e = 0; e < 32; ++e) {
+                    const int c = 2 * e;
+                    float p0 = dev::ex2(fmaf(__uint_as_float(sr[c]), a.scale_log2, nm));
+                    float p1 = dev::ex2(fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, nm));
+                    if (nv < 64) {
+                        p0 = c < nv ? p0 : 0.f;
+                        p1 = c + 1 < nv ? p1 : 0.f;
                     }
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                                 :: "r"(prow + ((c8 ^ (i & 7)) << 4)), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
-                                 : "memory");
+                    ls[e & 3] += p0;
+                    ls[4 + (e & 3)] += p1;
+                    pw[e] = dev::pack_bf16(p0, p1);
                 }
                 le += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-                tc::fence_async_smem();
+                tc::tmem_st32(t_s + 64 * bf, pw);
+                tc::tmem_wait_st();
                 tc::fence_before();
                 __syncwarp();
                 if (lane == 0) dev::mbar_arrive(p_full + 8 * (2 * t + bf));
@@ -1671,12 +1675,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (lane == 0) timed_out();
             } else {
                 // out row = O / le (partial), lse = (m + log2 le) ln 2. The warp's 32 rows leave
-                // through shared memory (the P buffers are idle once the last PV is done), so that
-                // each store writes whole 128-byte row segments (8 lanes a row, 4 rows a store)
-                // instead of a 16-byte piece of each of 32 rows: 8x fewer L2 transactions.
+                // through shared memory (the tile's Q region: its last S MMA ran before its last
+                // PV, which is done), so that each store writes whole 128-byte row segments (8
+                // lanes a row, 4 rows a store) instead of a 16-byte piece of each of 32 rows: 8x
+                // fewer L2 transactions.
                 const float inv = le > 0.f ? 1.f / le : 0.f;
-                // this tile's own two P buffers (the other tile's may still feed its last PV)
-                const uint32_t stg = sbase + TL::kP + static_cast<uint32_t>(2 * t * TL::kPTile + qd * 4096);  // 32 rows x 128 B
+                const uint32_t stg = sbase + TL::kQ + static_cast<uint32_t>(t * TL::kQTile + qd * 4096);  // 32 rows x 128 B
                 float *dst[8];  // rows 4k + lane / 8 of this warp (null past the readers)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {

@@ -2014,8 +2014,18 @@ __global__ void __launch_bounds__(1024) split_merge_kernel(const MergeHead *mh, 
         for (int u = 0; u < U; ++u) {
             const bool in = j + u < j1;
             l[u] = in ? pl[static_cast<int64_t>(j + u) * G] : -INFINITY;
+            // the lane's VEC consecutive floats in one 8- or 16-byte load (rows of D floats)
+            if constexpr (VEC == 4) {
+                const float4 x = in ? *reinterpret_cast<const float4 *>(po + (j + u) * pstride)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[u][0] = x.x;
+                v[u][1] = x.y;
+                v[u][2] = x.z;
+                v[u][3] = x.w;
+            } else {
 #pragma unroll
-            for (int c = 0; c < VEC; ++c) v[u][c] = in ? po[(j + u) * pstride + c] : 0.f;
+                for (int c = 0; c < VEC; ++c) v[u][c] = in ? po[(j + u) * pstride + c] : 0.f;
+            }
         }
         float mc = m;
 #pragma unroll
@@ -2064,12 +2074,23 @@ __global__ void __launch_bounds__(1024) split_merge_kernel(const MergeHead *mh, 
         m = M;
     }
     const float inv = m == -INFINITY ? 0.f : 1.f / sum;
+    if constexpr (VEC == 4) {
+        if (out_f32) {
+            *reinterpret_cast<float4 *>(out_f32 + row * D + lane * VEC) =
+                make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+        } else {
+            // four bf16 in one 8-byte store
+            *reinterpret_cast<uint2 *>(out + row * D + lane * VEC) =
+                make_uint2(dev::pack_bf16(acc[0] * inv, acc[1] * inv), dev::pack_bf16(acc[2] * inv, acc[3] * inv));
+        }
+    } else {
 #pragma unroll
-    for (int c = 0; c < VEC; ++c) {
-        if (out_f32)
-            out_f32[row * D + lane * VEC + c] = acc[c] * inv;
-        else
-            out[row * D + lane * VEC + c] = __float2bfloat16_rn(acc[c] * inv);
+        for (int c = 0; c < VEC; ++c) {
+            if (out_f32)
+                out_f32[row * D + lane * VEC + c] = acc[c] * inv;
+            else
+                out[row * D + lane * VEC + c] = __float2bfloat16_rn(acc[c] * inv);
+        }
     }
     if (lane == 0) lse[row] = m == -INFINITY ? -INFINITY : m + logf(sum);
 }

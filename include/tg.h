@@ -313,9 +313,10 @@ int tg_plan_timing_read(tg_plan *p, int32_t *n_calls, double *decode_ms, double 
 /* Worker timeline (a profiling aid). With on = 1 the plan allocates n_workers x 8 uint64
  * device words (here, not per call) and every later decode call records, per worker: the
  * global timer (ns) at CTA start, first copy issued, first page ready, stop marker seen and
- * worker done; then the number of dynamic items it took, the number of split heads it merged
- * and the ns it spent merging. tg_plan_trace_read synchronises the stream and copies the
- * last call's words to trace (host, n_workers x 8). on = 0 frees the buffer. */
+ * worker done; then the number of dynamic items it took; words 6 and 7 are written as zero
+ * (split heads are merged by the merge kernel, after the decode kernel). tg_plan_trace_read
+ * synchronises the stream and copies the last call's words to trace (host, n_workers x 8).
+ * on = 0 frees the buffer. */
 int tg_plan_trace_enable(tg_plan *p, int32_t on);
 int tg_plan_trace_read(tg_plan *p, uint64_t *trace, tg_stream stream);
 

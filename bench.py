@@ -139,7 +139,8 @@ def _traffic(cfg, alg_per_launch=None):
     """DRAM bytes per launch of the decode kernel from a committed ncu capture, if the kernel
     source is unchanged since the capture; else None. A capture of one layer of a multi-layer
     workload is stored as its traffic / algorithmic-bytes ratio and scaled to alg_per_launch
-    (the traffic grows with the pages a launch reads)."""
+    (the traffic grows with the pages a launch reads). A tiered workload with the INT4 slow tier
+    has its own entry."""
     src = os.path.join(ROOT, "non_uniform_paged_flash_b200", "csrc", "tg_kernels.cu")
     path = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
     try:
@@ -147,7 +148,8 @@ def _traffic(cfg, alg_per_launch=None):
             sha = hashlib.sha256(f.read()).hexdigest()[:16]
         with open(path) as f:
             j = json.load(f)
-        e = j.get(f"config{cfg}")
+        int4 = synth.preset(cfg).kind == "tiered" and SLOW_BITS == 4
+        e = j.get(f"config{cfg}" + ("_int4" if int4 else ""))  # the INT4 slow tier moves other bytes
         if e and e.get("kernel_sha") == sha:
             if "traffic_over_algorithmic" in e and alg_per_launch is not None:
                 return float(e["traffic_over_algorithmic"]) * float(alg_per_launch)

@@ -2095,6 +2095,90 @@ __global__ void __launch_bounds__(1024) split_merge_kernel(const MergeHead *mh, 
     if (lane == 0) lse[row] = m == -INFINITY ? -INFINITY : m + logf(sum);
 }
 
+// Merge of split heads of 9..kLaneParts parts: one warp per (split head, query row), 8 rows
+// per CTA. Lane j holds part j's lse; the row's maximum and the sum of the weights
+// w_j = exp(l_j - max) are warp reductions; each lane then sums its D/32 columns over the parts,
+// kPartBatch parts' loads at a time (all in flight), the weights broadcast from their lanes.
+// Fewer dependent rounds than the multi-warp merge for heads of 9..32 parts, and no shared
+// memory. The order of the sums is fixed, so the result does not depend on timing.
+constexpr int kLaneParts = 32;
+constexpr int kPartBatch = 16;
+
+template <int D>
+__global__ void __launch_bounds__(256) lane_merge_kernel(const MergeHead *mh, int64_t n_rows, int32_t G,
+                                                         int32_t Hq, int32_t Hkv, const float *part_o,
+                                                         const float *part_lse, __nv_bfloat16 *out,
+                                                         float *out_f32, float *lse) {
+    constexpr int VEC = D / 32;
+    constexpr unsigned FULL = 0xffffffffu;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t rid = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
+    if (rid >= n_rows) return;
+    const MergeHead h = mh[rid / G];
+    const int n = static_cast<int>(rid % G);
+    const int64_t pstride = static_cast<int64_t>(G) * D;
+    const float *pl = part_lse + static_cast<int64_t>(h.first_slot) * G + n;
+    const float *po = part_o + (static_cast<int64_t>(h.first_slot) * G + n) * D + lane * VEC;
+    const float l = lane < h.nsplit ? pl[static_cast<int64_t>(lane) * G] : -INFINITY;
+    float m = l;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+    const float w = (m == -INFINITY || l == -INFINITY) ? 0.f : expf(l - m);  // 0 for an empty part
+    float sum = w;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(FULL, sum, off);
+    float acc[VEC];
+#pragma unroll
+    for (int c = 0; c < VEC; ++c) acc[c] = 0.f;
+    for (int j0 = 0; j0 < h.nsplit; j0 += kPartBatch) {
+        float v[kPartBatch][VEC];
+#pragma unroll
+        for (int jj = 0; jj < kPartBatch; ++jj) {
+            const int j = j0 + jj;
+            if constexpr (VEC == 4) {
+                const float4 x = j < h.nsplit ? *reinterpret_cast<const float4 *>(po + j * pstride)
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[jj][0] = x.x;
+                v[jj][1] = x.y;
+                v[jj][2] = x.z;
+                v[jj][3] = x.w;
+            } else {
+#pragma unroll
+                for (int c = 0; c < VEC; ++c) v[jj][c] = j < h.nsplit ? po[j * pstride + c] : 0.f;
+            }
+        }
+#pragma unroll
+        for (int jj = 0; jj < kPartBatch; ++jj) {
+            const float wj = __shfl_sync(FULL, w, (j0 + jj) & 31);  // 0 past the parts
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) acc[c] += wj * v[jj][c];
+        }
+    }
+    const int32_t b = h.bh / Hkv, hh = h.bh - b * Hkv;
+    const int64_t row = static_cast<int64_t>(b) * Hq + static_cast<int64_t>(hh) * G + n;
+    const float inv = m == -INFINITY ? 0.f : 1.f / sum;
+    if constexpr (VEC == 4) {
+        if (out_f32) {
+            *reinterpret_cast<float4 *>(out_f32 + row * D + lane * VEC) =
+                make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+        } else {
+            *reinterpret_cast<uint2 *>(out + row * D + lane * VEC) =
+                make_uint2(dev::pack_bf16(acc[0] * inv, acc[1] * inv), dev::pack_bf16(acc[2] * inv, acc[3] * inv));
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) {
+            if (out_f32)
+                out_f32[row * D + lane * VEC + c] = acc[c] * inv;
+            else
+                out[row * D + lane * VEC + c] = __float2bfloat16_rn(acc[c] * inv);
+        }
+    }
+    if (lane == 0) lse[row] = m == -INFINITY ? -INFINITY : m + logf(sum);
+}
+
 // Generic merge (exported as tg_lse_merge): rows with contiguous split ranges.
 __global__ void lse_merge_kernel(int64_t n_rows, int32_t D, const int64_t *off, const float *po,
                                  const float *pl, __nv_bfloat16 *out, float *lse) {
@@ -2425,17 +2509,23 @@ static int launch_decode(tg_plan *p, DecodeFn fn, const DecodeArgs &a, const CUt
     return TG_OK;
 }
 
-// Merge kernel of the split heads (optionally a programmatic dependent launch). Heads of at
-// most 8 splits (merge_warps == 1) get one warp per query row, 8 rows per CTA.
+// Merge kernel of the split heads (optionally a programmatic dependent launch), by the most parts
+// a head of the plan has: up to 8 (merge_warps == 1), one warp per query row, 8 rows per CTA,
+// its parts loaded 4 at a time; 9 to kLaneParts (merge_warps <= 4), one warp per query row with
+// a lane per part (fewer dependent rounds for these heads; measured: config 2 103.8 -> 102.0
+// us, while heads of 3 parts ran slower this way, 83 -> 93 us on config 4, the kernel holding
+// twice the registers); more, one CTA per row, its warps splitting the head's parts.
 static int launch_merge(const tg_plan *p, const MergeHead *d_merge, const float *po, const float *pl,
                         void *out, float *lse, cudaStream_t stream, bool pdl) {
     constexpr int kRowsPerCta = 8;
+    static_assert(kLaneParts == 4 * 8, "lane merge: merge_warps <= 4 means at most 32 parts");
     const int64_t n_rows = static_cast<int64_t>(p->merge.size()) * p->G;
     const bool rows = p->merge_warps == 1;
+    const bool lanes = !rows && p->merge_warps <= 4;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(rows ? (n_rows + kRowsPerCta - 1) / kRowsPerCta : n_rows));
-    cfg.blockDim = dim3(static_cast<unsigned>(rows ? 32 * kRowsPerCta : 32 * p->merge_warps));
-    cfg.dynamicSmemBytes = !rows ? static_cast<size_t>(p->merge_warps) * (2 + p->shape.D) * 4 : 0;
+    cfg.gridDim = dim3(static_cast<unsigned>(rows || lanes ? (n_rows + kRowsPerCta - 1) / kRowsPerCta : n_rows));
+    cfg.blockDim = dim3(static_cast<unsigned>(rows || lanes ? 32 * kRowsPerCta : 32 * p->merge_warps));
+    cfg.dynamicSmemBytes = !rows && !lanes ? static_cast<size_t>(p->merge_warps) * (2 + p->shape.D) * 4 : 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -2447,9 +2537,11 @@ static int launch_merge(const tg_plan *p, const MergeHead *d_merge, const float 
     float *of = p->out_f32 ? static_cast<float *>(out) : nullptr;
     if (p->shape.D == 128) {
         if (rows) TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<128, true>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, of, lse));
+        else if (lanes) TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, lane_merge_kernel<128>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, of, lse));
         else TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<128, false>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, of, lse));
     } else {
         if (rows) TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<64, true>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, of, lse));
+        else if (lanes) TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, lane_merge_kernel<64>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, of, lse));
         else TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, split_merge_kernel<64, false>, d_merge, n_rows, G, Hq, Hkv, po, pl, o, of, lse));
     }
     return TG_OK;

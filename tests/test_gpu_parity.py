@@ -122,6 +122,22 @@ def test_split_heads_every_partition_size():
             assert info["n_partials"] > 0
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("workers, lo, hi", [(8, 2, 8), (48, 9, 32), (400, 33, 10**6)])
+def test_merge_by_parts_per_head(D, workers, lo, hi):
+    """Each merge kernel, chosen by the most parts a head of the plan has (up to 8: a warp per
+    row, parts 4 at a time; 9 to 32: a warp per row, a lane per part; more: a CTA per row),
+    at both head dimensions, against the oracle. A head's parts are the workers its pages land
+    on (at most one worker per 8 pages of the batch)."""
+    sp = synth.Spec("merge", "direct", B=2, Hq=8, Hkv=2, D=D, len_lo=2000, len_hi=9000,
+                    seed=0x7A4E3100 + D)
+    db, _ = _run(sp, num_workers=workers, static_permille=1000)
+    items = tg.tg_plan_items(db.plan)
+    mi = items[:, 7]
+    parts = np.bincount(mi[mi >= 0])
+    assert lo <= parts.max() <= hi, parts.max()
+
+
 def test_deterministic_repeat():
     """Dynamic items land on different workers from call to call; the merge order (split
     order) keeps the results bit-identical."""

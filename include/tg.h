@@ -249,7 +249,7 @@ void tg_plan_destroy(tg_plan *p);
 typedef struct tg_plan_info {
     int64_t n_items;          /* work items */
     int64_t n_partials;       /* items that write a partial result (heads with > 1 item) */
-    int64_t n_merge;          /* heads split over several items (merged in the kernel) */
+    int64_t n_merge;          /* heads split over several items (merged by the merge kernel) */
     int64_t n_empty;          /* heads with no retained token (out = 0, lse = -inf) */
     int64_t n_dynamic;        /* items taken from the shared ticket at run time */
     int32_t n_workers;        /* workers that have items */
